@@ -1,0 +1,360 @@
+"""Checks that pin the CPU oracle to things other than itself.
+
+Each ``check_*`` raises AssertionError when the oracle disagrees with the pin:
+a library routine computing the same definition (torch fp64
+scaled_dot_product_attention, torch.sort, torch.logsumexp), a closed form or
+invariant, or a hand-enumerated case from ``tests/golden``.  The pin tests call
+them on the oracle as written; the mutation tests call them on deliberately
+broken copies and expect them to fail.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+from oracle import csa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _sdpa(q, k, v, mask=None, scale=None, is_causal=False):
+    """torch fp64 attention: q [H, m, D], k/v [H, n, D], mask [H or 1, m, n] bool."""
+    return F.scaled_dot_product_attention(
+        torch.tensor(np.array(q), dtype=torch.float64)[None], torch.tensor(np.array(k), dtype=torch.float64)[None],
+        torch.tensor(np.array(v), dtype=torch.float64)[None],
+        attn_mask=None if mask is None else torch.tensor(np.array(mask))[None],
+        scale=scale, is_causal=is_causal)[0].numpy()
+
+
+# ---------------------------------------------------------------- attention
+
+def check_attention_vs_sdpa(seed=0, G=4, D=32, T=512, L=32, n_sel=5):
+    """Sparse attention over a chunk set == fp64 SDPA with a mask that keeps
+    exactly the tokens of those chunks; lse == logsumexp of the masked logits."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((G, D))
+    K = rng.standard_normal((T, D))
+    V = rng.standard_normal((T, D))
+    C = T // L
+    chunks = sorted(rng.choice(C, size=n_sel, replace=False).tolist())
+    scale = 1.0 / math.sqrt(D)
+    o, lse = O.decode_unit(q, K, V, chunks, L, scale)
+    keep = np.zeros(T, dtype=bool)
+    for c in chunks:
+        keep[c * L:(c + 1) * L] = True
+    mask = np.broadcast_to(keep, (G, 1, T))
+    ref = _sdpa(q[:, None, :], np.broadcast_to(K, (G, T, D)), np.broadcast_to(V, (G, T, D)),
+                mask=mask, scale=scale)[:, 0]
+    assert np.allclose(o, ref, rtol=0, atol=1e-12), np.abs(o - ref).max()
+    logits = torch.as_tensor(q @ K.T * scale)
+    logits[:, ~torch.as_tensor(keep)] = -math.inf
+    ref_lse = torch.logsumexp(logits, dim=1).numpy()
+    assert np.allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def check_dense_special_case(seed=1, G=2, D=16, T=256, L=32):
+    """Selecting every chunk (k_free covers the pool) reduces to dense
+    attention: fp64 SDPA with no mask."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((G, D))
+    K = rng.standard_normal((T, D))
+    V = rng.standard_normal((T, D))
+    C = T // L
+    summ = O.chunk_summaries(K, L)
+    s = O.score_chunks(q[None, None], summ[None, None], 1)[0, 0, 0]
+    chunks, _ = O.select_topk(s, C, 1, 1)
+    assert chunks == list(range(C))
+    o, _ = O.decode_unit(q, K, V, chunks, L, 0.25)
+    ref = _sdpa(q[:, None, :], np.broadcast_to(K, (G, T, D)), np.broadcast_to(V, (G, T, D)),
+                scale=0.25)[:, 0]
+    assert np.allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def check_empty_attention():
+    """An empty token set gives o = 0 and lse = -inf (no NaN)."""
+    o, lse = O.attend(np.ones((2, 4)), np.ones((8, 4)), np.ones((8, 4)), np.zeros(0, dtype=int), 1.0)
+    assert np.all(o == 0) and np.all(lse == -math.inf)
+
+
+# ---------------------------------------------------------------- summaries / scores
+
+def check_summary_closed_form():
+    """Keys that are constant within a chunk (row value = chunk id + column id)
+    have exactly that constant as summary; the projected summary equals the
+    mean of the projected keys (linearity)."""
+    L, C, D = 4, 5, 3
+    K = np.zeros((C * L, D))
+    for c in range(C):
+        K[c * L:(c + 1) * L] = c + np.arange(D)
+    s = O.chunk_summaries(K, L)
+    assert np.array_equal(s, np.arange(C)[:, None] + np.arange(D)[None, :])
+    rng = np.random.default_rng(3)
+    K = rng.standard_normal((8 * 16, 12))
+    P = rng.standard_normal((12, 4)) / 4
+    a = O.chunk_summaries(K, 16, P)
+    b = (K @ P).reshape(8, 16, 4).mean(axis=1)
+    assert np.allclose(a, b, rtol=0, atol=1e-12)
+
+
+def check_score_hand_case():
+    """s = q^T k_summary summed over the query heads of the KV head, on a case
+    worked by hand: heads q0 = (1, 2), q1 = (3, -1); summaries (1, 0), (0, 1),
+    (2, 2).  Group sum (4, 1): scores 4, 1, 10."""
+    q = np.array([[[[1.0, 2.0], [3.0, -1.0]]]])  # [B=1, Nq=1, Hq=2, D=2]
+    summ = np.array([[[[1.0, 0.0], [0.0, 1.0], [2.0, 2.0]]]])  # [1, Hkv=1, C=3, 2]
+    s = O.score_chunks(q, summ, 1)
+    assert np.array_equal(s[0, 0, 0], [4.0, 1.0, 10.0])
+    # two KV heads each with one query head: no mixing across groups
+    q2 = np.array([[[[1.0, 0.0], [0.0, 1.0]]]])
+    summ2 = np.array([[[[5.0, 7.0]], [[5.0, 7.0]]]])  # [1, 2, 1, 2]
+    s2 = O.score_chunks(q2, summ2, 2)
+    assert s2[0, 0, 0, 0] == 5.0 and s2[0, 1, 0, 0] == 7.0
+
+
+def check_projection_closed_form(seed=4):
+    """(P^T q) . (P^T kbar) == q^T (P P^T) kbar, computed two ways."""
+    rng = np.random.default_rng(seed)
+    D, R, C, G = 24, 6, 7, 3
+    q = rng.standard_normal((1, 1, G, D))
+    kbar = rng.standard_normal((C, D))
+    P = rng.standard_normal((D, R)) / 4
+    s = O.score_chunks(q, (kbar @ P)[None, None], 1, P)[0, 0, 0]
+    ref = (q[0, 0].sum(axis=0) @ P @ P.T) @ kbar.T
+    assert np.allclose(s, ref, rtol=0, atol=1e-12)
+
+
+def check_tile_mean():
+    """Tile mean of rows that are constant within the tile is that row; means
+    of a linear ramp are the ramp's midpoints."""
+    B, S, Hq, D, m = 1, 12, 2, 3, 4
+    Q = np.zeros((B, S, Hq, D))
+    for s_ in range(S):
+        Q[0, s_] = s_
+    tm = O.tile_mean_q(Q, m)
+    assert np.array_equal(tm[0, :, 0, 0], [1.5, 5.5, 9.5])
+
+
+# ---------------------------------------------------------------- selection
+
+def check_topk_golden():
+    for c in _golden("topk_cases.json")["cases"]:
+        got, _ = O.select_topk(np.array(c["scores"], dtype=np.float64), c["k_free"],
+                               c["n_sink"], c["n_local"], c["n_valid"])
+        assert got == c["expect"], (c["why"], got)
+
+
+def check_topk_vs_torch_sort(seed=5, C=64, trials=20):
+    """Library pin: the free part of the set is the first k_free of a stable
+    descending torch.sort over the non-forced chunks (stable sort keeps equal
+    scores in ascending index order)."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        s = rng.integers(-4, 5, size=C).astype(np.float64)  # many exact ties
+        n_sink, n_local = int(rng.integers(0, 3)), int(rng.integers(0, 3))
+        k_free = int(rng.integers(0, C))
+        got, _ = O.select_topk(s, k_free, n_sink, n_local)
+        forced = set(range(n_sink)) | set(range(C - n_local, C))
+        pool = torch.tensor([c for c in range(C) if c not in forced], dtype=torch.long)
+        order = torch.sort(torch.as_tensor(s)[pool], descending=True, stable=True).indices
+        ref = sorted(forced | set(pool[order[:k_free]].tolist()))
+        assert got == ref
+
+
+def check_topk_invariants(seed=6, C=40, trials=20):
+    """Forced chunks present; size = |F| + min(k_free, pool); every chosen
+    pool chunk scores >= every unchosen pool chunk; output ascending."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        s = rng.standard_normal(C)
+        v = int(rng.integers(1, C + 1))
+        k_free = int(rng.integers(0, C))
+        got, _ = O.select_topk(s, k_free, 1, 1, v)
+        F_ = {0, v - 1}
+        assert F_ <= set(got) and got == sorted(got) and all(c < v for c in got)
+        pool = [c for c in range(v) if c not in F_]
+        chosen = [c for c in got if c not in F_]
+        assert len(chosen) == min(k_free, len(pool))
+        rest = [c for c in pool if c not in chosen]
+        if chosen and rest:
+            assert min(s[chosen]) >= max(s[rest])
+
+
+def check_topp_golden():
+    for c in _golden("topp_cases.json")["cases"]:
+        got, n_p, _ = O.select_topp(np.array(c["scores"], dtype=np.float64), c["logit_scale"],
+                                    c["p"], c["budget"], c["n_sink"], c["n_local"])
+        assert got == c["expect"] and n_p == c["n_p"], (c["why"], got, n_p)
+
+
+def check_topp_invariants(seed=7, C=50, trials=30):
+    """cum(n_p - 1) < p <= cum(n_p) on the mass sorted by numpy (library);
+    forced chunks present; |set| <= budget + |F|; when n_p <= budget the free
+    part is exactly the n_p largest masses."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        s = rng.standard_normal(C) * rng.uniform(0.5, 8)
+        p = float(rng.uniform(0.05, 0.99))
+        budget = int(rng.integers(1, C))
+        scale = float(rng.uniform(0.1, 2))
+        got, n_p, _ = O.select_topp(s, scale, p, budget, 1, 2)
+        pi = np.exp(s * scale - (s * scale).max())
+        pi /= pi.sum()
+        cum = np.cumsum(np.sort(pi)[::-1])
+        assert cum[n_p - 1] >= p and (n_p == 1 or cum[n_p - 2] < p)
+        F_ = {0, C - 2, C - 1}
+        assert F_ <= set(got) and len(got) <= budget + len(F_)
+        if n_p <= budget:
+            top = set(np.argsort(-pi, kind="stable")[:n_p].tolist())
+            assert set(got) == top | F_
+
+
+def check_hier_golden():
+    for c in _golden("hier_cases.json")["cases"]:
+        summ = np.array(c["summ"], dtype=np.float64)[:, None]
+        meta = O.meta_summaries(summ, c["Gm"])
+        got, _, _ = O.select_hier(np.array(c["q"]), meta, summ, c["Gm"], c["top_meta"],
+                                  c["k_free"], c["n_sink"], c["n_local"])
+        assert got == c["expect"], (c["why"], got)
+
+
+def check_hier_all_metas_is_flat(seed=8, trials=10):
+    """Keeping every meta-chunk reduces the hierarchy to flat top-k over all
+    chunks with the same forced set and k_free."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        G, D, Gm, M = 4, 16, 8, 12
+        C = Gm * M
+        q = rng.standard_normal((G, D))
+        summ = rng.standard_normal((C, D))
+        meta = O.meta_summaries(summ, Gm)
+        k_free = int(rng.integers(1, 30))
+        got, _, _ = O.select_hier(q, meta, summ, Gm, M, k_free, 1, 2)
+        s = O.score_chunks(q[None, None], summ[None, None], 1)[0, 0, 0]
+        flat, _ = O.select_topk(s, k_free, 1, 2)
+        assert got == flat
+
+
+def check_meta_linearity(seed=9):
+    """A meta-summary (mean of Gm chunk means) equals the plain mean of all
+    Gm * L raw keys under it."""
+    rng = np.random.default_rng(seed)
+    L, Gm, M, D = 8, 4, 3, 5
+    K = rng.standard_normal((L * Gm * M, D))
+    meta = O.meta_summaries(O.chunk_summaries(K, L), Gm)
+    ref = K.reshape(M, Gm * L, D).mean(axis=1)
+    assert np.allclose(meta, ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- split-K and merge
+
+def check_merge_closed_form(seed=10, trials=10):
+    """Merging partials of any partition of a token set equals one-pass
+    attention over the set; an empty (-inf) split contributes nothing; one
+    partial merges to itself."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        G, D, n = 3, 8, int(rng.integers(2, 60))
+        q = rng.standard_normal((G, D)) * 2
+        K = rng.standard_normal((n, D))
+        V = rng.standard_normal((n, D))
+        tok = np.arange(n)
+        o_ref, lse_ref = O.attend(q, K, V, tok, 0.7)
+        cuts = sorted(rng.choice(np.arange(1, n), size=int(rng.integers(1, min(n, 6))),
+                             replace=False).tolist())
+        parts = np.split(tok, cuts)
+        op, lp = [], []
+        for pt in parts:
+            o, l = O.attend(q, K, V, pt, 0.7)
+            op.append(o)
+            lp.append(l)
+        op.append(np.full((G, D), 123.0))  # an empty split: o must not be read
+        lp.append(np.full(G, -math.inf))
+        o_part = np.stack(op, axis=1)
+        lse_part = np.stack(lp, axis=1)
+        om, lm = O.lse_merge(o_part, lse_part)
+        assert np.allclose(om, o_ref, rtol=0, atol=1e-12)
+        assert np.allclose(lm, lse_ref, rtol=0, atol=1e-12)
+        o1, l1 = O.lse_merge(o_ref[:, None], lse_ref[:, None])
+        assert np.allclose(o1, o_ref, rtol=0, atol=1e-14) and np.allclose(l1, lse_ref, atol=1e-14)
+
+
+def check_partition(seed=11, trials=20):
+    """The split-K layout covers each unit's list exactly once, in order, with
+    pieces whose sizes differ by at most one across the whole job."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        n = rng.integers(0, 40, size=int(rng.integers(1, 9))).tolist()
+        P = int(rng.integers(1, 50))
+        spl = O.decode_partition(n, P)
+        for u, s in enumerate(spl):
+            pos = 0
+            for (a, b) in s:
+                assert a == pos and b > a
+                pos = b
+            assert pos == n[u]
+        N = sum(n)
+        sizes = [((c + 1) * N) // P - (c * N) // P for c in range(P)]
+        assert max(sizes) - min(sizes) <= 1
+        assert sum(len(s) for s in spl) <= P + len(n) - 1
+    # hand-worked: lists of 5 and 3 chunks, 3 pieces: cuts at 0, 2, 5, 8
+    assert O.decode_partition([5, 3], 3) == [[(0, 2), (2, 5)], [(0, 3)]]
+    # lists of 4 and 4, 3 pieces: piece [2, 5) straddles the two units
+    assert O.decode_partition([4, 4], 3) == [[(0, 2), (2, 4)], [(0, 1), (1, 4)]]
+    # more pieces than chunks: empty pieces produce no split
+    assert O.decode_partition([2, 0, 1], 5) == [[(0, 1), (1, 2)], [], [(0, 1)]]
+
+
+# ---------------------------------------------------------------- prefill
+
+def check_prefill_dense_causal(seed=12, S=256, L=32, D=16, G=2):
+    """When every visible chunk is selected the block-sparse prefill is plain
+    causal attention: fp64 SDPA with is_causal=True."""
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((G, S, D))
+    K = rng.standard_normal((S, D))
+    V = rng.standard_normal((S, D))
+    ref = _sdpa(Q, np.broadcast_to(K, (G, S, D)), np.broadcast_to(V, (G, S, D)),
+                scale=0.3, is_causal=True)
+    for t in range(S // L):
+        for g in range(G):
+            o = O.prefill_tile(Q[g, t * L:(t + 1) * L], K, V, list(range(t + 1)), L, t * L, 0.3)
+            assert np.allclose(o, ref[g, t * L:(t + 1) * L], rtol=0, atol=1e-12)
+
+
+def check_prefill_masked(seed=13, S=256, L=32, D=16):
+    """A sparse chunk set per tile == fp64 SDPA with an explicit mask keeping
+    the tile's chunks and the causal triangle."""
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((S, D))
+    K = rng.standard_normal((S, D))
+    V = rng.standard_normal((S, D))
+    for t in range(S // L):
+        chunks = sorted({0, t} | set(rng.choice(t + 1, size=min(t + 1, 2), replace=False).tolist()))
+        mask = np.zeros((L, S), dtype=bool)
+        for c in chunks:
+            mask[:, c * L:(c + 1) * L] = True
+        pos = t * L + np.arange(L)
+        mask &= np.arange(S)[None, :] <= pos[:, None]
+        ref = _sdpa(Q[None, t * L:(t + 1) * L], K[None], V[None], mask=mask[None], scale=0.5)[0]
+        o = O.prefill_tile(Q[t * L:(t + 1) * L], K, V, chunks, L, t * L, 0.5)
+        assert np.allclose(o, ref, rtol=0, atol=1e-12)
+
+
+ALL_CHECKS = [
+    check_attention_vs_sdpa, check_dense_special_case, check_empty_attention,
+    check_summary_closed_form, check_score_hand_case, check_projection_closed_form,
+    check_tile_mean, check_topk_golden, check_topk_vs_torch_sort, check_topk_invariants,
+    check_topp_golden, check_topp_invariants, check_hier_golden, check_hier_all_metas_is_flat,
+    check_meta_linearity, check_merge_closed_form, check_partition,
+    check_prefill_dense_causal, check_prefill_masked,
+]

@@ -1,0 +1,198 @@
+"""Plant plausible mistakes in the CPU oracle and check that the pins catch
+each one.  Every mutant is a small edit of one oracle function (a dropped
+term, a wrong sign or index, a flipped comparison, a transposed operand); the
+test patches it in with monkeypatch, runs the pins and expects at least one
+to fail.  Nothing here touches a GPU."""
+import math
+
+import numpy as np
+import pytest
+
+import pins
+from oracle import csa_oracle as O
+
+_orig = {name: getattr(O, name) for name in
+         ["attend", "select_topk", "select_topp", "score_chunks", "lse_merge",
+          "causal_attend", "meta_summaries", "chunk_summaries", "select_hier",
+          "forced_set", "topp_probs", "decode_partition", "tile_mean_q"]}
+
+
+def attend_no_scale(q, K, V, tokens, scale):
+    return _orig["attend"](q, K, V, tokens, 1.0)
+
+
+def attend_no_max_shift_wrong_lse(q, K, V, tokens, scale):
+    o, lse = _orig["attend"](q, K, V, tokens, scale)
+    return o, lse - math.log(max(len(tokens), 1)) * 0 + 1e-3  # lse off by a constant
+
+
+def attend_last_token_dropped(q, K, V, tokens, scale):
+    return _orig["attend"](q, K, V, tokens[:-1], scale)
+
+
+def topk_ties_to_higher_index(scores, k_free, n_sink, n_local, n_valid=None):
+    scores = np.asarray(scores, dtype=np.float64)
+    v = len(scores) if n_valid is None else int(n_valid)
+    Fs = O.forced_set(v, n_sink, n_local)
+    cand = [c for c in range(v) if c not in Fs]
+    order = sorted(cand, key=lambda c: (-scores[c], -c))
+    return sorted(Fs | set(order[:k_free])), math.inf
+
+
+def topk_forced_inside_k(scores, k_free, n_sink, n_local, n_valid=None):
+    v = len(scores) if n_valid is None else int(n_valid)
+    nf = len(O.forced_set(v, n_sink, n_local))
+    return _orig["select_topk"](scores, max(k_free - nf, 0), n_sink, n_local, n_valid)
+
+
+def topk_ascending(scores, k_free, n_sink, n_local, n_valid=None):
+    return _orig["select_topk"](-np.asarray(scores, dtype=np.float64), k_free, n_sink,
+                                n_local, n_valid)
+
+
+def forced_local_off_by_one(n_valid, n_sink, n_local):
+    s = set(range(min(n_sink, n_valid)))
+    s.update(range(max(n_valid - n_local - 1, 0), n_valid - 1))
+    return s
+
+
+def topp_strict(scores, logit_scale, p, budget, n_sink, n_local):
+    # '>' instead of '>=': nudge p up by one ulp
+    return _orig["select_topp"](scores, logit_scale, np.nextafter(p, 2.0), budget, n_sink, n_local)
+
+
+def topp_cap_after_union(scores, logit_scale, p, budget, n_sink, n_local):
+    nf = len(O.forced_set(len(scores), n_sink, n_local))
+    return _orig["select_topp"](scores, logit_scale, p, max(budget - nf, 0), n_sink, n_local)
+
+
+def topp_probs_no_scale(scores, logit_scale):
+    return _orig["topp_probs"](scores, 1.0)
+
+
+def score_first_head_only(q, summ, Hkv, proj=None):
+    q = np.array(q, dtype=np.float64)
+    G = q.shape[2] // Hkv
+    for h in range(Hkv):
+        q[:, :, h * G + 1:(h + 1) * G] = 0.0
+    return _orig["score_chunks"](q, summ, Hkv, proj)
+
+
+def score_proj_transposed(q, summ, Hkv, proj=None):
+    if proj is None:
+        return _orig["score_chunks"](q, summ, Hkv, None)
+    P = np.asarray(proj)
+    PP = P @ P.T  # use the D x D Gram matrix's wrong side: q P P^T P^T ...
+    qq = np.einsum("bnhd,de->bnhe", np.asarray(q, dtype=np.float64), PP / np.abs(PP).max())
+    return _orig["score_chunks"](qq, summ, Hkv, proj)
+
+
+def merge_plain_average(o_part, lse_part):
+    o_part = np.asarray(o_part)
+    lse_part = np.asarray(lse_part)
+    o, lse = _orig["lse_merge"](o_part, lse_part)
+    valid = lse_part > -math.inf
+    avg = (o_part * valid[..., None]).sum(axis=1) / np.maximum(valid.sum(axis=1), 1)[:, None]
+    return avg, lse
+
+
+def merge_reads_empty(o_part, lse_part):
+    lse_part = np.where(np.asarray(lse_part) == -math.inf, 0.0, lse_part)  # zero-initialised slot
+    return _orig["lse_merge"](o_part, lse_part)
+
+
+def causal_off_by_one(Q_rows, k, v, key_pos, q_start, scale):
+    return _orig["causal_attend"](Q_rows, k, v, np.asarray(key_pos) + 1, q_start, scale)
+
+
+def causal_no_mask(Q_rows, k, v, key_pos, q_start, scale):
+    return _orig["causal_attend"](Q_rows, k, v, np.zeros_like(np.asarray(key_pos)), q_start, scale)
+
+
+def meta_sum_not_mean(summ, Gm):
+    return _orig["meta_summaries"](summ, Gm) * Gm
+
+
+def summaries_first_row(K, L, proj=None):
+    K = np.asarray(K, dtype=np.float64)
+    T, D = K.shape[-2:]
+    C = T // L
+    m = K[..., : C * L, :].reshape(K.shape[:-2] + (C, L, D))[..., 0, :]
+    return m if proj is None else m @ proj
+
+
+def hier_forced_in_pool(q_group, meta, summ, Gm, top_meta, k_free, n_sink, n_local):
+    res, a, b = _orig["select_hier"](q_group, meta, summ, Gm, top_meta, k_free, n_sink, n_local)
+    Fs = O.forced_set(summ.shape[0], n_sink, n_local)
+    free = [c for c in res if c not in Fs]
+    return sorted(Fs | set(free[: max(k_free - len(Fs), 0)])), a, b
+
+
+def hier_meta_ties_high(q_group, meta, summ, Gm, top_meta, k_free, n_sink, n_local):
+    return _orig["select_hier"](q_group, meta[::-1].copy(), summ, Gm, top_meta, k_free,
+                                n_sink, n_local)
+
+
+def partition_ceil(n_chunks, n_parts):
+    N = sum(n_chunks)
+    step = -(-N // n_parts) if n_parts else N
+    out, base = [], 0
+    for n in n_chunks:
+        spl, pos = [], 0
+        while pos < n:
+            nxt = min(n, pos + max(step, 1))
+            spl.append((pos, nxt))
+            pos = nxt
+        out.append(spl)
+        base += n
+    return out
+
+
+def tile_mean_first_row(Q, tile_m):
+    Q = np.asarray(Q, dtype=np.float64)
+    return Q[:, ::tile_m]
+
+
+MUTANTS = [
+    ("attend", attend_no_scale),
+    ("attend", attend_no_max_shift_wrong_lse),
+    ("attend", attend_last_token_dropped),
+    ("select_topk", topk_ties_to_higher_index),
+    ("select_topk", topk_forced_inside_k),
+    ("select_topk", topk_ascending),
+    ("forced_set", forced_local_off_by_one),
+    ("select_topp", topp_strict),
+    ("select_topp", topp_cap_after_union),
+    ("topp_probs", topp_probs_no_scale),
+    ("score_chunks", score_first_head_only),
+    ("score_chunks", score_proj_transposed),
+    ("lse_merge", merge_plain_average),
+    ("lse_merge", merge_reads_empty),
+    ("causal_attend", causal_off_by_one),
+    ("causal_attend", causal_no_mask),
+    ("meta_summaries", meta_sum_not_mean),
+    ("chunk_summaries", summaries_first_row),
+    ("select_hier", hier_forced_in_pool),
+    ("select_hier", hier_meta_ties_high),
+    ("decode_partition", partition_ceil),
+    ("tile_mean_q", tile_mean_first_row),
+]
+
+
+def _pins_fail():
+    for check in pins.ALL_CHECKS:
+        try:
+            check()
+        except (AssertionError, ValueError, IndexError):
+            return True
+    return False
+
+
+@pytest.mark.parametrize("name,mutant", MUTANTS, ids=lambda x: getattr(x, "__name__", x))
+def test_mutant_is_caught(monkeypatch, name, mutant):
+    monkeypatch.setattr(O, name, mutant)
+    assert _pins_fail(), f"no pin caught the planted mistake {mutant.__name__}"
+
+
+def test_unmutated_oracle_passes():
+    assert not _pins_fail()
