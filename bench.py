@@ -1,0 +1,500 @@
+"""Benchmark of query-adaptive chunk-sparse attention on B200.
+
+Headline: one decode step (score -> top-p select -> mixed full/sparse split-K
+decode -> LSE merge) on the 128K-token workload (B=1, 32 query / 8 KV heads,
+D=128, chunks of 128, top-p 0.9 capped at 256 chunks, KV heads 0-1 full),
+reported as µs/step (device time, CUDA events, CUDA-graph replay, L2 flushed
+between steps) with the HBM GB/s of the step and a roofline entry for the
+decode kernel.  The other workloads (top-k 32K, hierarchical 1M, tiny fp32,
+block-sparse prefill 32K in TFLOP/s) ride along under "workloads".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs its own replica (units shard across ranks with no collective on the data
+path) and rank 0 prints the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from query_adaptive_chunk_b200 import synth  # noqa: E402
+
+METRIC = "sparse-decode µs/step + HBM GB/s (% of peak) at 128K ctx; prefill TFLOP/s"
+HEADLINE = synth.TOPP_128K
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def dist_max(x: float, world: int, device) -> float:
+    """Max of a float over all ranks (identity for one rank)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_sum(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Each rank draws its own replica of the workload (weak scaling)."""
+    return w.scaled(seed=w.seed + 100 * rank) if rank else w
+
+
+# ---------------------------------------------------------------- measurement helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = f"/tmp/csa_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def file_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, name: str):
+    """DRAM traffic per launch recorded from an ncu capture, if the kernel
+    source has not changed since (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(name)
+    if not e or e.get("source_hash") != file_hash(kernel_file):
+        return None
+    return e.get("bytes_per_launch")
+
+
+def decoder_for(w, inp):
+    from query_adaptive_chunk_b200.steps import SparseDecoder
+    return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
+                         n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
+                         budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta)
+
+
+def selected_bytes(w, dec) -> tuple:
+    """(selected KV bytes, summary bytes) the step must read, from the actual
+    index counts (full heads: every chunk)."""
+    cnt = dec.count.cpu().tolist()
+    elt = 2 if w.dtype == "bf16" else 4
+    n = 0
+    for u, c in enumerate(cnt):
+        n += w.C if (u % w.Hkv) in w.full_heads else c
+    kv = n * w.L * w.D * elt * 2
+    U_sparse = sum(1 for u in range(w.B * w.Hkv) if (u % w.Hkv) not in w.full_heads)
+    if w.select == "hier":
+        summ = U_sparse * (w.C // w.Gm + w.top_meta * w.Gm) * w.D * 4
+    else:
+        Ds = w.proj_rank or w.D
+        summ = U_sparse * w.C * Ds * 4
+    return kv, summ, n
+
+
+def _ext_event():
+    try:
+        return torch.cuda.Event(enable_timing=True, external=True)
+    except TypeError:
+        return None
+
+
+def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
+    """Device time of `steps` decode steps (L2 flushed before each), with the
+    decode kernel's own duration from events around its launch."""
+    inp = synth.make_decode_inputs(w, device="cuda")
+    dec = decoder_for(w, inp)
+    q = inp["q"]
+    for _ in range(warmup):
+        dec.step(q)
+    torch.cuda.synchronize()
+    ev = [_ext_event() for _ in range(4)]
+    use_graph = graph and all(e is not None for e in ev)
+    g = None
+    if use_graph:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            dec.step(q)  # warm the side stream
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            ev[0].record()
+            dec.select_chunks(q)
+            ev[1].record()
+            from query_adaptive_chunk_b200 import csa
+            csa.csa_sparse_decode(q, dec.K, dec.V, dec.dtype, dec.idx, dec.count, dec.kmax,
+                                  dec.head_full, dec.B, dec.Hq, dec.Hkv, dec.D, dec.T, dec.L,
+                                  dec.scale, dec.P, dec.max_splits, dec.o_part, dec.lse_part)
+            ev[2].record()
+            csa.csa_lse_merge(dec.o_part, dec.lse_part, dec.B * dec.Hq, dec.max_splits, dec.D,
+                              dec.out, 0, dec.lse)
+            ev[3].record()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+    step_ms, dec_ms = [], []
+    for _ in range(steps):
+        flush()
+        if use_graph:
+            g.replay()
+            torch.cuda.synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[3]))
+            dec_ms.append(ev[1].elapsed_time(ev[2]))
+        else:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record()
+            dec.select_chunks(q)
+            e[1].record()
+            from query_adaptive_chunk_b200 import csa
+            csa.csa_sparse_decode(q, dec.K, dec.V, dec.dtype, dec.idx, dec.count, dec.kmax,
+                                  dec.head_full, dec.B, dec.Hq, dec.Hkv, dec.D, dec.T, dec.L,
+                                  dec.scale, dec.P, dec.max_splits, dec.o_part, dec.lse_part)
+            e[2].record()
+            csa.csa_lse_merge(dec.o_part, dec.lse_part, dec.B * dec.Hq, dec.max_splits, dec.D,
+                              dec.out, 0, dec.lse)
+            e[3].record()
+            torch.cuda.synchronize()
+            step_ms.append(e[0].elapsed_time(e[3]))
+            dec_ms.append(e[1].elapsed_time(e[2]))
+    kv, summ, n_chunks = selected_bytes(w, dec)
+    res = {"step_ms": step_ms, "decode_ms": dec_ms, "kv_bytes": kv, "summ_bytes": summ,
+           "chunks": n_chunks, "graph": use_graph, "dec": dec, "inp": inp}
+    return res
+
+
+def time_e2e(w, dec, inp, steps: int, flush):
+    """Same step through the public API with the query coming from pinned
+    host memory and the output read back to the host, per step."""
+    q_host = inp["q"].cpu().pin_memory()
+    out_host = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    q_dev = torch.empty_like(inp["q"])
+    ms = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        q_dev.copy_(q_host, non_blocking=True)
+        dec.step(q_dev)
+        out_host.copy_(dec.out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return ms, q_host.numel() * q_host.element_size(), out_host.numel() * out_host.element_size()
+
+
+def time_prefill(w, steps: int, warmup: int, flush):
+    from query_adaptive_chunk_b200.steps import BlockSparsePrefill
+    inp = synth.make_prefill_inputs(w, device="cuda")
+    pf = BlockSparsePrefill(inp["Q"], inp["K"], inp["V"], tile_m=w.tile_m, L=w.L, k_free=w.k_free,
+                            n_sink=w.n_sink, n_local=w.n_local)
+    for _ in range(warmup):
+        pf.step()
+    torch.cuda.synchronize()
+    sel_ms, att_ms = [], []
+    for _ in range(steps):
+        flush()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        pf.select_chunks()
+        e[1].record()
+        pf.attend()
+        e[2].record()
+        torch.cuda.synchronize()
+        sel_ms.append(e[0].elapsed_time(e[1]))
+        att_ms.append(e[1].elapsed_time(e[2]))
+    cnt = pf.count.cpu()
+    blocks = int(cnt.sum())
+    flops = blocks * w.G * 2 * (2 * w.tile_m * w.L * w.D)
+    return {"select_ms": sel_ms, "attend_ms": att_ms, "blocks": blocks, "flops": flops}
+
+
+def oracle_decode_seconds(w, inp, max_seconds: float = 20.0, max_steps: int = 5):
+    """The CPU oracle's per-step work (score + select + attention, summaries
+    precomputed) on this workload, single-threaded, a bounded number of steps."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import csa_oracle as O
+    from oracle import pipeline as OP
+    q, K, V = inp["q"].cpu(), inp["K"].cpu(), inp["V"].cpu()
+    proj = inp.get("proj")
+    projn = None if proj is None else OP.to_np(proj)
+    units = synth.decode_units(w)
+    with threadpool_limits(1):
+        summ = {u: OP.unit_summaries(K[u[0], u[1]], w.L, projn) for u in units
+                if u[1] not in w.full_heads}
+        times = []
+        t_start = time.perf_counter()
+        while len(times) < max_steps and (time.perf_counter() - t_start) < max_seconds:
+            t0 = time.perf_counter()
+            for (b, h) in units:
+                qg = OP.to_np(q[b, h * w.G:(h + 1) * w.G])
+                if h in w.full_heads:
+                    chunks = list(range(w.C))
+                else:
+                    s = O.score_chunks(qg[None, None], summ[(b, h)][None, None], 1, projn)[0, 0, 0]
+                    if w.select == "topp":
+                        chunks, _, _ = O.select_topp(s, 1.0 / math.sqrt(w.D), w.p, w.budget,
+                                                     w.n_sink, w.n_local)
+                    else:
+                        chunks, _ = O.select_topk(s, w.k_free, w.n_sink, w.n_local)
+                tok = O.chunk_tokens(chunks, w.L)
+                ti = torch.as_tensor(tok)
+                O.attend(qg, OP.to_np(K[b, h][ti]), OP.to_np(V[b, h][ti]),
+                         torch.arange(len(tok)).numpy(), w.scale)
+            times.append(time.perf_counter() - t0)
+    return times
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args):
+    """The CPU oracle timed as the reference arm, on the headline workload."""
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    w = HEADLINE
+    inp = synth.make_decode_inputs(w, device="cpu")
+    t = oracle_decode_seconds(w, inp, max_seconds=1e9, max_steps=args.warmup + args.steps)
+    t = t[args.warmup:] if len(t) > args.warmup else t
+    us = 1e6 * statistics.mean(t)
+    line = {"impl": "reference", "metric": METRIC, "value": us, "unit": "us/step",
+            "n_gpus": args.gpus, "steps": len(t), "warmup": args.warmup,
+            "ms_per_step": us / 1000, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                       "ctx": w.T, "L": w.L, "p": w.p, "budget": w.budget,
+                       "full_heads": list(w.full_heads)},
+            "cpu_baseline": {"value": us, "unit": "us/step", "cores": 1, "kind": "oracle",
+                             "sample": f"{len(t)} whole decode steps of {w.name} (all 8 units), "
+                                       "summaries precomputed, numpy fp64 single-threaded"},
+            "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = dist_init(world, "nccl")
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    w = rank_workload(HEADLINE, rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if "CUDA_VISIBLE_DEVICES" in os.environ else local
+    with ClockSampler(gpu_index) as clk:
+        r = time_decode(w, args.steps, args.warmup, flush)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = clk.summary()
+    step_us_local = 1000 * statistics.mean(r["step_ms"])
+    step_us = dist_max(step_us_local, world, dev)
+    dec_us = 1000 * statistics.mean(r["decode_ms"])
+    kv, summ = r["kv_bytes"], r["summ_bytes"]
+    step_gbs = (kv + summ) / (step_us * 1e-6) / 1e9
+    agg_gbs = dist_sum((kv + summ) / (step_us_local * 1e-6) / 1e9, world, dev)
+    dec_gbs = kv / (dec_us * 1e-6) / 1e9
+    e2e_ms, h2d, d2h = time_e2e(w, r["dec"], r["inp"], max(5, args.steps // 2), flush)
+    e2e_us = dist_max(1000 * statistics.mean(e2e_ms), world, dev)
+    extra = {}
+    if rank == 0 and not args.headline_only:
+        extra = other_workloads(args, flush, peaks)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t = oracle_decode_seconds(w, r["inp"], max_seconds=20.0, max_steps=5)
+        cpu = {"value": 1e6 * statistics.mean(t), "unit": "us/step", "cores": 1, "kind": "oracle",
+               "sample": f"{len(t)} whole decode steps of {w.name} (all {w.B * w.Hkv} units), "
+                         "summaries precomputed, numpy fp64 single-threaded"}
+    traffic = recorded_traffic(os.path.join(ROOT, "query_adaptive_chunk_b200", "csrc", "decode.cu"),
+                               "decode_bf16_kernel<128,128>/" + w.name)
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": round(step_us, 3), "unit": "us/step", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_us / 1000, 6),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "ctx": w.T,
+                   "L": w.L, "select": "top-p p=0.9 cap 256 + sink + 2 local",
+                   "full_heads": list(w.full_heads), "proj_rank": w.proj_rank,
+                   "l2": "flushed before every step (256 MB write)",
+                   "timing": "CUDA-graph replay, events inside the graph" if r["graph"]
+                             else "direct launches, CUDA events",
+                   "parallelism": f"replicas x{world} (units shard, no collective)"},
+        "hbm_gbs": round(step_gbs, 1), "hbm_frac_of_measured": round(step_gbs / peaks["hbm_gbs"], 4),
+        "hbm_frac_of_8tbs_nominal": round(step_gbs / 8000.0, 4),
+        "aggregate_hbm_gbs": round(agg_gbs, 1),
+        "step_bytes": {"selected_kv": kv, "summaries": summ, "chunks": r["chunks"]},
+        "roofline": {"kernel": "decode_bf16_kernel<128,128>", "bound": "hbm",
+                     "achieved": round(dec_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(dec_gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
+                     "algorithmic_bytes": kv, "duration_us": round(dec_us, 3),
+                     "peak_source": peaks["source"]},
+        "e2e": {"value": round(e2e_us, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "workloads": extra,
+    }
+    print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def other_workloads(args, flush, peaks):
+    out = {}
+    steps = max(5, args.steps // 2)
+    for w in (synth.TOPK_32K, synth.HIER_1M, synth.TINY_F32):
+        r = time_decode(w, steps, args.warmup, flush)
+        us = 1000 * statistics.mean(r["step_ms"])
+        dus = 1000 * statistics.mean(r["decode_ms"])
+        byt = r["kv_bytes"] + r["summ_bytes"]
+        out[w.name] = {"us_per_step": round(us, 3), "step_gbs": round(byt / (us * 1e-6) / 1e9, 1),
+                       "step_frac_of_measured_hbm": round(byt / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                       "decode_us": round(dus, 3),
+                       "decode_gbs": round(r["kv_bytes"] / (dus * 1e-6) / 1e9, 1),
+                       "selected_kv_bytes": r["kv_bytes"], "summary_bytes": r["summ_bytes"]}
+        del r
+        torch.cuda.empty_cache()
+    w = synth.PREFILL_32K
+    r = time_prefill(w, steps, args.warmup, flush)
+    att_ms = statistics.mean(r["attend_ms"])
+    tflops = r["flops"] / (att_ms * 1e-3) / 1e12
+    out[w.name] = {"attend_ms": round(att_ms, 4), "select_ms": round(statistics.mean(r["select_ms"]), 4),
+                   "executed_blocks": r["blocks"], "flops": r["flops"],
+                   "tflops": round(tflops, 1),
+                   "frac_of_measured_bf16": round(tflops / peaks["bf16_tflops"], 4),
+                   "frac_of_sustained_bf16": round(tflops / peaks["bf16_tflops_sustained"], 4)}
+    return out
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

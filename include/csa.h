@@ -1,0 +1,255 @@
+/*
+ * csa.h — C ABI of libcsa.so: query-adaptive chunk-sparse attention on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The method (pages of the surveyed subject):
+ *   - the KV sequence is cut into chunks of L tokens, each summarised by one
+ *     key (SSA summary, aitrends.kr/articles/69798, section "기술 상세";
+ *     HiLS review "Hierarchical Sparse Attention Done Right", section 1,
+ *     "Landmark Token"); this library summarises a chunk by the mean of its
+ *     keys, optionally projected to a low rank (RTPurbo review "Full Attention
+ *     Strikes Back", section 1, "Low-dimensional Projection");
+ *   - each chunk is scored by the inner product of the query with its
+ *     summary, s = q^T k_summary (SSA summary, section "방법론"), summed over
+ *     the query heads of a GQA group (HiLS review, section 1, "GQA");
+ *   - a chunk set is picked per (sequence, KV head) by top-k (SSA summary,
+ *     "방법론"), dynamic top-p (RTPurbo review, section 1, "Dynamic Top-p
+ *     Selection") or two-level meta-chunk -> chunk selection (SSA summary,
+ *     "핵심 기여", H-SSA), always keeping sink and local chunks;
+ *   - exact softmax attention runs over the raw KV of the chosen chunks as
+ *     split-K partials from a compact index list, combined afterwards (SSA
+ *     summary, "핵심 기여", decode kernel); full-attention and sparse heads run
+ *     in one launch (Elastic Attention summary, section 2.3, fused kernel);
+ *   - prefill runs block-sparse causal attention over a chunk set per query
+ *     tile (SSA summary, "핵심 기여", block-skip prefill; HiLS review, section 3,
+ *     union chunks of adjacent queries).
+ *
+ * Conventions for every call:
+ *   - Every data pointer is a DEVICE pointer (cudaMalloc'd, or managed)
+ *     owned by the caller.  The library allocates nothing, frees nothing and
+ *     never blocks the host; each call enqueues kernels on `stream` (a
+ *     cudaStream_t; NULL = legacy default stream) and returns.
+ *   - Tensors are dense, row-major (last index fastest), in the layouts given
+ *     per call.  K/V caches are [B, Hkv, T, D]: chunk c of head (b, h) is the
+ *     contiguous block of rows [c*L, (c+1)*L).
+ *   - Pointers must be 16-byte aligned.  A host pointer, a NULL required
+ *     pointer, a non-positive size, or an inconsistent shape is rejected with
+ *     CSA_ERR_INVALID_ARG before anything is launched; shapes outside what the
+ *     kernels implement are rejected with CSA_ERR_UNSUPPORTED.  On any error
+ *     nothing is enqueued, and csa_last_error_string() (thread-local) says why.
+ *   - Faults the kernels detect on the device (an index out of range, a wait
+ *     that exceeded its time limit) do not trap: the kernel records a code in
+ *     a device-side status word and carries on or returns.
+ *     csa_check_device_status() reads and clears it.
+ *   - Calls on one stream are ordered; the library keeps no state between
+ *     calls other than the device status word and process-wide settings
+ *     (wait limit).
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum csa_status {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,  /* NULL / host pointer, bad size, misalignment, kmax too small */
+  CSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. D not in {64,128}) */
+  CSA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  CSA_ERR_TIMEOUT = 4,      /* a device-side bounded wait expired (read back later) */
+  CSA_ERR_DEVICE_INDEX = 5  /* a kernel met a chunk index or count out of range */
+} csa_status;
+
+typedef enum csa_dtype { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype;
+
+typedef void* csa_stream; /* a cudaStream_t */
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+CSA_API int csa_version(void);
+
+/* Why the last call on this thread failed ("" after success). */
+CSA_API const char* csa_last_error_string(void);
+
+/* Waits for `stream` to finish, then reads and clears the device status
+ * word of the current device: CSA_OK, CSA_ERR_TIMEOUT or CSA_ERR_DEVICE_INDEX
+ * (or CSA_ERR_CUDA if the synchronisation itself failed).  This is the one
+ * call that blocks the host. */
+CSA_API csa_status csa_check_device_status(csa_stream stream);
+
+/* Time limit of every spin-wait inside the kernels, in nanoseconds (process
+ * wide; default 2e9, or the CSA_WAIT_LIMIT_NS environment variable).  A wait
+ * that exceeds it records CSA_ERR_TIMEOUT and the kernel returns. */
+CSA_API void csa_set_wait_limit_ns(uint64_t ns);
+CSA_API uint64_t csa_get_wait_limit_ns(void);
+
+/* Diagnostic (no counterpart in the pages): launches one CTA that waits on
+ * an mbarrier nothing ever arrives on, with a limit of `limit_ns`.  The wait
+ * runs out, the kernel records CSA_ERR_TIMEOUT and returns, and the next
+ * csa_check_device_status() reports it.  Shows that a stuck wait ends as a
+ * status code, not a hang or a trap, and that the context stays usable. */
+CSA_API csa_status csa_selftest_wait_timeout(uint64_t limit_ns, csa_stream stream);
+
+/* ---------------------------------------------------------------- a0
+ * Chunk summaries (precompute, once per cache).
+ * summ[b,h,c,:] = (1/L) * sum_{j<L} K[b,h,c*L+j,:]            (proj == NULL, Ds = D)
+ * summ[b,h,c,r] = sum_d proj[d,r] * (1/L) sum_j K[b,h,c*L+j,d]  (proj [D,R] fp32, Ds = R)
+ * Basis: chunk summary keys (SSA summary "기술 상세"; HiLS review section 1)
+ * with the chunk mean standing in for a learned gist/landmark key; low-rank
+ * projection (RTPurbo review section 1).
+ *   K     [B, Hkv, T, D] of `dtype`;  summ [B, Hkv, T/L, Ds] fp32 (output)
+ *   D in {64, 128}, L >= 1, T % L == 0, R in {16, 32, 64, 128} when proj != NULL.
+ * fp32 accumulation in row order. */
+CSA_API csa_status csa_chunk_summaries(const void* K, csa_dtype dtype, int B, int Hkv, int64_t T,
+                               int D, int L, const float* proj, int R, float* summ,
+                               csa_stream stream);
+
+/* Meta-summaries for two-level selection (H-SSA meta-gist stand-in, SSA
+ * summary "핵심 기여" and glossary "Hierarchical Gist-of-Gist"):
+ * meta[b,h,m,:] = (1/Gm) * sum_{j<Gm} summ[b,h,m*Gm+j,:].
+ *   summ [B, Hkv, C, Ds] fp32 -> meta [B, Hkv, C/Gm, Ds] fp32;  C % Gm == 0, Ds <= 1024. */
+CSA_API csa_status csa_meta_summaries(const float* summ, int B, int Hkv, int C, int Ds, int Gm,
+                              float* meta, csa_stream stream);
+
+/* ---------------------------------------------------------------- a7
+ * Tile-mean queries for prefill (HiLS review section 3: adjacent queries
+ * share one chunk union):  qbar[b,t,h,:] = (1/tile_m) sum_{i<tile_m} Q[b,t*tile_m+i,h,:].
+ *   Q [B, S, Hq, D] of `dtype` -> qbar [B, S/tile_m, Hq, D] fp32;  S % tile_m == 0, D <= 1024. */
+CSA_API csa_status csa_tile_mean_q(const void* Q, csa_dtype dtype, int B, int S, int Hq, int D,
+                           int tile_m, float* qbar, csa_stream stream);
+
+/* ---------------------------------------------------------------- a1
+ * Chunk scores (SSA summary "방법론": s_{t,m} = q_t^T k_{g_m}; group-level
+ * selection for GQA, HiLS review section 1):
+ *   scores[b,h,n,c] = sum_{g<G} qt[b,n,h*G+g,:] . summ[b,h,c,:],   G = Hq/Hkv,
+ *   qt = q (proj == NULL, Ds = D) or qt = proj^T q (proj [D,R] fp32, Ds = R).
+ *   q      [B, Nq, Hq, D] of `q_dtype` (decode: Nq = 1; prefill: the tile means, Nq = tiles)
+ *   summ   [B, Hkv, C, Ds] fp32;  scores [B, Hkv, Nq, C] fp32 (output)
+ *   head_full  NULL or [Hkv] bytes: rows of heads with head_full[h] != 0 are not
+ *              written (those heads attend to every chunk).
+ *   causal_tile_m, causal_L: 0, 0 for no mask; otherwise row n sees the chunks
+ *              c < ((n+1)*causal_tile_m - 1)/causal_L + 1 and the others get -inf.
+ *   Ds in {16, 32, 64, 128}; D <= 1024; Hq % Hkv == 0. */
+CSA_API csa_status csa_score_chunks(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                            const float* summ, int B, int Nq, int Hq, int Hkv, int D, int C,
+                            const uint8_t* head_full, int causal_tile_m, int causal_L,
+                            float* scores, csa_stream stream);
+
+/* ---------------------------------------------------------------- a2
+ * Top-k chunk selection per unit (SSA summary "방법론"; the compact list of
+ * the decode kernel, "핵심 기여").  Unit u sees chunks [0, v) with
+ * v = n_valid ? n_valid[u] : C.  Forced set F = the first n_sink and the last
+ * n_local of [0, v).  The other chunks are ranked by (score desc, index asc;
+ * -0 == +0) and the first k_free are kept.  Result F U top, ascending.
+ *   scores [U, C] fp32 (finite);  n_valid NULL or [U] int32 in [0, C]
+ *   idx [U, kmax] int32 (output, ascending, unused slots = -1);  count [U] int32 (output)
+ *   kmax >= min(C, k_free + n_sink + n_local);  C <= 32768. */
+CSA_API csa_status csa_select_topk(const float* scores, int U, int C, const int32_t* n_valid,
+                           int k_free, int n_sink, int n_local, int32_t* idx, int32_t* count,
+                           int kmax, csa_stream stream);
+
+/* ---------------------------------------------------------------- a3
+ * Dynamic top-p selection per unit (RTPurbo review section 1, "Dynamic Top-p
+ * Selection"; chunk mass from the HiLS review's chunk-mass surrogate):
+ * pi_c = softmax_c(scores[u,c] * logit_scale) over all C chunks; chunks
+ * ordered by (pi desc, index asc); n_p = smallest n with sum of the first n
+ * pi >= p; the first min(n_p, budget) are kept, then F (first n_sink, last
+ * n_local) is added.  Result ascending.
+ *   scores [U, C] fp32;  idx [U, kmax] int32, count [U] int32 (outputs)
+ *   n_p_out NULL or [U] int32: n_p when n_p <= budget, else budget + 1
+ *   0 < p <= 1;  1 <= budget <= 2048;  kmax >= min(C, budget + n_sink + n_local);  C <= 32768. */
+CSA_API csa_status csa_select_topp(const float* scores, int U, int C, float logit_scale, float p,
+                           int budget, int n_sink, int n_local, int32_t* idx, int32_t* count,
+                           int kmax, int32_t* n_p_out, csa_stream stream);
+
+/* ---------------------------------------------------------------- a4
+ * Two-level selection per unit (b, h) (SSA summary "핵심 기여", H-SSA:
+ * coarse selection on meta-gists, then re-scoring inside the kept segments):
+ * meta score = sum_g q[b,h*G+g,:] . meta[b,h,m,:]; keep the top_meta metas by
+ * (score desc, index asc); score their children the same way; among children
+ * not in F keep the k_free best; add F (first n_sink, last n_local of [0, C)).
+ *   q [B, Hq, D] of `q_dtype`;  meta [B, Hkv, C/Gm, D] fp32;  summ [B, Hkv, C, D] fp32
+ *   idx [B*Hkv, kmax] int32, count [B*Hkv] int32 (outputs, ascending)
+ *   D in {64, 128};  top_meta * Gm <= 8192;  C / Gm <= 8192;  C <= 32768;
+ *   kmax >= min(C, k_free + n_sink + n_local). */
+CSA_API csa_status csa_select_hier(const void* q, csa_dtype q_dtype, const float* meta,
+                           const float* summ, int B, int Hq, int Hkv, int D, int C, int Gm,
+                           int top_meta, int k_free, int n_sink, int n_local, int32_t* idx,
+                           int32_t* count, int kmax, csa_stream stream);
+
+/* ---------------------------------------------------------------- a5
+ * Sparse split-K decode (SSA summary "핵심 기여": compact index list + split-K
+ * partial attention; Elastic Attention summary section 2.3: full and sparse
+ * heads in one launch).
+ * Unit u = b*Hkv + h owns the chunk list idx[u, 0:count[u]] (or, if
+ * head_full[h] != 0, every chunk 0..T/L-1; idx/count of that unit are not
+ * read).  All units' lists are laid end to end (unit-major), N chunks in all,
+ * and cut into num_parts pieces [floor(c*N/P), floor((c+1)*N/P)); the s-th
+ * non-empty intersection of unit u with a piece is split s of that unit.  For
+ * every query head g of the unit and every split s:
+ *   o_part[b, h*G+g, s, :] = sum_j softmax(scale * q.k_j) v_j over the split's tokens,
+ *   lse_part[b, h*G+g, s]  = log sum_j exp(scale * q.k_j)          (natural log)
+ * and slots s >= the unit's split count get lse = -inf (their o is not written).
+ *   q [B, Hq, D], K/V [B, Hkv, T, D] of `dtype` (CSA_BF16: bf16 tensor-core
+ *   dot products with fp32 accumulation; CSA_F32: fp32 throughout)
+ *   idx [B*Hkv, kmax] int32 in [0, T/L);  count [B*Hkv] int32 in [0, kmax]
+ *   num_parts: 0 = csa_decode_default_parts(); max_splits >= the effective num_parts
+ *   o_part [B, Hq, max_splits, D] fp32;  lse_part [B, Hq, max_splits] fp32 (outputs)
+ *   D in {64, 128};  L in {64, 128};  T % L == 0;  Hq/Hkv in {1, 2, 4, 8};
+ *   B*Hkv <= 4096;  B*Hkv*T < 2^31.
+ * An idx entry out of range or count > kmax records CSA_ERR_DEVICE_INDEX
+ * (the chunk is replaced by chunk 0 / the count clamped) instead of faulting. */
+CSA_API csa_status csa_sparse_decode(const void* q, const void* K, const void* V, csa_dtype dtype,
+                             const int32_t* idx, const int32_t* count, int kmax,
+                             const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T,
+                             int L, float scale, int num_parts, int max_splits, float* o_part,
+                             float* lse_part, csa_stream stream);
+
+/* Number of pieces csa_sparse_decode uses when num_parts == 0, on the
+ * current device (a multiple of the SM count); < 0 on error. */
+CSA_API int csa_decode_default_parts(csa_dtype dtype, int D, int L);
+
+/* ---------------------------------------------------------------- a6
+ * Log-sum-exp merge of split-K partials (SSA summary "핵심 기여": split-K
+ * partials combined):
+ *   lse[r] = log sum_s exp(lse_part[r,s]);  out[r,:] = sum_s exp(lse_part[r,s] - lse[r]) o_part[r,s,:]
+ * over the slots with lse_part > -inf (others are not read; a row with none
+ * gives out = 0, lse = -inf).
+ *   o_part [rows, max_splits, D] fp32;  lse_part [rows, max_splits] fp32
+ *   out [rows, D] of out_dtype (output);  lse_out NULL or [rows] fp32 (output)
+ *   D % 4 == 0, D <= 512. */
+CSA_API csa_status csa_lse_merge(const float* o_part, const float* lse_part, int rows, int max_splits,
+                         int D, void* out, csa_dtype out_dtype, float* lse_out,
+                         csa_stream stream);
+
+/* ---------------------------------------------------------------- a8
+ * Block-sparse causal prefill (SSA summary "핵심 기여": block-skip prefill;
+ * HiLS review section 3: one chunk union per group of adjacent queries).
+ * For query tile t (rows t*tile_m .. +tile_m) and KV head h, the tile's chunk
+ * list is idx[u, 0:count[u]], u = (b*Hkv + h)*(S/tile_m) + t.  Query row i of
+ * head g in the group attends causally to the tokens j of those chunks with
+ * j <= t*tile_m + i:
+ *   O[b, t*tile_m+i, h*G+g, :] = sum_j softmax(scale * q.k_j) v_j   (bf16 out)
+ * Rows with no visible token get 0.  Tensor-core (tcgen05) bf16 products,
+ * fp32 accumulation and softmax.
+ *   Q [B, S, Hq, D] bf16;  K/V [B, Hkv, S, D] bf16;  O [B, S, Hq, D] bf16 (output)
+ *   idx [B*Hkv*(S/tile_m), kmax] int32 ascending in [0, S/L);  count [same] int32
+ *   implemented: D = 128, tile_m = L = 64, Hq/Hkv = 4;  B*Hkv*S < 2^31. */
+CSA_API csa_status csa_block_sparse_prefill(const void* Q, const void* K, const void* V,
+                                    const int32_t* idx, const int32_t* count, int kmax, int B,
+                                    int S, int Hq, int Hkv, int D, int tile_m, int L,
+                                    float scale, void* O, csa_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,185 @@
+"""Python binding of libcsa.so (the C ABI in include/csa.h).
+
+Argument marshalling only: each function has the name and the positional
+arguments of its C counterpart, accepts torch tensors (their data pointers
+are passed), ``None`` for NULL, and an optional ``stream`` (default: torch's
+current CUDA stream).  A non-OK status raises ``CsaError`` with the library's
+message.  Every step of the method runs in the library's CUDA kernels; there
+is no fallback when the library is missing: importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcsa.so")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "csa.h")
+
+CSA_F32, CSA_BF16 = 0, 1
+STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CUDA",
+          4: "CSA_ERR_TIMEOUT", 5: "CSA_ERR_DEVICE_INDEX"}
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m query_adaptive_chunk_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _i64, _f, _u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_uint64
+_SIGS = {
+    "csa_version": (_i, []),
+    "csa_last_error_string": (ctypes.c_char_p, []),
+    "csa_check_device_status": (_i, [_vp]),
+    "csa_set_wait_limit_ns": (None, [_u64]),
+    "csa_get_wait_limit_ns": (_u64, []),
+    "csa_selftest_wait_timeout": (_i, [_u64, _vp]),
+    "csa_chunk_summaries": (_i, [_vp, _i, _i, _i, _i64, _i, _i, _vp, _i, _vp, _vp]),
+    "csa_meta_summaries": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "csa_tile_mean_q": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
+    "csa_score_chunks": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
+                              _vp]),
+    "csa_select_topk": (_i, [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp, _i, _vp]),
+    "csa_select_topp": (_i, [_vp, _i, _i, _f, _f, _i, _i, _i, _vp, _vp, _i, _vp, _vp]),
+    "csa_select_hier": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                             _i, _vp]),
+    "csa_sparse_decode": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i64, _i, _f,
+                               _i, _i, _vp, _vp, _vp]),
+    "csa_decode_default_parts": (_i, [_i, _i, _i]),
+    "csa_lse_merge": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp]),
+    "csa_block_sparse_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                                      _vp, _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def header_functions() -> list:
+    """Names of the functions include/csa.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"CSA_API\s+[\w\s\*]*?\b(csa_\w+)\s*\(", text)))
+
+
+def _p(x):
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return ctypes.c_void_p(x.data_ptr())
+    return ctypes.c_void_p(int(x))
+
+
+def _s(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _dt(d) -> int:
+    if isinstance(d, torch.dtype):
+        return {torch.float32: CSA_F32, torch.bfloat16: CSA_BF16}[d]
+    return int(d)
+
+
+def _check(status: int):
+    if status != 0:
+        raise CsaError(status, lib.csa_last_error_string().decode())
+
+
+def csa_version() -> int:
+    return lib.csa_version()
+
+
+def csa_last_error_string() -> str:
+    return lib.csa_last_error_string().decode()
+
+
+def csa_check_device_status(stream=None) -> None:
+    _check(lib.csa_check_device_status(_s(stream)))
+
+
+def csa_set_wait_limit_ns(ns: int) -> None:
+    lib.csa_set_wait_limit_ns(int(ns))
+
+
+def csa_get_wait_limit_ns() -> int:
+    return lib.csa_get_wait_limit_ns()
+
+
+def csa_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(lib.csa_selftest_wait_timeout(int(limit_ns), _s(stream)))
+
+
+def csa_chunk_summaries(K, dtype, B, Hkv, T, D, L, proj, R, summ, stream=None):
+    _check(lib.csa_chunk_summaries(_p(K), _dt(dtype), B, Hkv, T, D, L, _p(proj), R, _p(summ),
+                                   _s(stream)))
+
+
+def csa_meta_summaries(summ, B, Hkv, C, Ds, Gm, meta, stream=None):
+    _check(lib.csa_meta_summaries(_p(summ), B, Hkv, C, Ds, Gm, _p(meta), _s(stream)))
+
+
+def csa_tile_mean_q(Q, dtype, B, S, Hq, D, tile_m, qbar, stream=None):
+    _check(lib.csa_tile_mean_q(_p(Q), _dt(dtype), B, S, Hq, D, tile_m, _p(qbar), _s(stream)))
+
+
+def csa_score_chunks(q, q_dtype, proj, R, summ, B, Nq, Hq, Hkv, D, C, head_full, causal_tile_m,
+                     causal_L, scores, stream=None):
+    _check(lib.csa_score_chunks(_p(q), _dt(q_dtype), _p(proj), R, _p(summ), B, Nq, Hq, Hkv, D, C,
+                                _p(head_full), causal_tile_m, causal_L, _p(scores), _s(stream)))
+
+
+def csa_select_topk(scores, U, C, n_valid, k_free, n_sink, n_local, idx, count, kmax, stream=None):
+    _check(lib.csa_select_topk(_p(scores), U, C, _p(n_valid), k_free, n_sink, n_local, _p(idx),
+                               _p(count), kmax, _s(stream)))
+
+
+def csa_select_topp(scores, U, C, logit_scale, p, budget, n_sink, n_local, idx, count, kmax,
+                    n_p_out=None, stream=None):
+    _check(lib.csa_select_topp(_p(scores), U, C, logit_scale, p, budget, n_sink, n_local, _p(idx),
+                               _p(count), kmax, _p(n_p_out), _s(stream)))
+
+
+def csa_select_hier(q, q_dtype, meta, summ, B, Hq, Hkv, D, C, Gm, top_meta, k_free, n_sink,
+                    n_local, idx, count, kmax, stream=None):
+    _check(lib.csa_select_hier(_p(q), _dt(q_dtype), _p(meta), _p(summ), B, Hq, Hkv, D, C, Gm,
+                               top_meta, k_free, n_sink, n_local, _p(idx), _p(count), kmax,
+                               _s(stream)))
+
+
+def csa_sparse_decode(q, K, V, dtype, idx, count, kmax, head_full, B, Hq, Hkv, D, T, L, scale,
+                      num_parts, max_splits, o_part, lse_part, stream=None):
+    _check(lib.csa_sparse_decode(_p(q), _p(K), _p(V), _dt(dtype), _p(idx), _p(count), kmax,
+                                 _p(head_full), B, Hq, Hkv, D, T, L, scale, num_parts, max_splits,
+                                 _p(o_part), _p(lse_part), _s(stream)))
+
+
+def csa_decode_default_parts(dtype, D, L) -> int:
+    n = lib.csa_decode_default_parts(_dt(dtype), D, L)
+    if n < 0:
+        raise CsaError(3, csa_last_error_string())
+    return n
+
+
+def csa_lse_merge(o_part, lse_part, rows, max_splits, D, out, out_dtype, lse_out, stream=None):
+    _check(lib.csa_lse_merge(_p(o_part), _p(lse_part), rows, max_splits, D, _p(out),
+                             _dt(out_dtype), _p(lse_out), _s(stream)))
+
+
+def csa_block_sparse_prefill(Q, K, V, idx, count, kmax, B, S, Hq, Hkv, D, tile_m, L, scale, O,
+                             stream=None):
+    _check(lib.csa_block_sparse_prefill(_p(Q), _p(K), _p(V), _p(idx), _p(count), kmax, B, S, Hq,
+                                        Hkv, D, tile_m, L, scale, _p(O), _s(stream)))

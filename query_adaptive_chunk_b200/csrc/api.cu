@@ -1,0 +1,416 @@
+// C ABI of libcsa (declared in include/csa.h): argument validation, error
+// reporting and the launches.  Nothing here allocates device memory.
+#include <algorithm>
+#include <atomic>
+#include <cstdlib>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/csa.h"
+#include "internal.h"
+
+// Device status word: [0] = first error code recorded by a kernel.
+__device__ int g_csa_status[4];
+
+// One thread waits on an mbarrier that never completes its first phase; the
+// bounded wait gives up after e.wait_ns and records DEV_TIMEOUT.
+__global__ void wait_timeout_selftest_kernel(csa::DevErr e) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = csa::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    csa::mbar_init(b, 1);
+    csa::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) csa::mbar_wait(b, 0u, e);
+}
+
+namespace {
+
+thread_local std::string t_err;
+
+std::atomic<uint64_t>& wait_limit() {
+  static std::atomic<uint64_t> v([] {
+    const char* e = std::getenv("CSA_WAIT_LIMIT_NS");
+    if (e && *e) {
+      const unsigned long long x = std::strtoull(e, nullptr, 10);
+      if (x > 0) return static_cast<uint64_t>(x);
+    }
+    return static_cast<uint64_t>(2000000000ull);
+  }());
+  return v;
+}
+
+struct DevState {
+  bool ready = false;
+  int* status = nullptr;
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+std::vector<DevState> g_dev;
+
+csa_status fail(csa_status s, const std::string& why) {
+  t_err = why;
+  return s;
+}
+
+csa_status cuda_fail(cudaError_t e, const char* what) {
+  t_err = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return CSA_ERR_CUDA;
+}
+
+// Per-device set-up (status word address, SM count), once per device.
+csa_status launch_ctx(csa_stream stream, csa::Launch* l) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (static_cast<int>(g_dev.size()) <= dev) g_dev.resize(dev + 1);
+  DevState& st = g_dev[dev];
+  if (!st.ready) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_csa_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    st.status = static_cast<int*>(p);
+    st.num_sms = sms;
+    st.ready = true;
+  }
+  l->stream = static_cast<cudaStream_t>(stream);
+  l->err.word = st.status;
+  l->err.wait_ns = wait_limit().load();
+  l->num_sms = st.num_sms;
+  return CSA_OK;
+}
+
+// A required device pointer: not NULL, 16-byte aligned, device or managed
+// memory of the current device.
+csa_status check_ptr(const void* p, const char* name, bool required = true) {
+  if (p == nullptr) {
+    if (!required) return CSA_OK;
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  }
+  if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " is not 16-byte aligned");
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " is not a CUDA pointer");
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " is not device memory");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (a.type == cudaMemoryTypeDevice && a.device != dev)
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " lives on another device");
+  return CSA_OK;
+}
+
+#define CSA_TRY(x)                     \
+  do {                                 \
+    csa_status _s = (x);               \
+    if (_s != CSA_OK) return _s;       \
+  } while (0)
+
+#define CSA_REQUIRE(cond, msg)                                   \
+  do {                                                           \
+    if (!(cond)) return fail(CSA_ERR_INVALID_ARG, (msg));        \
+  } while (0)
+
+#define CSA_SUPPORT(cond, msg)                                   \
+  do {                                                           \
+    if (!(cond)) return fail(CSA_ERR_UNSUPPORTED, (msg));        \
+  } while (0)
+
+bool valid_dtype(csa_dtype d) { return d == CSA_F32 || d == CSA_BF16; }
+
+csa_status finish(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  t_err.clear();
+  return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_version(void) { return 10000; }
+
+const char* csa_last_error_string(void) { return t_err.c_str(); }
+
+void csa_set_wait_limit_ns(uint64_t ns) { wait_limit().store(ns > 0 ? ns : 1); }
+
+uint64_t csa_get_wait_limit_ns(void) { return wait_limit().load(); }
+
+csa_status csa_check_device_status(csa_stream stream) {
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  cudaError_t e = cudaStreamSynchronize(l.stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int word[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(word, l.err.word, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (word[0] != 0) {
+    int zero[4] = {0, 0, 0, 0};
+    e = cudaMemcpy(l.err.word, zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+  }
+  switch (word[0]) {
+    case 0: t_err.clear(); return CSA_OK;
+    case csa::DEV_TIMEOUT: return fail(CSA_ERR_TIMEOUT, "a kernel wait exceeded its time limit");
+    case csa::DEV_BAD_INDEX:
+      return fail(CSA_ERR_DEVICE_INDEX, "a kernel met a chunk index or count out of range");
+    default: return fail(CSA_ERR_CUDA, "unknown device status " + std::to_string(word[0]));
+  }
+}
+
+csa_status csa_chunk_summaries(const void* K, csa_dtype dtype, int B, int Hkv, int64_t T, int D,
+                               int L, const float* proj, int R, float* summ, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(dtype), "dtype");
+  CSA_REQUIRE(B >= 0 && Hkv >= 0 && T >= 0 && D > 0 && L > 0, "sizes must be non-negative, D and L positive");
+  CSA_REQUIRE(T % L == 0, "T must be a multiple of L");
+  CSA_SUPPORT(D == 64 || D == 128, "D must be 64 or 128");
+  if (proj) CSA_SUPPORT(R == 16 || R == 32 || R == 64 || R == 128, "R must be 16, 32, 64 or 128");
+  CSA_SUPPORT(T / L <= 2147483647LL, "too many chunks");
+  if (static_cast<int64_t>(B) * Hkv * T == 0) return CSA_OK;
+  CSA_TRY(check_ptr(K, "K"));
+  CSA_TRY(check_ptr(summ, "summ"));
+  CSA_TRY(check_ptr(proj, "proj", false));
+  CSA_SUPPORT(static_cast<int64_t>(B) * Hkv <= 65535, "B*Hkv must be <= 65535");
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_chunk_summaries(l, K, dtype == CSA_BF16, B * Hkv, T, D, L, proj, R, summ),
+                "chunk summaries launch");
+}
+
+csa_status csa_meta_summaries(const float* summ, int B, int Hkv, int C, int Ds, int Gm, float* meta,
+                              csa_stream stream) {
+  CSA_REQUIRE(B >= 0 && Hkv >= 0 && C >= 0 && Ds > 0 && Gm > 0, "bad sizes");
+  CSA_REQUIRE(C % Gm == 0, "C must be a multiple of Gm");
+  CSA_SUPPORT(Ds <= 1024, "Ds must be <= 1024");
+  if (static_cast<int64_t>(B) * Hkv * C == 0) return CSA_OK;
+  CSA_SUPPORT(static_cast<int64_t>(B) * Hkv <= 65535, "B*Hkv must be <= 65535");
+  CSA_TRY(check_ptr(summ, "summ"));
+  CSA_TRY(check_ptr(meta, "meta"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_meta_summaries(l, summ, B * Hkv, C, Ds, Gm, meta), "meta summaries launch");
+}
+
+csa_status csa_tile_mean_q(const void* Q, csa_dtype dtype, int B, int S, int Hq, int D, int tile_m,
+                           float* qbar, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(dtype), "dtype");
+  CSA_REQUIRE(B >= 0 && S >= 0 && Hq >= 0 && D > 0 && tile_m > 0, "bad sizes");
+  CSA_REQUIRE(S % tile_m == 0, "S must be a multiple of tile_m");
+  CSA_SUPPORT(D <= 1024 && Hq <= 65535 && B <= 65535, "D <= 1024, Hq and B <= 65535");
+  if (static_cast<int64_t>(B) * S * Hq == 0) return CSA_OK;
+  CSA_TRY(check_ptr(Q, "Q"));
+  CSA_TRY(check_ptr(qbar, "qbar"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_tile_mean(l, Q, dtype == CSA_BF16, B, S, Hq, D, tile_m, qbar), "tile mean launch");
+}
+
+csa_status csa_score_chunks(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                            const float* summ, int B, int Nq, int Hq, int Hkv, int D, int C,
+                            const uint8_t* head_full, int causal_tile_m, int causal_L,
+                            float* scores, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
+  CSA_REQUIRE(B >= 0 && Nq >= 0 && Hq > 0 && Hkv > 0 && D > 0 && C >= 0, "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_REQUIRE(causal_tile_m >= 0 && (causal_tile_m == 0 || causal_L > 0), "causal_tile_m / causal_L");
+  CSA_SUPPORT(D <= 1024, "D must be <= 1024");
+  const int Ds = proj ? R : D;
+  CSA_SUPPORT(Ds == 16 || Ds == 32 || Ds == 64 || Ds == 128, "summary width must be 16, 32, 64 or 128");
+  CSA_SUPPORT(Nq <= 65535 && static_cast<int64_t>(B) * Hkv <= 65535, "Nq and B*Hkv must be <= 65535");
+  if (static_cast<int64_t>(B) * Nq * C == 0) return CSA_OK;
+  CSA_TRY(check_ptr(q, "q"));
+  CSA_TRY(check_ptr(proj, "proj", false));
+  CSA_TRY(check_ptr(summ, "summ"));
+  CSA_TRY(check_ptr(head_full, "head_full", false));
+  CSA_TRY(check_ptr(scores, "scores"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_score(l, q, q_dtype == CSA_BF16, proj, R, summ, B, Nq, Hq, Hkv, D, C,
+                                  head_full, causal_tile_m, causal_L, scores),
+                "score launch");
+}
+
+csa_status csa_select_topk(const float* scores, int U, int C, const int32_t* n_valid, int k_free,
+                           int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                           csa_stream stream) {
+  CSA_REQUIRE(kmax > 0, "kmax must be positive");
+  CSA_REQUIRE(U >= 0 && C >= 0 && k_free >= 0 && n_sink >= 0 && n_local >= 0, "U, C, k_free, n_sink and n_local must be non-negative");
+  CSA_SUPPORT(C <= 32768, "C must be <= 32768");
+  const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(k_free) + n_sink + n_local);
+  CSA_REQUIRE(kmax >= need, "kmax < min(C, k_free + n_sink + n_local)");
+  if (U == 0) return CSA_OK;
+  CSA_SUPPORT(U <= 2147483647, "U");
+  CSA_TRY(check_ptr(scores, "scores", C > 0));
+  CSA_TRY(check_ptr(n_valid, "n_valid", false));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_select_topk(l, scores, U, C, n_valid, k_free, n_sink, n_local, idx, count, kmax),
+                "select_topk launch");
+}
+
+csa_status csa_select_topp(const float* scores, int U, int C, float logit_scale, float p, int budget,
+                           int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                           int32_t* n_p_out, csa_stream stream) {
+  CSA_REQUIRE(kmax > 0, "kmax must be positive");
+  CSA_REQUIRE(U >= 0 && C > 0 && n_sink >= 0 && n_local >= 0, "U, n_sink and n_local must be non-negative and C positive");
+  CSA_REQUIRE(p > 0.f && p <= 1.f, "p must be in (0, 1]");
+  CSA_REQUIRE(budget >= 1, "budget must be >= 1");
+  CSA_REQUIRE(logit_scale == logit_scale, "logit_scale is NaN");
+  CSA_SUPPORT(budget <= 2048 && C <= 32768, "budget <= 2048 and C <= 32768");
+  const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(budget) + n_sink + n_local);
+  CSA_REQUIRE(kmax >= need, "kmax < min(C, budget + n_sink + n_local)");
+  if (U == 0) return CSA_OK;
+  CSA_TRY(check_ptr(scores, "scores"));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  CSA_TRY(check_ptr(n_p_out, "n_p_out", false));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_select_topp(l, scores, U, C, logit_scale, p, budget, n_sink, n_local, idx,
+                                        count, kmax, n_p_out),
+                "select_topp launch");
+}
+
+csa_status csa_select_hier(const void* q, csa_dtype q_dtype, const float* meta, const float* summ,
+                           int B, int Hq, int Hkv, int D, int C, int Gm, int top_meta, int k_free,
+                           int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                           csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
+  CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && C > 0 && Gm > 0 && top_meta >= 0 && k_free >= 0 &&
+                  n_sink >= 0 && n_local >= 0 && kmax > 0,
+              "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_REQUIRE(C % Gm == 0, "C must be a multiple of Gm");
+  CSA_SUPPORT(D == 64 || D == 128, "D must be 64 or 128");
+  CSA_SUPPORT(C <= 32768 && C / Gm <= 8192, "C <= 32768 and C/Gm <= 8192");
+  CSA_SUPPORT(static_cast<int64_t>(std::min(top_meta, C / Gm)) * Gm <= 8192, "top_meta * Gm must be <= 8192");
+  const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(k_free) + n_sink + n_local);
+  CSA_REQUIRE(kmax >= need, "kmax < min(C, k_free + n_sink + n_local)");
+  if (B == 0) return CSA_OK;
+  CSA_TRY(check_ptr(q, "q"));
+  CSA_TRY(check_ptr(meta, "meta"));
+  CSA_TRY(check_ptr(summ, "summ"));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_select_hier(l, q, q_dtype == CSA_BF16, meta, summ, B, Hq, Hkv, D, C, Gm,
+                                        top_meta, k_free, n_sink, n_local, idx, count, kmax),
+                "select_hier launch");
+}
+
+csa_status csa_selftest_wait_timeout(uint64_t limit_ns, csa_stream stream) {
+  CSA_REQUIRE(limit_ns > 0 && limit_ns <= 10000000000ull, "limit_ns must be in (0, 1e10]");
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  csa::DevErr e = l.err;
+  e.wait_ns = limit_ns;
+  wait_timeout_selftest_kernel<<<1, 32, 0, l.stream>>>(e);
+  return finish(cudaGetLastError(), "wait-timeout self-test launch");
+}
+
+int csa_decode_default_parts(csa_dtype dtype, int D, int L) {
+  csa::Launch l;
+  if (launch_ctx(nullptr, &l) != CSA_OK) return -1;
+  return csa::decode_default_parts(dtype == CSA_BF16, D, L, l.num_sms);
+}
+
+csa_status csa_sparse_decode(const void* q, const void* K, const void* V, csa_dtype dtype,
+                             const int32_t* idx, const int32_t* count, int kmax,
+                             const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T, int L,
+                             float scale, int num_parts, int max_splits, float* o_part,
+                             float* lse_part, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(dtype), "dtype");
+  CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && T >= 0 && L > 0 && kmax > 0 && num_parts >= 0 &&
+                  max_splits > 0,
+              "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_REQUIRE(T % L == 0, "T must be a multiple of L");
+  CSA_SUPPORT(D == 64 || D == 128, "D must be 64 or 128");
+  CSA_SUPPORT(L == 64 || L == 128, "L must be 64 or 128");
+  const int G = Hq / Hkv;
+  CSA_SUPPORT(G == 1 || G == 2 || G == 4 || G == 8, "Hq/Hkv must be 1, 2, 4 or 8");
+  CSA_SUPPORT(static_cast<int64_t>(B) * Hkv <= 2048, "B*Hkv must be <= 2048");
+  CSA_SUPPORT(static_cast<int64_t>(B) * Hkv * T < 2147483648LL, "B*Hkv*T must be < 2^31");
+  CSA_REQUIRE(scale == scale, "scale is NaN");
+  if (B == 0) return CSA_OK;
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  const int P = num_parts > 0 ? num_parts : csa::decode_default_parts(dtype == CSA_BF16, D, L, l.num_sms);
+  CSA_REQUIRE(max_splits >= P, "max_splits must be >= the number of pieces (num_parts)");
+  CSA_SUPPORT(P <= 65535, "num_parts must be <= 65535");
+  CSA_TRY(check_ptr(q, "q"));
+  CSA_TRY(check_ptr(K, "K"));
+  CSA_TRY(check_ptr(V, "V"));
+  CSA_TRY(check_ptr(head_full, "head_full", false));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  CSA_TRY(check_ptr(o_part, "o_part"));
+  CSA_TRY(check_ptr(lse_part, "lse_part"));
+  std::string why;
+  cudaError_t e = csa::launch_decode(l, q, K, V, dtype == CSA_BF16, idx, count, kmax, head_full, B, Hq,
+                                     Hkv, D, T, L, scale, P, max_splits, o_part, lse_part, &why);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  return finish(e, "sparse decode launch");
+}
+
+csa_status csa_lse_merge(const float* o_part, const float* lse_part, int rows, int max_splits, int D,
+                         void* out, csa_dtype out_dtype, float* lse_out, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(out_dtype), "out_dtype");
+  CSA_REQUIRE(rows >= 0 && max_splits > 0 && D > 0, "bad sizes");
+  CSA_SUPPORT(D % 4 == 0 && D <= 512, "D must be a multiple of 4, <= 512");
+  if (rows == 0) return CSA_OK;
+  CSA_TRY(check_ptr(o_part, "o_part"));
+  CSA_TRY(check_ptr(lse_part, "lse_part"));
+  CSA_TRY(check_ptr(out, "out"));
+  CSA_TRY(check_ptr(lse_out, "lse_out", false));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_merge(l, o_part, lse_part, rows, max_splits, D, out, out_dtype == CSA_BF16,
+                                  lse_out),
+                "lse merge launch");
+}
+
+csa_status csa_block_sparse_prefill(const void* Q, const void* K, const void* V, const int32_t* idx,
+                                    const int32_t* count, int kmax, int B, int S, int Hq, int Hkv,
+                                    int D, int tile_m, int L, float scale, void* O,
+                                    csa_stream stream) {
+  CSA_REQUIRE(B >= 0 && S >= 0 && Hq > 0 && Hkv > 0 && D > 0 && tile_m > 0 && L > 0 && kmax > 0,
+              "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_REQUIRE(S % tile_m == 0 && S % L == 0, "S must be a multiple of tile_m and of L");
+  CSA_SUPPORT(D == 128 && tile_m == 64 && L == 64 && Hq / Hkv == 4,
+              "implemented for D = 128, tile_m = L = 64, Hq/Hkv = 4");
+  CSA_SUPPORT(static_cast<int64_t>(B) * Hkv * S < 2147483648LL && static_cast<int64_t>(B) * S < 2147483648LL,
+              "B*Hkv*S must be < 2^31");
+  CSA_REQUIRE(scale == scale, "scale is NaN");
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  CSA_TRY(check_ptr(Q, "Q"));
+  CSA_TRY(check_ptr(K, "K"));
+  CSA_TRY(check_ptr(V, "V"));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  CSA_TRY(check_ptr(O, "O"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  std::string why;
+  cudaError_t e = csa::launch_prefill(l, Q, K, V, idx, count, kmax, B, S, Hq, Hkv, D, tile_m, L, scale, O,
+                                      &why);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  return finish(e, "block-sparse prefill launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,641 @@
+// Sparse split-K decode over the gathered raw KV of the selected chunks, and
+// the log-sum-exp merge of its partials.
+//
+// bf16 path (the hot one).  A persistent grid of P CTAs, one per SM.  The
+// units' chunk lists are laid end to end and cut into P equal pieces, so
+// every CTA streams the same number of chunks whatever mix of full-attention
+// heads (all chunks) and sparse heads (a few hundred) the step holds.
+//   * warp 4 (producer): resolves chunk ids 32 at a time (one lane each) and
+//     issues, per chunk, 2-D TMA loads of the chunk's K and V rows
+//     ([L x 64] boxes, 128-byte swizzle) into a ring of stages that fills
+//     ~192 KB of shared memory (3 stages of 64 KB at L = 128, D = 128), i.e.
+//     enough bytes in flight per SM to cover HBM latency.
+//   * warps 0-3 (consumers): each takes L/4 tokens of every chunk.  S^T =
+//     K q^T runs on the tensor cores as mma.m16n8k16 with the tokens as M and
+//     the query heads of the GQA group as N (up to 8); the online softmax
+//     stays in registers (per-head running max/sum); P is moved into the B
+//     layout with movmatrix and O^T += V^T P^T runs as a second mma.  The
+//     math per 64 KB chunk is a few hundred warp instructions, so the SM
+//     stays bound by the copy engine, not by issue.
+//   * at a unit boundary the four warps combine their (m, l, O) through
+//     shared memory and write one split partial (o normalised, lse).
+// Every wait is an mbarrier wait with a time limit; there is no named
+// barrier, so a timeout anywhere makes the kernel wind down, never hang.
+//
+// fp32 path: a plain CUDA-core kernel with the same partition, used for fp32
+// caches (parity workloads); it does the dot products in fp32.
+#include <algorithm>
+
+#include "internal.h"
+
+namespace csa {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStageBudget = 192 * 1024;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecodeParams {
+  const void* q;  // [B, Hq, D]
+  const float* Kf;  // fp32 path only
+  const float* Vf;
+  const int32_t* idx;
+  const int32_t* count;
+  int kmax;
+  const uint8_t* head_full;
+  int U, Hkv, G, Hq, C, L;
+  int64_t T;
+  float scale_log2;
+  int max_splits;
+  float* o_part;
+  float* lse_part;
+  DevErr err;
+};
+
+__device__ __forceinline__ int unit_count(const DecodeParams& p, int u) {
+  if (p.head_full != nullptr && p.head_full[u % p.Hkv]) return p.C;
+  int n = p.count[u];
+  if (n < 0 || n > p.kmax) {
+    dev_flag(p.err, DEV_BAD_INDEX);
+    n = max(0, min(n, p.kmax));
+  }
+  return n;
+}
+
+__device__ __forceinline__ int unit_chunk(const DecodeParams& p, int u, int pos) {
+  if (p.head_full != nullptr && p.head_full[u % p.Hkv]) return pos;
+  int c = p.idx[static_cast<int64_t>(u) * p.kmax + pos];
+  if (c < 0 || c >= p.C) {
+    dev_flag(p.err, DEV_BAD_INDEX);
+    c = 0;
+  }
+  return c;
+}
+
+// prefix[0..U] of the effective chunk counts (all threads of the block).
+__device__ void build_prefix(const DecodeParams& p, int* prefix, int* scan_sh) {
+  const int seg = (p.U + blockDim.x - 1) / blockDim.x;
+  const int lo = min(p.U, static_cast<int>(threadIdx.x) * seg), hi = min(p.U, lo + seg);
+  int loc = 0;
+  for (int u = lo; u < hi; ++u) loc += unit_count(p, u);
+  int total = 0;
+  int run = block_exclusive_scan(loc, scan_sh, &total);
+  for (int u = lo; u < hi; ++u) {
+    prefix[u] = run;
+    run += unit_count(p, u);
+  }
+  if (threadIdx.x == 0) prefix[p.U] = total;
+  __syncthreads();
+}
+
+// Unit owning global chunk g (prefix[u] <= g < prefix[u+1]); empty units skipped.
+__device__ __forceinline__ int unit_of(const int* prefix, int U, int64_t g) {
+  int lo = 0, hi = U - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= g) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int64_t piece_of(int64_t g, int64_t N, int64_t P) {
+  return ((g + 1) * P - 1) / N;
+}
+
+// Slots of unit u beyond its split count get lse = -inf (CTA c covers units
+// u = c, c + P, ...).  Threads [0, nthreads) of the block take part.
+__device__ void fill_empty_slots(const DecodeParams& p, const int* prefix, int nthreads) {
+  const int64_t N = prefix[p.U], P = gridDim.x;
+  for (int u = blockIdx.x; u < p.U; u += gridDim.x) {
+    const int64_t lo = prefix[u], hi = prefix[u + 1];
+    const int nsplit = hi > lo ? static_cast<int>(piece_of(hi - 1, N, P) - piece_of(lo, N, P) + 1) : 0;
+    const int b = u / p.Hkv, h = u % p.Hkv;
+    const int nfill = p.max_splits - nsplit;
+    for (int e = threadIdx.x; e < p.G * nfill; e += nthreads) {
+      const int g = e / nfill, s = nsplit + e % nfill;
+      p.lse_part[(static_cast<int64_t>(b) * p.Hq + h * p.G + g) * p.max_splits + s] = -INFINITY;
+    }
+  }
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <int D, int L>
+struct DecodeLayout {
+  static constexpr int KV_BYTES = L * D * 2;
+  static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+  static constexpr int NS = kStageBudget / STAGE_BYTES;
+  static constexpr int BOX_BYTES = L * 128;
+  static constexpr int FLUSH_BYTES = kConsumerWarps * 8 * D * 4 + kConsumerWarps * 8 * 2 * 4;
+  static constexpr int BAR_OFF = NS * STAGE_BYTES;
+  static constexpr int FLUSH_OFF = BAR_OFF + 2 * NS * 8 + 16;  // + flush mbarrier
+  static constexpr int PREFIX_OFF = FLUSH_OFF + FLUSH_BYTES;
+  static size_t bytes(int U) { return 1024 + PREFIX_OFF + static_cast<size_t>(U + 1) * 4; }
+};
+
+template <int D, int L>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
+  using Lay = DecodeLayout<D, L>;
+  constexpr int NS = Lay::NS;
+  constexpr int TOK_W = L / kConsumerWarps;  // tokens per consumer warp
+  constexpr int MT = TOK_W / 16;             // 16-token m-tiles per warp
+  constexpr int KS = D / 16;                 // k-steps (QK) / d-tiles (PV)
+  constexpr int NBOX = D / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t full_bar = sbase + Lay::BAR_OFF;
+  const uint32_t empty_bar = full_bar + NS * 8;
+  const uint32_t flush_bar = empty_bar + NS * 8;
+  float* fo = reinterpret_cast<float*>(smem + Lay::FLUSH_OFF);          // [4][8][D]
+  float* fm = fo + kConsumerWarps * 8 * D;                              // [4][8]
+  float* fl = fm + kConsumerWarps * 8;                                  // [4][8]
+  int* prefix = reinterpret_cast<int*>(smem + Lay::PREFIX_OFF);         // [U+1]
+  __shared__ int scan_sh[33];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full_bar + 8 * s, 1);
+      mbar_init(empty_bar + 8 * s, kConsumerWarps);
+    }
+    mbar_init(flush_bar, kConsumerWarps * 32);
+    fence_barrier_init();
+  }
+  if (warp == kConsumerWarps && lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  build_prefix(p, prefix, scan_sh);  // ends with __syncthreads (also publishes the barriers)
+
+  const int64_t N = prefix[p.U];
+  const int64_t P = gridDim.x;
+  const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+
+  if (warp == kConsumerWarps) {
+    // ---------------------------------------------------------------- producer
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t g0 = a; g0 < bnd && ok; g0 += 32) {
+      const int64_t g = g0 + lane;
+      int row = 0;
+      if (g < bnd) {
+        const int u = unit_of(prefix, p.U, g);
+        const int c = unit_chunk(p, u, static_cast<int>(g - prefix[u]));
+        row = static_cast<int>(u * p.T + static_cast<int64_t>(c) * L);
+      }
+      const int nb = static_cast<int>(bnd - g0 < 32 ? bnd - g0 : 32);
+      for (int j = 0; j < nb; ++j) {
+        const int row_j = __shfl_sync(0xffffffffu, row, j);
+        int good = 1;
+        if (lane == 0) {
+          const int64_t i = g0 - a + j;
+          const int s = static_cast<int>(i % NS);
+          const uint32_t it = static_cast<uint32_t>(i / NS);
+          if (!mbar_wait(empty_bar + 8 * s, (it & 1u) ^ 1u, p.err)) {
+            good = 0;
+          } else {
+            const uint32_t fb = full_bar + 8 * s;
+            mbar_arrive_expect_tx(fb, Lay::STAGE_BYTES);
+            const uint32_t dst = sbase + s * Lay::STAGE_BYTES;
+#pragma unroll
+            for (int bx = 0; bx < NBOX; ++bx) {
+              tma_load_2d(dst + bx * Lay::BOX_BYTES, &tmK, bx * 64, row_j, fb);
+              tma_load_2d(dst + Lay::KV_BYTES + bx * Lay::BOX_BYTES, &tmV, bx * 64, row_j, fb);
+            }
+            ++issued;
+          }
+        }
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
+          ok = false;
+          break;
+        }
+      }
+    }
+    // no copy may still be landing when the CTA retires
+    if (lane == 0) {
+      const int64_t first = issued > NS ? issued - NS : 0;
+      for (int64_t i = first; i < issued; ++i)
+        mbar_wait(full_bar + 8 * static_cast<int>(i % NS), static_cast<uint32_t>(i / NS) & 1u, p.err);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  fill_empty_slots(p, prefix, kConsumerWarps * 32);
+  const float scale_log2 = p.scale_log2;
+  const int hA = 2 * (lane & 3), hB = hA + 1;
+  uint32_t qf[KS][2];
+  float o[KS][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  int cur_u = -1;
+  uint32_t flush_phase = 0;
+  bool ok = true;
+
+  auto load_q = [&](int u) {
+    const int b = u / p.Hkv, h = u % p.Hkv;
+    const int n = lane >> 2;
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int d0 = ks * 16 + 2 * (lane & 3);
+      if (n < p.G) {
+        const __nv_bfloat16* r = qb + (static_cast<int64_t>(b) * p.Hq + h * p.G + n) * D;
+        qf[ks][0] = *reinterpret_cast<const uint32_t*>(r + d0);
+        qf[ks][1] = *reinterpret_cast<const uint32_t*>(r + d0 + 8);
+      } else {
+        qf[ks][0] = 0u;
+        qf[ks][1] = 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[ks][e] = 0.f;
+    }
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+  };
+
+  auto group_sync = [&]() -> bool {
+    mbar_arrive(flush_bar);
+    const bool r = mbar_wait(flush_bar, flush_phase, p.err);
+    flush_phase ^= 1u;
+    return r;
+  };
+
+  auto flush = [&](int u) -> bool {
+#pragma unroll
+    for (int x = 4; x < 32; x <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, x);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, x);
+    }
+    float* fow = fo + warp * 8 * D;
+    if (lane < 4) {
+      fm[warp * 8 + hA] = m0;
+      fm[warp * 8 + hB] = m1;
+      fl[warp * 8 + hA] = l0;
+      fl[warp * 8 + hB] = l1;
+    }
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const int d = dt * 16 + (lane >> 2);
+      fow[hA * D + d] = o[dt][0];
+      fow[hB * D + d] = o[dt][1];
+      fow[hA * D + d + 8] = o[dt][2];
+      fow[hB * D + d + 8] = o[dt][3];
+    }
+    if (!group_sync()) return false;
+    const int b = u / p.Hkv, h = u % p.Hkv;
+    const int slot = static_cast<int>(blockIdx.x - piece_of(prefix[u], N, P));
+    for (int e = threadIdx.x; e < p.G * D; e += kConsumerWarps * 32) {
+      const int g = e / D, d = e % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + g]);
+      float Ls = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float sc = exp2f(fm[w * 8 + g] - M);
+        Ls += fl[w * 8 + g] * sc;
+        acc += fo[(w * 8 + g) * D + d] * sc;
+      }
+      const int64_t row = static_cast<int64_t>(b) * p.Hq + h * p.G + g;
+      p.o_part[(row * p.max_splits + slot) * D + d] = acc / Ls;
+      if (d == 0) p.lse_part[row * p.max_splits + slot] = (M + log2f(Ls)) * kLn2;
+    }
+    return group_sync();
+  };
+
+  for (int64_t g = a, i = 0; g < bnd; ++g, ++i) {
+    if (cur_u < 0 || g >= prefix[cur_u + 1]) {
+      if (cur_u >= 0 && !flush(cur_u)) {
+        ok = false;
+        break;
+      }
+      cur_u = unit_of(prefix, p.U, g);
+      load_q(cur_u);
+    }
+    const int s = static_cast<int>(i % NS);
+    const uint32_t it = static_cast<uint32_t>(i / NS);
+    if (!mbar_wait(full_bar + 8 * s, it & 1u, p.err)) {
+      ok = false;
+      break;
+    }
+    const uint32_t sK = sbase + s * Lay::STAGE_BYTES;
+    const uint32_t sV = sK + Lay::KV_BYTES;
+    const int tok0 = warp * TOK_W;
+
+    // S^T = K q^T over this warp's tokens
+    float sc[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int bx = ks >> 2, colb = (ks & 3) * 16;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int row = tok0 + mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int col = colb + (lane >> 4) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(sK + bx * Lay::BOX_BYTES + sw128_offset(row, col), a0, a1, a2, a3);
+        mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+      }
+    }
+    // online softmax (log2 domain), per head hA / hB of this lane
+    float cm0 = -INFINITY, cm1 = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[mt][e] *= scale_log2;
+      cm0 = fmaxf(cm0, fmaxf(sc[mt][0], sc[mt][2]));
+      cm1 = fmaxf(cm1, fmaxf(sc[mt][1], sc[mt][3]));
+    }
+#pragma unroll
+    for (int x = 4; x < 32; x <<= 1) {
+      cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, x));
+      cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, x));
+    }
+    const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
+    const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    uint32_t pb[MT][2];
+    float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const float p0 = fast_exp2(sc[mt][0] - mn0), p1 = fast_exp2(sc[mt][1] - mn1);
+      const float p2 = fast_exp2(sc[mt][2] - mn0), p3 = fast_exp2(sc[mt][3] - mn1);
+      ps0 += p0 + p2;
+      ps1 += p1 + p3;
+      pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+      pb[mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+    }
+    l0 = l0 * al0 + ps0;
+    l1 = l1 * al1 + ps1;
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      o[dt][0] *= al0;
+      o[dt][1] *= al1;
+      o[dt][2] *= al0;
+      o[dt][3] *= al1;
+    }
+    // O^T += V^T P^T
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+      for (int dt = 0; dt < KS; ++dt) {
+        const int bx = dt >> 2, colb = (dt & 3) * 16;
+        const int mi = lane >> 3;
+        const int tok = tok0 + mt * 16 + (lane & 7) + (mi >> 1) * 8;
+        const int col = colb + (mi & 1) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(sV + bx * Lay::BOX_BYTES + sw128_offset(tok, col), a0, a1, a2, a3);
+        mma_bf16_16816(o[dt], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar + 8 * s);
+  }
+  if (ok && cur_u >= 0) flush(cur_u);
+}
+
+// ------------------------------------------------------------------ fp32 path
+
+constexpr int kF32Threads = 128;
+
+template <int D>
+__global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t smem_f[];
+  float* qs = reinterpret_cast<float*>(smem_f);   // [8][D]
+  float* sc = qs + 8 * D;                          // [8][128]
+  float* mh = sc + 8 * 128;                        // [8]
+  float* lh = mh + 8;                              // [8]
+  float* ah = lh + 8;                              // [8]
+  int* prefix = reinterpret_cast<int*>(ah + 8);    // [U+1]
+  __shared__ int scan_sh[33];
+  build_prefix(p, prefix, scan_sh);
+  fill_empty_slots(p, prefix, kF32Threads);
+  const int64_t N = prefix[p.U], P = gridDim.x;
+  const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+  const int L = p.L, G = p.G;
+  const int tid = threadIdx.x;
+  float o[8];
+  int cur_u = -1;
+
+  auto flush = [&](int u) {
+    const int b = u / p.Hkv, h = u % p.Hkv;
+    const int slot = static_cast<int>(blockIdx.x - piece_of(prefix[u], N, P));
+    for (int g = 0; g < G; ++g) {
+      const int64_t row = static_cast<int64_t>(b) * p.Hq + h * G + g;
+      if (tid < D) p.o_part[(row * p.max_splits + slot) * D + tid] = o[g] / lh[g];
+      if (tid == 0) p.lse_part[row * p.max_splits + slot] = (mh[g] + log2f(lh[g])) * kLn2;
+    }
+    __syncthreads();
+  };
+
+  for (int64_t g = a; g < bnd; ++g) {
+    if (cur_u < 0 || g >= prefix[cur_u + 1]) {
+      if (cur_u >= 0) flush(cur_u);
+      cur_u = unit_of(prefix, p.U, g);
+      const int b = cur_u / p.Hkv, h = cur_u % p.Hkv;
+      const float* qf = static_cast<const float*>(p.q);
+      for (int e = tid; e < G * D; e += kF32Threads)
+        qs[e] = qf[(static_cast<int64_t>(b) * p.Hq + h * G) * D + e];
+      if (tid < 8) {
+        mh[tid] = -INFINITY;
+        lh[tid] = 0.f;
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x) o[x] = 0.f;
+      __syncthreads();
+    }
+    const int u = cur_u;
+    const int c = unit_chunk(p, u, static_cast<int>(g - prefix[u]));
+    const int64_t row0 = u * p.T + static_cast<int64_t>(c) * L;
+    if (tid < L) {
+      const float* kr = p.Kf + (row0 + tid) * D;
+      for (int x = 0; x < G; ++x) {
+        float acc = 0.f;
+        for (int d = 0; d < D; ++d) acc += qs[x * D + d] * kr[d];
+        sc[x * 128 + tid] = acc * p.scale_log2;
+      }
+    }
+    __syncthreads();
+    if (tid < G) {
+      float cm = -INFINITY;
+      for (int j = 0; j < L; ++j) cm = fmaxf(cm, sc[tid * 128 + j]);
+      const float mn = fmaxf(mh[tid], cm);
+      ah[tid] = exp2f(mh[tid] - mn);
+      mh[tid] = mn;
+    }
+    __syncthreads();
+    if (tid < L)
+      for (int x = 0; x < G; ++x) sc[x * 128 + tid] = exp2f(sc[x * 128 + tid] - mh[x]);
+    __syncthreads();
+    if (tid < G) {
+      float s = 0.f;
+      for (int j = 0; j < L; ++j) s += sc[tid * 128 + j];
+      lh[tid] = lh[tid] * ah[tid] + s;
+    }
+    if (tid < D) {
+      for (int x = 0; x < G; ++x) {
+        float acc = 0.f;
+        for (int j = 0; j < L; ++j) acc += sc[x * 128 + j] * p.Vf[(row0 + j) * D + tid];
+        o[x] = o[x] * ah[x] + acc;
+      }
+    }
+    __syncthreads();
+  }
+  if (cur_u >= 0) flush(cur_u);
+}
+
+// ------------------------------------------------------------------ merge
+
+constexpr int kMergeThreads = 128;
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(
+    const float* __restrict__ o_part, const float* __restrict__ lse_part, int rows, int S, int D,
+    void* __restrict__ out, int out_bf16, float* __restrict__ lse_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (kMergeThreads / 32) + warp;
+  if (r >= rows) return;
+  const float* lrow = lse_part + static_cast<int64_t>(r) * S;
+  float mx = -INFINITY;
+  for (int s = lane; s < S; s += 32) mx = fmaxf(mx, lrow[s]);
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+  float tot = 0.f;
+  if (mx != -INFINITY)
+    for (int s = lane; s < S; s += 32) {
+      const float v = lrow[s];
+      if (v != -INFINITY) tot += expf(v - mx);
+    }
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, x);
+  const float lse = mx == -INFINITY ? -INFINITY : mx + logf(tot);
+  if (lane == 0 && lse_out) lse_out[r] = lse;
+  const int nv = D / 4;
+  for (int v4 = lane; v4 < nv; v4 += 32) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (mx != -INFINITY) {
+      for (int s = 0; s < S; ++s) {
+        const float l = lrow[s];
+        if (l == -INFINITY) continue;
+        const float w = expf(l - lse);
+        const float4 x = __ldg(reinterpret_cast<const float4*>(o_part + (static_cast<int64_t>(r) * S + s) * D) + v4);
+        acc.x += w * x.x;
+        acc.y += w * x.y;
+        acc.z += w * x.z;
+        acc.w += w * x.w;
+      }
+    }
+    if (out_bf16) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out) + static_cast<int64_t>(r) * D + v4 * 4;
+      reinterpret_cast<uint32_t*>(ob)[0] = pack_bf16x2(acc.x, acc.y);
+      reinterpret_cast<uint32_t*>(ob)[1] = pack_bf16x2(acc.z, acc.w);
+    } else {
+      reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(r) * D)[v4] = acc;
+    }
+  }
+}
+
+template <int D, int L>
+cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, const void* V,
+                        int B, int Hkv, int P, std::string* why) {
+  using Lay = DecodeLayout<D, L>;
+  CUtensorMap tmK, tmV;
+  const uint64_t rows = static_cast<uint64_t>(B) * Hkv * p.T;
+  if (!make_tmap_bf16_2d(&tmK, K, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tmV, V, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+  const size_t sh = Lay::bytes(p.U);
+  auto fn = decode_bf16_kernel<D, L>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sh));
+  if (e != cudaSuccess) return e;
+  fn<<<P, kDecodeThreads, sh, l.stream>>>(tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_default_parts(bool bf16, int D, int L, int num_sms) {
+  (void)bf16;
+  (void)D;
+  (void)L;
+  return num_sms;  // one persistent CTA per SM
+}
+
+size_t decode_smem_bytes(bool bf16, int D, int L, int U) {
+  if (!bf16) return static_cast<size_t>(8 * D + 8 * 128 + 24 + U + 1) * 4;
+  if (D == 128 && L == 128) return DecodeLayout<128, 128>::bytes(U);
+  if (D == 128 && L == 64) return DecodeLayout<128, 64>::bytes(U);
+  if (D == 64 && L == 128) return DecodeLayout<64, 128>::bytes(U);
+  return DecodeLayout<64, 64>::bytes(U);
+}
+
+cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,
+                          const int32_t* idx, const int32_t* count, int kmax,
+                          const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T,
+                          int L, float scale, int num_parts, int max_splits, float* o_part,
+                          float* lse_part, std::string* why) {
+  DecodeParams p{};
+  p.q = q;
+  p.Kf = static_cast<const float*>(K);
+  p.Vf = static_cast<const float*>(V);
+  p.idx = idx;
+  p.count = count;
+  p.kmax = kmax;
+  p.head_full = head_full;
+  p.U = B * Hkv;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.Hq = Hq;
+  p.C = static_cast<int>(T / L);
+  p.L = L;
+  p.T = T;
+  p.scale_log2 = scale * kLog2e;
+  p.max_splits = max_splits;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.err = l.err;
+  const int P = num_parts > 0 ? num_parts : decode_default_parts(bf16, D, L, l.num_sms);
+  if (p.U == 0) return cudaSuccess;
+  if (!bf16) {
+    const size_t sh = decode_smem_bytes(false, D, L, p.U);
+    cudaError_t e;
+    if (D == 128) {
+      e = cudaFuncSetAttribute(decode_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sh));
+      if (e != cudaSuccess) return e;
+      decode_f32_kernel<128><<<P, kF32Threads, sh, l.stream>>>(p);
+    } else {
+      e = cudaFuncSetAttribute(decode_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sh));
+      if (e != cudaSuccess) return e;
+      decode_f32_kernel<64><<<P, kF32Threads, sh, l.stream>>>(p);
+    }
+    return cudaGetLastError();
+  }
+  if (D == 128 && L == 128) return launch_bf16<128, 128>(l, p, K, V, B, Hkv, P, why);
+  if (D == 128 && L == 64) return launch_bf16<128, 64>(l, p, K, V, B, Hkv, P, why);
+  if (D == 64 && L == 128) return launch_bf16<64, 128>(l, p, K, V, B, Hkv, P, why);
+  return launch_bf16<64, 64>(l, p, K, V, B, Hkv, P, why);
+}
+
+cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_part, int rows,
+                         int max_splits, int D, void* out, bool out_bf16, float* lse_out) {
+  if (rows == 0) return cudaSuccess;
+  const int per = kMergeThreads / 32;
+  merge_kernel<<<(rows + per - 1) / per, kMergeThreads, 0, l.stream>>>(
+      o_part, lse_part, rows, max_splits, D, out, out_bf16 ? 1 : 0, lse_out);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

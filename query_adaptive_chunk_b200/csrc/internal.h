@@ -1,0 +1,69 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernel files.
+// Launchers assume validated arguments and return the launch's cudaError_t.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "common.cuh"
+
+namespace csa {
+
+struct Launch {
+  cudaStream_t stream;
+  DevErr err;
+  int num_sms;
+};
+
+// summaries.cu
+cudaError_t launch_chunk_summaries(const Launch& l, const void* K, bool bf16, int U, int64_t T,
+                                   int D, int L, const float* proj, int R, float* summ);
+cudaError_t launch_meta_summaries(const Launch& l, const float* summ, int U, int C, int Ds, int Gm,
+                                  float* meta);
+cudaError_t launch_tile_mean(const Launch& l, const void* Q, bool bf16, int B, int S, int Hq, int D,
+                             int tile_m, float* qbar);
+
+// score.cu
+cudaError_t launch_score(const Launch& l, const void* q, bool bf16, const float* proj, int R,
+                         const float* summ, int B, int Nq, int Hq, int Hkv, int D, int C,
+                         const uint8_t* head_full, int causal_tile_m, int causal_L,
+                         float* scores);
+
+// select.cu
+cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
+                               const int32_t* n_valid, int k_free, int n_sink, int n_local,
+                               int32_t* idx, int32_t* count, int kmax);
+cudaError_t launch_select_topp(const Launch& l, const float* scores, int U, int C,
+                               float logit_scale, float p, int budget, int n_sink, int n_local,
+                               int32_t* idx, int32_t* count, int kmax, int32_t* n_p_out);
+cudaError_t launch_select_hier(const Launch& l, const void* q, bool bf16, const float* meta,
+                               const float* summ, int B, int Hq, int Hkv, int D, int C, int Gm,
+                               int top_meta, int k_free, int n_sink, int n_local, int32_t* idx,
+                               int32_t* count, int kmax);
+
+// decode.cu
+int decode_default_parts(bool bf16, int D, int L, int num_sms);
+cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,
+                          const int32_t* idx, const int32_t* count, int kmax,
+                          const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T,
+                          int L, float scale, int num_parts, int max_splits, float* o_part,
+                          float* lse_part, std::string* why);
+cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_part, int rows,
+                         int max_splits, int D, void* out, bool out_bf16, float* lse_out);
+
+// prefill.cu
+cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const void* V,
+                           const int32_t* idx, const int32_t* count, int kmax, int B, int S,
+                           int Hq, int Hkv, int D, int tile_m, int L, float scale, void* O,
+                           std::string* why);
+
+// tma_host.cu: 2-D bf16 tensor map over a row-major [rows, cols] matrix with
+// `row_stride` elements between rows, box [box_rows, box_cols], 128-byte swizzle.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint64_t row_stride, uint32_t box_rows, uint32_t box_cols,
+                       std::string* why);
+
+}  // namespace csa

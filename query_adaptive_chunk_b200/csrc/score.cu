@@ -1,0 +1,114 @@
+// Chunk scores: S[b,h,n,c] = (sum_g qt[b,n,h*G+g]) . summ[b,h,c]  (qt = q or P^T q).
+//
+// The group sum of the query heads is taken first (one dot product per chunk
+// instead of G), then every warp streams summary rows with 128-bit loads:
+// a row of Ds floats is spread over Ds/4 lanes, all eight rows of a warp are
+// loaded before any arithmetic so that 8 x 512 B are in flight per warp, and
+// the partial dot products are reduced with xor-shuffles inside the row's
+// lanes.  One CTA covers 32 KB of summaries.
+#include "internal.h"
+
+namespace csa {
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kScoreIters = 8;  // rows per lane-group per warp
+
+template <int DS>
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ proj, int R,
+    const float* __restrict__ summ, int Nq, int Hq, int Hkv, int D, int C,
+    const uint8_t* __restrict__ head_full, int causal_tile_m, int causal_L,
+    float* __restrict__ scores) {
+  constexpr int LPR = DS / 4;          // lanes per summary row
+  constexpr int RPI = 32 / LPR;        // rows per warp iteration
+  constexpr int ROWS_WARP = RPI * kScoreIters;
+  constexpr int ROWS_CTA = ROWS_WARP * kScoreWarps;
+  __shared__ float qs[1024];
+  __shared__ float qp[DS];
+
+  const int u = blockIdx.z;  // b * Hkv + h
+  const int n = blockIdx.y;
+  const int h = u % Hkv, b = u / Hkv;
+  if (head_full != nullptr && head_full[h]) return;
+  const int G = Hq / Hkv;
+
+  // group-summed query row (fp32)
+  for (int d = threadIdx.x; d < D; d += kScoreThreads) {
+    float acc = 0.f;
+    for (int g = 0; g < G; ++g) {
+      const int64_t off = ((static_cast<int64_t>(b) * Nq + n) * Hq + h * G + g) * D + d;
+      acc += q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
+                    : static_cast<const float*>(q)[off];
+    }
+    qs[d] = acc;
+  }
+  __syncthreads();
+  const float* qv = qs;
+  if (proj != nullptr) {
+    for (int r = threadIdx.x; r < R; r += kScoreThreads) {
+      float acc = 0.f;
+      for (int d = 0; d < D; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * qs[d];
+      qp[r] = acc;
+    }
+    __syncthreads();
+    qv = qp;
+  }
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % LPR, rsub = lane / LPR;
+  const float4 q4 = make_float4(qv[sub * 4], qv[sub * 4 + 1], qv[sub * 4 + 2], qv[sub * 4 + 3]);
+  const int n_valid =
+      causal_tile_m > 0 ? min(C, ((n + 1) * causal_tile_m - 1) / causal_L + 1) : C;
+  const int row0 = blockIdx.x * ROWS_CTA + warp * ROWS_WARP + rsub;
+  const float* sbase = summ + static_cast<int64_t>(u) * C * DS;
+  float4 v[kScoreIters];
+#pragma unroll
+  for (int it = 0; it < kScoreIters; ++it) {
+    const int c = row0 + it * RPI;
+    if (c < n_valid)
+      v[it] = __ldg(reinterpret_cast<const float4*>(sbase + static_cast<int64_t>(c) * DS) + sub);
+    else
+      v[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float* out = scores + (static_cast<int64_t>(u) * Nq + n) * C;
+#pragma unroll
+  for (int it = 0; it < kScoreIters; ++it) {
+    float s = v[it].x * q4.x + v[it].y * q4.y + v[it].z * q4.z + v[it].w * q4.w;
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const int c = row0 + it * RPI;
+    if (sub == 0 && c < C) out[c] = c < n_valid ? s : -INFINITY;
+  }
+}
+
+template <int DS>
+cudaError_t launch_ds(const Launch& l, const void* q, bool bf16, const float* proj, int R,
+                      const float* summ, int B, int Nq, int Hq, int Hkv, int D, int C,
+                      const uint8_t* head_full, int ctm, int cL, float* scores) {
+  constexpr int ROWS_CTA = (32 / (DS / 4)) * kScoreIters * kScoreWarps;
+  dim3 grid((C + ROWS_CTA - 1) / ROWS_CTA, Nq, B * Hkv);
+  score_kernel<DS><<<grid, kScoreThreads, 0, l.stream>>>(q, bf16 ? 1 : 0, proj, R, summ, Nq, Hq,
+                                                        Hkv, D, C, head_full, ctm, cL, scores);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score(const Launch& l, const void* q, bool bf16, const float* proj, int R,
+                         const float* summ, int B, int Nq, int Hq, int Hkv, int D, int C,
+                         const uint8_t* head_full, int causal_tile_m, int causal_L,
+                         float* scores) {
+  if (B == 0 || Nq == 0 || C == 0) return cudaSuccess;
+  const int Ds = proj ? R : D;
+  switch (Ds) {
+    case 16: return launch_ds<16>(l, q, bf16, proj, R, summ, B, Nq, Hq, Hkv, D, C, head_full, causal_tile_m, causal_L, scores);
+    case 32: return launch_ds<32>(l, q, bf16, proj, R, summ, B, Nq, Hq, Hkv, D, C, head_full, causal_tile_m, causal_L, scores);
+    case 64: return launch_ds<64>(l, q, bf16, proj, R, summ, B, Nq, Hq, Hkv, D, C, head_full, causal_tile_m, causal_L, scores);
+    case 128: return launch_ds<128>(l, q, bf16, proj, R, summ, B, Nq, Hq, Hkv, D, C, head_full, causal_tile_m, causal_L, scores);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace csa

@@ -1,0 +1,154 @@
+"""Decode and prefill steps assembled from the C-ABI calls.
+
+``SparseDecoder`` owns the buffers of one decode configuration (chunk
+summaries, scores, index lists, split-K partials, outputs) and runs a step
+as: score -> select (top-k / top-p / hierarchical) -> sparse decode ->
+LSE merge.  ``BlockSparsePrefill`` runs tile means -> causal scores -> top-k
+-> block-sparse prefill.  Buffers come from torch (device memory); every
+computation is a call into libcsa.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import csa
+
+
+def _dt(t: torch.Tensor) -> int:
+    return csa.CSA_BF16 if t.dtype == torch.bfloat16 else csa.CSA_F32
+
+
+class SparseDecoder:
+    """Query-adaptive chunk-sparse decode over a fixed KV cache.
+
+    K, V: [B, Hkv, T, D] (bf16 or fp32, contiguous, on the current device).
+    select: "topk" | "topp" | "hier".  The summaries (and meta-summaries)
+    are computed once here, as part of building the cache."""
+
+    def __init__(self, K: torch.Tensor, V: torch.Tensor, *, Hq: int, L: int, select: str,
+                 n_sink: int, n_local: int, k_free: int = 0, proj: torch.Tensor | None = None,
+                 p: float = 0.9, budget: int = 256, full_heads=(), Gm: int = 0, top_meta: int = 0,
+                 scale: float | None = None, num_parts: int = 0, out_dtype=torch.float32):
+        assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
+        self.K, self.V = K, V
+        B, Hkv, T, D = K.shape
+        self.B, self.Hq, self.Hkv, self.T, self.D, self.L = B, Hq, Hkv, T, D, L
+        self.C = T // L
+        self.select, self.n_sink, self.n_local, self.k_free = select, n_sink, n_local, k_free
+        self.p, self.budget, self.Gm, self.top_meta = p, budget, Gm, top_meta
+        self.scale = 1.0 / math.sqrt(D) if scale is None else scale
+        self.proj = proj
+        self.R = 0 if proj is None else proj.shape[1]
+        self.dtype = _dt(K)
+        dev = K.device
+        U = B * Hkv
+        Ds = self.R if proj is not None else D
+        self.summ = torch.empty(B, Hkv, self.C, Ds, dtype=torch.float32, device=dev)
+        csa.csa_chunk_summaries(K, self.dtype, B, Hkv, T, D, L, proj, self.R, self.summ)
+        self.meta = None
+        if select == "hier":
+            self.meta = torch.empty(B, Hkv, self.C // Gm, Ds, dtype=torch.float32, device=dev)
+            csa.csa_meta_summaries(self.summ, B, Hkv, self.C, Ds, Gm, self.meta)
+        self.head_full = None
+        if full_heads:
+            hf = torch.zeros(Hkv, dtype=torch.uint8)
+            hf[list(full_heads)] = 1
+            self.head_full = hf.to(dev)
+        extra = budget if select == "topp" else k_free
+        self.kmax = min(self.C, extra + n_sink + n_local)
+        self.scores = torch.zeros(B, Hkv, 1, self.C, dtype=torch.float32, device=dev)
+        self.idx = torch.full((U, self.kmax), -1, dtype=torch.int32, device=dev)
+        self.count = torch.zeros(U, dtype=torch.int32, device=dev)
+        self.n_p = torch.zeros(U, dtype=torch.int32, device=dev)
+        self.P = num_parts if num_parts > 0 else csa.csa_decode_default_parts(self.dtype, D, L)
+        self.max_splits = self.P
+        self.o_part = torch.empty(B, Hq, self.max_splits, D, dtype=torch.float32, device=dev)
+        self.lse_part = torch.empty(B, Hq, self.max_splits, dtype=torch.float32, device=dev)
+        self.out = torch.empty(B, Hq, D, dtype=out_dtype, device=dev)
+        self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+
+    def select_chunks(self, q: torch.Tensor, stream=None):
+        """Score + select: fills self.idx / self.count (and self.n_p for top-p)."""
+        B, Hq, Hkv, D, C = self.B, self.Hq, self.Hkv, self.D, self.C
+        U = B * Hkv
+        qd = _dt(q)
+        if self.select == "hier":
+            csa.csa_select_hier(q, qd, self.meta, self.summ, B, Hq, Hkv, D, C, self.Gm,
+                                self.top_meta, self.k_free, self.n_sink, self.n_local, self.idx,
+                                self.count, self.kmax, stream=stream)
+            return
+        csa.csa_score_chunks(q, qd, self.proj, self.R, self.summ, B, 1, Hq, Hkv, D, C,
+                             self.head_full, 0, 0, self.scores, stream=stream)
+        if self.select == "topk":
+            csa.csa_select_topk(self.scores, U, C, None, self.k_free, self.n_sink, self.n_local,
+                                self.idx, self.count, self.kmax, stream=stream)
+        elif self.select == "topp":
+            csa.csa_select_topp(self.scores, U, C, 1.0 / math.sqrt(D), self.p, self.budget,
+                                self.n_sink, self.n_local, self.idx, self.count, self.kmax,
+                                self.n_p, stream=stream)
+        else:
+            raise ValueError(self.select)
+
+    def attend(self, q: torch.Tensor, stream=None):
+        """Sparse split-K decode over the current index lists, then the LSE merge."""
+        csa.csa_sparse_decode(q, self.K, self.V, self.dtype, self.idx, self.count, self.kmax,
+                              self.head_full, self.B, self.Hq, self.Hkv, self.D, self.T, self.L,
+                              self.scale, self.P, self.max_splits, self.o_part, self.lse_part,
+                              stream=stream)
+        csa.csa_lse_merge(self.o_part, self.lse_part, self.B * self.Hq, self.max_splits, self.D,
+                          self.out, _dt(self.out), self.lse, stream=stream)
+
+    def step(self, q: torch.Tensor, stream=None):
+        self.select_chunks(q, stream)
+        self.attend(q, stream)
+        return self.out, self.lse
+
+
+class BlockSparsePrefill:
+    """Block-sparse causal prefill: per (tile, KV head) the top-k_free chunks by
+    tile-mean score plus the sink and the diagonal chunk."""
+
+    def __init__(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, *, tile_m: int, L: int,
+                 k_free: int, n_sink: int = 1, n_local: int = 1, scale: float | None = None):
+        B, S, Hq, D = Q.shape
+        Hkv = K.shape[1]
+        self.Q, self.K, self.V = Q, K, V
+        self.B, self.S, self.Hq, self.Hkv, self.D = B, S, Hq, Hkv, D
+        self.tile_m, self.L, self.k_free, self.n_sink, self.n_local = tile_m, L, k_free, n_sink, n_local
+        self.scale = 1.0 / math.sqrt(D) if scale is None else scale
+        self.n_tiles = S // tile_m
+        self.C = S // L
+        dev = Q.device
+        self.kmax = min(self.C, k_free + n_sink + n_local)
+        self.summ = torch.empty(B, Hkv, self.C, D, dtype=torch.float32, device=dev)
+        csa.csa_chunk_summaries(K, _dt(K), B, Hkv, S, D, L, None, 0, self.summ)
+        self.qbar = torch.empty(B, self.n_tiles, Hq, D, dtype=torch.float32, device=dev)
+        self.scores = torch.empty(B, Hkv, self.n_tiles, self.C, dtype=torch.float32, device=dev)
+        U = B * Hkv * self.n_tiles
+        t = torch.arange(self.n_tiles, dtype=torch.int64)
+        n_valid = ((t + 1) * tile_m - 1) // L + 1
+        self.n_valid = n_valid.repeat(B * Hkv).to(torch.int32).to(dev)
+        self.idx = torch.full((U, self.kmax), -1, dtype=torch.int32, device=dev)
+        self.count = torch.zeros(U, dtype=torch.int32, device=dev)
+        self.O = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=dev)
+
+    def select_chunks(self, stream=None):
+        B, S, Hq, Hkv, D = self.B, self.S, self.Hq, self.Hkv, self.D
+        csa.csa_tile_mean_q(self.Q, _dt(self.Q), B, S, Hq, D, self.tile_m, self.qbar, stream=stream)
+        csa.csa_score_chunks(self.qbar, csa.CSA_F32, None, 0, self.summ, B, self.n_tiles, Hq, Hkv,
+                             D, self.C, None, self.tile_m, self.L, self.scores, stream=stream)
+        csa.csa_select_topk(self.scores, B * Hkv * self.n_tiles, self.C, self.n_valid, self.k_free,
+                            self.n_sink, self.n_local, self.idx, self.count, self.kmax,
+                            stream=stream)
+
+    def attend(self, stream=None):
+        csa.csa_block_sparse_prefill(self.Q, self.K, self.V, self.idx, self.count, self.kmax,
+                                     self.B, self.S, self.Hq, self.Hkv, self.D, self.tile_m,
+                                     self.L, self.scale, self.O, stream=stream)
+
+    def step(self, stream=None):
+        self.select_chunks(stream)
+        self.attend(stream)
+        return self.O

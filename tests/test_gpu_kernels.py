@@ -1,0 +1,407 @@
+"""Per-call parity of the CUDA library against the CPU oracle, through the C
+ABI, on seeded inputs that span several tiles and a ragged tail, plus the
+edge cases (empty and one-element sets, n_valid = 0/1, ties, more pieces
+than chunks, group sizes 1..8, both head dims and chunk lengths)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import parity
+from oracle import csa_oracle as O
+from oracle.pipeline import to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def csa():
+    from query_adaptive_chunk_b200 import csa as mod
+    return mod
+
+
+def _gen(seed):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, seed, dtype=torch.float32):
+    return torch.randn(shape, generator=_gen(seed), device="cuda").to(dtype)
+
+
+def _dt(name):
+    return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
+
+
+# ---------------------------------------------------------------- precompute
+
+@pytest.mark.parametrize("dtype,D,L,R", [("f32", 64, 64, 0), ("bf16", 128, 64, 0),
+                                         ("bf16", 128, 128, 16), ("bf16", 64, 128, 32),
+                                         ("f32", 128, 64, 128)])
+def test_chunk_summaries(csa, dtype, D, L, R):
+    B, Hkv, C = 2, 3, 7
+    K = _randn((B, Hkv, C * L, D), 1, _dt(dtype))
+    P = _randn((D, R), 2) / 4 if R else None
+    Ds = R if R else D
+    out = torch.empty(B, Hkv, C, Ds, device="cuda")
+    csa.csa_chunk_summaries(K, K.dtype, B, Hkv, C * L, D, L, P, R, out)
+    ref = O.chunk_summaries(to_np(K), L, None if P is None else to_np(P))
+    assert np.abs(out.cpu().double().numpy() - ref).max() < 1e-5
+
+
+def test_meta_summaries_and_tile_mean(csa):
+    summ = _randn((2, 3, 64, 128), 3)
+    meta = torch.empty(2, 3, 8, 128, device="cuda")
+    csa.csa_meta_summaries(summ, 2, 3, 64, 128, 8, meta)
+    assert np.abs(meta.cpu().double().numpy() - O.meta_summaries(to_np(summ), 8)).max() < 1e-6
+    Q = _randn((2, 320, 8, 64), 4, torch.bfloat16)
+    qbar = torch.empty(2, 5, 8, 64, device="cuda")
+    csa.csa_tile_mean_q(Q, Q.dtype, 2, 320, 8, 64, 64, qbar)
+    assert np.abs(qbar.cpu().double().numpy() - O.tile_mean_q(to_np(Q), 64)).max() < 1e-5
+
+
+# ---------------------------------------------------------------- scores
+
+@pytest.mark.parametrize("G,D,R,C,causal", [(4, 128, 0, 517, False), (4, 128, 16, 1029, False),
+                                            (1, 64, 0, 70, False), (8, 128, 32, 300, False),
+                                            (4, 128, 0, 96, True)])
+def test_score_chunks(csa, G, D, R, C, causal):
+    B, Hkv = 2, 3
+    Hq = G * Hkv
+    Nq = 96 if causal else 1
+    q = _randn((B, Nq, Hq, D), 5, torch.bfloat16 if not causal else torch.float32)
+    P = _randn((D, R), 6) / 4 if R else None
+    Ds = R if R else D
+    summ = _randn((B, Hkv, C, Ds), 7) * 0.2
+    full = torch.tensor([0, 1, 0], dtype=torch.uint8, device="cuda")
+    scores = torch.full((B, Hkv, Nq, C), 12345.0, device="cuda")
+    csa.csa_score_chunks(q, q.dtype, P, R, summ, B, Nq, Hq, Hkv, D, C, None if causal else full,
+                         64 if causal else 0, 64 if causal else 0, scores)
+    got = scores.cpu().double().numpy()
+    ref = O.score_chunks(to_np(q), to_np(summ), Hkv, None if P is None else to_np(P))
+    for b in range(B):
+        for h in range(Hkv):
+            if not causal and h == 1:
+                assert np.all(got[b, h] == 12345.0)  # full head: row not written
+                continue
+            for n in range(Nq):
+                vis = min(C, n + 1) if causal else C
+                assert np.allclose(got[b, h, n, :vis], ref[b, h, n, :vis], rtol=1e-5, atol=1e-4)
+                assert np.all(np.isneginf(got[b, h, n, vis:]))
+
+
+# ---------------------------------------------------------------- top-k
+
+def _run_topk(csa, scores, k_free, n_sink, n_local, n_valid=None, kmax=None):
+    U, C = scores.shape
+    kmax = kmax or max(1, min(C, k_free + n_sink + n_local))
+    idx = torch.full((U, kmax), 777, dtype=torch.int32, device="cuda")
+    cnt = torch.full((U,), 777, dtype=torch.int32, device="cuda")
+    nv = None if n_valid is None else torch.tensor(n_valid, dtype=torch.int32, device="cuda")
+    csa.csa_select_topk(scores, U, C, nv, k_free, n_sink, n_local, idx, cnt, kmax)
+    return parity.gpu_sets(idx, cnt)
+
+
+@pytest.mark.parametrize("C,U,kind", [(16, 3, "normal"), (512, 32, "normal"), (1000, 5, "ints"),
+                                      (8192, 2, "normal"), (32768, 1, "normal"), (300, 4, "zeros"),
+                                      (513, 4, "ints")])
+def test_select_topk_exact(csa, C, U, kind):
+    """Same fp32 scores on both sides: the sets must agree exactly (ties to
+    the lower index, -0 == +0)."""
+    if kind == "normal":
+        s = _randn((U, C), 8)
+    elif kind == "ints":
+        s = torch.randint(-3, 4, (U, C), generator=_gen(9), device="cuda").float()
+    else:
+        s = torch.zeros(U, C, device="cuda")
+        s[:, ::3] = -0.0
+        s[:, 5::7] = 1.0
+    rng = np.random.default_rng(C)
+    for k_free, n_sink, n_local in [(2, 1, 1), (29, 1, 2), (0, 1, 1), (C, 0, 0), (C + 5, 2, 3),
+                                    (int(rng.integers(1, C)), 0, 1)]:
+        got = _run_topk(csa, s, k_free, n_sink, n_local)
+        sn = s.cpu().double().numpy()
+        for u in range(U):
+            ref, _ = O.select_topk(sn[u], k_free, n_sink, n_local)
+            assert got[u] == ref, (u, k_free, n_sink, n_local)
+
+
+def test_select_topk_n_valid(csa):
+    """Causal units: each sees only chunks [0, n_valid) (0, 1, 2 and ragged)."""
+    C, U = 515, 40
+    s = _randn((U, C), 10)
+    nv = [0, 1, 2, 3, 17, 18, 19, 515] + list(np.random.default_rng(1).integers(0, C + 1, U - 8))
+    got = _run_topk(csa, s, 16, 1, 1, n_valid=[int(x) for x in nv])
+    sn = s.cpu().double().numpy()
+    for u in range(U):
+        ref, _ = O.select_topk(sn[u], 16, 1, 1, n_valid=int(nv[u]))
+        assert got[u] == ref, (u, nv[u])
+
+
+def test_select_topk_golden(csa):
+    for c in pins_golden("topk_cases.json"):
+        s = torch.tensor([c["scores"]], dtype=torch.float32, device="cuda")
+        nv = None if c["n_valid"] is None else [c["n_valid"]]
+        got = _run_topk(csa, s, c["k_free"], c["n_sink"], c["n_local"], n_valid=nv,
+                        kmax=len(c["scores"]))
+        assert got[0] == c["expect"], c["why"]
+
+
+def pins_golden(name):
+    import pins
+    return pins._golden(name)["cases"]
+
+
+# ---------------------------------------------------------------- top-p
+
+def _run_topp(csa, s, scale, p, budget, n_sink, n_local):
+    U, C = s.shape
+    kmax = min(C, budget + n_sink + n_local)
+    idx = torch.full((U, kmax), 777, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(U, dtype=torch.int32, device="cuda")
+    n_p = torch.zeros(U, dtype=torch.int32, device="cuda")
+    csa.csa_select_topp(s, U, C, scale, p, budget, n_sink, n_local, idx, cnt, kmax, n_p)
+    return parity.gpu_sets(idx, cnt), n_p.cpu().numpy()
+
+
+def test_select_topp_golden(csa):
+    for c in pins_golden("topp_cases.json"):
+        s = torch.tensor([c["scores"]], dtype=torch.float32, device="cuda")
+        got, n_p = _run_topp(csa, s, c["logit_scale"], c["p"], c["budget"], c["n_sink"],
+                             c["n_local"])
+        assert got[0] == c["expect"], c["why"]
+        if c["n_p"] <= c["budget"]:
+            assert n_p[0] == c["n_p"], c["why"]
+
+
+@pytest.mark.parametrize("C,U,budget,spread", [(1024, 6, 256, 4.0), (1024, 6, 256, 40.0),
+                                               (100, 8, 64, 10.0), (2000, 3, 2048, 3.0),
+                                               (37, 5, 5, 1.0)])
+def test_select_topp_vs_oracle(csa, C, U, budget, spread):
+    """Same fp32 scores; the mass cut is fp32 on the GPU and fp64 in the oracle,
+    so a mismatch is accepted only at a near-tie (reported)."""
+    s = _randn((U, C), 11) * spread
+    scale = 1.0 / math.sqrt(128)
+    for p in [0.5, 0.9, 0.99]:
+        got, n_p = _run_topp(csa, s, scale, p, budget, 1, 2)
+        sn = s.cpu().double().numpy()
+        refs, gaps = [], []
+        for u in range(U):
+            r, rn, gap = O.select_topp(sn[u], scale, p, budget, 1, 2)
+            refs.append(r)
+            gaps.append(gap)
+            if rn <= budget and got[u] == r:
+                assert n_p[u] == rn
+        parity.compare_sets(got, refs, gaps, f"topp C={C} p={p}")
+
+
+# ---------------------------------------------------------------- hierarchical
+
+@pytest.mark.parametrize("D,C,Gm,top_meta,k_free,G", [(128, 8192, 32, 8, 32, 4),
+                                                      (64, 1024, 16, 5, 20, 2),
+                                                      (128, 640, 64, 10, 700, 4)])
+def test_select_hier_vs_oracle(csa, D, C, Gm, top_meta, k_free, G):
+    B, Hkv = 2, 2
+    Hq = G * Hkv
+    q = _randn((B, Hq, D), 12, torch.bfloat16)
+    summ = _randn((B, Hkv, C, D), 13) * 0.1
+    meta = torch.empty(B, Hkv, C // Gm, D, device="cuda")
+    csa.csa_meta_summaries(summ, B, Hkv, C, D, Gm, meta)
+    kmax = min(C, k_free + 3)
+    idx = torch.full((B * Hkv, kmax), 777, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B * Hkv, dtype=torch.int32, device="cuda")
+    csa.csa_select_hier(q, q.dtype, meta, summ, B, Hq, Hkv, D, C, Gm, top_meta, k_free, 1, 2,
+                        idx, cnt, kmax)
+    got = parity.gpu_sets(idx, cnt)
+    qn, mn, sn = to_np(q), to_np(meta), to_np(summ)
+    refs, gaps = [], []
+    for b in range(B):
+        for h in range(Hkv):
+            r, g1, g2 = O.select_hier(qn[b, h * G:(h + 1) * G], mn[b, h], sn[b, h], Gm, top_meta,
+                                      k_free, 1, 2)
+            refs.append(r)
+            gaps.append(min(g1, g2))
+    parity.compare_sets(got, refs, gaps, "hier")
+
+
+def test_select_hier_golden(csa):
+    for c in pins_golden("hier_cases.json"):
+        qv = np.array(c["q"], dtype=np.float32)  # [G, 1] scalars
+        G = qv.shape[0]
+        D = 64
+        summ_s = np.array(c["summ"], dtype=np.float32)
+        C = len(summ_s)
+        q = torch.zeros(1, G, D, device="cuda")
+        q[0, :, 0] = torch.tensor(qv[:, 0])
+        summ = torch.zeros(1, 1, C, D, device="cuda")
+        summ[0, 0, :, 0] = torch.tensor(summ_s)
+        meta = torch.empty(1, 1, C // c["Gm"], D, device="cuda")
+        csa.csa_meta_summaries(summ, 1, 1, C, D, c["Gm"], meta)
+        kmax = C
+        idx = torch.full((1, kmax), 777, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+        csa.csa_select_hier(q, torch.float32, meta, summ, 1, G, 1, D, C, c["Gm"], c["top_meta"],
+                            c["k_free"], c["n_sink"], c["n_local"], idx, cnt, kmax)
+        assert parity.gpu_sets(idx, cnt)[0] == c["expect"], c["why"]
+
+
+# ---------------------------------------------------------------- merge
+
+def test_lse_merge(csa):
+    rows, S, D = 37, 20, 128
+    o = _randn((rows, S, D), 14)
+    lse = _randn((rows, S), 15) * 3
+    lse[::2, 5:] = -math.inf
+    lse[3, :] = -math.inf  # a row with no tokens at all
+    out = torch.empty(rows, D, device="cuda")
+    lo = torch.empty(rows, device="cuda")
+    csa.csa_lse_merge(o, lse, rows, S, D, out, torch.float32, lo)
+    ro, rl = O.lse_merge(to_np(o), to_np(lse))
+    assert np.abs(out.cpu().double().numpy() - ro).max() < 1e-5
+    got_l = lo.cpu().double().numpy()
+    assert np.isneginf(got_l[3]) and np.all(out[3].cpu().numpy() == 0)
+    fin = np.isfinite(rl)
+    assert np.abs(got_l[fin] - rl[fin]).max() < 1e-5
+    outb = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
+    csa.csa_lse_merge(o, lse, rows, S, D, outb, torch.bfloat16, None)
+    assert np.abs(outb.float().cpu().double().numpy() - ro).max() < 2e-2
+
+
+# ---------------------------------------------------------------- decode
+
+def _decode_case(csa, dtype, B, Hkv, G, D, T, L, sets, full=(), num_parts=0, max_splits=None,
+                 seed=16):
+    Hq = G * Hkv
+    C = T // L
+    dt = _dt(dtype)
+    q = _randn((B, Hq, D), seed, dt)
+    K = _randn((B, Hkv, T, D), seed + 1, dt)
+    V = _randn((B, Hkv, T, D), seed + 2, dt)
+    U = B * Hkv
+    kmax = max(1, max(len(s) for s in sets))
+    idx = torch.full((U, kmax), -1, dtype=torch.int32)
+    cnt = torch.zeros(U, dtype=torch.int32)
+    for u, s in enumerate(sets):
+        idx[u, :len(s)] = torch.tensor(sorted(s), dtype=torch.int32)
+        cnt[u] = len(s)
+    idx, cnt = idx.cuda(), cnt.cuda()
+    hf = None
+    if full:
+        hf = torch.zeros(Hkv, dtype=torch.uint8)
+        hf[list(full)] = 1
+        hf = hf.cuda()
+    P = num_parts or csa.csa_decode_default_parts(dt, D, L)
+    S = max_splits or P
+    o_part = torch.full((B, Hq, S, D), float("nan"), device="cuda")
+    lse_part = torch.full((B, Hq, S), float("nan"), device="cuda")
+    scale = 1.0 / math.sqrt(D)
+    csa.csa_sparse_decode(q, K, V, dt, idx, cnt, kmax, hf, B, Hq, Hkv, D, T, L, scale, num_parts,
+                          S, o_part, lse_part)
+    out = torch.empty(B, Hq, D, device="cuda")
+    lse = torch.empty(B, Hq, device="cuda")
+    csa.csa_lse_merge(o_part, lse_part, B * Hq, S, D, out, torch.float32, lse)
+    csa.csa_check_device_status()
+    eff = [list(range(C)) if (u % Hkv) in full else sorted(s) for u, s in enumerate(sets)]
+    qn = to_np(q)
+    Kc, Vc = K.cpu(), V.cpu()
+    # merged output per unit
+    for u, s in enumerate(eff):
+        b, h = divmod(u, Hkv)
+        ro, rl = O.decode_unit(qn[b, h * G:(h + 1) * G], to_np(Kc[b, h]), to_np(Vc[b, h]), s, L,
+                               scale)
+        got = out[b, h * G:(h + 1) * G].cpu().double().numpy()
+        if not s:
+            assert np.all(got == 0) and np.all(np.isneginf(lse[b, h * G:(h + 1) * G].cpu().numpy()))
+            continue
+        parity.assert_close(got, ro, dtype, f"decode unit {u}")
+        assert np.abs(lse[b, h * G:(h + 1) * G].cpu().double().numpy() - rl).max() < 1e-3
+    # every split partial against the oracle over that split's chunks
+    spl = O.decode_partition([len(s) for s in eff], P)
+    op, lp = o_part.cpu(), lse_part.cpu()
+    for u, s in enumerate(eff):
+        b, h = divmod(u, Hkv)
+        for slot in range(S):
+            rows = slice(h * G, (h + 1) * G)
+            if slot < len(spl[u]):
+                a0, a1 = spl[u][slot]
+                ro, rl = O.decode_unit(qn[b, rows], to_np(Kc[b, h]), to_np(Vc[b, h]), s[a0:a1], L,
+                                       scale)
+                parity.assert_close(op[b, rows, slot].double().numpy(), ro, dtype,
+                                    f"partial u{u} s{slot}")
+                assert np.abs(lp[b, rows, slot].double().numpy() - rl).max() < 1e-3
+            else:
+                assert torch.all(torch.isneginf(lp[b, rows, slot])), (u, slot)
+
+
+@pytest.mark.parametrize("dtype,D,L,G", [("bf16", 128, 128, 4), ("bf16", 128, 64, 4),
+                                         ("bf16", 64, 64, 8), ("bf16", 64, 128, 1),
+                                         ("bf16", 128, 64, 2), ("f32", 64, 64, 4),
+                                         ("f32", 128, 128, 8)])
+def test_sparse_decode_shapes(csa, dtype, D, L, G):
+    B, Hkv, C = 2, 3, 24
+    rng = np.random.default_rng(D + L + G)
+    sets = [sorted(rng.choice(C, size=int(rng.integers(1, 12)), replace=False).tolist())
+            for _ in range(B * Hkv)]
+    _decode_case(csa, dtype, B, Hkv, G, D, C * L, L, sets, num_parts=13)
+
+
+def test_sparse_decode_edge_cases(csa):
+    # empty unit, single chunk, a full head, more pieces than chunks, one piece
+    B, Hkv, G, D, L, C = 1, 4, 4, 128, 64, 9
+    sets = [[], [0], [2, 5, 8], [0, 1, 2, 3, 4, 5, 6, 7, 8]]
+    _decode_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=40, max_splits=45)
+    _decode_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=1)
+    _decode_case(csa, "bf16", B, Hkv, G, D, C * L, L, [[3], [0, 8], [], [1]], full=(2,),
+                 num_parts=7)
+    _decode_case(csa, "f32", B, Hkv, G, 64, C * L, L, sets, num_parts=40, max_splits=45)
+    # T == L: one chunk per head
+    _decode_case(csa, "bf16", 2, 2, 4, 128, 128, 128, [[0], [0], [], [0]], num_parts=3)
+
+
+def test_sparse_decode_mixed_heads_default_parts(csa):
+    """Full heads (every chunk) and sparse heads in one launch, default grid."""
+    B, Hkv, G, D, L, C = 1, 8, 4, 128, 128, 96
+    rng = np.random.default_rng(3)
+    sets = [sorted(rng.choice(C, size=20, replace=False).tolist()) for _ in range(B * Hkv)]
+    _decode_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, full=(0, 1))
+
+
+def test_device_index_error_reported(csa):
+    """An out-of-range chunk index is caught by the kernel's own check (the
+    chunk is replaced by chunk 0), reported by csa_check_device_status, and
+    the status is cleared afterwards."""
+    B, Hkv, G, D, L, C = 1, 1, 4, 128, 64, 4
+    q = _randn((B, G, D), 20, torch.bfloat16)
+    K = _randn((B, Hkv, C * L, D), 21, torch.bfloat16)
+    idx = torch.tensor([[0, 99]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([2], dtype=torch.int32, device="cuda")
+    o = torch.empty(B, G, 4, D, device="cuda")
+    l = torch.empty(B, G, 4, device="cuda")
+    csa.csa_sparse_decode(q, K, K, torch.bfloat16, idx, cnt, 2, None, B, G, Hkv, D, C * L, L, 0.1,
+                          4, 4, o, l)
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_check_device_status()
+    assert ei.value.status == 5
+    csa.csa_check_device_status()  # cleared
+
+
+def test_bounded_wait_times_out_without_trap(csa):
+    """A wait on a barrier nothing arrives on ends as CSA_ERR_TIMEOUT after the
+    limit; the context stays usable."""
+    csa.csa_selftest_wait_timeout(20_000_000)  # 20 ms
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_check_device_status()
+    assert ei.value.status == 4
+    csa.csa_check_device_status()
+    x = torch.ones(1000, device="cuda")
+    assert float(x.sum()) == 1000.0
+
+
+def test_host_pointer_rejected(csa):
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16)  # host memory
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_sparse_decode(q, q, q, torch.bfloat16, q, q, 1, None, 1, 4, 1, 128, 128, 128, 0.1,
+                              1, 1, q, q)
+    assert ei.value.status == 1

@@ -1,0 +1,105 @@
+"""Whole decode steps through the C ABI (summaries -> score -> select ->
+sparse split-K decode -> LSE merge) against the oracle's independent chain
+on the same seeded inputs: reduced sizes first, then the full workload sizes
+(every unit where the oracle finishes in seconds, sampled units at 1M)."""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from oracle import csa_oracle as O
+from oracle import pipeline as OP
+from oracle.pipeline import to_np
+from query_adaptive_chunk_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _decoder(w, inp):
+    from query_adaptive_chunk_b200.steps import SparseDecoder
+    return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
+                         n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
+                         budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta)
+
+
+def run_and_check(w, units=None):
+    from query_adaptive_chunk_b200 import csa
+    inp = synth.make_decode_inputs(w, device="cuda")
+    dec = _decoder(w, inp)
+    out, lse = dec.step(inp["q"])
+    csa.csa_check_device_status()
+    all_units = synth.decode_units(w)
+    units = units or all_units
+    ref = OP.decode_step(inp["q"], inp["K"], inp["V"], L=w.L, scale=w.scale, select=w.select,
+                         n_sink=w.n_sink, n_local=w.n_local, k_free=w.k_free,
+                         proj=inp.get("proj"), p=w.p, budget=w.budget, full_heads=w.full_heads,
+                         Gm=w.Gm, top_meta=w.top_meta, units=units)
+    gsets_all = parity.gpu_sets(dec.idx, dec.count)
+    sparse = [u for u in units if u[1] not in w.full_heads]
+    uidx = {u: i for i, u in enumerate(all_units)}
+    n_tie = parity.compare_sets([gsets_all[uidx[u]] for u in sparse],
+                                [ref["sets"][u] for u in sparse],
+                                [ref["gap"][u] for u in sparse], w.name)
+    G = w.G
+    worst = 0.0
+    for (b, h) in units:
+        got = out[b, h * G:(h + 1) * G].cpu().double().numpy()
+        gset = list(range(w.C)) if h in w.full_heads else gsets_all[uidx[(b, h)]]
+        if gset == ref["sets"][(b, h)]:
+            ro, rl = ref["o"][(b, h)], ref["lse"][(b, h)]
+        else:  # near-tie: check attention over the GPU's own set
+            ro, rl = O.decode_unit(to_np(inp["q"][b, h * G:(h + 1) * G]), to_np(inp["K"][b, h]),
+                                   to_np(inp["V"][b, h]), gset, w.L, w.scale)
+        mx, _ = parity.assert_close(got, ro, w.dtype, f"{w.name} unit {(b, h)}")
+        worst = max(worst, mx)
+        assert np.abs(lse[b, h * G:(h + 1) * G].cpu().double().numpy() - rl).max() < 1e-3
+    if w.select == "topp":
+        n_p = dec.n_p.cpu().numpy()
+        for (b, h) in sparse:
+            rn = ref["n_p"][(b, h)]
+            if rn <= w.budget:
+                assert n_p[uidx[(b, h)]] == rn or ref["gap"][(b, h)] < parity.NEAR_TIE
+            else:
+                assert n_p[uidx[(b, h)]] == w.budget + 1 or ref["gap"][(b, h)] < parity.NEAR_TIE
+    print(f"{w.name}: units {len(units)} near-ties {n_tie} worst max-abs {worst:.3g}")
+    return dec, inp
+
+
+def test_tiny_f32_decode():
+    run_and_check(synth.TINY_F32)
+
+
+def test_topk_decode_reduced():
+    run_and_check(synth.TOPK_32K.scaled(B=2, T=8192))
+
+
+def test_topk_decode_full_size():
+    run_and_check(synth.TOPK_32K)
+
+
+def test_topp_decode_prefix_cut():
+    """C = 128 < budget: the cap cannot bind, the mass cut p decides."""
+    run_and_check(synth.TOPP_128K.scaled(T=16384))
+
+
+def test_topp_decode_reduced():
+    run_and_check(synth.TOPP_128K.scaled(T=65536))
+
+
+def test_topp_mixed_decode_full_size():
+    run_and_check(synth.TOPP_128K)
+
+
+def test_hier_decode_reduced():
+    run_and_check(synth.HIER_1M.scaled(T=131072, planted=8))
+
+
+def test_hier_decode_full_size_sampled():
+    run_and_check(synth.HIER_1M, units=[(0, 0), (0, 5)])
+
+
+def test_decode_batch_with_gqa8_and_d64():
+    w = synth.DecodeWorkload(name="topk_gqa8_d64", seed=11, B=3, Hq=16, Hkv=2, D=64, T=64 * 40,
+                             L=64, dtype="bf16", select="topk", n_sink=1, n_local=2, k_free=9,
+                             planted=3)
+    run_and_check(w)
