@@ -165,6 +165,20 @@ def recorded_traffic(kernel_file: str, name: str):
     return e.get("bytes_per_launch")
 
 
+def make_flush(dev):
+    """Evict the inputs from L2 between timed steps: write a 256 MB buffer,
+    then read another 256 MB buffer so that the dirty lines of the write are
+    written back before the next timed step starts (not inside it)."""
+    wbuf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        wbuf.zero_()
+        rbuf.sum()
+
+    return flush
+
+
 def decoder_for(w, inp):
     from query_adaptive_chunk_b200.steps import SparseDecoder
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
@@ -379,10 +393,9 @@ def run_ours(args):
     dist = dist_init(world, "nccl")
     dev = torch.device("cuda", local)
     peaks = load_peaks()
-    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def flush():
-        flush_buf.zero_()
+    flush = make_flush(dev)
+    if args.only:
+        return run_only(args, flush, load_peaks())
 
     w = rank_workload(HEADLINE, rank)
     if world > 1:
@@ -426,7 +439,7 @@ def run_ours(args):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "ctx": w.T,
                    "L": w.L, "select": "top-p p=0.9 cap 256 + sink + 2 local",
                    "full_heads": list(w.full_heads), "proj_rank": w.proj_rank,
-                   "l2": "flushed before every step (256 MB write)",
+                   "l2": "flushed before every step (256 MB write + 256 MB read)",
                    "timing": "CUDA-graph replay, events inside the graph" if r["graph"]
                              else "direct launches, CUDA events",
                    "parallelism": f"replicas x{world} (units shard, no collective)"},
@@ -480,6 +493,24 @@ def other_workloads(args, flush, peaks):
     return out
 
 
+def run_only(args, flush, peaks):
+    """Time one named workload alone and print its figures (profiling aid)."""
+    byname = {w.name: w for w in synth.ALL_WORKLOADS}
+    w = byname[args.only]
+    if isinstance(w, synth.PrefillWorkload):
+        r = time_prefill(w, args.steps, args.warmup, flush)
+        ms = statistics.mean(r["attend_ms"])
+        d = {"workload": w.name, "attend_ms": ms, "tflops": r["flops"] / (ms * 1e-3) / 1e12}
+    else:
+        r = time_decode(w, args.steps, args.warmup, flush)
+        us = 1000 * statistics.mean(r["step_ms"])
+        dus = 1000 * statistics.mean(r["decode_ms"])
+        d = {"workload": w.name, "us_per_step": us, "decode_us": dus,
+             "decode_gbs": r["kv_bytes"] / (dus * 1e-6) / 1e9}
+    print(json.dumps(d))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -488,6 +519,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None, help="time one named workload alone")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -225,7 +225,7 @@ CSA_API int csa_decode_default_parts(csa_dtype dtype, int D, int L);
  * gives out = 0, lse = -inf).
  *   o_part [rows, max_splits, D] fp32;  lse_part [rows, max_splits] fp32
  *   out [rows, D] of out_dtype (output);  lse_out NULL or [rows] fp32 (output)
- *   D % 4 == 0, D <= 512. */
+ *   D % 4 == 0, D <= 512, max_splits <= 16384. */
 CSA_API csa_status csa_lse_merge(const float* o_part, const float* lse_part, int rows, int max_splits,
                          int D, void* out, csa_dtype out_dtype, float* lse_out,
                          csa_stream stream);

@@ -372,6 +372,7 @@ csa_status csa_lse_merge(const float* o_part, const float* lse_part, int rows, i
   CSA_REQUIRE(valid_dtype(out_dtype), "out_dtype");
   CSA_REQUIRE(rows >= 0 && max_splits > 0 && D > 0, "bad sizes");
   CSA_SUPPORT(D % 4 == 0 && D <= 512, "D must be a multiple of 4, <= 512");
+  CSA_SUPPORT(max_splits <= 16384, "max_splits must be <= 16384");
   if (rows == 0) return CSA_OK;
   CSA_TRY(check_ptr(o_part, "o_part"));
   CSA_TRY(check_ptr(lse_part, "lse_part"));

@@ -105,13 +105,27 @@ __device__ __forceinline__ int64_t piece_of(int64_t g, int64_t N, int64_t P) {
   return ((g + 1) * P - 1) / N;
 }
 
+// Splits of a unit = the non-empty pieces meeting its range [lo, hi).  With
+// N >= P every piece holds >= 1 chunk; with N < P a non-empty piece holds
+// exactly one chunk, so splits are counted in chunks.
+__device__ __forceinline__ int split_count(int64_t lo, int64_t hi, int64_t N, int64_t P) {
+  if (hi <= lo) return 0;
+  return N >= P ? static_cast<int>(piece_of(hi - 1, N, P) - piece_of(lo, N, P) + 1)
+                : static_cast<int>(hi - lo);
+}
+
+// Split index, within unit [lo, ...), of the piece `c` that starts at chunk a.
+__device__ __forceinline__ int split_slot(int64_t lo, int64_t a, int64_t c, int64_t N, int64_t P) {
+  return N >= P ? static_cast<int>(c - piece_of(lo, N, P)) : static_cast<int>(a - lo);
+}
+
 // Slots of unit u beyond its split count get lse = -inf (CTA c covers units
 // u = c, c + P, ...).  Threads [0, nthreads) of the block take part.
 __device__ void fill_empty_slots(const DecodeParams& p, const int* prefix, int nthreads) {
   const int64_t N = prefix[p.U], P = gridDim.x;
   for (int u = blockIdx.x; u < p.U; u += gridDim.x) {
     const int64_t lo = prefix[u], hi = prefix[u + 1];
-    const int nsplit = hi > lo ? static_cast<int>(piece_of(hi - 1, N, P) - piece_of(lo, N, P) + 1) : 0;
+    const int nsplit = split_count(lo, hi, N, P);
     const int b = u / p.Hkv, h = u % p.Hkv;
     const int nfill = p.max_splits - nsplit;
     for (int e = threadIdx.x; e < p.G * nfill; e += nthreads) {
@@ -293,7 +307,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     if (!group_sync()) return false;
     const int b = u / p.Hkv, h = u % p.Hkv;
-    const int slot = static_cast<int>(blockIdx.x - piece_of(prefix[u], N, P));
+    const int slot = split_slot(prefix[u], a, blockIdx.x, N, P);
     for (int e = threadIdx.x; e < p.G * D; e += kConsumerWarps * 32) {
       const int g = e / D, d = e % D;
       float M = -INFINITY;
@@ -433,7 +447,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
 
   auto flush = [&](int u) {
     const int b = u / p.Hkv, h = u % p.Hkv;
-    const int slot = static_cast<int>(blockIdx.x - piece_of(prefix[u], N, P));
+    const int slot = split_slot(prefix[u], a, blockIdx.x, N, P);
     for (int g = 0; g < G; ++g) {
       const int64_t row = static_cast<int64_t>(b) * p.Hq + h * G + g;
       if (tid < D) p.o_part[(row * p.max_splits + slot) * D + tid] = o[g] / lh[g];
@@ -501,50 +515,98 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
 // ------------------------------------------------------------------ merge
 
 constexpr int kMergeThreads = 128;
+constexpr int kMergeWarps = kMergeThreads / 32;
 
+// One CTA per row.  The valid slots (lse > -inf) are compacted in slot order
+// with their weights exp(lse_s - lse); warp w then accumulates slots w, w+4,
+// ... over its lanes' float4 columns and the four partial sums are added in
+// a fixed order, so the result does not depend on timing.
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part, int rows, int S, int D,
     void* __restrict__ out, int out_bf16, float* __restrict__ lse_out) {
+  extern __shared__ __align__(16) float msm[];
+  float* acc_sh = msm;                                        // [kMergeWarps][D] (float4 stores)
+  float* wts = msm + kMergeWarps * D;                         // [S]
+  int* slots = reinterpret_cast<int*>(wts + S);               // [S]
+  __shared__ int scan_sh[33];
+  __shared__ float red[kMergeWarps];
+  __shared__ float lse_sh;
+  const int r = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * (kMergeThreads / 32) + warp;
-  if (r >= rows) return;
   const float* lrow = lse_part + static_cast<int64_t>(r) * S;
+  // row max
   float mx = -INFINITY;
-  for (int s = lane; s < S; s += 32) mx = fmaxf(mx, lrow[s]);
+  for (int s = threadIdx.x; s < S; s += kMergeThreads) mx = fmaxf(mx, lrow[s]);
 #pragma unroll
   for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
-  float tot = 0.f;
-  if (mx != -INFINITY)
-    for (int s = lane; s < S; s += 32) {
-      const float v = lrow[s];
-      if (v != -INFINITY) tot += expf(v - mx);
-    }
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
 #pragma unroll
-  for (int x = 16; x > 0; x >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, x);
-  const float lse = mx == -INFINITY ? -INFINITY : mx + logf(tot);
-  if (lane == 0 && lse_out) lse_out[r] = lse;
-  const int nv = D / 4;
-  for (int v4 = lane; v4 < nv; v4 += 32) {
+  for (int w = 1; w < kMergeWarps; ++w) mx = fmaxf(mx, red[w]);
+  __syncthreads();
+  // ordered compaction of the valid slots (contiguous segments per thread)
+  const int seg = (S + kMergeThreads - 1) / kMergeThreads;
+  const int lo = min(S, static_cast<int>(threadIdx.x) * seg), hi = min(S, lo + seg);
+  int nv = 0;
+  for (int s = lo; s < hi; ++s) nv += (mx != -INFINITY && lrow[s] != -INFINITY);
+  int total = 0;
+  int pos = block_exclusive_scan(nv, scan_sh, &total);
+  for (int s = lo; s < hi; ++s)
+    if (mx != -INFINITY && lrow[s] != -INFINITY) {
+      slots[pos] = s;
+      wts[pos] = expf(lrow[s] - mx);
+      ++pos;
+    }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int i = 0; i < total; ++i) tot += wts[i];
+    lse_sh = total > 0 ? mx + logf(tot) : -INFINITY;
+    if (lse_out) lse_out[r] = lse_sh;
+    const float inv = total > 0 ? 1.0f / tot : 0.f;
+    for (int i = 0; i < total; ++i) wts[i] *= inv;
+  }
+  __syncthreads();
+  const int nv4 = D / 4;
+  for (int v4 = lane; v4 < nv4; v4 += 32) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (mx != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const float l = lrow[s];
-        if (l == -INFINITY) continue;
-        const float w = expf(l - lse);
-        const float4 x = __ldg(reinterpret_cast<const float4*>(o_part + (static_cast<int64_t>(r) * S + s) * D) + v4);
-        acc.x += w * x.x;
-        acc.y += w * x.y;
-        acc.z += w * x.z;
-        acc.w += w * x.w;
+    int i = warp;
+    for (; i + 3 * kMergeWarps < total; i += 4 * kMergeWarps) {
+      float4 x[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        x[k] = __ldg(reinterpret_cast<const float4*>(
+                         o_part + (static_cast<int64_t>(r) * S + slots[i + k * kMergeWarps]) * D) + v4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float wgt = wts[i + k * kMergeWarps];
+        acc.x += wgt * x[k].x;
+        acc.y += wgt * x[k].y;
+        acc.z += wgt * x[k].z;
+        acc.w += wgt * x[k].w;
       }
     }
-    if (out_bf16) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out) + static_cast<int64_t>(r) * D + v4 * 4;
-      reinterpret_cast<uint32_t*>(ob)[0] = pack_bf16x2(acc.x, acc.y);
-      reinterpret_cast<uint32_t*>(ob)[1] = pack_bf16x2(acc.z, acc.w);
-    } else {
-      reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(r) * D)[v4] = acc;
+    for (; i < total; i += kMergeWarps) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(
+                                 o_part + (static_cast<int64_t>(r) * S + slots[i]) * D) + v4);
+      const float wgt = wts[i];
+      acc.x += wgt * x.x;
+      acc.y += wgt * x.y;
+      acc.z += wgt * x.z;
+      acc.w += wgt * x.w;
     }
+    reinterpret_cast<float4*>(acc_sh + warp * D)[v4] = acc;
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += kMergeThreads) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) v += acc_sh[w * D + d];
+    if (out_bf16)
+      static_cast<__nv_bfloat16*>(out)[static_cast<int64_t>(r) * D + d] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(out)[static_cast<int64_t>(r) * D + d] = v;
   }
 }
 
@@ -632,9 +694,14 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
 cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_part, int rows,
                          int max_splits, int D, void* out, bool out_bf16, float* lse_out) {
   if (rows == 0) return cudaSuccess;
-  const int per = kMergeThreads / 32;
-  merge_kernel<<<(rows + per - 1) / per, kMergeThreads, 0, l.stream>>>(
-      o_part, lse_part, rows, max_splits, D, out, out_bf16 ? 1 : 0, lse_out);
+  const size_t sh = (2 * static_cast<size_t>(max_splits) + kMergeWarps * D) * 4;
+  if (sh > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sh));
+    if (e != cudaSuccess) return e;
+  }
+  merge_kernel<<<rows, kMergeThreads, sh, l.stream>>>(o_part, lse_part, rows, max_splits, D, out,
+                                                      out_bf16 ? 1 : 0, lse_out);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(
   constexpr int ROWS_CTA = ROWS_WARP * kScoreWarps;
   __shared__ float qs[1024];
   __shared__ float qp[DS];
+  __shared__ float qpart[kScoreThreads];
 
   const int u = blockIdx.z;  // b * Hkv + h
   const int n = blockIdx.y;
@@ -47,10 +48,22 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(
   __syncthreads();
   const float* qv = qs;
   if (proj != nullptr) {
-    for (int r = threadIdx.x; r < R; r += kScoreThreads) {
-      float acc = 0.f;
-      for (int d = 0; d < D; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * qs[d];
-      qp[r] = acc;
+    // qp[r] = sum_d proj[d, r] qs[d]: the 256 threads split the d range into
+    // 256/R parts, each a short run of independent loads, then R threads add
+    // the parts in a fixed order
+    const int parts = kScoreThreads / R;
+    const int r = threadIdx.x % R, part = threadIdx.x / R;
+    const int dchunk = (D + parts - 1) / parts;
+    const int d0 = part * dchunk, d1 = min(D, d0 + dchunk);
+    float acc = 0.f;
+#pragma unroll 4
+    for (int d = d0; d < d1; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * qs[d];
+    qpart[part * R + r] = acc;
+    __syncthreads();
+    if (threadIdx.x < R) {
+      float t = 0.f;
+      for (int k = 0; k < parts; ++k) t += qpart[k * R + threadIdx.x];
+      qp[threadIdx.x] = t;
     }
     __syncthreads();
     qv = qp;

@@ -250,6 +250,22 @@ __global__ void __launch_bounds__(kSelThreads) select_topp_kernel(
   // the nb best chunks (by score, lower index first) into flags as a pool
   const int nb = min(budget, C);
   choose_best(keys, C, C, nb, flags, s);
+  // if even those nb chunks hold less than p of the mass, n_p > budget and the
+  // cap decides: the pool is the answer, no ordering of it is needed
+  {
+    float mpart = 0.f;
+    for (int c = threadIdx.x; c < C; c += blockDim.x)
+      if (flags[c]) mpart += expf((key_to_float(keys[c]) - mx) * logit_scale);
+    const float mass_nb = block_sum(mpart, s);
+    if (nb < C && mass_nb < p * Z) {
+      for (int c = threadIdx.x; c < C; c += blockDim.x)
+        if (is_forced(c, C, n_sink, n_local)) flags[c] = 1;
+      __syncthreads();
+      if (n_p_out && threadIdx.x == 0) n_p_out[u] = nb + 1;
+      emit_ascending(flags, C, idx + static_cast<int64_t>(u) * kmax, count + u, kmax, s);
+      return;
+    }
+  }
   // compact them, in index order, into the sort buffer as 64-bit keys
   {
     const int seg = (C + blockDim.x - 1) / blockDim.x;
