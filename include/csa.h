@@ -217,6 +217,54 @@ CSA_API csa_status csa_sparse_decode(const void* q, const void* K, const void* V
  * current device (a multiple of the SM count); < 0 on error. */
 CSA_API int csa_decode_default_parts(csa_dtype dtype, int D, int L);
 
+/* Fused a1 + a2 (decode, Nq = 1): the scores of csa_score_chunks computed
+ * straight into shared memory, one CTA per unit, then the top-k of
+ * csa_select_topk; same arithmetic, so the index lists equal the two-call
+ * path's bit for bit.  Units of heads with head_full[h] != 0 get count 0 and
+ * an all -1 row (csa_sparse_decode reads every chunk for them).
+ *   q [B, Hq, D];  proj NULL or [D, R];  summ [B, Hkv, C, Ds] fp32
+ *   idx [B*Hkv, kmax], count [B*Hkv] (outputs);  same limits as the two calls. */
+CSA_API csa_status csa_score_select_topk(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                         const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                         const uint8_t* head_full, int k_free, int n_sink,
+                                         int n_local, int32_t* idx, int32_t* count, int kmax,
+                                         csa_stream stream);
+
+/* Fused a1 + a3 (decode): csa_score_chunks then csa_select_topp in one CTA
+ * per unit (bit-identical to the two calls); full heads as above (n_p_out 0). */
+CSA_API csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                         const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                         const uint8_t* head_full, float logit_scale, float p,
+                                         int budget, int n_sink, int n_local, int32_t* idx,
+                                         int32_t* count, int kmax, int32_t* n_p_out,
+                                         csa_stream stream);
+
+/* Bytes of device workspace csa_sparse_decode_merged needs (num_parts 0 =
+ * the default piece count of the current device); < 0 on bad sizes. */
+CSA_API int64_t csa_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int num_parts);
+
+/* a5 + a6 in one launch (SSA summary "핵심 기여": split-K partials combined):
+ * the decode of csa_sparse_decode, after which the last CTA to finish a unit
+ * merges that unit's splits (the log-sum-exp merge of csa_lse_merge) into
+ *   out[b, h*G+g, :] (out_dtype) and lse_out[b, h*G+g] (natural log; NULL ok).
+ * A unit with a single split writes its output directly; a unit with no
+ * chunks gets out = 0, lse = -inf.
+ * `workspace` (caller-owned device memory, >= csa_decode_workspace_bytes())
+ * holds the split partials and one arrival counter per unit.  The counters
+ * must be zero before the first call (zero the workspace once); every call
+ * that completes leaves them zero again.  After a call that reported
+ * CSA_ERR_TIMEOUT, zero the workspace before reusing it.  Calls that share a
+ * workspace must not overlap on the GPU.
+ *   num_parts <= 256 (0 = default); other arguments as csa_sparse_decode. */
+CSA_API csa_status csa_sparse_decode_merged(const void* q, const void* K, const void* V,
+                                            csa_dtype dtype, const int32_t* idx,
+                                            const int32_t* count, int kmax,
+                                            const uint8_t* head_full, int B, int Hq, int Hkv,
+                                            int D, int64_t T, int L, float scale, int num_parts,
+                                            void* workspace, int64_t workspace_bytes, void* out,
+                                            csa_dtype out_dtype, float* lse_out,
+                                            csa_stream stream);
+
 /* ---------------------------------------------------------------- a6
  * Log-sum-exp merge of split-K partials (SSA summary "핵심 기여": split-K
  * partials combined):

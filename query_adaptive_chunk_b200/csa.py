@@ -55,6 +55,13 @@ _SIGS = {
     "csa_sparse_decode": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i64, _i, _f,
                                _i, _i, _vp, _vp, _vp]),
     "csa_decode_default_parts": (_i, [_i, _i, _i]),
+    "csa_score_select_topk": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i,
+                                   _vp, _vp, _i, _vp]),
+    "csa_score_select_topp": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _f, _f, _i,
+                                   _i, _i, _vp, _vp, _i, _vp, _vp]),
+    "csa_decode_workspace_bytes": (_i64, [_i, _i, _i, _i, _i]),
+    "csa_sparse_decode_merged": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i64,
+                                      _i, _f, _i, _vp, _i64, _vp, _i, _vp, _vp]),
     "csa_lse_merge": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp]),
     "csa_block_sparse_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                       _vp, _vp]),
@@ -172,6 +179,36 @@ def csa_decode_default_parts(dtype, D, L) -> int:
     if n < 0:
         raise CsaError(3, csa_last_error_string())
     return n
+
+
+def csa_score_select_topk(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full, k_free, n_sink,
+                          n_local, idx, count, kmax, stream=None):
+    _check(lib.csa_score_select_topk(_p(q), _dt(q_dtype), _p(proj), R, _p(summ), B, Hq, Hkv, D, C,
+                                     _p(head_full), k_free, n_sink, n_local, _p(idx), _p(count),
+                                     kmax, _s(stream)))
+
+
+def csa_score_select_topp(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full, logit_scale, p,
+                          budget, n_sink, n_local, idx, count, kmax, n_p_out=None, stream=None):
+    _check(lib.csa_score_select_topp(_p(q), _dt(q_dtype), _p(proj), R, _p(summ), B, Hq, Hkv, D, C,
+                                     _p(head_full), logit_scale, p, budget, n_sink, n_local,
+                                     _p(idx), _p(count), kmax, _p(n_p_out), _s(stream)))
+
+
+def csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts) -> int:
+    n = lib.csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts)
+    if n < 0:
+        raise CsaError(1, "csa_decode_workspace_bytes: bad sizes")
+    return n
+
+
+def csa_sparse_decode_merged(q, K, V, dtype, idx, count, kmax, head_full, B, Hq, Hkv, D, T, L,
+                             scale, num_parts, workspace, workspace_bytes, out, out_dtype, lse_out,
+                             stream=None):
+    _check(lib.csa_sparse_decode_merged(_p(q), _p(K), _p(V), _dt(dtype), _p(idx), _p(count), kmax,
+                                        _p(head_full), B, Hq, Hkv, D, T, L, scale, num_parts,
+                                        _p(workspace), workspace_bytes, _p(out), _dt(out_dtype),
+                                        _p(lse_out), _s(stream)))
 
 
 def csa_lse_merge(o_part, lse_part, rows, max_splits, D, out, out_dtype, lse_out, stream=None):

@@ -328,15 +328,16 @@ int csa_decode_default_parts(csa_dtype dtype, int D, int L) {
   return csa::decode_default_parts(dtype == CSA_BF16, D, L, l.num_sms);
 }
 
-csa_status csa_sparse_decode(const void* q, const void* K, const void* V, csa_dtype dtype,
-                             const int32_t* idx, const int32_t* count, int kmax,
-                             const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T, int L,
-                             float scale, int num_parts, int max_splits, float* o_part,
-                             float* lse_part, csa_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// Shape checks shared by the two decode entry points (no CUDA call).
+csa_status decode_shape_checks(csa_dtype dtype, int kmax, int B, int Hq, int Hkv, int D, int64_t T,
+                               int L, float scale, int num_parts) {
   CSA_REQUIRE(valid_dtype(dtype), "dtype");
-  CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && T >= 0 && L > 0 && kmax > 0 && num_parts >= 0 &&
-                  max_splits > 0,
-              "bad sizes");
+  CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && T >= 0 && L > 0 && kmax > 0 && num_parts >= 0,
+              "B, T, num_parts must be non-negative; Hq, Hkv, L, kmax positive");
   CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
   CSA_REQUIRE(T % L == 0, "T must be a multiple of L");
   CSA_SUPPORT(D == 64 || D == 128, "D must be 64 or 128");
@@ -345,26 +346,170 @@ csa_status csa_sparse_decode(const void* q, const void* K, const void* V, csa_dt
   CSA_SUPPORT(G == 1 || G == 2 || G == 4 || G == 8, "Hq/Hkv must be 1, 2, 4 or 8");
   CSA_SUPPORT(static_cast<int64_t>(B) * Hkv <= 2048, "B*Hkv must be <= 2048");
   CSA_SUPPORT(static_cast<int64_t>(B) * Hkv * T < 2147483648LL, "B*Hkv*T must be < 2^31");
+  CSA_SUPPORT(num_parts <= 65535, "num_parts must be <= 65535");
   CSA_REQUIRE(scale == scale, "scale is NaN");
-  if (B == 0) return CSA_OK;
-  csa::Launch l;
-  CSA_TRY(launch_ctx(stream, &l));
-  const int P = num_parts > 0 ? num_parts : csa::decode_default_parts(dtype == CSA_BF16, D, L, l.num_sms);
-  CSA_REQUIRE(max_splits >= P, "max_splits must be >= the number of pieces (num_parts)");
-  CSA_SUPPORT(P <= 65535, "num_parts must be <= 65535");
+  return CSA_OK;
+}
+
+// Pointer checks shared by the two decode entry points; returns the piece count.
+csa_status decode_ptr_checks(const void* q, const void* K, const void* V, const int32_t* idx,
+                             const int32_t* count, const uint8_t* head_full, bool bf16, int D,
+                             int L, int num_parts, const csa::Launch& l, int* P_out) {
   CSA_TRY(check_ptr(q, "q"));
   CSA_TRY(check_ptr(K, "K"));
   CSA_TRY(check_ptr(V, "V"));
   CSA_TRY(check_ptr(head_full, "head_full", false));
   CSA_TRY(check_ptr(idx, "idx"));
   CSA_TRY(check_ptr(count, "count"));
+  *P_out = num_parts > 0 ? num_parts : csa::decode_default_parts(bf16, D, L, l.num_sms);
+  return CSA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WorkspaceLayout {
+  size_t counters, lse, o, total;
+};
+
+WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int D, int P) {
+  WorkspaceLayout w;
+  w.counters = 0;
+  w.lse = round256(static_cast<size_t>(B) * Hkv * 4);
+  w.o = w.lse + round256(static_cast<size_t>(B) * Hq * P * 4);
+  w.total = w.o + static_cast<size_t>(B) * Hq * P * D * 4;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+csa_status csa_sparse_decode(const void* q, const void* K, const void* V, csa_dtype dtype,
+                             const int32_t* idx, const int32_t* count, int kmax,
+                             const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T, int L,
+                             float scale, int num_parts, int max_splits, float* o_part,
+                             float* lse_part, csa_stream stream) {
+  CSA_REQUIRE(max_splits > 0, "max_splits must be positive");
+  CSA_TRY(decode_shape_checks(dtype, kmax, B, Hq, Hkv, D, T, L, scale, num_parts));
+  if (num_parts > 0) CSA_REQUIRE(max_splits >= num_parts, "max_splits must be >= num_parts");
+  if (B == 0) return CSA_OK;
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  int P = 0;
+  CSA_TRY(decode_ptr_checks(q, K, V, idx, count, head_full, dtype == CSA_BF16, D, L, num_parts, l, &P));
+  CSA_REQUIRE(max_splits >= P, "max_splits must be >= the number of pieces (num_parts)");
   CSA_TRY(check_ptr(o_part, "o_part"));
   CSA_TRY(check_ptr(lse_part, "lse_part"));
   std::string why;
   cudaError_t e = csa::launch_decode(l, q, K, V, dtype == CSA_BF16, idx, count, kmax, head_full, B, Hq,
-                                     Hkv, D, T, L, scale, P, max_splits, o_part, lse_part, &why);
+                                     Hkv, D, T, L, scale, P, max_splits, o_part, lse_part, nullptr, &why);
   if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
   return finish(e, "sparse decode launch");
+}
+
+int64_t csa_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int num_parts) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return -1;
+  int P = num_parts;
+  if (P <= 0) {
+    csa::Launch l;
+    if (launch_ctx(nullptr, &l) != CSA_OK) return -1;
+    P = csa::decode_default_parts(true, D, 128, l.num_sms);
+  }
+  return static_cast<int64_t>(workspace_layout(B, Hq, Hkv, D, P).total);
+}
+
+csa_status csa_sparse_decode_merged(const void* q, const void* K, const void* V, csa_dtype dtype,
+                                    const int32_t* idx, const int32_t* count, int kmax,
+                                    const uint8_t* head_full, int B, int Hq, int Hkv, int D,
+                                    int64_t T, int L, float scale, int num_parts, void* workspace,
+                                    int64_t workspace_bytes, void* out, csa_dtype out_dtype,
+                                    float* lse_out, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(out_dtype), "out_dtype");
+  CSA_TRY(decode_shape_checks(dtype, kmax, B, Hq, Hkv, D, T, L, scale, num_parts));
+  CSA_SUPPORT(num_parts <= csa::kMergedMaxParts, "num_parts must be <= 256 for the merged decode");
+  if (B == 0) return CSA_OK;
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  int P = 0;
+  CSA_TRY(decode_ptr_checks(q, K, V, idx, count, head_full, dtype == CSA_BF16, D, L, num_parts, l, &P));
+  CSA_SUPPORT(P <= csa::kMergedMaxParts, "num_parts must be <= 256 for the merged decode");
+  const WorkspaceLayout w = workspace_layout(B, Hq, Hkv, D, P);
+  CSA_REQUIRE(workspace_bytes >= static_cast<int64_t>(w.total),
+              "workspace smaller than csa_decode_workspace_bytes()");
+  CSA_TRY(check_ptr(workspace, "workspace"));
+  CSA_TRY(check_ptr(out, "out"));
+  CSA_TRY(check_ptr(lse_out, "lse_out", false));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  csa::MergeOut m{reinterpret_cast<int*>(ws + w.counters), out, out_dtype == CSA_BF16, lse_out};
+  std::string why;
+  cudaError_t e = csa::launch_decode(l, q, K, V, dtype == CSA_BF16, idx, count, kmax, head_full, B, Hq,
+                                     Hkv, D, T, L, scale, P, P, reinterpret_cast<float*>(ws + w.o),
+                                     reinterpret_cast<float*>(ws + w.lse), &m, &why);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  return finish(e, "merged sparse decode launch");
+}
+
+csa_status csa_score_select_topk(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                 const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                 const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                                 int32_t* idx, int32_t* count, int kmax, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
+  CSA_REQUIRE(kmax > 0, "kmax must be positive");
+  CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && D > 0 && C >= 0 && k_free >= 0 && n_sink >= 0 &&
+                  n_local >= 0,
+              "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_SUPPORT(D <= 1024 && C <= 32768, "D <= 1024 and C <= 32768");
+  const int Ds = proj ? R : D;
+  CSA_SUPPORT(Ds == 16 || Ds == 32 || Ds == 64 || Ds == 128, "summary width must be 16, 32, 64 or 128");
+  const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(k_free) + n_sink + n_local);
+  CSA_REQUIRE(kmax >= need, "kmax < min(C, k_free + n_sink + n_local)");
+  if (B == 0 || C == 0) return CSA_OK;
+  CSA_TRY(check_ptr(q, "q"));
+  CSA_TRY(check_ptr(proj, "proj", false));
+  CSA_TRY(check_ptr(summ, "summ"));
+  CSA_TRY(check_ptr(head_full, "head_full", false));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_score_select_topk(l, q, q_dtype == CSA_BF16, proj, R, summ, B, Hq, Hkv, D,
+                                              C, head_full, k_free, n_sink, n_local, idx, count, kmax),
+                "score_select_topk launch");
+}
+
+csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                 const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                 const uint8_t* head_full, float logit_scale, float p, int budget,
+                                 int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                                 int32_t* n_p_out, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
+  CSA_REQUIRE(kmax > 0, "kmax must be positive");
+  CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && D > 0 && C > 0 && n_sink >= 0 && n_local >= 0,
+              "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_REQUIRE(p > 0.f && p <= 1.f, "p must be in (0, 1]");
+  CSA_REQUIRE(budget >= 1, "budget must be >= 1");
+  CSA_REQUIRE(logit_scale == logit_scale, "logit_scale is NaN");
+  CSA_SUPPORT(budget <= 2048 && C <= 32768 && D <= 1024, "budget <= 2048, C <= 32768, D <= 1024");
+  const int Ds = proj ? R : D;
+  CSA_SUPPORT(Ds == 16 || Ds == 32 || Ds == 64 || Ds == 128, "summary width must be 16, 32, 64 or 128");
+  const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(budget) + n_sink + n_local);
+  CSA_REQUIRE(kmax >= need, "kmax < min(C, budget + n_sink + n_local)");
+  if (B == 0) return CSA_OK;
+  CSA_TRY(check_ptr(q, "q"));
+  CSA_TRY(check_ptr(proj, "proj", false));
+  CSA_TRY(check_ptr(summ, "summ"));
+  CSA_TRY(check_ptr(head_full, "head_full", false));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  CSA_TRY(check_ptr(n_p_out, "n_p_out", false));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_score_select_topp(l, q, q_dtype == CSA_BF16, proj, R, summ, B, Hq, Hkv, D,
+                                              C, head_full, logit_scale, p, budget, n_sink, n_local,
+                                              idx, count, kmax, n_p_out),
+                "score_select_topp launch");
 }
 
 csa_status csa_lse_merge(const float* o_part, const float* lse_part, int rows, int max_splits, int D,

@@ -45,13 +45,19 @@ struct DecodeParams {
   const int32_t* count;
   int kmax;
   const uint8_t* head_full;
-  int U, Hkv, G, Hq, C, L;
+  int U, Hkv, G, Hq, C, L, D;
   int64_t T;
   float scale_log2;
   int max_splits;
   float* o_part;
   float* lse_part;
   DevErr err;
+  // merged variant: the last CTA of a unit combines its splits into out/lse_out
+  int merged;
+  int* counters;   // [U] arrivals, zero between calls
+  void* out;       // [B, Hq, D] fp32 or bf16
+  int out_bf16;
+  float* lse_out;  // [B, Hq] or null
 };
 
 __device__ __forceinline__ int unit_count(const DecodeParams& p, int u) {
@@ -119,6 +125,13 @@ __device__ __forceinline__ int split_slot(int64_t lo, int64_t a, int64_t c, int6
   return N >= P ? static_cast<int>(c - piece_of(lo, N, P)) : static_cast<int>(a - lo);
 }
 
+__device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, float v) {
+  if (p.out_bf16)
+    static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+  else
+    static_cast<float*>(p.out)[idx] = v;
+}
+
 // Slots of unit u beyond its split count get lse = -inf (CTA c covers units
 // u = c, c + P, ...).  Threads [0, nthreads) of the block take part.
 __device__ void fill_empty_slots(const DecodeParams& p, const int* prefix, int nthreads) {
@@ -127,12 +140,102 @@ __device__ void fill_empty_slots(const DecodeParams& p, const int* prefix, int n
     const int64_t lo = prefix[u], hi = prefix[u + 1];
     const int nsplit = split_count(lo, hi, N, P);
     const int b = u / p.Hkv, h = u % p.Hkv;
+    if (p.merged && nsplit == 0) {  // no split will merge this unit: write its rows here
+      const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * p.G;
+      const int D = p.D;
+      for (int e = threadIdx.x; e < p.G * D; e += nthreads) store_out(p, row0 * D + e, 0.f);
+      if (p.lse_out)
+        for (int g = threadIdx.x; g < p.G; g += nthreads) p.lse_out[row0 + g] = -INFINITY;
+    }
     const int nfill = p.max_splits - nsplit;
     for (int e = threadIdx.x; e < p.G * nfill; e += nthreads) {
       const int g = e / nfill, s = nsplit + e % nfill;
       p.lse_part[(static_cast<int64_t>(b) * p.Hq + h * p.G + g) * p.max_splits + s] = -INFINITY;
     }
   }
+}
+
+// Combine the ns split partials of unit u (already in L2, read with ld.cg)
+// into the unit's G output rows.  `wts` holds >= G * ns floats of shared
+// memory; `nthr` threads take part; `sync` is a barrier over them that
+// returns false on a timeout.
+template <int D, typename Sync>
+__device__ bool merge_unit(const DecodeParams& p, int u, int ns, float* wts, int nthr, Sync sync) {
+  constexpr int D4 = D / 4;
+  constexpr int BATCH = 24;
+  const int b = u / p.Hkv, h = u % p.Hkv, G = p.G;
+  const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+  // Output items e = (head g, float4 column c4).  The partial loads of this
+  // thread's first item do not depend on the weights: issue them first so
+  // they are in flight during the lse phase.
+  const int n_items = G * D4;
+  float4 pre[BATCH];
+  const int e0 = tid;
+  if (e0 < n_items) {
+    const float4* src = reinterpret_cast<const float4*>(
+                            p.o_part + (row0 + e0 / D4) * p.max_splits * D) + (e0 % D4);
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k)
+      pre[k] = k < ns ? __ldcg(src + static_cast<int64_t>(k) * D4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int e = tid; e < G * ns; e += nthr) {
+    const int g = e / ns, sl = e % ns;
+    wts[e] = __ldcg(p.lse_part + (row0 + g) * p.max_splits + sl);
+  }
+  if (!sync()) return false;
+  for (int g = warp; g < G; g += nw) {
+    float mx = -INFINITY;
+    for (int sl = lane; sl < ns; sl += 32) mx = fmaxf(mx, wts[g * ns + sl]);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+    float sum = 0.f;
+    for (int sl = lane; sl < ns; sl += 32) sum += expf(wts[g * ns + sl] - mx);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
+    const float lse = mx + logf(sum);
+    __syncwarp();
+    for (int sl = lane; sl < ns; sl += 32) wts[g * ns + sl] = expf(wts[g * ns + sl] - lse);
+    if (lane == 0 && p.lse_out) p.lse_out[row0 + g] = lse;
+  }
+  if (!sync()) return false;
+  for (int e = tid; e < n_items; e += nthr) {
+    const int g = e / D4, c4 = e % D4;
+    const float4* src = reinterpret_cast<const float4*>(p.o_part + (row0 + g) * p.max_splits * D) + c4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s0 = 0;
+    if (e == e0) {
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) {
+        const float wk = k < ns ? wts[g * ns + k] : 0.f;
+        acc.x += wk * pre[k].x;
+        acc.y += wk * pre[k].y;
+        acc.z += wk * pre[k].z;
+        acc.w += wk * pre[k].w;
+      }
+      s0 = BATCH;
+    }
+    for (; s0 < ns; s0 += BATCH) {
+      float4 x[BATCH];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k)
+        x[k] = s0 + k < ns ? __ldcg(src + static_cast<int64_t>(s0 + k) * D4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) {
+        const float wk = s0 + k < ns ? wts[g * ns + s0 + k] : 0.f;
+        acc.x += wk * x[k].x;
+        acc.y += wk * x[k].y;
+        acc.z += wk * x[k].z;
+        acc.w += wk * x[k].w;
+      }
+    }
+    const int64_t o = (row0 + g) * D + c4 * 4;
+    store_out(p, o, acc.x);
+    store_out(p, o + 1, acc.y);
+    store_out(p, o + 2, acc.z);
+    store_out(p, o + 3, acc.w);
+  }
+  return sync();
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -174,6 +277,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   float* fl = fm + kConsumerWarps * 8;                                  // [4][8]
   int* prefix = reinterpret_cast<int*>(smem + Lay::PREFIX_OFF);         // [U+1]
   __shared__ int scan_sh[33];
+  __shared__ int last_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -308,6 +412,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (!group_sync()) return false;
     const int b = u / p.Hkv, h = u % p.Hkv;
     const int slot = split_slot(prefix[u], a, blockIdx.x, N, P);
+    const int ns = split_count(prefix[u], prefix[u + 1], N, P);
+    const bool direct = p.merged && ns == 1;  // the only split: it is the output
     for (int e = threadIdx.x; e < p.G * D; e += kConsumerWarps * 32) {
       const int g = e / D, d = e % D;
       float M = -INFINITY;
@@ -321,10 +427,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         acc += fo[(w * 8 + g) * D + d] * sc;
       }
       const int64_t row = static_cast<int64_t>(b) * p.Hq + h * p.G + g;
-      p.o_part[(row * p.max_splits + slot) * D + d] = acc / Ls;
-      if (d == 0) p.lse_part[row * p.max_splits + slot] = (M + log2f(Ls)) * kLn2;
+      const float lse = (M + log2f(Ls)) * kLn2;
+      if (direct) {
+        store_out(p, row * D + d, acc / Ls);
+        if (d == 0 && p.lse_out) p.lse_out[row] = lse;
+      } else {
+        p.o_part[(row * p.max_splits + slot) * D + d] = acc / Ls;
+        if (d == 0) p.lse_part[row * p.max_splits + slot] = lse;
+      }
     }
-    return group_sync();
+    if (!group_sync()) return false;
+    if (!p.merged || direct) return true;
+    if (threadIdx.x == 0) {
+      __threadfence();
+      last_sh = atomicAdd(p.counters + u, 1) == ns - 1;
+    }
+    if (!group_sync()) return false;
+    if (!last_sh) return true;
+    __threadfence();
+    if (!merge_unit<D>(p, u, ns, fo, kConsumerWarps * 32, group_sync)) return false;
+    if (threadIdx.x == 0) p.counters[u] = 0;  // ready for the next call
+    return true;
   };
 
   for (int64_t g = a, i = 0; g < bnd; ++g, ++i) {
@@ -425,6 +548,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 // ------------------------------------------------------------------ fp32 path
 
 constexpr int kF32Threads = 128;
+constexpr int kMergeWts = 2048;  // G * splits per unit in merged mode (8 * 256)
 
 template <int D>
 __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodeParams p) {
@@ -434,8 +558,10 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
   float* mh = sc + 8 * 128;                        // [8]
   float* lh = mh + 8;                              // [8]
   float* ah = lh + 8;                              // [8]
-  int* prefix = reinterpret_cast<int*>(ah + 8);    // [U+1]
+  float* wts = ah + 8;                             // [kMergeWts] merge weights
+  int* prefix = reinterpret_cast<int*>(wts + kMergeWts);  // [U+1]
   __shared__ int scan_sh[33];
+  __shared__ int last_sh;
   build_prefix(p, prefix, scan_sh);
   fill_empty_slots(p, prefix, kF32Threads);
   const int64_t N = prefix[p.U], P = gridDim.x;
@@ -448,10 +574,31 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
   auto flush = [&](int u) {
     const int b = u / p.Hkv, h = u % p.Hkv;
     const int slot = split_slot(prefix[u], a, blockIdx.x, N, P);
+    const int ns = split_count(prefix[u], prefix[u + 1], N, P);
+    const bool direct = p.merged && ns == 1;
     for (int g = 0; g < G; ++g) {
       const int64_t row = static_cast<int64_t>(b) * p.Hq + h * G + g;
-      if (tid < D) p.o_part[(row * p.max_splits + slot) * D + tid] = o[g] / lh[g];
-      if (tid == 0) p.lse_part[row * p.max_splits + slot] = (mh[g] + log2f(lh[g])) * kLn2;
+      const float lse = (mh[g] + log2f(lh[g])) * kLn2;
+      if (direct) {
+        if (tid < D) store_out(p, row * D + tid, o[g] / lh[g]);
+        if (tid == 0 && p.lse_out) p.lse_out[row] = lse;
+      } else {
+        if (tid < D) p.o_part[(row * p.max_splits + slot) * D + tid] = o[g] / lh[g];
+        if (tid == 0) p.lse_part[row * p.max_splits + slot] = lse;
+      }
+    }
+    __syncthreads();
+    if (p.merged && !direct) {
+      if (tid == 0) {
+        __threadfence();
+        last_sh = atomicAdd(p.counters + u, 1) == ns - 1;
+      }
+      __syncthreads();
+      if (last_sh) {
+        __threadfence();
+        merge_unit<D>(p, u, ns, wts, kF32Threads, [] { __syncthreads(); return true; });
+        if (tid == 0) p.counters[u] = 0;
+      }
     }
     __syncthreads();
   };
@@ -637,7 +784,7 @@ int decode_default_parts(bool bf16, int D, int L, int num_sms) {
 }
 
 size_t decode_smem_bytes(bool bf16, int D, int L, int U) {
-  if (!bf16) return static_cast<size_t>(8 * D + 8 * 128 + 24 + U + 1) * 4;
+  if (!bf16) return static_cast<size_t>(8 * D + 8 * 128 + 24 + kMergeWts + U + 1) * 4;
   if (D == 128 && L == 128) return DecodeLayout<128, 128>::bytes(U);
   if (D == 128 && L == 64) return DecodeLayout<128, 64>::bytes(U);
   if (D == 64 && L == 128) return DecodeLayout<64, 128>::bytes(U);
@@ -648,8 +795,16 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
                           const int32_t* idx, const int32_t* count, int kmax,
                           const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T,
                           int L, float scale, int num_parts, int max_splits, float* o_part,
-                          float* lse_part, std::string* why) {
+                          float* lse_part, const MergeOut* merge, std::string* why) {
   DecodeParams p{};
+  if (merge != nullptr) {
+    p.merged = 1;
+    p.counters = merge->counters;
+    p.out = merge->out;
+    p.out_bf16 = merge->out_bf16 ? 1 : 0;
+    p.lse_out = merge->lse_out;
+  }
+  p.D = D;
   p.q = q;
   p.Kf = static_cast<const float*>(K);
   p.Vf = static_cast<const float*>(V);

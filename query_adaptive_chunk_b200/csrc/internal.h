@@ -44,13 +44,31 @@ cudaError_t launch_select_hier(const Launch& l, const void* q, bool bf16, const 
                                int top_meta, int k_free, int n_sink, int n_local, int32_t* idx,
                                int32_t* count, int kmax);
 
+cudaError_t launch_score_select_topk(const Launch& l, const void* q, bool bf16, const float* proj,
+                                     int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                     const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                                     int32_t* idx, int32_t* count, int kmax);
+cudaError_t launch_score_select_topp(const Launch& l, const void* q, bool bf16, const float* proj,
+                                     int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                     const uint8_t* head_full, float logit_scale, float p,
+                                     int budget, int n_sink, int n_local, int32_t* idx,
+                                     int32_t* count, int kmax, int32_t* n_p_out);
+
 // decode.cu
 int decode_default_parts(bool bf16, int D, int L, int num_sms);
+// Merged mode: the last CTA of each unit combines the unit's splits.
+struct MergeOut {
+  int* counters;   // [B*Hkv], zero on entry, left zero on a normal exit
+  void* out;       // [B, Hq, D]
+  bool out_bf16;
+  float* lse_out;  // [B, Hq] or null
+};
+constexpr int kMergedMaxParts = 256;
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,
                           const int32_t* idx, const int32_t* count, int kmax,
                           const uint8_t* head_full, int B, int Hq, int Hkv, int D, int64_t T,
                           int L, float scale, int num_parts, int max_splits, float* o_part,
-                          float* lse_part, std::string* why);
+                          float* lse_part, const MergeOut* merge, std::string* why);
 cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_part, int rows,
                          int max_splits, int D, void* out, bool out_bf16, float* lse_out);
 

@@ -27,7 +27,6 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(
   constexpr int ROWS_CTA = ROWS_WARP * kScoreWarps;
   __shared__ float qs[1024];
   __shared__ float qp[DS];
-  __shared__ float qpart[kScoreThreads];
 
   const int u = blockIdx.z;  // b * Hkv + h
   const int n = blockIdx.y;
@@ -48,23 +47,18 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(
   __syncthreads();
   const float* qv = qs;
   if (proj != nullptr) {
-    // qp[r] = sum_d proj[d, r] qs[d]: the 256 threads split the d range into
-    // 256/R parts, each a short run of independent loads, then R threads add
-    // the parts in a fixed order
+    // qp[r] = sum_d proj[d, r] qs[d]: thread t handles r = t / parts over the
+    // d range of part t % parts (parts = 256 / R); the parts of one r sit in
+    // adjacent lanes and are added by an xor-shuffle tree
     const int parts = kScoreThreads / R;
-    const int r = threadIdx.x % R, part = threadIdx.x / R;
+    const int r = threadIdx.x / parts, pt = threadIdx.x % parts;
     const int dchunk = (D + parts - 1) / parts;
-    const int d0 = part * dchunk, d1 = min(D, d0 + dchunk);
+    const int d0 = pt * dchunk, d1 = min(D, d0 + dchunk);
     float acc = 0.f;
 #pragma unroll 4
     for (int d = d0; d < d1; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * qs[d];
-    qpart[part * R + r] = acc;
-    __syncthreads();
-    if (threadIdx.x < R) {
-      float t = 0.f;
-      for (int k = 0; k < parts; ++k) t += qpart[k * R + threadIdx.x];
-      qp[threadIdx.x] = t;
-    }
+    for (int o = parts >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (pt == 0) qp[r] = acc;
     __syncthreads();
     qv = qp;
   }

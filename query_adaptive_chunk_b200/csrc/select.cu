@@ -1,18 +1,22 @@
-// Chunk selection, one CTA per unit, entirely in shared memory.
+// Chunk selection, one CTA per unit, entirely on chip.
 //
-// Scores become order-preserving uint32 keys (0 = not a candidate).  The
-// k-th largest key tau is found by an MSB-first radix select (4 passes of
-// 8 bits, warp-aggregated shared-memory histograms).  The chosen set is every
-// candidate with key > tau plus the first (k - #greater) candidates with key
-// == tau in index order, which realises the (score desc, index asc) order
-// exactly.  Results are written ascending through a block-wide scan.
+// Scores become order-preserving uint32 keys (0 = not a candidate) and
+// 64-bit composites (key << 32 | ~index), whose descending order is exactly
+// (score desc, index asc).
 //
-// top-k: radix select over the non-forced chunks.
-// top-p: radix select of the `budget` best chunks, a bitonic sort of just
-//        those, an ordered prefix scan of their softmax mass, and a cut at the
-//        first prefix reaching p (or at the budget).
-// hier:  meta scores -> radix select of top_meta metas -> child scores ->
-//        radix select of k_free children.
+// Up to 2048 candidates (every workload here): a register-resident bitonic
+// sort of the composites (shuffles inside a warp, shared memory only for the
+// cross-warp stages) gives the order directly.
+//   top-k: the first k_free sort positions of the non-forced chunks;
+//   top-p: an ordered block scan of exp((s - max) * scale) over the first
+//          `budget` positions; the cut is the first position whose prefix
+//          reaches p * Z (Z from a fixed-order (max, sum-exp) reduction), or
+//          the budget when none does;
+//   hier:  the same sort-and-mark for the metas, then for their children.
+// Larger C falls back to an MSB-first radix select (4 passes of 8 bits over
+// shared-memory histograms) that finds the k-th key, keeps the keys above it
+// and the first of the equal keys in index order.
+// Results are written ascending through a block-wide scan of per-chunk flags.
 #include "internal.h"
 
 namespace csa {
@@ -20,17 +24,36 @@ namespace {
 
 constexpr int kSelThreads = 512;
 
+// Shared-memory exchange buffer of the register sort (0 when C is too large
+// for it): one 64-bit slot per sort position, at least one per thread.
+__host__ __device__ __forceinline__ int sort_exch_bytes(int C) {
+  int p = 1;
+  while (p < C) p <<= 1;
+  if (p > 2048) return 0;
+  return 8 * (p < kSelThreads ? kSelThreads : p);
+}
+
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   uint32_t b = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
   return __uint_as_float(b);
 }
 
-struct SelScratch {
+struct __align__(16) SelScratch {
   int hist[256];
   int bcast[2];
   int scan[33];
   float fscan[33];
   int misc[4];
+};
+
+// Bucket-select scratch (see bucket_mark).
+constexpr int kBuckets = 1024;
+constexpr int kBoundaryMax = 256;
+
+struct BucketScratch {
+  int hist[kBuckets];
+  uint64_t bnd[kBoundaryMax];
+  int n_bnd, above, bstar;
 };
 
 // k-th largest candidate key among keys[0, n) (0 = not a candidate);
@@ -53,12 +76,13 @@ __device__ uint32_t radix_select(const uint32_t* keys, int n, int k, SelScratch&
     }
     __syncthreads();
     if (threadIdx.x < 32) {
-      int cnt[8], tot = 0;
+      // lane j owns buckets 255-8j down to 248-8j (two 16-byte reads)
+      const int4 hi = reinterpret_cast<const int4*>(s.hist)[(252 - 8 * lane) >> 2];
+      const int4 lo = reinterpret_cast<const int4*>(s.hist)[(248 - 8 * lane) >> 2];
+      const int cnt[8] = {hi.w, hi.z, hi.y, hi.x, lo.w, lo.z, lo.y, lo.x};
+      int tot = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        cnt[i] = s.hist[255 - 8 * lane - i];
-        tot += cnt[i];
-      }
+      for (int i = 0; i < 8; ++i) tot += cnt[i];
       int inc = tot;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -89,43 +113,56 @@ __device__ uint32_t radix_select(const uint32_t* keys, int n, int k, SelScratch&
   return prefix;
 }
 
+__device__ __forceinline__ float key_to_float(uint32_t k);
+__device__ float block_sum(float v, SelScratch& s);
+
 // Mark in flags[] the candidates with key > tau and the first take_eq with
 // key == tau (index order).  Threads own contiguous segments so that the
-// block scan follows index order.
+// block scan follows index order.  With mass != null, also returns the sum
+// of exp((score - mx) * scale) over the marked candidates.
 __device__ void mark_top(const uint32_t* keys, int n, uint32_t tau, int take_eq, uint8_t* flags,
-                         SelScratch& s) {
+                         SelScratch& s, float* mass = nullptr, float mx = 0.f, float scale = 0.f) {
   const int seg = (n + blockDim.x - 1) / blockDim.x;
   const int lo = min(n, static_cast<int>(threadIdx.x) * seg), hi = min(n, lo + seg);
   int eq = 0;
   for (int c = lo; c < hi; ++c) eq += keys[c] == tau;
   int rank = block_exclusive_scan(eq, s.scan, nullptr);
+  float m = 0.f;
   for (int c = lo; c < hi; ++c) {
     const uint32_t k = keys[c];
     if (k == 0u) continue;
-    if (k > tau) flags[c] = 1;
+    bool take = false;
+    if (k > tau) take = true;
     else if (k == tau) {
-      if (rank < take_eq) flags[c] = 1;
+      take = rank < take_eq;
       ++rank;
     }
+    if (take) {
+      flags[c] = 1;
+      if (mass) m += expf((key_to_float(k) - mx) * scale);
+    }
   }
-  __syncthreads();
+  if (mass) *mass = block_sum(m, s);  // ends with a barrier
+  else __syncthreads();
 }
 
 // Choose the k best candidates of keys[0, n) into flags (k clamped to the
-// number of candidates n_cand).
+// number of candidates n_cand); optionally the softmax mass of the chosen.
 __device__ void choose_best(const uint32_t* keys, int n, int n_cand, int k, uint8_t* flags,
-                            SelScratch& s) {
+                            SelScratch& s, float* mass = nullptr, float mx = 0.f,
+                            float scale = 0.f) {
   k = min(k, n_cand);
-  if (k <= 0) return;
+  if (k <= 0) {
+    if (mass) *mass = 0.f;
+    return;
+  }
   if (k == n_cand) {
-    for (int c = threadIdx.x; c < n; c += blockDim.x)
-      if (keys[c] != 0u) flags[c] = 1;
-    __syncthreads();
+    mark_top(keys, n, 0u, 0, flags, s, mass, mx, scale);  // every non-zero key is > 0
     return;
   }
   int n_gt = 0;
   const uint32_t tau = radix_select(keys, n, k, s, &n_gt);
-  mark_top(keys, n, tau, k - n_gt, flags, s);
+  mark_top(keys, n, tau, k - n_gt, flags, s, mass, mx, scale);
 }
 
 // Write the positions of set flags in [0, n) ascending into row[0:total],
@@ -157,13 +194,31 @@ __device__ __forceinline__ int forced_count(int v, int n_sink, int n_local) {
   return a + (v - b0) - max(0, a - b0);  // |[0,a) U [b0,v)|
 }
 
+// Top-k over keys[0, v) already loaded (forced chunks: key 0, flag 1).
+__device__ bool try_sorted_mark(const uint32_t* keys, uint8_t* flags, int v, int k_take,
+                                uint64_t* exch);
+
+__device__ void mark_best(const uint32_t* keys, uint8_t* flags, int n, int n_cand, int k,
+                          uint64_t* exch, BucketScratch& bs, SelScratch& s);
+
+__device__ void topk_from_keys(const uint32_t* keys, uint8_t* flags, int v, int n_sink,
+                               int n_local, int k_free, int32_t* row, int32_t* cnt, int kmax,
+                               SelScratch& s, uint64_t* exch, BucketScratch& bs) {
+  const int n_cand = v - forced_count(v, n_sink, n_local);
+  mark_best(keys, flags, v, n_cand, k_free, exch, bs, s);
+  emit_ascending(flags, v, row, cnt, kmax, s);
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
     const float* __restrict__ scores, int C, const int32_t* __restrict__ n_valid, int k_free,
     int n_sink, int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sm);
-  uint8_t* flags = sm + static_cast<size_t>(C) * 4;
+  __shared__ BucketScratch bs;
+  const int exch_bytes = sort_exch_bytes(C);
+  uint64_t* exch = exch_bytes ? reinterpret_cast<uint64_t*>(sm) : nullptr;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + exch_bytes);
+  uint8_t* flags = sm + exch_bytes + static_cast<size_t>(C) * 4;
   const int u = blockIdx.x;
   const int v = n_valid ? max(0, min(C, n_valid[u])) : C;
   const float* row = scores + static_cast<int64_t>(u) * C;
@@ -173,34 +228,69 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
     flags[c] = f ? 1 : 0;
   }
   __syncthreads();
-  const int n_cand = v - forced_count(v, n_sink, n_local);
-  choose_best(keys, v, n_cand, k_free, flags, s);
-  emit_ascending(flags, v, idx + static_cast<int64_t>(u) * kmax, count + u, kmax, s);
+  topk_from_keys(keys, flags, v, n_sink, n_local, k_free, idx + static_cast<int64_t>(u) * kmax,
+                 count + u, kmax, s, exch, bs);
 }
 
-// Block sum of one float per thread in a fixed order (deterministic).
+// Block sum of one float per thread in a fixed order (deterministic): a
+// warp xor-tree, then every warp reduces the per-warp totals the same way.
 __device__ float block_sum(float v, SelScratch& s) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if (lane == 0) s.fscan[warp] = v;
   __syncthreads();
-  float t = 0.f;
-  for (int w = 0; w < nw; ++w) t += s.fscan[w];
+  float t = lane < nw ? s.fscan[lane] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
   __syncthreads();
   return t;
 }
 
-__device__ float block_max(float v, SelScratch& s) {
+
+// Running (max m, sum s of exp((x - m) * scale)) of a stream of scores.
+__device__ __forceinline__ void ms_add(float& m, float& sum, float x, float scale) {
+  if (x > m) {
+    sum = sum * expf((m - x) * scale) + 1.f;
+    m = x;
+  } else {
+    sum += expf((x - m) * scale);
+  }
+}
+
+__device__ __forceinline__ void ms_merge(float& m, float& sum, float m2, float s2, float scale) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = m2;
+    sum = s2;
+    return;
+  }
+  const float M = fmaxf(m, m2);
+  sum = sum * expf((m - M) * scale) + s2 * expf((m2 - M) * scale);
+  m = M;
+}
+
+// Block-wide (max, sum-exp) in a fixed tree order; every thread gets the result.
+__device__ void block_max_sumexp(float& m, float& sum, float scale, SelScratch& s) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if (lane == 0) s.fscan[warp] = v;
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
+    ms_merge(m, sum, m2, s2, scale);
+  }
+  if (lane == 0) {
+    s.fscan[warp] = m;
+    s.fscan[16 + warp] = sum;
+  }
   __syncthreads();
-  float t = -INFINITY;
-  for (int w = 0; w < nw; ++w) t = fmaxf(t, s.fscan[w]);
+  m = lane < nw ? s.fscan[lane] : -INFINITY;
+  sum = lane < nw ? s.fscan[16 + lane] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
+    ms_merge(m, sum, m2, s2, scale);
+  }
   __syncthreads();
-  return t;
 }
 
 // Exclusive block scan of floats, fixed order.
@@ -221,50 +311,338 @@ __device__ float block_exclusive_scan_f(float v, SelScratch& s) {
   return base + x - v;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_topp_kernel(
-    const float* __restrict__ scores, int C, float logit_scale, float p, int budget, int n_sink,
-    int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax,
-    int32_t* __restrict__ n_p_out, int SN) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  __shared__ SelScratch s;
-  uint64_t* sortbuf = reinterpret_cast<uint64_t*>(sm);            // [SN]
-  float* cum = reinterpret_cast<float*>(sm + static_cast<size_t>(SN) * 8);  // [SN]
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + static_cast<size_t>(SN) * 12);  // [C]
-  uint8_t* flags = sm + static_cast<size_t>(SN) * 12 + static_cast<size_t>(C) * 4;  // [C]
-  const int u = blockIdx.x;
-  const float* row = scores + static_cast<int64_t>(u) * C;
+// Top-p over keys[0, C) already loaded (every chunk a candidate, flags 0)
+// with mx = the largest score.
+// ---------------------------------------------------------------- register bitonic sort
+//
+// For up to 2048 candidates the whole selection is a sort: thread t holds
+// the E = SN/256 consecutive sort positions t*E .. t*E+E-1 in registers as
+// 64-bit composites (score key << 32 | ~index), so descending order is
+// (score desc, index asc) and 0 marks padding or an excluded chunk.  Stages
+// whose partner is in the same thread need nothing, partners in another
+// lane of the warp come by shuffle, and only partners in another warp go
+// through shared memory with a barrier (6 of the 55 stages at SN = 1024).
 
-  float mx = -INFINITY;
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    const float x = row[c];
-    keys[c] = float_key(x);
-    flags[c] = 0;
-    mx = fmaxf(mx, x);
+constexpr int kSortedMax = 2048;
+
+__device__ __forceinline__ uint64_t composite(uint32_t key, int c) {
+  return key ? ((static_cast<uint64_t>(key) << 32) | (0xffffffffu - static_cast<uint32_t>(c))) : 0ull;
+}
+__device__ __forceinline__ int comp_index(uint64_t v) {
+  return static_cast<int>(0xffffffffu - static_cast<uint32_t>(v & 0xffffffffull));
+}
+__device__ __forceinline__ uint32_t comp_key(uint64_t v) { return static_cast<uint32_t>(v >> 32); }
+
+__device__ __forceinline__ int pow2_at_least(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <int E>
+__device__ void bitonic_desc(uint64_t (&v)[E], uint64_t* exch, int SN) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int k = 2; k <= SN; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j < E) {
+        // partner in this thread: unrolled per stride so indices are constants
+#pragma unroll
+        for (int jj = 1; jj < E; jj <<= 1) {
+          if (jj != j) continue;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const int pe = e ^ jj;
+            if (pe > e) {
+              const bool desc = ((tid * E + e) & k) == 0;
+              const uint64_t a = v[e], b = v[pe];
+              if (desc ? (a < b) : (a > b)) {
+                v[e] = b;
+                v[pe] = a;
+              }
+            }
+          }
+        }
+      } else if (j < 32 * E) {
+        const int lm = j / E;
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], lm);
+          const bool keep_max = (((tid * E + e) & k) == 0) == lower;
+          v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) exch[tid * E + e] = v[e];
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const uint64_t o = exch[i ^ j];
+          const bool keep_max = ((i & k) == 0) == ((i & j) == 0);
+          v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+        }
+        __syncthreads();
+      }
+    }
   }
-  mx = block_max(mx, s);  // includes the __syncthreads that publishes keys
-  float part = 0.f;
-  for (int c = threadIdx.x; c < C; c += blockDim.x)
-    part += expf((key_to_float(keys[c]) - mx) * logit_scale);
-  const float Z = block_sum(part, s);
+}
 
-  // the nb best chunks (by score, lower index first) into flags as a pool
+// Mark in flags the k_take best of keys[0, v) (0 = excluded) by sorting.
+template <int E>
+__device__ void sorted_mark(const uint32_t* keys, uint8_t* flags, int v, int k_take,
+                            uint64_t* exch) {
+  const int SN = pow2_at_least(max(v, 1));
+  uint64_t x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int c = threadIdx.x * E + e;
+    x[e] = c < v ? composite(keys[c], c) : 0ull;
+  }
+  bitonic_desc<E>(x, exch, SN);
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (static_cast<int>(threadIdx.x) * E + e < k_take && x[e] != 0ull) flags[comp_index(x[e])] = 1;
+  __syncthreads();
+}
+
+// Dispatch on the sort width; false (nothing done) when v is too large.
+__device__ bool try_sorted_mark(const uint32_t* keys, uint8_t* flags, int v, int k_take,
+                                uint64_t* exch) {
+  const int SN = pow2_at_least(max(v, 1));
+  if (exch == nullptr || SN > kSortedMax) return false;
+  // E sort positions per thread: E * blockDim.x >= SN, and the exchange
+  // buffer holds E * blockDim.x = max(SN, blockDim.x) entries
+  const int E = SN <= static_cast<int>(blockDim.x) ? 1 : SN / static_cast<int>(blockDim.x);
+  if (E == 1) sorted_mark<1>(keys, flags, v, k_take, exch);
+  else if (E == 2) sorted_mark<2>(keys, flags, v, k_take, exch);
+  else if (E == 4) sorted_mark<4>(keys, flags, v, k_take, exch);
+  else sorted_mark<8>(keys, flags, v, k_take, exch);
+  return true;
+}
+
+// ---------------------------------------------------------------- bucket select
+//
+// Top-k without ordering the whole set: scores are binned linearly between
+// their min and max (the map x -> floor((x - lo) * NB / (hi - lo)) is
+// monotone, and equal scores share a bin), one shared-memory histogram and
+// one descending scan find the bin b* holding the k-th best; every chunk in
+// a higher bin is chosen, and only the few chunks of bin b* are ranked
+// exactly by (key desc, index asc).  Degenerate inputs (all candidates
+// equal, or too many in one bin) report false and the caller sorts.
+
+
+__device__ void block_minmax(float& lo, float& hi, SelScratch& s) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    s.fscan[warp] = lo;
+    s.fscan[16 + warp] = hi;
+  }
+  __syncthreads();
+  lo = lane < nw ? s.fscan[lane] : INFINITY;
+  hi = lane < nw ? s.fscan[16 + lane] : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ int bucket_of(float x, float lo, float scale) {
+  return min(kBuckets - 1, static_cast<int>((x - lo) * scale));
+}
+
+// Marks in flags the k_take best of keys[0, v) (0 = excluded); returns
+// false when the input is degenerate for binning (flags then hold a subset
+// of the answer, which a sort on top completes).
+__device__ bool bucket_mark(const uint32_t* keys, uint8_t* flags, int v, int k_take,
+                            BucketScratch& bs, SelScratch& s) {
+  if (k_take <= 0) return true;
+  float lo = INFINITY, hi = -INFINITY;
+  for (int c = threadIdx.x; c < v; c += blockDim.x)
+    if (keys[c]) {
+      const float x = key_to_float(keys[c]);
+      lo = fminf(lo, x);
+      hi = fmaxf(hi, x);
+    }
+  for (int b = threadIdx.x; b < kBuckets; b += blockDim.x) bs.hist[b] = 0;
+  if (threadIdx.x == 0) {
+    bs.n_bnd = 0;
+    bs.bstar = -1;
+  }
+  block_minmax(lo, hi, s);  // barriers also publish the cleared histogram
+  if (!(hi > lo)) return false;
+  const float scale = static_cast<float>(kBuckets) / (hi - lo);
+  if (!(scale < INFINITY)) return false;
+  for (int c = threadIdx.x; c < v; c += blockDim.x)
+    if (keys[c]) atomicAdd(&bs.hist[bucket_of(key_to_float(keys[c]), lo, scale)], 1);
+  __syncthreads();
+  // descending scan over the bins: thread t owns bins NB-1-t*seg down to NB-(t+1)*seg
+  const int seg = kBuckets / blockDim.x;
+  const int top = kBuckets - 1 - static_cast<int>(threadIdx.x) * seg;
+  int loc = 0;
+  for (int i = 0; i < seg; ++i) loc += bs.hist[top - i];
+  const int exc = block_exclusive_scan(loc, s.scan, nullptr);
+  if (exc < k_take && k_take <= exc + loc) {
+    int run = exc;
+    for (int i = 0; i < seg; ++i) {
+      const int h = bs.hist[top - i];
+      if (run + h >= k_take) {
+        bs.bstar = top - i;
+        bs.above = run;
+        break;
+      }
+      run += h;
+    }
+  }
+  __syncthreads();
+  const int bstar = bs.bstar;
+  if (bstar < 0) return false;
+  for (int c = threadIdx.x; c < v; c += blockDim.x) {
+    const uint32_t k = keys[c];
+    if (!k) continue;
+    const int b = bucket_of(key_to_float(k), lo, scale);
+    if (b > bstar) {
+      flags[c] = 1;
+    } else if (b == bstar) {
+      const int pos = atomicAdd(&bs.n_bnd, 1);
+      if (pos < kBoundaryMax) bs.bnd[pos] = composite(k, c);
+    }
+  }
+  __syncthreads();
+  const int m = bs.n_bnd, need = k_take - bs.above;
+  if (m > kBoundaryMax) return false;
+  for (int j = threadIdx.x; j < m; j += blockDim.x) {
+    const uint64_t mine = bs.bnd[j];
+    int rank = 0;
+    for (int i = 0; i < m; ++i) rank += bs.bnd[i] > mine;
+    if (rank < need) flags[comp_index(mine)] = 1;
+  }
+  __syncthreads();
+  return true;
+}
+
+// Top-p by sorting all C chunks: the ordered prefix mass over the first
+// nb = min(budget, C) sort positions is a block scan; the cut is the first
+// position where it reaches p * Z, or nb when it never does.
+template <int E>
+__device__ void sorted_topp(const uint32_t* keys, uint8_t* flags, int C, float mx, float Z,
+                            float logit_scale, float p, int budget, int n_sink, int n_local,
+                            uint64_t* exch, int32_t* row, int32_t* cnt, int kmax,
+                            int32_t* n_p_slot, SelScratch& s) {
+  const int SN = pow2_at_least(C);
+  uint64_t x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int c = threadIdx.x * E + e;
+    x[e] = c < C ? composite(keys[c], c) : 0ull;
+  }
+  bitonic_desc<E>(x, exch, SN);
   const int nb = min(budget, C);
-  choose_best(keys, C, C, nb, flags, s);
+  float ev[E];
+  float loc = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int r = threadIdx.x * E + e;
+    ev[e] = (r < nb && x[e] != 0ull) ? expf((key_to_float(comp_key(x[e])) - mx) * logit_scale) : 0.f;
+    loc += ev[e];
+  }
+  if (threadIdx.x == 0) s.misc[0] = 0x7fffffff;
+  float run = block_exclusive_scan_f(loc, s);  // its barriers also publish misc[0]
+  const float target = p * Z;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    run += ev[e];
+    const int r = threadIdx.x * E + e;
+    if (r < nb && run >= target) {
+      atomicMin(&s.misc[0], r);
+      break;
+    }
+  }
+  __syncthreads();
+  const int first = s.misc[0];
+  const bool found = first != 0x7fffffff;
+  const int n_take = found ? first + 1 : nb;
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (static_cast<int>(threadIdx.x) * E + e < n_take && x[e] != 0ull) flags[comp_index(x[e])] = 1;
+  for (int c = threadIdx.x; c < C; c += blockDim.x)
+    if (is_forced(c, C, n_sink, n_local)) flags[c] = 1;
+  __syncthreads();
+  if (n_p_slot && threadIdx.x == 0) *n_p_slot = found ? first + 1 : (nb < C ? nb + 1 : C);
+  emit_ascending(flags, C, row, cnt, kmax, s);
+}
+
+__device__ bool try_sorted_topp(const uint32_t* keys, uint8_t* flags, int C, float mx, float Z,
+                                float logit_scale, float p, int budget, int n_sink, int n_local,
+                                uint64_t* exch, int32_t* row, int32_t* cnt, int kmax,
+                                int32_t* n_p_slot, SelScratch& s) {
+  const int SN = pow2_at_least(C);
+  if (SN > kSortedMax) return false;
+  const int E = SN <= static_cast<int>(blockDim.x) ? 1 : SN / static_cast<int>(blockDim.x);
+  if (E == 1)
+    sorted_topp<1>(keys, flags, C, mx, Z, logit_scale, p, budget, n_sink, n_local, exch, row, cnt, kmax, n_p_slot, s);
+  else if (E == 2)
+    sorted_topp<2>(keys, flags, C, mx, Z, logit_scale, p, budget, n_sink, n_local, exch, row, cnt, kmax, n_p_slot, s);
+  else if (E == 4)
+    sorted_topp<4>(keys, flags, C, mx, Z, logit_scale, p, budget, n_sink, n_local, exch, row, cnt, kmax, n_p_slot, s);
+  else
+    sorted_topp<8>(keys, flags, C, mx, Z, logit_scale, p, budget, n_sink, n_local, exch, row, cnt, kmax, n_p_slot, s);
+  return true;
+}
+
+// Mark the k best of keys[0, n) (n_cand candidates, 0 = excluded): bucket
+// select, else a register sort (n <= 2048), else radix select.
+__device__ void mark_best(const uint32_t* keys, uint8_t* flags, int n, int n_cand, int k,
+                          uint64_t* exch, BucketScratch& bs, SelScratch& s) {
+  const int k_take = min(k, n_cand);
+  if (k_take <= 0) return;
+  if (k_take >= n_cand) {
+    for (int c = threadIdx.x; c < n; c += blockDim.x)
+      if (keys[c]) flags[c] = 1;
+    __syncthreads();
+    return;
+  }
+  if (bucket_mark(keys, flags, n, k_take, bs, s)) return;
+  if (try_sorted_mark(keys, flags, n, k_take, exch)) return;
+  choose_best(keys, n, n_cand, k_take, flags, s);
+}
+
+// Bytes before the keys in the top-p kernels' shared memory: the register
+// sort's exchange buffer when C is small enough, else the radix path's
+// sort buffer and prefix array for the budget's SN entries.
+__host__ __device__ __forceinline__ size_t topp_head_bytes(int C, int SN) {
+  const int ex = sort_exch_bytes(C);
+  const size_t radix = static_cast<size_t>(SN) * 12;
+  return ex ? (static_cast<size_t>(ex) > radix ? static_cast<size_t>(ex) : radix) : radix;
+}
+
+// Top-p over keys[0, C) already loaded (every chunk a candidate, flags 0),
+// mx = the largest score, Z = sum_c exp((score_c - mx) * logit_scale).
+__device__ void topp_from_keys(const uint32_t* keys, uint8_t* flags, uint64_t* sortbuf,
+                               float* cum, int C, float mx, float Z, float logit_scale, float p,
+                               int budget, int n_sink, int n_local, int32_t* idx, int32_t* count,
+                               int kmax, int32_t* n_p_out, int SN, int u, SelScratch& s) {
+  // the nb best chunks (by score, lower index first) into flags as a pool,
+  // with their softmax mass
+  const int nb = min(budget, C);
+  float mass_nb = 0.f;
+  choose_best(keys, C, C, nb, flags, s, &mass_nb, mx, logit_scale);
   // if even those nb chunks hold less than p of the mass, n_p > budget and the
   // cap decides: the pool is the answer, no ordering of it is needed
-  {
-    float mpart = 0.f;
+  if (nb < C && mass_nb < p * Z) {
     for (int c = threadIdx.x; c < C; c += blockDim.x)
-      if (flags[c]) mpart += expf((key_to_float(keys[c]) - mx) * logit_scale);
-    const float mass_nb = block_sum(mpart, s);
-    if (nb < C && mass_nb < p * Z) {
-      for (int c = threadIdx.x; c < C; c += blockDim.x)
-        if (is_forced(c, C, n_sink, n_local)) flags[c] = 1;
-      __syncthreads();
-      if (n_p_out && threadIdx.x == 0) n_p_out[u] = nb + 1;
-      emit_ascending(flags, C, idx + static_cast<int64_t>(u) * kmax, count + u, kmax, s);
-      return;
-    }
+      if (is_forced(c, C, n_sink, n_local)) flags[c] = 1;
+    __syncthreads();
+    if (n_p_out && threadIdx.x == 0) n_p_out[u] = nb + 1;
+    emit_ascending(flags, C, idx + static_cast<int64_t>(u) * kmax, count + u, kmax, s);
+    return;
   }
   // compact them, in index order, into the sort buffer as 64-bit keys
   {
@@ -333,13 +711,73 @@ __global__ void __launch_bounds__(kSelThreads) select_topp_kernel(
   emit_ascending(flags, C, idx + static_cast<int64_t>(u) * kmax, count + u, kmax, s);
 }
 
+
+// Top-p driver: when the budget caps the prefix (the usual case on long
+// contexts) the answer is the budget's best set, found by bucket select,
+// whose mass is checked against p; only when that set reaches p is the exact
+// ordered prefix needed, from a sort (or the radix path beyond 2048 chunks).
+__device__ void topp_select(const uint32_t* keys, uint8_t* flags, uint64_t* sortbuf, float* cum,
+                            int C, float mx, float Z, float logit_scale, float p, int budget,
+                            int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                            int32_t* n_p_out, int SN, int u, SelScratch& s, BucketScratch& bs) {
+  const int nb = min(budget, C);
+  int32_t* row = idx + static_cast<int64_t>(u) * kmax;
+  if (nb < C && bucket_mark(keys, flags, C, nb, bs, s)) {
+    float m = 0.f;
+    for (int c = threadIdx.x; c < C; c += blockDim.x)
+      if (flags[c]) m += expf((key_to_float(keys[c]) - mx) * logit_scale);
+    const float mass_nb = block_sum(m, s);
+    if (mass_nb < p * Z) {
+      for (int c = threadIdx.x; c < C; c += blockDim.x)
+        if (is_forced(c, C, n_sink, n_local)) flags[c] = 1;
+      __syncthreads();
+      if (n_p_out && threadIdx.x == 0) n_p_out[u] = nb + 1;
+      emit_ascending(flags, C, row, count + u, kmax, s);
+      return;
+    }
+  }
+  for (int c = threadIdx.x; c < C; c += blockDim.x) flags[c] = 0;
+  __syncthreads();
+  if (try_sorted_topp(keys, flags, C, mx, Z, logit_scale, p, budget, n_sink, n_local, sortbuf, row,
+                      count + u, kmax, n_p_out ? n_p_out + u : nullptr, s))
+    return;
+  topp_from_keys(keys, flags, sortbuf, cum, C, mx, Z, logit_scale, p, budget, n_sink, n_local, idx,
+                 count, kmax, n_p_out, SN, u, s);
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_topp_kernel(
+    const float* __restrict__ scores, int C, float logit_scale, float p, int budget, int n_sink,
+    int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax,
+    int32_t* __restrict__ n_p_out, int SN) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ SelScratch s;
+  __shared__ BucketScratch bs;
+  const size_t head = topp_head_bytes(C, SN);
+  uint64_t* sortbuf = reinterpret_cast<uint64_t*>(sm);            // [SN] or the sort exchange
+  float* cum = reinterpret_cast<float*>(sm + static_cast<size_t>(SN) * 8);  // [SN]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + head);  // [C]
+  uint8_t* flags = sm + head + static_cast<size_t>(C) * 4;  // [C]
+  const int u = blockIdx.x;
+  const float* row = scores + static_cast<int64_t>(u) * C;
+  float mx = -INFINITY, Z = 0.f;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    const float x = row[c];
+    keys[c] = float_key(x);
+    flags[c] = 0;
+    ms_add(mx, Z, x, logit_scale);
+  }
+  block_max_sumexp(mx, Z, logit_scale, s);  // its barriers also publish keys
+  topp_select(keys, flags, sortbuf, cum, C, mx, Z, logit_scale, p, budget, n_sink, n_local, idx,
+              count, kmax, n_p_out, SN, u, s, bs);
+}
+
 // Group-summed dot products of `nrows` rows (row ids rows[i], or i when rows
 // is null) of a [*, D] fp32 matrix with qs, into keys (0 where skip(c)).
 template <bool kSkipForced>
 __device__ void score_rows(const float* __restrict__ mat, int D, const float* qs, const int* rows,
                            int nrows, uint32_t* keys, int C, int n_sink, int n_local) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  constexpr int BATCH = 8;
+  constexpr int BATCH = 16;
   for (int i0 = warp * BATCH; i0 < nrows; i0 += nw * BATCH) {
     float4 v[BATCH];
 #pragma unroll
@@ -376,6 +814,7 @@ __global__ void __launch_bounds__(kSelThreads) select_hier_kernel(
     int kmax) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
+  __shared__ BucketScratch bs;
   __shared__ float qs[128];
   const int M = C / Gm;
   const int k1 = min(top_meta, M);
@@ -387,6 +826,10 @@ __global__ void __launch_bounds__(kSelThreads) select_hier_kernel(
   uint8_t* mflags = reinterpret_cast<uint8_t*>(mlist + k1);                 // [M]
   uint8_t* cflags = mflags + M;                                             // [NCH]
   uint8_t* flags = cflags + NCH;                                            // [C]
+  const int exch_bytes = sort_exch_bytes(max(M, NCH));
+  uint64_t* exch = exch_bytes ? reinterpret_cast<uint64_t*>(
+                                    sm + ((static_cast<size_t>(5) * M + 9 * NCH + 4 * k1 + C + 15) & ~size_t(15)))
+                              : nullptr;
 
   const int u = blockIdx.x;
   const int h = u % Hkv, b = u / Hkv;
@@ -408,7 +851,7 @@ __global__ void __launch_bounds__(kSelThreads) select_hier_kernel(
   // level 1: meta-chunks
   score_rows<false>(meta + static_cast<int64_t>(u) * M * D, D, qs, nullptr, M, mkeys, C, 0, 0);
   __syncthreads();
-  choose_best(mkeys, M, M, k1, mflags, s);
+  mark_best(mkeys, mflags, M, M, k1, exch, bs, s);
   {  // ascending list of kept metas -> ascending list of their children
     const int seg = (M + blockDim.x - 1) / blockDim.x;
     const int lo = min(M, static_cast<int>(threadIdx.x) * seg), hi = min(M, lo + seg);
@@ -433,11 +876,186 @@ __global__ void __launch_bounds__(kSelThreads) select_hier_kernel(
     block_exclusive_scan(loc, s.scan, &tot);
     n_cand = tot;
   }
-  choose_best(ckeys, NCH, n_cand, k_free, cflags, s);
+  mark_best(ckeys, cflags, NCH, n_cand, k_free, exch, bs, s);
   for (int i = threadIdx.x; i < NCH; i += blockDim.x)
     if (cflags[i]) flags[clist[i]] = 1;
   __syncthreads();
   emit_ascending(flags, C, idx + static_cast<int64_t>(u) * kmax, count + u, kmax, s);
+}
+
+// ---------------------------------------------------------------- fused score + select
+
+// Group-summed query of unit (b, h) into qs[0, D) and, with a projection,
+// proj^T qs into qv[0, R).  Same partition and order as the score kernel
+// (256 threads split the d range), so the scores match it bit for bit.
+__device__ void unit_query(const void* __restrict__ q, int q_bf16, int64_t head0, int G, int D,
+                           const float* __restrict__ proj, int R, float* qs, float* qv,
+                           float* part) {
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int g = 0; g < G; ++g) {
+      const int64_t off = (head0 + g) * D + d;
+      acc += q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
+                    : static_cast<const float*>(q)[off];
+    }
+    qs[d] = acc;
+  }
+  __syncthreads();
+  if (proj == nullptr) return;
+  // 256 threads: thread t handles r = t / parts over the d range of part
+  // t % parts; the parts of one r sit in adjacent lanes and are added by an
+  // xor-shuffle tree (same order as the score kernel)
+  const int parts = 256 / R;
+  if (threadIdx.x < 256) {
+    const int r = threadIdx.x / parts, pt = threadIdx.x % parts;
+    const int dchunk = (D + parts - 1) / parts;
+    const int d0 = pt * dchunk, d1 = min(D, d0 + dchunk);
+    float acc = 0.f;
+#pragma unroll 4
+    for (int d = d0; d < d1; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * qs[d];
+    for (int o = parts >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (pt == 0) qv[r] = acc;
+  }
+  (void)part;
+  __syncthreads();
+}
+
+constexpr int kRowBatch = 8;  // summary rows per lane group in flight
+
+// First round of summary rows of a unit (issued before the query is ready).
+template <int DS>
+__device__ __forceinline__ void rows_load(const float* __restrict__ summ_u, int C, int base,
+                                          float4 (&v)[kRowBatch]) {
+  constexpr int LPR = DS / 4, RPI = 32 / LPR;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane % LPR, rsub = lane / LPR;
+#pragma unroll
+  for (int b = 0; b < kRowBatch; ++b) {
+    const int c = base + b * RPI + rsub;
+    v[b] = c < C ? __ldg(reinterpret_cast<const float4*>(summ_u + static_cast<int64_t>(c) * DS) + sub)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+template <int DS>
+__device__ __forceinline__ int rows_first_base() {
+  constexpr int RPI = 32 / (DS / 4);
+  return (threadIdx.x >> 5) * RPI * kRowBatch;
+}
+
+// keys[c] = key of (qv . summ_u[c]) for c < C (0 for forced chunks when
+// skip_forced), with the running (max, sum-exp) of the scores when scale != 0.
+// Rows of DS floats over DS/4 lanes, kRowBatch rows per lane group in flight;
+// `pre` holds the first round, loaded by rows_load.
+template <int DS>
+__device__ void summaries_to_keys(const float* __restrict__ summ_u, int C, const float* qv,
+                                  uint32_t* keys, int n_sink, int n_local, bool skip_forced,
+                                  float& mx, float& sum, float scale,
+                                  const float4 (&pre)[kRowBatch]) {
+  constexpr int LPR = DS / 4, RPI = 32 / LPR;
+  const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int sub = lane % LPR, rsub = lane / LPR;
+  const float4 q4 = make_float4(qv[sub * 4], qv[sub * 4 + 1], qv[sub * 4 + 2], qv[sub * 4 + 3]);
+  mx = -INFINITY;
+  sum = 0.f;
+  const int first = rows_first_base<DS>();
+  for (int base = first; base < C; base += nw * RPI * kRowBatch) {
+    float4 v[kRowBatch];
+    if (base == first) {
+#pragma unroll
+      for (int b = 0; b < kRowBatch; ++b) v[b] = pre[b];
+    } else {
+      rows_load<DS>(summ_u, C, base, v);
+    }
+#pragma unroll
+    for (int b = 0; b < kRowBatch; ++b) {
+      float x = v[b].x * q4.x + v[b].y * q4.y + v[b].z * q4.z + v[b].w * q4.w;
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      const int c = base + b * RPI + rsub;
+      if (sub == 0 && c < C) {
+        keys[c] = (skip_forced && is_forced(c, C, n_sink, n_local)) ? 0u : float_key(x);
+        if (scale != 0.f) ms_add(mx, sum, x, scale);
+      }
+    }
+  }
+}
+
+struct FusedSmem {
+  float qs[1024];
+  float qv[128];
+  float part[256];
+};
+
+template <int DS>
+__global__ void __launch_bounds__(kSelThreads) score_select_topk_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ proj, int R,
+    const float* __restrict__ summ, int Hq, int Hkv, int D, int C,
+    const uint8_t* __restrict__ head_full, int k_free, int n_sink, int n_local,
+    int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ SelScratch s;
+  __shared__ BucketScratch bs;
+  __shared__ FusedSmem f;
+  const int exch_bytes = sort_exch_bytes(C);
+  uint64_t* exch = exch_bytes ? reinterpret_cast<uint64_t*>(sm) : nullptr;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + exch_bytes);
+  uint8_t* flags = sm + exch_bytes + static_cast<size_t>(C) * 4;
+  const int u = blockIdx.x, h = u % Hkv, b = u / Hkv, G = Hq / Hkv;
+  int32_t* row = idx + static_cast<int64_t>(u) * kmax;
+  if (head_full != nullptr && head_full[h]) {  // full heads read every chunk: no list
+    for (int i = threadIdx.x; i < kmax; i += blockDim.x) row[i] = -1;
+    if (threadIdx.x == 0) count[u] = 0;
+    return;
+  }
+  const float* summ_u = summ + static_cast<int64_t>(u) * C * DS;
+  float4 pre[kRowBatch];
+  rows_load<DS>(summ_u, C, rows_first_base<DS>(), pre);  // in flight during the query phase
+  unit_query(q, q_bf16, static_cast<int64_t>(b) * Hq + h * G, G, D, proj, R, f.qs, f.qv, f.part);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) flags[c] = is_forced(c, C, n_sink, n_local);
+  float mx_unused = 0.f, sum_unused = 0.f;
+  summaries_to_keys<DS>(summ_u, C, proj ? f.qv : f.qs, keys, n_sink, n_local, true, mx_unused,
+                        sum_unused, 0.f, pre);
+  __syncthreads();
+  topk_from_keys(keys, flags, C, n_sink, n_local, k_free, row, count + u, kmax, s, exch, bs);
+}
+
+template <int DS>
+__global__ void __launch_bounds__(kSelThreads) score_select_topp_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ proj, int R,
+    const float* __restrict__ summ, int Hq, int Hkv, int D, int C,
+    const uint8_t* __restrict__ head_full, float logit_scale, float p, int budget, int n_sink,
+    int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax,
+    int32_t* __restrict__ n_p_out, int SN) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ SelScratch s;
+  __shared__ BucketScratch bs;
+  __shared__ FusedSmem f;
+  const size_t head = topp_head_bytes(C, SN);
+  uint64_t* sortbuf = reinterpret_cast<uint64_t*>(sm);
+  float* cum = reinterpret_cast<float*>(sm + static_cast<size_t>(SN) * 8);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + head);
+  uint8_t* flags = sm + head + static_cast<size_t>(C) * 4;
+  const int u = blockIdx.x, h = u % Hkv, b = u / Hkv, G = Hq / Hkv;
+  if (head_full != nullptr && head_full[h]) {
+    int32_t* row = idx + static_cast<int64_t>(u) * kmax;
+    for (int i = threadIdx.x; i < kmax; i += blockDim.x) row[i] = -1;
+    if (threadIdx.x == 0) {
+      count[u] = 0;
+      if (n_p_out) n_p_out[u] = 0;
+    }
+    return;
+  }
+  const float* summ_u = summ + static_cast<int64_t>(u) * C * DS;
+  float4 pre[kRowBatch];
+  rows_load<DS>(summ_u, C, rows_first_base<DS>(), pre);  // in flight during the query phase
+  unit_query(q, q_bf16, static_cast<int64_t>(b) * Hq + h * G, G, D, proj, R, f.qs, f.qv, f.part);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) flags[c] = 0;
+  float mx = -INFINITY, Z = 0.f;
+  summaries_to_keys<DS>(summ_u, C, proj ? f.qv : f.qs, keys, 0, 0, false, mx, Z, logit_scale, pre);
+  block_max_sumexp(mx, Z, logit_scale, s);  // its barriers also publish keys
+  topp_select(keys, flags, sortbuf, cum, C, mx, Z, logit_scale, p, budget, n_sink, n_local, idx,
+              count, kmax, n_p_out, SN, u, s, bs);
 }
 
 int next_pow2(int x) {
@@ -458,7 +1076,7 @@ cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int 
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax) {
   if (U == 0) return cudaSuccess;
-  const size_t sh = static_cast<size_t>(C) * 5 + 16;
+  const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_topk_kernel), sh);
   if (e != cudaSuccess) return e;
   select_topk_kernel<<<U, kSelThreads, sh, l.stream>>>(scores, C, n_valid, k_free, n_sink, n_local,
@@ -471,7 +1089,7 @@ cudaError_t launch_select_topp(const Launch& l, const float* scores, int U, int 
                                int32_t* idx, int32_t* count, int kmax, int32_t* n_p_out) {
   if (U == 0) return cudaSuccess;
   const int SN = next_pow2(std::min(budget, C));
-  const size_t sh = static_cast<size_t>(SN) * 12 + static_cast<size_t>(C) * 5 + 16;
+  const size_t sh = topp_head_bytes(C, SN) + static_cast<size_t>(C) * 5 + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_topp_kernel), sh);
   if (e != cudaSuccess) return e;
   select_topp_kernel<<<U, kSelThreads, sh, l.stream>>>(scores, C, logit_scale, p, budget, n_sink,
@@ -488,14 +1106,79 @@ cudaError_t launch_select_hier(const Launch& l, const void* q, bool bf16, const 
   const int M = C / Gm;
   const int k1 = std::min(top_meta, M);
   const int NCH = k1 * Gm;
-  const size_t sh = static_cast<size_t>(M) * 5 + static_cast<size_t>(NCH) * 9 +
-                    static_cast<size_t>(k1) * 4 + static_cast<size_t>(C) + 16;
+  const size_t base = (static_cast<size_t>(M) * 5 + static_cast<size_t>(NCH) * 9 +
+                       static_cast<size_t>(k1) * 4 + static_cast<size_t>(C) + 15) & ~size_t(15);
+  const size_t sh = base + sort_exch_bytes(std::max(M, NCH)) + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_hier_kernel), sh);
   if (e != cudaSuccess) return e;
   select_hier_kernel<<<U, kSelThreads, sh, l.stream>>>(q, bf16 ? 1 : 0, meta, summ, Hq, Hkv, D, C,
                                                        Gm, top_meta, k_free, n_sink, n_local, idx,
                                                        count, kmax);
   return cudaGetLastError();
+}
+
+
+namespace {
+template <int DS>
+cudaError_t fused_topk_ds(const Launch& l, const void* q, bool bf16, const float* proj, int R,
+                          const float* summ, int U, int Hq, int Hkv, int D, int C,
+                          const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                          int32_t* idx, int32_t* count, int kmax) {
+  const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
+  cudaError_t e = set_smem(reinterpret_cast<const void*>(score_select_topk_kernel<DS>), sh);
+  if (e != cudaSuccess) return e;
+  score_select_topk_kernel<DS><<<U, kSelThreads, sh, l.stream>>>(
+      q, bf16 ? 1 : 0, proj, R, summ, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx,
+      count, kmax);
+  return cudaGetLastError();
+}
+
+template <int DS>
+cudaError_t fused_topp_ds(const Launch& l, const void* q, bool bf16, const float* proj, int R,
+                          const float* summ, int U, int Hq, int Hkv, int D, int C,
+                          const uint8_t* head_full, float logit_scale, float p, int budget,
+                          int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                          int32_t* n_p_out) {
+  const int SN = next_pow2(std::min(budget, C));
+  const size_t sh = topp_head_bytes(C, SN) + static_cast<size_t>(C) * 5 + 16;
+  cudaError_t e = set_smem(reinterpret_cast<const void*>(score_select_topp_kernel<DS>), sh);
+  if (e != cudaSuccess) return e;
+  score_select_topp_kernel<DS><<<U, kSelThreads, sh, l.stream>>>(
+      q, bf16 ? 1 : 0, proj, R, summ, Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink,
+      n_local, idx, count, kmax, n_p_out, SN);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_score_select_topk(const Launch& l, const void* q, bool bf16, const float* proj,
+                                     int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                     const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                                     int32_t* idx, int32_t* count, int kmax) {
+  const int U = B * Hkv;
+  if (U == 0) return cudaSuccess;
+  switch (proj ? R : D) {
+    case 16: return fused_topk_ds<16>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
+    case 32: return fused_topk_ds<32>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
+    case 64: return fused_topk_ds<64>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
+    case 128: return fused_topk_ds<128>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_score_select_topp(const Launch& l, const void* q, bool bf16, const float* proj,
+                                     int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                     const uint8_t* head_full, float logit_scale, float p,
+                                     int budget, int n_sink, int n_local, int32_t* idx,
+                                     int32_t* count, int kmax, int32_t* n_p_out) {
+  const int U = B * Hkv;
+  if (U == 0) return cudaSuccess;
+  switch (proj ? R : D) {
+    case 16: return fused_topp_ds<16>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink, n_local, idx, count, kmax, n_p_out);
+    case 32: return fused_topp_ds<32>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink, n_local, idx, count, kmax, n_p_out);
+    case 64: return fused_topp_ds<64>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink, n_local, idx, count, kmax, n_p_out);
+    case 128: return fused_topp_ds<128>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink, n_local, idx, count, kmax, n_p_out);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace csa

@@ -25,12 +25,16 @@ class SparseDecoder:
 
     K, V: [B, Hkv, T, D] (bf16 or fp32, contiguous, on the current device).
     select: "topk" | "topp" | "hier".  The summaries (and meta-summaries)
-    are computed once here, as part of building the cache."""
+    are computed once here, as part of building the cache.  With fused=True
+    (default) a step is two launches: fused score+select (one CTA per unit)
+    and the merged split-K decode; fused=False runs the separate calls
+    (score, select, decode, merge)."""
 
     def __init__(self, K: torch.Tensor, V: torch.Tensor, *, Hq: int, L: int, select: str,
                  n_sink: int, n_local: int, k_free: int = 0, proj: torch.Tensor | None = None,
                  p: float = 0.9, budget: int = 256, full_heads=(), Gm: int = 0, top_meta: int = 0,
-                 scale: float | None = None, num_parts: int = 0, out_dtype=torch.float32):
+                 scale: float | None = None, num_parts: int = 0, out_dtype=torch.float32,
+                 fused: bool = True):
         assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
         self.K, self.V = K, V
         B, Hkv, T, D = K.shape
@@ -68,6 +72,10 @@ class SparseDecoder:
         self.lse_part = torch.empty(B, Hq, self.max_splits, dtype=torch.float32, device=dev)
         self.out = torch.empty(B, Hq, D, dtype=out_dtype, device=dev)
         self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+        self.fused = fused
+        if fused:
+            self.ws_bytes = csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, self.P)
+            self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
 
     def select_chunks(self, q: torch.Tensor, stream=None):
         """Score + select: fills self.idx / self.count (and self.n_p for top-p)."""
@@ -78,6 +86,17 @@ class SparseDecoder:
             csa.csa_select_hier(q, qd, self.meta, self.summ, B, Hq, Hkv, D, C, self.Gm,
                                 self.top_meta, self.k_free, self.n_sink, self.n_local, self.idx,
                                 self.count, self.kmax, stream=stream)
+            return
+        if self.fused and self.select == "topk":
+            csa.csa_score_select_topk(q, qd, self.proj, self.R, self.summ, B, Hq, Hkv, D, C,
+                                      self.head_full, self.k_free, self.n_sink, self.n_local,
+                                      self.idx, self.count, self.kmax, stream=stream)
+            return
+        if self.fused and self.select == "topp":
+            csa.csa_score_select_topp(q, qd, self.proj, self.R, self.summ, B, Hq, Hkv, D, C,
+                                      self.head_full, 1.0 / math.sqrt(D), self.p, self.budget,
+                                      self.n_sink, self.n_local, self.idx, self.count, self.kmax,
+                                      self.n_p, stream=stream)
             return
         csa.csa_score_chunks(q, qd, self.proj, self.R, self.summ, B, 1, Hq, Hkv, D, C,
                              self.head_full, 0, 0, self.scores, stream=stream)
@@ -92,7 +111,15 @@ class SparseDecoder:
             raise ValueError(self.select)
 
     def attend(self, q: torch.Tensor, stream=None):
-        """Sparse split-K decode over the current index lists, then the LSE merge."""
+        """Sparse split-K decode over the current index lists, then the LSE merge
+        (one launch when fused)."""
+        if self.fused:
+            csa.csa_sparse_decode_merged(q, self.K, self.V, self.dtype, self.idx, self.count,
+                                         self.kmax, self.head_full, self.B, self.Hq, self.Hkv,
+                                         self.D, self.T, self.L, self.scale, self.P,
+                                         self.workspace, self.ws_bytes, self.out, _dt(self.out),
+                                         self.lse, stream=stream)
+            return
         csa.csa_sparse_decode(q, self.K, self.V, self.dtype, self.idx, self.count, self.kmax,
                               self.head_full, self.B, self.Hq, self.Hkv, self.D, self.T, self.L,
                               self.scale, self.P, self.max_splits, self.o_part, self.lse_part,

@@ -405,3 +405,137 @@ def test_host_pointer_rejected(csa):
         csa.csa_sparse_decode(q, q, q, torch.bfloat16, q, q, 1, None, 1, 4, 1, 128, 128, 128, 0.1,
                               1, 1, q, q)
     assert ei.value.status == 1
+
+
+# ---------------------------------------------------------------- fused paths
+
+@pytest.mark.parametrize("select,R,G,C", [("topk", 0, 4, 512), ("topk", 32, 8, 300),
+                                          ("topp", 16, 4, 1024), ("topp", 0, 2, 700)])
+def test_fused_score_select_equals_two_calls(csa, select, R, G, C):
+    """One CTA per unit computing scores into shared memory gives the same
+    index lists as csa_score_chunks followed by csa_select_*."""
+    B, Hkv, D = 2, 4, 128
+    Hq = G * Hkv
+    q = _randn((B, Hq, D), 30, torch.bfloat16)
+    P = _randn((D, R), 31) / 4 if R else None
+    Ds = R or D
+    summ = _randn((B, Hkv, C, Ds), 32) * 0.3
+    full = torch.tensor([0, 1, 0, 0], dtype=torch.uint8, device="cuda")
+    U = B * Hkv
+    kmax = min(C, (20 if select == "topk" else 64) + 3)
+    scores = torch.zeros(B, Hkv, 1, C, device="cuda")
+    csa.csa_score_chunks(q, q.dtype, P, R, summ, B, 1, Hq, Hkv, D, C, full, 0, 0, scores)
+    i1 = torch.full((U, kmax), 7, dtype=torch.int32, device="cuda")
+    c1 = torch.zeros(U, dtype=torch.int32, device="cuda")
+    i2, c2 = i1.clone(), c1.clone()
+    n1 = torch.zeros(U, dtype=torch.int32, device="cuda")
+    n2 = n1.clone()
+    if select == "topk":
+        csa.csa_select_topk(scores, U, C, None, 20, 1, 2, i1, c1, kmax)
+        csa.csa_score_select_topk(q, q.dtype, P, R, summ, B, Hq, Hkv, D, C, full, 20, 1, 2, i2, c2,
+                                  kmax)
+    else:
+        for p in (0.9, 0.3):
+            csa.csa_select_topp(scores, U, C, D ** -0.5, p, 64, 1, 2, i1, c1, kmax, n1)
+            csa.csa_score_select_topp(q, q.dtype, P, R, summ, B, Hq, Hkv, D, C, full, D ** -0.5,
+                                      p, 64, 1, 2, i2, c2, kmax, n2)
+    for u in range(U):
+        if u % Hkv == 1:
+            assert int(c2[u]) == 0 and torch.all(i2[u] == -1)
+            continue
+        assert torch.equal(i1[u], i2[u]) and int(c1[u]) == int(c2[u]), u
+        if select == "topp":
+            assert int(n1[u]) == int(n2[u])
+
+
+def _merged_case(csa, dtype, B, Hkv, G, D, T, L, sets, full=(), num_parts=0, out_bf16=False,
+                 with_lse=True, seed=40):
+    Hq = G * Hkv
+    C = T // L
+    dt = _dt(dtype)
+    q = _randn((B, Hq, D), seed, dt)
+    K = _randn((B, Hkv, T, D), seed + 1, dt)
+    V = _randn((B, Hkv, T, D), seed + 2, dt)
+    U = B * Hkv
+    kmax = max(1, max(len(s) for s in sets))
+    idx = torch.full((U, kmax), -1, dtype=torch.int32)
+    cnt = torch.zeros(U, dtype=torch.int32)
+    for u, s in enumerate(sets):
+        idx[u, :len(s)] = torch.tensor(sorted(s), dtype=torch.int32)
+        cnt[u] = len(s)
+    idx, cnt = idx.cuda(), cnt.cuda()
+    hf = None
+    if full:
+        hf = torch.zeros(Hkv, dtype=torch.uint8)
+        hf[list(full)] = 1
+        hf = hf.cuda()
+    scale = D ** -0.5
+    nbytes = csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    odt = torch.bfloat16 if out_bf16 else torch.float32
+    outs = []
+    for _ in range(2):  # the second call must see the counters reset by the first
+        out = torch.full((B, Hq, D), float("nan"), device="cuda").to(odt)
+        lse = torch.full((B, Hq), float("nan"), device="cuda") if with_lse else None
+        csa.csa_sparse_decode_merged(q, K, V, dt, idx, cnt, kmax, hf, B, Hq, Hkv, D, T, L, scale,
+                                     num_parts, ws, nbytes, out, odt, lse)
+        csa.csa_check_device_status()
+        outs.append((out.clone(), None if lse is None else lse.clone()))
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert int(ws[:4 * U].view(torch.int32).abs().sum()) == 0  # counters back at zero
+    out, lse = outs[1]
+    eff = [list(range(C)) if (u % Hkv) in full else sorted(s) for u, s in enumerate(sets)]
+    qn = to_np(q)
+    Kc, Vc = K.cpu(), V.cpu()
+    tol = "bf16" if (dtype == "bf16" or out_bf16) else "f32"
+    for u, s in enumerate(eff):
+        b, h = divmod(u, Hkv)
+        rows = slice(h * G, (h + 1) * G)
+        got = out[b, rows].float().cpu().double().numpy()
+        if not s:
+            assert np.all(got == 0)
+            if lse is not None:
+                assert torch.all(torch.isneginf(lse[b, rows]))
+            continue
+        ro, rl = O.decode_unit(qn[b, rows], to_np(Kc[b, h]), to_np(Vc[b, h]), s, L, scale)
+        parity.assert_close(got, ro, tol, f"merged unit {u}")
+        if lse is not None:
+            assert np.abs(lse[b, rows].cpu().double().numpy() - rl).max() < 1e-3
+    # same result as the split path (decode + separate merge), to fp32 rounding
+    if not out_bf16:
+        P = num_parts or csa.csa_decode_default_parts(dt, D, L)
+        o_part = torch.empty(B, Hq, P, D, device="cuda")
+        l_part = torch.empty(B, Hq, P, device="cuda")
+        csa.csa_sparse_decode(q, K, V, dt, idx, cnt, kmax, hf, B, Hq, Hkv, D, T, L, scale,
+                              num_parts, P, o_part, l_part)
+        ref = torch.empty(B, Hq, D, device="cuda")
+        csa.csa_lse_merge(o_part, l_part, B * Hq, P, D, ref, torch.float32, None)
+        assert (out - ref).abs().max().item() < 1e-5
+
+
+@pytest.mark.parametrize("dtype,D,L,G,parts", [("bf16", 128, 128, 4, 0), ("bf16", 128, 64, 4, 13),
+                                               ("bf16", 64, 64, 8, 7), ("f32", 64, 64, 4, 5),
+                                               ("f32", 128, 128, 2, 0), ("bf16", 64, 128, 1, 256)])
+def test_merged_decode_shapes(csa, dtype, D, L, G, parts):
+    B, Hkv, C = 2, 3, 24
+    rng = np.random.default_rng(D + L + G + parts)
+    sets = [sorted(rng.choice(C, size=int(rng.integers(1, 14)), replace=False).tolist())
+            for _ in range(B * Hkv)]
+    _merged_case(csa, dtype, B, Hkv, G, D, C * L, L, sets, num_parts=parts)
+
+
+def test_merged_decode_edge_cases(csa):
+    B, Hkv, G, D, L, C = 1, 4, 4, 128, 64, 9
+    sets = [[], [0], [2, 5, 8], list(range(9))]
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=1)      # one split each
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=200)    # more pieces than chunks
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, [[3], [0, 8], [], [1]], full=(2,), num_parts=7)
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=5, out_bf16=True)
+    _merged_case(csa, "f32", B, Hkv, G, 64, C * L, L, sets, num_parts=3, with_lse=False)
+
+
+def test_merged_decode_mixed_heads(csa):
+    B, Hkv, G, D, L, C = 1, 8, 4, 128, 128, 96
+    rng = np.random.default_rng(7)
+    sets = [sorted(rng.choice(C, size=20, replace=False).tolist()) for _ in range(B * Hkv)]
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, full=(0, 1))

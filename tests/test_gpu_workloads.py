@@ -15,17 +15,18 @@ from query_adaptive_chunk_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-def _decoder(w, inp):
+def _decoder(w, inp, fused=True):
     from query_adaptive_chunk_b200.steps import SparseDecoder
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
                          n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
-                         budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta)
+                         budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta,
+                         fused=fused)
 
 
-def run_and_check(w, units=None):
+def run_and_check(w, units=None, fused=True):
     from query_adaptive_chunk_b200 import csa
     inp = synth.make_decode_inputs(w, device="cuda")
-    dec = _decoder(w, inp)
+    dec = _decoder(w, inp, fused)
     out, lse = dec.step(inp["q"])
     csa.csa_check_device_status()
     all_units = synth.decode_units(w)
@@ -77,6 +78,10 @@ def test_topk_decode_full_size():
     run_and_check(synth.TOPK_32K)
 
 
+def test_topk_decode_full_size_separate_calls():
+    run_and_check(synth.TOPK_32K, fused=False)
+
+
 def test_topp_decode_prefix_cut():
     """C = 128 < budget: the cap cannot bind, the mass cut p decides."""
     run_and_check(synth.TOPP_128K.scaled(T=16384))
@@ -88,6 +93,10 @@ def test_topp_decode_reduced():
 
 def test_topp_mixed_decode_full_size():
     run_and_check(synth.TOPP_128K)
+
+
+def test_topp_mixed_decode_full_size_separate_calls():
+    run_and_check(synth.TOPP_128K, fused=False)
 
 
 def test_hier_decode_reduced():
