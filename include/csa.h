@@ -265,6 +265,34 @@ CSA_API csa_status csa_sparse_decode_merged(const void* q, const void* K, const 
                                             csa_dtype out_dtype, float* lse_out,
                                             csa_stream stream);
 
+/* The merged decode above for callers that cannot allocate device memory
+ * (the pages have no counterpart: this is a deployment convenience).  An
+ * application that manages all device memory through its own pool and
+ * forbids other allocations, or a serving loop that must not call cudaMalloc
+ * (which can synchronise the device) on its hot path, can call this instead
+ * of csa_sparse_decode_merged: it takes the same arguments minus the
+ * workspace and allocates nothing.  Its scratch (split partials and per-unit
+ * counters) is a fixed 16 MiB area inside the library, held by every GPU
+ * that loads the library until the process exits.
+ *   - Shapes whose scratch (csa_decode_workspace_bytes()) exceeds 16 MiB are
+ *     rejected with CSA_ERR_UNSUPPORTED (use fewer pieces, or the
+ *     workspace variant).
+ *   - The first call on a device looks up the area's device address; make
+ *     that first call before any stream capture on that device.
+ *   - The area starts zeroed when the library loads and keeps what each
+ *     call leaves; every call clears its counters on `stream` after its
+ *     decode, so the next call starts clean.  All calls share the one area:
+ *     calls that overlap on the GPU (other streams, other host threads)
+ *     race and must be serialised by the caller.  A call rejected on its
+ *     arguments enqueues nothing. */
+CSA_API csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K, const void* V,
+                                                    csa_dtype dtype, const int32_t* idx,
+                                                    const int32_t* count, int kmax,
+                                                    const uint8_t* head_full, int B, int Hq,
+                                                    int Hkv, int D, int64_t T, int L, float scale,
+                                                    int num_parts, void* out, csa_dtype out_dtype,
+                                                    float* lse_out, csa_stream stream);
+
 /* ---------------------------------------------------------------- a6
  * Log-sum-exp merge of split-K partials (SSA summary "핵심 기여": split-K
  * partials combined):

@@ -62,6 +62,8 @@ _SIGS = {
     "csa_decode_workspace_bytes": (_i64, [_i, _i, _i, _i, _i]),
     "csa_sparse_decode_merged": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i64,
                                       _i, _f, _i, _vp, _i64, _vp, _i, _vp, _vp]),
+    "csa_sparse_decode_merged_noalloc": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i,
+                                              _i64, _i, _f, _i, _vp, _i, _vp, _vp]),
     "csa_lse_merge": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp]),
     "csa_block_sparse_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                       _vp, _vp]),
@@ -209,6 +211,16 @@ def csa_sparse_decode_merged(q, K, V, dtype, idx, count, kmax, head_full, B, Hq,
                                         _p(head_full), B, Hq, Hkv, D, T, L, scale, num_parts,
                                         _p(workspace), workspace_bytes, _p(out), _dt(out_dtype),
                                         _p(lse_out), _s(stream)))
+
+
+def csa_sparse_decode_merged_noalloc(q, K, V, dtype, idx, count, kmax, head_full, B, Hq, Hkv, D,
+                                     T, L, scale, num_parts, out, out_dtype, lse_out, stream=None):
+    """csa_sparse_decode_merged without a workspace: the library's built-in
+    16 MiB scratch is used, so nothing is allocated (see include/csa.h)."""
+    _check(lib.csa_sparse_decode_merged_noalloc(_p(q), _p(K), _p(V), _dt(dtype), _p(idx),
+                                                _p(count), kmax, _p(head_full), B, Hq, Hkv, D, T,
+                                                L, scale, num_parts, _p(out), _dt(out_dtype),
+                                                _p(lse_out), _s(stream)))
 
 
 def csa_lse_merge(o_part, lse_part, rows, max_splits, D, out, out_dtype, lse_out, stream=None):

@@ -137,6 +137,10 @@ csa_status finish(cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace csa {
+void set_last_error(const std::string& why) { t_err = why; }
+}  // namespace csa
+
 extern "C" {
 
 int csa_version(void) { return 10000; }

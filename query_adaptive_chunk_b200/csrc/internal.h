@@ -12,6 +12,9 @@
 
 namespace csa {
 
+// Sets the thread-local message returned by csa_last_error_string().
+void set_last_error(const std::string& why);
+
 struct Launch {
   cudaStream_t stream;
   DevErr err;
