@@ -214,11 +214,14 @@ def _ext_event():
 def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
     """Device time of `steps` decode steps (L2 flushed before each).
 
-    Two CUDA graphs of the same step are replayed alternately inside the
-    timed loop: G1 (plain) gives the step time from events recorded around
-    the replay; G2 carries events around its select and decode nodes and
-    gives the decode kernel's own duration.  Without graph support the step
-    is timed from direct launches."""
+    Two CUDA graphs are replayed alternately inside the timed loop: G1 is
+    the step as a user runs it (one csa_decode_step call: selection, then
+    the decode launched behind it with programmatic dependent launch) and
+    gives the step time from events recorded around the replay; G2 runs the
+    selection and the merged decode as two plain launches with events
+    between them and gives the decode kernel's own duration (with the
+    overlap of G1 the kernel has no duration of its own).  Without graph
+    support the step is timed from direct launches."""
     inp = synth.make_decode_inputs(w, device="cuda")
     dec = decoder_for(w, inp)
     q = inp["q"]
@@ -236,8 +239,7 @@ def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
         torch.cuda.synchronize()
         g1 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g1, capture_error_mode="relaxed"):
-            dec.select_chunks(q)
-            dec.attend(q)
+            dec.step(q)
         g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2, capture_error_mode="relaxed"):
             ev[0].record()

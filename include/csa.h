@@ -293,6 +293,66 @@ CSA_API csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K
                                                     int num_parts, void* out, csa_dtype out_dtype,
                                                     float* lse_out, csa_stream stream);
 
+/* ---------------------------------------------------------------- a1-a6 in one call
+ * A whole decode step: the selection (csa_score_select_topk,
+ * csa_score_select_topp or csa_select_hier) followed by the merged split-K
+ * decode (csa_sparse_decode_merged), with the same results.  The decode is
+ * launched with programmatic dependent launch and works in two phases: the
+ * chunks of full-attention heads first, which do not depend on the
+ * selection and so stream while it runs, then the selected chunks of the
+ * sparse heads once the selection has completed (SSA summary "핵심 기여";
+ * Elastic Attention summary section 2.3: full and sparse heads in one pass).
+ * bf16 caches only.  Fields of the descriptor are the arguments of those
+ * calls.  num_parts 0 = the number of SMs minus B*Hkv (the selection's CTAs,
+ * which run beside the first phase) when head_full is given, else the
+ * number of SMs; at most 256.  The workspace must be sized for the P the
+ * call uses (csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts) with the
+ * same num_parts, 0 included, is always enough) and start zeroed once; each
+ * call leaves it zeroed again.  Errors: as the underlying calls; nothing is
+ * enqueued when an argument is rejected, and CSA_ERR_UNSUPPORTED for a
+ * fp32 cache (use the separate calls).  The step is two kernel launches on
+ * one stream and is safe to capture in a CUDA graph. */
+typedef enum csa_select_mode {
+  CSA_SELECT_TOPK = 0,
+  CSA_SELECT_TOPP = 1,
+  CSA_SELECT_HIER = 2
+} csa_select_mode;
+
+typedef struct csa_decode_step_desc {
+  /* query and KV cache */
+  const void* q;       /* [B, Hq, D] bf16 */
+  const void* K;       /* [B, Hkv, T, D] bf16 */
+  const void* V;       /* [B, Hkv, T, D] bf16 */
+  int B, Hq, Hkv, D;
+  int64_t T;
+  int L;
+  float scale;
+  const uint8_t* head_full; /* NULL or [Hkv] */
+  /* selection */
+  int mode;            /* csa_select_mode */
+  const float* summ;   /* [B, Hkv, C, Ds] fp32 */
+  const float* proj;   /* top-k / top-p: NULL or [D, R] fp32 */
+  int R;
+  const float* meta;   /* hierarchical: [B, Hkv, C/Gm, D] fp32 */
+  int Gm, top_meta;
+  int k_free, n_sink, n_local;
+  float logit_scale, p;  /* top-p */
+  int budget;            /* top-p */
+  int32_t* idx;          /* [B*Hkv, kmax] (output) */
+  int32_t* count;        /* [B*Hkv] (output) */
+  int kmax;
+  int32_t* n_p_out;      /* top-p: NULL or [B*Hkv] (output) */
+  /* decode and merge */
+  int num_parts;
+  void* workspace;       /* >= csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts) */
+  int64_t workspace_bytes;
+  void* out;             /* [B, Hq, D] of out_dtype (output) */
+  csa_dtype out_dtype;
+  float* lse_out;        /* NULL or [B, Hq] (output) */
+} csa_decode_step_desc;
+
+CSA_API csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream);
+
 /* ---------------------------------------------------------------- a6
  * Log-sum-exp merge of split-K partials (SSA summary "핵심 기여": split-K
  * partials combined):

@@ -65,6 +65,7 @@ _SIGS = {
     "csa_sparse_decode_merged_noalloc": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i,
                                               _i64, _i, _f, _i, _vp, _i, _vp, _vp]),
     "csa_lse_merge": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp]),
+    "csa_decode_step": (_i, [_vp, _vp]),
     "csa_block_sparse_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                       _vp, _vp]),
 }
@@ -221,6 +222,41 @@ def csa_sparse_decode_merged_noalloc(q, K, V, dtype, idx, count, kmax, head_full
                                                 _p(count), kmax, _p(head_full), B, Hq, Hkv, D, T,
                                                 L, scale, num_parts, _p(out), _dt(out_dtype),
                                                 _p(lse_out), _s(stream)))
+
+
+CSA_SELECT_TOPK, CSA_SELECT_TOPP, CSA_SELECT_HIER = 0, 1, 2
+
+
+class DecodeStepDesc(ctypes.Structure):
+    """ctypes mirror of csa_decode_step_desc (field order and types as in
+    include/csa.h)."""
+    _fields_ = [
+        ("q", _vp), ("K", _vp), ("V", _vp),
+        ("B", _i), ("Hq", _i), ("Hkv", _i), ("D", _i),
+        ("T", _i64), ("L", _i), ("scale", _f), ("head_full", _vp),
+        ("mode", _i), ("summ", _vp), ("proj", _vp), ("R", _i), ("meta", _vp),
+        ("Gm", _i), ("top_meta", _i), ("k_free", _i), ("n_sink", _i), ("n_local", _i),
+        ("logit_scale", _f), ("p", _f), ("budget", _i),
+        ("idx", _vp), ("count", _vp), ("kmax", _i), ("n_p_out", _vp),
+        ("num_parts", _i), ("workspace", _vp), ("workspace_bytes", _i64),
+        ("out", _vp), ("out_dtype", _i), ("lse_out", _vp),
+    ]
+
+
+def decode_step_desc(**kw) -> DecodeStepDesc:
+    """Build a descriptor; tensors become their data pointers, dtypes their codes."""
+    d = DecodeStepDesc()
+    for k, v in kw.items():
+        if k == "out_dtype":
+            v = _dt(v)
+        elif isinstance(v, torch.Tensor) or (v is None and k not in ("scale", "p")):
+            v = None if v is None else v.data_ptr()
+        setattr(d, k, v)
+    return d
+
+
+def csa_decode_step(desc: DecodeStepDesc, stream=None):
+    _check(lib.csa_decode_step(ctypes.byref(desc), _s(stream)))
 
 
 def csa_lse_merge(o_part, lse_part, rows, max_splits, D, out, out_dtype, lse_out, stream=None):

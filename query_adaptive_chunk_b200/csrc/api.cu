@@ -516,6 +516,63 @@ csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* 
                 "score_select_topp launch");
 }
 
+csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
+  CSA_REQUIRE(d != nullptr, "descriptor is NULL");
+  CSA_REQUIRE(d->mode == CSA_SELECT_TOPK || d->mode == CSA_SELECT_TOPP || d->mode == CSA_SELECT_HIER,
+              "mode must be CSA_SELECT_TOPK, CSA_SELECT_TOPP or CSA_SELECT_HIER");
+  CSA_REQUIRE(valid_dtype(d->out_dtype), "out_dtype");
+  CSA_TRY(decode_shape_checks(CSA_BF16, d->kmax, d->B, d->Hq, d->Hkv, d->D, d->T, d->L, d->scale,
+                              d->num_parts));
+  CSA_SUPPORT(d->num_parts <= csa::kMergedMaxParts, "num_parts must be <= 256");
+  if (d->B == 0) return CSA_OK;
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  // decode arguments first, so that a rejected call enqueues nothing
+  int P = 0;
+  CSA_TRY(decode_ptr_checks(d->q, d->K, d->V, d->idx, d->count, d->head_full, true, d->D, d->L,
+                            d->num_parts, l, &P));
+  if (d->num_parts == 0 && d->head_full != nullptr) {
+    // The selection runs one CTA per (batch, KV head) unit beside the
+    // decode's first phase: leave it those SMs (counted without reading
+    // head_full, so that the call stays free of host-device copies).
+    P = std::max(1, std::min(csa::kMergedMaxParts, l.num_sms - d->B * d->Hkv));
+  } else if (d->num_parts == 0) {
+    P = std::min(csa::kMergedMaxParts, l.num_sms);
+  }
+  const WorkspaceLayout w = workspace_layout(d->B, d->Hq, d->Hkv, d->D, P);
+  CSA_REQUIRE(d->workspace_bytes >= static_cast<int64_t>(w.total),
+              "workspace smaller than csa_decode_workspace_bytes()");
+  CSA_TRY(check_ptr(d->workspace, "workspace"));
+  CSA_TRY(check_ptr(d->out, "out"));
+  CSA_TRY(check_ptr(d->lse_out, "lse_out", false));
+  const int C = static_cast<int>(d->T / d->L);
+  // the selection (validates its own arguments before launching)
+  csa_status st;
+  if (d->mode == CSA_SELECT_TOPK)
+    st = csa_score_select_topk(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
+                               d->head_full, d->k_free, d->n_sink, d->n_local, d->idx, d->count,
+                               d->kmax, stream);
+  else if (d->mode == CSA_SELECT_TOPP)
+    st = csa_score_select_topp(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
+                               d->head_full, d->logit_scale, d->p, d->budget, d->n_sink, d->n_local,
+                               d->idx, d->count, d->kmax, d->n_p_out, stream);
+  else
+    st = csa_select_hier(d->q, CSA_BF16, d->meta, d->summ, d->B, d->Hq, d->Hkv, d->D, C, d->Gm,
+                         d->top_meta, d->k_free, d->n_sink, d->n_local, d->idx, d->count, d->kmax,
+                         stream);
+  if (st != CSA_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(d->workspace);
+  csa::MergeOut m{reinterpret_cast<int*>(ws + w.counters), d->out, d->out_dtype == CSA_BF16,
+                  d->lse_out, true};
+  std::string why;
+  cudaError_t e = csa::launch_decode(l, d->q, d->K, d->V, true, d->idx, d->count, d->kmax,
+                                     d->head_full, d->B, d->Hq, d->Hkv, d->D, d->T, d->L, d->scale,
+                                     P, P, reinterpret_cast<float*>(ws + w.o),
+                                     reinterpret_cast<float*>(ws + w.lse), &m, &why);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  return finish(e, "decode step launch");
+}
+
 csa_status csa_lse_merge(const float* o_part, const float* lse_part, int rows, int max_splits, int D,
                          void* out, csa_dtype out_dtype, float* lse_out, csa_stream stream) {
   CSA_REQUIRE(valid_dtype(out_dtype), "out_dtype");

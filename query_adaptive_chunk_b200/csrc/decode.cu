@@ -36,6 +36,7 @@ constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kStageBudget = 192 * 1024;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kDeferMax = 32;  // merges a CTA can postpone to the end of its work
 
 struct DecodeParams {
   const void* q;  // [B, Hq, D]
@@ -58,10 +59,23 @@ struct DecodeParams {
   void* out;       // [B, Hq, D] fp32 or bf16
   int out_bf16;
   float* lse_out;  // [B, Hq] or null
+  // phased: full-head units first (no dependency on the selection), then,
+  // after griddepcontrol.wait, the sparse units (launched with programmatic
+  // dependent launch behind the selection kernel)
+  int phased;
 };
 
-__device__ __forceinline__ int unit_count(const DecodeParams& p, int u) {
-  if (p.head_full != nullptr && p.head_full[u % p.Hkv]) return p.C;
+// Unit sets of a phase: 0 = every unit, 1 = full-head units, 2 = sparse units.
+__device__ __forceinline__ bool unit_in(const DecodeParams& p, int u, int mode) {
+  if (mode == 0) return true;
+  const bool full = p.head_full != nullptr && p.head_full[u % p.Hkv];
+  return mode == 1 ? full : !full;
+}
+
+__device__ __forceinline__ int unit_count(const DecodeParams& p, int u, int mode = 0) {
+  const bool full = p.head_full != nullptr && p.head_full[u % p.Hkv];
+  if (mode == 1) return full ? p.C : 0;
+  if (full) return mode == 2 ? 0 : p.C;
   int n = p.count[u];
   if (n < 0 || n > p.kmax) {
     dev_flag(p.err, DEV_BAD_INDEX);
@@ -80,20 +94,46 @@ __device__ __forceinline__ int unit_chunk(const DecodeParams& p, int u, int pos)
   return c;
 }
 
-// prefix[0..U] of the effective chunk counts (all threads of the block).
-__device__ void build_prefix(const DecodeParams& p, int* prefix, int* scan_sh) {
+// prefix[0..U] of the effective chunk counts of a phase (all threads of the block).
+__device__ void build_prefix(const DecodeParams& p, int* prefix, int* scan_sh, int mode = 0) {
   const int seg = (p.U + blockDim.x - 1) / blockDim.x;
   const int lo = min(p.U, static_cast<int>(threadIdx.x) * seg), hi = min(p.U, lo + seg);
   int loc = 0;
-  for (int u = lo; u < hi; ++u) loc += unit_count(p, u);
+  for (int u = lo; u < hi; ++u) loc += unit_count(p, u, mode);
   int total = 0;
   int run = block_exclusive_scan(loc, scan_sh, &total);
   for (int u = lo; u < hi; ++u) {
     prefix[u] = run;
-    run += unit_count(p, u);
+    run += unit_count(p, u, mode);
   }
   if (threadIdx.x == 0) prefix[p.U] = total;
   __syncthreads();
+}
+
+// The same by one warp (the producer), without a block barrier.
+__device__ void warp_build_prefix(const DecodeParams& p, int* prefix, int mode) {
+  const int lane = threadIdx.x & 31;
+  const int seg = (p.U + 31) / 32;
+  const int lo = min(p.U, lane * seg), hi = min(p.U, lo + seg);
+  int loc = 0;
+  for (int u = lo; u < hi; ++u) loc += unit_count(p, u, mode);
+  int inc = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  int run = inc - loc;
+  for (int u = lo; u < hi; ++u) {
+    prefix[u] = run;
+    run += unit_count(p, u, mode);
+  }
+  if (lane == 31) prefix[p.U] = inc;
+  __syncwarp();
+}
+
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Unit owning global chunk g (prefix[u] <= g < prefix[u+1]); empty units skipped.
@@ -132,6 +172,19 @@ __device__ __forceinline__ void store_out(const DecodeParams& p, int64_t idx, fl
     static_cast<float*>(p.out)[idx] = v;
 }
 
+// Merged mode: units of the phase with no chunk get out = 0, lse = -inf
+// (no split exists to merge them); CTA c covers units c, c + P, ...
+__device__ void zero_empty_units(const DecodeParams& p, const int* prefix, int mode, int nthreads) {
+  for (int u = blockIdx.x; u < p.U; u += gridDim.x) {
+    if (!unit_in(p, u, mode) || prefix[u + 1] > prefix[u]) continue;
+    const int b = u / p.Hkv, h = u % p.Hkv;
+    const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * p.G;
+    for (int e = threadIdx.x; e < p.G * p.D; e += nthreads) store_out(p, row0 * p.D + e, 0.f);
+    if (p.lse_out)
+      for (int g = threadIdx.x; g < p.G; g += nthreads) p.lse_out[row0 + g] = -INFINITY;
+  }
+}
+
 // Slots of unit u beyond its split count get lse = -inf (CTA c covers units
 // u = c, c + P, ...).  Threads [0, nthreads) of the block take part.
 __device__ void fill_empty_slots(const DecodeParams& p, const int* prefix, int nthreads) {
@@ -159,10 +212,9 @@ __device__ void fill_empty_slots(const DecodeParams& p, const int* prefix, int n
 // into the unit's G output rows.  `wts` holds >= G * ns floats of shared
 // memory; `nthr` threads take part; `sync` is a barrier over them that
 // returns false on a timeout.
-template <int D, typename Sync>
+template <int D, int BATCH, typename Sync>
 __device__ bool merge_unit(const DecodeParams& p, int u, int ns, float* wts, int nthr, Sync sync) {
   constexpr int D4 = D / 4;
-  constexpr int BATCH = 24;
   const int b = u / p.Hkv, h = u % p.Hkv, G = p.G;
   const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
@@ -252,7 +304,7 @@ struct DecodeLayout {
   static constexpr int BAR_OFF = NS * STAGE_BYTES;
   static constexpr int FLUSH_OFF = BAR_OFF + 2 * NS * 8 + 16;  // + flush mbarrier
   static constexpr int PREFIX_OFF = FLUSH_OFF + FLUSH_BYTES;
-  static size_t bytes(int U) { return 1024 + PREFIX_OFF + static_cast<size_t>(U + 1) * 4; }
+  static size_t bytes(int U) { return 1024 + PREFIX_OFF + 2 * static_cast<size_t>(U + 1) * 4; }
 };
 
 template <int D, int L>
@@ -278,6 +330,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   int* prefix = reinterpret_cast<int*>(smem + Lay::PREFIX_OFF);         // [U+1]
   __shared__ int scan_sh[33];
   __shared__ int last_sh;
+  __shared__ int defer_u[kDeferMax], defer_ns[kDeferMax];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -292,52 +345,73 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
-  build_prefix(p, prefix, scan_sh);  // ends with __syncthreads (also publishes the barriers)
-
-  const int64_t N = prefix[p.U];
+  build_prefix(p, prefix, scan_sh, p.phased ? 1 : 0);  // ends with __syncthreads (also publishes the barriers)
+  int* prefix2 = prefix + (p.U + 1);  // phase 2 (sparse units), built by the producer
+  const uint32_t phase_bar = flush_bar + 8;
+  if (threadIdx.x == 0) {
+    mbar_init(phase_bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int n_phase = p.phased ? 2 : 1;
   const int64_t P = gridDim.x;
-  const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
 
   if (warp == kConsumerWarps) {
     // ---------------------------------------------------------------- producer
     int64_t issued = 0;
     bool ok = true;
-    for (int64_t g0 = a; g0 < bnd && ok; g0 += 32) {
-      const int64_t g = g0 + lane;
-      int row = 0;
-      if (g < bnd) {
-        const int u = unit_of(prefix, p.U, g);
-        const int c = unit_chunk(p, u, static_cast<int>(g - prefix[u]));
-        row = static_cast<int>(u * p.T + static_cast<int64_t>(c) * L);
+    for (int ph = 0; ph < n_phase && ok; ++ph) {
+      const int* pre = prefix;
+      if (ph == 1) {  // the selection has to be complete from here on
+        grid_dependency_wait();
+        warp_build_prefix(p, prefix2, 2);
+        if (lane == 0) mbar_arrive(phase_bar);
+        pre = prefix2;
       }
-      const int nb = static_cast<int>(bnd - g0 < 32 ? bnd - g0 : 32);
-      for (int j = 0; j < nb; ++j) {
-        const int row_j = __shfl_sync(0xffffffffu, row, j);
-        int good = 1;
-        if (lane == 0) {
-          const int64_t i = g0 - a + j;
-          const int s = static_cast<int>(i % NS);
-          const uint32_t it = static_cast<uint32_t>(i / NS);
-          if (!mbar_wait(empty_bar + 8 * s, (it & 1u) ^ 1u, p.err)) {
-            good = 0;
-          } else {
-            const uint32_t fb = full_bar + 8 * s;
-            mbar_arrive_expect_tx(fb, Lay::STAGE_BYTES);
-            const uint32_t dst = sbase + s * Lay::STAGE_BYTES;
+      const int64_t N = pre[p.U];
+      const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+      for (int64_t g0 = a; g0 < bnd && ok; g0 += 32) {
+        const int64_t g = g0 + lane;
+        int row = 0;
+        if (g < bnd) {
+          const int u = unit_of(pre, p.U, g);
+          const int c = unit_chunk(p, u, static_cast<int>(g - pre[u]));
+          row = static_cast<int>(u * p.T + static_cast<int64_t>(c) * L);
+        }
+        const int nb = static_cast<int>(bnd - g0 < 32 ? bnd - g0 : 32);
+        for (int j = 0; j < nb; ++j) {
+          const int row_j = __shfl_sync(0xffffffffu, row, j);
+          int good = 1;
+          if (lane == 0) {
+            const int64_t i = issued;
+            const int s = static_cast<int>(i % NS);
+            const uint32_t it = static_cast<uint32_t>(i / NS);
+            if (!mbar_wait(empty_bar + 8 * s, (it & 1u) ^ 1u, p.err)) {
+              good = 0;
+            } else {
+              const uint32_t fb = full_bar + 8 * s;
+              mbar_arrive_expect_tx(fb, Lay::STAGE_BYTES);
+              const uint32_t dst = sbase + s * Lay::STAGE_BYTES;
 #pragma unroll
-            for (int bx = 0; bx < NBOX; ++bx) {
-              tma_load_2d(dst + bx * Lay::BOX_BYTES, &tmK, bx * 64, row_j, fb);
-              tma_load_2d(dst + Lay::KV_BYTES + bx * Lay::BOX_BYTES, &tmV, bx * 64, row_j, fb);
+              for (int bx = 0; bx < NBOX; ++bx) {
+                tma_load_2d(dst + bx * Lay::BOX_BYTES, &tmK, bx * 64, row_j, fb);
+                tma_load_2d(dst + Lay::KV_BYTES + bx * Lay::BOX_BYTES, &tmV, bx * 64, row_j, fb);
+              }
             }
-            ++issued;
+          }
+          issued = __shfl_sync(0xffffffffu, issued + good, 0);
+          good = __shfl_sync(0xffffffffu, good, 0);
+          if (!good) {
+            ok = false;
+            break;
           }
         }
-        good = __shfl_sync(0xffffffffu, good, 0);
-        if (!good) {
-          ok = false;
-          break;
-        }
       }
+    }
+    if (!ok && p.phased) {  // never leave the consumers waiting: hand them an empty phase
+      for (int u = lane; u <= p.U; u += 32) prefix2[u] = 0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(phase_bar);
     }
     // no copy may still be landing when the CTA retires
     if (lane == 0) {
@@ -349,7 +423,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
 
   // ------------------------------------------------------------------ consumers
-  fill_empty_slots(p, prefix, kConsumerWarps * 32);
+  const int* pre = prefix;
+  int64_t N = pre[p.U];
+  int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+  if (p.merged) zero_empty_units(p, pre, p.phased ? 1 : 0, kConsumerWarps * 32);
+  else fill_empty_slots(p, pre, kConsumerWarps * 32);
   const float scale_log2 = p.scale_log2;
   const int hA = 2 * (lane & 3), hB = hA + 1;
   uint32_t qf[KS][2];
@@ -358,6 +436,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   int cur_u = -1;
   uint32_t flush_phase = 0;
   bool ok = true;
+  int n_defer = 0;  // units whose merge falls to this CTA, done after the loop
 
   auto load_q = [&](int u) {
     const int b = u / p.Hkv, h = u % p.Hkv;
@@ -411,8 +490,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     if (!group_sync()) return false;
     const int b = u / p.Hkv, h = u % p.Hkv;
-    const int slot = split_slot(prefix[u], a, blockIdx.x, N, P);
-    const int ns = split_count(prefix[u], prefix[u + 1], N, P);
+    const int slot = split_slot(pre[u], a, blockIdx.x, N, P);
+    const int ns = split_count(pre[u], pre[u + 1], N, P);
     const bool direct = p.merged && ns == 1;  // the only split: it is the output
     for (int e = threadIdx.x; e < p.G * D; e += kConsumerWarps * 32) {
       const int g = e / D, d = e % D;
@@ -444,105 +523,144 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     if (!group_sync()) return false;
     if (!last_sh) return true;
+    if (n_defer < kDeferMax) {  // merge after the main loop, off the hot path
+      if (threadIdx.x == 0) {
+        defer_u[n_defer] = u;
+        defer_ns[n_defer] = ns;
+      }
+      ++n_defer;
+      return true;
+    }
     __threadfence();
-    if (!merge_unit<D>(p, u, ns, fo, kConsumerWarps * 32, group_sync)) return false;
+    if (!merge_unit<D, 8>(p, u, ns, fo, kConsumerWarps * 32, group_sync)) return false;
     if (threadIdx.x == 0) p.counters[u] = 0;  // ready for the next call
     return true;
   };
 
-  for (int64_t g = a, i = 0; g < bnd; ++g, ++i) {
-    if (cur_u < 0 || g >= prefix[cur_u + 1]) {
-      if (cur_u >= 0 && !flush(cur_u)) {
+  int64_t i = 0;
+  for (int ph = 0; ph < n_phase && ok; ++ph) {
+    if (ph == 1) {
+      if (cur_u >= 0) {  // phases hold different units
+        if (!flush(cur_u)) {
+          ok = false;
+          break;
+        }
+        cur_u = -1;
+      }
+      if (!mbar_wait(phase_bar, 0u, p.err)) {
         ok = false;
         break;
       }
-      cur_u = unit_of(prefix, p.U, g);
-      load_q(cur_u);
+      grid_dependency_wait();
+      pre = prefix2;
+      N = pre[p.U];
+      a = N * blockIdx.x / P;
+      bnd = N * (blockIdx.x + 1) / P;
+      zero_empty_units(p, pre, 2, kConsumerWarps * 32);
     }
-    const int s = static_cast<int>(i % NS);
-    const uint32_t it = static_cast<uint32_t>(i / NS);
-    if (!mbar_wait(full_bar + 8 * s, it & 1u, p.err)) {
-      ok = false;
-      break;
-    }
-    const uint32_t sK = sbase + s * Lay::STAGE_BYTES;
-    const uint32_t sV = sK + Lay::KV_BYTES;
-    const int tok0 = warp * TOK_W;
+    for (int64_t g = a; g < bnd; ++g, ++i) {
+      if (cur_u < 0 || g >= pre[cur_u + 1]) {
+        if (cur_u >= 0 && !flush(cur_u)) {
+          ok = false;
+          break;
+        }
+        cur_u = unit_of(pre, p.U, g);
+        load_q(cur_u);
+      }
+      const int s = static_cast<int>(i % NS);
+      const uint32_t it = static_cast<uint32_t>(i / NS);
+      if (!mbar_wait(full_bar + 8 * s, it & 1u, p.err)) {
+        ok = false;
+        break;
+      }
+      const uint32_t sK = sbase + s * Lay::STAGE_BYTES;
+      const uint32_t sV = sK + Lay::KV_BYTES;
+      const int tok0 = warp * TOK_W;
 
-    // S^T = K q^T over this warp's tokens
-    float sc[MT][4];
+      // S^T = K q^T over this warp's tokens
+      float sc[MT][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+      for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int bx = ks >> 2, colb = (ks & 3) * 16;
+      for (int ks = 0; ks < KS; ++ks) {
+        const int bx = ks >> 2, colb = (ks & 3) * 16;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int row = tok0 + mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int col = colb + (lane >> 4) * 8;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(sK + bx * Lay::BOX_BYTES + sw128_offset(row, col), a0, a1, a2, a3);
+          mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        }
+      }
+      // online softmax (log2 domain), per head hA / hB of this lane
+      float cm0 = -INFINITY, cm1 = -INFINITY;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        const int row = tok0 + mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int col = colb + (lane >> 4) * 8;
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(sK + bx * Lay::BOX_BYTES + sw128_offset(row, col), a0, a1, a2, a3);
-        mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[mt][e] *= scale_log2;
+        cm0 = fmaxf(cm0, fmaxf(sc[mt][0], sc[mt][2]));
+        cm1 = fmaxf(cm1, fmaxf(sc[mt][1], sc[mt][3]));
       }
-    }
-    // online softmax (log2 domain), per head hA / hB of this lane
-    float cm0 = -INFINITY, cm1 = -INFINITY;
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
+      for (int x = 4; x < 32; x <<= 1) {
+        cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, x));
+        cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, x));
+      }
+      const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
+      const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      uint32_t pb[MT][2];
+      float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sc[mt][e] *= scale_log2;
-      cm0 = fmaxf(cm0, fmaxf(sc[mt][0], sc[mt][2]));
-      cm1 = fmaxf(cm1, fmaxf(sc[mt][1], sc[mt][3]));
-    }
-#pragma unroll
-    for (int x = 4; x < 32; x <<= 1) {
-      cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, x));
-      cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, x));
-    }
-    const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
-    const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    uint32_t pb[MT][2];
-    float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const float p0 = fast_exp2(sc[mt][0] - mn0), p1 = fast_exp2(sc[mt][1] - mn1);
-      const float p2 = fast_exp2(sc[mt][2] - mn0), p3 = fast_exp2(sc[mt][3] - mn1);
-      ps0 += p0 + p2;
-      ps1 += p1 + p3;
-      pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
-      pb[mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
-    }
-    l0 = l0 * al0 + ps0;
-    l1 = l1 * al1 + ps1;
-#pragma unroll
-    for (int dt = 0; dt < KS; ++dt) {
-      o[dt][0] *= al0;
-      o[dt][1] *= al1;
-      o[dt][2] *= al0;
-      o[dt][3] *= al1;
-    }
-    // O^T += V^T P^T
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
+      for (int mt = 0; mt < MT; ++mt) {
+        const float p0 = fast_exp2(sc[mt][0] - mn0), p1 = fast_exp2(sc[mt][1] - mn1);
+        const float p2 = fast_exp2(sc[mt][2] - mn0), p3 = fast_exp2(sc[mt][3] - mn1);
+        ps0 += p0 + p2;
+        ps1 += p1 + p3;
+        pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+        pb[mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+      }
+      l0 = l0 * al0 + ps0;
+      l1 = l1 * al1 + ps1;
 #pragma unroll
       for (int dt = 0; dt < KS; ++dt) {
-        const int bx = dt >> 2, colb = (dt & 3) * 16;
-        const int mi = lane >> 3;
-        const int tok = tok0 + mt * 16 + (lane & 7) + (mi >> 1) * 8;
-        const int col = colb + (mi & 1) * 8;
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_trans(sV + bx * Lay::BOX_BYTES + sw128_offset(tok, col), a0, a1, a2, a3);
-        mma_bf16_16816(o[dt], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+        o[dt][0] *= al0;
+        o[dt][1] *= al1;
+        o[dt][2] *= al0;
+        o[dt][3] *= al1;
       }
+      // O^T += V^T P^T
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt) {
+          const int bx = dt >> 2, colb = (dt & 3) * 16;
+          const int mi = lane >> 3;
+          const int tok = tok0 + mt * 16 + (lane & 7) + (mi >> 1) * 8;
+          const int col = colb + (mi & 1) * 8;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(sV + bx * Lay::BOX_BYTES + sw128_offset(tok, col), a0, a1, a2, a3);
+          mma_bf16_16816(o[dt], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar + 8 * s);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty_bar + 8 * s);
   }
-  if (ok && cur_u >= 0) flush(cur_u);
+  if (ok && cur_u >= 0) ok = flush(cur_u);
+  if (!ok || n_defer == 0) return;
+  // deferred merges: thread 0 wrote the list after the flushes' last barrier
+  if (!group_sync()) return;
+  __threadfence();
+  for (int k = 0; k < n_defer && k < kDeferMax; ++k) {
+    const int u = defer_u[k];
+    if (!merge_unit<D, 24>(p, u, defer_ns[k], fo, kConsumerWarps * 32, group_sync)) return;
+    if (threadIdx.x == 0) p.counters[u] = 0;  // ready for the next call
+  }
 }
 
 // ------------------------------------------------------------------ fp32 path
@@ -596,7 +714,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
       __syncthreads();
       if (last_sh) {
         __threadfence();
-        merge_unit<D>(p, u, ns, wts, kF32Threads, [] { __syncthreads(); return true; });
+        merge_unit<D, 8>(p, u, ns, wts, kF32Threads, [] { __syncthreads(); return true; });
         if (tid == 0) p.counters[u] = 0;
       }
     }
@@ -770,8 +888,24 @@ cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, c
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sh));
   if (e != cudaSuccess) return e;
-  fn<<<P, kDecodeThreads, sh, l.stream>>>(tmK, tmV, p);
-  return cudaGetLastError();
+  if (!p.phased) {
+    fn<<<P, kDecodeThreads, sh, l.stream>>>(tmK, tmV, p);
+    return cudaGetLastError();
+  }
+  // programmatic dependent launch: the grid may start while the selection
+  // kernel before it still runs; the kernel waits (griddepcontrol.wait)
+  // before it reads anything the selection writes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P);
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = sh;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, tmK, tmV, p);
 }
 
 }  // namespace
@@ -803,6 +937,7 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
     p.out = merge->out;
     p.out_bf16 = merge->out_bf16 ? 1 : 0;
     p.lse_out = merge->lse_out;
+    p.phased = (merge->phased && bf16) ? 1 : 0;
   }
   p.D = D;
   p.q = q;

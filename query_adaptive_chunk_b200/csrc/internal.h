@@ -65,6 +65,10 @@ struct MergeOut {
   void* out;       // [B, Hq, D]
   bool out_bf16;
   float* lse_out;  // [B, Hq] or null
+  // bf16 only: full-head units first, then (after the selection kernel that
+  // precedes it on the stream completes) the sparse units; the decode is
+  // launched with programmatic dependent launch
+  bool phased = false;
 };
 constexpr int kMergedMaxParts = 256;
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,

@@ -33,6 +33,13 @@ __host__ __device__ __forceinline__ int sort_exch_bytes(int C) {
   return 8 * (p < kSelThreads ? kSelThreads : p);
 }
 
+// Lets a grid launched behind this one with programmatic dependent launch
+// start now; that grid still waits for this one's completion before it reads
+// what this one writes.
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   uint32_t b = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
   return __uint_as_float(b);
@@ -812,6 +819,7 @@ __global__ void __launch_bounds__(kSelThreads) select_hier_kernel(
     const float* __restrict__ summ, int Hq, int Hkv, int D, int C, int Gm, int top_meta,
     int k_free, int n_sink, int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count,
     int kmax) {
+  allow_dependent_launch();
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
   __shared__ BucketScratch bs;
@@ -993,6 +1001,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_topk_kernel(
     const float* __restrict__ summ, int Hq, int Hkv, int D, int C,
     const uint8_t* __restrict__ head_full, int k_free, int n_sink, int n_local,
     int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
+  allow_dependent_launch();
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
   __shared__ BucketScratch bs;
@@ -1027,6 +1036,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_topp_kernel(
     const uint8_t* __restrict__ head_full, float logit_scale, float p, int budget, int n_sink,
     int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax,
     int32_t* __restrict__ n_p_out, int SN) {
+  allow_dependent_launch();
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
   __shared__ BucketScratch bs;

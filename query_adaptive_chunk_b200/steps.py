@@ -28,7 +28,9 @@ class SparseDecoder:
     are computed once here, as part of building the cache.  With fused=True
     (default) a step is two launches: fused score+select (one CTA per unit)
     and the merged split-K decode; fused=False runs the separate calls
-    (score, select, decode, merge)."""
+    (score, select, decode, merge).  With a bf16 cache and fused=True,
+    ``step`` is one call of csa_decode_step, whose decode streams the
+    full-attention heads while the selection runs."""
 
     def __init__(self, K: torch.Tensor, V: torch.Tensor, *, Hq: int, L: int, select: str,
                  n_sink: int, n_local: int, k_free: int = 0, proj: torch.Tensor | None = None,
@@ -73,9 +75,24 @@ class SparseDecoder:
         self.out = torch.empty(B, Hq, D, dtype=out_dtype, device=dev)
         self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
         self.fused = fused
+        self.num_parts = num_parts
         if fused:
-            self.ws_bytes = csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, self.P)
+            # sized for the larger of the two P the merged paths may use
+            self.ws_bytes = max(csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, self.P),
+                                csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts))
             self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.desc = None
+        if fused and self.dtype == csa.CSA_BF16:
+            mode = {"topk": csa.CSA_SELECT_TOPK, "topp": csa.CSA_SELECT_TOPP,
+                    "hier": csa.CSA_SELECT_HIER}[select]
+            self.desc = csa.decode_step_desc(
+                K=K, V=V, B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, L=L, scale=self.scale,
+                head_full=self.head_full, mode=mode, summ=self.summ, proj=proj, R=self.R,
+                meta=self.meta, Gm=Gm, top_meta=top_meta, k_free=k_free, n_sink=n_sink,
+                n_local=n_local, logit_scale=1.0 / math.sqrt(D), p=p, budget=budget, idx=self.idx,
+                count=self.count, kmax=self.kmax, n_p_out=self.n_p, num_parts=num_parts,
+                workspace=self.workspace, workspace_bytes=self.ws_bytes, out=self.out,
+                out_dtype=self.out.dtype, lse_out=self.lse)
 
     def select_chunks(self, q: torch.Tensor, stream=None):
         """Score + select: fills self.idx / self.count (and self.n_p for top-p)."""
@@ -128,6 +145,10 @@ class SparseDecoder:
                           self.out, _dt(self.out), self.lse, stream=stream)
 
     def step(self, q: torch.Tensor, stream=None):
+        if self.desc is not None and q.dtype == torch.bfloat16:
+            self.desc.q = q.data_ptr()
+            csa.csa_decode_step(self.desc, stream=stream)
+            return self.out, self.lse
         self.select_chunks(q, stream)
         self.attend(q, stream)
         return self.out, self.lse

@@ -76,3 +76,32 @@ def test_wait_limit_setting(csa):
         assert csa.csa_get_wait_limit_ns() == 123456
     finally:
         csa.csa_set_wait_limit_ns(old)
+
+
+def test_decode_step_descriptor_layout(csa):
+    """The ctypes mirror of csa_decode_step_desc has the C struct's size and
+    field offsets (compiled from include/csa.h by the host compiler)."""
+    import tempfile
+    fields = [f for f, _ in csa.DecodeStepDesc._fields_]
+    prog = ['#include <stdio.h>', '#include <stddef.h>', '#include "csa.h"', 'int main(void) {',
+            '  printf("%zu\\n", sizeof(csa_decode_step_desc));']
+    prog += [f'  printf("%zu\\n", offsetof(csa_decode_step_desc, {f}));' for f in fields]
+    prog += ['  return 0;', '}']
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(B.__file__))), "include")
+    with tempfile.TemporaryDirectory() as d:
+        src, exe = os.path.join(d, "l.c"), os.path.join(d, "l")
+        with open(src, "w") as f:
+            f.write("\n".join(prog) + "\n")
+        subprocess.run(["gcc", "-I", inc, src, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True,
+                                               check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(csa.DecodeStepDesc)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(csa.DecodeStepDesc, f).offset == off, f
+
+
+def test_decode_step_rejects_on_host(csa):
+    d = csa.decode_step_desc(B=1, Hq=4, Hkv=1, D=128, T=1024, L=64, scale=0.1, mode=7, kmax=4)
+    assert csa.lib.csa_decode_step(ctypes.byref(d), ctypes.c_void_p(0)) == 1
+    assert "mode" in csa.csa_last_error_string()
+    assert csa.lib.csa_decode_step(None, ctypes.c_void_p(0)) == 1

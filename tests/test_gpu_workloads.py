@@ -112,3 +112,19 @@ def test_decode_batch_with_gqa8_and_d64():
                              L=64, dtype="bf16", select="topk", n_sink=1, n_local=2, k_free=9,
                              planted=3)
     run_and_check(w)
+
+
+def test_topk_decode_full_heads_one_call_step():
+    """Full and sparse heads in one csa_decode_step: the full heads' chunks
+    are decoded while the selection runs, the sparse heads' after it."""
+    w = synth.DecodeWorkload(name="topk_mixed_step", seed=12, B=2, Hq=32, Hkv=8, D=128,
+                             T=128 * 96, L=128, dtype="bf16", select="topk", n_sink=1, n_local=2,
+                             k_free=13, planted=4, full_heads=(0, 3, 7))
+    run_and_check(w)
+
+
+def test_hier_decode_full_heads_one_call_step():
+    import dataclasses
+    w = dataclasses.replace(synth.HIER_1M.scaled(T=65536, planted=4), name="hier_mixed_step",
+                            full_heads=(2,))
+    run_and_check(w)
