@@ -81,6 +81,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const D
   }
 }
 
+// mbar_wait by all 32 lanes of a warp, with a warp-uniform result: warp-
+// collective instructions (shuffles, ldmatrix, mma.sync, tcgen05.ld/st) that
+// follow must not see a warp split by a timeout that only some lanes met.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DevErr& e) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, e));
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,

@@ -9,16 +9,23 @@
 //     issues, per chunk, 2-D TMA loads of the chunk's K and V rows
 //     ([L x 64] boxes, 128-byte swizzle) into a ring of stages that fills
 //     ~192 KB of shared memory (3 stages of 64 KB at L = 128, D = 128), i.e.
-//     enough bytes in flight per SM to cover HBM latency.
+//     enough bytes in flight per SM to cover HBM latency.  With the first
+//     chunk of each unit it also copies the unit's query rows into the
+//     stage's q slot, on the same barrier.
 //   * warps 0-3 (consumers): each takes L/4 tokens of every chunk.  S^T =
 //     K q^T runs on the tensor cores as mma.m16n8k16 with the tokens as M and
 //     the query heads of the GQA group as N (up to 8); the online softmax
 //     stays in registers (per-head running max/sum); P is moved into the B
 //     layout with movmatrix and O^T += V^T P^T runs as a second mma.  The
 //     math per 64 KB chunk is a few hundred warp instructions, so the SM
-//     stays bound by the copy engine, not by issue.
-//   * at a unit boundary the four warps combine their (m, l, O) through
-//     shared memory and write one split partial (o normalised, lse).
+//     stays bound by the copy engine, not by issue.  At a unit boundary each
+//     warp drops its (m, l, O) into a flush buffer (two, double-buffered)
+//     and streams on.
+//   * warp 5 (epilogue): combines the four warps' partials of each unit into
+//     one split partial (o normalised, lse), or the output when the unit has
+//     a single split, and in merged mode counts the split in; the CTA that
+//     brings a unit's last split merges it after its main loop, with the
+//     partials staged through shared memory.
 // Every wait is an mbarrier wait with a time limit; there is no named
 // barrier, so a timeout anywhere makes the kernel wind down, never hang.
 //
@@ -31,8 +38,10 @@
 namespace csa {
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kConsumerWarps = 4;                    // warps 0-3
+constexpr int kProducerWarp = kConsumerWarps;        // warp 4
+constexpr int kEpilogueWarp = kConsumerWarps + 1;    // warp 5
+constexpr int kDecodeThreads = (kConsumerWarps + 2) * 32;
 constexpr int kStageBudget = 192 * 1024;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -210,14 +219,15 @@ __device__ void fill_empty_slots(const DecodeParams& p, const int* prefix, int n
 
 // Combine the ns split partials of unit u (already in L2, read with ld.cg)
 // into the unit's G output rows.  `wts` holds >= G * ns floats of shared
-// memory; `nthr` threads take part; `sync` is a barrier over them that
-// returns false on a timeout.
+// memory; `nthr` threads take part, `tid` in [0, nthr) numbering them by
+// whole warps; `sync` is a barrier over them that returns false on a timeout.
 template <int D, int BATCH, typename Sync>
-__device__ bool merge_unit(const DecodeParams& p, int u, int ns, float* wts, int nthr, Sync sync) {
+__device__ bool merge_unit(const DecodeParams& p, int u, int ns, float* wts, int tid, int nthr,
+                           Sync sync) {
   constexpr int D4 = D / 4;
   const int b = u / p.Hkv, h = u % p.Hkv, G = p.G;
   const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+  const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
   // Output items e = (head g, float4 column c4).  The partial loads of this
   // thread's first item do not depend on the weights: issue them first so
   // they are in flight during the lse phase.
@@ -294,43 +304,194 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// Shared-memory layout of the bf16 kernel, offsets from the 1024-aligned base:
+// K/V stages | q slots (one per stage) | flush buffers | mbarriers | prefix[2][U+1].
+struct DecLayout {
+  int nf;        // flush buffers: 2, or 1 when two do not fit
+  int fb_bytes;  // one flush buffer: per consumer warp O [G][D], m [8], l [8]
+  int q_off, fb_off, bar_off, prefix_off;
+  size_t total;  // dynamic shared memory to request (with the alignment slack)
+};
+
+constexpr int kQSlotHeads = 8;          // a q slot holds up to 8 query heads
+constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block
+
 template <int D, int L>
-struct DecodeLayout {
+struct DecodeShape {
   static constexpr int KV_BYTES = L * D * 2;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES;
   static constexpr int NS = kStageBudget / STAGE_BYTES;
   static constexpr int BOX_BYTES = L * 128;
-  static constexpr int FLUSH_BYTES = kConsumerWarps * 8 * D * 4 + kConsumerWarps * 8 * 2 * 4;
-  static constexpr int BAR_OFF = NS * STAGE_BYTES;
-  static constexpr int FLUSH_OFF = BAR_OFF + 2 * NS * 8 + 16;  // + flush mbarrier
-  static constexpr int PREFIX_OFF = FLUSH_OFF + FLUSH_BYTES;
-  static size_t bytes(int U) { return 1024 + PREFIX_OFF + 2 * static_cast<size_t>(U + 1) * 4; }
+  static constexpr int QSLOT_BYTES = kQSlotHeads * D * 2;
 };
+
+__host__ __device__ inline DecLayout dec_layout(int D, int L, int G, int U, int nf) {
+  const int stage_bytes = 2 * L * D * 2;
+  const int ns = kStageBudget / stage_bytes;
+  DecLayout y;
+  y.nf = nf;
+  y.fb_bytes = (kConsumerWarps * G * D * 4 + 2 * kConsumerWarps * 8 * 4 + 127) & ~127;
+  y.q_off = ns * stage_bytes;
+  y.fb_off = y.q_off + ns * kQSlotHeads * D * 2;
+  y.bar_off = y.fb_off + nf * y.fb_bytes;
+  y.prefix_off = y.bar_off + (2 * ns + 6) * 8;  // full[ns], empty[ns], fb_full[2], fb_empty[2], phase, end
+  y.total = 1024 + static_cast<size_t>(y.prefix_off) + 2 * static_cast<size_t>(U + 1) * 4;
+  return y;
+}
+
+__host__ __device__ inline DecLayout dec_layout(int D, int L, int G, int U) {
+  DecLayout y = dec_layout(D, L, G, U, 2);
+  if (y.total > kMaxDynSmem) y = dec_layout(D, L, G, U, 1);
+  return y;
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Merge of unit u by one warp, straight from global memory (rarely used:
+// more merges fell to one CTA than its deferred list holds).
+template <int D>
+__device__ void merge_unit_warp(const DecodeParams& p, int u, int ns) {
+  constexpr int D4 = D / 4;
+  const int lane = threadIdx.x & 31;
+  const int b = u / p.Hkv, h = u % p.Hkv;
+  for (int g = 0; g < p.G; ++g) {
+    const int64_t row = static_cast<int64_t>(b) * p.Hq + h * p.G + g;
+    const float* ls = p.lse_part + row * p.max_splits;
+    float mx = -INFINITY;
+    for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldcg(ls + s));
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+    float sum = 0.f;
+    for (int s = lane; s < ns; s += 32) sum += expf(__ldcg(ls + s) - mx);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
+    const float lse = mx + logf(sum);
+    if (lane < D4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4* src = reinterpret_cast<const float4*>(p.o_part + row * p.max_splits * D) + lane;
+      for (int s = 0; s < ns; ++s) {
+        const float wgt = expf(__ldcg(ls + s) - lse);
+        const float4 x = __ldcg(src + static_cast<int64_t>(s) * D4);
+        acc.x += wgt * x.x;
+        acc.y += wgt * x.y;
+        acc.z += wgt * x.z;
+        acc.w += wgt * x.w;
+      }
+      const int64_t o = row * D + lane * 4;
+      store_out(p, o, acc.x);
+      store_out(p, o + 1, acc.y);
+      store_out(p, o + 2, acc.z);
+      store_out(p, o + 3, acc.w);
+    }
+    if (lane == 0 && p.lse_out) p.lse_out[row] = lse;
+  }
+}
+
+// Merge of unit u with its partials first copied into shared memory (one
+// round trip to L2 for all of them), by `nthr` threads numbered `tid`.
+// `area` (area_bytes, the idle K/V stage ring) holds the partials and, in
+// its last 8 KB, the split weights.  Falls back to merge_unit when the
+// partials do not fit.
+template <int D, typename Sync>
+__device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area, int area_bytes,
+                             int tid, int nthr, Sync sync) {
+  constexpr int D4 = D / 4;
+  const int G = p.G;
+  float* wts = reinterpret_cast<float*>(area + area_bytes - 8192);
+  if (static_cast<size_t>(G) * ns * D * 4 > static_cast<size_t>(area_bytes) - 8192)
+    return merge_unit<D, 8>(p, u, ns, wts, tid, nthr, sync);
+  const int b = u / p.Hkv, h = u % p.Hkv;
+  const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
+  float* st = reinterpret_cast<float*>(area);  // [G][ns][D]
+  const int n16 = G * ns * D4;
+  for (int e = tid; e < n16; e += nthr) {
+    const int c4 = e % D4, gs = e / D4, g = gs / ns, s = gs % ns;
+    cp_async16(smem_u32(st + static_cast<size_t>(gs) * D + c4 * 4),
+               p.o_part + ((row0 + g) * p.max_splits + s) * D + c4 * 4);
+  }
+  for (int e = tid; e < G * ns; e += nthr) {
+    const int g = e / ns, sl = e % ns;
+    wts[e] = __ldcg(p.lse_part + (row0 + g) * p.max_splits + sl);
+  }
+  cp_async_wait_all();
+  if (!sync()) return false;
+  const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+  for (int g = warp; g < G; g += nw) {
+    float mx = -INFINITY;
+    for (int sl = lane; sl < ns; sl += 32) mx = fmaxf(mx, wts[g * ns + sl]);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+    float sum = 0.f;
+    for (int sl = lane; sl < ns; sl += 32) sum += expf(wts[g * ns + sl] - mx);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
+    const float lse = mx + logf(sum);
+    __syncwarp();
+    for (int sl = lane; sl < ns; sl += 32) wts[g * ns + sl] = expf(wts[g * ns + sl] - lse);
+    if (lane == 0 && p.lse_out) p.lse_out[row0 + g] = lse;
+  }
+  if (!sync()) return false;
+  for (int e = tid; e < G * D4; e += nthr) {
+    const int g = e / D4, c4 = e % D4;
+    const float* src = st + static_cast<size_t>(g) * ns * D + c4 * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < ns; ++s) {
+      const float wk = wts[g * ns + s];
+      const float4 x = *reinterpret_cast<const float4*>(src + static_cast<size_t>(s) * D);
+      acc.x += wk * x.x;
+      acc.y += wk * x.y;
+      acc.z += wk * x.z;
+      acc.w += wk * x.w;
+    }
+    const int64_t o = (row0 + g) * D + c4 * 4;
+    store_out(p, o, acc.x);
+    store_out(p, o + 1, acc.y);
+    store_out(p, o + 2, acc.z);
+    store_out(p, o + 3, acc.w);
+  }
+  return sync();
+}
 
 template <int D, int L>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
-  using Lay = DecodeLayout<D, L>;
-  constexpr int NS = Lay::NS;
+  using Sh = DecodeShape<D, L>;
+  constexpr int NS = Sh::NS;
   constexpr int TOK_W = L / kConsumerWarps;  // tokens per consumer warp
   constexpr int MT = TOK_W / 16;             // 16-token m-tiles per warp
   constexpr int KS = D / 16;                 // k-steps (QK) / d-tiles (PV)
   constexpr int NBOX = D / 64;
+  const DecLayout Y = dec_layout(D, L, p.G, p.U);
+  const int G = p.G;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t full_bar = sbase + Lay::BAR_OFF;
+  const uint32_t full_bar = sbase + Y.bar_off;
   const uint32_t empty_bar = full_bar + NS * 8;
-  const uint32_t flush_bar = empty_bar + NS * 8;
-  float* fo = reinterpret_cast<float*>(smem + Lay::FLUSH_OFF);          // [4][8][D]
-  float* fm = fo + kConsumerWarps * 8 * D;                              // [4][8]
-  float* fl = fm + kConsumerWarps * 8;                                  // [4][8]
-  int* prefix = reinterpret_cast<int*>(smem + Lay::PREFIX_OFF);         // [U+1]
+  const uint32_t fb_full = empty_bar + NS * 8;  // [2]
+  const uint32_t fb_empty = fb_full + 16;       // [2]
+  const uint32_t phase_bar = fb_empty + 16;
+  const uint32_t end_bar = phase_bar + 8;
+  int* prefix = reinterpret_cast<int*>(smem + Y.prefix_off);  // [U+1]
+  int* prefix2 = prefix + (p.U + 1);  // phase 2 (sparse units), built by the producer
   __shared__ int scan_sh[33];
-  __shared__ int last_sh;
   __shared__ int defer_u[kDeferMax], defer_ns[kDeferMax];
+  __shared__ int n_defer_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -338,26 +499,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       mbar_init(full_bar + 8 * s, 1);
       mbar_init(empty_bar + 8 * s, kConsumerWarps);
     }
-    mbar_init(flush_bar, kConsumerWarps * 32);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(fb_full + 8 * k, kConsumerWarps * 32);
+      mbar_init(fb_empty + 8 * k, 1);
+    }
+    mbar_init(phase_bar, 1);
+    mbar_init(end_bar, (kConsumerWarps + 1) * 32);
+    n_defer_sh = 0;
     fence_barrier_init();
   }
-  if (warp == kConsumerWarps && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
   build_prefix(p, prefix, scan_sh, p.phased ? 1 : 0);  // ends with __syncthreads (also publishes the barriers)
-  int* prefix2 = prefix + (p.U + 1);  // phase 2 (sparse units), built by the producer
-  const uint32_t phase_bar = flush_bar + 8;
-  if (threadIdx.x == 0) {
-    mbar_init(phase_bar, 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
   const int n_phase = p.phased ? 2 : 1;
   const int64_t P = gridDim.x;
 
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer
+    const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
+    const uint32_t q_bytes = static_cast<uint32_t>(G) * D * 2;
     int64_t issued = 0;
     bool ok = true;
     for (int ph = 0; ph < n_phase && ok; ++ph) {
@@ -372,15 +534,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
       for (int64_t g0 = a; g0 < bnd && ok; g0 += 32) {
         const int64_t g = g0 + lane;
-        int row = 0;
+        int row = 0, qu = -1;
         if (g < bnd) {
           const int u = unit_of(pre, p.U, g);
           const int c = unit_chunk(p, u, static_cast<int>(g - pre[u]));
           row = static_cast<int>(u * p.T + static_cast<int64_t>(c) * L);
+          if (g == a || g == pre[u]) qu = u;  // first chunk of a unit here: its q rides along
         }
         const int nb = static_cast<int>(bnd - g0 < 32 ? bnd - g0 : 32);
         for (int j = 0; j < nb; ++j) {
           const int row_j = __shfl_sync(0xffffffffu, row, j);
+          const int qu_j = __shfl_sync(0xffffffffu, qu, j);
           int good = 1;
           if (lane == 0) {
             const int64_t i = issued;
@@ -390,12 +554,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               good = 0;
             } else {
               const uint32_t fb = full_bar + 8 * s;
-              mbar_arrive_expect_tx(fb, Lay::STAGE_BYTES);
-              const uint32_t dst = sbase + s * Lay::STAGE_BYTES;
+              mbar_arrive_expect_tx(fb, Sh::STAGE_BYTES + (qu_j >= 0 ? q_bytes : 0u));
+              if (qu_j >= 0) {
+                const int64_t qrow = static_cast<int64_t>(qu_j / p.Hkv) * p.Hq + (qu_j % p.Hkv) * G;
+                bulk_load(sbase + Y.q_off + s * Sh::QSLOT_BYTES, qg + qrow * D, q_bytes, fb);
+              }
+              const uint32_t dst = sbase + s * Sh::STAGE_BYTES;
 #pragma unroll
               for (int bx = 0; bx < NBOX; ++bx) {
-                tma_load_2d(dst + bx * Lay::BOX_BYTES, &tmK, bx * 64, row_j, fb);
-                tma_load_2d(dst + Lay::KV_BYTES + bx * Lay::BOX_BYTES, &tmV, bx * 64, row_j, fb);
+                tma_load_2d(dst + bx * Sh::BOX_BYTES, &tmK, bx * 64, row_j, fb);
+                tma_load_2d(dst + Sh::KV_BYTES + bx * Sh::BOX_BYTES, &tmV, bx * 64, row_j, fb);
               }
             }
           }
@@ -408,7 +576,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
       }
     }
-    if (!ok && p.phased) {  // never leave the consumers waiting: hand them an empty phase
+    if (!ok && p.phased) {  // never leave the other warps waiting: hand them an empty phase
       for (int u = lane; u <= p.U; u += 32) prefix2[u] = 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(phase_bar);
@@ -419,6 +587,130 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int64_t i = first; i < issued; ++i)
         mbar_wait(full_bar + 8 * static_cast<int>(i % NS), static_cast<uint32_t>(i / NS) & 1u, p.err);
     }
+    return;
+  }
+
+  // consumers and the epilogue warp meet at the end (merged mode) to run
+  // the merges that fell to this CTA
+  uint32_t end_phase = 0;
+  auto end_sync = [&]() -> bool {
+    mbar_arrive(end_bar);
+    const bool r = warp_wait(end_bar, end_phase, p.err);
+    end_phase ^= 1u;
+    return r;
+  };
+  auto final_merges = [&](int tid) {
+    if (!end_sync()) return;
+    const int nd = n_defer_sh;
+    if (nd == 0) return;
+    __threadfence();
+    for (int k = 0; k < nd; ++k) {
+      const int u = defer_u[k];
+      if (!merge_staged<D>(p, u, defer_ns[k], smem, NS * Sh::STAGE_BYTES, tid,
+                           (kConsumerWarps + 1) * 32, end_sync))
+        return;
+      if (tid == 0) p.counters[u] = 0;  // ready for the next call
+    }
+  };
+
+  if (warp == kEpilogueWarp) {
+    // ---------------------------------------------------------------- epilogue
+    // Takes each unit's four per-warp partials from a flush buffer, combines
+    // them into the unit's split partial (or its output when it has one
+    // split), and counts the split in (merged mode) while the consumers
+    // stream on.
+    bool ok = true;
+    int nseen = 0, n_defer = 0;
+    for (int ph = 0; ph < n_phase && ok; ++ph) {
+      const int* pre = prefix;
+      if (ph == 1) {
+        if (!warp_wait(phase_bar, 0u, p.err)) {
+          ok = false;
+          break;
+        }
+        pre = prefix2;
+      }
+      const int64_t N = pre[p.U];
+      const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+      if (a >= bnd) continue;
+      const int u0 = unit_of(pre, p.U, a), u1 = unit_of(pre, p.U, bnd - 1);
+      for (int u = u0; u <= u1 && ok; ++u) {
+        if (pre[u + 1] <= pre[u]) continue;  // no chunk: never flushed
+        const int k = Y.nf == 2 ? (nseen & 1) : 0;
+        const int use = Y.nf == 2 ? (nseen >> 1) : nseen;
+        if (!warp_wait(fb_full + 8 * k, static_cast<uint32_t>(use) & 1u, p.err)) {
+          ok = false;
+          break;
+        }
+        ++nseen;
+        const float* fo = reinterpret_cast<const float*>(smem + Y.fb_off + k * Y.fb_bytes);
+        const float* fm = fo + kConsumerWarps * G * D;
+        const float* fl = fm + kConsumerWarps * 8;
+        const int b = u / p.Hkv, h = u % p.Hkv;
+        const int slot = split_slot(pre[u], a, blockIdx.x, N, P);
+        const int ns = split_count(pre[u], pre[u + 1], N, P);
+        const bool direct = p.merged && ns == 1;  // the only split: it is the output
+        // per head g = lane: max over the warps, warp weights, total sum
+        float M = -INFINITY, Ls = 0.f, scw[kConsumerWarps];
+        if (lane < G) {
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + lane]);
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            scw[w] = exp2f(fm[w * 8 + lane] - M);
+            Ls += fl[w * 8 + lane] * scw[w];
+          }
+        }
+        for (int g = 0; g < G; ++g) {
+          const float Mg = __shfl_sync(0xffffffffu, M, g), Lg = __shfl_sync(0xffffffffu, Ls, g);
+          float sc[kConsumerWarps];
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) sc[w] = __shfl_sync(0xffffffffu, scw[w], g);
+          const float inv = 1.0f / Lg;
+          const int64_t row = static_cast<int64_t>(b) * p.Hq + h * G + g;
+          for (int d = lane; d < D; d += 32) {
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) acc += fo[(w * G + g) * D + d] * sc[w];
+            if (direct) store_out(p, row * D + d, acc * inv);
+            else p.o_part[(row * p.max_splits + slot) * D + d] = acc * inv;
+          }
+          if (lane == 0) {
+            const float lse = (Mg + log2f(Lg)) * kLn2;
+            if (direct) {
+              if (p.lse_out) p.lse_out[row] = lse;
+            } else {
+              p.lse_part[row * p.max_splits + slot] = lse;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(fb_empty + 8 * k);  // the consumers may refill it
+        if (!p.merged || direct) continue;
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(p.counters + u, 1) == ns - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        if (n_defer < kDeferMax) {  // merged after the main loop, off the hot path
+          if (lane == 0) {
+            defer_u[n_defer] = u;
+            defer_ns[n_defer] = ns;
+          }
+          ++n_defer;
+        } else {
+          __threadfence();
+          merge_unit_warp<D>(p, u, ns);
+          __syncwarp();
+          if (lane == 0) p.counters[u] = 0;
+        }
+      }
+    }
+    if (!p.merged) return;
+    if (lane == 0) n_defer_sh = n_defer;
+    __syncwarp();
+    final_merges(kConsumerWarps * 32 + lane);
     return;
   }
 
@@ -433,47 +725,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint32_t qf[KS][2];
   float o[KS][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  int cur_u = -1;
-  uint32_t flush_phase = 0;
+  int cur_u = -1, nflush = 0;
   bool ok = true;
-  int n_defer = 0;  // units whose merge falls to this CTA, done after the loop
 
-  auto load_q = [&](int u) {
-    const int b = u / p.Hkv, h = u % p.Hkv;
-    const int n = lane >> 2;
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q);
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int d0 = ks * 16 + 2 * (lane & 3);
-      if (n < p.G) {
-        const __nv_bfloat16* r = qb + (static_cast<int64_t>(b) * p.Hq + h * p.G + n) * D;
-        qf[ks][0] = *reinterpret_cast<const uint32_t*>(r + d0);
-        qf[ks][1] = *reinterpret_cast<const uint32_t*>(r + d0 + 8);
-      } else {
-        qf[ks][0] = 0u;
-        qf[ks][1] = 0u;
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[ks][e] = 0.f;
-    }
-    m0 = m1 = -INFINITY;
-    l0 = l1 = 0.f;
-  };
-
-  auto group_sync = [&]() -> bool {
-    mbar_arrive(flush_bar);
-    const bool r = mbar_wait(flush_bar, flush_phase, p.err);
-    flush_phase ^= 1u;
-    return r;
-  };
-
-  auto flush = [&](int u) -> bool {
+  // Hand this warp's (m, l, O) of unit u to the epilogue warp and go on.
+  auto flush_async = [&](int u) -> bool {
 #pragma unroll
     for (int x = 4; x < 32; x <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, x);
       l1 += __shfl_xor_sync(0xffffffffu, l1, x);
     }
-    float* fow = fo + warp * 8 * D;
+    (void)u;
+    const int k = Y.nf == 2 ? (nflush & 1) : 0;
+    const int use = Y.nf == 2 ? (nflush >> 1) : nflush;
+    if (use > 0 && !warp_wait(fb_empty + 8 * k, static_cast<uint32_t>(use - 1) & 1u, p.err))
+      return false;
+    float* fo = reinterpret_cast<float*>(smem + Y.fb_off + k * Y.fb_bytes);
+    float* fm = fo + kConsumerWarps * G * D;
+    float* fl = fm + kConsumerWarps * 8;
     if (lane < 4) {
       fm[warp * 8 + hA] = m0;
       fm[warp * 8 + hB] = m1;
@@ -483,57 +752,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
     for (int dt = 0; dt < KS; ++dt) {
       const int d = dt * 16 + (lane >> 2);
-      fow[hA * D + d] = o[dt][0];
-      fow[hB * D + d] = o[dt][1];
-      fow[hA * D + d + 8] = o[dt][2];
-      fow[hB * D + d + 8] = o[dt][3];
-    }
-    if (!group_sync()) return false;
-    const int b = u / p.Hkv, h = u % p.Hkv;
-    const int slot = split_slot(pre[u], a, blockIdx.x, N, P);
-    const int ns = split_count(pre[u], pre[u + 1], N, P);
-    const bool direct = p.merged && ns == 1;  // the only split: it is the output
-    for (int e = threadIdx.x; e < p.G * D; e += kConsumerWarps * 32) {
-      const int g = e / D, d = e % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + g]);
-      float Ls = 0.f, acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float sc = exp2f(fm[w * 8 + g] - M);
-        Ls += fl[w * 8 + g] * sc;
-        acc += fo[(w * 8 + g) * D + d] * sc;
+      if (hA < G) {
+        fo[(warp * G + hA) * D + d] = o[dt][0];
+        fo[(warp * G + hA) * D + d + 8] = o[dt][2];
       }
-      const int64_t row = static_cast<int64_t>(b) * p.Hq + h * p.G + g;
-      const float lse = (M + log2f(Ls)) * kLn2;
-      if (direct) {
-        store_out(p, row * D + d, acc / Ls);
-        if (d == 0 && p.lse_out) p.lse_out[row] = lse;
-      } else {
-        p.o_part[(row * p.max_splits + slot) * D + d] = acc / Ls;
-        if (d == 0) p.lse_part[row * p.max_splits + slot] = lse;
+      if (hB < G) {
+        fo[(warp * G + hB) * D + d] = o[dt][1];
+        fo[(warp * G + hB) * D + d + 8] = o[dt][3];
       }
     }
-    if (!group_sync()) return false;
-    if (!p.merged || direct) return true;
-    if (threadIdx.x == 0) {
-      __threadfence();
-      last_sh = atomicAdd(p.counters + u, 1) == ns - 1;
-    }
-    if (!group_sync()) return false;
-    if (!last_sh) return true;
-    if (n_defer < kDeferMax) {  // merge after the main loop, off the hot path
-      if (threadIdx.x == 0) {
-        defer_u[n_defer] = u;
-        defer_ns[n_defer] = ns;
-      }
-      ++n_defer;
-      return true;
-    }
-    __threadfence();
-    if (!merge_unit<D, 8>(p, u, ns, fo, kConsumerWarps * 32, group_sync)) return false;
-    if (threadIdx.x == 0) p.counters[u] = 0;  // ready for the next call
+    mbar_arrive(fb_full + 8 * k);
+    ++nflush;
     return true;
   };
 
@@ -541,13 +770,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   for (int ph = 0; ph < n_phase && ok; ++ph) {
     if (ph == 1) {
       if (cur_u >= 0) {  // phases hold different units
-        if (!flush(cur_u)) {
+        if (!flush_async(cur_u)) {
           ok = false;
           break;
         }
         cur_u = -1;
       }
-      if (!mbar_wait(phase_bar, 0u, p.err)) {
+      if (!warp_wait(phase_bar, 0u, p.err)) {
         ok = false;
         break;
       }
@@ -559,22 +788,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       zero_empty_units(p, pre, 2, kConsumerWarps * 32);
     }
     for (int64_t g = a; g < bnd; ++g, ++i) {
+      const int s = static_cast<int>(i % NS);
+      const uint32_t it = static_cast<uint32_t>(i / NS);
+      if (!warp_wait(full_bar + 8 * s, it & 1u, p.err)) {
+        ok = false;
+        break;
+      }
       if (cur_u < 0 || g >= pre[cur_u + 1]) {
-        if (cur_u >= 0 && !flush(cur_u)) {
+        if (cur_u >= 0 && !flush_async(cur_u)) {
           ok = false;
           break;
         }
         cur_u = unit_of(pre, p.U, g);
-        load_q(cur_u);
+        // the unit's q arrived with this stage
+        const __nv_bfloat16* qs =
+            reinterpret_cast<const __nv_bfloat16*>(smem + Y.q_off + s * Sh::QSLOT_BYTES);
+        const int n = lane >> 2;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int d0 = ks * 16 + 2 * (lane & 3);
+          if (n < G) {
+            qf[ks][0] = *reinterpret_cast<const uint32_t*>(qs + n * D + d0);
+            qf[ks][1] = *reinterpret_cast<const uint32_t*>(qs + n * D + d0 + 8);
+          } else {
+            qf[ks][0] = 0u;
+            qf[ks][1] = 0u;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[ks][e] = 0.f;
+        }
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
       }
-      const int s = static_cast<int>(i % NS);
-      const uint32_t it = static_cast<uint32_t>(i / NS);
-      if (!mbar_wait(full_bar + 8 * s, it & 1u, p.err)) {
-        ok = false;
-        break;
-      }
-      const uint32_t sK = sbase + s * Lay::STAGE_BYTES;
-      const uint32_t sV = sK + Lay::KV_BYTES;
+      const uint32_t sK = sbase + s * Sh::STAGE_BYTES;
+      const uint32_t sV = sK + Sh::KV_BYTES;
       const int tok0 = warp * TOK_W;
 
       // S^T = K q^T over this warp's tokens
@@ -591,7 +838,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           const int row = tok0 + mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
           const int col = colb + (lane >> 4) * 8;
           uint32_t a0, a1, a2, a3;
-          ldsm_x4(sK + bx * Lay::BOX_BYTES + sw128_offset(row, col), a0, a1, a2, a3);
+          ldsm_x4(sK + bx * Sh::BOX_BYTES + sw128_offset(row, col), a0, a1, a2, a3);
           mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
         }
       }
@@ -643,7 +890,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           const int tok = tok0 + mt * 16 + (lane & 7) + (mi >> 1) * 8;
           const int col = colb + (mi & 1) * 8;
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_trans(sV + bx * Lay::BOX_BYTES + sw128_offset(tok, col), a0, a1, a2, a3);
+          ldsm_x4_trans(sV + bx * Sh::BOX_BYTES + sw128_offset(tok, col), a0, a1, a2, a3);
           mma_bf16_16816(o[dt], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
         }
       }
@@ -651,16 +898,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (lane == 0) mbar_arrive(empty_bar + 8 * s);
     }
   }
-  if (ok && cur_u >= 0) ok = flush(cur_u);
-  if (!ok || n_defer == 0) return;
-  // deferred merges: thread 0 wrote the list after the flushes' last barrier
-  if (!group_sync()) return;
-  __threadfence();
-  for (int k = 0; k < n_defer && k < kDeferMax; ++k) {
-    const int u = defer_u[k];
-    if (!merge_unit<D, 24>(p, u, defer_ns[k], fo, kConsumerWarps * 32, group_sync)) return;
-    if (threadIdx.x == 0) p.counters[u] = 0;  // ready for the next call
-  }
+  if (ok && cur_u >= 0) ok = flush_async(cur_u);
+  if (!p.merged) return;
+  final_merges(threadIdx.x);
 }
 
 // ------------------------------------------------------------------ fp32 path
@@ -714,7 +954,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
       __syncthreads();
       if (last_sh) {
         __threadfence();
-        merge_unit<D, 8>(p, u, ns, wts, kF32Threads, [] { __syncthreads(); return true; });
+        merge_unit<D, 8>(p, u, ns, wts, tid, kF32Threads, [] { __syncthreads(); return true; });
         if (tid == 0) p.counters[u] = 0;
       }
     }
@@ -878,12 +1118,15 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
 template <int D, int L>
 cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, const void* V,
                         int B, int Hkv, int P, std::string* why) {
-  using Lay = DecodeLayout<D, L>;
   CUtensorMap tmK, tmV;
   const uint64_t rows = static_cast<uint64_t>(B) * Hkv * p.T;
   if (!make_tmap_bf16_2d(&tmK, K, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tmV, V, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
-  const size_t sh = Lay::bytes(p.U);
+  const size_t sh = dec_layout(D, L, p.G, p.U).total;
+  if (sh > kMaxDynSmem) {
+    *why = "too many (batch, KV head) units for one decode launch: " + std::to_string(p.U);
+    return cudaErrorInvalidValue;
+  }
   auto fn = decode_bf16_kernel<D, L>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sh));
@@ -917,12 +1160,8 @@ int decode_default_parts(bool bf16, int D, int L, int num_sms) {
   return num_sms;  // one persistent CTA per SM
 }
 
-size_t decode_smem_bytes(bool bf16, int D, int L, int U) {
-  if (!bf16) return static_cast<size_t>(8 * D + 8 * 128 + 24 + kMergeWts + U + 1) * 4;
-  if (D == 128 && L == 128) return DecodeLayout<128, 128>::bytes(U);
-  if (D == 128 && L == 64) return DecodeLayout<128, 64>::bytes(U);
-  if (D == 64 && L == 128) return DecodeLayout<64, 128>::bytes(U);
-  return DecodeLayout<64, 64>::bytes(U);
+size_t decode_f32_smem_bytes(int D, int U) {
+  return static_cast<size_t>(8 * D + 8 * 128 + 24 + kMergeWts + U + 1) * 4;
 }
 
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,
@@ -962,7 +1201,7 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
   const int P = num_parts > 0 ? num_parts : decode_default_parts(bf16, D, L, l.num_sms);
   if (p.U == 0) return cudaSuccess;
   if (!bf16) {
-    const size_t sh = decode_smem_bytes(false, D, L, p.U);
+    const size_t sh = decode_f32_smem_bytes(D, p.U);
     cudaError_t e;
     if (D == 128) {
       e = cudaFuncSetAttribute(decode_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sh));

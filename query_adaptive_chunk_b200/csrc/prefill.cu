@@ -5,28 +5,29 @@
 // the tile for each of the G = 4 query heads of the group, stacked into 256
 // rows (head-major) that share the tile's chunk list.  The 256 rows are two
 // 128-row halves, each an M = 128 MMA operand.  Per selected chunk (64 keys):
-//   S_half = Q_half K^T      tcgen05.mma M=128 N=64 K=128, A/B from shared memory
-//   P_half = softmax rows    two warpgroups (one per half) read S from TMEM with
-//                            tcgen05.ld, keep the running max/sum per row, write
-//                            P back to TMEM as packed bf16
-//   O_half += P_half V       tcgen05.mma M=128 N=128 K=64, A = P from TMEM,
-//                            B = V from shared memory (MN-major)
-// The running max is lazily updated: O is rescaled (tcgen05.ld/st by the
-// owning softmax thread) only when a row max grows by more than 2^8.
-// Warp roles: warp 0 issues TMA (Q tile once per unit, K/V per chunk into a
-// 4-stage ring), warp 1 allocates TMEM and one of its threads issues every MMA
-// and tcgen05.commit, warps 4-7 and 8-11 are the softmax/epilogue warpgroups
-// of half 0 and half 1 (a warpgroup's warp w may touch TMEM lanes
-// 32*(w%4)..+31, so the four warps cover the 128 rows).  MMA order
-//   QK0(0) QK1(0) | PV0(j) QK0(j+1) PV1(j) QK1(j+1) | ...
-// lets one half's softmax run while the tensor core works on the other half.
-// A commit tracks every earlier MMA of the issuing thread, so "S_h(j+1) is
-// ready" also means "PV_h(j) has finished": the softmax may then overwrite P_h
-// and rescale O_h without a separate wait.
+//   S_half = Q_half K^T      tcgen05.mma M=128 N=64 K=128, A/B from shared memory,
+//                            D into one of two TMEM buffers per half
+//   P_half = softmax rows    one warpgroup per half reads S with tcgen05.ld,
+//                            keeps the running max/sum per row and writes P as
+//                            bf16 into shared memory (128-byte swizzled, K-major)
+//   O_half += P_half V       tcgen05.mma M=128 N=128 K=64, A = P, B = V (MN-major)
+// Double-buffered S lets QK^T of chunk j+1 run while the softmax works on
+// chunk j; the running max is lazily updated (O is rescaled in TMEM only when
+// a row max grows by more than 2^8).  A quarter of the exponentials are
+// computed on the FMA pipe (2^x = 2^rint(x) * cubic(x - rint(x))) so that the
+// special-function unit, which otherwise needs as many cycles per chunk as
+// the tensor core, stops being the bound.
+// Warp roles: warp 0 issues TMA (each half of the Q tile once per unit, K/V
+// per chunk into a 4-stage ring), warp 1 allocates TMEM and one of its
+// threads issues every MMA and tcgen05.commit, warps 4-7 and 8-11 are the
+// softmax/epilogue warpgroups of half 0 and half 1 (a warpgroup's warp w may
+// touch TMEM lanes 32*(w%4)..+31, so the four warps cover the 128 rows).
+// MMA issue order per chunk j:  QK0(j+1) PV0(j) QK1(j+1) PV1(j).
 // Every wait is a bounded mbarrier wait; the grid is persistent (one CTA per
 // SM, the whole 512-column TMEM), heaviest tiles first.
 #include <algorithm>
 
+#include "exp2_poly.h"
 #include "internal.h"
 
 namespace csa {
@@ -34,19 +35,21 @@ namespace {
 
 constexpr int kPfThreads = 384;
 constexpr int kNS = 4;                         // K/V stages
-constexpr int kQBytes = 256 * 128 * 2;         // 64 KB Q tile
+constexpr int kQHalfBytes = 128 * 128 * 2;     // 32 KB: one 128-row half of the Q tile
 constexpr int kKVBytes = 64 * 128 * 2;         // 16 KB per K (or V) chunk
 constexpr int kStageBytes = 2 * kKVBytes;
+constexpr int kPBytes = 128 * 64 * 2;          // 16 KB: P of one half
 constexpr int kQOff = 0;
-constexpr int kKVOff = kQBytes;
-constexpr int kBarOff = kKVOff + kNS * kStageBytes;
+constexpr int kKVOff = 2 * kQHalfBytes;
+constexpr int kPOff = kKVOff + kNS * kStageBytes;
+constexpr int kBarOff = kPOff + 2 * kPBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kEmuPeriod = 4;  // one pair of exponentials in kEmuPeriod on the FMA pipe
 
-// TMEM columns
-constexpr uint32_t kColS0 = 0, kColS1 = 64, kColP0 = 128, kColP1 = 160, kColO0 = 256,
-                   kColO1 = 384;
+// TMEM columns: S of half h, buffer b at 128 h + 64 b; O of half h at 256 + 128 h
+constexpr uint32_t kColO = 256;
 
 // instruction descriptors (kind::f16): D fp32, A/B bf16, M = 128
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (0u << 16) |
@@ -156,6 +159,35 @@ __device__ __forceinline__ int unit_chunk(const PrefillParams& p, int sel_row, i
   return c;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair, x <= 8, on the FMA and integer pipes (Cody-Waite range
+// reduction): j = rint(x) by the round-to-nearest of adding 1.5 * 2^23,
+// f = x - j in [-1/2, 1/2], 2^f by the minimax cubic of exp2_poly.h (relative
+// error < 1e-4), and 2^j added to the exponent field.  Inputs below -125
+// give 2^-125 (the result stays a normal number).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, magic);
+  const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(jf, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(f, make_float2(CSA_EXP2_C3, CSA_EXP2_C3), make_float2(CSA_EXP2_C2, CSA_EXP2_C2));
+  q = __ffma2_rn(q, f, make_float2(CSA_EXP2_C1, CSA_EXP2_C1));
+  q = __ffma2_rn(q, f, make_float2(CSA_EXP2_C0, CSA_EXP2_C0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -165,29 +197,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const uint32_t sQ = sb + kQOff;
   const uint32_t sKV = sb + kKVOff;
+  const uint32_t sP = sb + kPOff;
   const uint32_t bar = sb + kBarOff;
-  const uint32_t q_full = bar, q_empty = bar + 8;
-  const uint32_t kv_full = bar + 16, kv_empty = kv_full + 8 * kNS;
-  const uint32_t s_full = kv_empty + 8 * kNS;  // [2]
-  const uint32_t p_full = s_full + 16;         // [2]
-  const uint32_t o_full = p_full + 16;         // [2]
-  const uint32_t o_empty = o_full + 16;        // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * (2 + 2 * kNS + 8));
+  const uint32_t q_full = bar, q_empty = bar + 16;          // [2] each
+  const uint32_t kv_full = bar + 32, kv_empty = kv_full + 8 * kNS;
+  const uint32_t s_full = kv_empty + 8 * kNS;               // [half][buffer]
+  const uint32_t p_full = s_full + 32;                      // [2]
+  const uint32_t pv_done = p_full + 16;                     // [2]
+  const uint32_t drain = pv_done + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + (drain + 8 - bar));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(q_full + 8 * h, 1);
+      mbar_init(q_empty + 8 * h, 1);
+      mbar_init(s_full + 8 * (2 * h), 1);
+      mbar_init(s_full + 8 * (2 * h + 1), 1);
+      mbar_init(p_full + 8 * h, 128);
+      mbar_init(pv_done + 8 * h, 1);
+    }
     for (int s = 0; s < kNS; ++s) {
       mbar_init(kv_full + 8 * s, 1);
       mbar_init(kv_empty + 8 * s, 1);
     }
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(s_full + 8 * h, 1);
-      mbar_init(p_full + 8 * h, 128);
-      mbar_init(o_full + 8 * h, 1);
-      mbar_init(o_empty + 8 * h, 128);
-    }
+    mbar_init(drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -204,7 +238,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    uint32_t q_phase = 0, kv_it = 0;
+    uint32_t q_phase[2] = {0, 0}, kv_it = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       int b, h, t;
@@ -213,15 +247,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int n = unit_n(p, sel);
       if (n == 0) continue;
       if (lane == 0) {
-        if (!mbar_wait(q_empty, q_phase ^ 1u, p.err)) ok = false;
-        q_phase ^= 1u;
-        if (ok) {
-          mbar_arrive_expect_tx(q_full, kQBytes);
-          const int qrow = b * p.S + t * 64;
-          for (int g = 0; g < 4; ++g)
+        const int qrow = b * p.S + t * 64;
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          // a half is free once the last QK^T of the previous unit that reads it is done
+          if (!mbar_wait(q_empty + 8 * hf, q_phase[hf] ^ 1u, p.err)) ok = false;
+          q_phase[hf] ^= 1u;
+          if (!ok) break;
+          const uint32_t fb = q_full + 8 * hf;
+          mbar_arrive_expect_tx(fb, kQHalfBytes);
+          for (int gg = 0; gg < 2; ++gg)
             for (int dbx = 0; dbx < 2; ++dbx)
-              tma_load_2d(sQ + (g >> 1) * 32768 + dbx * 16384 + (g & 1) * 8192, &tmQ,
-                          (h * 4 + g) * 128 + dbx * 64, qrow, q_full);
+              tma_load_2d(sQ + hf * kQHalfBytes + dbx * 16384 + gg * 8192, &tmQ,
+                          (h * 4 + 2 * hf + gg) * 128 + dbx * 64, qrow, fb);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -264,12 +301,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      uint32_t q_phase = 0, kv_it = 0;
-      uint32_t p_phase[2] = {0, 0}, oe_phase[2] = {0, 0};
+      uint32_t q_phase[2] = {0, 0}, p_phase[2] = {0, 0}, s_cnt[2] = {0, 0}, kv_it = 0;
       bool ok = true;
       auto qk = [&](int half, uint32_t stage) {
-        const uint32_t d = tmem + (half ? kColS1 : kColS0);
-        const uint32_t qa = sQ + half * 32768;
+        const uint32_t buf = s_cnt[half] & 1u;
+        const uint32_t d = tmem + half * 128 + buf * 64;
+        const uint32_t qa = sQ + half * kQHalfBytes;
         const uint32_t kb = sKV + stage * kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -278,70 +315,60 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           umma_ss(d, smem_desc(qa + off_q, 16, 1024), smem_desc(kb + off_k, 16, 1024), kIdescQK,
                   kk > 0 ? 1u : 0u);
         }
+        umma_commit(s_full + 8 * (2 * half + buf));
+        ++s_cnt[half];
       };
       auto pv = [&](int half, uint32_t stage, bool acc) {
-        const uint32_t d = tmem + (half ? kColO1 : kColO0);
-        const uint32_t a = tmem + (half ? kColP1 : kColP0);
+        const uint32_t d = tmem + kColO + half * 128;
+        const uint32_t pa = sP + half * kPBytes;
         const uint32_t vb = sKV + stage * kStageBytes + kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ts(d, a + kk * 8, smem_desc(vb + kk * 2048, 8192, 1024), kIdescPV,
-                  (acc || kk > 0) ? 1u : 0u);
+          umma_ss(d, smem_desc(pa + kk * 32, 16, 1024), smem_desc(vb + kk * 2048, 8192, 1024),
+                  kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        umma_commit(pv_done + 8 * half);
       };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
         int b, h, t;
         unit_coords(p, w, b, h, t);
         const int n = unit_n(p, (b * p.Hkv + h) * p.n_tiles + t);
         if (n == 0) continue;
-        if (!mbar_wait(q_full, q_phase, p.err)) break;
-        q_phase ^= 1u;
-        uint32_t st = kv_it % kNS;
-        if (!mbar_wait(kv_full + 8 * st, (kv_it / kNS) & 1u, p.err)) break;
-        tc_fence_after();
-        qk(0, st);
-        umma_commit(s_full);
-        qk(1, st);
-        umma_commit(s_full + 8);
-        for (int j = 0; j < n; ++j) {
-          const uint32_t cur = kv_it % kNS;
-          const bool last = j + 1 == n;
-          // half 0
-          if (!mbar_wait(p_full, p_phase[0], p.err)) { ok = false; break; }
-          p_phase[0] ^= 1u;
-          if (j == 0) {
-            if (!mbar_wait(o_empty, oe_phase[0] ^ 1u, p.err)) { ok = false; break; }
-            oe_phase[0] ^= 1u;
-          }
+        const uint32_t st0 = kv_it % kNS;
+        if (!mbar_wait(kv_full + 8 * st0, (kv_it / kNS) & 1u, p.err)) break;
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          if (!mbar_wait(q_full + 8 * hf, q_phase[hf], p.err)) { ok = false; break; }
+          q_phase[hf] ^= 1u;
           tc_fence_after();
-          pv(0, cur, j > 0);
-          if (last) umma_commit(o_full);
-          uint32_t nxt = (kv_it + 1) % kNS;
+          qk(hf, st0);
+          if (n == 1) umma_commit(q_empty + 8 * hf);
+        }
+        for (int j = 0; j < n && ok; ++j) {
+          const uint32_t cur = kv_it % kNS, nxt = (kv_it + 1) % kNS;
+          const bool last = j + 1 == n;
           if (!last) {
             if (!mbar_wait(kv_full + 8 * nxt, ((kv_it + 1) / kNS) & 1u, p.err)) { ok = false; break; }
+          }
+          for (int hf = 0; hf < 2; ++hf) {
+            if (!last) {
+              // the buffer was last read by the softmax of chunk j - 1, whose
+              // P (p_full) has been waited for
+              tc_fence_after();
+              qk(hf, nxt);
+              if (j + 2 == n) umma_commit(q_empty + 8 * hf);
+            }
+            if (!mbar_wait(p_full + 8 * hf, p_phase[hf], p.err)) { ok = false; break; }
+            p_phase[hf] ^= 1u;
             tc_fence_after();
-            qk(0, nxt);
-            umma_commit(s_full);
+            pv(hf, cur, j > 0);
           }
-          // half 1
-          if (!mbar_wait(p_full + 8, p_phase[1], p.err)) { ok = false; break; }
-          p_phase[1] ^= 1u;
-          if (j == 0) {
-            if (!mbar_wait(o_empty + 8, oe_phase[1] ^ 1u, p.err)) { ok = false; break; }
-            oe_phase[1] ^= 1u;
-          }
-          tc_fence_after();
-          pv(1, cur, j > 0);
+          if (!ok) break;
           umma_commit(kv_empty + 8 * cur);
-          if (last) {
-            umma_commit(o_full + 8);
-            umma_commit(q_empty);
-          } else {
-            qk(1, nxt);
-            umma_commit(s_full + 8);
-          }
           ++kv_it;
         }
       }
+      // every MMA issued has finished before TMEM is released
+      umma_commit(drain);
+      mbar_wait(drain, 0u, p.err);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -349,14 +376,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int half = (warp - 4) >> 2;
     const int r = ((warp & 3) << 5) + lane;  // row within the half == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + (half ? kColS1 : kColS0);
-    const uint32_t tP = tmem + lane_base + (half ? kColP1 : kColP0);
-    const uint32_t tO = tmem + lane_base + (half ? kColO1 : kColO0);
-    const uint32_t my_s_full = s_full + 8 * half, my_p_full = p_full + 8 * half;
-    const uint32_t my_o_full = o_full + 8 * half, my_o_empty = o_empty + 8 * half;
+    const uint32_t tS = tmem + lane_base + half * 128;
+    const uint32_t tO = tmem + lane_base + kColO + half * 128;
+    uint8_t* prow = smem + kPOff + half * kPBytes + r * 128;
+    const uint32_t my_p_full = p_full + 8 * half, my_pv_done = pv_done + 8 * half;
     const int g = half * 2 + (r >> 6);  // query head within the group
     const int i = r & 63;               // row within the tile
-    uint32_t s_phase = 0, of_phase = 0;
+    const float sl = p.scale_log2;
+    uint32_t s_cnt = 0, pv_phase = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       int b, h, t;
@@ -369,32 +396,64 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // running max of the raw scores, sum of 2^((s - m) sl)
+      int c_next = unit_chunk(p, sel, 0);
       for (int j = 0; j < n; ++j) {
-        const int c = unit_chunk(p, sel, j);
-        if (!mbar_wait(my_s_full, s_phase, p.err)) { ok = false; break; }
-        s_phase ^= 1u;
+        const int c = c_next;
+        if (j + 1 < n) c_next = unit_chunk(p, sel, j + 1);
+        const uint32_t buf = s_cnt & 1u, sph = (s_cnt >> 1) & 1u;
+        ++s_cnt;
+        // wait results are made warp-uniform: the TMEM accesses below are
+        // warp-collective
+        if (!warp_wait(s_full + 8 * (2 * half + buf), sph, p.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         uint32_t sr[2][32];
-        tmem_ld32(tS, sr[0]);
-        tmem_ld32(tS + 32, sr[1]);
+        tmem_ld32(tS + buf * 64, sr[0]);
+        tmem_ld32(tS + buf * 64 + 32, sr[1]);
         tmem_wait_ld();
-        const int lim = qpos - c * 64;  // keys jj <= lim are visible
         float x[64];
-        float rmax = -INFINITY;
 #pragma unroll
-        for (int jj = 0; jj < 64; ++jj) {
-          const float v = __uint_as_float(sr[jj >> 5][jj & 31]) * p.scale_log2;
-          x[jj] = jj <= lim ? v : -INFINITY;
-          rmax = fmaxf(rmax, x[jj]);
+        for (int jj = 0; jj < 64; ++jj) x[jj] = __uint_as_float(sr[jj >> 5][jj & 31]);
+        // only a chunk reaching past the tile's first row needs the causal mask
+        const bool masked = c * 64 + 63 > t * 64;
+        if (masked) {
+          const int lim = qpos - c * 64;  // keys jj <= lim are visible
+#pragma unroll
+          for (int jj = 0; jj < 64; ++jj) x[jj] = jj <= lim ? x[jj] : -INFINITY;
         }
-        float mnew = fmaxf(m, rmax);
-        if (m == -INFINITY) {
-          m = mnew;  // first visible keys: nothing accumulated in O yet
-        } else if (mnew > m + kRescaleLog2) {
-          const float alpha = fast_exp2(m - mnew);
+        float mq[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          float v = fmax3(x[16 * a], x[16 * a + 1], x[16 * a + 2]);
+#pragma unroll
+          for (int k = 3; k < 15; k += 2) v = fmax3(v, x[16 * a + k], x[16 * a + k + 1]);
+          mq[a] = fmaxf(v, x[16 * a + 15]);
+        }
+        const float mnew = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmaxf(mq[3], m));
+        // P and O of this half are free once the previous chunk's PV is done
+        if (j > 0) {
+          if (!warp_wait(my_pv_done, pv_phase, p.err)) {
+            ok = false;
+            break;
+          }
+          pv_phase ^= 1u;
+          tc_fence_after();
+        }
+        // Lazy rescale: a row moves its max only when it grew by more than
+        // 2^8.  tcgen05.ld/st are warp-collective, so the warp rescales
+        // together when any of its rows needs it (the others by 1).
+        const bool grow = m != -INFINITY && (mnew - m) * sl > kRescaleLog2;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = fast_exp2((m - mnew) * sl);
           l *= alpha;
           m = mnew;
+        }
+        if (m == -INFINITY) m = mnew;  // first visible keys: nothing accumulated in O yet
+        if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
           for (int cc = 0; cc < 128; cc += 32) {
             uint32_t ov[32];
@@ -404,26 +463,54 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
             tmem_st32(tO + cc, ov);
           }
+          tmem_wait_st();
         }
-        const float mu = m == -INFINITY ? 0.f : m;
+        const float nm = m == -INFINITY ? 0.f : -m * sl;
+        const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(nm, nm);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
         uint32_t pk[32];
-        float ls = 0.f;
+        if (!masked) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = fast_exp2(x[2 * e] - mu), p1 = fast_exp2(x[2 * e + 1] - mu);
-          ls += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 32; ++e) {
+            const float2 xe = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sl2, nm2);
+            float2 pe;
+            if (e % kEmuPeriod == kEmuPeriod - 1) {
+              pe = exp2_fma2(xe);
+            } else {
+              pe.x = fast_exp2(xe.x);
+              pe.y = fast_exp2(xe.y);
+            }
+            acc[e & 3] = __fadd2_rn(acc[e & 3], pe);
+            pk[e] = pack_bf16x2(pe.x, pe.y);
+          }
+        } else {  // masked keys must give exactly 0: special-function unit only
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float2 xe = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sl2, nm2);
+            const float2 pe = make_float2(fast_exp2(xe.x), fast_exp2(xe.y));
+            acc[e & 3] = __fadd2_rn(acc[e & 3], pe);
+            pk[e] = pack_bf16x2(pe.x, pe.y);
+          }
         }
-        l += ls;
-        tmem_st32(tP, pk);
-        tmem_wait_st();
+        l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
+             (acc[3].x + acc[3].y);
+        // P row r -> shared memory, 16-byte chunk q at q ^ (r % 8) (128-byte swizzle)
+#pragma unroll
+        for (int q16 = 0; q16 < 8; ++q16)
+          *reinterpret_cast<uint4*>(prow + ((q16 ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * q16], pk[4 * q16 + 1], pk[4 * q16 + 2], pk[4 * q16 + 3]);
+        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(my_p_full);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 rows
-      if (!mbar_wait(my_o_full, of_phase, p.err)) { ok = false; break; }
-      of_phase ^= 1u;
+      // epilogue: O / l -> bf16 rows, once the unit's last PV is done
+      if (!warp_wait(my_pv_done, pv_phase, p.err)) {
+        ok = false;
+        break;
+      }
+      pv_phase ^= 1u;
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll 1
@@ -439,8 +526,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
+      // the next unit's first PV overwrites O: it is issued after this
+      // warpgroup's next p_full arrival, which follows these loads
       tc_fence_before();
-      mbar_arrive(my_o_empty);
     }
   }
   tc_fence_before();

@@ -124,3 +124,46 @@ def test_prefill_handbuilt_lists():
         want = np.stack([O.prefill_tile(to_np(Q[0, rows, h * G + gg]), to_np(K[0, h]), to_np(V[0, h]),
                                         s, 64, t * 64, D ** -0.5) for gg in range(G)])
         parity.assert_close(got, want, "bf16", f"handbuilt {(h, t)} {s}")
+
+
+def test_prefill_large_logits_rescale_path():
+    """Logits spread over hundreds of units (queries scaled by 8, one chunk
+    per KV head with keys scaled by 6): the running row max grows by more
+    than 2^8 within a tile, so O is rescaled in tensor memory, and many
+    exponentials sit near the bottom of the fp32 range."""
+    from query_adaptive_chunk_b200 import csa
+    B, S, Hq, Hkv, D = 1, 1024, 8, 2, 128
+    n_tiles = S // 64
+    g = torch.Generator(device="cuda")
+    g.manual_seed(9)
+    Q = (8 * torch.randn(B, S, Hq, D, generator=g, device="cuda")).bfloat16()
+    K = torch.randn(B, Hkv, S, D, generator=g, device="cuda")
+    K[:, :, 5 * 64:6 * 64] *= 6
+    K = K.bfloat16()
+    V = torch.randn(B, Hkv, S, D, generator=g, device="cuda").bfloat16()
+    rng = np.random.default_rng(3)
+    lists = {}
+    for h in range(Hkv):
+        for t in range(n_tiles):
+            s = set(rng.choice(t + 1, size=min(t + 1, 6), replace=False).tolist()) | {0, t}
+            if t > 5:
+                s |= {5}
+            lists[(h, t)] = sorted(s)
+    kmax = 9  # up to 6 random chunks + sink + the large-key chunk + diagonal
+    idx = torch.full((B * Hkv * n_tiles, kmax), -1, dtype=torch.int32)
+    cnt = torch.zeros(B * Hkv * n_tiles, dtype=torch.int32)
+    for (h, t), s in lists.items():
+        r = h * n_tiles + t
+        idx[r, :len(s)] = torch.tensor(s, dtype=torch.int32)
+        cnt[r] = len(s)
+    Og = torch.empty(B, S, Hq, D, device="cuda").bfloat16()
+    csa.csa_block_sparse_prefill(Q, K, V, idx.cuda(), cnt.cuda(), kmax, B, S, Hq, Hkv, D, 64, 64,
+                                 D ** -0.5, Og)
+    csa.csa_check_device_status()
+    G = Hq // Hkv
+    for (h, t), s in lists.items():
+        rows = slice(t * 64, (t + 1) * 64)
+        got = Og[0, rows, h * G:(h + 1) * G].permute(1, 0, 2).cpu().double().numpy()
+        want = np.stack([O.prefill_tile(to_np(Q[0, rows, h * G + gg]), to_np(K[0, h]), to_np(V[0, h]),
+                                        s, 64, t * 64, D ** -0.5) for gg in range(G)])
+        parity.assert_close(got, want, "bf16", f"large logits {(h, t)} {s}")
