@@ -326,9 +326,14 @@ def time_prefill(w, steps: int, warmup: int, flush):
     return {"select_ms": sel_ms, "attend_ms": att_ms, "blocks": blocks, "flops": flops}
 
 
-def oracle_decode_seconds(w, inp, max_seconds: float = 20.0, max_steps: int = 5):
+def oracle_decode_seconds(w, inp, max_seconds: float = 20.0, max_steps: int = 5, threads: int = 1):
     """The CPU oracle's per-step work (score + select + attention, summaries
-    precomputed) on this workload, single-threaded, a bounded number of steps."""
+    precomputed) on this workload, a bounded number of steps.  threads == 1:
+    single-threaded; threads > 1: the units of a step spread over that many
+    host threads (numpy releases the GIL inside its array kernels), each
+    single-threaded inside."""
+    import concurrent.futures as cf
+
     from threadpoolctl import threadpool_limits
 
     from oracle import csa_oracle as O
@@ -337,29 +342,42 @@ def oracle_decode_seconds(w, inp, max_seconds: float = 20.0, max_steps: int = 5)
     proj = inp.get("proj")
     projn = None if proj is None else OP.to_np(proj)
     units = synth.decode_units(w)
+
+    def unit_work(bh):
+        b, h = bh
+        qg = OP.to_np(q[b, h * w.G:(h + 1) * w.G])
+        if h in w.full_heads:
+            chunks = list(range(w.C))
+        else:
+            s = O.score_chunks(qg[None, None], summ[(b, h)][None, None], 1, projn)[0, 0, 0]
+            if w.select == "topp":
+                chunks, _, _ = O.select_topp(s, 1.0 / math.sqrt(w.D), w.p, w.budget,
+                                             w.n_sink, w.n_local)
+            else:
+                chunks, _ = O.select_topk(s, w.k_free, w.n_sink, w.n_local)
+        tok = O.chunk_tokens(chunks, w.L)
+        ti = torch.as_tensor(tok)
+        O.attend(qg, OP.to_np(K[b, h][ti]), OP.to_np(V[b, h][ti]),
+                 torch.arange(len(tok)).numpy(), w.scale)
+
     with threadpool_limits(1):
         summ = {u: OP.unit_summaries(K[u[0], u[1]], w.L, projn) for u in units
                 if u[1] not in w.full_heads}
         times = []
-        t_start = time.perf_counter()
-        while len(times) < max_steps and (time.perf_counter() - t_start) < max_seconds:
-            t0 = time.perf_counter()
-            for (b, h) in units:
-                qg = OP.to_np(q[b, h * w.G:(h + 1) * w.G])
-                if h in w.full_heads:
-                    chunks = list(range(w.C))
+        ex = cf.ThreadPoolExecutor(max_workers=threads) if threads > 1 else None
+        try:
+            t_start = time.perf_counter()
+            while len(times) < max_steps and (time.perf_counter() - t_start) < max_seconds:
+                t0 = time.perf_counter()
+                if ex is None:
+                    for u in units:
+                        unit_work(u)
                 else:
-                    s = O.score_chunks(qg[None, None], summ[(b, h)][None, None], 1, projn)[0, 0, 0]
-                    if w.select == "topp":
-                        chunks, _, _ = O.select_topp(s, 1.0 / math.sqrt(w.D), w.p, w.budget,
-                                                     w.n_sink, w.n_local)
-                    else:
-                        chunks, _ = O.select_topk(s, w.k_free, w.n_sink, w.n_local)
-                tok = O.chunk_tokens(chunks, w.L)
-                ti = torch.as_tensor(tok)
-                O.attend(qg, OP.to_np(K[b, h][ti]), OP.to_np(V[b, h][ti]),
-                         torch.arange(len(tok)).numpy(), w.scale)
-            times.append(time.perf_counter() - t0)
+                    list(ex.map(unit_work, units))
+                times.append(time.perf_counter() - t0)
+        finally:
+            if ex is not None:
+                ex.shutdown()
     return times
 
 
@@ -431,6 +449,13 @@ def run_ours(args):
         cpu = {"value": 1e6 * statistics.mean(t), "unit": "us/step", "cores": 1, "kind": "oracle",
                "sample": f"{len(t)} whole decode steps of {w.name} (all {w.B * w.Hkv} units), "
                          "summaries precomputed, numpy fp64 single-threaded"}
+        n_thr = min(os.cpu_count() or 1, w.B * w.Hkv)
+        if n_thr > 1:
+            tp = oracle_decode_seconds(w, r["inp"], max_seconds=10.0, max_steps=5, threads=n_thr)
+            cpu["parallel"] = {"value": 1e6 * statistics.mean(tp), "unit": "us/step",
+                               "cores": n_thr, "host_cores": os.cpu_count(),
+                               "sample": f"{len(tp)} whole steps, units spread over {n_thr} "
+                                         "host threads (one unit per thread)"}
     traffic = recorded_traffic(os.path.join(ROOT, "query_adaptive_chunk_b200", "csrc", "decode.cu"),
                                "decode_bf16_kernel<128,128>/" + w.name)
     if rank != 0:

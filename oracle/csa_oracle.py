@@ -155,6 +155,34 @@ def select_topk(scores: np.ndarray, k_free: int, n_sink: int, n_local: int,
     return sorted(F | set(chosen)), gap
 
 
+def score_chunks_per_head(q_group: np.ndarray, summ_unit: np.ndarray,
+                          proj: np.ndarray | None = None) -> np.ndarray:
+    """Relevance of every chunk for each query head of one unit, without the
+    group sum: S[g, c] = q~_g . summ[c] (SSA summary, "방법론": s = q^T k_gist,
+    evaluated per query head).  q_group [G, D]; summ_unit [C, Ds] -> [G, C]."""
+    q = np.asarray(q_group, dtype=np.float64)
+    if proj is not None:
+        q = q @ np.asarray(proj, dtype=np.float64)
+    return q @ np.asarray(summ_unit, dtype=np.float64).T
+
+
+def select_topk_union(scores_heads: np.ndarray, k_free: int, n_sink: int, n_local: int,
+                      n_valid: int | None = None) -> tuple[list, float]:
+    """Per-head top-k with the GQA union (SSA summary, glossary entry
+    "Grouped-Query Attention": every query head makes its own top-k choice and
+    the group loads the union of the chosen chunks once).
+
+    scores_heads [G, C]: each head's own top-k (forced set plus its k_free best
+    non-forced chunks, select_topk); the result is the ascending union over
+    the heads.  The returned gap is the smallest of the heads' boundary gaps."""
+    out, gap = set(), math.inf
+    for row in np.asarray(scores_heads, dtype=np.float64):
+        chunks, g = select_topk(row, k_free, n_sink, n_local, n_valid)
+        out.update(chunks)
+        gap = min(gap, g)
+    return sorted(out), gap
+
+
 def topp_probs(scores: np.ndarray, logit_scale: float) -> np.ndarray:
     """Chunk-level attention mass pi_c = softmax(S_c * logit_scale) over all
     chunks of the unit: the first-order chunk-mass estimate of the HiLS review

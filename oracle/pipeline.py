@@ -58,6 +58,10 @@ def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_lo
             summ = unit_summaries(K[b, h], L, projn)
             s = O.score_chunks(qg[None, None], summ[None, None], 1, projn)[0, 0, 0]
             chunks, gap = O.select_topk(s, k_free, n_sink, n_local)
+        elif select == "topk_union":
+            summ = unit_summaries(K[b, h], L, projn)
+            s = O.score_chunks_per_head(qg, summ, projn)
+            chunks, gap = O.select_topk_union(s, k_free, n_sink, n_local)
         elif select == "topp":
             summ = unit_summaries(K[b, h], L, projn)
             s = O.score_chunks(qg[None, None], summ[None, None], 1, projn)[0, 0, 0]

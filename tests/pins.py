@@ -189,6 +189,55 @@ def check_topk_invariants(seed=6, C=40, trials=20):
             assert min(s[chosen]) >= max(s[rest])
 
 
+def check_topk_union_golden():
+    for c in _golden("topk_union_cases.json")["cases"]:
+        got, _ = O.select_topk_union(np.array(c["scores"], dtype=np.float64), c["k_free"],
+                                     c["n_sink"], c["n_local"])
+        assert got == c["expect"], (c["why"], got)
+
+
+def check_topk_union_brute_force(seed=14, G=3, C=12, trials=40):
+    """Brute force on tiny inputs with many exact ties: a non-forced chunk is
+    in the union iff, for some head, fewer than k_free non-forced chunks beat
+    it (higher score, or equal score and lower index).  A single head gives
+    the unit top-k."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        s = rng.integers(-2, 3, size=(G, C)).astype(np.float64)
+        n_sink, n_local = int(rng.integers(0, 3)), int(rng.integers(0, 3))
+        k_free = int(rng.integers(0, C))
+        got, _ = O.select_topk_union(s, k_free, n_sink, n_local)
+        forced = set(range(min(n_sink, C))) | set(range(max(C - n_local, 0), C))
+        pool = [c for c in range(C) if c not in forced]
+        ref = set(forced)
+        for c in pool:
+            for g in range(G):
+                beaten_by = sum(1 for d in pool if s[g, d] > s[g, c] or (s[g, d] == s[g, c] and d < c))
+                if beaten_by < k_free:
+                    ref.add(c)
+                    break
+        assert got == sorted(ref), (got, sorted(ref))
+        one, _ = O.select_topk_union(s[:1], k_free, n_sink, n_local)
+        flat, _ = O.select_topk(s[0], k_free, n_sink, n_local)
+        assert one == flat
+
+
+def check_per_head_scores(seed=15):
+    """Per-head scores: a hand case, and their sum over the heads equals the
+    group-summed score of score_chunks (pinned by its own hand case)."""
+    q = np.array([[1.0, 0.0], [0.0, 2.0]])
+    summ = np.array([[3.0, 4.0], [1.0, -1.0], [0.5, 0.0]])
+    assert np.array_equal(O.score_chunks_per_head(q, summ), [[3.0, 1.0, 0.5], [8.0, -2.0, 0.0]])
+    rng = np.random.default_rng(seed)
+    G, D, C, R = 4, 16, 9, 8
+    q = rng.standard_normal((G, D))
+    summ = rng.standard_normal((C, R))
+    P = rng.standard_normal((D, R))
+    per = O.score_chunks_per_head(q, summ, P)
+    grp = O.score_chunks(q[None, None], summ[None, None], 1, P)[0, 0, 0]
+    assert np.allclose(per.sum(axis=0), grp, rtol=0, atol=1e-12)
+
+
 def check_topp_golden():
     for c in _golden("topp_cases.json")["cases"]:
         got, n_p, _ = O.select_topp(np.array(c["scores"], dtype=np.float64), c["logit_scale"],
@@ -354,6 +403,7 @@ ALL_CHECKS = [
     check_attention_vs_sdpa, check_dense_special_case, check_empty_attention,
     check_summary_closed_form, check_score_hand_case, check_projection_closed_form,
     check_tile_mean, check_topk_golden, check_topk_vs_torch_sort, check_topk_invariants,
+    check_topk_union_golden, check_topk_union_brute_force, check_per_head_scores,
     check_topp_golden, check_topp_invariants, check_hier_golden, check_hier_all_metas_is_flat,
     check_meta_linearity, check_merge_closed_form, check_partition,
     check_prefill_dense_causal, check_prefill_masked,

@@ -14,7 +14,8 @@ from oracle import csa_oracle as O
 _orig = {name: getattr(O, name) for name in
          ["attend", "select_topk", "select_topp", "score_chunks", "lse_merge",
           "causal_attend", "meta_summaries", "chunk_summaries", "select_hier",
-          "forced_set", "topp_probs", "decode_partition", "tile_mean_q"]}
+          "forced_set", "topp_probs", "decode_partition", "tile_mean_q",
+          "select_topk_union", "score_chunks_per_head"]}
 
 
 def attend_no_scale(q, K, V, tokens, scale):
@@ -153,6 +154,26 @@ def tile_mean_first_row(Q, tile_m):
     return Q[:, ::tile_m]
 
 
+def union_is_intersection(scores_heads, k_free, n_sink, n_local, n_valid=None):
+    sets = [set(_orig["select_topk"](row, k_free, n_sink, n_local, n_valid)[0])
+            for row in np.asarray(scores_heads, dtype=np.float64)]
+    return sorted(set.intersection(*sets)), math.inf
+
+
+def union_first_head_only(scores_heads, k_free, n_sink, n_local, n_valid=None):
+    return _orig["select_topk_union"](np.asarray(scores_heads)[:1], k_free, n_sink, n_local, n_valid)
+
+
+def union_of_group_sum(scores_heads, k_free, n_sink, n_local, n_valid=None):
+    s = np.asarray(scores_heads, dtype=np.float64).sum(axis=0, keepdims=True)
+    return _orig["select_topk_union"](s, k_free, n_sink, n_local, n_valid)
+
+
+def per_head_scores_group_summed(q_group, summ_unit, proj=None):
+    per = _orig["score_chunks_per_head"](q_group, summ_unit, proj)
+    return np.repeat(per.sum(axis=0, keepdims=True), per.shape[0], axis=0)
+
+
 MUTANTS = [
     ("attend", attend_no_scale),
     ("attend", attend_no_max_shift_wrong_lse),
@@ -176,6 +197,10 @@ MUTANTS = [
     ("select_hier", hier_meta_ties_high),
     ("decode_partition", partition_ceil),
     ("tile_mean_q", tile_mean_first_row),
+    ("select_topk_union", union_is_intersection),
+    ("select_topk_union", union_first_head_only),
+    ("select_topk_union", union_of_group_sum),
+    ("score_chunks_per_head", per_head_scores_group_summed),
 ]
 
 
