@@ -499,7 +499,7 @@ def run_ours(args):
 def other_workloads(args, flush, peaks):
     out = {}
     steps = max(5, args.steps // 2)
-    for w in (synth.TOPK_32K, synth.HIER_1M, synth.TINY_F32):
+    for w in (synth.TOPK_32K, synth.HIER_1M, synth.TINY_F32, synth.TOPK_UNION_32K):
         r = time_decode(w, steps, args.warmup, flush)
         us = 1000 * statistics.mean(r["step_ms"])
         dus = 1000 * statistics.mean(r["decode_ms"])

@@ -230,6 +230,22 @@ CSA_API csa_status csa_score_select_topk(const void* q, csa_dtype q_dtype, const
                                          int n_local, int32_t* idx, int32_t* count, int kmax,
                                          csa_stream stream);
 
+/* Per-head top-k with the GQA union (SSA summary, glossary entry
+ * "Grouped-Query Attention": each query head selects its own top-k chunks and
+ * the group loads the union of the selected chunks once, so the decode reads
+ * each KV chunk once per group).  Per unit (b, h): for each query head g of
+ * the group, S_g[c] = q~_g . summ[b, h, c] (q~ = P^T q_g with a projection);
+ * head g keeps its k_free best non-forced chunks by (score desc, index asc);
+ * the list is the ascending union over the heads plus the forced set (first
+ * n_sink and last n_local chunks).  Arguments, layouts, full-head handling
+ * and errors as csa_score_select_topk, except that kmax must be
+ * >= min(C, (Hq/Hkv) * k_free + n_sink + n_local). */
+CSA_API csa_status csa_score_select_topk_union(const void* q, csa_dtype q_dtype, const float* proj,
+                                               int R, const float* summ, int B, int Hq, int Hkv,
+                                               int D, int C, const uint8_t* head_full, int k_free,
+                                               int n_sink, int n_local, int32_t* idx,
+                                               int32_t* count, int kmax, csa_stream stream);
+
 /* Fused a1 + a3 (decode): csa_score_chunks then csa_select_topp in one CTA
  * per unit (bit-identical to the two calls); full heads as above (n_p_out 0). */
 CSA_API csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* proj, int R,
@@ -295,7 +311,8 @@ CSA_API csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K
 
 /* ---------------------------------------------------------------- a1-a6 in one call
  * A whole decode step: the selection (csa_score_select_topk,
- * csa_score_select_topp or csa_select_hier) followed by the merged split-K
+ * csa_score_select_topk_union, csa_score_select_topp or csa_select_hier,
+ * by `mode`) followed by the merged split-K
  * decode (csa_sparse_decode_merged), with the same results.  The decode is
  * launched with programmatic dependent launch and works in two phases: the
  * chunks of full-attention heads first, which do not depend on the
@@ -315,7 +332,8 @@ CSA_API csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K
 typedef enum csa_select_mode {
   CSA_SELECT_TOPK = 0,
   CSA_SELECT_TOPP = 1,
-  CSA_SELECT_HIER = 2
+  CSA_SELECT_HIER = 2,
+  CSA_SELECT_TOPK_UNION = 3 /* csa_score_select_topk_union */
 } csa_select_mode;
 
 typedef struct csa_decode_step_desc {

@@ -57,6 +57,8 @@ _SIGS = {
     "csa_decode_default_parts": (_i, [_i, _i, _i]),
     "csa_score_select_topk": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i, _i,
                                    _vp, _vp, _i, _vp]),
+    "csa_score_select_topk_union": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _i, _i,
+                                         _i, _vp, _vp, _i, _vp]),
     "csa_score_select_topp": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _f, _f, _i,
                                    _i, _i, _vp, _vp, _i, _vp, _vp]),
     "csa_decode_workspace_bytes": (_i64, [_i, _i, _i, _i, _i]),
@@ -191,6 +193,13 @@ def csa_score_select_topk(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full
                                      kmax, _s(stream)))
 
 
+def csa_score_select_topk_union(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full, k_free,
+                                n_sink, n_local, idx, count, kmax, stream=None):
+    _check(lib.csa_score_select_topk_union(_p(q), _dt(q_dtype), _p(proj), R, _p(summ), B, Hq, Hkv,
+                                           D, C, _p(head_full), k_free, n_sink, n_local, _p(idx),
+                                           _p(count), kmax, _s(stream)))
+
+
 def csa_score_select_topp(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full, logit_scale, p,
                           budget, n_sink, n_local, idx, count, kmax, n_p_out=None, stream=None):
     _check(lib.csa_score_select_topp(_p(q), _dt(q_dtype), _p(proj), R, _p(summ), B, Hq, Hkv, D, C,
@@ -224,7 +233,7 @@ def csa_sparse_decode_merged_noalloc(q, K, V, dtype, idx, count, kmax, head_full
                                                 _p(lse_out), _s(stream)))
 
 
-CSA_SELECT_TOPK, CSA_SELECT_TOPP, CSA_SELECT_HIER = 0, 1, 2
+CSA_SELECT_TOPK, CSA_SELECT_TOPP, CSA_SELECT_HIER, CSA_SELECT_TOPK_UNION = 0, 1, 2, 3
 
 
 class DecodeStepDesc(ctypes.Structure):

@@ -453,10 +453,12 @@ csa_status csa_sparse_decode_merged(const void* q, const void* K, const void* V,
   return finish(e, "merged sparse decode launch");
 }
 
-csa_status csa_score_select_topk(const void* q, csa_dtype q_dtype, const float* proj, int R,
-                                 const float* summ, int B, int Hq, int Hkv, int D, int C,
-                                 const uint8_t* head_full, int k_free, int n_sink, int n_local,
-                                 int32_t* idx, int32_t* count, int kmax, csa_stream stream) {
+namespace {
+csa_status score_select_topk_common(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                    const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                    const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                                    int32_t* idx, int32_t* count, int kmax, csa_stream stream,
+                                    bool per_head_union) {
   CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
   CSA_REQUIRE(kmax > 0, "kmax must be positive");
   CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && D > 0 && C >= 0 && k_free >= 0 && n_sink >= 0 &&
@@ -466,8 +468,14 @@ csa_status csa_score_select_topk(const void* q, csa_dtype q_dtype, const float* 
   CSA_SUPPORT(D <= 1024 && C <= 32768, "D <= 1024 and C <= 32768");
   const int Ds = proj ? R : D;
   CSA_SUPPORT(Ds == 16 || Ds == 32 || Ds == 64 || Ds == 128, "summary width must be 16, 32, 64 or 128");
-  const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(k_free) + n_sink + n_local);
-  CSA_REQUIRE(kmax >= need, "kmax < min(C, k_free + n_sink + n_local)");
+  if (per_head_union) {
+    const int64_t need = std::min<int64_t>(
+        C, static_cast<int64_t>(Hq / Hkv) * k_free + n_sink + n_local);
+    CSA_REQUIRE(kmax >= need, "kmax < min(C, (Hq/Hkv) * k_free + n_sink + n_local)");
+  } else {
+    const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(k_free) + n_sink + n_local);
+    CSA_REQUIRE(kmax >= need, "kmax < min(C, k_free + n_sink + n_local)");
+  }
   if (B == 0 || C == 0) return CSA_OK;
   CSA_TRY(check_ptr(q, "q"));
   CSA_TRY(check_ptr(proj, "proj", false));
@@ -478,8 +486,27 @@ csa_status csa_score_select_topk(const void* q, csa_dtype q_dtype, const float* 
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
   return finish(csa::launch_score_select_topk(l, q, q_dtype == CSA_BF16, proj, R, summ, B, Hq, Hkv, D,
-                                              C, head_full, k_free, n_sink, n_local, idx, count, kmax),
-                "score_select_topk launch");
+                                              C, head_full, k_free, n_sink, n_local, idx, count, kmax,
+                                              per_head_union),
+                per_head_union ? "score_select_topk_union launch" : "score_select_topk launch");
+}
+}  // namespace
+
+csa_status csa_score_select_topk(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                 const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                 const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                                 int32_t* idx, int32_t* count, int kmax, csa_stream stream) {
+  return score_select_topk_common(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full, k_free,
+                                  n_sink, n_local, idx, count, kmax, stream, false);
+}
+
+csa_status csa_score_select_topk_union(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                       const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                       const uint8_t* head_full, int k_free, int n_sink,
+                                       int n_local, int32_t* idx, int32_t* count, int kmax,
+                                       csa_stream stream) {
+  return score_select_topk_common(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full, k_free,
+                                  n_sink, n_local, idx, count, kmax, stream, true);
 }
 
 csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* proj, int R,
@@ -518,8 +545,10 @@ csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* 
 
 csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
   CSA_REQUIRE(d != nullptr, "descriptor is NULL");
-  CSA_REQUIRE(d->mode == CSA_SELECT_TOPK || d->mode == CSA_SELECT_TOPP || d->mode == CSA_SELECT_HIER,
-              "mode must be CSA_SELECT_TOPK, CSA_SELECT_TOPP or CSA_SELECT_HIER");
+  CSA_REQUIRE(d->mode == CSA_SELECT_TOPK || d->mode == CSA_SELECT_TOPP ||
+                  d->mode == CSA_SELECT_HIER || d->mode == CSA_SELECT_TOPK_UNION,
+              "mode must be CSA_SELECT_TOPK, CSA_SELECT_TOPP, CSA_SELECT_HIER or "
+              "CSA_SELECT_TOPK_UNION");
   CSA_REQUIRE(valid_dtype(d->out_dtype), "out_dtype");
   CSA_TRY(decode_shape_checks(CSA_BF16, d->kmax, d->B, d->Hq, d->Hkv, d->D, d->T, d->L, d->scale,
                               d->num_parts));
@@ -552,6 +581,10 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
     st = csa_score_select_topk(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
                                d->head_full, d->k_free, d->n_sink, d->n_local, d->idx, d->count,
                                d->kmax, stream);
+  else if (d->mode == CSA_SELECT_TOPK_UNION)
+    st = csa_score_select_topk_union(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
+                                     d->D, C, d->head_full, d->k_free, d->n_sink, d->n_local,
+                                     d->idx, d->count, d->kmax, stream);
   else if (d->mode == CSA_SELECT_TOPP)
     st = csa_score_select_topp(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
                                d->head_full, d->logit_scale, d->p, d->budget, d->n_sink, d->n_local,

@@ -416,16 +416,16 @@ __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
   float* st = reinterpret_cast<float*>(area);  // [G][ns][D]
-  const int n16 = G * ns * D4;
-  for (int e = tid; e < n16; e += nthr) {
-    const int c4 = e % D4, gs = e / D4, g = gs / ns, s = gs % ns;
-    cp_async16(smem_u32(st + static_cast<size_t>(gs) * D + c4 * 4),
-               p.o_part + ((row0 + g) * p.max_splits + s) * D + c4 * 4);
+  // thread tid copies float4 column tid % D4 of splits tid / D4, tid / D4 + nthr / D4, ...
+  const int c4 = tid % D4, s0 = tid / D4, ds = nthr / D4;
+  for (int g = 0; g < G; ++g) {
+    const float* src = p.o_part + (row0 + g) * p.max_splits * D + c4 * 4;
+    float* dst = st + static_cast<size_t>(g) * ns * D + c4 * 4;
+    for (int s = s0; s < ns; s += ds) cp_async16(smem_u32(dst + s * D), src + static_cast<int64_t>(s) * D);
   }
-  for (int e = tid; e < G * ns; e += nthr) {
-    const int g = e / ns, sl = e % ns;
-    wts[e] = __ldcg(p.lse_part + (row0 + g) * p.max_splits + sl);
-  }
+  for (int g = 0; g < G; ++g)
+    for (int sl = tid; sl < ns; sl += nthr)
+      wts[g * ns + sl] = __ldcg(p.lse_part + (row0 + g) * p.max_splits + sl);
   cp_async_wait_all();
   if (!sync()) return false;
   const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;

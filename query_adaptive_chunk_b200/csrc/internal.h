@@ -50,7 +50,8 @@ cudaError_t launch_select_hier(const Launch& l, const void* q, bool bf16, const 
 cudaError_t launch_score_select_topk(const Launch& l, const void* q, bool bf16, const float* proj,
                                      int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
                                      const uint8_t* head_full, int k_free, int n_sink, int n_local,
-                                     int32_t* idx, int32_t* count, int kmax);
+                                     int32_t* idx, int32_t* count, int kmax,
+                                     bool per_head_union = false);
 cudaError_t launch_score_select_topp(const Launch& l, const void* q, bool bf16, const float* proj,
                                      int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
                                      const uint8_t* head_full, float logit_scale, float p,

@@ -995,7 +995,11 @@ struct FusedSmem {
   float part[256];
 };
 
-template <int DS>
+// Fused score + top-k, one CTA per unit.  kUnion: per-head top-k with the
+// GQA union (each query head of the group scores the chunks with its own
+// query and marks its k_free best; the unit keeps the union, loaded once by
+// the decode); otherwise one top-k over the group-summed score.
+template <int DS, bool kUnion>
 __global__ void __launch_bounds__(kSelThreads) score_select_topk_kernel(
     const void* __restrict__ q, int q_bf16, const float* __restrict__ proj, int R,
     const float* __restrict__ summ, int Hq, int Hkv, int D, int C,
@@ -1018,15 +1022,31 @@ __global__ void __launch_bounds__(kSelThreads) score_select_topk_kernel(
     return;
   }
   const float* summ_u = summ + static_cast<int64_t>(u) * C * DS;
+  const int64_t head0 = static_cast<int64_t>(b) * Hq + h * G;
   float4 pre[kRowBatch];
   rows_load<DS>(summ_u, C, rows_first_base<DS>(), pre);  // in flight during the query phase
-  unit_query(q, q_bf16, static_cast<int64_t>(b) * Hq + h * G, G, D, proj, R, f.qs, f.qv, f.part);
+  unit_query(q, q_bf16, head0, kUnion ? 1 : G, D, proj, R, f.qs, f.qv, f.part);
   for (int c = threadIdx.x; c < C; c += blockDim.x) flags[c] = is_forced(c, C, n_sink, n_local);
   float mx_unused = 0.f, sum_unused = 0.f;
   summaries_to_keys<DS>(summ_u, C, proj ? f.qv : f.qs, keys, n_sink, n_local, true, mx_unused,
                         sum_unused, 0.f, pre);
   __syncthreads();
-  topk_from_keys(keys, flags, C, n_sink, n_local, k_free, row, count + u, kmax, s, exch, bs);
+  if (!kUnion) {
+    topk_from_keys(keys, flags, C, n_sink, n_local, k_free, row, count + u, kmax, s, exch, bs);
+    return;
+  }
+  const int n_cand = C - forced_count(C, n_sink, n_local);
+  for (int g = 0;;) {
+    mark_best(keys, flags, C, n_cand, k_free, exch, bs, s);  // sets flags; never clears them
+    __syncthreads();
+    if (++g == G) break;
+    rows_load<DS>(summ_u, C, rows_first_base<DS>(), pre);
+    unit_query(q, q_bf16, head0 + g, 1, D, proj, R, f.qs, f.qv, f.part);
+    summaries_to_keys<DS>(summ_u, C, proj ? f.qv : f.qs, keys, n_sink, n_local, true, mx_unused,
+                          sum_unused, 0.f, pre);
+    __syncthreads();
+  }
+  emit_ascending(flags, C, row, count + u, kmax, s);
 }
 
 template <int DS>
@@ -1129,18 +1149,30 @@ cudaError_t launch_select_hier(const Launch& l, const void* q, bool bf16, const 
 
 
 namespace {
+template <int DS, bool kUnion>
+cudaError_t fused_topk_kernel(const Launch& l, const void* q, bool bf16, const float* proj, int R,
+                              const float* summ, int U, int Hq, int Hkv, int D, int C,
+                              const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                              int32_t* idx, int32_t* count, int kmax) {
+  const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
+  cudaError_t e = set_smem(reinterpret_cast<const void*>(score_select_topk_kernel<DS, kUnion>), sh);
+  if (e != cudaSuccess) return e;
+  score_select_topk_kernel<DS, kUnion><<<U, kSelThreads, sh, l.stream>>>(
+      q, bf16 ? 1 : 0, proj, R, summ, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx,
+      count, kmax);
+  return cudaGetLastError();
+}
+
 template <int DS>
 cudaError_t fused_topk_ds(const Launch& l, const void* q, bool bf16, const float* proj, int R,
                           const float* summ, int U, int Hq, int Hkv, int D, int C,
                           const uint8_t* head_full, int k_free, int n_sink, int n_local,
-                          int32_t* idx, int32_t* count, int kmax) {
-  const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
-  cudaError_t e = set_smem(reinterpret_cast<const void*>(score_select_topk_kernel<DS>), sh);
-  if (e != cudaSuccess) return e;
-  score_select_topk_kernel<DS><<<U, kSelThreads, sh, l.stream>>>(
-      q, bf16 ? 1 : 0, proj, R, summ, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx,
-      count, kmax);
-  return cudaGetLastError();
+                          int32_t* idx, int32_t* count, int kmax, bool per_head_union) {
+  if (per_head_union)
+    return fused_topk_kernel<DS, true>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full,
+                                       k_free, n_sink, n_local, idx, count, kmax);
+  return fused_topk_kernel<DS, false>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full,
+                                      k_free, n_sink, n_local, idx, count, kmax);
 }
 
 template <int DS>
@@ -1163,14 +1195,15 @@ cudaError_t fused_topp_ds(const Launch& l, const void* q, bool bf16, const float
 cudaError_t launch_score_select_topk(const Launch& l, const void* q, bool bf16, const float* proj,
                                      int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
                                      const uint8_t* head_full, int k_free, int n_sink, int n_local,
-                                     int32_t* idx, int32_t* count, int kmax) {
+                                     int32_t* idx, int32_t* count, int kmax, bool per_head_union) {
   const int U = B * Hkv;
   if (U == 0) return cudaSuccess;
+  const bool pu = per_head_union;
   switch (proj ? R : D) {
-    case 16: return fused_topk_ds<16>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
-    case 32: return fused_topk_ds<32>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
-    case 64: return fused_topk_ds<64>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
-    case 128: return fused_topk_ds<128>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax);
+    case 16: return fused_topk_ds<16>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, pu);
+    case 32: return fused_topk_ds<32>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, pu);
+    case 64: return fused_topk_ds<64>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, pu);
+    case 128: return fused_topk_ds<128>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, pu);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -24,7 +24,7 @@ class SparseDecoder:
     """Query-adaptive chunk-sparse decode over a fixed KV cache.
 
     K, V: [B, Hkv, T, D] (bf16 or fp32, contiguous, on the current device).
-    select: "topk" | "topp" | "hier".  The summaries (and meta-summaries)
+    select: "topk" | "topk_union" (per-head top-k, GQA union) | "topp" | "hier".  The summaries (and meta-summaries)
     are computed once here, as part of building the cache.  With fused=True
     (default) a step is two launches: fused score+select (one CTA per unit)
     and the merged split-K decode; fused=False runs the separate calls
@@ -63,6 +63,8 @@ class SparseDecoder:
             hf[list(full_heads)] = 1
             self.head_full = hf.to(dev)
         extra = budget if select == "topp" else k_free
+        if select == "topk_union":
+            extra = (Hq // Hkv) * k_free
         self.kmax = min(self.C, extra + n_sink + n_local)
         self.scores = torch.zeros(B, Hkv, 1, self.C, dtype=torch.float32, device=dev)
         self.idx = torch.full((U, self.kmax), -1, dtype=torch.int32, device=dev)
@@ -84,7 +86,7 @@ class SparseDecoder:
         self.desc = None
         if fused and self.dtype == csa.CSA_BF16:
             mode = {"topk": csa.CSA_SELECT_TOPK, "topp": csa.CSA_SELECT_TOPP,
-                    "hier": csa.CSA_SELECT_HIER}[select]
+                    "hier": csa.CSA_SELECT_HIER, "topk_union": csa.CSA_SELECT_TOPK_UNION}[select]
             self.desc = csa.decode_step_desc(
                 K=K, V=V, B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, L=L, scale=self.scale,
                 head_full=self.head_full, mode=mode, summ=self.summ, proj=proj, R=self.R,
@@ -108,6 +110,12 @@ class SparseDecoder:
             csa.csa_score_select_topk(q, qd, self.proj, self.R, self.summ, B, Hq, Hkv, D, C,
                                       self.head_full, self.k_free, self.n_sink, self.n_local,
                                       self.idx, self.count, self.kmax, stream=stream)
+            return
+        if self.select == "topk_union":  # one call: per-head scores never leave the SM
+            csa.csa_score_select_topk_union(q, qd, self.proj, self.R, self.summ, B, Hq, Hkv, D, C,
+                                            self.head_full, self.k_free, self.n_sink,
+                                            self.n_local, self.idx, self.count, self.kmax,
+                                            stream=stream)
             return
         if self.fused and self.select == "topp":
             csa.csa_score_select_topp(q, qd, self.proj, self.R, self.summ, B, Hq, Hkv, D, C,

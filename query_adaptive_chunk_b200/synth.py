@@ -52,7 +52,7 @@ class DecodeWorkload:
     T: int
     L: int
     dtype: str  # "f32" or "bf16"
-    select: str  # "topk", "topp" or "hier"
+    select: str  # "topk", "topk_union", "topp" or "hier"
     n_sink: int
     n_local: int
     k_free: int = 0  # top-k / hierarchical: chunks picked besides the forced ones
@@ -78,6 +78,8 @@ class DecodeWorkload:
     def kmax(self) -> int:
         """Width of one unit's index row: an upper bound on the set size."""
         extra = self.budget if self.select == "topp" else self.k_free
+        if self.select == "topk_union":  # one k_free per query head
+            extra = self.G * self.k_free
         return min(self.C, extra + self.n_sink + self.n_local)
 
     @property
@@ -152,7 +154,12 @@ PREFILL_32K = PrefillWorkload(
     name="block_sparse_prefill_bf16_seq32k", seed=5, B=1, S=32768, Hq=32, Hkv=8, D=128,
     tile_m=64, L=64, k_free=16)
 
-DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M)
+# Per-head top-k with the GQA union on the 32K shapes: each of the 4 query
+# heads of a group keeps its own 29 best chunks, the group reads the union.
+TOPK_UNION_32K = dataclasses.replace(TOPK_32K, name="topk_union_decode_bf16_ctx32k", seed=6,
+                                     select="topk_union")
+
+DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M, TOPK_UNION_32K)
 ALL_WORKLOADS = DECODE_WORKLOADS + (PREFILL_32K,)
 
 

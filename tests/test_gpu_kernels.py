@@ -539,3 +539,65 @@ def test_merged_decode_mixed_heads(csa):
     rng = np.random.default_rng(7)
     sets = [sorted(rng.choice(C, size=20, replace=False).tolist()) for _ in range(B * Hkv)]
     _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, full=(0, 1))
+
+
+# ---------------------------------------------------------------- per-head top-k, GQA union
+
+def _union_from_scores(csa, scores, k_free, n_sink, n_local):
+    """Run csa_score_select_topk_union on one unit whose per-head scores are
+    exactly `scores` [G][C]: one-hot summaries (chunk c = unit vector c) and
+    head g's query = its score row, so q_g . summ_c = scores[g][c]."""
+    G, C = len(scores), len(scores[0])
+    D = 64
+    q = torch.zeros(1, G, D, device="cuda")
+    q[0, :, :C] = torch.tensor(scores, dtype=torch.float32, device="cuda")
+    summ = torch.zeros(1, 1, C, D, device="cuda")
+    summ[0, 0, torch.arange(C), torch.arange(C)] = 1.0
+    kmax = min(C, G * k_free + n_sink + n_local)
+    idx = torch.full((1, max(kmax, 1)), 777, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa.csa_score_select_topk_union(q, torch.float32, None, 0, summ, 1, G, 1, D, C, None, k_free,
+                                    n_sink, n_local, idx, cnt, max(kmax, 1))
+    csa.csa_check_device_status()
+    return parity.gpu_sets(idx, cnt)[0]
+
+
+def test_select_topk_union_golden(csa):
+    for c in pins_golden("topk_union_cases.json"):
+        got = _union_from_scores(csa, c["scores"], c["k_free"], c["n_sink"], c["n_local"])
+        assert got == c["expect"], c["why"]
+
+
+def test_select_topk_union_random_ties(csa):
+    """Integer scores (many exact ties) through the kernel against the oracle."""
+    rng = np.random.default_rng(21)
+    for trial in range(12):
+        G = int(rng.choice([1, 2, 4, 8]))
+        C = int(rng.integers(3, 65))
+        s = rng.integers(-3, 4, size=(G, C)).astype(np.float64)
+        k_free, n_sink, n_local = int(rng.integers(0, C)), int(rng.integers(0, 3)), int(rng.integers(0, 3))
+        got = _union_from_scores(csa, s.tolist(), k_free, n_sink, n_local)
+        ref, _ = O.select_topk_union(s, k_free, n_sink, n_local)
+        assert got == ref, (trial, G, C, k_free)
+
+
+def test_select_topk_union_single_head_equals_topk(csa):
+    """G = 1: the union kernel and the fused top-k give the same lists."""
+    B, Hkv, D, C = 2, 3, 128, 777
+    q = _randn((B, Hkv, D), 40, torch.bfloat16)
+    summ = _randn((B, Hkv, C, D), 41) * 0.3
+    kmax = 24 + 3
+    outs = []
+    for fn in (csa.csa_score_select_topk, csa.csa_score_select_topk_union):
+        idx = torch.full((B * Hkv, kmax), 5, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(B * Hkv, dtype=torch.int32, device="cuda")
+        fn(q, q.dtype, None, 0, summ, B, Hkv, Hkv, D, C, None, 24, 1, 2, idx, cnt, kmax)
+        outs.append(parity.gpu_sets(idx, cnt))
+    assert outs[0] == outs[1]
+
+
+def test_select_topk_union_kmax_too_small_rejected(csa):
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_score_select_topk_union(None, torch.bfloat16, None, 0, None, 1, 8, 2, 128, 512,
+                                        None, 10, 1, 1, None, None, 20)
+    assert ei.value.status == 1 and "kmax" in str(ei.value)

@@ -128,3 +128,20 @@ def test_hier_decode_full_heads_one_call_step():
     w = dataclasses.replace(synth.HIER_1M.scaled(T=65536, planted=4), name="hier_mixed_step",
                             full_heads=(2,))
     run_and_check(w)
+
+
+def test_topk_union_decode_reduced():
+    """Per-head top-k with the GQA union (each query head's own top-k, the
+    group reads the union once)."""
+    run_and_check(synth.TOPK_UNION_32K.scaled(B=2, T=8192))
+
+
+def test_topk_union_decode_full_size():
+    run_and_check(synth.TOPK_UNION_32K)
+
+
+def test_topk_union_with_projection_and_full_head():
+    import dataclasses
+    w = dataclasses.replace(synth.TOPK_UNION_32K.scaled(B=1, T=16384, planted=4),
+                            name="topk_union_proj_mixed", proj_rank=16, full_heads=(3,))
+    run_and_check(w)
