@@ -18,11 +18,12 @@
 // special-function unit, which otherwise needs as many cycles per chunk as
 // the tensor core, stops being the bound.
 // Warp roles: warp 0 issues TMA (each half of the Q tile once per unit, K/V
-// per chunk into a 4-stage ring), warp 1 allocates TMEM and one of its
-// threads issues every MMA and tcgen05.commit, warps 4-7 and 8-11 are the
-// softmax/epilogue warpgroups of half 0 and half 1 (a warpgroup's warp w may
-// touch TMEM lanes 32*(w%4)..+31, so the four warps cover the 128 rows).
-// MMA issue order per chunk j:  QK0(j+1) PV0(j) QK1(j+1) PV1(j).
+// per chunk into a 4-stage ring), warp 1 allocates TMEM, one thread of warp
+// 1 issues the MMAs of half 0 and one thread of warp 2 those of half 1 (in
+// the order QK(j+1) PV(j) per chunk j, so that neither half's chain waits
+// on the other's softmax), warps 4-7 and 8-11 are the softmax/epilogue
+// warpgroups of half 0 and half 1 (a warpgroup's warp w may touch TMEM
+// lanes 32*(w%4)..+31, so the four warps cover the 128 rows).
 // Every wait is a bounded mbarrier wait; the grid is persistent (one CTA per
 // SM, the whole 512-column TMEM), heaviest tiles first.
 #include <algorithm>
@@ -204,8 +205,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t s_full = kv_empty + 8 * kNS;               // [half][buffer]
   const uint32_t p_full = s_full + 32;                      // [2]
   const uint32_t pv_done = p_full + 16;                     // [2]
-  const uint32_t drain = pv_done + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + (drain + 8 - bar));
+  const uint32_t drain = pv_done + 16;                      // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + (drain + 16 - bar));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -219,9 +220,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int s = 0; s < kNS; ++s) {
       mbar_init(kv_full + 8 * s, 1);
-      mbar_init(kv_empty + 8 * s, 1);
+      mbar_init(kv_empty + 8 * s, 2);  // released by both halves' MMA issuers
     }
     mbar_init(drain, 1);
+    mbar_init(drain + 8, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -298,15 +300,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (uint32_t i = first; i < kv_it; ++i)
         mbar_wait(kv_full + 8 * (i % kNS), (i / kNS) & 1u, p.err);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ---------------------------------------------------------------- MMA issuers
+    // One thread per 128-row half (warp 1: half 0, warp 2: half 1), so each
+    // half's QK^T -> softmax -> PV chain runs at its own pace.
+    const int hf = warp - 1;
     if (lane == 0) {
-      uint32_t q_phase[2] = {0, 0}, p_phase[2] = {0, 0}, s_cnt[2] = {0, 0}, kv_it = 0;
+      uint32_t q_phase = 0, p_phase = 0, s_cnt = 0, kv_it = 0;
       bool ok = true;
-      auto qk = [&](int half, uint32_t stage) {
-        const uint32_t buf = s_cnt[half] & 1u;
-        const uint32_t d = tmem + half * 128 + buf * 64;
-        const uint32_t qa = sQ + half * kQHalfBytes;
+      const uint32_t qa = sQ + hf * kQHalfBytes;
+      auto qk = [&](uint32_t stage) {
+        const uint32_t buf = s_cnt & 1u;
+        const uint32_t d = tmem + hf * 128 + buf * 64;
         const uint32_t kb = sKV + stage * kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -315,18 +320,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           umma_ss(d, smem_desc(qa + off_q, 16, 1024), smem_desc(kb + off_k, 16, 1024), kIdescQK,
                   kk > 0 ? 1u : 0u);
         }
-        umma_commit(s_full + 8 * (2 * half + buf));
-        ++s_cnt[half];
+        umma_commit(s_full + 8 * (2 * hf + buf));
+        ++s_cnt;
       };
-      auto pv = [&](int half, uint32_t stage, bool acc) {
-        const uint32_t d = tmem + kColO + half * 128;
-        const uint32_t pa = sP + half * kPBytes;
+      auto pv = [&](uint32_t stage, bool acc) {
+        const uint32_t d = tmem + kColO + hf * 128;
+        const uint32_t pa = sP + hf * kPBytes;
         const uint32_t vb = sKV + stage * kStageBytes + kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_ss(d, smem_desc(pa + kk * 32, 16, 1024), smem_desc(vb + kk * 2048, 8192, 1024),
                   kIdescPV, (acc || kk > 0) ? 1u : 0u);
-        umma_commit(pv_done + 8 * half);
+        umma_commit(pv_done + 8 * hf);
       };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
         int b, h, t;
@@ -335,40 +340,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (n == 0) continue;
         const uint32_t st0 = kv_it % kNS;
         if (!mbar_wait(kv_full + 8 * st0, (kv_it / kNS) & 1u, p.err)) break;
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          if (!mbar_wait(q_full + 8 * hf, q_phase[hf], p.err)) { ok = false; break; }
-          q_phase[hf] ^= 1u;
-          tc_fence_after();
-          qk(hf, st0);
-          if (n == 1) umma_commit(q_empty + 8 * hf);
-        }
-        for (int j = 0; j < n && ok; ++j) {
+        if (!mbar_wait(q_full + 8 * hf, q_phase, p.err)) break;
+        q_phase ^= 1u;
+        tc_fence_after();
+        qk(st0);
+        if (n == 1) umma_commit(q_empty + 8 * hf);
+        for (int j = 0; j < n; ++j) {
           const uint32_t cur = kv_it % kNS, nxt = (kv_it + 1) % kNS;
-          const bool last = j + 1 == n;
-          if (!last) {
+          if (j + 1 < n) {
+            // the buffer was last read by the softmax of chunk j - 1, whose P
+            // (p_full) has been waited for
             if (!mbar_wait(kv_full + 8 * nxt, ((kv_it + 1) / kNS) & 1u, p.err)) { ok = false; break; }
-          }
-          for (int hf = 0; hf < 2; ++hf) {
-            if (!last) {
-              // the buffer was last read by the softmax of chunk j - 1, whose
-              // P (p_full) has been waited for
-              tc_fence_after();
-              qk(hf, nxt);
-              if (j + 2 == n) umma_commit(q_empty + 8 * hf);
-            }
-            if (!mbar_wait(p_full + 8 * hf, p_phase[hf], p.err)) { ok = false; break; }
-            p_phase[hf] ^= 1u;
             tc_fence_after();
-            pv(hf, cur, j > 0);
+            qk(nxt);
+            if (j + 2 == n) umma_commit(q_empty + 8 * hf);
           }
-          if (!ok) break;
-          umma_commit(kv_empty + 8 * cur);
+          if (!mbar_wait(p_full + 8 * hf, p_phase, p.err)) { ok = false; break; }
+          p_phase ^= 1u;
+          tc_fence_after();
+          pv(cur, j > 0);
+          umma_commit(kv_empty + 8 * cur);  // the stage is free once both halves' reads are done
           ++kv_it;
         }
       }
-      // every MMA issued has finished before TMEM is released
-      umma_commit(drain);
-      mbar_wait(drain, 0u, p.err);
+      // every MMA this thread issued has finished before TMEM is released
+      umma_commit(drain + 8 * hf);
+      mbar_wait(drain + 8 * hf, 0u, p.err);
     }
     __syncwarp();
   } else if (warp >= 4) {
