@@ -334,7 +334,7 @@ __host__ __device__ inline DecLayout dec_layout(int D, int L, int G, int U, int 
   y.q_off = ns * stage_bytes;
   y.fb_off = y.q_off + ns * kQSlotHeads * D * 2;
   y.bar_off = y.fb_off + nf * y.fb_bytes;
-  y.prefix_off = y.bar_off + (2 * ns + 6) * 8;  // full[ns], empty[ns], fb_full[2], fb_empty[2], phase, end
+  y.prefix_off = y.bar_off + (2 * ns + 8) * 8;  // full[ns], empty[ns], fb_full[2], fb_empty[2], phase, end, merge, spare
   y.total = 1024 + static_cast<size_t>(y.prefix_off) + 2 * static_cast<size_t>(U + 1) * 4;
   return y;
 }
@@ -352,12 +352,8 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Merge of unit u by one warp, straight from global memory (rarely used:
@@ -400,69 +396,79 @@ __device__ void merge_unit_warp(const DecodeParams& p, int u, int ns) {
   }
 }
 
-// Merge of unit u with its partials first copied into shared memory (one
-// round trip to L2 for all of them), by `nthr` threads numbered `tid`.
-// `area` (area_bytes, the idle K/V stage ring) holds the partials and, in
-// its last 8 KB, the split weights.  Falls back to merge_unit when the
-// partials do not fit.
+// Merge of unit u with its partials first copied into shared memory: one
+// bulk copy per head (the head's ns partial rows are contiguous), so the
+// partials cross from L2 in a single round trip.  `area` (area_bytes, the
+// idle K/V stage ring) receives them in all but its last 8 KB, which hold
+// the split weights; `bar` is an mbarrier of this CTA (count 1) and
+// `n_bulk` counts the copies that completed it so far.  Then each warp
+// takes whole heads: the head's lse and split weights stay in the warp
+// (shuffles and a per-warp slice of the weights), and the lanes accumulate
+// float4 columns, with no block barrier in between.  `nthr` (<= 256)
+// threads numbered `tid` by whole warps take part; `sync` is a barrier over
+// them (bounded).  Falls back to merge_unit when the partials do not fit.
 template <int D, typename Sync>
 __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area, int area_bytes,
-                             int tid, int nthr, Sync sync) {
+                             uint32_t bar, uint32_t& n_bulk, int tid, int nthr, Sync sync) {
   constexpr int D4 = D / 4;
   const int G = p.G;
-  float* wts = reinterpret_cast<float*>(area + area_bytes - 8192);
-  if (static_cast<size_t>(G) * ns * D * 4 > static_cast<size_t>(area_bytes) - 8192)
-    return merge_unit<D, 8>(p, u, ns, wts, tid, nthr, sync);
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
+  const uint32_t head_bytes = static_cast<uint32_t>(ns) * D * 4;
+  float* wts = reinterpret_cast<float*>(area + area_bytes - 8192);
+  if (static_cast<size_t>(G) * head_bytes > static_cast<size_t>(area_bytes) - 8192 || ns > 256)
+    return merge_unit<D, 8>(p, u, ns, wts, tid, nthr, sync);
+  const uint32_t phase = n_bulk & 1u;
+  ++n_bulk;
   float* st = reinterpret_cast<float*>(area);  // [G][ns][D]
-  // thread tid copies float4 column tid % D4 of splits tid / D4, tid / D4 + nthr / D4, ...
-  const int c4 = tid % D4, s0 = tid / D4, ds = nthr / D4;
-  for (int g = 0; g < G; ++g) {
-    const float* src = p.o_part + (row0 + g) * p.max_splits * D + c4 * 4;
-    float* dst = st + static_cast<size_t>(g) * ns * D + c4 * 4;
-    for (int s = s0; s < ns; s += ds) cp_async16(smem_u32(dst + s * D), src + static_cast<int64_t>(s) * D);
+  if (tid == 0) {
+    fence_proxy_async_global();  // partials written by other CTAs, read through the async proxy
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(G) * head_bytes);
+    for (int g = 0; g < G; ++g)
+      bulk_load(smem_u32(st + static_cast<size_t>(g) * ns * D),
+                p.o_part + (row0 + g) * p.max_splits * D, head_bytes, bar);
   }
-  for (int g = 0; g < G; ++g)
-    for (int sl = tid; sl < ns; sl += nthr)
-      wts[g * ns + sl] = __ldcg(p.lse_part + (row0 + g) * p.max_splits + sl);
-  cp_async_wait_all();
-  if (!sync()) return false;
   const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
-  for (int g = warp; g < G; g += nw) {
+  float* ww = wts + warp * 256;  // this warp's split weights
+  bool ok = warp_wait(bar, phase, p.err);
+  for (int g = warp; g < G && ok; g += nw) {
+    const float* lsp = p.lse_part + (row0 + g) * p.max_splits;
     float mx = -INFINITY;
-    for (int sl = lane; sl < ns; sl += 32) mx = fmaxf(mx, wts[g * ns + sl]);
+    for (int sl = lane; sl < ns; sl += 32) {
+      const float v = __ldcg(lsp + sl);
+      ww[sl] = v;
+      mx = fmaxf(mx, v);
+    }
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
     float sum = 0.f;
-    for (int sl = lane; sl < ns; sl += 32) sum += expf(wts[g * ns + sl] - mx);
+    for (int sl = lane; sl < ns; sl += 32) sum += expf(ww[sl] - mx);
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
     const float lse = mx + logf(sum);
+    for (int sl = lane; sl < ns; sl += 32) ww[sl] = expf(ww[sl] - lse);
     __syncwarp();
-    for (int sl = lane; sl < ns; sl += 32) wts[g * ns + sl] = expf(wts[g * ns + sl] - lse);
     if (lane == 0 && p.lse_out) p.lse_out[row0 + g] = lse;
-  }
-  if (!sync()) return false;
-  for (int e = tid; e < G * D4; e += nthr) {
-    const int g = e / D4, c4 = e % D4;
-    const float* src = st + static_cast<size_t>(g) * ns * D + c4 * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < ns; ++s) {
-      const float wk = wts[g * ns + s];
-      const float4 x = *reinterpret_cast<const float4*>(src + static_cast<size_t>(s) * D);
-      acc.x += wk * x.x;
-      acc.y += wk * x.y;
-      acc.z += wk * x.z;
-      acc.w += wk * x.w;
+    for (int c4 = lane; c4 < D4; c4 += 32) {
+      const float* src = st + static_cast<size_t>(g) * ns * D + c4 * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sl = 0; sl < ns; ++sl) {
+        const float wk = ww[sl];
+        const float4 x = *reinterpret_cast<const float4*>(src + static_cast<size_t>(sl) * D);
+        acc.x += wk * x.x;
+        acc.y += wk * x.y;
+        acc.z += wk * x.z;
+        acc.w += wk * x.w;
+      }
+      const int64_t o = (row0 + g) * D + c4 * 4;
+      store_out(p, o, acc.x);
+      store_out(p, o + 1, acc.y);
+      store_out(p, o + 2, acc.z);
+      store_out(p, o + 3, acc.w);
     }
-    const int64_t o = (row0 + g) * D + c4 * 4;
-    store_out(p, o, acc.x);
-    store_out(p, o + 1, acc.y);
-    store_out(p, o + 2, acc.z);
-    store_out(p, o + 3, acc.w);
+    __syncwarp();
   }
-  return sync();
+  return sync() && ok;  // the area is free again
 }
 
 template <int D, int L>
@@ -487,6 +493,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const uint32_t fb_empty = fb_full + 16;       // [2]
   const uint32_t phase_bar = fb_empty + 16;
   const uint32_t end_bar = phase_bar + 8;
+  const uint32_t merge_bar = end_bar + 8;  // completed by the final merges' bulk copies
   int* prefix = reinterpret_cast<int*>(smem + Y.prefix_off);  // [U+1]
   int* prefix2 = prefix + (p.U + 1);  // phase 2 (sparse units), built by the producer
   __shared__ int scan_sh[33];
@@ -505,6 +512,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     mbar_init(phase_bar, 1);
     mbar_init(end_bar, (kConsumerWarps + 1) * 32);
+    mbar_init(merge_bar, 1);
     n_defer_sh = 0;
     fence_barrier_init();
   }
@@ -604,9 +612,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const int nd = n_defer_sh;
     if (nd == 0) return;
     __threadfence();
+    uint32_t n_bulk = 0;
     for (int k = 0; k < nd; ++k) {
       const int u = defer_u[k];
-      if (!merge_staged<D>(p, u, defer_ns[k], smem, NS * Sh::STAGE_BYTES, tid,
+      if (!merge_staged<D>(p, u, defer_ns[k], smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk, tid,
                            (kConsumerWarps + 1) * 32, end_sync))
         return;
       if (tid == 0) p.counters[u] = 0;  // ready for the next call
