@@ -5,20 +5,21 @@
 // the tile for each of the G = 4 query heads of the group, stacked into 256
 // rows (head-major) that share the tile's chunk list.  The 256 rows are two
 // 128-row halves, each an M = 128 MMA operand.  Per selected chunk (64 keys):
-//   S_half = Q_half K^T      tcgen05.mma M=128 N=64 K=128, A/B from shared memory,
-//                            D into one of two TMEM buffers per half
+//   S_half = Q_half K^T      tcgen05.mma M=128 N=64 K=128, A/B from shared memory
 //   P_half = softmax rows    one warpgroup per half reads S with tcgen05.ld,
-//                            keeps the running max/sum per row and writes P as
-//                            bf16 into shared memory (128-byte swizzled, K-major)
-//   O_half += P_half V       tcgen05.mma M=128 N=128 K=64, A = P, B = V (MN-major)
-// Double-buffered S lets QK^T of chunk j+1 run while the softmax works on
-// chunk j; the running max is lazily updated (O is rescaled in TMEM only when
-// a row max grows by more than 2^8).  A quarter of the exponentials are
+//                            keeps the running max/sum per row and writes P
+//                            back to tensor memory as bf16 pairs (tcgen05.st)
+//   O_half += P_half V       tcgen05.mma M=128 N=128 K=64, A = P from tensor
+//                            memory, B = V from shared memory (MN-major)
+// The softmax releases S as soon as it holds it in registers, so QK^T of
+// chunk j+1 runs while it computes the exponentials of chunk j; the running
+// max is lazily updated (O is rescaled in TMEM only when a row max grows by
+// more than 2^8).  A quarter of the exponentials are
 // computed on the FMA pipe (2^x = 2^rint(x) * cubic(x - rint(x))) so that the
 // special-function unit, which otherwise needs as many cycles per chunk as
 // the tensor core, stops being the bound.
 // Warp roles: warp 0 issues TMA (each half of the Q tile once per unit, K/V
-// per chunk into a 4-stage ring), warp 1 allocates TMEM, one thread of warp
+// per chunk into a 5-stage ring), warp 1 allocates TMEM, one thread of warp
 // 1 issues the MMAs of half 0 and one thread of warp 2 those of half 1 (in
 // the order QK(j+1) PV(j) per chunk j, so that neither half's chain waits
 // on the other's softmax), warps 4-7 and 8-11 are the softmax/epilogue
@@ -35,22 +36,21 @@ namespace csa {
 namespace {
 
 constexpr int kPfThreads = 384;
-constexpr int kNS = 4;                         // K/V stages
+constexpr int kNS = 5;                         // K/V stages
 constexpr int kQHalfBytes = 128 * 128 * 2;     // 32 KB: one 128-row half of the Q tile
 constexpr int kKVBytes = 64 * 128 * 2;         // 16 KB per K (or V) chunk
 constexpr int kStageBytes = 2 * kKVBytes;
-constexpr int kPBytes = 128 * 64 * 2;          // 16 KB: P of one half
 constexpr int kQOff = 0;
 constexpr int kKVOff = 2 * kQHalfBytes;
-constexpr int kPOff = kKVOff + kNS * kStageBytes;
-constexpr int kBarOff = kPOff + 2 * kPBytes;
+constexpr int kBarOff = kKVOff + kNS * kStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kEmuPeriod = 4;  // one pair of exponentials in kEmuPeriod on the FMA pipe
 
-// TMEM columns: S of half h, buffer b at 128 h + 64 b; O of half h at 256 + 128 h
-constexpr uint32_t kColO = 256;
+// TMEM columns: S of half h at 64 h, P (bf16 pairs) of half h at 128 + 32 h,
+// O of half h at 256 + 128 h
+constexpr uint32_t kColP = 128, kColO = 256;
 
 // instruction descriptors (kind::f16): D fp32, A/B bf16, M = 128
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (0u << 16) |
@@ -185,10 +185,6 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -198,12 +194,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const uint32_t sQ = sb + kQOff;
   const uint32_t sKV = sb + kKVOff;
-  const uint32_t sP = sb + kPOff;
   const uint32_t bar = sb + kBarOff;
   const uint32_t q_full = bar, q_empty = bar + 16;          // [2] each
   const uint32_t kv_full = bar + 32, kv_empty = kv_full + 8 * kNS;
-  const uint32_t s_full = kv_empty + 8 * kNS;               // [half][buffer]
-  const uint32_t p_full = s_full + 32;                      // [2]
+  const uint32_t s_full = kv_empty + 8 * kNS;               // [2]
+  const uint32_t s_free = s_full + 16;                      // [2]
+  const uint32_t p_full = s_free + 16;                      // [2]
   const uint32_t pv_done = p_full + 16;                     // [2]
   const uint32_t drain = pv_done + 16;                      // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + (drain + 16 - bar));
@@ -213,8 +209,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int h = 0; h < 2; ++h) {
       mbar_init(q_full + 8 * h, 1);
       mbar_init(q_empty + 8 * h, 1);
-      mbar_init(s_full + 8 * (2 * h), 1);
-      mbar_init(s_full + 8 * (2 * h + 1), 1);
+      mbar_init(s_full + 8 * h, 1);
+      mbar_init(s_free + 8 * h, 128);
       mbar_init(p_full + 8 * h, 128);
       mbar_init(pv_done + 8 * h, 1);
     }
@@ -309,9 +305,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t q_phase = 0, p_phase = 0, s_cnt = 0, kv_it = 0;
       bool ok = true;
       const uint32_t qa = sQ + hf * kQHalfBytes;
-      auto qk = [&](uint32_t stage) {
-        const uint32_t buf = s_cnt & 1u;
-        const uint32_t d = tmem + hf * 128 + buf * 64;
+      // S of this half is overwritten only after the softmax has loaded the
+      // previous S (s_free), so QK^T of chunk j+1 runs during its exponentials
+      auto qk = [&](uint32_t stage) -> bool {
+        if (s_cnt > 0 && !mbar_wait(s_free + 8 * hf, (s_cnt - 1) & 1u, p.err)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + hf * 64;
         const uint32_t kb = sKV + stage * kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -320,17 +319,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           umma_ss(d, smem_desc(qa + off_q, 16, 1024), smem_desc(kb + off_k, 16, 1024), kIdescQK,
                   kk > 0 ? 1u : 0u);
         }
-        umma_commit(s_full + 8 * (2 * hf + buf));
+        umma_commit(s_full + 8 * hf);
         ++s_cnt;
+        return true;
       };
       auto pv = [&](uint32_t stage, bool acc) {
         const uint32_t d = tmem + kColO + hf * 128;
-        const uint32_t pa = sP + hf * kPBytes;
+        const uint32_t pa = tmem + kColP + hf * 32;
         const uint32_t vb = sKV + stage * kStageBytes + kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ss(d, smem_desc(pa + kk * 32, 16, 1024), smem_desc(vb + kk * 2048, 8192, 1024),
-                  kIdescPV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts(d, pa + kk * 8, smem_desc(vb + kk * 2048, 8192, 1024), kIdescPV,
+                  (acc || kk > 0) ? 1u : 0u);
         umma_commit(pv_done + 8 * hf);
       };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
@@ -342,19 +342,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!mbar_wait(kv_full + 8 * st0, (kv_it / kNS) & 1u, p.err)) break;
         if (!mbar_wait(q_full + 8 * hf, q_phase, p.err)) break;
         q_phase ^= 1u;
-        tc_fence_after();
-        qk(st0);
+        if (!qk(st0)) break;
         if (n == 1) umma_commit(q_empty + 8 * hf);
         for (int j = 0; j < n; ++j) {
           const uint32_t cur = kv_it % kNS, nxt = (kv_it + 1) % kNS;
           if (j + 1 < n) {
-            // the buffer was last read by the softmax of chunk j - 1, whose P
-            // (p_full) has been waited for
             if (!mbar_wait(kv_full + 8 * nxt, ((kv_it + 1) / kNS) & 1u, p.err)) { ok = false; break; }
-            tc_fence_after();
-            qk(nxt);
+            if (!qk(nxt)) { ok = false; break; }
             if (j + 2 == n) umma_commit(q_empty + 8 * hf);
           }
+          // P of chunk j written, and (implied) the PV of chunk j - 1 done
           if (!mbar_wait(p_full + 8 * hf, p_phase, p.err)) { ok = false; break; }
           p_phase ^= 1u;
           tc_fence_after();
@@ -373,9 +370,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int half = (warp - 4) >> 2;
     const int r = ((warp & 3) << 5) + lane;  // row within the half == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + half * 128;
+    const uint32_t tS = tmem + lane_base + half * 64;
+    const uint32_t tP = tmem + lane_base + kColP + half * 32;
     const uint32_t tO = tmem + lane_base + kColO + half * 128;
-    uint8_t* prow = smem + kPOff + half * kPBytes + r * 128;
     const uint32_t my_p_full = p_full + 8 * half, my_pv_done = pv_done + 8 * half;
     const int g = half * 2 + (r >> 6);  // query head within the group
     const int i = r & 63;               // row within the tile
@@ -398,19 +395,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int c = c_next;
         if (j + 1 < n) c_next = unit_chunk(p, sel, j + 1);
-        const uint32_t buf = s_cnt & 1u, sph = (s_cnt >> 1) & 1u;
+        const uint32_t sph = s_cnt & 1u;
         ++s_cnt;
         // wait results are made warp-uniform: the TMEM accesses below are
         // warp-collective
-        if (!warp_wait(s_full + 8 * (2 * half + buf), sph, p.err)) {
+        if (!warp_wait(s_full + 8 * half, sph, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sr[2][32];
-        tmem_ld32(tS + buf * 64, sr[0]);
-        tmem_ld32(tS + buf * 64 + 32, sr[1]);
+        tmem_ld32(tS, sr[0]);
+        tmem_ld32(tS + 32, sr[1]);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_free + 8 * half);  // S is in registers: QK^T of the next chunk may overwrite it
         float x[64];
 #pragma unroll
         for (int jj = 0; jj < 64; ++jj) x[jj] = __uint_as_float(sr[jj >> 5][jj & 31]);
@@ -492,12 +491,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
              (acc[3].x + acc[3].y);
-        // P row r -> shared memory, 16-byte chunk q at q ^ (r % 8) (128-byte swizzle)
-#pragma unroll
-        for (int q16 = 0; q16 < 8; ++q16)
-          *reinterpret_cast<uint4*>(prow + ((q16 ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * q16], pk[4 * q16 + 1], pk[4 * q16 + 2], pk[4 * q16 + 3]);
-        fence_proxy_async_smem();
+        tmem_st32(tP, pk);  // P row r (bf16 pairs), the A operand of this half's PV
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(my_p_full);
       }
