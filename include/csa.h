@@ -122,7 +122,8 @@ CSA_API csa_status csa_meta_summaries(const float* summ, int B, int Hkv, int C, 
 /* ---------------------------------------------------------------- a7
  * Tile-mean queries for prefill (HiLS review section 3: adjacent queries
  * share one chunk union):  qbar[b,t,h,:] = (1/tile_m) sum_{i<tile_m} Q[b,t*tile_m+i,h,:].
- *   Q [B, S, Hq, D] of `dtype` -> qbar [B, S/tile_m, Hq, D] fp32;  S % tile_m == 0, D <= 1024. */
+ *   Q [B, S, Hq, D] of `dtype` -> qbar [B, S/tile_m, Hq, D] fp32;  S % tile_m == 0, D <= 1024,
+ *   Hq*D a multiple of 8 (bf16) or 4 (fp32), else CSA_ERR_UNSUPPORTED. */
 CSA_API csa_status csa_tile_mean_q(const void* Q, csa_dtype dtype, int B, int S, int Hq, int D,
                            int tile_m, float* qbar, csa_stream stream);
 
@@ -320,9 +321,10 @@ CSA_API csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K
  * sparse heads once the selection has completed (SSA summary "핵심 기여";
  * Elastic Attention summary section 2.3: full and sparse heads in one pass).
  * bf16 caches only.  Fields of the descriptor are the arguments of those
- * calls.  num_parts 0 = the number of SMs minus B*Hkv (the selection's CTAs,
- * which run beside the first phase) when head_full is given, else the
- * number of SMs; at most 256.  The workspace must be sized for the P the
+ * calls.  num_parts 0 = the number of SMs (at most 256).  When head_full is
+ * given, the last min(B*Hkv + P - #SMs, P - 1) CTAs (those that find the
+ * selection's CTAs on their SMs and start late) take only selected chunks.
+ * The workspace must be sized for the P the
  * call uses (csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts) with the
  * same num_parts, 0 included, is always enough) and start zeroed once; each
  * call leaves it zeroed again.  Errors: as the underlying calls; nothing is

@@ -212,6 +212,8 @@ csa_status csa_tile_mean_q(const void* Q, csa_dtype dtype, int B, int S, int Hq,
   CSA_REQUIRE(B >= 0 && S >= 0 && Hq >= 0 && D > 0 && tile_m > 0, "bad sizes");
   CSA_REQUIRE(S % tile_m == 0, "S must be a multiple of tile_m");
   CSA_SUPPORT(D <= 1024 && Hq <= 65535 && B <= 65535, "D <= 1024, Hq and B <= 65535");
+  CSA_SUPPORT((static_cast<int64_t>(Hq) * D) % (dtype == CSA_BF16 ? 8 : 4) == 0,
+              "Hq * D must be a multiple of 8 (bf16) or 4 (fp32): rows are read 16 bytes at a time");
   if (static_cast<int64_t>(B) * S * Hq == 0) return CSA_OK;
   CSA_TRY(check_ptr(Q, "Q"));
   CSA_TRY(check_ptr(qbar, "qbar"));
@@ -560,14 +562,15 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
   int P = 0;
   CSA_TRY(decode_ptr_checks(d->q, d->K, d->V, d->idx, d->count, d->head_full, true, d->D, d->L,
                             d->num_parts, l, &P));
-  if (d->num_parts == 0 && d->head_full != nullptr) {
-    // The selection runs one CTA per (batch, KV head) unit beside the
-    // decode's first phase: leave it those SMs (counted without reading
-    // head_full, so that the call stays free of host-device copies).
-    P = std::max(1, std::min(csa::kMergedMaxParts, l.num_sms - d->B * d->Hkv));
-  } else if (d->num_parts == 0) {
-    P = std::min(csa::kMergedMaxParts, l.num_sms);
-  }
+  if (d->num_parts == 0) P = std::min(csa::kMergedMaxParts, l.num_sms);
+  // The selection runs one CTA per (batch, KV head) unit; while it runs the
+  // decode CTAs that find no free SM start late.  Those (the last ones of the
+  // grid) take no full-head work, only the selected chunks, which cannot
+  // start before the selection ends anyway.  Counted without reading
+  // head_full, so the call stays free of host-device copies.
+  int late = 0;
+  if (d->head_full != nullptr)
+    late = std::max(0, std::min(P - 1, P + d->B * d->Hkv - l.num_sms));
   const WorkspaceLayout w = workspace_layout(d->B, d->Hq, d->Hkv, d->D, P);
   CSA_REQUIRE(d->workspace_bytes >= static_cast<int64_t>(w.total),
               "workspace smaller than csa_decode_workspace_bytes()");
@@ -596,7 +599,7 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
   if (st != CSA_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(d->workspace);
   csa::MergeOut m{reinterpret_cast<int*>(ws + w.counters), d->out, d->out_dtype == CSA_BF16,
-                  d->lse_out, true};
+                  d->lse_out, true, late};
   std::string why;
   cudaError_t e = csa::launch_decode(l, d->q, d->K, d->V, true, d->idx, d->count, d->kmax,
                                      d->head_full, d->B, d->Hq, d->Hkv, d->D, d->T, d->L, d->scale,

@@ -72,6 +72,9 @@ struct DecodeParams {
   // after griddepcontrol.wait, the sparse units (launched with programmatic
   // dependent launch behind the selection kernel)
   int phased;
+  // phased: the last `late` CTAs of the grid take no phase-1 work (they can
+  // only start once the selection's CTAs have left their SMs)
+  int late;
 };
 
 // Unit sets of a phase: 0 = every unit, 1 = full-head units, 2 = sparse units.
@@ -154,6 +157,14 @@ __device__ __forceinline__ int unit_of(const int* prefix, int U, int64_t g) {
     else hi = mid - 1;
   }
   return lo;
+}
+
+// Piece c of P over N chunks: [N c / P, N (c + 1) / P); CTAs c >= P (the
+// late ones of phase 1) get an empty piece at N.
+__device__ __forceinline__ void piece_range(int64_t N, int64_t P, int64_t c, int64_t& a,
+                                            int64_t& bnd) {
+  a = c < P ? N * c / P : N;
+  bnd = c < P ? N * (c + 1) / P : N;
 }
 
 __device__ __forceinline__ int64_t piece_of(int64_t g, int64_t N, int64_t P) {
@@ -352,6 +363,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+// Release/acquire fence at GPU scope: orders this thread's partial writes
+// before its arrival count (release), and the count before the reads of a
+// merge (acquire).  Lighter than the sequentially consistent __threadfence.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -415,18 +433,29 @@ __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area
   const int b = u / p.Hkv, h = u % p.Hkv;
   const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
   const uint32_t head_bytes = static_cast<uint32_t>(ns) * D * 4;
+  // lse rows come along when they start on 16-byte boundaries; a row is
+  // copied rounded up to 4 floats (the workspace holds more after the last)
+  const int ns4 = (ns + 3) & ~3;
+  const bool lse_bulk = (p.max_splits & 3) == 0;
+  const uint32_t lse_bytes = lse_bulk ? static_cast<uint32_t>(ns4) * 4 : 0u;
   float* wts = reinterpret_cast<float*>(area + area_bytes - 8192);
-  if (static_cast<size_t>(G) * head_bytes > static_cast<size_t>(area_bytes) - 8192 || ns > 256)
+  if (static_cast<size_t>(G) * (head_bytes + lse_bytes) > static_cast<size_t>(area_bytes) - 8192 ||
+      ns > 256)
     return merge_unit<D, 8>(p, u, ns, wts, tid, nthr, sync);
   const uint32_t phase = n_bulk & 1u;
   ++n_bulk;
-  float* st = reinterpret_cast<float*>(area);  // [G][ns][D]
+  float* st = reinterpret_cast<float*>(area);                    // [G][ns][D]
+  float* sl_rows = st + static_cast<size_t>(G) * ns * D;         // [G][ns4]
   if (tid == 0) {
     fence_proxy_async_global();  // partials written by other CTAs, read through the async proxy
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(G) * head_bytes);
-    for (int g = 0; g < G; ++g)
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(G) * (head_bytes + lse_bytes));
+    for (int g = 0; g < G; ++g) {
       bulk_load(smem_u32(st + static_cast<size_t>(g) * ns * D),
                 p.o_part + (row0 + g) * p.max_splits * D, head_bytes, bar);
+      if (lse_bulk)
+        bulk_load(smem_u32(sl_rows + g * ns4), p.lse_part + (row0 + g) * p.max_splits, lse_bytes,
+                  bar);
+    }
   }
   const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
   float* ww = wts + warp * 256;  // this warp's split weights
@@ -435,7 +464,7 @@ __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area
     const float* lsp = p.lse_part + (row0 + g) * p.max_splits;
     float mx = -INFINITY;
     for (int sl = lane; sl < ns; sl += 32) {
-      const float v = __ldcg(lsp + sl);
+      const float v = lse_bulk ? sl_rows[g * ns4 + sl] : __ldcg(lsp + sl);
       ww[sl] = v;
       mx = fmaxf(mx, v);
     }
@@ -522,7 +551,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   }
   build_prefix(p, prefix, scan_sh, p.phased ? 1 : 0);  // ends with __syncthreads (also publishes the barriers)
   const int n_phase = p.phased ? 2 : 1;
-  const int64_t P = gridDim.x;
+  // pieces per phase: phase 1 of a phased launch leaves out the late CTAs
+  const int64_t P_all = gridDim.x;
+  auto phase_parts = [&](int ph) -> int64_t {
+    return (p.phased && ph == 0) ? P_all - p.late : P_all;
+  };
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer
@@ -539,7 +572,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         pre = prefix2;
       }
       const int64_t N = pre[p.U];
-      const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+      int64_t a, bnd;
+      piece_range(N, phase_parts(ph), blockIdx.x, a, bnd);
       for (int64_t g0 = a; g0 < bnd && ok; g0 += 32) {
         const int64_t g = g0 + lane;
         int row = 0, qu = -1;
@@ -611,7 +645,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (!end_sync()) return;
     const int nd = n_defer_sh;
     if (nd == 0) return;
-    __threadfence();
+    fence_acq_rel_gpu();  // the arrival counts seen before the partials are read
     uint32_t n_bulk = 0;
     for (int k = 0; k < nd; ++k) {
       const int u = defer_u[k];
@@ -639,8 +673,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
         pre = prefix2;
       }
-      const int64_t N = pre[p.U];
-      const int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+      const int64_t N = pre[p.U], P = phase_parts(ph);
+      int64_t a, bnd;
+      piece_range(N, P, blockIdx.x, a, bnd);
       if (a >= bnd) continue;
       const int u0 = unit_of(pre, p.U, a), u1 = unit_of(pre, p.U, bnd - 1);
       for (int u = u0; u <= u1 && ok; ++u) {
@@ -696,7 +731,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(fb_empty + 8 * k);  // the consumers may refill it
         if (!p.merged || direct) continue;
-        __threadfence();
+        fence_acq_rel_gpu();  // this lane's partial writes before the arrival count
         __syncwarp();
         int last = 0;
         if (lane == 0) last = atomicAdd(p.counters + u, 1) == ns - 1;
@@ -709,7 +744,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           }
           ++n_defer;
         } else {
-          __threadfence();
+          fence_acq_rel_gpu();
           merge_unit_warp<D>(p, u, ns);
           __syncwarp();
           if (lane == 0) p.counters[u] = 0;
@@ -726,7 +761,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // ------------------------------------------------------------------ consumers
   const int* pre = prefix;
   int64_t N = pre[p.U];
-  int64_t a = N * blockIdx.x / P, bnd = N * (blockIdx.x + 1) / P;
+  int64_t a, bnd;
+  piece_range(N, phase_parts(0), blockIdx.x, a, bnd);
   if (p.merged) zero_empty_units(p, pre, p.phased ? 1 : 0, kConsumerWarps * 32);
   else fill_empty_slots(p, pre, kConsumerWarps * 32);
   const float scale_log2 = p.scale_log2;
@@ -792,8 +828,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       grid_dependency_wait();
       pre = prefix2;
       N = pre[p.U];
-      a = N * blockIdx.x / P;
-      bnd = N * (blockIdx.x + 1) / P;
+      piece_range(N, phase_parts(1), blockIdx.x, a, bnd);
       zero_empty_units(p, pre, 2, kConsumerWarps * 32);
     }
     for (int64_t g = a; g < bnd; ++g, ++i) {
@@ -1186,6 +1221,7 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
     p.out_bf16 = merge->out_bf16 ? 1 : 0;
     p.lse_out = merge->lse_out;
     p.phased = (merge->phased && bf16) ? 1 : 0;
+    p.late = p.phased ? merge->late : 0;
   }
   p.D = D;
   p.q = q;

@@ -70,6 +70,9 @@ struct MergeOut {
   // precedes it on the stream completes) the sparse units; the decode is
   // launched with programmatic dependent launch
   bool phased = false;
+  // phased: CTAs at the end of the grid that take no full-head work (they
+  // start only after the selection's CTAs leave their SMs)
+  int late = 0;
 };
 constexpr int kMergedMaxParts = 256;
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,

@@ -14,7 +14,7 @@
 // The softmax releases S as soon as it holds it in registers, so QK^T of
 // chunk j+1 runs while it computes the exponentials of chunk j; the running
 // max is lazily updated (O is rescaled in TMEM only when a row max grows by
-// more than 2^8).  A quarter of the exponentials are
+// more than 2^8).  A third of the exponentials are
 // computed on the FMA pipe (2^x = 2^rint(x) * cubic(x - rint(x))) so that the
 // special-function unit, which otherwise needs as many cycles per chunk as
 // the tensor core, stops being the bound.
@@ -46,7 +46,7 @@ constexpr int kBarOff = kKVOff + kNS * kStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kEmuPeriod = 4;  // one pair of exponentials in kEmuPeriod on the FMA pipe
+constexpr int kEmuPeriod = 3;  // one pair of exponentials in kEmuPeriod on the FMA pipe
 
 // TMEM columns: S of half h at 64 h, P (bf16 pairs) of half h at 128 + 32 h,
 // O of half h at 256 + 128 h
@@ -505,18 +505,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       pv_phase ^= 1u;
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
+      // two 32-column loads in flight at a time
 #pragma unroll 1
-      for (int cc = 0; cc < 128; cc += 32) {
-        uint32_t ov[32];
-        tmem_ld32(tO + cc, ov);
+      for (int cc = 0; cc < 128; cc += 64) {
+        uint32_t ov[2][32];
+        tmem_ld32(tO + cc, ov[0]);
+        tmem_ld32(tO + cc + 32, ov[1]);
         tmem_wait_ld();
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + cc);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(ov[hh][2 * e]) * inv,
+                                __uint_as_float(ov[hh][2 * e + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc + 32 * hh);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
       }
       // the next unit's first PV overwrites O: it is issued after this
       // warpgroup's next p_full arrival, which follows these loads

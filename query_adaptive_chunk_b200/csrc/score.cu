@@ -90,6 +90,89 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(
   }
 }
 
+// Many query rows per unit (prefill tile means): the scores of one unit are
+// the product of its [Nq, DS] group-summed query rows with its [C, DS]
+// summaries, so the CTA stages a 64-row block of each in shared memory
+// (padded rows, no bank conflicts) and every thread accumulates a 4 x 4
+// block of outputs in registers; each summary row is read once per 64 query
+// rows instead of once per row.  Blocks above the causal diagonal are only
+// filled with -inf.
+constexpr int kTileRows = 64;
+constexpr int kTileThreads = 256;
+
+template <int DS>
+__global__ void __launch_bounds__(kTileThreads) score_tiles_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ summ, int Nq, int Hq,
+    int Hkv, int C, const uint8_t* __restrict__ head_full, int causal_tile_m, int causal_L,
+    float* __restrict__ scores) {
+  constexpr int LD = DS + 1;
+  extern __shared__ float sm_tile[];
+  float* As = sm_tile;                   // [64][LD] query rows
+  float* Bs = sm_tile + kTileRows * LD;  // [64][LD] summary rows
+  const int u = blockIdx.z;
+  const int h = u % Hkv, b = u / Hkv;
+  if (head_full != nullptr && head_full[h]) return;
+  const int G = Hq / Hkv;
+  const int n0 = blockIdx.y * kTileRows, c0 = blockIdx.x * kTileRows;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16 threads, 4 x 4 outputs each
+  float* out = scores + static_cast<int64_t>(u) * Nq * C;
+  auto visible = [&](int n) {  // chunks [0, visible(n)) of query row n
+    return causal_tile_m > 0 ? min(C, ((n + 1) * causal_tile_m - 1) / causal_L + 1) : C;
+  };
+  const int n_last = min(Nq, n0 + kTileRows) - 1;
+  if (c0 >= visible(n_last)) {  // the whole block is masked
+    for (int i = threadIdx.x; i < kTileRows * kTileRows; i += kTileThreads) {
+      const int n = n0 + i / kTileRows, c = c0 + i % kTileRows;
+      if (n < Nq && c < C) out[static_cast<int64_t>(n) * C + c] = -INFINITY;
+    }
+    return;
+  }
+  // stage the group-summed query rows and the summary rows
+  for (int i = threadIdx.x; i < kTileRows * DS; i += kTileThreads) {
+    const int r = i / DS, d = i % DS, n = n0 + r;
+    float acc = 0.f;
+    if (n < Nq) {
+      for (int g = 0; g < G; ++g) {
+        const int64_t off = ((static_cast<int64_t>(b) * Nq + n) * Hq + h * G + g) * DS + d;
+        acc += q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
+                      : static_cast<const float*>(q)[off];
+      }
+    }
+    As[r * LD + d] = acc;
+    const int c = c0 + r;
+    Bs[r * LD + d] = c < C ? __ldg(summ + (static_cast<int64_t>(u) * C + c) * DS + d) : 0.f;
+  }
+  __syncthreads();
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < DS; ++d) {
+    float a[4], bb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = As[(ty * 4 + i) * LD + d];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bb[j] = Bs[(tx * 4 + j) * LD + d];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += a[i] * bb[j];
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = n0 + ty * 4 + i;
+    if (n >= Nq) continue;
+    const int v = visible(n);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx * 4 + j;
+      if (c < C) out[static_cast<int64_t>(n) * C + c] = c < v ? acc[i][j] : -INFINITY;
+    }
+  }
+}
+
 template <int DS>
 cudaError_t launch_ds(const Launch& l, const void* q, bool bf16, const float* proj, int R,
                       const float* summ, int B, int Nq, int Hq, int Hkv, int D, int C,
@@ -108,6 +191,21 @@ cudaError_t launch_score(const Launch& l, const void* q, bool bf16, const float*
                          const uint8_t* head_full, int causal_tile_m, int causal_L,
                          float* scores) {
   if (B == 0 || Nq == 0 || C == 0) return cudaSuccess;
+  if (proj == nullptr && Nq >= 16 && (D == 128 || D == 64)) {
+    dim3 grid((C + kTileRows - 1) / kTileRows, (Nq + kTileRows - 1) / kTileRows, B * Hkv);
+    const size_t sh = 2 * kTileRows * static_cast<size_t>(D + 1) * sizeof(float);
+    if (D == 128) {
+      cudaError_t e = cudaFuncSetAttribute(score_tiles_kernel<128>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+      if (e != cudaSuccess) return e;
+      score_tiles_kernel<128><<<grid, kTileThreads, sh, l.stream>>>(
+          q, bf16 ? 1 : 0, summ, Nq, Hq, Hkv, C, head_full, causal_tile_m, causal_L, scores);
+    } else {
+      score_tiles_kernel<64><<<grid, kTileThreads, sh, l.stream>>>(
+          q, bf16 ? 1 : 0, summ, Nq, Hq, Hkv, C, head_full, causal_tile_m, causal_L, scores);
+    }
+    return cudaGetLastError();
+  }
   const int Ds = proj ? R : D;
   switch (Ds) {
     case 16: return launch_ds<16>(l, q, bf16, proj, R, summ, B, Nq, Hq, Hkv, D, C, head_full, causal_tile_m, causal_L, scores);

@@ -1,7 +1,7 @@
 // Precompute kernels: chunk summaries (chunk-mean keys, optionally projected
 // to a low rank), meta-summaries (mean of Gm chunk summaries) and tile-mean
 // queries.  These run once per cache / per prefill, outside the per-step path;
-// each is a plain coalesced reduction with one thread per column.
+// each is a coalesced reduction over rows.
 #include "internal.h"
 
 namespace csa {
@@ -60,18 +60,57 @@ __global__ void meta_summaries_kernel(const float* __restrict__ summ, int C, int
   }
 }
 
-template <typename T>
-__global__ void tile_mean_kernel(const T* __restrict__ Q, int S, int Hq, int D, int tile_m,
-                                 float* __restrict__ qbar) {
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int n_tiles = S / tile_m;
-  const float inv = 1.0f / static_cast<float>(tile_m);
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    const T* p = Q + ((static_cast<int64_t>(b) * S + static_cast<int64_t>(t) * tile_m) * Hq + h) * D + d;
-    for (int i = 0; i < tile_m; ++i) acc += ld_f<T>(p + static_cast<int64_t>(i) * Hq * D);
-    qbar[((static_cast<int64_t>(b) * n_tiles + t) * Hq + h) * D + d] = acc * inv;
+// Tile means: a position's Hq*D query values are one contiguous row; each
+// thread owns 16 bytes of it (8 bf16 or 4 fp32 values, so a warp reads 512
+// contiguous bytes per row) and sums them over the tile's rows in row order,
+// eight rows in flight.  Grid: (tiles, row segments of 128 threads, batch).
+constexpr int kTileMeanThreads = 128;
+
+__device__ __forceinline__ void add16(float* acc, const uint4& v, const __nv_bfloat16*) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    acc[2 * e] += f.x;
+    acc[2 * e + 1] += f.y;
   }
+}
+__device__ __forceinline__ void add16(float* acc, const uint4& v, const float*) {
+  acc[0] += __uint_as_float(v.x);
+  acc[1] += __uint_as_float(v.y);
+  acc[2] += __uint_as_float(v.z);
+  acc[3] += __uint_as_float(v.w);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTileMeanThreads) tile_mean_kernel(
+    const T* __restrict__ Q, int S, int HD, int tile_m, float* __restrict__ qbar) {
+  constexpr int E = 16 / sizeof(T);  // values per thread
+  const int t = blockIdx.x, b = blockIdx.z;
+  const int n_tiles = S / tile_m;
+  const int col = (blockIdx.y * kTileMeanThreads + threadIdx.x) * E;
+  if (col >= HD) return;
+  const T* p = Q + (static_cast<int64_t>(b) * S + static_cast<int64_t>(t) * tile_m) * HD + col;
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  int i = 0;
+  for (; i + 8 <= tile_m; i += 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      v[k] = __ldg(reinterpret_cast<const uint4*>(p + static_cast<int64_t>(i + k) * HD));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) add16(acc, v[k], static_cast<const T*>(nullptr));
+  }
+  for (; i < tile_m; ++i)
+    add16(acc, __ldg(reinterpret_cast<const uint4*>(p + static_cast<int64_t>(i) * HD)),
+          static_cast<const T*>(nullptr));
+  const float inv = 1.0f / static_cast<float>(tile_m);
+  float4* out = reinterpret_cast<float4*>(qbar + (static_cast<int64_t>(b) * n_tiles + t) * HD + col);
+#pragma unroll
+  for (int e = 0; e < E; e += 4)
+    out[e / 4] = make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
 }
 
 }  // namespace
@@ -106,14 +145,15 @@ cudaError_t launch_tile_mean(const Launch& l, const void* Q, bool bf16, int B, i
                              int tile_m, float* qbar) {
   const int n = S / tile_m;
   if (n == 0 || B == 0 || Hq == 0) return cudaSuccess;
-  dim3 grid(n, Hq, B);
-  const int threads = D >= 128 ? 128 : ((D + 31) / 32) * 32;
+  const int HD = Hq * D;  // a multiple of 8 (D is 64 or 128)
+  const int E = bf16 ? 8 : 4;
+  dim3 grid(n, (HD / E + kTileMeanThreads - 1) / kTileMeanThreads, B);
   if (bf16)
-    tile_mean_kernel<__nv_bfloat16><<<grid, threads, 0, l.stream>>>(
-        static_cast<const __nv_bfloat16*>(Q), S, Hq, D, tile_m, qbar);
+    tile_mean_kernel<__nv_bfloat16><<<grid, kTileMeanThreads, 0, l.stream>>>(
+        static_cast<const __nv_bfloat16*>(Q), S, HD, tile_m, qbar);
   else
-    tile_mean_kernel<float><<<grid, threads, 0, l.stream>>>(static_cast<const float*>(Q), S, Hq, D,
-                                                           tile_m, qbar);
+    tile_mean_kernel<float><<<grid, kTileMeanThreads, 0, l.stream>>>(static_cast<const float*>(Q),
+                                                                    S, HD, tile_m, qbar);
   return cudaGetLastError();
 }
 

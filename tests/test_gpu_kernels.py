@@ -51,6 +51,15 @@ def test_chunk_summaries(csa, dtype, D, L, R):
     assert np.abs(out.cpu().double().numpy() - ref).max() < 1e-5
 
 
+def test_tile_mean_fp32_ragged_tile(csa):
+    """fp32 queries and a tile length that is not a multiple of the kernel's
+    8-row batches."""
+    Q = _randn((1, 12 * 7, 4, 64), 61)
+    qbar = torch.empty(1, 7, 4, 64, device="cuda")
+    csa.csa_tile_mean_q(Q, Q.dtype, 1, 12 * 7, 4, 64, 12, qbar)
+    assert np.abs(qbar.cpu().double().numpy() - O.tile_mean_q(to_np(Q), 12)).max() < 1e-5
+
+
 def test_meta_summaries_and_tile_mean(csa):
     summ = _randn((2, 3, 64, 128), 3)
     meta = torch.empty(2, 3, 8, 128, device="cuda")
@@ -66,7 +75,7 @@ def test_meta_summaries_and_tile_mean(csa):
 
 @pytest.mark.parametrize("G,D,R,C,causal", [(4, 128, 0, 517, False), (4, 128, 16, 1029, False),
                                             (1, 64, 0, 70, False), (8, 128, 32, 300, False),
-                                            (4, 128, 0, 96, True)])
+                                            (4, 128, 0, 96, True), (2, 64, 0, 150, True)])
 def test_score_chunks(csa, G, D, R, C, causal):
     B, Hkv = 2, 3
     Hq = G * Hkv
