@@ -127,20 +127,43 @@ __global__ void __launch_bounds__(kTileThreads) score_tiles_kernel(
     }
     return;
   }
-  // stage the group-summed query rows and the summary rows
-  for (int i = threadIdx.x; i < kTileRows * DS; i += kTileThreads) {
-    const int r = i / DS, d = i % DS, n = n0 + r;
-    float acc = 0.f;
+  // stage the group-summed query rows and the summary rows, 4 floats per load
+  constexpr int D4 = DS / 4;
+  for (int i = threadIdx.x; i < kTileRows * D4; i += kTileThreads) {
+    const int r = i / D4, d = (i % D4) * 4, n = n0 + r;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (n < Nq) {
+      const int64_t row = (static_cast<int64_t>(b) * Nq + n) * Hq + h * G;
       for (int g = 0; g < G; ++g) {
-        const int64_t off = ((static_cast<int64_t>(b) * Nq + n) * Hq + h * G + g) * DS + d;
-        acc += q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
-                      : static_cast<const float*>(q)[off];
+        float4 x;
+        if (q_bf16) {
+          const __nv_bfloat162* qp = reinterpret_cast<const __nv_bfloat162*>(
+              static_cast<const __nv_bfloat16*>(q) + (row + g) * DS + d);
+          const float2 lo = __bfloat1622float2(qp[0]), hi = __bfloat1622float2(qp[1]);
+          x = make_float4(lo.x, lo.y, hi.x, hi.y);
+        } else {
+          x = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(q) + (row + g) * DS + d));
+        }
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
       }
     }
-    As[r * LD + d] = acc;
+    float* ar = As + r * LD + d;
+    ar[0] = acc.x;
+    ar[1] = acc.y;
+    ar[2] = acc.z;
+    ar[3] = acc.w;
     const int c = c0 + r;
-    Bs[r * LD + d] = c < C ? __ldg(summ + (static_cast<int64_t>(u) * C + c) * DS + d) : 0.f;
+    const float4 sv = c < C ? __ldg(reinterpret_cast<const float4*>(
+                                  summ + (static_cast<int64_t>(u) * C + c) * DS + d))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    float* br = Bs + r * LD + d;
+    br[0] = sv.x;
+    br[1] = sv.y;
+    br[2] = sv.z;
+    br[3] = sv.w;
   }
   __syncthreads();
   float acc[4][4];
