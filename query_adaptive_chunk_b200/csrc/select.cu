@@ -891,6 +891,93 @@ __global__ void __launch_bounds__(kSelThreads) select_hier_kernel(
   emit_ascending(flags, C, idx + static_cast<int64_t>(u) * kmax, count + u, kmax, s);
 }
 
+// Selection by rank for small candidate sets (n <= kRankMax): thread i counts
+// the composite keys above its own (composites are unique: ties go to the
+// lower chunk index), and keeps i when fewer than k are above it.  Key 0 is
+// "not a candidate".  n^2 / blockDim comparisons, all shared-memory
+// broadcasts, and a single barrier.
+constexpr int kRankMax = 512;
+
+__device__ void rank_select(const uint64_t* comp, int n, int k, uint8_t* sel) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint64_t me = comp[i];
+    int above = 0;
+    if (me != 0ull)
+      for (int j = 0; j < n; ++j) above += comp[j] > me;
+    sel[i] = (me != 0ull && above < k) ? 1 : 0;
+  }
+  __syncthreads();
+}
+
+// Hierarchical selection when both levels have at most kRankMax candidates:
+// rank selection at each level, and the list written directly as sink
+// chunks, the chosen children (ascending already: the kept metas are
+// ascending and so are their children) and the local chunks.
+__global__ void __launch_bounds__(kSelThreads) select_hier_rank_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ meta,
+    const float* __restrict__ summ, int Hq, int Hkv, int D, int C, int Gm, int top_meta,
+    int k_free, int n_sink, int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count,
+    int kmax) {
+  allow_dependent_launch();
+  __shared__ SelScratch s;
+  __shared__ float qs[128];
+  __shared__ uint32_t keys[kRankMax];
+  __shared__ uint64_t comp[kRankMax];
+  __shared__ int clist[kRankMax];
+  __shared__ uint8_t sel[kRankMax];
+  __shared__ int mlist[kRankMax];
+  const int M = C / Gm;
+  const int k1 = min(top_meta, M);
+  const int NCH = k1 * Gm;
+  const int u = blockIdx.x;
+  const int h = u % Hkv, b = u / Hkv;
+  const int G = Hq / Hkv;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int g = 0; g < G; ++g) {
+      const int64_t off = (static_cast<int64_t>(b) * Hq + h * G + g) * D + d;
+      acc += q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
+                    : static_cast<const float*>(q)[off];
+    }
+    qs[d] = acc;
+  }
+  __syncthreads();
+  // level 1: meta-chunks (every meta is a candidate)
+  score_rows<false>(meta + static_cast<int64_t>(u) * M * D, D, qs, nullptr, M, keys, C, 0, 0);
+  __syncthreads();
+  for (int i = threadIdx.x; i < M; i += blockDim.x) comp[i] = composite(keys[i], i);
+  __syncthreads();
+  rank_select(comp, M, k1, sel);
+  {  // ascending list of the kept metas, then their children
+    int pos = block_exclusive_scan(threadIdx.x < M ? sel[threadIdx.x] : 0, s.scan, nullptr);
+    if (threadIdx.x < M && sel[threadIdx.x]) mlist[pos] = threadIdx.x;
+    __syncthreads();
+    for (int i = threadIdx.x; i < NCH; i += blockDim.x) clist[i] = mlist[i / Gm] * Gm + (i % Gm);
+    __syncthreads();
+  }
+  // level 2: the children, forced chunks excluded from the pool (key 0)
+  score_rows<true>(summ + static_cast<int64_t>(u) * C * D, D, qs, clist, NCH, keys, C, n_sink,
+                   n_local);
+  __syncthreads();
+  for (int i = threadIdx.x; i < NCH; i += blockDim.x) comp[i] = composite(keys[i], clist[i]);
+  __syncthreads();
+  rank_select(comp, NCH, k_free, sel);
+  // list = sink chunks, chosen children (ascending), local chunks
+  int nsel = 0;
+  const int pos = block_exclusive_scan(threadIdx.x < NCH ? sel[threadIdx.x] : 0, s.scan, &nsel);
+  const int n_s = min(n_sink, C);
+  const int loc0 = max(C - n_local, n_s);
+  const int n_l = C - loc0;
+  const int total = n_s + nsel + n_l;
+  int32_t* row = idx + static_cast<int64_t>(u) * kmax;
+  if (threadIdx.x < NCH && sel[threadIdx.x] && n_s + pos < kmax) row[n_s + pos] = clist[threadIdx.x];
+  for (int j = threadIdx.x; j < n_s && j < kmax; j += blockDim.x) row[j] = j;
+  for (int j = threadIdx.x; j < n_l; j += blockDim.x)
+    if (n_s + nsel + j < kmax) row[n_s + nsel + j] = loc0 + j;
+  for (int j = total + threadIdx.x; j < kmax; j += blockDim.x) row[j] = -1;
+  if (threadIdx.x == 0) count[u] = min(total, kmax);
+}
+
 // ---------------------------------------------------------------- fused score + select
 
 // Group-summed query of unit (b, h) into qs[0, D) and, with a projection,
@@ -1136,6 +1223,12 @@ cudaError_t launch_select_hier(const Launch& l, const void* q, bool bf16, const 
   const int M = C / Gm;
   const int k1 = std::min(top_meta, M);
   const int NCH = k1 * Gm;
+  if (M <= kRankMax && NCH <= kRankMax && D <= 128) {
+    select_hier_rank_kernel<<<U, kSelThreads, 0, l.stream>>>(q, bf16 ? 1 : 0, meta, summ, Hq, Hkv,
+                                                             D, C, Gm, top_meta, k_free, n_sink,
+                                                             n_local, idx, count, kmax);
+    return cudaGetLastError();
+  }
   const size_t base = (static_cast<size_t>(M) * 5 + static_cast<size_t>(NCH) * 9 +
                        static_cast<size_t>(k1) * 4 + static_cast<size_t>(C) + 15) & ~size_t(15);
   const size_t sh = base + sort_exch_bytes(std::max(M, NCH)) + 16;
