@@ -370,6 +370,12 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* ptr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -414,49 +420,76 @@ __device__ void merge_unit_warp(const DecodeParams& p, int u, int ns) {
   }
 }
 
-// Merge of unit u with its partials first copied into shared memory: one
-// bulk copy per head (the head's ns partial rows are contiguous), so the
-// partials cross from L2 in a single round trip.  `area` (area_bytes, the
-// idle K/V stage ring) receives them in all but its last 8 KB, which hold
-// the split weights; `bar` is an mbarrier of this CTA (count 1) and
-// `n_bulk` counts the copies that completed it so far.  Then each warp
-// takes whole heads: the head's lse and split weights stay in the warp
-// (shuffles and a per-warp slice of the weights), and the lanes accumulate
-// float4 columns, with no block barrier in between.  `nthr` (<= 256)
-// threads numbered `tid` by whole warps take part; `sync` is a barrier over
-// them (bounded).  Falls back to merge_unit when the partials do not fit.
+// Shared-memory staging of a unit's merge: the ns partial rows of each head
+// ([G][ns][D]) and, when rows start on 16-byte boundaries, its lse rows
+// ([G][ns4], each copied rounded up to 4 floats: the workspace holds more
+// after the last row), in the idle K/V stage ring; its last 8 KB hold the
+// split weights.
+struct MergeGeom {
+  uint32_t head_bytes, lse_bytes;
+  int ns4;
+  bool fits;
+};
+
+template <int D>
+__device__ __forceinline__ MergeGeom merge_geom(const DecodeParams& p, int ns, int area_bytes) {
+  MergeGeom m;
+  m.head_bytes = static_cast<uint32_t>(ns) * D * 4;
+  m.ns4 = (ns + 3) & ~3;
+  m.lse_bytes = (p.max_splits & 3) == 0 ? static_cast<uint32_t>(m.ns4) * 4 : 0u;
+  m.fits = ns <= 256 && static_cast<size_t>(p.G) * (m.head_bytes + m.lse_bytes) <=
+                            static_cast<size_t>(area_bytes) - 8192;
+  return m;
+}
+
+// Issues the bulk copies of unit u's partials (and lse rows) into `area`,
+// completing mbarrier `bar`.  The calling thread must have acquired the
+// unit's final arrival count (the partials are other CTAs' writes).
+template <int D>
+__device__ void merge_bulk_issue(const DecodeParams& p, int u, int ns, const MergeGeom& m,
+                                 uint8_t* area, uint32_t bar) {
+  const int G = p.G;
+  const int64_t row0 = static_cast<int64_t>(u / p.Hkv) * p.Hq + (u % p.Hkv) * G;
+  float* st = reinterpret_cast<float*>(area);
+  float* sl_rows = st + static_cast<size_t>(G) * ns * D;
+  fence_proxy_async_global();  // read through the async proxy
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(G) * (m.head_bytes + m.lse_bytes));
+  for (int g = 0; g < G; ++g) {
+    bulk_load(smem_u32(st + static_cast<size_t>(g) * ns * D),
+              p.o_part + (row0 + g) * p.max_splits * D, m.head_bytes, bar);
+    if (m.lse_bytes)
+      bulk_load(smem_u32(sl_rows + g * m.ns4), p.lse_part + (row0 + g) * p.max_splits,
+                m.lse_bytes, bar);
+  }
+}
+
+// Merge of unit u from its staged partials (merge_geom): one bulk copy per
+// head row set, so the partials cross from L2 in a single round trip (issued
+// here by tid 0, or earlier when `issued`); `bar` is an mbarrier of this CTA
+// (count 1) and `n_bulk` counts the copies that completed it so far.  Then
+// each warp takes whole heads: the head's lse and split weights stay in the
+// warp (shuffles and a per-warp slice of the weights), and the lanes
+// accumulate float4 columns, with no block barrier in between.  `nthr`
+// (<= 256) threads numbered `tid` by whole warps take part; `sync` is a
+// barrier over them (bounded).  Falls back to merge_unit when the partials
+// do not fit.
 template <int D, typename Sync>
 __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area, int area_bytes,
-                             uint32_t bar, uint32_t& n_bulk, int tid, int nthr, Sync sync) {
+                             uint32_t bar, uint32_t& n_bulk, bool issued, int tid, int nthr,
+                             Sync sync) {
   constexpr int D4 = D / 4;
   const int G = p.G;
-  const int b = u / p.Hkv, h = u % p.Hkv;
-  const int64_t row0 = static_cast<int64_t>(b) * p.Hq + h * G;
-  const uint32_t head_bytes = static_cast<uint32_t>(ns) * D * 4;
-  // lse rows come along when they start on 16-byte boundaries; a row is
-  // copied rounded up to 4 floats (the workspace holds more after the last)
-  const int ns4 = (ns + 3) & ~3;
-  const bool lse_bulk = (p.max_splits & 3) == 0;
-  const uint32_t lse_bytes = lse_bulk ? static_cast<uint32_t>(ns4) * 4 : 0u;
+  const int64_t row0 = static_cast<int64_t>(u / p.Hkv) * p.Hq + (u % p.Hkv) * G;
+  const MergeGeom m = merge_geom<D>(p, ns, area_bytes);
   float* wts = reinterpret_cast<float*>(area + area_bytes - 8192);
-  if (static_cast<size_t>(G) * (head_bytes + lse_bytes) > static_cast<size_t>(area_bytes) - 8192 ||
-      ns > 256)
-    return merge_unit<D, 8>(p, u, ns, wts, tid, nthr, sync);
+  if (!m.fits) return merge_unit<D, 8>(p, u, ns, wts, tid, nthr, sync);
   const uint32_t phase = n_bulk & 1u;
   ++n_bulk;
   float* st = reinterpret_cast<float*>(area);                    // [G][ns][D]
   float* sl_rows = st + static_cast<size_t>(G) * ns * D;         // [G][ns4]
-  if (tid == 0) {
-    fence_proxy_async_global();  // partials written by other CTAs, read through the async proxy
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(G) * (head_bytes + lse_bytes));
-    for (int g = 0; g < G; ++g) {
-      bulk_load(smem_u32(st + static_cast<size_t>(g) * ns * D),
-                p.o_part + (row0 + g) * p.max_splits * D, head_bytes, bar);
-      if (lse_bulk)
-        bulk_load(smem_u32(sl_rows + g * ns4), p.lse_part + (row0 + g) * p.max_splits, lse_bytes,
-                  bar);
-    }
-  }
+  const bool lse_bulk = m.lse_bytes != 0;
+  const int ns4 = m.ns4;
+  if (!issued && tid == 0) merge_bulk_issue<D>(p, u, ns, m, area, bar);
   const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
   float* ww = wts + warp * 256;  // this warp's split weights
   bool ok = warp_wait(bar, phase, p.err);
@@ -500,10 +533,80 @@ __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area
   return sync() && ok;  // the area is free again
 }
 
+// The epilogue warp's work for one flushed unit: combine the four consumer
+// warps' (m, l, O) from flush buffer `fo` into the unit's split partial (or
+// its output when ns == 1), release the buffer, and count the split in.
+// Returns 1 when this CTA brought the unit's last split (its merge is
+// deferred), 2 when it also started the merge's copy already (the CTA's last
+// flush), else 0.
+template <int D>
+__device__ __forceinline__ int epilogue_unit(const DecodeParams& p, const float* fo, int u,
+                                             int slot, int ns, bool final_flush, uint8_t* area,
+                                             int area_bytes, uint32_t merge_bar,
+                                             uint32_t fb_empty, int* pre_u, int* pre_ns) {
+  const int lane = threadIdx.x & 31, G = p.G;
+  const float* fm = fo + kConsumerWarps * G * D;
+  const float* fl = fm + kConsumerWarps * 8;
+  const int b = u / p.Hkv, h = u % p.Hkv;
+  const bool direct = p.merged && ns == 1;  // the only split: it is the output
+  // per head g = lane: max over the warps, warp weights, total sum
+  float M = -INFINITY, Ls = 0.f, scw[kConsumerWarps];
+  if (lane < G) {
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + lane]);
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      scw[w] = exp2f(fm[w * 8 + lane] - M);
+      Ls += fl[w * 8 + lane] * scw[w];
+    }
+  }
+  for (int g = 0; g < G; ++g) {
+    const float Mg = __shfl_sync(0xffffffffu, M, g), Lg = __shfl_sync(0xffffffffu, Ls, g);
+    float sc[kConsumerWarps];
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) sc[w] = __shfl_sync(0xffffffffu, scw[w], g);
+    const float inv = 1.0f / Lg;
+    const int64_t row = static_cast<int64_t>(b) * p.Hq + h * G + g;
+    for (int d = lane; d < D; d += 32) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) acc += fo[(w * G + g) * D + d] * sc[w];
+      if (direct) store_out(p, row * D + d, acc * inv);
+      else p.o_part[(row * p.max_splits + slot) * D + d] = acc * inv;
+    }
+    if (lane == 0) {
+      const float lse = (Mg + log2f(Lg)) * kLn2;
+      if (direct) {
+        if (p.lse_out) p.lse_out[row] = lse;
+      } else {
+        p.lse_part[row * p.max_splits + slot] = lse;
+      }
+    }
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(fb_empty);  // the consumers may refill it
+  if (!p.merged || direct) return 0;
+  fence_acq_rel_gpu();  // this lane's partial writes before the arrival count
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) {
+    last = atom_add_acq_rel_gpu(p.counters + u, 1) == ns - 1;
+    const MergeGeom mg = merge_geom<D>(p, ns, area_bytes);
+    if (last && final_flush && mg.fits) {  // start the merge's copy now, before the CTA barrier
+      merge_bulk_issue<D>(p, u, ns, mg, area, merge_bar);
+      *pre_u = u;
+      *pre_ns = ns;
+      last = 2;
+    }
+  }
+  return __shfl_sync(0xffffffffu, last, 0);
+}
+
 template <int D, int L>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ DecodeParams p) {
   using Sh = DecodeShape<D, L>;
   constexpr int NS = Sh::NS;
   constexpr int TOK_W = L / kConsumerWarps;  // tokens per consumer warp
@@ -527,7 +630,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   int* prefix2 = prefix + (p.U + 1);  // phase 2 (sparse units), built by the producer
   __shared__ int scan_sh[33];
   __shared__ int defer_u[kDeferMax], defer_ns[kDeferMax];
-  __shared__ int n_defer_sh;
+  __shared__ int n_defer_sh, pre_u_sh, pre_ns_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -543,6 +646,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     mbar_init(end_bar, (kConsumerWarps + 1) * 32);
     mbar_init(merge_bar, 1);
     n_defer_sh = 0;
+    pre_u_sh = -1;
     fence_barrier_init();
   }
   if (warp == kProducerWarp && lane == 0) {
@@ -561,6 +665,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // ---------------------------------------------------------------- producer
     const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
     const uint32_t q_bytes = static_cast<uint32_t>(G) * D * 2;
+    // K/V is read once: first out of L2, so that what the kernel reads again
+    // (its instructions, parameters, the partials and counters) stays there
+    const uint64_t kv_policy = l2_policy_evict_first();
     int64_t issued = 0;
     bool ok = true;
     for (int ph = 0; ph < n_phase && ok; ++ph) {
@@ -604,8 +711,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               const uint32_t dst = sbase + s * Sh::STAGE_BYTES;
 #pragma unroll
               for (int bx = 0; bx < NBOX; ++bx) {
-                tma_load_2d(dst + bx * Sh::BOX_BYTES, &tmK, bx * 64, row_j, fb);
-                tma_load_2d(dst + Sh::KV_BYTES + bx * Sh::BOX_BYTES, &tmV, bx * 64, row_j, fb);
+                tma_load_2d_hint(dst + bx * Sh::BOX_BYTES, &tmK, bx * 64, row_j, fb, kv_policy);
+                tma_load_2d_hint(dst + Sh::KV_BYTES + bx * Sh::BOX_BYTES, &tmV, bx * 64, row_j, fb,
+                                 kv_policy);
               }
             }
           }
@@ -643,14 +751,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   };
   auto final_merges = [&](int tid) {
     if (!end_sync()) return;
-    const int nd = n_defer_sh;
-    if (nd == 0) return;
-    fence_acq_rel_gpu();  // the arrival counts seen before the partials are read
+    const int nd = n_defer_sh, pu = pre_u_sh;
+    if (nd == 0 && pu < 0) return;
+    // the arrival counts seen (by the epilogue's atomics) before partials are
+    // read by these threads; not needed when the only merge's partials and
+    // lse rows come by the bulk copy its own issuer ordered
+    if (nd > 0 || (p.max_splits & 3) != 0) fence_acq_rel_gpu();
     uint32_t n_bulk = 0;
+    if (pu >= 0) {  // the last unit of the CTA: its copy is already in flight
+      if (!merge_staged<D>(p, pu, pre_ns_sh, smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk, true,
+                           tid, (kConsumerWarps + 1) * 32, end_sync))
+        return;
+      if (tid == 0) p.counters[pu] = 0;  // ready for the next call
+    }
     for (int k = 0; k < nd; ++k) {
       const int u = defer_u[k];
-      if (!merge_staged<D>(p, u, defer_ns[k], smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk, tid,
-                           (kConsumerWarps + 1) * 32, end_sync))
+      if (!merge_staged<D>(p, u, defer_ns[k], smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk, false,
+                           tid, (kConsumerWarps + 1) * 32, end_sync))
         return;
       if (tid == 0) p.counters[u] = 0;  // ready for the next call
     }
@@ -688,55 +805,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
         ++nseen;
         const float* fo = reinterpret_cast<const float*>(smem + Y.fb_off + k * Y.fb_bytes);
-        const float* fm = fo + kConsumerWarps * G * D;
-        const float* fl = fm + kConsumerWarps * 8;
-        const int b = u / p.Hkv, h = u % p.Hkv;
         const int slot = split_slot(pre[u], a, blockIdx.x, N, P);
         const int ns = split_count(pre[u], pre[u + 1], N, P);
-        const bool direct = p.merged && ns == 1;  // the only split: it is the output
-        // per head g = lane: max over the warps, warp weights, total sum
-        float M = -INFINITY, Ls = 0.f, scw[kConsumerWarps];
-        if (lane < G) {
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + lane]);
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) {
-            scw[w] = exp2f(fm[w * 8 + lane] - M);
-            Ls += fl[w * 8 + lane] * scw[w];
-          }
-        }
-        for (int g = 0; g < G; ++g) {
-          const float Mg = __shfl_sync(0xffffffffu, M, g), Lg = __shfl_sync(0xffffffffu, Ls, g);
-          float sc[kConsumerWarps];
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) sc[w] = __shfl_sync(0xffffffffu, scw[w], g);
-          const float inv = 1.0f / Lg;
-          const int64_t row = static_cast<int64_t>(b) * p.Hq + h * G + g;
-          for (int d = lane; d < D; d += 32) {
-            float acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) acc += fo[(w * G + g) * D + d] * sc[w];
-            if (direct) store_out(p, row * D + d, acc * inv);
-            else p.o_part[(row * p.max_splits + slot) * D + d] = acc * inv;
-          }
-          if (lane == 0) {
-            const float lse = (Mg + log2f(Lg)) * kLn2;
-            if (direct) {
-              if (p.lse_out) p.lse_out[row] = lse;
-            } else {
-              p.lse_part[row * p.max_splits + slot] = lse;
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(fb_empty + 8 * k);  // the consumers may refill it
-        if (!p.merged || direct) continue;
-        fence_acq_rel_gpu();  // this lane's partial writes before the arrival count
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = atomicAdd(p.counters + u, 1) == ns - 1;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) continue;
+        // the CTA's last flush: the consumers are done with the stage ring
+        const bool final_flush = ph == n_phase - 1 && u == u1;
+        int last = epilogue_unit<D>(p, fo, u, slot, ns, final_flush, smem, NS * Sh::STAGE_BYTES,
+                                    merge_bar, fb_empty + 8 * k, &pre_u_sh, &pre_ns_sh);
+        if (last != 1) continue;
         if (n_defer < kDeferMax) {  // merged after the main loop, off the hot path
           if (lane == 0) {
             defer_u[n_defer] = u;
