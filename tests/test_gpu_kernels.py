@@ -543,6 +543,19 @@ def test_merged_decode_edge_cases(csa):
     _merged_case(csa, "f32", B, Hkv, G, 64, C * L, L, sets, num_parts=3, with_lse=False)
 
 
+def test_merged_decode_second_wave(csa):
+    """More pieces than SMs with long chunk lists: the CTAs of the second wave
+    start only when CTAs of the first have retired, and still bring their
+    splits to the right units."""
+    B, Hkv, G, D, L, C = 2, 4, 4, 128, 64, 400
+    rng = np.random.default_rng(11)
+    sets = [sorted(rng.choice(C, size=int(rng.integers(150, 400)), replace=False).tolist())
+            for _ in range(B * Hkv)]
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=256)
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, full=(1,), num_parts=37,
+                 out_bf16=True)
+
+
 def test_merged_decode_mixed_heads(csa):
     B, Hkv, G, D, L, C = 1, 8, 4, 128, 128, 96
     rng = np.random.default_rng(7)
