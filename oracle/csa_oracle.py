@@ -25,7 +25,9 @@ What it computes, in the order the pages give it:
   glossary entry "Hierarchical Gist-of-Gist").  Sink and local chunks are
   always kept.
 * Exact attention over the raw KV of the selected chunks (SSA summary,
-  "방법론": standard attention over the hybrid context), computed as split-K
+  "방법론": standard attention over the hybrid context), and over the hybrid
+  context itself, the gist KV of every chunk plus the raw KV of the selected
+  ones ("방법론", "기술 상세"), computed as split-K
   partials combined afterwards (SSA summary, "핵심 기여": compact index list and
   split-K partial attention).
 * Block-sparse causal prefill over per-query-tile chunk sets (SSA summary,
@@ -303,6 +305,26 @@ def attend(q_heads: np.ndarray, K: np.ndarray, V: np.ndarray, tokens: np.ndarray
 def decode_unit(q_group, K_unit, V_unit, chunks, L: int, scale: float):
     """Attention of one unit's query heads over the raw KV of its chunk set."""
     return attend(q_group, K_unit, V_unit, chunk_tokens(sorted(chunks), L), scale)
+
+
+def hybrid_unit(q_group, K_unit, V_unit, Kg_unit, Vg_unit, chunks, L: int, scale: float):
+    """Attention of one unit's query heads over its hybrid context (SSA
+    summary, "방법론" and "기술 상세": K_hybrid and V_hybrid are the gist KV
+    together with the raw KV of the selected chunks I_t, attended with
+    standard attention).
+
+    Reading: every chunk keeps its gist token in the context (glossary entry
+    "Selective Unfolding": the query first meets the gist tokens of all
+    chunks), and the raw tokens of the selected chunks are added next to
+    them.  One softmax runs over the union, with the same scale for gist and
+    raw logits.  K_unit/V_unit [T, D] raw; Kg_unit/Vg_unit [C, D], one gist
+    key/value per chunk -> o [G, D], lse [G]."""
+    tok = chunk_tokens(sorted(chunks), L)
+    Kr = np.asarray(K_unit, dtype=np.float64)[tok]
+    Vr = np.asarray(V_unit, dtype=np.float64)[tok]
+    Kh = np.concatenate([Kr, np.asarray(Kg_unit, dtype=np.float64)], axis=0)
+    Vh = np.concatenate([Vr, np.asarray(Vg_unit, dtype=np.float64)], axis=0)
+    return attend(q_group, Kh, Vh, np.arange(Kh.shape[0]), scale)
 
 
 def lse_merge(o_part: np.ndarray, lse_part: np.ndarray) -> tuple[np.ndarray, np.ndarray]:

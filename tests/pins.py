@@ -86,6 +86,46 @@ def check_empty_attention():
     assert np.all(o == 0) and np.all(lse == -math.inf)
 
 
+def check_hybrid_golden():
+    """Hybrid context (gist KV of every chunk + raw KV of the selected ones):
+    the hand-worked cases of tests/golden/hybrid_cases.json."""
+    g = _golden("hybrid_cases.json")
+    q, K, V = (np.array(g[k], dtype=np.float64) for k in ("q", "K", "V"))
+    Kg, Vg = np.array(g["Kg"], dtype=np.float64), np.array(g["Vg"], dtype=np.float64)
+    for c in g["cases"]:
+        o, lse = O.hybrid_unit(q, K, V, Kg, Vg, c["chunks"], g["L"], g["scale"])
+        assert np.allclose(o, np.array(c["o"]), rtol=0, atol=1e-12), (c["chunks"], o)
+        assert np.allclose(lse, np.array(c["lse"]), rtol=0, atol=1e-12), (c["chunks"], lse)
+
+
+def check_hybrid_vs_sdpa(seed=16, G=4, D=16, T=256, L=32):
+    """Hybrid context == fp64 SDPA over the raw cache with the C gist rows
+    appended, masked to keep the selected chunks' raw tokens and every gist
+    row; lse == logsumexp of the same masked logits.  Chunk sets from empty
+    to all chunks."""
+    rng = np.random.default_rng(seed)
+    C = T // L
+    for n_sel in (0, 1, 3, C):
+        q = rng.standard_normal((G, D))
+        K, V = rng.standard_normal((T, D)), rng.standard_normal((T, D))
+        Kg, Vg = rng.standard_normal((C, D)), rng.standard_normal((C, D))
+        chunks = sorted(rng.choice(C, size=n_sel, replace=False).tolist())
+        scale = 1.0 / math.sqrt(D)
+        o, lse = O.hybrid_unit(q, K, V, Kg, Vg, chunks, L, scale)
+        Ke, Ve = np.concatenate([K, Kg]), np.concatenate([V, Vg])
+        keep = np.zeros(T + C, dtype=bool)
+        keep[T:] = True
+        for c in chunks:
+            keep[c * L:(c + 1) * L] = True
+        mask = np.broadcast_to(keep, (G, 1, T + C))
+        ref = _sdpa(q[:, None, :], np.broadcast_to(Ke, (G, T + C, D)),
+                    np.broadcast_to(Ve, (G, T + C, D)), mask=mask, scale=scale)[:, 0]
+        assert np.allclose(o, ref, rtol=0, atol=1e-12), np.abs(o - ref).max()
+        logits = torch.as_tensor(q @ Ke.T * scale)
+        logits[:, ~torch.as_tensor(keep)] = -math.inf
+        assert np.allclose(lse, torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- summaries / scores
 
 def check_summary_closed_form():
@@ -406,5 +446,5 @@ ALL_CHECKS = [
     check_topk_union_golden, check_topk_union_brute_force, check_per_head_scores,
     check_topp_golden, check_topp_invariants, check_hier_golden, check_hier_all_metas_is_flat,
     check_meta_linearity, check_merge_closed_form, check_partition,
-    check_prefill_dense_causal, check_prefill_masked,
+    check_prefill_dense_causal, check_prefill_masked, check_hybrid_golden, check_hybrid_vs_sdpa,
 ]

@@ -15,7 +15,7 @@ _orig = {name: getattr(O, name) for name in
          ["attend", "select_topk", "select_topp", "score_chunks", "lse_merge",
           "causal_attend", "meta_summaries", "chunk_summaries", "select_hier",
           "forced_set", "topp_probs", "decode_partition", "tile_mean_q",
-          "select_topk_union", "score_chunks_per_head"]}
+          "select_topk_union", "score_chunks_per_head", "hybrid_unit"]}
 
 
 def attend_no_scale(q, K, V, tokens, scale):
@@ -174,6 +174,21 @@ def per_head_scores_group_summed(q_group, summ_unit, proj=None):
     return np.repeat(per.sum(axis=0, keepdims=True), per.shape[0], axis=0)
 
 
+def hybrid_selected_gists_only(q, K, V, Kg, Vg, chunks, L, scale):
+    sel = sorted(chunks)
+    return _orig["hybrid_unit"](q, K, V, np.asarray(Kg)[sel], np.asarray(Vg)[sel], chunks, L,
+                                scale)
+
+
+def hybrid_no_gists(q, K, V, Kg, Vg, chunks, L, scale):
+    return O.decode_unit(q, K, V, chunks, L, scale)
+
+
+def hybrid_gist_logits_unscaled(q, K, V, Kg, Vg, chunks, L, scale):
+    return _orig["hybrid_unit"](q, K, V, np.asarray(Kg, dtype=np.float64) / scale, Vg, chunks,
+                                L, scale)
+
+
 MUTANTS = [
     ("attend", attend_no_scale),
     ("attend", attend_no_max_shift_wrong_lse),
@@ -201,6 +216,9 @@ MUTANTS = [
     ("select_topk_union", union_first_head_only),
     ("select_topk_union", union_of_group_sum),
     ("score_chunks_per_head", per_head_scores_group_summed),
+    ("hybrid_unit", hybrid_selected_gists_only),
+    ("hybrid_unit", hybrid_no_gists),
+    ("hybrid_unit", hybrid_gist_logits_unscaled),
 ]
 
 
