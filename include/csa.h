@@ -310,6 +310,34 @@ CSA_API csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K
                                                     int num_parts, void* out, csa_dtype out_dtype,
                                                     float* lse_out, csa_stream stream);
 
+/* ---------------------------------------------------------------- hybrid context
+ * The merged decode over the hybrid context of the SSA summary (sections
+ * "방법론" and "기술 상세": K_hybrid / V_hybrid are the gist KV together with
+ * the raw KV of the selected chunks, attended with standard attention): each
+ * sparse unit's query heads attend, in one softmax, over the raw tokens of
+ * its selected chunks and over the gist token of EVERY chunk of the unit
+ * (reading: the gist tokens stay in the context, as the summary's glossary
+ * entry "Selective Unfolding" describes; the raw tokens of the selected
+ * chunks come next to them).  Full-attention KV heads (head_full) attend
+ * over their raw tokens only.
+ *   Kg, Vg [B, Hkv, C, D] bf16, C = T / L: gist key / value of chunk c of
+ *   unit (b, h) at row c (the model's gist KV; the synthetic workloads use the
+ *   chunk means as a stand-in).  Same scale for gist and raw logits.
+ *   Other arguments, outputs, workspace and errors as
+ *   csa_sparse_decode_merged; bf16 caches only (CSA_ERR_UNSUPPORTED for
+ *   fp32).  The gist rows stream as ceil(C/L) extra chunks of each sparse
+ *   unit (K and V: 2*C*D*2 bytes per unit). */
+CSA_API csa_status csa_sparse_decode_merged_hybrid(const void* q, const void* K, const void* V,
+                                                   const void* Kg, const void* Vg,
+                                                   csa_dtype dtype, const int32_t* idx,
+                                                   const int32_t* count, int kmax,
+                                                   const uint8_t* head_full, int B, int Hq,
+                                                   int Hkv, int D, int64_t T, int L, float scale,
+                                                   int num_parts, void* workspace,
+                                                   int64_t workspace_bytes, void* out,
+                                                   csa_dtype out_dtype, float* lse_out,
+                                                   csa_stream stream);
+
 /* ---------------------------------------------------------------- a1-a6 in one call
  * A whole decode step: the selection (csa_score_select_topk,
  * csa_score_select_topk_union, csa_score_select_topp or csa_select_hier,
@@ -369,6 +397,10 @@ typedef struct csa_decode_step_desc {
   void* out;             /* [B, Hq, D] of out_dtype (output) */
   csa_dtype out_dtype;
   float* lse_out;        /* NULL or [B, Hq] (output) */
+  /* hybrid context (as csa_sparse_decode_merged_hybrid): NULL, NULL = off,
+   * else both [B, Hkv, T/L, D] bf16 gist keys and values */
+  const void* Kg;
+  const void* Vg;
 } csa_decode_step_desc;
 
 CSA_API csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream);

@@ -64,6 +64,9 @@ _SIGS = {
     "csa_decode_workspace_bytes": (_i64, [_i, _i, _i, _i, _i]),
     "csa_sparse_decode_merged": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i64,
                                       _i, _f, _i, _vp, _i64, _vp, _i, _vp, _vp]),
+    "csa_sparse_decode_merged_hybrid": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i,
+                                             _i, _i, _i, _i64, _i, _f, _i, _vp, _i64, _vp, _i,
+                                             _vp, _vp]),
     "csa_sparse_decode_merged_noalloc": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i,
                                               _i64, _i, _f, _i, _vp, _i, _vp, _vp]),
     "csa_lse_merge": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp]),
@@ -223,6 +226,18 @@ def csa_sparse_decode_merged(q, K, V, dtype, idx, count, kmax, head_full, B, Hq,
                                         _p(lse_out), _s(stream)))
 
 
+def csa_sparse_decode_merged_hybrid(q, K, V, Kg, Vg, dtype, idx, count, kmax, head_full, B, Hq,
+                                    Hkv, D, T, L, scale, num_parts, workspace, workspace_bytes,
+                                    out, out_dtype, lse_out, stream=None):
+    """The merged decode over the hybrid context: gist K/V rows [B, Hkv, T/L, D]
+    of every chunk plus the raw KV of the selected chunks (see include/csa.h)."""
+    _check(lib.csa_sparse_decode_merged_hybrid(_p(q), _p(K), _p(V), _p(Kg), _p(Vg), _dt(dtype),
+                                               _p(idx), _p(count), kmax, _p(head_full), B, Hq,
+                                               Hkv, D, T, L, scale, num_parts, _p(workspace),
+                                               workspace_bytes, _p(out), _dt(out_dtype),
+                                               _p(lse_out), _s(stream)))
+
+
 def csa_sparse_decode_merged_noalloc(q, K, V, dtype, idx, count, kmax, head_full, B, Hq, Hkv, D,
                                      T, L, scale, num_parts, out, out_dtype, lse_out, stream=None):
     """csa_sparse_decode_merged without a workspace: the library's built-in
@@ -249,6 +264,7 @@ class DecodeStepDesc(ctypes.Structure):
         ("idx", _vp), ("count", _vp), ("kmax", _i), ("n_p_out", _vp),
         ("num_parts", _i), ("workspace", _vp), ("workspace_bytes", _i64),
         ("out", _vp), ("out_dtype", _i), ("lse_out", _vp),
+        ("Kg", _vp), ("Vg", _vp),
     ]
 
 

@@ -424,21 +424,30 @@ int64_t csa_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int num_parts)
   return static_cast<int64_t>(workspace_layout(B, Hq, Hkv, D, P).total);
 }
 
-csa_status csa_sparse_decode_merged(const void* q, const void* K, const void* V, csa_dtype dtype,
-                                    const int32_t* idx, const int32_t* count, int kmax,
-                                    const uint8_t* head_full, int B, int Hq, int Hkv, int D,
-                                    int64_t T, int L, float scale, int num_parts, void* workspace,
-                                    int64_t workspace_bytes, void* out, csa_dtype out_dtype,
-                                    float* lse_out, csa_stream stream) {
+}  // extern "C"
+
+namespace {
+// csa_sparse_decode_merged, with the hybrid context when Kg/Vg are given.
+csa_status merged_decode(const void* q, const void* K, const void* V, const void* Kg,
+                         const void* Vg, csa_dtype dtype, const int32_t* idx,
+                         const int32_t* count, int kmax, const uint8_t* head_full, int B, int Hq,
+                         int Hkv, int D, int64_t T, int L, float scale, int num_parts,
+                         void* workspace, int64_t workspace_bytes, void* out,
+                         csa_dtype out_dtype, float* lse_out, csa_stream stream, bool hybrid) {
   CSA_REQUIRE(valid_dtype(out_dtype), "out_dtype");
   CSA_TRY(decode_shape_checks(dtype, kmax, B, Hq, Hkv, D, T, L, scale, num_parts));
   CSA_SUPPORT(num_parts <= csa::kMergedMaxParts, "num_parts must be <= 256 for the merged decode");
+  if (hybrid) CSA_SUPPORT(dtype == CSA_BF16, "the hybrid context needs a bf16 cache");
   if (B == 0) return CSA_OK;
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
   int P = 0;
   CSA_TRY(decode_ptr_checks(q, K, V, idx, count, head_full, dtype == CSA_BF16, D, L, num_parts, l, &P));
   CSA_SUPPORT(P <= csa::kMergedMaxParts, "num_parts must be <= 256 for the merged decode");
+  if (hybrid) {
+    CSA_TRY(check_ptr(Kg, "Kg"));
+    CSA_TRY(check_ptr(Vg, "Vg"));
+  }
   const WorkspaceLayout w = workspace_layout(B, Hq, Hkv, D, P);
   CSA_REQUIRE(workspace_bytes >= static_cast<int64_t>(w.total),
               "workspace smaller than csa_decode_workspace_bytes()");
@@ -447,12 +456,43 @@ csa_status csa_sparse_decode_merged(const void* q, const void* K, const void* V,
   CSA_TRY(check_ptr(lse_out, "lse_out", false));
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   csa::MergeOut m{reinterpret_cast<int*>(ws + w.counters), out, out_dtype == CSA_BF16, lse_out};
+  if (hybrid) {
+    m.Kg = Kg;
+    m.Vg = Vg;
+  }
   std::string why;
   cudaError_t e = csa::launch_decode(l, q, K, V, dtype == CSA_BF16, idx, count, kmax, head_full, B, Hq,
                                      Hkv, D, T, L, scale, P, P, reinterpret_cast<float*>(ws + w.o),
                                      reinterpret_cast<float*>(ws + w.lse), &m, &why);
   if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
-  return finish(e, "merged sparse decode launch");
+  return finish(e, hybrid ? "hybrid merged decode launch" : "merged sparse decode launch");
+}
+}  // namespace
+
+extern "C" {
+
+csa_status csa_sparse_decode_merged(const void* q, const void* K, const void* V, csa_dtype dtype,
+                                    const int32_t* idx, const int32_t* count, int kmax,
+                                    const uint8_t* head_full, int B, int Hq, int Hkv, int D,
+                                    int64_t T, int L, float scale, int num_parts, void* workspace,
+                                    int64_t workspace_bytes, void* out, csa_dtype out_dtype,
+                                    float* lse_out, csa_stream stream) {
+  return merged_decode(q, K, V, nullptr, nullptr, dtype, idx, count, kmax, head_full, B, Hq, Hkv,
+                       D, T, L, scale, num_parts, workspace, workspace_bytes, out, out_dtype,
+                       lse_out, stream, false);
+}
+
+csa_status csa_sparse_decode_merged_hybrid(const void* q, const void* K, const void* V,
+                                           const void* Kg, const void* Vg, csa_dtype dtype,
+                                           const int32_t* idx, const int32_t* count, int kmax,
+                                           const uint8_t* head_full, int B, int Hq, int Hkv,
+                                           int D, int64_t T, int L, float scale, int num_parts,
+                                           void* workspace, int64_t workspace_bytes, void* out,
+                                           csa_dtype out_dtype, float* lse_out,
+                                           csa_stream stream) {
+  return merged_decode(q, K, V, Kg, Vg, dtype, idx, count, kmax, head_full, B, Hq, Hkv, D, T, L,
+                       scale, num_parts, workspace, workspace_bytes, out, out_dtype, lse_out,
+                       stream, true);
 }
 
 namespace {
@@ -577,6 +617,11 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
   CSA_TRY(check_ptr(d->workspace, "workspace"));
   CSA_TRY(check_ptr(d->out, "out"));
   CSA_TRY(check_ptr(d->lse_out, "lse_out", false));
+  const bool hybrid = d->Kg != nullptr || d->Vg != nullptr;
+  if (hybrid) {  // both or neither
+    CSA_TRY(check_ptr(d->Kg, "Kg"));
+    CSA_TRY(check_ptr(d->Vg, "Vg"));
+  }
   const int C = static_cast<int>(d->T / d->L);
   // the selection (validates its own arguments before launching)
   csa_status st;
@@ -600,6 +645,10 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
   uint8_t* ws = static_cast<uint8_t*>(d->workspace);
   csa::MergeOut m{reinterpret_cast<int*>(ws + w.counters), d->out, d->out_dtype == CSA_BF16,
                   d->lse_out, true, late};
+  if (hybrid) {
+    m.Kg = d->Kg;
+    m.Vg = d->Vg;
+  }
   std::string why;
   cudaError_t e = csa::launch_decode(l, d->q, d->K, d->V, true, d->idx, d->count, d->kmax,
                                      d->head_full, d->B, d->Hq, d->Hkv, d->D, d->T, d->L, d->scale,

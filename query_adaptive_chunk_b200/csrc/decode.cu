@@ -75,6 +75,12 @@ struct DecodeParams {
   // phased: the last `late` CTAs of the grid take no phase-1 work (they can
   // only start once the selection's CTAs have left their SMs)
   int late;
+  // hybrid context (bf16 merged): every sparse unit also attends over its
+  // gist rows, gist_rows (= C) per unit in [B*Hkv*gist_rows, D] bf16 tensors,
+  // streamed as n_gist = ceil(gist_rows / L) extra chunks after its selected
+  // ones (the last one ragged, its rows past gist_rows masked); 0 = off
+  int n_gist;
+  int gist_rows;
 };
 
 // Unit sets of a phase: 0 = every unit, 1 = full-head units, 2 = sparse units.
@@ -93,7 +99,7 @@ __device__ __forceinline__ int unit_count(const DecodeParams& p, int u, int mode
     dev_flag(p.err, DEV_BAD_INDEX);
     n = max(0, min(n, p.kmax));
   }
-  return n;
+  return n + p.n_gist;  // a sparse unit's gist chunks come after its selected ones
 }
 
 __device__ __forceinline__ int unit_chunk(const DecodeParams& p, int u, int pos) {
@@ -104,6 +110,18 @@ __device__ __forceinline__ int unit_chunk(const DecodeParams& p, int u, int pos)
     c = 0;
   }
   return c;
+}
+
+// Row of the chunk at position pos of unit u (n = the unit's chunk count):
+// the raw K/V row of a selected (or, for a full unit, every) chunk, or for a
+// hybrid unit's gist chunk j the gist row, encoded as -(row + 1).
+__device__ __forceinline__ int unit_row(const DecodeParams& p, int u, int pos, int n, int L) {
+  if (p.n_gist > 0 && !(p.head_full != nullptr && p.head_full[u % p.Hkv])) {
+    const int j = pos - (n - p.n_gist);
+    if (j >= 0) return -(u * p.gist_rows + j * L) - 1;
+  }
+  const int c = unit_chunk(p, u, pos);
+  return static_cast<int>(u * p.T + static_cast<int64_t>(c) * L);
 }
 
 // prefix[0..U] of the effective chunk counts of a phase (all threads of the block).
@@ -606,6 +624,8 @@ template <int D, int L>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmKg,
+                       const __grid_constant__ CUtensorMap tmVg,
                        const __grid_constant__ DecodeParams p) {
   using Sh = DecodeShape<D, L>;
   constexpr int NS = Sh::NS;
@@ -652,6 +672,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
+    if (p.n_gist > 0) {
+      prefetch_tensormap(&tmKg);
+      prefetch_tensormap(&tmVg);
+    }
   }
   build_prefix(p, prefix, scan_sh, p.phased ? 1 : 0);  // ends with __syncthreads (also publishes the barriers)
   const int n_phase = p.phased ? 2 : 1;
@@ -686,8 +710,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         int row = 0, qu = -1;
         if (g < bnd) {
           const int u = unit_of(pre, p.U, g);
-          const int c = unit_chunk(p, u, static_cast<int>(g - pre[u]));
-          row = static_cast<int>(u * p.T + static_cast<int64_t>(c) * L);
+          row = unit_row(p, u, static_cast<int>(g - pre[u]), pre[u + 1] - pre[u], L);
           if (g == a || g == pre[u]) qu = u;  // first chunk of a unit here: its q rides along
         }
         const int nb = static_cast<int>(bnd - g0 < 32 ? bnd - g0 : 32);
@@ -709,10 +732,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 bulk_load(sbase + Y.q_off + s * Sh::QSLOT_BYTES, qg + qrow * D, q_bytes, fb);
               }
               const uint32_t dst = sbase + s * Sh::STAGE_BYTES;
+              const bool gist = row_j < 0;  // rows of a ragged last gist chunk past
+              const int r = gist ? -row_j - 1 : row_j;  // the tensor read as zeros
+              const CUtensorMap* mk = gist ? &tmKg : &tmK;
+              const CUtensorMap* mv = gist ? &tmVg : &tmV;
 #pragma unroll
               for (int bx = 0; bx < NBOX; ++bx) {
-                tma_load_2d_hint(dst + bx * Sh::BOX_BYTES, &tmK, bx * 64, row_j, fb, kv_policy);
-                tma_load_2d_hint(dst + Sh::KV_BYTES + bx * Sh::BOX_BYTES, &tmV, bx * 64, row_j, fb,
+                tma_load_2d_hint(dst + bx * Sh::BOX_BYTES, mk, bx * 64, r, fb, kv_policy);
+                tma_load_2d_hint(dst + Sh::KV_BYTES + bx * Sh::BOX_BYTES, mv, bx * 64, r, fb,
                                  kv_policy);
               }
             }
@@ -846,6 +873,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   float o[KS][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   int cur_u = -1, nflush = 0;
+  bool cur_full = false;  // hybrid launches: the current unit is a full-attention one
   bool ok = true;
 
   // Hand this warp's (m, l, O) of unit u to the epilogue warp and go on.
@@ -919,6 +947,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           break;
         }
         cur_u = unit_of(pre, p.U, g);
+        cur_full = p.n_gist > 0 && p.head_full != nullptr && p.head_full[cur_u % p.Hkv];
         // the unit's q arrived with this stage
         const __nv_bfloat16* qs =
             reinterpret_cast<const __nv_bfloat16*>(smem + Y.q_off + s * Sh::QSLOT_BYTES);
@@ -961,6 +990,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
         }
       }
+      if (p.n_gist > 0 && !cur_full) {
+        // a hybrid unit's last gist chunk is ragged: rows past its gist rows
+        // (the next unit's, or zeros past the tensor) take no part
+        const int n_all = pre[cur_u + 1] - pre[cur_u];
+        const int j = static_cast<int>(g - pre[cur_u]) - (n_all - p.n_gist);
+        const int valid = j >= 0 ? p.gist_rows - j * L : L;
+        if (valid < L) {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (tok0 + mt * 16 + (lane >> 2) + (e >> 1) * 8 >= valid) sc[mt][e] = -INFINITY;
+        }
+      }
       // online softmax (log2 domain), per head hA / hB of this lane
       float cm0 = -INFINITY, cm1 = -INFINITY;
 #pragma unroll
@@ -976,15 +1019,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, x));
       }
       const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
-      const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+      // exponent reference: 0 while every row this warp has seen was masked
+      // (max -inf), so that no -inf - -inf arises
+      const float rf0 = mn0 == -INFINITY ? 0.f : mn0, rf1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = fast_exp2(m0 - rf0), al1 = fast_exp2(m1 - rf1);
       m0 = mn0;
       m1 = mn1;
       uint32_t pb[MT][2];
       float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        const float p0 = fast_exp2(sc[mt][0] - mn0), p1 = fast_exp2(sc[mt][1] - mn1);
-        const float p2 = fast_exp2(sc[mt][2] - mn0), p3 = fast_exp2(sc[mt][3] - mn1);
+        const float p0 = fast_exp2(sc[mt][0] - rf0), p1 = fast_exp2(sc[mt][1] - rf1);
+        const float p2 = fast_exp2(sc[mt][2] - rf0), p3 = fast_exp2(sc[mt][3] - rf1);
         ps0 += p0 + p2;
         ps1 += p1 + p3;
         pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
@@ -1236,11 +1282,19 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
 
 template <int D, int L>
 cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, const void* V,
-                        int B, int Hkv, int P, std::string* why) {
-  CUtensorMap tmK, tmV;
+                        const void* Kg, const void* Vg, int B, int Hkv, int P, std::string* why) {
+  CUtensorMap tmK, tmV, tmKg, tmVg;
   const uint64_t rows = static_cast<uint64_t>(B) * Hkv * p.T;
   if (!make_tmap_bf16_2d(&tmK, K, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tmV, V, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+  if (p.n_gist > 0) {  // the gist rows: [B*Hkv*gist_rows, D], the same boxes
+    const uint64_t grows = static_cast<uint64_t>(B) * Hkv * p.gist_rows;
+    if (!make_tmap_bf16_2d(&tmKg, Kg, grows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tmVg, Vg, grows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+  } else {
+    tmKg = tmK;
+    tmVg = tmV;
+  }
   const size_t sh = dec_layout(D, L, p.G, p.U).total;
   if (sh > kMaxDynSmem) {
     *why = "too many (batch, KV head) units for one decode launch: " + std::to_string(p.U);
@@ -1251,7 +1305,7 @@ cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, c
                                        static_cast<int>(sh));
   if (e != cudaSuccess) return e;
   if (!p.phased) {
-    fn<<<P, kDecodeThreads, sh, l.stream>>>(tmK, tmV, p);
+    fn<<<P, kDecodeThreads, sh, l.stream>>>(tmK, tmV, tmKg, tmVg, p);
     return cudaGetLastError();
   }
   // programmatic dependent launch: the grid may start while the selection
@@ -1267,7 +1321,7 @@ cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fn, tmK, tmV, p);
+  return cudaLaunchKernelEx(&cfg, fn, tmK, tmV, tmKg, tmVg, p);
 }
 
 }  // namespace
@@ -1297,6 +1351,10 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
     p.lse_out = merge->lse_out;
     p.phased = (merge->phased && bf16) ? 1 : 0;
     p.late = p.phased ? merge->late : 0;
+    if (merge->Kg != nullptr && bf16) {
+      p.gist_rows = static_cast<int>(T / L);
+      p.n_gist = (p.gist_rows + L - 1) / L;
+    }
   }
   p.D = D;
   p.q = q;
@@ -1334,10 +1392,12 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
     }
     return cudaGetLastError();
   }
-  if (D == 128 && L == 128) return launch_bf16<128, 128>(l, p, K, V, B, Hkv, P, why);
-  if (D == 128 && L == 64) return launch_bf16<128, 64>(l, p, K, V, B, Hkv, P, why);
-  if (D == 64 && L == 128) return launch_bf16<64, 128>(l, p, K, V, B, Hkv, P, why);
-  return launch_bf16<64, 64>(l, p, K, V, B, Hkv, P, why);
+  const void* Kg = merge != nullptr ? merge->Kg : nullptr;
+  const void* Vg = merge != nullptr ? merge->Vg : nullptr;
+  if (D == 128 && L == 128) return launch_bf16<128, 128>(l, p, K, V, Kg, Vg, B, Hkv, P, why);
+  if (D == 128 && L == 64) return launch_bf16<128, 64>(l, p, K, V, Kg, Vg, B, Hkv, P, why);
+  if (D == 64 && L == 128) return launch_bf16<64, 128>(l, p, K, V, Kg, Vg, B, Hkv, P, why);
+  return launch_bf16<64, 64>(l, p, K, V, Kg, Vg, B, Hkv, P, why);
 }
 
 cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_part, int rows,

@@ -73,6 +73,10 @@ struct MergeOut {
   // phased: CTAs at the end of the grid that take no full-head work (they
   // start only after the selection's CTAs leave their SMs)
   int late = 0;
+  // bf16 hybrid context: gist K/V rows [B, Hkv, C, D] (C = T / L) that every
+  // sparse unit attends over next to its selected chunks; null = off
+  const void* Kg = nullptr;
+  const void* Vg = nullptr;
 };
 constexpr int kMergedMaxParts = 256;
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,

@@ -556,6 +556,108 @@ def test_merged_decode_second_wave(csa):
                  out_bf16=True)
 
 
+def _hybrid_case(csa, B, Hkv, G, D, L, C, sets, full=(), num_parts=0, out_bf16=False,
+                 with_lse=True, seed=60, via_step=False):
+    """csa_sparse_decode_merged_hybrid against the oracle's hybrid context:
+    random bf16 gist rows (any gist KV is a valid input), every sparse unit
+    over all its gist rows plus its selected chunks, full units over their
+    raw chunks only."""
+    Hq, T = G * Hkv, C * L
+    dt = _dt("bf16")
+    q = _randn((B, Hq, D), seed, dt)
+    K = _randn((B, Hkv, T, D), seed + 1, dt)
+    V = _randn((B, Hkv, T, D), seed + 2, dt)
+    Kg = _randn((B, Hkv, C, D), seed + 3, dt)
+    Vg = _randn((B, Hkv, C, D), seed + 4, dt)
+    U = B * Hkv
+    kmax = max(1, max(len(s) for s in sets))
+    idx = torch.full((U, kmax), -1, dtype=torch.int32)
+    cnt = torch.zeros(U, dtype=torch.int32)
+    for u, st in enumerate(sets):
+        idx[u, :len(st)] = torch.tensor(sorted(st), dtype=torch.int32)
+        cnt[u] = len(st)
+    idx, cnt = idx.cuda(), cnt.cuda()
+    hf = None
+    if full:
+        hf = torch.zeros(Hkv, dtype=torch.uint8)
+        hf[list(full)] = 1
+        hf = hf.cuda()
+    scale = D ** -0.5
+    nbytes = csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    odt = torch.bfloat16 if out_bf16 else torch.float32
+    out = torch.full((B, Hq, D), float("nan"), device="cuda").to(odt)
+    lse = torch.full((B, Hq), float("nan"), device="cuda") if with_lse else None
+    for _ in range(2):  # the second call sees the counters the first left
+        csa.csa_sparse_decode_merged_hybrid(q, K, V, Kg, Vg, dt, idx, cnt, kmax, hf, B, Hq, Hkv,
+                                            D, T, L, scale, num_parts, ws, nbytes, out, odt, lse)
+        csa.csa_check_device_status()
+    qn = to_np(q)
+    Kc, Vc, Kgc, Vgc = K.cpu(), V.cpu(), Kg.cpu(), Vg.cpu()
+    for u, st in enumerate(sets):
+        b, h = divmod(u, Hkv)
+        rows = slice(h * G, (h + 1) * G)
+        got = out[b, rows].float().cpu().double().numpy()
+        if h in full:
+            ro, rl = O.decode_unit(qn[b, rows], to_np(Kc[b, h]), to_np(Vc[b, h]), range(C), L,
+                                   scale)
+        else:
+            ro, rl = O.hybrid_unit(qn[b, rows], to_np(Kc[b, h]), to_np(Vc[b, h]),
+                                   to_np(Kgc[b, h]), to_np(Vgc[b, h]), st, L, scale)
+        parity.assert_close(got, ro, "bf16", f"hybrid unit {u}")
+        if lse is not None:
+            assert np.abs(lse[b, rows].cpu().double().numpy() - rl).max() < 1e-3, u
+    return out
+
+
+@pytest.mark.parametrize("D,L,G,C,parts", [(128, 128, 4, 24, 0), (128, 64, 4, 150, 13),
+                                           (64, 64, 8, 40, 7), (64, 128, 2, 300, 256),
+                                           (128, 128, 1, 9, 3)])
+def test_hybrid_decode_shapes(csa, D, L, G, C, parts):
+    """Gist rows from one ragged chunk (C < L) to several with a ragged last
+    one (C % L != 0), GQA groups 1-8, few and many pieces."""
+    B, Hkv = 2, 3
+    rng = np.random.default_rng(D + L + G + C)
+    sets = [sorted(rng.choice(C, size=int(rng.integers(1, min(C, 14) + 1)),
+                              replace=False).tolist()) for _ in range(B * Hkv)]
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=parts)
+
+
+def test_hybrid_decode_edge_cases(csa):
+    """A unit with no selected chunk attends over its gist rows alone; full
+    heads ignore the gist rows; bf16 output; one piece; no lse output."""
+    B, Hkv, G, D, L, C = 1, 4, 4, 128, 64, 9
+    sets = [[], [0], [2, 5, 8], list(range(9))]
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=1)
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=200, out_bf16=True)
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, full=(2,), num_parts=7, with_lse=False)
+    _hybrid_case(csa, 2, 8, 4, 128, 128, 96, [list(range(0, 96, 5))] * 16, full=(0, 1))
+
+
+def test_hybrid_decode_rejects_fp32_and_unaligned(csa):
+    """The hybrid context needs a bf16 cache and 16-byte aligned gist rows;
+    a rejected call enqueues nothing."""
+    from query_adaptive_chunk_b200.csa import CsaError
+    B, Hq, Hkv, D, L, C = 1, 4, 1, 64, 64, 4
+    q = torch.zeros(B, Hq, D, device="cuda")
+    K = torch.zeros(B, Hkv, C * L, D, device="cuda")
+    g = torch.zeros(B, Hkv, C, D, device="cuda")
+    idx = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+    cnt = torch.ones(1, dtype=torch.int32, device="cuda")
+    nbytes = csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, 0)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    out = torch.zeros(B, Hq, D, device="cuda")
+    with pytest.raises(CsaError):
+        csa.csa_sparse_decode_merged_hybrid(q, K, K, g, g, torch.float32, idx, cnt, 1, None, B, Hq,
+                                            Hkv, D, C * L, L, 0.1, 0, ws, nbytes, out,
+                                            torch.float32, None)
+    qb, Kb, gb = q.bfloat16(), K.bfloat16(), g.bfloat16()
+    with pytest.raises(CsaError):
+        csa.csa_sparse_decode_merged_hybrid(qb, Kb, Kb, gb.view(-1)[1:].data_ptr(), gb, torch.bfloat16,
+                                            idx, cnt, 1, None, B, Hq, Hkv, D, C * L, L, 0.1, 0, ws,
+                                            nbytes, out, torch.float32, None)
+
+
 def test_merged_decode_mixed_heads(csa):
     B, Hkv, G, D, L, C = 1, 8, 4, 128, 128, 96
     rng = np.random.default_rng(7)
