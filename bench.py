@@ -183,12 +183,13 @@ def decoder_for(w, inp):
     from query_adaptive_chunk_b200.steps import SparseDecoder
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
                          n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
-                         budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta)
+                         budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta,
+                         hybrid=w.hybrid)
 
 
 def selected_bytes(w, dec) -> tuple:
     """(selected KV bytes, summary bytes) the step must read, from the actual
-    index counts (full heads: every chunk)."""
+    index counts (full heads: every chunk; hybrid: plus the gist rows)."""
     cnt = dec.count.cpu().tolist()
     elt = 2 if w.dtype == "bf16" else 4
     n = 0
@@ -196,6 +197,8 @@ def selected_bytes(w, dec) -> tuple:
         n += w.C if (u % w.Hkv) in w.full_heads else c
     kv = n * w.L * w.D * elt * 2
     U_sparse = sum(1 for u in range(w.B * w.Hkv) if (u % w.Hkv) not in w.full_heads)
+    if w.hybrid:  # every sparse unit also reads one gist key and value row per chunk
+        kv += U_sparse * w.C * w.D * elt * 2
     if w.select == "hier":
         summ = U_sparse * (w.C // w.Gm + w.top_meta * w.Gm) * w.D * 4
     else:
@@ -499,7 +502,8 @@ def run_ours(args):
 def other_workloads(args, flush, peaks):
     out = {}
     steps = max(5, args.steps // 2)
-    for w in (synth.TOPK_32K, synth.HIER_1M, synth.TINY_F32, synth.TOPK_UNION_32K):
+    for w in (synth.TOPK_32K, synth.HIER_1M, synth.TINY_F32, synth.TOPK_UNION_32K,
+              synth.HYBRID_TOPK_32K):
         r = time_decode(w, steps, args.warmup, flush)
         us = 1000 * statistics.mean(r["step_ms"])
         dus = 1000 * statistics.mean(r["decode_ms"])

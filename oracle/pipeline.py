@@ -36,12 +36,14 @@ def unit_summaries(K_unit, L: int, proj=None, block_chunks: int = 2048) -> np.nd
 def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_local: int,
                 k_free: int = 0, proj=None, p: float = 0.0, budget: int = 0,
                 full_heads=(), Gm: int = 0, top_meta: int = 0, units=None,
-                with_attention: bool = True) -> dict:
+                with_attention: bool = True, gist=None) -> dict:
     """One decode step of the units (b, kvh) listed (default: all).
 
     q [B, Hq, D]; K, V [B, Hkv, T, D].  Returns a dict with, per unit, the
     ascending chunk set, the boundary gap(s), n_p for top-p, and when
-    ``with_attention`` the output rows o [G, D] and lse [G]."""
+    ``with_attention`` the output rows o [G, D] and lse [G].  gist = (Kg, Vg),
+    each [B, Hkv, T // L, D]: the sparse units attend over the hybrid context
+    (their gist rows plus the raw KV of their chunks, ``hybrid_unit``)."""
     B, Hkv, T, D = K.shape
     Hq = q.shape[1]
     G = Hq // Hkv
@@ -77,7 +79,12 @@ def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_lo
             raise ValueError(select)
         res["sets"][(b, h)] = chunks
         res["gap"][(b, h)] = gap
-        if with_attention:
+        if with_attention and gist is not None and h not in tuple(full_heads):
+            o, lse = O.hybrid_unit(qg, to_np(K[b, h]), to_np(V[b, h]), to_np(gist[0][b, h]),
+                                   to_np(gist[1][b, h]), chunks, L, scale)
+            res["o"][(b, h)] = o
+            res["lse"][(b, h)] = lse
+        elif with_attention:
             tok = O.chunk_tokens(chunks, L)
             Kt = to_np(K[b, h][_index(K, tok)])
             Vt = to_np(V[b, h][_index(V, tok)])

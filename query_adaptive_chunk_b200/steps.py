@@ -30,13 +30,18 @@ class SparseDecoder:
     and the merged split-K decode; fused=False runs the separate calls
     (score, select, decode, merge).  With a bf16 cache and fused=True,
     ``step`` is one call of csa_decode_step, whose decode streams the
-    full-attention heads while the selection runs."""
+    full-attention heads while the selection runs.
+
+    hybrid=True (bf16, fused): every sparse head also attends over one gist
+    key/value row per chunk (the hybrid context of SSA).  The gist rows are
+    built here with the cache, as the chunk means of K and V in bf16: the
+    stand-in for a trained model's gist KV."""
 
     def __init__(self, K: torch.Tensor, V: torch.Tensor, *, Hq: int, L: int, select: str,
                  n_sink: int, n_local: int, k_free: int = 0, proj: torch.Tensor | None = None,
                  p: float = 0.9, budget: int = 256, full_heads=(), Gm: int = 0, top_meta: int = 0,
                  scale: float | None = None, num_parts: int = 0, out_dtype=torch.float32,
-                 fused: bool = True):
+                 fused: bool = True, hybrid: bool = False):
         assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
         self.K, self.V = K, V
         B, Hkv, T, D = K.shape
@@ -57,6 +62,14 @@ class SparseDecoder:
         if select == "hier":
             self.meta = torch.empty(B, Hkv, self.C // Gm, Ds, dtype=torch.float32, device=dev)
             csa.csa_meta_summaries(self.summ, B, Hkv, self.C, Ds, Gm, self.meta)
+        self.Kg = self.Vg = None
+        if hybrid:
+            assert fused and K.dtype == torch.bfloat16, "the hybrid context needs a fused bf16 decode"
+            means = torch.empty(B, Hkv, self.C, D, dtype=torch.float32, device=dev)
+            csa.csa_chunk_summaries(K, self.dtype, B, Hkv, T, D, L, None, 0, means)
+            self.Kg = means.to(torch.bfloat16)
+            csa.csa_chunk_summaries(V, self.dtype, B, Hkv, T, D, L, None, 0, means)
+            self.Vg = means.to(torch.bfloat16)
         self.head_full = None
         if full_heads:
             hf = torch.zeros(Hkv, dtype=torch.uint8)
@@ -94,7 +107,7 @@ class SparseDecoder:
                 n_local=n_local, logit_scale=1.0 / math.sqrt(D), p=p, budget=budget, idx=self.idx,
                 count=self.count, kmax=self.kmax, n_p_out=self.n_p, num_parts=num_parts,
                 workspace=self.workspace, workspace_bytes=self.ws_bytes, out=self.out,
-                out_dtype=self.out.dtype, lse_out=self.lse)
+                out_dtype=self.out.dtype, lse_out=self.lse, Kg=self.Kg, Vg=self.Vg)
 
     def select_chunks(self, q: torch.Tensor, stream=None):
         """Score + select: fills self.idx / self.count (and self.n_p for top-p)."""
@@ -138,6 +151,13 @@ class SparseDecoder:
     def attend(self, q: torch.Tensor, stream=None):
         """Sparse split-K decode over the current index lists, then the LSE merge
         (one launch when fused)."""
+        if self.Kg is not None:
+            csa.csa_sparse_decode_merged_hybrid(q, self.K, self.V, self.Kg, self.Vg, self.dtype,
+                                                self.idx, self.count, self.kmax, self.head_full,
+                                                self.B, self.Hq, self.Hkv, self.D, self.T, self.L,
+                                                self.scale, self.P, self.workspace, self.ws_bytes,
+                                                self.out, _dt(self.out), self.lse, stream=stream)
+            return
         if self.fused:
             csa.csa_sparse_decode_merged(q, self.K, self.V, self.dtype, self.idx, self.count,
                                          self.kmax, self.head_full, self.B, self.Hq, self.Hkv,

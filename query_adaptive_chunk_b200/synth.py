@@ -65,6 +65,7 @@ class DecodeWorkload:
     full_heads: tuple = ()  # KV heads that attend to every chunk
     Gm: int = 0  # hierarchical: chunks per meta-chunk
     top_meta: int = 0  # hierarchical: meta-chunks kept
+    hybrid: bool = False  # sparse heads also attend over one gist row per chunk
 
     @property
     def C(self) -> int:
@@ -159,7 +160,12 @@ PREFILL_32K = PrefillWorkload(
 TOPK_UNION_32K = dataclasses.replace(TOPK_32K, name="topk_union_decode_bf16_ctx32k", seed=6,
                                      select="topk_union")
 
-DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M, TOPK_UNION_32K)
+# SSA's hybrid context: the 32K top-k step with every chunk's gist row in the
+# context of each sparse head (8 extra 64-row chunks per unit)
+HYBRID_TOPK_32K = dataclasses.replace(TOPK_32K, name="hybrid_topk_decode_bf16_ctx32k", seed=7,
+                                      hybrid=True)
+
+DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M, TOPK_UNION_32K, HYBRID_TOPK_32K)
 ALL_WORKLOADS = DECODE_WORKLOADS + (PREFILL_32K,)
 
 

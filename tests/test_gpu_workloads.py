@@ -20,7 +20,7 @@ def _decoder(w, inp, fused=True):
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
                          n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
                          budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta,
-                         fused=fused)
+                         fused=fused, hybrid=w.hybrid)
 
 
 def run_and_check(w, units=None, fused=True):
@@ -34,7 +34,8 @@ def run_and_check(w, units=None, fused=True):
     ref = OP.decode_step(inp["q"], inp["K"], inp["V"], L=w.L, scale=w.scale, select=w.select,
                          n_sink=w.n_sink, n_local=w.n_local, k_free=w.k_free,
                          proj=inp.get("proj"), p=w.p, budget=w.budget, full_heads=w.full_heads,
-                         Gm=w.Gm, top_meta=w.top_meta, units=units)
+                         Gm=w.Gm, top_meta=w.top_meta, units=units,
+                         gist=(dec.Kg, dec.Vg) if w.hybrid else None)
     gsets_all = parity.gpu_sets(dec.idx, dec.count)
     sparse = [u for u in units if u[1] not in w.full_heads]
     uidx = {u: i for i, u in enumerate(all_units)}
@@ -48,6 +49,10 @@ def run_and_check(w, units=None, fused=True):
         gset = list(range(w.C)) if h in w.full_heads else gsets_all[uidx[(b, h)]]
         if gset == ref["sets"][(b, h)]:
             ro, rl = ref["o"][(b, h)], ref["lse"][(b, h)]
+        elif w.hybrid:  # near-tie: the hybrid context over the GPU's own set
+            ro, rl = O.hybrid_unit(to_np(inp["q"][b, h * G:(h + 1) * G]), to_np(inp["K"][b, h]),
+                                   to_np(inp["V"][b, h]), to_np(dec.Kg[b, h]),
+                                   to_np(dec.Vg[b, h]), gset, w.L, w.scale)
         else:  # near-tie: check attention over the GPU's own set
             ro, rl = O.decode_unit(to_np(inp["q"][b, h * G:(h + 1) * G]), to_np(inp["K"][b, h]),
                                    to_np(inp["V"][b, h]), gset, w.L, w.scale)
@@ -145,3 +150,35 @@ def test_topk_union_with_projection_and_full_head():
     w = dataclasses.replace(synth.TOPK_UNION_32K.scaled(B=1, T=16384, planted=4),
                             name="topk_union_proj_mixed", proj_rank=16, full_heads=(3,))
     run_and_check(w)
+
+
+def test_hybrid_topk_decode_reduced():
+    """SSA's hybrid context through the one-call step: each sparse head over
+    its top-k chunks plus the gist row of every chunk (chunk means of K and V
+    as the gist stand-in, built with the cache)."""
+    run_and_check(synth.HYBRID_TOPK_32K.scaled(B=2, T=8192))
+
+
+def test_hybrid_topk_decode_full_size():
+    run_and_check(synth.HYBRID_TOPK_32K)
+
+
+def test_hybrid_with_projection_full_head_and_topp():
+    """Hybrid context next to a full-attention head, with projected top-p
+    scores (the full head attends over its raw tokens only)."""
+    import dataclasses
+    w = dataclasses.replace(synth.TOPP_128K.scaled(B=1, T=16384), name="hybrid_topp_mixed",
+                            seed=17, hybrid=True)
+    run_and_check(w)
+
+
+def test_hybrid_separate_decode_call_matches_step():
+    """csa_sparse_decode_merged_hybrid over the step's own index lists gives
+    the step's output (same chunk sets, same gist rows)."""
+    from query_adaptive_chunk_b200 import csa
+    w = synth.HYBRID_TOPK_32K.scaled(B=2, T=8192)
+    dec, inp = run_and_check(w)
+    out_step = dec.out.clone()
+    dec.attend(inp["q"])
+    csa.csa_check_device_status()
+    assert (dec.out - out_step).abs().max().item() < 1e-5
