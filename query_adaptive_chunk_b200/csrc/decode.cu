@@ -562,42 +562,51 @@ __device__ __forceinline__ int epilogue_unit(const DecodeParams& p, const float*
                                              int slot, int ns, bool final_flush, uint8_t* area,
                                              int area_bytes, uint32_t merge_bar,
                                              uint32_t fb_empty, int* pre_u, int* pre_ns) {
+  static_assert(kConsumerWarps == 4, "four partials per head");
   const int lane = threadIdx.x & 31, G = p.G;
   const float* fm = fo + kConsumerWarps * G * D;
   const float* fl = fm + kConsumerWarps * 8;
-  const int b = u / p.Hkv, h = u % p.Hkv;
+  const int64_t row0 = static_cast<int64_t>(u / p.Hkv) * p.Hq + (u % p.Hkv) * G;
   const bool direct = p.merged && ns == 1;  // the only split: it is the output
-  // per head g = lane: max over the warps, warp weights, total sum
-  float M = -INFINITY, Ls = 0.f, scw[kConsumerWarps];
+  // Lane g < G: head g's max over the warps, and the weights of the warps'
+  // partials normalised by the total sum; it also writes the head's lse.
+  float wn[kConsumerWarps] = {0.f, 0.f, 0.f, 0.f};
   if (lane < G) {
+    float M = -INFINITY, Ls = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + lane]);
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      scw[w] = exp2f(fm[w * 8 + lane] - M);
-      Ls += fl[w * 8 + lane] * scw[w];
+      wn[w] = exp2f(fm[w * 8 + lane] - M);
+      Ls += fl[w * 8 + lane] * wn[w];
     }
+    const float inv = 1.0f / Ls;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) wn[w] *= inv;
+    const float lse = (M + log2f(Ls)) * kLn2;
+    if (!direct)
+      p.lse_part[(row0 + lane) * p.max_splits + slot] = lse;
+    else if (p.lse_out)
+      p.lse_out[row0 + lane] = lse;
   }
-  for (int g = 0; g < G; ++g) {
-    const float Mg = __shfl_sync(0xffffffffu, M, g), Lg = __shfl_sync(0xffffffffu, Ls, g);
-    float sc[kConsumerWarps];
+  // Every lane: columns lane + 32 j of every head, all independent (the
+  // weights of all heads first, then the loads and stores).
+  float wg[8][kConsumerWarps];
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) sc[w] = __shfl_sync(0xffffffffu, scw[w], g);
-    const float inv = 1.0f / Lg;
-    const int64_t row = static_cast<int64_t>(b) * p.Hq + h * G + g;
-    for (int d = lane; d < D; d += 32) {
-      float acc = 0.f;
+  for (int g = 0; g < 8; ++g)
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) acc += fo[(w * G + g) * D + d] * sc[w];
-      if (direct) store_out(p, row * D + d, acc * inv);
-      else p.o_part[(row * p.max_splits + slot) * D + d] = acc * inv;
-    }
-    if (lane == 0) {
-      const float lse = (Mg + log2f(Lg)) * kLn2;
-      if (direct) {
-        if (p.lse_out) p.lse_out[row] = lse;
-      } else {
-        p.lse_part[row * p.max_splits + slot] = lse;
+    for (int w = 0; w < kConsumerWarps; ++w) wg[g][w] = __shfl_sync(0xffffffffu, wn[w], g);
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    if (g < G) {
+      const int64_t row = row0 + g;
+#pragma unroll
+      for (int d = lane; d < D; d += 32) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) acc += fo[(w * G + g) * D + d] * wg[g][w];
+        if (direct) store_out(p, row * D + d, acc);
+        else p.o_part[(row * p.max_splits + slot) * D + d] = acc;
       }
     }
   }
@@ -824,6 +833,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int u0 = unit_of(pre, p.U, a), u1 = unit_of(pre, p.U, bnd - 1);
       for (int u = u0; u <= u1 && ok; ++u) {
         if (pre[u + 1] <= pre[u]) continue;  // no chunk: never flushed
+        // the split's slot and count before the wait (64-bit divisions)
+        const int slot = split_slot(pre[u], a, blockIdx.x, N, P);
+        const int ns = split_count(pre[u], pre[u + 1], N, P);
         const int k = Y.nf == 2 ? (nseen & 1) : 0;
         const int use = Y.nf == 2 ? (nseen >> 1) : nseen;
         if (!warp_wait(fb_full + 8 * k, static_cast<uint32_t>(use) & 1u, p.err)) {
@@ -832,8 +844,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
         ++nseen;
         const float* fo = reinterpret_cast<const float*>(smem + Y.fb_off + k * Y.fb_bytes);
-        const int slot = split_slot(pre[u], a, blockIdx.x, N, P);
-        const int ns = split_count(pre[u], pre[u + 1], N, P);
         // the CTA's last flush: the consumers are done with the stage ring
         const bool final_flush = ph == n_phase - 1 && u == u1;
         int last = epilogue_unit<D>(p, fo, u, slot, ns, final_flush, smem, NS * Sh::STAGE_BYTES,
