@@ -184,7 +184,7 @@ def decoder_for(w, inp):
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
                          n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
                          budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta,
-                         hybrid=w.hybrid)
+                         hybrid=w.hybrid, rope_theta=w.rope_theta)
 
 
 def selected_bytes(w, dec) -> tuple:
@@ -503,7 +503,7 @@ def other_workloads(args, flush, peaks):
     out = {}
     steps = max(5, args.steps // 2)
     for w in (synth.TOPK_32K, synth.HIER_1M, synth.TINY_F32, synth.TOPK_UNION_32K,
-              synth.HYBRID_TOPK_32K):
+              synth.HYBRID_TOPK_32K, synth.ROPE_TOPK_32K):
         r = time_decode(w, steps, args.warmup, flush)
         us = 1000 * statistics.mean(r["step_ms"])
         dus = 1000 * statistics.mean(r["decode_ms"])

@@ -119,6 +119,23 @@ CSA_API csa_status csa_chunk_summaries(const void* K, csa_dtype dtype, int B, in
 CSA_API csa_status csa_meta_summaries(const float* summ, int B, int Hkv, int C, int Ds, int Gm,
                               float* meta, csa_stream stream);
 
+/* ---------------------------------------------------------------- RoPE
+ * Rotary position embedding, for the RoPE-aware split of the RTPurbo review
+ * (section 1, "Low-dimensional Projection": the scoring projection is taken
+ * before RoPE, which makes scores depend on distance): chunks are scored on
+ * the pre-RoPE keys and query (summaries of the pre-RoPE cache,
+ * csa_decode_step_desc.q_score), and attention runs on the rotated ones made
+ * here.  The pages do not write RoPE out; this is the rotate-half form:
+ * row r of x sits at position p = pos0 + (r mod period), and for i < D/2
+ *   y[r,i]     = x[r,i] cos(p w_i) - x[r,i+D/2] sin(p w_i)
+ *   y[r,i+D/2] = x[r,i+D/2] cos(p w_i) + x[r,i] sin(p w_i),  w_i = theta^(-2i/D).
+ * The angle is reduced modulo 2 pi in double precision.
+ *   x, y [rows, D] of `dtype` (y == x allowed); a K cache [B, H, T, D] is
+ *   rows = B*H*T with period T, pos0 0; a decode query [B, Hq, D] at position
+ *   t is rows = B*Hq with period 1, pos0 t.  D even, D <= 512, theta > 1. */
+CSA_API csa_status csa_rope(const void* x, void* y, csa_dtype dtype, int64_t rows, int D,
+                            int64_t period, int64_t pos0, float theta, csa_stream stream);
+
 /* ---------------------------------------------------------------- a7
  * Tile-mean queries for prefill (HiLS review section 3: adjacent queries
  * share one chunk union):  qbar[b,t,h,:] = (1/tile_m) sum_{i<tile_m} Q[b,t*tile_m+i,h,:].
@@ -401,6 +418,11 @@ typedef struct csa_decode_step_desc {
    * else both [B, Hkv, T/L, D] bf16 gist keys and values */
   const void* Kg;
   const void* Vg;
+  /* RoPE-aware split (see csa_rope): NULL = score with q; else the pre-RoPE
+   * query [B, Hq, D] bf16 the selection scores with (against summaries of
+   * the pre-RoPE keys), while the decode attends with q (rotated) over the
+   * rotated cache K */
+  const void* q_score;
 } csa_decode_step_desc;
 
 CSA_API csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream);

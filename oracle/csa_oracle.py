@@ -307,6 +307,25 @@ def decode_unit(q_group, K_unit, V_unit, chunks, L: int, scale: float):
     return attend(q_group, K_unit, V_unit, chunk_tokens(sorted(chunks), L), scale)
 
 
+def rope(x: np.ndarray, pos, theta: float) -> np.ndarray:
+    """Rotary position embedding of rows x [..., n, D] at positions pos
+    (broadcast against the row axis), rotate-half pairing: for i < D/2 the
+    pair (x_i, x_{i+D/2}) turns by the angle pos * theta^(-2i/D).
+
+    The RTPurbo review (section 1, "Low-dimensional Projection") scores on a
+    projection taken before RoPE because RoPE makes scores depend on the
+    distance; the pages do not write RoPE out, so this is the common
+    rotate-half form with base theta."""
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    h = D // 2
+    freq = theta ** (-2.0 * np.arange(h) / D)                      # [h]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * freq      # [..., n, h]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., :h], x[..., h:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
 def hybrid_unit(q_group, K_unit, V_unit, Kg_unit, Vg_unit, chunks, L: int, scale: float):
     """Attention of one unit's query heads over its hybrid context (SSA
     summary, "방법론" and "기술 상세": K_hybrid and V_hybrid are the gist KV

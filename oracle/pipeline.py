@@ -36,14 +36,19 @@ def unit_summaries(K_unit, L: int, proj=None, block_chunks: int = 2048) -> np.nd
 def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_local: int,
                 k_free: int = 0, proj=None, p: float = 0.0, budget: int = 0,
                 full_heads=(), Gm: int = 0, top_meta: int = 0, units=None,
-                with_attention: bool = True, gist=None) -> dict:
+                with_attention: bool = True, gist=None, rope_theta: float = 0.0) -> dict:
     """One decode step of the units (b, kvh) listed (default: all).
 
     q [B, Hq, D]; K, V [B, Hkv, T, D].  Returns a dict with, per unit, the
     ascending chunk set, the boundary gap(s), n_p for top-p, and when
     ``with_attention`` the output rows o [G, D] and lse [G].  gist = (Kg, Vg),
     each [B, Hkv, T // L, D]: the sparse units attend over the hybrid context
-    (their gist rows plus the raw KV of their chunks, ``hybrid_unit``)."""
+    (their gist rows plus the raw KV of their chunks, ``hybrid_unit``).
+    rope_theta > 0: the RoPE-aware split (RTPurbo review, section 1): q and K
+    are the pre-RoPE ones and score as they are; attention runs on the
+    rotated query (position T - 1, the context's last token) and keys
+    (positions 0 .. T - 1), each stored in the cache's dtype as a decode
+    step would hold them."""
     B, Hkv, T, D = K.shape
     Hq = q.shape[1]
     G = Hq // Hkv
@@ -79,7 +84,14 @@ def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_lo
             raise ValueError(select)
         res["sets"][(b, h)] = chunks
         res["gap"][(b, h)] = gap
-        if with_attention and gist is not None and h not in tuple(full_heads):
+        if with_attention and rope_theta > 0:
+            tok = O.chunk_tokens(chunks, L)
+            qr = _stored(O.rope(qg, np.full(G, T - 1), rope_theta), q)
+            Kr = _stored(O.rope(to_np(K[b, h][_index(K, tok)]), tok, rope_theta), K)
+            o, lse = O.attend(qr, Kr, to_np(V[b, h][_index(V, tok)]), np.arange(len(tok)), scale)
+            res["o"][(b, h)] = o
+            res["lse"][(b, h)] = lse
+        elif with_attention and gist is not None and h not in tuple(full_heads):
             o, lse = O.hybrid_unit(qg, to_np(K[b, h]), to_np(V[b, h]), to_np(gist[0][b, h]),
                                    to_np(gist[1][b, h]), chunks, L, scale)
             res["o"][(b, h)] = o
@@ -92,6 +104,15 @@ def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_lo
             res["o"][(b, h)] = o
             res["lse"][(b, h)] = lse
     return res
+
+
+def _stored(x: np.ndarray, like) -> np.ndarray:
+    """x rounded to the element type of `like` (a bf16 cache holds bf16), as
+    fp64.  torch's round-to-nearest-even conversion is the library step."""
+    if hasattr(like, "dtype") and str(like.dtype) == "torch.bfloat16":
+        import torch
+        return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
 
 
 def _index(t, idx: np.ndarray):

@@ -46,6 +46,7 @@ _SIGS = {
     "csa_chunk_summaries": (_i, [_vp, _i, _i, _i, _i64, _i, _i, _vp, _i, _vp, _vp]),
     "csa_meta_summaries": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "csa_tile_mean_q": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
+    "csa_rope": (_i, [_vp, _vp, _i, _i64, _i, _i64, _i64, _f, _vp]),
     "csa_score_chunks": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
                               _vp]),
     "csa_select_topk": (_i, [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp, _i, _vp]),
@@ -210,6 +211,12 @@ def csa_score_select_topp(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full
                                      _p(idx), _p(count), kmax, _p(n_p_out), _s(stream)))
 
 
+def csa_rope(x, y, dtype, rows, D, period, pos0, theta, stream=None):
+    """Rotary position embedding of x [rows, D] into y (may be x): row r at
+    position pos0 + r % period (see include/csa.h)."""
+    _check(lib.csa_rope(_p(x), _p(y), _dt(dtype), rows, D, period, pos0, theta, _s(stream)))
+
+
 def csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts) -> int:
     n = lib.csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts)
     if n < 0:
@@ -264,7 +271,7 @@ class DecodeStepDesc(ctypes.Structure):
         ("idx", _vp), ("count", _vp), ("kmax", _i), ("n_p_out", _vp),
         ("num_parts", _i), ("workspace", _vp), ("workspace_bytes", _i64),
         ("out", _vp), ("out_dtype", _i), ("lse_out", _vp),
-        ("Kg", _vp), ("Vg", _vp),
+        ("Kg", _vp), ("Vg", _vp), ("q_score", _vp),
     ]
 
 

@@ -1,6 +1,7 @@
 // C ABI of libcsa (declared in include/csa.h): argument validation, error
 // reporting and the launches.  Nothing here allocates device memory.
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdlib>
 #include <mutex>
@@ -220,6 +221,22 @@ csa_status csa_tile_mean_q(const void* Q, csa_dtype dtype, int B, int S, int Hq,
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
   return finish(csa::launch_tile_mean(l, Q, dtype == CSA_BF16, B, S, Hq, D, tile_m, qbar), "tile mean launch");
+}
+
+csa_status csa_rope(const void* x, void* y, csa_dtype dtype, int64_t rows, int D, int64_t period,
+                    int64_t pos0, float theta, csa_stream stream) {
+  CSA_REQUIRE(valid_dtype(dtype), "dtype");
+  CSA_REQUIRE(rows >= 0 && D > 0 && period > 0 && pos0 >= 0, "bad sizes");
+  CSA_REQUIRE(D % 2 == 0, "D must be even");
+  CSA_SUPPORT(D <= 512, "D <= 512");
+  CSA_REQUIRE(std::isfinite(theta) && theta > 1.0f, "theta must be finite and > 1");
+  if (rows == 0) return CSA_OK;
+  CSA_TRY(check_ptr(x, "x"));
+  CSA_TRY(check_ptr(y, "y"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_rope(l, x, y, dtype == CSA_BF16, rows, D, period, pos0, theta),
+                "rope launch");
 }
 
 csa_status csa_score_chunks(const void* q, csa_dtype q_dtype, const float* proj, int R,
@@ -623,22 +640,25 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
     CSA_TRY(check_ptr(d->Vg, "Vg"));
   }
   const int C = static_cast<int>(d->T / d->L);
+  // the selection scores with the pre-RoPE query when one is given
+  const void* qs = d->q_score != nullptr ? d->q_score : d->q;
+  if (d->q_score != nullptr) CSA_TRY(check_ptr(d->q_score, "q_score"));
   // the selection (validates its own arguments before launching)
   csa_status st;
   if (d->mode == CSA_SELECT_TOPK)
-    st = csa_score_select_topk(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
+    st = csa_score_select_topk(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
                                d->head_full, d->k_free, d->n_sink, d->n_local, d->idx, d->count,
                                d->kmax, stream);
   else if (d->mode == CSA_SELECT_TOPK_UNION)
-    st = csa_score_select_topk_union(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
+    st = csa_score_select_topk_union(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
                                      d->D, C, d->head_full, d->k_free, d->n_sink, d->n_local,
                                      d->idx, d->count, d->kmax, stream);
   else if (d->mode == CSA_SELECT_TOPP)
-    st = csa_score_select_topp(d->q, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
+    st = csa_score_select_topp(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
                                d->head_full, d->logit_scale, d->p, d->budget, d->n_sink, d->n_local,
                                d->idx, d->count, d->kmax, d->n_p_out, stream);
   else
-    st = csa_select_hier(d->q, CSA_BF16, d->meta, d->summ, d->B, d->Hq, d->Hkv, d->D, C, d->Gm,
+    st = csa_select_hier(qs, CSA_BF16, d->meta, d->summ, d->B, d->Hq, d->Hkv, d->D, C, d->Gm,
                          d->top_meta, d->k_free, d->n_sink, d->n_local, d->idx, d->count, d->kmax,
                          stream);
   if (st != CSA_OK) return st;

@@ -58,6 +58,10 @@ cudaError_t launch_score_select_topp(const Launch& l, const void* q, bool bf16, 
                                      int budget, int n_sink, int n_local, int32_t* idx,
                                      int32_t* count, int kmax, int32_t* n_p_out);
 
+// rope.cu
+cudaError_t launch_rope(const Launch& l, const void* x, void* y, bool bf16, int64_t rows, int D,
+                        int64_t period, int64_t pos0, float theta);
+
 // decode.cu
 int decode_default_parts(bool bf16, int D, int L, int num_sms);
 // Merged mode: the last CTA of each unit combines the unit's splits.

@@ -35,13 +35,18 @@ class SparseDecoder:
     hybrid=True (bf16, fused): every sparse head also attends over one gist
     key/value row per chunk (the hybrid context of SSA).  The gist rows are
     built here with the cache, as the chunk means of K and V in bf16: the
-    stand-in for a trained model's gist KV."""
+    stand-in for a trained model's gist KV.
+
+    rope_theta > 0 (the RoPE-aware split): K and the queries given to ``step``
+    are pre-RoPE; chunks are scored on them, and attention runs on rotated
+    copies (csa_rope): the cache is rotated once here (positions 0..T-1) and
+    each step rotates its query at position T - 1."""
 
     def __init__(self, K: torch.Tensor, V: torch.Tensor, *, Hq: int, L: int, select: str,
                  n_sink: int, n_local: int, k_free: int = 0, proj: torch.Tensor | None = None,
                  p: float = 0.9, budget: int = 256, full_heads=(), Gm: int = 0, top_meta: int = 0,
                  scale: float | None = None, num_parts: int = 0, out_dtype=torch.float32,
-                 fused: bool = True, hybrid: bool = False):
+                 fused: bool = True, hybrid: bool = False, rope_theta: float = 0.0):
         assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
         self.K, self.V = K, V
         B, Hkv, T, D = K.shape
@@ -62,6 +67,13 @@ class SparseDecoder:
         if select == "hier":
             self.meta = torch.empty(B, Hkv, self.C // Gm, Ds, dtype=torch.float32, device=dev)
             csa.csa_meta_summaries(self.summ, B, Hkv, self.C, Ds, Gm, self.meta)
+        self.rope_theta = float(rope_theta)
+        self.K_att, self.q_rot = K, None
+        if self.rope_theta > 0:
+            assert not hybrid, "the hybrid context is not combined with RoPE here"
+            self.K_att = torch.empty_like(K)
+            csa.csa_rope(K, self.K_att, self.dtype, B * Hkv * T, D, T, 0, self.rope_theta)
+            self.q_rot = torch.empty(B, Hq, D, dtype=K.dtype, device=dev)
         self.Kg = self.Vg = None
         if hybrid:
             assert fused and K.dtype == torch.bfloat16, "the hybrid context needs a fused bf16 decode"
@@ -101,7 +113,7 @@ class SparseDecoder:
             mode = {"topk": csa.CSA_SELECT_TOPK, "topp": csa.CSA_SELECT_TOPP,
                     "hier": csa.CSA_SELECT_HIER, "topk_union": csa.CSA_SELECT_TOPK_UNION}[select]
             self.desc = csa.decode_step_desc(
-                K=K, V=V, B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, L=L, scale=self.scale,
+                K=self.K_att, V=V, B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, L=L, scale=self.scale,
                 head_full=self.head_full, mode=mode, summ=self.summ, proj=proj, R=self.R,
                 meta=self.meta, Gm=Gm, top_meta=top_meta, k_free=k_free, n_sink=n_sink,
                 n_local=n_local, logit_scale=1.0 / math.sqrt(D), p=p, budget=budget, idx=self.idx,
@@ -152,20 +164,20 @@ class SparseDecoder:
         """Sparse split-K decode over the current index lists, then the LSE merge
         (one launch when fused)."""
         if self.Kg is not None:
-            csa.csa_sparse_decode_merged_hybrid(q, self.K, self.V, self.Kg, self.Vg, self.dtype,
+            csa.csa_sparse_decode_merged_hybrid(q, self.K_att, self.V, self.Kg, self.Vg, self.dtype,
                                                 self.idx, self.count, self.kmax, self.head_full,
                                                 self.B, self.Hq, self.Hkv, self.D, self.T, self.L,
                                                 self.scale, self.P, self.workspace, self.ws_bytes,
                                                 self.out, _dt(self.out), self.lse, stream=stream)
             return
         if self.fused:
-            csa.csa_sparse_decode_merged(q, self.K, self.V, self.dtype, self.idx, self.count,
+            csa.csa_sparse_decode_merged(q, self.K_att, self.V, self.dtype, self.idx, self.count,
                                          self.kmax, self.head_full, self.B, self.Hq, self.Hkv,
                                          self.D, self.T, self.L, self.scale, self.P,
                                          self.workspace, self.ws_bytes, self.out, _dt(self.out),
                                          self.lse, stream=stream)
             return
-        csa.csa_sparse_decode(q, self.K, self.V, self.dtype, self.idx, self.count, self.kmax,
+        csa.csa_sparse_decode(q, self.K_att, self.V, self.dtype, self.idx, self.count, self.kmax,
                               self.head_full, self.B, self.Hq, self.Hkv, self.D, self.T, self.L,
                               self.scale, self.P, self.max_splits, self.o_part, self.lse_part,
                               stream=stream)
@@ -173,12 +185,18 @@ class SparseDecoder:
                           self.out, _dt(self.out), self.lse, stream=stream)
 
     def step(self, q: torch.Tensor, stream=None):
+        qa = q  # the query attention runs with
+        if self.q_rot is not None:
+            csa.csa_rope(q, self.q_rot, self.dtype, self.B * self.Hq, self.D, 1, self.T - 1,
+                         self.rope_theta, stream=stream)
+            qa = self.q_rot
         if self.desc is not None and q.dtype == torch.bfloat16:
-            self.desc.q = q.data_ptr()
+            self.desc.q = qa.data_ptr()
+            self.desc.q_score = q.data_ptr() if self.q_rot is not None else None
             csa.csa_decode_step(self.desc, stream=stream)
             return self.out, self.lse
         self.select_chunks(q, stream)
-        self.attend(q, stream)
+        self.attend(qa, stream)
         return self.out, self.lse
 
 

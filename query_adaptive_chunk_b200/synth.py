@@ -66,6 +66,7 @@ class DecodeWorkload:
     Gm: int = 0  # hierarchical: chunks per meta-chunk
     top_meta: int = 0  # hierarchical: meta-chunks kept
     hybrid: bool = False  # sparse heads also attend over one gist row per chunk
+    rope_theta: float = 0.0  # > 0: K/q are pre-RoPE; attention on the rotated ones
 
     @property
     def C(self) -> int:
@@ -165,7 +166,13 @@ TOPK_UNION_32K = dataclasses.replace(TOPK_32K, name="topk_union_decode_bf16_ctx3
 HYBRID_TOPK_32K = dataclasses.replace(TOPK_32K, name="hybrid_topk_decode_bf16_ctx32k", seed=7,
                                       hybrid=True)
 
-DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M, TOPK_UNION_32K, HYBRID_TOPK_32K)
+# RTPurbo's RoPE-aware split: the 32K top-k step scored on the pre-RoPE keys
+# and query, attending with the rotated ones (base 500000)
+ROPE_TOPK_32K = dataclasses.replace(TOPK_32K, name="rope_topk_decode_bf16_ctx32k", seed=20,
+                                    rope_theta=500000.0)
+
+DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M, TOPK_UNION_32K, HYBRID_TOPK_32K,
+                    ROPE_TOPK_32K)
 ALL_WORKLOADS = DECODE_WORKLOADS + (PREFILL_32K,)
 
 

@@ -126,6 +126,33 @@ def check_hybrid_vs_sdpa(seed=16, G=4, D=16, T=256, L=32):
         assert np.allclose(lse, torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
 
 
+def check_rope_closed_forms(seed=18):
+    """RoPE: hand-worked pairs (D = 2: a rotation by pos radians; D = 4: the
+    pairing and the frequencies);
+    position 0 is the identity; norms are kept; and the textbook relative
+    property q(m).k(n) = q(m - n).k(0) for every pair of positions."""
+    x = np.array([[1.0, 0.0], [0.0, 2.0]])
+    y = O.rope(x, [math.pi / 2, math.pi / 6], 10000.0)
+    assert np.allclose(y, [[0.0, 1.0], [-1.0, math.sqrt(3.0)]], atol=1e-15), y
+    # D = 4, theta = 100: pairs (0, 2) at frequency 1 and (1, 3) at 100^(-1/2)
+    # = 0.1 (rotate-half pairing, frequency theta^(-2i/D)); position pi/2
+    y = O.rope(np.eye(4)[:2], [math.pi / 2, math.pi / 2], 100.0)
+    c, s_ = math.cos(math.pi / 20), math.sin(math.pi / 20)
+    assert np.allclose(y, [[0.0, 0.0, 1.0, 0.0], [0.0, c, 0.0, s_]], atol=1e-15), y
+    rng = np.random.default_rng(seed)
+    D = 16
+    q, k = rng.standard_normal((5, D)), rng.standard_normal((5, D))
+    assert np.array_equal(O.rope(q, np.zeros(5), 500.0), q)
+    m = np.array([0, 3, 17, 1000, 131071], dtype=np.float64)
+    assert np.allclose(np.linalg.norm(O.rope(q, m, 500.0), axis=1), np.linalg.norm(q, axis=1),
+                       rtol=1e-12)
+    for mi in m:
+        for ni in (0.0, 5.0, 999.0):
+            lhs = O.rope(q, np.full(5, mi), 500.0) @ O.rope(k, np.full(5, ni), 500.0).T
+            rhs = O.rope(q, np.full(5, mi - ni), 500.0) @ k.T
+            assert np.allclose(lhs, rhs, rtol=0, atol=1e-9), (mi, ni)
+
+
 # ---------------------------------------------------------------- summaries / scores
 
 def check_summary_closed_form():
@@ -447,4 +474,5 @@ ALL_CHECKS = [
     check_topp_golden, check_topp_invariants, check_hier_golden, check_hier_all_metas_is_flat,
     check_meta_linearity, check_merge_closed_form, check_partition,
     check_prefill_dense_causal, check_prefill_masked, check_hybrid_golden, check_hybrid_vs_sdpa,
+    check_rope_closed_forms,
 ]

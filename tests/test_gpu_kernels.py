@@ -725,3 +725,43 @@ def test_select_topk_union_kmax_too_small_rejected(csa):
         csa.csa_score_select_topk_union(None, torch.bfloat16, None, 0, None, 1, 8, 2, 128, 512,
                                         None, 10, 1, 1, None, None, 20)
     assert ei.value.status == 1 and "kmax" in str(ei.value)
+
+
+# ---------------------------------------------------------------- RoPE
+
+@pytest.mark.parametrize("dtype,D,period,pos0,theta", [("f32", 128, 4096, 0, 10000.0),
+                                                       ("bf16", 128, 131072, 0, 500000.0),
+                                                       ("f32", 64, 1, 1048575, 10000.0),
+                                                       ("bf16", 64, 7, 123, 100.0)])
+def test_rope_matches_oracle(csa, dtype, D, period, pos0, theta):
+    """csa_rope against the oracle's fp64 rotation: fp32 to 2e-6 (the angle is
+    reduced in double, so positions near 2^20 keep their accuracy); bf16 to
+    one rounding of the output."""
+    rows = 3 * period if period < 5000 else period
+    rows = min(rows, 40000)
+    x = _randn((rows, D), 70 + D, _dt(dtype))
+    y = torch.empty_like(x)
+    csa.csa_rope(x, y, x.dtype, rows, D, period, pos0, theta)
+    csa.csa_check_device_status()
+    pos = pos0 + np.arange(rows) % period
+    ref = O.rope(to_np(x), pos, theta)
+    got = y.cpu().double().numpy()
+    if dtype == "f32":
+        assert np.abs(got - ref).max() < 2e-6
+    else:
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
+    # in place gives the same bits
+    csa.csa_rope(x, x, x.dtype, rows, D, period, pos0, theta)
+    assert torch.equal(x, y)
+
+
+def test_rope_rejects_bad_arguments(csa):
+    from query_adaptive_chunk_b200.csa import CsaError
+    x = torch.zeros(4, 63, device="cuda")
+    with pytest.raises(CsaError):
+        csa.csa_rope(x, x, x.dtype, 4, 63, 4, 0, 10000.0)  # odd D
+    x = torch.zeros(4, 64, device="cuda")
+    with pytest.raises(CsaError):
+        csa.csa_rope(x, x, x.dtype, 4, 64, 0, 0, 10000.0)  # period 0
+    with pytest.raises(CsaError):
+        csa.csa_rope(x, x, x.dtype, 4, 64, 4, 0, 1.0)  # theta must be > 1

@@ -20,7 +20,7 @@ def _decoder(w, inp, fused=True):
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
                          n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
                          budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta,
-                         fused=fused, hybrid=w.hybrid)
+                         fused=fused, hybrid=w.hybrid, rope_theta=w.rope_theta)
 
 
 def run_and_check(w, units=None, fused=True):
@@ -35,7 +35,7 @@ def run_and_check(w, units=None, fused=True):
                          n_sink=w.n_sink, n_local=w.n_local, k_free=w.k_free,
                          proj=inp.get("proj"), p=w.p, budget=w.budget, full_heads=w.full_heads,
                          Gm=w.Gm, top_meta=w.top_meta, units=units,
-                         gist=(dec.Kg, dec.Vg) if w.hybrid else None)
+                         gist=(dec.Kg, dec.Vg) if w.hybrid else None, rope_theta=w.rope_theta)
     gsets_all = parity.gpu_sets(dec.idx, dec.count)
     sparse = [u for u in units if u[1] not in w.full_heads]
     uidx = {u: i for i, u in enumerate(all_units)}
@@ -49,6 +49,12 @@ def run_and_check(w, units=None, fused=True):
         gset = list(range(w.C)) if h in w.full_heads else gsets_all[uidx[(b, h)]]
         if gset == ref["sets"][(b, h)]:
             ro, rl = ref["o"][(b, h)], ref["lse"][(b, h)]
+        elif w.rope_theta:  # near-tie: rotated attention over the GPU's own set
+            tok = O.chunk_tokens(gset, w.L)
+            qg = to_np(inp["q"][b, h * G:(h + 1) * G])
+            qr = OP._stored(O.rope(qg, np.full(G, w.T - 1), w.rope_theta), inp["q"])
+            Kr = OP._stored(O.rope(to_np(inp["K"][b, h][tok]), tok, w.rope_theta), inp["K"])
+            ro, rl = O.attend(qr, Kr, to_np(inp["V"][b, h][tok]), np.arange(len(tok)), w.scale)
         elif w.hybrid:  # near-tie: the hybrid context over the GPU's own set
             ro, rl = O.hybrid_unit(to_np(inp["q"][b, h * G:(h + 1) * G]), to_np(inp["K"][b, h]),
                                    to_np(inp["V"][b, h]), to_np(dec.Kg[b, h]),
@@ -180,5 +186,34 @@ def test_hybrid_separate_decode_call_matches_step():
     dec, inp = run_and_check(w)
     out_step = dec.out.clone()
     dec.attend(inp["q"])
+    csa.csa_check_device_status()
+    assert (dec.out - out_step).abs().max().item() < 1e-5
+
+
+def test_rope_aware_topp_mixed_reduced():
+    """RoPE-aware split (RTPurbo review, section 1): chunks scored on the
+    pre-RoPE projected keys and query, attention on the rotated cache and
+    query (rotated by csa_rope), full and top-p heads in one step."""
+    import dataclasses
+    w = dataclasses.replace(synth.TOPP_128K.scaled(B=1, T=16384), name="rope_topp_mixed",
+                            seed=19, rope_theta=10000.0)
+    run_and_check(w)
+
+
+def test_rope_aware_topk_full_size():
+    run_and_check(synth.ROPE_TOPK_32K)
+
+
+def test_rope_aware_separate_calls_match_step():
+    """The separate calls (score on the pre-RoPE query, decode with the
+    rotated one) give the one-call step's output."""
+    import dataclasses
+    from query_adaptive_chunk_b200 import csa
+    w = dataclasses.replace(synth.TOPK_32K.scaled(B=2, T=8192), name="rope_topk_small", seed=21,
+                            rope_theta=10000.0)
+    dec, inp = run_and_check(w)
+    out_step = dec.out.clone()
+    dec.select_chunks(inp["q"])
+    dec.attend(dec.q_rot)
     csa.csa_check_device_status()
     assert (dec.out - out_step).abs().max().item() < 1e-5

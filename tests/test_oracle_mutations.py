@@ -15,7 +15,7 @@ _orig = {name: getattr(O, name) for name in
          ["attend", "select_topk", "select_topp", "score_chunks", "lse_merge",
           "causal_attend", "meta_summaries", "chunk_summaries", "select_hier",
           "forced_set", "topp_probs", "decode_partition", "tile_mean_q",
-          "select_topk_union", "score_chunks_per_head", "hybrid_unit"]}
+          "select_topk_union", "score_chunks_per_head", "hybrid_unit", "rope"]}
 
 
 def attend_no_scale(q, K, V, tokens, scale):
@@ -189,6 +189,29 @@ def hybrid_gist_logits_unscaled(q, K, V, Kg, Vg, chunks, L, scale):
                                 L, scale)
 
 
+def rope_sin_sign_flipped(x, pos, theta):
+    return _orig["rope"](x, -np.asarray(pos, dtype=np.float64), theta)
+
+
+def rope_adjacent_pairs(x, pos, theta):
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    perm = np.concatenate([np.arange(0, D, 2), np.arange(1, D, 2)])  # pairs (2i, 2i+1)
+    inv = np.argsort(perm)
+    return _orig["rope"](x[..., perm], pos, theta)[..., inv]
+
+
+def rope_freq_exponent_off(x, pos, theta):
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    h = D // 2
+    freq = theta ** (-1.0 * np.arange(h) / D)  # i/D instead of 2i/D
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * freq
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., :h], x[..., h:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
 MUTANTS = [
     ("attend", attend_no_scale),
     ("attend", attend_no_max_shift_wrong_lse),
@@ -219,6 +242,9 @@ MUTANTS = [
     ("hybrid_unit", hybrid_selected_gists_only),
     ("hybrid_unit", hybrid_no_gists),
     ("hybrid_unit", hybrid_gist_logits_unscaled),
+    ("rope", rope_sin_sign_flipped),
+    ("rope", rope_adjacent_pairs),
+    ("rope", rope_freq_exponent_off),
 ]
 
 
