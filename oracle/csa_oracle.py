@@ -422,3 +422,75 @@ def prefill_tile(Q_tile: np.ndarray, K_head: np.ndarray, V_head: np.ndarray, chu
     tok = chunk_tokens(sorted(chunks), L)
     return causal_attend(Q_tile, np.asarray(K_head)[tok], np.asarray(V_head)[tok], tok,
                          q_start, scale)
+
+
+# ------------------------------------------------------ token-level sparsity
+
+def token_importance(Q_obs: np.ndarray, K: np.ndarray, obs_pos: np.ndarray,
+                     scale: float) -> np.ndarray:
+    """Importance of every key of one KV head from a proxy attention map of
+    the recent queries (Token Sparse Attention summary, section 2, "동적 토큰
+    커버리지": recent queries against all keys, scores summed over the query
+    axis of the attention weights).
+
+    Q_obs [r, D]: the recent query rows of the KV head's query heads (the GQA
+    group, reading: one importance per KV head, summed over its query heads);
+    obs_pos [r]: their positions.  Row i attends causally (key j <= obs_pos[i])
+    with softmax(scale * q.k); the importance of key j is the sum over the rows
+    of its weight.  K [S, D] -> [S]."""
+    q = np.asarray(Q_obs, dtype=np.float64)
+    k = np.asarray(K, dtype=np.float64)
+    a = (q @ k.T) * scale                                   # [r, S]
+    S = k.shape[0]
+    vis = np.arange(S)[None, :] <= np.asarray(obs_pos)[:, None]
+    a = np.where(vis, a, NEG_INF)
+    w = np.exp(a - a.max(axis=1, keepdims=True))
+    w /= w.sum(axis=1, keepdims=True)
+    return w.sum(axis=0)
+
+
+def coverage_budget(mass: np.ndarray, tau: float) -> int:
+    """Dynamic Token Coverage budget (Token Sparse Attention summary, section
+    2): sort the tokens by importance ascending and drop them from the least
+    important while the dropped mass stays <= tau; the budget is the number
+    of tokens left.  mass [S], normalised here to sum 1; ties in the order go
+    to the higher index first (so the lower index is kept)."""
+    m = np.asarray(mass, dtype=np.float64)
+    m = m / m.sum()
+    order = sorted(range(len(m)), key=lambda j: (m[j], -j))   # ascending mass
+    dropped, acc = 0, 0.0
+    for j in order:
+        if acc + m[j] > tau:
+            break
+        acc += m[j]
+        dropped += 1
+    return len(m) - dropped
+
+
+def select_tokens(importance: np.ndarray, k: int) -> list:
+    """The k most important tokens of one KV head (score desc, lower index
+    first on ties), ascending: each head keeps its own top-k under the global
+    budget (Token Sparse Attention summary, section 2, "헤드별 선택")."""
+    return sorted(_rank_order(np.asarray(importance, dtype=np.float64),
+                              range(len(importance)))[:k])
+
+
+def token_sparse_head(Q_group: np.ndarray, K_head: np.ndarray, V_head: np.ndarray, tokens,
+                      scale: float) -> np.ndarray:
+    """Compress, attend, decompress for one KV head (Token Sparse Attention
+    summary, section 2, "핵심 아키텍처"): gather the query rows of the group's
+    heads and the key/value rows at the selected tokens (ascending), run dense
+    causal attention on the compressed sequence, and scatter the outputs back
+    to their positions of a zero output.  Q_group [S, G, D], K/V [S, D] ->
+    O [S, G, D]."""
+    Q_group = np.asarray(Q_group, dtype=np.float64)
+    S, G, D = Q_group.shape
+    out = np.zeros((S, G, np.asarray(V_head).shape[-1]))
+    t = np.asarray(sorted(tokens), dtype=np.int64)
+    if len(t) == 0:
+        return out
+    k, v = np.asarray(K_head, dtype=np.float64)[t], np.asarray(V_head, dtype=np.float64)[t]
+    for g in range(G):
+        # compressed index i sees compressed j <= i: positions stay in order
+        out[t, g] = causal_attend(Q_group[t, g], k, v, np.arange(len(t)), 0, scale)
+    return out

@@ -153,6 +153,67 @@ def check_rope_closed_forms(seed=18):
             assert np.allclose(lhs, rhs, rtol=0, atol=1e-9), (mi, ni)
 
 
+def check_token_sparse_golden():
+    """Token importance and the coverage budget on the hand-worked cases of
+    tests/golden/token_sparse_cases.json."""
+    g = _golden("token_sparse_cases.json")
+    im = g["importance"]
+    got = O.token_importance(np.array(im["Q_obs"]), np.array(im["K"]), np.array(im["obs_pos"]),
+                             im["scale"])
+    assert np.allclose(got, im["expected"], rtol=0, atol=1e-12), got
+    for tau, k in g["budget"]["cases"]:
+        assert O.coverage_budget(g["budget"]["mass"], tau) == k, (tau, k)
+
+
+def check_token_sparse_invariants(seed=22, trials=30):
+    """Importance: every query row spends a total weight of 1; keys after a
+    row's position get none from it.  Budget: equals the smallest m whose m
+    most important tokens hold >= 1 - tau of the mass (the same cut counted
+    from the top), on cases without near-ties.  Token choice: torch.sort on
+    (score desc, index asc)."""
+    rng = np.random.default_rng(seed)
+    S, D, r = 40, 8, 6
+    q, k = rng.standard_normal((r, D)), rng.standard_normal((S, D))
+    pos = np.array([39, 38, 30, 20, 5, 0])
+    im = O.token_importance(q, k, pos, 0.5)
+    assert abs(im.sum() - r) < 1e-9
+    assert im[39] > 0 and abs(O.token_importance(q[4:5], k, pos[4:5], 0.5)[6:].sum()) == 0.0
+    for _ in range(trials):
+        n = int(rng.integers(2, 60))
+        m = rng.random(n) ** 3
+        m /= m.sum()
+        tau = float(rng.random() * 0.5)
+        srt = np.sort(m)[::-1]
+        cum = np.cumsum(srt)
+        if np.min(np.abs(cum - (1 - tau))) < 1e-9:
+            continue
+        m_top = int(np.argmax(cum >= 1 - tau - 1e-15)) + 1
+        assert O.coverage_budget(m, tau) == m_top, (n, tau)
+        kk = int(rng.integers(0, n + 1))
+        sc = np.round(rng.standard_normal(n), 1)  # ties on purpose
+        ref = sorted(torch.sort(torch.tensor(-sc * 1000.0 + np.arange(n) * 1e-3)).indices[:kk].tolist())
+        assert O.select_tokens(sc, kk) == ref
+
+
+def check_token_sparse_vs_sdpa(seed=23, S=96, G=2, D=16):
+    """Compress, dense causal attention, decompress == fp64 SDPA over the
+    whole sequence with a mask keeping, for a selected query row, the
+    selected keys at or before it; rows not selected are 0."""
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((S, G, D))
+    K, V = rng.standard_normal((S, D)), rng.standard_normal((S, D))
+    sel = sorted(rng.choice(S, size=37, replace=False).tolist())
+    out = O.token_sparse_head(Q, K, V, sel, 0.25)
+    keep = np.zeros(S, dtype=bool)
+    keep[sel] = True
+    mask = keep[:, None] & keep[None, :] & (np.arange(S)[None, :] <= np.arange(S)[:, None])
+    mask[~keep, 0] = True  # rows left out get a dummy key; compared as zeros below
+    for g in range(G):
+        ref = _sdpa(Q[None, :, g], K[None], V[None], mask=mask[None], scale=0.25)[0]
+        assert np.allclose(out[keep, g], ref[keep], rtol=0, atol=1e-12)
+        assert np.all(out[~keep, g] == 0)
+
+
 # ---------------------------------------------------------------- summaries / scores
 
 def check_summary_closed_form():
@@ -474,5 +535,6 @@ ALL_CHECKS = [
     check_topp_golden, check_topp_invariants, check_hier_golden, check_hier_all_metas_is_flat,
     check_meta_linearity, check_merge_closed_form, check_partition,
     check_prefill_dense_causal, check_prefill_masked, check_hybrid_golden, check_hybrid_vs_sdpa,
-    check_rope_closed_forms,
+    check_rope_closed_forms, check_token_sparse_golden, check_token_sparse_invariants,
+    check_token_sparse_vs_sdpa,
 ]

@@ -15,7 +15,8 @@ _orig = {name: getattr(O, name) for name in
          ["attend", "select_topk", "select_topp", "score_chunks", "lse_merge",
           "causal_attend", "meta_summaries", "chunk_summaries", "select_hier",
           "forced_set", "topp_probs", "decode_partition", "tile_mean_q",
-          "select_topk_union", "score_chunks_per_head", "hybrid_unit", "rope"]}
+          "select_topk_union", "score_chunks_per_head", "hybrid_unit", "rope",
+          "token_importance", "coverage_budget", "select_tokens", "token_sparse_head"]}
 
 
 def attend_no_scale(q, K, V, tokens, scale):
@@ -212,6 +213,58 @@ def rope_freq_exponent_off(x, pos, theta):
     return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
 
 
+def importance_not_causal(Q_obs, K, obs_pos, scale):
+    return _orig["token_importance"](Q_obs, K, np.full(len(obs_pos), len(K)), scale)
+
+
+def budget_strict(mass, tau):
+    m = np.asarray(mass, dtype=np.float64)
+    m = m / m.sum()
+    dropped, acc = 0, 0.0
+    for j in sorted(range(len(m)), key=lambda j: (m[j], -j)):
+        if acc + m[j] >= tau:  # stops at equality
+            break
+        acc += m[j]
+        dropped += 1
+    return len(m) - dropped
+
+
+def budget_keeps_tail(mass, tau):
+    m = np.asarray(mass, dtype=np.float64)
+    m = m / m.sum()
+    kept, acc = 0, 0.0  # counts from the top until the kept mass reaches tau
+    for j in sorted(range(len(m)), key=lambda j: (-m[j], j)):
+        if acc >= tau:
+            break
+        acc += m[j]
+        kept += 1
+    return kept
+
+
+def tokens_least_important(importance, k):
+    return _orig["select_tokens"](-np.asarray(importance, dtype=np.float64), k)
+
+
+def token_sparse_dense_rows(Q_group, K_head, V_head, tokens, scale):
+    out = _orig["token_sparse_head"](Q_group, K_head, V_head, tokens, scale)
+    full = _orig["token_sparse_head"](Q_group, K_head, V_head, range(len(K_head)), scale)
+    keep = np.zeros(len(K_head), dtype=bool)
+    keep[list(tokens)] = True
+    out[~keep] = full[~keep]  # rows left out attend densely instead of 0
+    return out
+
+
+def token_sparse_not_causal(Q_group, K_head, V_head, tokens, scale):
+    Q_group = np.asarray(Q_group, dtype=np.float64)
+    S, G, D = Q_group.shape
+    out = np.zeros((S, G, np.asarray(V_head).shape[-1]))
+    t = np.asarray(sorted(tokens), dtype=np.int64)
+    for g in range(G):
+        out[t, g] = O.causal_attend(Q_group[t, g], np.asarray(K_head)[t], np.asarray(V_head)[t],
+                                    np.zeros(len(t)), 0, scale)
+    return out
+
+
 MUTANTS = [
     ("attend", attend_no_scale),
     ("attend", attend_no_max_shift_wrong_lse),
@@ -245,6 +298,12 @@ MUTANTS = [
     ("rope", rope_sin_sign_flipped),
     ("rope", rope_adjacent_pairs),
     ("rope", rope_freq_exponent_off),
+    ("token_importance", importance_not_causal),
+    ("coverage_budget", budget_strict),
+    ("coverage_budget", budget_keeps_tail),
+    ("select_tokens", tokens_least_important),
+    ("token_sparse_head", token_sparse_dense_rows),
+    ("token_sparse_head", token_sparse_not_causal),
 ]
 
 
