@@ -136,6 +136,54 @@ CSA_API csa_status csa_meta_summaries(const float* summ, int B, int Hkv, int C, 
 CSA_API csa_status csa_rope(const void* x, void* y, csa_dtype dtype, int64_t rows, int D,
                             int64_t period, int64_t pos0, float theta, csa_stream stream);
 
+/* ---------------------------------------------------------------- token-level sparsity
+ * Token Sparse Attention for prefill (Token Sparse Attention summary,
+ * gist.science/ko/paper/2602.03216, section 2).  bf16 Q [B, S, Hq, D] and
+ * K, V [B, Hkv, S, D]; the GQA group of KV head h is query heads h*G..h*G+G-1.
+ *
+ * csa_token_importance: importance of every key from a proxy attention map
+ * of the recent queries ("동적 토큰 커버리지"): the last n_obs query rows of
+ * every query head of the group attend causally (key j <= the row's
+ * position) with softmax(scale * q.k); imp[b, h, j] = the sum over those
+ * G*n_obs rows of key j's weight.  Two passes over K on the tensor cores.
+ * imp [B, Hkv, S] fp32 (output); scratch >= csa_token_importance_scratch_bytes.
+ * D 64 or 128; n_obs a multiple of 8 with (Hq/Hkv) * n_obs <= 512. */
+CSA_API int64_t csa_token_importance_scratch_bytes(int B, int S, int Hq, int Hkv, int n_obs);
+CSA_API csa_status csa_token_importance(const void* Q, const void* K, int B, int S, int Hq,
+                                        int Hkv, int D, int n_obs, float scale, float* imp,
+                                        void* scratch, int64_t scratch_bytes,
+                                        csa_stream stream);
+
+/* csa_token_budget: Dynamic Token Coverage.  The masses m_j = sum_h
+ * imp[b, h, j] are normalised; the least important tokens are dropped while
+ * their mass stays <= tau, i.e. k_seq[b] = the fewest tokens whose mass
+ * reaches 1 - tau.  k_unit[b*Hkv + h] = k_seq[b] rounded up to a multiple of
+ * `tile` (at most S): the token count every KV head of sequence b keeps.
+ * Float sums: a cut within rounding of a tie may land one token apart from
+ * exact arithmetic.  tau in [0, 1); S <= 32768. */
+CSA_API csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, float tau, int tile,
+                                    int32_t* k_seq, int32_t* k_unit, csa_stream stream);
+
+/* csa_token_sparse_prefill: the whole prefill ("핵심 아키텍처", "헤드별 선택"):
+ * importance and budget as above (tile 64), each KV head's own k_unit most
+ * important tokens (score desc, lower index on ties; csa_select_topk's
+ * order), then compress: the kept tokens' K and V rows and the group's query
+ * rows, in position order, into dense tensors; dense causal attention of the
+ * compressed sequences on the tensor cores (the block-sparse prefill kernel
+ * with every earlier tile visible); decompress: each output row back to its
+ * position, every other row of O set to 0.
+ *   O [B, S, Hq, D] bf16 (output); budget_out [B] int32 device (output, the
+ *   unrounded k_seq).  D = 128, Hq/Hkv = 4, S % 64 == 0, S <= 32768.
+ *   workspace >= csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs).
+ * The call reads the budgets back to the host to size the dense attention:
+ * it synchronises `stream` once and cannot be captured in a CUDA graph. */
+CSA_API int64_t csa_token_sparse_workspace_bytes(int B, int S, int Hq, int Hkv, int D, int n_obs);
+CSA_API csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V, int B,
+                                            int S, int Hq, int Hkv, int D, int n_obs, float tau,
+                                            float scale, void* workspace,
+                                            int64_t workspace_bytes, void* O,
+                                            int32_t* budget_out, csa_stream stream);
+
 /* ---------------------------------------------------------------- a7
  * Tile-mean queries for prefill (HiLS review section 3: adjacent queries
  * share one chunk union):  qbar[b,t,h,:] = (1/tile_m) sum_{i<tile_m} Q[b,t*tile_m+i,h,:].

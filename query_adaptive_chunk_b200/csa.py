@@ -47,6 +47,12 @@ _SIGS = {
     "csa_meta_summaries": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "csa_tile_mean_q": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp]),
     "csa_rope": (_i, [_vp, _vp, _i, _i64, _i, _i64, _i64, _f, _vp]),
+    "csa_token_importance_scratch_bytes": (_i64, [_i, _i, _i, _i, _i]),
+    "csa_token_importance": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _i64, _vp]),
+    "csa_token_budget": (_i, [_vp, _i, _i, _i, _f, _i, _vp, _vp, _vp]),
+    "csa_token_sparse_workspace_bytes": (_i64, [_i, _i, _i, _i, _i, _i]),
+    "csa_token_sparse_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _i64,
+                                      _vp, _vp, _vp]),
     "csa_score_chunks": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
                               _vp]),
     "csa_select_topk": (_i, [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp, _i, _vp]),
@@ -215,6 +221,40 @@ def csa_rope(x, y, dtype, rows, D, period, pos0, theta, stream=None):
     """Rotary position embedding of x [rows, D] into y (may be x): row r at
     position pos0 + r % period (see include/csa.h)."""
     _check(lib.csa_rope(_p(x), _p(y), _dt(dtype), rows, D, period, pos0, theta, _s(stream)))
+
+
+def csa_token_importance_scratch_bytes(B, S, Hq, Hkv, n_obs) -> int:
+    n = lib.csa_token_importance_scratch_bytes(B, S, Hq, Hkv, n_obs)
+    if n < 0:
+        raise CsaError(1, "csa_token_importance_scratch_bytes: bad sizes")
+    return n
+
+
+def csa_token_importance(Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp, scratch, scratch_bytes,
+                         stream=None):
+    _check(lib.csa_token_importance(_p(Q), _p(K), B, S, Hq, Hkv, D, n_obs, scale, _p(imp),
+                                    _p(scratch), scratch_bytes, _s(stream)))
+
+
+def csa_token_budget(imp, B, S, Hkv, tau, tile, k_seq, k_unit, stream=None):
+    _check(lib.csa_token_budget(_p(imp), B, S, Hkv, tau, tile, _p(k_seq), _p(k_unit), _s(stream)))
+
+
+def csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs) -> int:
+    n = lib.csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs)
+    if n < 0:
+        raise CsaError(1, "csa_token_sparse_workspace_bytes: bad sizes")
+    return n
+
+
+def csa_token_sparse_prefill(Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale, workspace,
+                             workspace_bytes, O, budget_out, stream=None):
+    """Token Sparse Attention prefill: importance, coverage budget, each KV
+    head's own tokens, dense causal attention of the compressed sequences,
+    scatter back (see include/csa.h)."""
+    _check(lib.csa_token_sparse_prefill(_p(Q), _p(K), _p(V), B, S, Hq, Hkv, D, n_obs, tau, scale,
+                                        _p(workspace), workspace_bytes, _p(O), _p(budget_out),
+                                        _s(stream)))
 
 
 def csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts) -> int:

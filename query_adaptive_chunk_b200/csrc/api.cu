@@ -725,4 +725,156 @@ csa_status csa_block_sparse_prefill(const void* Q, const void* K, const void* V,
   return finish(e, "block-sparse prefill launch");
 }
 
+
+// ---------------------------------------------------------------- token-level sparsity
+
+int64_t csa_token_importance_scratch_bytes(int B, int S, int Hq, int Hkv, int n_obs) {
+  if (B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_obs <= 0) return -1;
+  return static_cast<int64_t>(csa::token_importance_scratch_bytes(B, S, Hkv, Hq / Hkv, n_obs));
+}
+
+namespace {
+csa_status importance_checks(const void* Q, const void* K, int B, int S, int Hq, int Hkv, int D,
+                             int n_obs, float scale) {
+  CSA_REQUIRE(B >= 0 && S >= 0 && Hq > 0 && Hkv > 0 && D > 0 && n_obs > 0, "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_REQUIRE(n_obs <= S || S == 0, "n_obs must be <= S");
+  CSA_SUPPORT(D == 64 || D == 128, "D must be 64 or 128");
+  CSA_SUPPORT(n_obs % 8 == 0 && (Hq / Hkv) * n_obs <= 512,
+              "n_obs a multiple of 8 and (Hq/Hkv) * n_obs <= 512");
+  CSA_REQUIRE(scale == scale && scale > 0.f, "scale must be positive");
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  CSA_TRY(check_ptr(Q, "Q"));
+  CSA_TRY(check_ptr(K, "K"));
+  return CSA_OK;
+}
+}  // namespace
+
+csa_status csa_token_importance(const void* Q, const void* K, int B, int S, int Hq, int Hkv,
+                                int D, int n_obs, float scale, float* imp, void* scratch,
+                                int64_t scratch_bytes, csa_stream stream) {
+  CSA_TRY(importance_checks(Q, K, B, S, Hq, Hkv, D, n_obs, scale));
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  CSA_REQUIRE(scratch_bytes >= csa_token_importance_scratch_bytes(B, S, Hq, Hkv, n_obs),
+              "scratch smaller than csa_token_importance_scratch_bytes()");
+  CSA_TRY(check_ptr(imp, "imp"));
+  CSA_TRY(check_ptr(scratch, "scratch"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_token_importance(l, Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp,
+                                             static_cast<float*>(scratch)),
+                "token importance launch");
+}
+
+csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, float tau, int tile,
+                            int32_t* k_seq, int32_t* k_unit, csa_stream stream) {
+  CSA_REQUIRE(B >= 0 && S >= 0 && Hkv > 0 && tile > 0, "bad sizes");
+  CSA_REQUIRE(tau == tau && tau >= 0.f && tau < 1.f, "tau must be in [0, 1)");
+  CSA_SUPPORT(S <= 32768, "S must be <= 32768");
+  if (B == 0) return CSA_OK;
+  CSA_TRY(check_ptr(imp, "imp"));
+  CSA_TRY(check_ptr(k_seq, "k_seq"));
+  CSA_TRY(check_ptr(k_unit, "k_unit"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_token_budget(l, imp, B, S, Hkv, tau, tile, k_seq, k_unit),
+                "token budget launch");
+}
+
+namespace {
+struct TsaLayout {
+  size_t imp, scratch, k_unit, idx, count, qc, kc, vc, oc, lists, counts2, inv, total;
+};
+TsaLayout tsa_layout(int B, int S, int Hq, int Hkv, int D, int n_obs) {
+  auto r = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t U = static_cast<size_t>(B) * Hkv, T = S / 64;
+  TsaLayout w;
+  size_t o = 0;
+  w.imp = o; o += r(U * S * 4);
+  w.scratch = o; o += r(csa::token_importance_scratch_bytes(B, S, Hkv, Hq / Hkv, n_obs));
+  w.k_unit = o; o += r(U * 4);
+  w.idx = o; o += r(U * S * 4);
+  w.count = o; o += r(U * 4);
+  w.qc = o; o += r(static_cast<size_t>(B) * S * Hq * D * 2);
+  w.kc = o; o += r(U * S * D * 2);
+  w.vc = o; o += r(U * S * D * 2);
+  w.oc = o; o += r(static_cast<size_t>(B) * S * Hq * D * 2);
+  w.lists = o; o += r(U * T * T * 4);
+  w.counts2 = o; o += r(U * T * 4);
+  w.inv = o; o += r(U * S * 4);
+  w.total = o;
+  return w;
+}
+}  // namespace
+
+int64_t csa_token_sparse_workspace_bytes(int B, int S, int Hq, int Hkv, int D, int n_obs) {
+  if (B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || n_obs <= 0 ||
+      S % 64 != 0)
+    return -1;
+  return static_cast<int64_t>(tsa_layout(B, S, Hq, Hkv, D, n_obs).total);
+}
+
+csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V, int B, int S,
+                                    int Hq, int Hkv, int D, int n_obs, float tau, float scale,
+                                    void* workspace, int64_t workspace_bytes, void* O,
+                                    int32_t* budget_out, csa_stream stream) {
+  CSA_TRY(importance_checks(Q, K, B, S, Hq, Hkv, D, n_obs, scale));
+  CSA_REQUIRE(tau == tau && tau >= 0.f && tau < 1.f, "tau must be in [0, 1)");
+  CSA_REQUIRE(S % 64 == 0, "S must be a multiple of 64");
+  CSA_SUPPORT(D == 128 && Hq / Hkv == 4 && S <= 32768,
+              "implemented for D = 128, Hq/Hkv = 4 and S <= 32768");
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  const TsaLayout w = tsa_layout(B, S, Hq, Hkv, D, n_obs);
+  CSA_REQUIRE(workspace_bytes >= static_cast<int64_t>(w.total),
+              "workspace smaller than csa_token_sparse_workspace_bytes()");
+  CSA_TRY(check_ptr(V, "V"));
+  CSA_TRY(check_ptr(workspace, "workspace"));
+  CSA_TRY(check_ptr(O, "O"));
+  CSA_TRY(check_ptr(budget_out, "budget_out"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* imp = reinterpret_cast<float*>(ws + w.imp);
+  int32_t* k_unit = reinterpret_cast<int32_t*>(ws + w.k_unit);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + w.count);
+  const int U = B * Hkv;
+  cudaError_t e = csa::launch_token_importance(l, Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp,
+                                               reinterpret_cast<float*>(ws + w.scratch));
+  if (e == cudaSuccess) e = csa::launch_token_budget(l, imp, B, S, Hkv, tau, 64, budget_out, k_unit);
+  if (e == cudaSuccess)  // each KV head's own top tokens under the (rounded) budget
+    e = csa::launch_select_topk(l, imp, U, S, nullptr, 0, 0, 0, idx, cnt, S, k_unit);
+  if (e != cudaSuccess) return finish(e, "token selection launch");
+  // The compressed length sizes the dense attention: read back the budgets.
+  std::vector<int32_t> ku(U);
+  e = cudaMemcpyAsync(ku.data(), k_unit, U * sizeof(int32_t), cudaMemcpyDeviceToHost, l.stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(l.stream);
+  if (e != cudaSuccess) return finish(e, "token budget read-back");
+  int Sc = 0;
+  for (int v : ku) Sc = std::max(Sc, v);
+  if (Sc <= 0 || Sc > S || Sc % 64 != 0) {
+    if (Sc != 0) return fail(CSA_ERR_CUDA, "token budget out of range");
+  }
+  void* Qc = ws + w.qc;
+  void* Kc = ws + w.kc;
+  void* Vc = ws + w.vc;
+  void* Oc = ws + w.oc;
+  if (Sc > 0) {
+    e = csa::launch_tsa_gather(l, Q, K, V, idx, cnt, S, B, S, Sc, Hq, Hkv, D, Qc, Kc, Vc);
+    const int T = Sc / 64;
+    int32_t* lists = reinterpret_cast<int32_t*>(ws + w.lists);
+    int32_t* counts2 = reinterpret_cast<int32_t*>(ws + w.counts2);
+    if (e == cudaSuccess) e = csa::launch_tsa_lists(l, k_unit, U, T, 64, lists, counts2);
+    std::string why;
+    if (e == cudaSuccess)
+      e = csa::launch_prefill(l, Qc, Kc, Vc, lists, counts2, T, B, Sc, Hq, Hkv, D, 64, 64, scale,
+                              Oc, &why);
+    if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  }
+  if (e == cudaSuccess)
+    e = csa::launch_tsa_scatter(l, Oc, idx, cnt, S, B, S, Sc, Hq, Hkv, D,
+                                reinterpret_cast<int32_t*>(ws + w.inv), O);
+  return finish(e, "token sparse prefill launch");
+}
+
 }  // extern "C"

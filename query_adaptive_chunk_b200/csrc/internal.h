@@ -38,7 +38,8 @@ cudaError_t launch_score(const Launch& l, const void* q, bool bf16, const float*
 // select.cu
 cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
-                               int32_t* idx, int32_t* count, int kmax);
+                               int32_t* idx, int32_t* count, int kmax,
+                               const int32_t* k_dev = nullptr);
 cudaError_t launch_select_topp(const Launch& l, const float* scores, int U, int C,
                                float logit_scale, float p, int budget, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax, int32_t* n_p_out);
@@ -57,6 +58,22 @@ cudaError_t launch_score_select_topp(const Launch& l, const void* q, bool bf16, 
                                      const uint8_t* head_full, float logit_scale, float p,
                                      int budget, int n_sink, int n_local, int32_t* idx,
                                      int32_t* count, int kmax, int32_t* n_p_out);
+
+// token_sparse.cu
+size_t token_importance_scratch_bytes(int B, int S, int Hkv, int G, int n_obs);
+cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* K, int B, int S,
+                                    int Hq, int Hkv, int D, int n_obs, float scale, float* imp,
+                                    float* scratch);
+cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S, int Hkv,
+                                float tau, int tile, int32_t* k_seq, int32_t* k_unit);
+cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, const void* V,
+                              const int32_t* idx, const int32_t* count, int kmax, int B, int S,
+                              int Sc, int Hq, int Hkv, int D, void* Qc, void* Kc, void* Vc);
+cudaError_t launch_tsa_lists(const Launch& l, const int32_t* k_unit, int U, int n_tiles, int tile,
+                             int32_t* lists, int32_t* counts);
+cudaError_t launch_tsa_scatter(const Launch& l, const void* Oc, const int32_t* idx,
+                               const int32_t* count, int kmax, int B, int S, int Sc, int Hq,
+                               int Hkv, int D, int32_t* inv, void* O);
 
 // rope.cu
 cudaError_t launch_rope(const Launch& l, const void* x, void* y, bool bf16, int64_t rows, int D,

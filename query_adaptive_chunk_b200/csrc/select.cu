@@ -218,7 +218,8 @@ __device__ void topk_from_keys(const uint32_t* keys, uint8_t* flags, int v, int 
 
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
     const float* __restrict__ scores, int C, const int32_t* __restrict__ n_valid, int k_free,
-    int n_sink, int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
+    int n_sink, int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax,
+    const int32_t* __restrict__ k_dev) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
   __shared__ BucketScratch bs;
@@ -235,7 +236,9 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
     flags[c] = f ? 1 : 0;
   }
   __syncthreads();
-  topk_from_keys(keys, flags, v, n_sink, n_local, k_free, idx + static_cast<int64_t>(u) * kmax,
+  // k_dev: a per-unit k computed on the device (token budgets), else k_free
+  const int k = k_dev ? max(0, min(k_dev[u], kmax)) : k_free;
+  topk_from_keys(keys, flags, v, n_sink, n_local, k, idx + static_cast<int64_t>(u) * kmax,
                  count + u, kmax, s, exch, bs);
 }
 
@@ -1191,13 +1194,13 @@ cudaError_t set_smem(const void* fn, size_t bytes) {
 
 cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
-                               int32_t* idx, int32_t* count, int kmax) {
+                               int32_t* idx, int32_t* count, int kmax, const int32_t* k_dev) {
   if (U == 0) return cudaSuccess;
   const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_topk_kernel), sh);
   if (e != cudaSuccess) return e;
   select_topk_kernel<<<U, kSelThreads, sh, l.stream>>>(scores, C, n_valid, k_free, n_sink, n_local,
-                                                       idx, count, kmax);
+                                                       idx, count, kmax, k_dev);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,528 @@
+// Token Sparse Attention for prefill (gist.science/ko/paper/2602.03216,
+// section 2): which tokens each KV head keeps, and the gather / scatter
+// around the dense causal attention of the kept tokens.
+//
+//   importance   a proxy attention map of the last n_obs query rows of every
+//                query head against all keys of its KV head; the importance
+//                of key j is the sum over those rows of its softmax weight
+//                (the rows of the GQA group's heads summed: one importance
+//                per KV head).  Two passes over K on the tensor cores
+//                (mma.m16n8k16, keys as M, query rows as N): per-row max and
+//                sum over key blocks, then, with the rows' final max and sum,
+//                the weights summed per key.  HBM-bound on K (read twice).
+//   budget       Dynamic Token Coverage: the fewest tokens whose importance
+//                (summed over the KV heads, normalised) reaches 1 - tau, i.e.
+//                the least important ones are dropped while their mass stays
+//                within tau.  One CTA per sequence: an MSB-first radix select
+//                over the masses' bits that carries each bucket's mass, so
+//                the cut is found without sorting.  The budget is rounded up
+//                to whole 64-row tiles for the dense attention.
+//   gather       per KV head, its kept tokens' K and V rows and the group's
+//                query rows, in position order, into dense compressed
+//                tensors (rows past a sequence's budget are zero).
+//   scatter      the compressed output back to the kept positions; every
+//                other row of the output is 0 (the residual path carries the
+//                skipped tokens in the model).
+#include "internal.h"
+
+namespace csa {
+namespace {
+
+constexpr int kImpThreads = 128;  // 4 warps
+constexpr int kImpKeys = 128;     // keys per CTA, 32 per warp
+constexpr float kLog2eF = 1.4426950408889634f;
+
+// Row r of the observed block of KV head h: query head h*G + r / n_obs at
+// position S - n_obs + r % n_obs.
+__device__ __forceinline__ int obs_pos(int r, int n_obs, int S) { return S - n_obs + r % n_obs; }
+
+// Loads the observed query rows of (b, h) [R][D] and the key block [128][D]
+// into padded shared memory (row stride D + 8 bf16: conflict-free fragment loads).
+template <int D>
+__device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, int h, int S,
+                         int Hq, int Hkv, int G, int n_obs, int j0, __nv_bfloat16* qs,
+                         __nv_bfloat16* ks) {
+  constexpr int LD = D + 8, V8 = D / 8;
+  const int R = G * n_obs;
+  for (int e = threadIdx.x; e < R * V8; e += blockDim.x) {
+    const int r = e / V8, c = (e % V8) * 8;
+    const int g = r / n_obs, pos = obs_pos(r, n_obs, S);
+    const int4 v = *reinterpret_cast<const int4*>(
+        Q + ((static_cast<int64_t>(b) * S + pos) * Hq + h * G + g) * D + c);
+    *reinterpret_cast<int4*>(qs + r * LD + c) = v;
+  }
+  const __nv_bfloat16* kb = K + ((static_cast<int64_t>(b) * Hkv + h) * S) * D;
+  for (int e = threadIdx.x; e < kImpKeys * V8; e += blockDim.x) {
+    const int r = e / V8, c = (e % V8) * 8;
+    const int j = j0 + r;
+    int4 v = make_int4(0, 0, 0, 0);
+    if (j < S) v = *reinterpret_cast<const int4*>(kb + static_cast<int64_t>(j) * D + c);
+    *reinterpret_cast<int4*>(ks + r * LD + c) = v;
+  }
+}
+
+// S^T tile of this warp's 32 keys (two 16-key m-tiles) against query rows
+// [n0 .. n0 + 8): acc[mt][0..3] as the mma C layout (key = lane/4 (+8),
+// row = n0 + 2 (lane%4) (+1)); scaled to the log2 domain.
+template <int D>
+__device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const __nv_bfloat16* ks,
+                                         int kw, int n0, float sl2, float (&acc)[2][4]) {
+  constexpr int LD = D + 8;
+  const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+#pragma unroll
+  for (int k0 = 0; k0 < D; k0 += 16) {
+    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qs + (n0 + rr) * LD + k0 + cc);
+    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qs + (n0 + rr) * LD + k0 + cc + 8);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const __nv_bfloat16* kr = ks + (kw + mt * 16 + rr) * LD + k0 + cc;
+      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(kr);
+      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(kr + 8 * LD);
+      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(kr + 8);
+      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(kr + 8 * LD + 8);
+      mma_bf16_16816(acc[mt], a0, a1, a2, a3, b0, b1);
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[mt][e] *= sl2;
+}
+
+// Pass 1: per (b, h, key block) and observed row, the max and the sum of
+// 2^(s - max) over the block's visible keys -> part [b, h, block, R, 2].
+template <int D>
+__global__ void __launch_bounds__(kImpThreads) imp_stats_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, int S, int Hq,
+    int Hkv, int G, int n_obs, float sl2, float* __restrict__ part) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  constexpr int LD = D + 8;
+  const int R = G * n_obs;
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);
+  __nv_bfloat16* ks = qs + R * LD;
+  float* red = reinterpret_cast<float*>(ks + kImpKeys * LD);  // [4 warps][R][2]
+  const int nblk = gridDim.x, blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int j0 = blk * kImpKeys;
+  imp_load<D>(Q, K, b, h, S, Hq, Hkv, G, n_obs, j0, qs, ks);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kw = warp * 32, rr = lane >> 2, cc = 2 * (lane & 3);
+  for (int n0 = 0; n0 < R; n0 += 8) {
+    float acc[2][4];
+    imp_tile<D>(qs, ks, kw, n0, sl2, acc);
+    // this lane: rows n0 + cc, n0 + cc + 1; keys j0 + kw + {rr, rr+8, rr+16, rr+24}
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = j0 + kw + mt * 16 + rr + (e >> 1) * 8, r = n0 + cc + (e & 1);
+        if (j >= S || j > obs_pos(r, n_obs, S)) acc[mt][e] = -INFINITY;
+        mx[e & 1] = fmaxf(mx[e & 1], acc[mt][e]);
+      }
+#pragma unroll
+    for (int x = 4; x < 32; x <<= 1) {
+      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], x));
+      mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], x));
+    }
+    float sm_[2] = {0.f, 0.f};
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (mx[e & 1] != -INFINITY) sm_[e & 1] += exp2f(acc[mt][e] - mx[e & 1]);
+#pragma unroll
+    for (int x = 4; x < 32; x <<= 1) {
+      sm_[0] += __shfl_xor_sync(0xffffffffu, sm_[0], x);
+      sm_[1] += __shfl_xor_sync(0xffffffffu, sm_[1], x);
+    }
+    if (rr == 0) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        red[(warp * R + n0 + cc + t) * 2] = mx[t];
+        red[(warp * R + n0 + cc + t) * 2 + 1] = sm_[t];
+      }
+    }
+  }
+  __syncthreads();
+  float* out = part + ((static_cast<int64_t>(b) * Hkv + h) * nblk + blk) * R * 2;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    float m = -INFINITY, l = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      const float mw = red[(w * R + r) * 2], lw = red[(w * R + r) * 2 + 1];
+      if (mw == -INFINITY) continue;
+      const float mn = fmaxf(m, mw);
+      l = l * exp2f(m - mn) + lw * exp2f(mw - mn);
+      m = mn;
+    }
+    out[r * 2] = m;
+    out[r * 2 + 1] = l;
+  }
+}
+
+// The rows' max and sum over all key blocks: part -> stats [b, h, R, 2]
+// (one CTA per (b, h)).
+__global__ void imp_combine_kernel(const float* __restrict__ part, int nblk, int R,
+                                   float* __restrict__ stats) {
+  const int64_t bh = blockIdx.x;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    float m = -INFINITY, l = 0.f;
+    for (int k = 0; k < nblk; ++k) {
+      const float mw = part[((bh * nblk + k) * R + r) * 2], lw = part[((bh * nblk + k) * R + r) * 2 + 1];
+      if (mw == -INFINITY) continue;
+      const float mn = fmaxf(m, mw);
+      l = l * exp2f(m - mn) + lw * exp2f(mw - mn);
+      m = mn;
+    }
+    stats[(bh * R + r) * 2] = m;
+    stats[(bh * R + r) * 2 + 1] = l;
+  }
+}
+
+// Pass 2: importance of each key = sum over the observed rows of
+// 2^(s - max_r) / sum_r -> imp [b, h, S].
+template <int D>
+__global__ void __launch_bounds__(kImpThreads) imp_weight_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, int S, int Hq,
+    int Hkv, int G, int n_obs, float sl2, const float* __restrict__ stats, float* __restrict__ imp) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  constexpr int LD = D + 8;
+  const int R = G * n_obs;
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);
+  __nv_bfloat16* ks = qs + R * LD;
+  float* st = reinterpret_cast<float*>(ks + kImpKeys * LD);  // [R][2]: max, 1/sum
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int j0 = blk * kImpKeys;
+  const int64_t bh = static_cast<int64_t>(b) * Hkv + h;
+  imp_load<D>(Q, K, b, h, S, Hq, Hkv, G, n_obs, j0, qs, ks);
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    st[r * 2] = stats[(bh * R + r) * 2];
+    const float l = stats[(bh * R + r) * 2 + 1];
+    st[r * 2 + 1] = l > 0.f ? 1.0f / l : 0.f;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kw = warp * 32, rr = lane >> 2, cc = 2 * (lane & 3);
+  float wsum[4] = {0.f, 0.f, 0.f, 0.f};  // keys kw + rr + 8 t
+  for (int n0 = 0; n0 < R; n0 += 8) {
+    float acc[2][4];
+    imp_tile<D>(qs, ks, kw, n0, sl2, acc);
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = mt * 2 + (e >> 1);
+        const int j = j0 + kw + rr + t * 8, r = n0 + cc + (e & 1);
+        if (j < S && j <= obs_pos(r, n_obs, S))
+          wsum[t] += exp2f(acc[mt][e] - st[r * 2]) * st[r * 2 + 1];
+      }
+  }
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    wsum[t] += __shfl_xor_sync(0xffffffffu, wsum[t], 1);
+    wsum[t] += __shfl_xor_sync(0xffffffffu, wsum[t], 2);
+  }
+  if ((lane & 3) == 0) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int j = j0 + kw + rr + t * 8;
+      if (j < S) imp[bh * S + j] = wsum[t];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- budget
+
+constexpr int kBudgetThreads = 1024;
+
+// One CTA per sequence b: the masses m_j = sum_h imp[b,h,j] (kept in shared
+// memory), then the smallest k whose k largest masses reach (1 - tau) of the
+// total.  Non-negative floats order like their bit patterns, so an MSB-first
+// radix select over the bits, carrying each bucket's count and mass, finds
+// the cut value; equal masses at the cut are taken as few as needed.
+// k_seq[b] = k; k_unit[b*Hkv + h] = k rounded up to whole `tile`s (<= S).
+__global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __restrict__ imp,
+                                                                int S, int Hkv, float tau, int tile,
+                                                                int32_t* __restrict__ k_seq,
+                                                                int32_t* __restrict__ k_unit) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  float* ms = reinterpret_cast<float*>(sm);  // [S]
+  __shared__ unsigned int hc[256];
+  __shared__ float hm[256];
+  __shared__ float wsum[32];
+  __shared__ unsigned int sel_sh, prefix_sh;
+  __shared__ float above_m_sh;
+  __shared__ unsigned int above_c_sh;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const float* ib = imp + static_cast<int64_t>(b) * Hkv * S;
+  float part = 0.f;
+  for (int j = tid; j < S; j += blockDim.x) {
+    float m = 0.f;
+    for (int h = 0; h < Hkv; ++h) m += ib[static_cast<int64_t>(h) * S + j];
+    m = fmaxf(m, 0.f);
+    ms[j] = m;
+    part += m;
+  }
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) part += __shfl_xor_sync(0xffffffffu, part, x);
+  if ((tid & 31) == 0) wsum[tid >> 5] = part;
+  if (tid == 0) {
+    prefix_sh = 0u;
+    above_m_sh = 0.f;
+    above_c_sh = 0u;
+  }
+  __syncthreads();
+  float total = 0.f;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) total += wsum[w];
+  const float target = (1.0f - tau) * total;
+  unsigned int mask = 0u;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int d = tid; d < 256; d += blockDim.x) {
+      hc[d] = 0u;
+      hm[d] = 0.f;
+    }
+    __syncthreads();
+    const unsigned int prefix = prefix_sh;
+    for (int j = tid; j < S; j += blockDim.x) {
+      const unsigned int key = __float_as_uint(ms[j]);
+      if ((key & mask) == prefix) {
+        const int d = (key >> shift) & 255u;
+        atomicAdd(&hc[d], 1u);
+        atomicAdd(&hm[d], ms[j]);
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      float am = above_m_sh;
+      unsigned int ac = above_c_sh;
+      int sel = -1, low = -1;
+      for (int d = 255; d >= 0; --d) {
+        if (hc[d] == 0u) continue;
+        if (am + hm[d] >= target) {
+          sel = d;
+          break;
+        }
+        am += hm[d];
+        ac += hc[d];
+        low = d;
+      }
+      if (sel < 0) {  // the sums fell short of the target by rounding: cut in the lowest bucket
+        sel = low < 0 ? 0 : low;
+        if (low >= 0) {
+          am -= hm[low];
+          ac -= hc[low];
+        }
+      }
+      above_m_sh = am;
+      above_c_sh = ac;
+      sel_sh = static_cast<unsigned int>(sel);
+      prefix_sh = prefix | (static_cast<unsigned int>(sel) << shift);
+    }
+    __syncthreads();
+    mask |= 255u << shift;
+    if (shift == 0) break;
+  }
+  if (tid == 0) {
+    int k;
+    if (!(target > 0.f)) {
+      k = 0;
+    } else {
+      const float v = __uint_as_float(prefix_sh);
+      const unsigned int n_eq = hc[sel_sh];
+      const float need = target - above_m_sh;
+      unsigned int take = n_eq;
+      if (v > 0.f && need > 0.f) {
+        const float t = ceilf(need / v);
+        take = t < static_cast<float>(n_eq) ? static_cast<unsigned int>(fmaxf(t, 1.f)) : n_eq;
+      } else if (!(need > 0.f)) {
+        take = 0u;
+      }
+      k = static_cast<int>(above_c_sh + take);
+    }
+    k = min(k, S);
+    k_seq[b] = k;
+    const int kt = min(S, (k + tile - 1) / tile * tile);
+    for (int h = 0; h < Hkv; ++h) k_unit[static_cast<int64_t>(b) * Hkv + h] = kt;
+  }
+}
+
+// ---------------------------------------------------------------- gather / scatter
+
+// Compressed row t of (b, h): the kept token idx[u, t] (t < count[u]) or a
+// zero row.  Q^ [B, Sc, Hq, D] takes the G query heads of the group; K^, V^
+// [B, Hkv, Sc, D].  16 bytes per thread.
+__global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
+                                  const __nv_bfloat16* __restrict__ K,
+                                  const __nv_bfloat16* __restrict__ V,
+                                  const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
+                                  int kmax, int S, int Sc, int Hq, int Hkv, int D,
+                                  __nv_bfloat16* __restrict__ Qc, __nv_bfloat16* __restrict__ Kc,
+                                  __nv_bfloat16* __restrict__ Vc) {
+  const int G = Hq / Hkv, V8 = D / 8;
+  const int per_row = (G + 2) * V8;  // 16-byte pieces of one compressed row of (b, h)
+  const int64_t u = blockIdx.y;      // b * Hkv + h
+  const int b = static_cast<int>(u / Hkv), h = static_cast<int>(u % Hkv);
+  const int n = count[u];
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       e < static_cast<int64_t>(Sc) * per_row; e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(e / per_row), w = static_cast<int>(e % per_row);
+    const int part = w / V8, c = (w % V8) * 8;
+    const int p = t < n ? idx[u * kmax + t] : -1;
+    int4 v = make_int4(0, 0, 0, 0);
+    if (part < G) {  // query head h*G + part
+      if (p >= 0)
+        v = *reinterpret_cast<const int4*>(Q + ((static_cast<int64_t>(b) * S + p) * Hq + h * G + part) * D + c);
+      *reinterpret_cast<int4*>(Qc + ((static_cast<int64_t>(b) * Sc + t) * Hq + h * G + part) * D + c) = v;
+    } else {
+      const __nv_bfloat16* src = part == G ? K : V;
+      __nv_bfloat16* dst = part == G ? Kc : Vc;
+      if (p >= 0) v = *reinterpret_cast<const int4*>(src + (u * S + p) * D + c);
+      *reinterpret_cast<int4*>(dst + (u * Sc + t) * D + c) = v;
+    }
+  }
+}
+
+// Dense causal chunk lists of the compressed sequences: tile t of (b, h)
+// sees chunks 0..t (chunk = tile = 64 rows); tiles past the budget of
+// sequence b see none (their rows are padding and come out 0).
+__global__ void tsa_lists_kernel(const int32_t* __restrict__ k_unit, int n_tiles, int tile,
+                                 int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
+  const int64_t ut = blockIdx.x;  // (b * Hkv + h) * n_tiles + t
+  const int t = static_cast<int>(ut % n_tiles);
+  const int64_t u = ut / n_tiles;
+  const bool live = t * tile < k_unit[u];
+  for (int c = threadIdx.x; c < n_tiles; c += blockDim.x)
+    lists[ut * n_tiles + c] = (live && c <= t) ? c : -1;
+  if (threadIdx.x == 0) counts[ut] = live ? t + 1 : 0;
+}
+
+__global__ void tsa_inverse_kernel(const int32_t* __restrict__ idx,
+                                   const int32_t* __restrict__ count, int kmax, int S,
+                                   int32_t* __restrict__ inv) {
+  const int64_t u = blockIdx.x;
+  for (int s = threadIdx.x; s < S; s += blockDim.x) inv[u * S + s] = -1;
+  __syncthreads();
+  const int n = count[u];
+  for (int t = threadIdx.x; t < n; t += blockDim.x) {
+    const int p = idx[u * kmax + t];
+    if (p >= 0 && p < S) inv[u * S + p] = t;
+  }
+}
+
+// O[b, s, h*G + g] = O^[b, inv, h*G + g] for kept positions, else 0.
+__global__ void tsa_scatter_kernel(const __nv_bfloat16* __restrict__ Oc,
+                                   const int32_t* __restrict__ inv, int S, int Sc, int Hq, int Hkv,
+                                   int D, int B, __nv_bfloat16* __restrict__ O) {
+  const int G = Hq / Hkv, V8 = D / 8;
+  const int64_t total = static_cast<int64_t>(B) * S * Hq * V8;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(e % V8) * 8;
+    const int64_t row = e / V8;  // (b * S + s) * Hq + hq
+    const int hq = static_cast<int>(row % Hq);
+    const int64_t bs = row / Hq;
+    const int s = static_cast<int>(bs % S), b = static_cast<int>(bs / S);
+    const int t = inv[(static_cast<int64_t>(b) * Hkv + hq / G) * S + s];
+    int4 v = make_int4(0, 0, 0, 0);
+    if (t >= 0)
+      v = *reinterpret_cast<const int4*>(Oc + ((static_cast<int64_t>(b) * Sc + t) * Hq + hq) * D + c);
+    *reinterpret_cast<int4*>(O + row * D + c) = v;
+  }
+}
+
+cudaError_t set_smem_ts(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes));
+}
+
+}  // namespace
+
+cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S, int Hkv,
+                                float tau, int tile, int32_t* k_seq, int32_t* k_unit) {
+  if (B == 0) return cudaSuccess;
+  const size_t sh = static_cast<size_t>(S) * 4;
+  cudaError_t e = set_smem_ts(reinterpret_cast<const void*>(budget_kernel), sh);
+  if (e != cudaSuccess) return e;
+  budget_kernel<<<B, kBudgetThreads, sh, l.stream>>>(imp, S, Hkv, tau, tile, k_seq, k_unit);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, const void* V,
+                              const int32_t* idx, const int32_t* count, int kmax, int B, int S,
+                              int Sc, int Hq, int Hkv, int D, void* Qc, void* Kc, void* Vc) {
+  if (B == 0 || Sc == 0) return cudaSuccess;
+  const dim3 grid(4 * l.num_sms / (B * Hkv) + 1, B * Hkv);
+  tsa_gather_kernel<<<grid, 256, 0, l.stream>>>(
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
+      static_cast<const __nv_bfloat16*>(V), idx, count, kmax, S, Sc, Hq, Hkv, D,
+      static_cast<__nv_bfloat16*>(Qc), static_cast<__nv_bfloat16*>(Kc),
+      static_cast<__nv_bfloat16*>(Vc));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tsa_lists(const Launch& l, const int32_t* k_unit, int U, int n_tiles, int tile,
+                             int32_t* lists, int32_t* counts) {
+  if (U == 0 || n_tiles == 0) return cudaSuccess;
+  tsa_lists_kernel<<<U * n_tiles, 128, 0, l.stream>>>(k_unit, n_tiles, tile, lists, counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tsa_scatter(const Launch& l, const void* Oc, const int32_t* idx,
+                               const int32_t* count, int kmax, int B, int S, int Sc, int Hq,
+                               int Hkv, int D, int32_t* inv, void* O) {
+  if (B == 0 || S == 0) return cudaSuccess;
+  tsa_inverse_kernel<<<B * Hkv, 512, 0, l.stream>>>(idx, count, kmax, S, inv);
+  tsa_scatter_kernel<<<8 * l.num_sms, 256, 0, l.stream>>>(
+      static_cast<const __nv_bfloat16*>(Oc), inv, S, Sc, Hq, Hkv, D, B,
+      static_cast<__nv_bfloat16*>(O));
+  return cudaGetLastError();
+}
+
+size_t token_importance_scratch_bytes(int B, int S, int Hkv, int G, int n_obs) {
+  const int64_t nblk = (S + kImpKeys - 1) / kImpKeys;
+  const int64_t R = static_cast<int64_t>(G) * n_obs;
+  return static_cast<size_t>(B) * Hkv * R * 2 * 4 * (nblk + 1);
+}
+
+cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* K, int B, int S,
+                                    int Hq, int Hkv, int D, int n_obs, float scale, float* imp,
+                                    float* scratch) {
+  if (B == 0 || S == 0) return cudaSuccess;
+  const int G = Hq / Hkv, R = G * n_obs;
+  const int nblk = (S + kImpKeys - 1) / kImpKeys;
+  float* part = scratch;
+  float* stats = scratch + static_cast<size_t>(B) * Hkv * nblk * R * 2;
+  const size_t lds = static_cast<size_t>(D + 8) * 2;
+  const size_t sh1 = (R + kImpKeys) * lds + 4 * static_cast<size_t>(R) * 2 * 4;
+  const size_t sh2 = (R + kImpKeys) * lds + static_cast<size_t>(R) * 2 * 4;
+  const dim3 grid(nblk, Hkv, B);
+  const float sl2 = scale * kLog2eF;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K);
+  cudaError_t e;
+  if (D == 128) {
+    e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<128>), sh1);
+    if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<128>), sh2);
+    if (e != cudaSuccess) return e;
+    imp_stats_kernel<128><<<grid, kImpThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
+    imp_combine_kernel<<<B * Hkv, 256, 0, l.stream>>>(part, nblk, R, stats);
+    imp_weight_kernel<128><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
+                                                                 stats, imp);
+  } else {
+    e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<64>), sh1);
+    if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<64>), sh2);
+    if (e != cudaSuccess) return e;
+    imp_stats_kernel<64><<<grid, kImpThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
+    imp_combine_kernel<<<B * Hkv, 256, 0, l.stream>>>(part, nblk, R, stats);
+    imp_weight_kernel<64><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
+                                                                stats, imp);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace csa
