@@ -329,6 +329,46 @@ def time_prefill(w, steps: int, warmup: int, flush):
     return {"select_ms": sel_ms, "attend_ms": att_ms, "blocks": blocks, "flops": flops}
 
 
+def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1):
+    """Token Sparse Attention prefill on the 32K prefill inputs: the whole
+    call (importance, budget, token choice, gather, dense causal attention of
+    the kept tokens, scatter) between two events.  The call reads the budget
+    back to the host once (so it is not graph-replayed)."""
+    from query_adaptive_chunk_b200 import csa
+    inp = synth.make_prefill_inputs(w, device="cuda")
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    scale = 1.0 / math.sqrt(w.D)
+    nb = csa.csa_token_sparse_workspace_bytes(w.B, w.S, w.Hq, w.Hkv, w.D, n_obs)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    O = torch.empty_like(Q)
+    budget = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+
+    def call():
+        csa.csa_token_sparse_prefill(Q, K, V, w.B, w.S, w.Hq, w.Hkv, w.D, n_obs, tau, scale, ws,
+                                     nb, O, budget)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    csa.csa_check_device_status()
+    k = int(budget.max())
+    kt = min(w.S, (k + 63) // 64 * 64)
+    n_t = kt // 64
+    # dense causal attention of the kept tokens: tile t sees tiles 0..t
+    flops = w.B * w.Hkv * (n_t * (n_t + 1) // 2) * w.G * 2 * (2 * 64 * 64 * w.D)
+    return {"ms": ms, "budget": k, "kept_tokens": kt, "flops": flops, "n_obs": n_obs,
+            "tau": tau}
+
+
 def oracle_decode_seconds(w, inp, max_seconds: float = 20.0, max_steps: int = 5, threads: int = 1):
     """The CPU oracle's per-step work (score + select + attention, summaries
     precomputed) on this workload, a bounded number of steps.  threads == 1:
@@ -516,6 +556,16 @@ def other_workloads(args, flush, peaks):
         del r
         torch.cuda.empty_cache()
     w = synth.PREFILL_32K
+    r = time_token_sparse(w, steps, args.warmup, flush)
+    ms = statistics.mean(r["ms"])
+    out["token_sparse_prefill_bf16_seq32k"] = {
+        "ms_per_step": round(ms, 4), "n_obs": r["n_obs"], "tau": r["tau"],
+        "budget_tokens": r["budget"], "kept_tokens_per_head": r["kept_tokens"],
+        "kept_fraction": round(r["kept_tokens"] / w.S, 4),
+        "attention_flops": r["flops"],
+        "effective_tflops_whole_step": round(r["flops"] / (ms * 1e-3) / 1e12, 1)}
+    del r
+    torch.cuda.empty_cache()
     r = time_prefill(w, steps, args.warmup, flush)
     att_ms = statistics.mean(r["attend_ms"])
     tflops = r["flops"] / (att_ms * 1e-3) / 1e12
