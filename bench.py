@@ -579,6 +579,11 @@ def other_workloads(args, flush, peaks):
 
 def run_only(args, flush, peaks):
     """Time one named workload alone and print its figures (profiling aid)."""
+    if args.only == "token_sparse_prefill_bf16_seq32k":
+        r = time_token_sparse(synth.PREFILL_32K, args.steps, args.warmup, flush)
+        print(json.dumps({"workload": args.only, "ms": statistics.mean(r["ms"]),
+                          "budget": r["budget"], "flops": r["flops"]}))
+        return 0
     byname = {w.name: w for w in synth.ALL_WORKLOADS}
     w = byname[args.only]
     if isinstance(w, synth.PrefillWorkload):

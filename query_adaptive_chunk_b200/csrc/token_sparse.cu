@@ -61,12 +61,31 @@ __device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, 
   }
 }
 
-// S^T tile of this warp's 32 keys (two 16-key m-tiles) against query rows
-// [n0 .. n0 + 8): acc[mt][0..3] as the mma C layout (key = lane/4 (+8),
-// row = n0 + 2 (lane%4) (+1)); scaled to the log2 domain.
+// This warp's 32 keys (two 16-key m-tiles) as mma A fragments for every
+// 16-wide slice of D, loaded once and reused for every block of query rows.
 template <int D>
-__device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const __nv_bfloat16* ks,
-                                         int kw, int n0, float sl2, float (&acc)[2][4]) {
+__device__ __forceinline__ void imp_load_a(const __nv_bfloat16* ks, int kw,
+                                           uint32_t (&af)[D / 16][2][4]) {
+  constexpr int LD = D + 8;
+  const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
+#pragma unroll
+  for (int ks16 = 0; ks16 < D / 16; ++ks16)
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const __nv_bfloat16* kr = ks + (kw + mt * 16 + rr) * LD + ks16 * 16 + cc;
+      af[ks16][mt][0] = *reinterpret_cast<const uint32_t*>(kr);
+      af[ks16][mt][1] = *reinterpret_cast<const uint32_t*>(kr + 8 * LD);
+      af[ks16][mt][2] = *reinterpret_cast<const uint32_t*>(kr + 8);
+      af[ks16][mt][3] = *reinterpret_cast<const uint32_t*>(kr + 8 * LD + 8);
+    }
+}
+
+// S^T tile of this warp's 32 keys against query rows [n0 .. n0 + 8):
+// acc[mt][0..3] as the mma C layout (key = lane/4 (+8), row = n0 + 2 (lane%4)
+// (+1)); scaled to the log2 domain.
+template <int D>
+__device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const uint32_t (&af)[D / 16][2][4],
+                                         int n0, float sl2, float (&acc)[2][4]) {
   constexpr int LD = D + 8;
   const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
 #pragma unroll
@@ -74,18 +93,14 @@ __device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const __nv_bfl
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
 #pragma unroll
-  for (int k0 = 0; k0 < D; k0 += 16) {
-    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qs + (n0 + rr) * LD + k0 + cc);
-    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qs + (n0 + rr) * LD + k0 + cc + 8);
+  for (int ks16 = 0; ks16 < D / 16; ++ks16) {
+    const __nv_bfloat16* qr = qs + (n0 + rr) * LD + ks16 * 16 + cc;
+    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qr);
+    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qr + 8);
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      const __nv_bfloat16* kr = ks + (kw + mt * 16 + rr) * LD + k0 + cc;
-      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(kr);
-      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(kr + 8 * LD);
-      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(kr + 8);
-      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(kr + 8 * LD + 8);
-      mma_bf16_16816(acc[mt], a0, a1, a2, a3, b0, b1);
-    }
+    for (int mt = 0; mt < 2; ++mt)
+      mma_bf16_16816(acc[mt], af[ks16][mt][0], af[ks16][mt][1], af[ks16][mt][2], af[ks16][mt][3],
+                     b0, b1);
   }
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
@@ -111,9 +126,11 @@ __global__ void __launch_bounds__(kImpThreads) imp_stats_kernel(
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kw = warp * 32, rr = lane >> 2, cc = 2 * (lane & 3);
+  uint32_t af[D / 16][2][4];
+  imp_load_a<D>(ks, kw, af);
   for (int n0 = 0; n0 < R; n0 += 8) {
     float acc[2][4];
-    imp_tile<D>(qs, ks, kw, n0, sl2, acc);
+    imp_tile<D>(qs, af, n0, sl2, acc);
     // this lane: rows n0 + cc, n0 + cc + 1; keys j0 + kw + {rr, rr+8, rr+16, rr+24}
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -208,9 +225,11 @@ __global__ void __launch_bounds__(kImpThreads) imp_weight_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kw = warp * 32, rr = lane >> 2, cc = 2 * (lane & 3);
   float wsum[4] = {0.f, 0.f, 0.f, 0.f};  // keys kw + rr + 8 t
+  uint32_t af[D / 16][2][4];
+  imp_load_a<D>(ks, kw, af);
   for (int n0 = 0; n0 < R; n0 += 8) {
     float acc[2][4];
-    imp_tile<D>(qs, ks, kw, n0, sl2, acc);
+    imp_tile<D>(qs, af, n0, sl2, acc);
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -287,12 +306,31 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
     }
     __syncthreads();
     const unsigned int prefix = prefix_sh;
-    for (int j = tid; j < S; j += blockDim.x) {
-      const unsigned int key = __float_as_uint(ms[j]);
-      if ((key & mask) == prefix) {
-        const int d = (key >> shift) & 255u;
-        atomicAdd(&hc[d], 1u);
-        atomicAdd(&hm[d], ms[j]);
+    // Most masses share a few buckets: lanes of a warp with the same bucket
+    // add their count and mass through one leader (one atomic per bucket per
+    // warp, not per element).
+    const int lane = tid & 31;
+    for (int j0 = 0; j0 < S; j0 += blockDim.x) {
+      const int j = j0 + tid;
+      int d = -1;
+      float m = 0.f;
+      if (j < S) {
+        const unsigned int key = __float_as_uint(ms[j]);
+        if ((key & mask) == prefix) {
+          d = (key >> shift) & 255u;
+          m = ms[j];
+        }
+      }
+      const unsigned int peers = __match_any_sync(0xffffffffu, d);
+      const int leader = __ffs(peers) - 1;
+      float tot = 0.f;
+      for (unsigned int b = peers; b != 0u; b &= b - 1) {  // the group's masses, in lane order
+        const float v = __shfl_sync(peers, m, __ffs(b) - 1);
+        tot += v;
+      }
+      if (d >= 0 && lane == leader) {
+        atomicAdd(&hc[d], static_cast<unsigned int>(__popc(peers)));
+        atomicAdd(&hm[d], tot);
       }
     }
     __syncthreads();
