@@ -36,8 +36,17 @@ constexpr float kLog2eF = 1.4426950408889634f;
 // position S - n_obs + r % n_obs.
 __device__ __forceinline__ int obs_pos(int r, int n_obs, int S) { return S - n_obs + r % n_obs; }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+  // 16-byte asynchronous copy; src-size 0 fills the destination with zeros
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gsrc), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
 // Loads the observed query rows of (b, h) [R][D] and the key block [128][D]
-// into padded shared memory (row stride D + 8 bf16: conflict-free fragment loads).
+// into padded shared memory (row stride D + 8 bf16: conflict-free fragment
+// loads) with asynchronous 16-byte copies, all in flight at once; waits for
+// them (the caller's barrier then publishes them).
 template <int D>
 __device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, int h, int S,
                          int Hq, int Hkv, int G, int n_obs, int j0, __nv_bfloat16* qs,
@@ -47,18 +56,16 @@ __device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, 
   for (int e = threadIdx.x; e < R * V8; e += blockDim.x) {
     const int r = e / V8, c = (e % V8) * 8;
     const int g = r / n_obs, pos = obs_pos(r, n_obs, S);
-    const int4 v = *reinterpret_cast<const int4*>(
-        Q + ((static_cast<int64_t>(b) * S + pos) * Hq + h * G + g) * D + c);
-    *reinterpret_cast<int4*>(qs + r * LD + c) = v;
+    cp_async16(qs + r * LD + c, Q + ((static_cast<int64_t>(b) * S + pos) * Hq + h * G + g) * D + c,
+               true);
   }
   const __nv_bfloat16* kb = K + ((static_cast<int64_t>(b) * Hkv + h) * S) * D;
   for (int e = threadIdx.x; e < kImpKeys * V8; e += blockDim.x) {
     const int r = e / V8, c = (e % V8) * 8;
     const int j = j0 + r;
-    int4 v = make_int4(0, 0, 0, 0);
-    if (j < S) v = *reinterpret_cast<const int4*>(kb + static_cast<int64_t>(j) * D + c);
-    *reinterpret_cast<int4*>(ks + r * LD + c) = v;
+    cp_async16(ks + r * LD + c, kb + static_cast<int64_t>(j < S ? j : 0) * D + c, j < S);
   }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
 // This warp's 32 keys (two 16-key m-tiles) as mma A fragments for every
