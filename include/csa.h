@@ -26,7 +26,8 @@
  *
  * Conventions for every call:
  *   - Every data pointer is a DEVICE pointer (cudaMalloc'd, or managed)
- *     owned by the caller.  The library allocates nothing, frees nothing and
+ *     owned by the caller, except the pinned host buffers of
+ *     csa_decode_step_host.  The library allocates nothing, frees nothing and
  *     never blocks the host; each call enqueues kernels on `stream` (a
  *     cudaStream_t; NULL = legacy default stream) and returns.
  *   - Tensors are dense, row-major (last index fastest), in the layouts given
@@ -474,6 +475,28 @@ typedef struct csa_decode_step_desc {
 } csa_decode_step_desc;
 
 CSA_API csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream);
+
+/* The same step with the query and the result in host memory, for a caller
+ * whose query arrives on the host: q_host ([B, Hq, D] bf16) is brought into
+ * the device buffer d->q, the step of csa_decode_step runs, and its output
+ * ([B, Hq, D] of out_dtype) lands in out_host and, when lse_host is given,
+ * its lse ([B, Hq] fp32; d->lse_out then required) in lse_host.  All on
+ * `stream`, asynchronous: the host reads out_host after synchronising it.
+ * q_host, out_host and lse_host must be pinned host memory (cudaHostAlloc
+ * or cudaHostRegister), else CSA_ERR_INVALID_ARG.  When that memory is
+ * mapped into the device's address space (every pinned allocation under
+ * unified addressing) and 16-byte aligned, the SMs read the query from it
+ * (one small copy kernel) and the decode stores the result straight into
+ * it; d->out and d->lse_out are then left as they were.  Otherwise the
+ * copies are cudaMemcpyAsync transfers and d->out / d->lse_out hold the
+ * result too.  The call captures into a CUDA graph, whose replays read and
+ * write the same host buffers.  CSA_ERR_UNSUPPORTED with q_score set (the
+ * RoPE-aware split rotates the query on the device: csa_rope, then
+ * csa_decode_step).  Once the decode's own arguments have passed their
+ * checks the query copy is enqueued, so a selection argument rejected
+ * after that leaves the copy enqueued (it writes only d->q). */
+CSA_API csa_status csa_decode_step_host(const csa_decode_step_desc* d, const void* q_host,
+                                        void* out_host, float* lse_host, csa_stream stream);
 
 /* ---------------------------------------------------------------- a6
  * Log-sum-exp merge of split-K partials (SSA summary "핵심 기여": split-K

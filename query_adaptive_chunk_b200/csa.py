@@ -78,6 +78,7 @@ _SIGS = {
                                               _i64, _i, _f, _i, _vp, _i, _vp, _vp]),
     "csa_lse_merge": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp]),
     "csa_decode_step": (_i, [_vp, _vp]),
+    "csa_decode_step_host": (_i, [_vp, _vp, _vp, _vp, _vp]),
     "csa_block_sparse_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                       _vp, _vp]),
 }
@@ -329,6 +330,11 @@ def decode_step_desc(**kw) -> DecodeStepDesc:
 
 def csa_decode_step(desc: DecodeStepDesc, stream=None):
     _check(lib.csa_decode_step(ctypes.byref(desc), _s(stream)))
+
+
+def csa_decode_step_host(desc: DecodeStepDesc, q_host, out_host, lse_host=None, stream=None):
+    _check(lib.csa_decode_step_host(ctypes.byref(desc), _p(q_host), _p(out_host), _p(lse_host),
+                                    _s(stream)))
 
 
 def csa_lse_merge(o_part, lse_part, rows, max_splits, D, out, out_dtype, lse_out, stream=None):

@@ -602,7 +602,50 @@ csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* 
                 "score_select_topp launch");
 }
 
-csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// Pinned host memory (page-locked by cudaHostAlloc or cudaHostRegister):
+// the only host memory an asynchronous copy, and a CUDA graph, can take.
+csa_status check_host_ptr(const void* p, const char* name, bool required = true) {
+  if (p == nullptr) {
+    if (!required) return CSA_OK;
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  }
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " is not a valid pointer");
+  }
+  if (a.type != cudaMemoryTypeHost)
+    return fail(CSA_ERR_INVALID_ARG, std::string(name) + " is not pinned host memory");
+  return CSA_OK;
+}
+
+// Device address of pinned host memory (the same address under unified
+// addressing), or NULL when the memory is not mapped or the address is not
+// 16-byte aligned.
+void* mapped_ptr(const void* h) {
+  void* dp = nullptr;
+  if (cudaHostGetDevicePointer(&dp, const_cast<void*>(h), 0) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return reinterpret_cast<uintptr_t>(dp) % 16 == 0 ? dp : nullptr;
+}
+
+// Host side of a step: where the query comes from and where the result goes.
+struct HostIO {
+  const void* q = nullptr;  // the query's source, or NULL (d->q already holds it)
+  bool q_mapped = false;    // q is a device address of pinned host memory: copied by the SMs
+  bool out_mapped = false;  // d->out (and d->lse_out) are device addresses of pinned host memory
+};
+
+// The decode step; with io->q the query is first copied into d->q on the
+// stream, after every check of the decode's own arguments.
+csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stream stream) {
   CSA_REQUIRE(d != nullptr, "descriptor is NULL");
   CSA_REQUIRE(d->mode == CSA_SELECT_TOPK || d->mode == CSA_SELECT_TOPP ||
                   d->mode == CSA_SELECT_HIER || d->mode == CSA_SELECT_TOPK_UNION,
@@ -632,8 +675,10 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
   CSA_REQUIRE(d->workspace_bytes >= static_cast<int64_t>(w.total),
               "workspace smaller than csa_decode_workspace_bytes()");
   CSA_TRY(check_ptr(d->workspace, "workspace"));
-  CSA_TRY(check_ptr(d->out, "out"));
-  CSA_TRY(check_ptr(d->lse_out, "lse_out", false));
+  if (io == nullptr || !io->out_mapped) {
+    CSA_TRY(check_ptr(d->out, "out"));
+    CSA_TRY(check_ptr(d->lse_out, "lse_out", false));
+  }
   const bool hybrid = d->Kg != nullptr || d->Vg != nullptr;
   if (hybrid) {  // both or neither
     CSA_TRY(check_ptr(d->Kg, "Kg"));
@@ -643,6 +688,16 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
   // the selection scores with the pre-RoPE query when one is given
   const void* qs = d->q_score != nullptr ? d->q_score : d->q;
   if (d->q_score != nullptr) CSA_TRY(check_ptr(d->q_score, "q_score"));
+  if (io != nullptr && io->q != nullptr) {
+    const size_t nq = static_cast<size_t>(d->B) * d->Hq * d->D * sizeof(__nv_bfloat16);
+    if (io->q_mapped)
+      CSA_TRY(finish(csa::launch_copy16(l, io->q, const_cast<void*>(d->q), nq),
+                     "query copy to the device"));
+    else
+      CSA_TRY(finish(cudaMemcpyAsync(const_cast<void*>(d->q), io->q, nq, cudaMemcpyHostToDevice,
+                                     l.stream),
+                     "query copy to the device"));
+  }
   // the selection (validates its own arguments before launching)
   csa_status st;
   if (d->mode == CSA_SELECT_TOPK)
@@ -676,6 +731,56 @@ csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
                                      reinterpret_cast<float*>(ws + w.lse), &m, &why);
   if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
   return finish(e, "decode step launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream stream) {
+  return decode_step(d, nullptr, stream);
+}
+
+csa_status csa_decode_step_host(const csa_decode_step_desc* d, const void* q_host, void* out_host,
+                                float* lse_host, csa_stream stream) {
+  CSA_REQUIRE(d != nullptr, "descriptor is NULL");
+  CSA_SUPPORT(d->q_score == nullptr,
+              "q_score (the RoPE-aware split) needs the query rotated on the device: use "
+              "csa_rope and csa_decode_step");
+  CSA_TRY(check_host_ptr(q_host, "q_host"));
+  CSA_TRY(check_host_ptr(out_host, "out_host"));
+  CSA_TRY(check_host_ptr(lse_host, "lse_host", false));
+  CSA_REQUIRE(lse_host == nullptr || d->lse_out != nullptr, "lse_host needs lse_out");
+  CSA_TRY(check_ptr(d->out, "out"));
+  CSA_TRY(check_ptr(d->lse_out, "lse_out", false));
+  // Mapped host memory (every pinned allocation under unified addressing):
+  // the SMs read the query and the decode stores its result straight into
+  // the host buffers, with no copy-engine transfer on either side.
+  HostIO io;
+  void* qd = mapped_ptr(q_host);
+  io.q = qd != nullptr ? qd : q_host;
+  io.q_mapped = qd != nullptr;
+  void* od = mapped_ptr(out_host);
+  void* ld = lse_host != nullptr ? mapped_ptr(lse_host) : nullptr;
+  csa_decode_step_desc dd = *d;
+  if (od != nullptr && (lse_host == nullptr || ld != nullptr)) {
+    io.out_mapped = true;
+    dd.out = od;
+    dd.lse_out = lse_host != nullptr ? static_cast<float*>(ld) : d->lse_out;
+  }
+  CSA_TRY(decode_step(&dd, &io, stream));
+  if (d->B == 0 || io.out_mapped) return CSA_OK;
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  const size_t rows = static_cast<size_t>(d->B) * d->Hq;
+  const size_t no = rows * d->D * (d->out_dtype == CSA_BF16 ? 2 : 4);
+  CSA_TRY(finish(cudaMemcpyAsync(out_host, d->out, no, cudaMemcpyDeviceToHost, l.stream),
+                 "output copy to the host"));
+  if (lse_host != nullptr)
+    CSA_TRY(finish(cudaMemcpyAsync(lse_host, d->lse_out, rows * sizeof(float),
+                                   cudaMemcpyDeviceToHost, l.stream),
+                   "lse copy to the host"));
+  return CSA_OK;
 }
 
 csa_status csa_lse_merge(const float* o_part, const float* lse_part, int rows, int max_splits, int D,

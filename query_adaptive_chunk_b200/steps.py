@@ -199,6 +199,39 @@ class SparseDecoder:
         self.attend(qa, stream)
         return self.out, self.lse
 
+    def step_host(self, q_host: torch.Tensor, out_host: torch.Tensor,
+                  lse_host: torch.Tensor | None = None, stream=None):
+        """One step whose query and result live in pinned host memory
+        (csa_decode_step_host): q_host [B, Hq, D] bf16 is copied into the
+        decoder's own device query buffer, the step runs, and the output
+        (and lse, when lse_host is given) are copied into out_host, all
+        asynchronously on `stream`: synchronise it before reading out_host.
+        Needs the one-call bf16 step without RoPE."""
+        if self.desc is None or self.q_rot is not None:
+            raise ValueError("step_host needs a fused bf16 decoder without RoPE")
+        if getattr(self, "q_dev", None) is None:
+            self.q_dev = torch.empty(self.B, self.Hq, self.D, dtype=torch.bfloat16,
+                                     device=self.out.device)
+        self.desc.q = self.q_dev.data_ptr()
+        self.desc.q_score = None
+        csa.csa_decode_step_host(self.desc, q_host, out_host, lse_host, stream=stream)
+
+    def host_step_graph(self, q_host: torch.Tensor, out_host: torch.Tensor,
+                        lse_host: torch.Tensor | None = None) -> "torch.cuda.CUDAGraph":
+        """``step_host`` on these host buffers captured as a CUDA graph: each
+        ``replay()`` copies the current contents of q_host in, runs the step
+        and copies the result out (synchronise before reading out_host)."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step_host(q_host, out_host, lse_host)  # warm the capture stream
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            self.step_host(q_host, out_host, lse_host)
+        return g
+
 
 class BlockSparsePrefill:
     """Block-sparse causal prefill: per (tile, KV head) the top-k_free chunks by

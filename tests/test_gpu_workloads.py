@@ -217,3 +217,52 @@ def test_rope_aware_separate_calls_match_step():
     dec.attend(dec.q_rot)
     csa.csa_check_device_status()
     assert (dec.out - out_step).abs().max().item() < 1e-5
+
+
+def test_decode_step_host_matches_device_step():
+    """csa_decode_step_host (query and result in pinned host memory) gives
+    the device step's output bit for bit, called directly and replayed as a
+    CUDA graph with a new query written into the same host buffer; the
+    device step itself is pinned to the oracle by run_and_check."""
+    from query_adaptive_chunk_b200 import csa
+    w = synth.TOPP_128K.scaled(B=1, T=16384)
+    dec, inp = run_and_check(w)
+    ref_out, ref_lse = dec.out.clone(), dec.lse.clone()
+    q_host = inp["q"].cpu().pin_memory()
+    out_host = torch.full(dec.out.shape, float("nan"), dtype=dec.out.dtype).pin_memory()
+    lse_host = torch.full(dec.lse.shape, float("nan")).pin_memory()
+    dec.step_host(q_host, out_host, lse_host)
+    torch.cuda.synchronize()
+    csa.csa_check_device_status()
+    assert torch.equal(out_host, ref_out.cpu()) and torch.equal(lse_host, ref_lse.cpu())
+    # a second query through a graph of the same call
+    q2 = (inp["q"].float() * -0.5 + 0.25).to(torch.bfloat16)
+    dec.step(q2)
+    ref2 = dec.out.clone()
+    out_host.fill_(float("nan"))
+    g = dec.host_step_graph(q_host, out_host)
+    q_host.copy_(q2.cpu())
+    out_host.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    csa.csa_check_device_status()
+    assert torch.equal(out_host, ref2.cpu())
+    del g
+
+
+def test_decode_step_host_rejects_pageable_and_rope():
+    from query_adaptive_chunk_b200 import csa
+    w = synth.TOPK_32K.scaled(B=1, T=4096)
+    inp = synth.make_decode_inputs(w, device="cuda")
+    dec = _decoder(w, inp)
+    q_pageable = inp["q"].cpu()
+    out_host = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    with pytest.raises(csa.CsaError, match="pinned host memory"):
+        dec.step_host(q_pageable, out_host)
+    with pytest.raises(csa.CsaError, match="pinned host memory"):
+        dec.step_host(inp["q"].cpu().pin_memory(), torch.empty(dec.out.shape))
+    dec.desc.q_score = inp["q"].data_ptr()
+    with pytest.raises(csa.CsaError, match="CSA_ERR_UNSUPPORTED"):
+        csa.csa_decode_step_host(dec.desc, inp["q"].cpu().pin_memory(), out_host)
+    dec.desc.q_score = None
+    csa.csa_check_device_status()
