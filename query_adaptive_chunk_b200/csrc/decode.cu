@@ -1410,28 +1410,6 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
   return launch_bf16<64, 64>(l, p, K, V, Kg, Vg, B, Hkv, P, why);
 }
 
-namespace {
-
-// 16-byte words from src to dst, one word per thread.  Used to bring a
-// decode query in from mapped pinned host memory: the loads cross the host
-// link from the SMs, with no copy-engine transfer in between.
-__global__ void copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < n) dst[i] = src[i];
-}
-
-}  // namespace
-
-cudaError_t launch_copy16(const Launch& l, const void* src, void* dst, size_t bytes) {
-  const int64_t n = static_cast<int64_t>(bytes / 16);
-  if (n == 0) return cudaSuccess;
-  const int threads = 256;
-  const int64_t blocks = (n + threads - 1) / threads;
-  copy16_kernel<<<static_cast<unsigned>(blocks), threads, 0, l.stream>>>(
-      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_part, int rows,
                          int max_splits, int D, void* out, bool out_bf16, float* lse_out) {
   if (rows == 0) return cudaSuccess;

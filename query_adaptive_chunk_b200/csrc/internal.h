@@ -107,8 +107,9 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
                           float* lse_part, const MergeOut* merge, std::string* why);
 cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_part, int rows,
                          int max_splits, int D, void* out, bool out_bf16, float* lse_out);
-// bytes / 16 words from src to dst (both 16-byte aligned; src may be mapped
-// pinned host memory)
+
+// hostio.cu: bytes / 16 words from src to dst (both 16-byte aligned; src may
+// be mapped pinned host memory)
 cudaError_t launch_copy16(const Launch& l, const void* src, void* dst, size_t bytes);
 
 // prefill.cu
