@@ -7,9 +7,10 @@
 //                of key j is the sum over those rows of its softmax weight
 //                (the rows of the GQA group's heads summed: one importance
 //                per KV head).  Two passes over K on the tensor cores
-//                (mma.m16n8k16, keys as M, query rows as N): per-row max and
-//                sum over key blocks, then, with the rows' final max and sum,
-//                the weights summed per key.  HBM-bound on K (read twice).
+//                (mma.m16n8k16): per-row max and sum over key blocks (rows
+//                as M, keys as N), then, with the rows' final max and sum,
+//                the weights summed per key (keys as M, rows as N).  K is
+//                read twice from HBM.
 //   budget       Dynamic Token Coverage: the fewest tokens whose importance
 //                (summed over the KV heads, normalised) reaches 1 - tau, i.e.
 //                the least important ones are dropped while their mass stays
@@ -28,8 +29,9 @@
 namespace csa {
 namespace {
 
-constexpr int kImpThreads = 128;  // 4 warps
-constexpr int kImpKeys = 128;     // keys per CTA, 32 per warp
+constexpr int kImpThreads = 128;    // pass 2: 4 warps, 32 keys each
+constexpr int kStatsThreads = 256;  // pass 1: 8 warps, 32 observed rows each per turn
+constexpr int kImpKeys = 128;       // keys per CTA
 constexpr float kLog2eF = 1.4426950408889634f;
 
 // Row r of the observed block of KV head h: query head h*G + r / n_obs at
@@ -89,10 +91,10 @@ __device__ __forceinline__ void imp_load_a(const __nv_bfloat16* ks, int kw,
 
 // S^T tile of this warp's 32 keys against query rows [n0 .. n0 + 8):
 // acc[mt][0..3] as the mma C layout (key = lane/4 (+8), row = n0 + 2 (lane%4)
-// (+1)); scaled to the log2 domain.
+// (+1)), unscaled.
 template <int D>
 __device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const uint32_t (&af)[D / 16][2][4],
-                                         int n0, float sl2, float (&acc)[2][4]) {
+                                         int n0, float (&acc)[2][4]) {
   constexpr int LD = D + 8;
   const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
 #pragma unroll
@@ -109,82 +111,147 @@ __device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const uint32_t
       mma_bf16_16816(acc[mt], af[ks16][mt][0], af[ks16][mt][1], af[ks16][mt][2], af[ks16][mt][3],
                      b0, b1);
   }
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[mt][e] *= sl2;
 }
 
 // Pass 1: per (b, h, key block) and observed row, the max and the sum of
 // 2^(s - max) over the block's visible keys -> part [b, h, block, R, 2].
+// Here the observed rows are the mma M dimension and the keys N (the layout
+// of a flash-attention forward pass): a warp holds the A fragments of 32
+// rows, runs over the block's keys 64 at a time, and every lane keeps a
+// running (max, sum) of its rows over its own key columns; the four lanes of
+// a row merge once at the end, so no cross-lane reduction runs per tile.
+// Only blocks that reach past the first observed position need the causal
+// mask; the others take the unmasked path.
 template <int D>
-__global__ void __launch_bounds__(kImpThreads) imp_stats_kernel(
+__global__ void __launch_bounds__(kStatsThreads) imp_stats_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, int S, int Hq,
     int Hkv, int G, int n_obs, float sl2, float* __restrict__ part) {
   extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int LD = D + 8;
-  const int R = G * n_obs;
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);
-  __nv_bfloat16* ks = qs + R * LD;
-  float* red = reinterpret_cast<float*>(ks + kImpKeys * LD);  // [4 warps][R][2]
+  constexpr int LD = D + 8, V8 = D / 8;
+  const int R = G * n_obs, Rp = (R + 31) & ~31;
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);  // [Rp][LD]
+  __nv_bfloat16* ks = qs + Rp * LD;                          // [kImpKeys][LD]
   const int nblk = gridDim.x, blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int j0 = blk * kImpKeys;
+  // rows R .. Rp - 1 of the last row group are zero (their results are dropped)
+  for (int e = threadIdx.x; e < (Rp - R) * V8; e += blockDim.x)
+    *reinterpret_cast<uint4*>(qs + (R + e / V8) * LD + (e % V8) * 8) = make_uint4(0u, 0u, 0u, 0u);
   imp_load<D>(Q, K, b, h, S, Hq, Hkv, G, n_obs, j0, qs, ks);
   __syncthreads();
+  // key j is visible to row r iff j <= S - n_obs + r % n_obs (which also
+  // keeps j < S): every key of the block is visible to every row iff the
+  // block ends at or before the first observed position
+  const bool masked = j0 + kImpKeys - 1 > S - n_obs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kw = warp * 32, rr = lane >> 2, cc = 2 * (lane & 3);
-  uint32_t af[D / 16][2][4];
-  imp_load_a<D>(ks, kw, af);
-  for (int n0 = 0; n0 < R; n0 += 8) {
-    float acc[2][4];
-    imp_tile<D>(qs, af, n0, sl2, acc);
-    // this lane: rows n0 + cc, n0 + cc + 1; keys j0 + kw + {rr, rr+8, rr+16, rr+24}
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = j0 + kw + mt * 16 + rr + (e >> 1) * 8, r = n0 + cc + (e & 1);
-        if (j >= S || j > obs_pos(r, n_obs, S)) acc[mt][e] = -INFINITY;
-        mx[e & 1] = fmaxf(mx[e & 1], acc[mt][e]);
-      }
-#pragma unroll
-    for (int x = 4; x < 32; x <<= 1) {
-      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], x));
-      mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], x));
-    }
-    float sm_[2] = {0.f, 0.f};
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (mx[e & 1] != -INFINITY) sm_[e & 1] += exp2f(acc[mt][e] - mx[e & 1]);
-#pragma unroll
-    for (int x = 4; x < 32; x <<= 1) {
-      sm_[0] += __shfl_xor_sync(0xffffffffu, sm_[0], x);
-      sm_[1] += __shfl_xor_sync(0xffffffffu, sm_[1], x);
-    }
-    if (rr == 0) {
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        red[(warp * R + n0 + cc + t) * 2] = mx[t];
-        red[(warp * R + n0 + cc + t) * 2 + 1] = sm_[t];
-      }
-    }
-  }
-  __syncthreads();
+  const int rr = lane >> 2, cc = 2 * (lane & 3);
   float* out = part + ((static_cast<int64_t>(b) * Hkv + h) * nblk + blk) * R * 2;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    float m = -INFINITY, l = 0.f;
-    for (int w = 0; w < 4; ++w) {
-      const float mw = red[(w * R + r) * 2], lw = red[(w * R + r) * 2 + 1];
-      if (mw == -INFINITY) continue;
-      const float mn = fmaxf(m, mw);
-      l = l * exp2f(m - mn) + lw * exp2f(mw - mn);
-      m = mn;
+  for (int r0 = warp * 32; r0 < R; r0 += (kStatsThreads / 32) * 32) {
+    uint32_t qa[D / 16][2][4];
+#pragma unroll
+    for (int k16 = 0; k16 < D / 16; ++k16)
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const __nv_bfloat16* qr = qs + (r0 + mt * 16 + rr) * LD + k16 * 16 + cc;
+        qa[k16][mt][0] = *reinterpret_cast<const uint32_t*>(qr);
+        qa[k16][mt][1] = *reinterpret_cast<const uint32_t*>(qr + 8 * LD);
+        qa[k16][mt][2] = *reinterpret_cast<const uint32_t*>(qr + 8);
+        qa[k16][mt][3] = *reinterpret_cast<const uint32_t*>(qr + 8 * LD + 8);
+      }
+    int lim[2][2];  // last key visible to this lane's rows [mt][+0 / +8]
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = r0 + mt * 16 + rr + 8 * hh;
+        lim[mt][hh] = r < R ? S - n_obs + r % n_obs : -1;
+      }
+    float m[2][2], l[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        m[mt][hh] = -INFINITY;
+        l[mt][hh] = 0.f;
+      }
+#pragma unroll 1
+    for (int half = 0; half < kImpKeys / 64; ++half) {
+      float acc[8][2][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+#pragma unroll
+      for (int k16 = 0; k16 < D / 16; ++k16)
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const __nv_bfloat16* kr = ks + (half * 64 + nt * 8 + rr) * LD + k16 * 16 + cc;
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 8);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            mma_bf16_16816(acc[nt][mt], qa[k16][mt][0], qa[k16][mt][1], qa[k16][mt][2],
+                           qa[k16][mt][3], b0, b1);
+        }
+      // C layout: acc[nt][mt][e] = row r0 + mt*16 + rr + 8 (e >> 1), key
+      // j0 + half*64 + nt*8 + cc + (e & 1); to the log2 domain, masked
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v = acc[nt][mt][e] * sl2;
+            if (masked && j0 + half * 64 + nt * 8 + cc + (e & 1) > lim[mt][e >> 1]) v = -INFINITY;
+            acc[nt][mt][e] = v;
+          }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+            mx = fmaxf(mx, fmaxf(acc[nt][mt][2 * hh], acc[nt][mt][2 * hh + 1]));
+          const float mn = fmaxf(m[mt][hh], mx);
+          if (mn != -INFINITY) {
+            float sum = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+              sum += fast_exp2(acc[nt][mt][2 * hh] - mn) + fast_exp2(acc[nt][mt][2 * hh + 1] - mn);
+            l[mt][hh] = l[mt][hh] * fast_exp2(m[mt][hh] - mn) + sum;
+            m[mt][hh] = mn;
+          }
+        }
     }
-    out[r * 2] = m;
-    out[r * 2 + 1] = l;
+    // merge the four lanes of each row (lanes 4 rr .. 4 rr + 3)
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int x = 1; x <= 2; x <<= 1) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m[mt][hh], x);
+          const float lo = __shfl_xor_sync(0xffffffffu, l[mt][hh], x);
+          const float mn = fmaxf(m[mt][hh], mo);
+          if (mn != -INFINITY) {
+            l[mt][hh] = l[mt][hh] * fast_exp2(m[mt][hh] - mn) + lo * fast_exp2(mo - mn);
+            m[mt][hh] = mn;
+          }
+        }
+    if ((lane & 3) == 0) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int r = r0 + mt * 16 + rr + 8 * hh;
+          if (r < R) {
+            out[r * 2] = m[mt][hh];
+            out[r * 2 + 1] = l[mt][hh];
+          }
+        }
+    }
   }
 }
 
@@ -234,18 +301,32 @@ __global__ void __launch_bounds__(kImpThreads) imp_weight_kernel(
   float wsum[4] = {0.f, 0.f, 0.f, 0.f};  // keys kw + rr + 8 t
   uint32_t af[D / 16][2][4];
   imp_load_a<D>(ks, kw, af);
+  // as in pass 1: only blocks reaching past the first observed position mask
+  const bool masked = j0 + kImpKeys - 1 > S - n_obs;
+  const float2* st2 = reinterpret_cast<const float2*>(st);
   for (int n0 = 0; n0 < R; n0 += 8) {
     float acc[2][4];
-    imp_tile<D>(qs, af, n0, sl2, acc);
+    imp_tile<D>(qs, af, n0, acc);
+    // (max, 1/sum) of this lane's two rows
+    const float2 s0 = st2[n0 + cc], s1 = st2[n0 + cc + 1];
+    const float nm[2] = {-s0.x, -s1.x}, il[2] = {s0.y, s1.y};
+    if (!masked) {
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = mt * 2 + (e >> 1);
-        const int j = j0 + kw + rr + t * 8, r = n0 + cc + (e & 1);
-        if (j < S && j <= obs_pos(r, n_obs, S))
-          wsum[t] += exp2f(acc[mt][e] - st[r * 2]) * st[r * 2 + 1];
-      }
+        for (int e = 0; e < 4; ++e)
+          wsum[mt * 2 + (e >> 1)] += fast_exp2(fmaf(acc[mt][e], sl2, nm[e & 1])) * il[e & 1];
+    } else {
+      const int lim[2] = {obs_pos(n0 + cc, n_obs, S), obs_pos(n0 + cc + 1, n_obs, S)};
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int t = mt * 2 + (e >> 1);
+          if (j0 + kw + rr + t * 8 <= lim[e & 1])
+            wsum[t] += fast_exp2(fmaf(acc[mt][e], sl2, nm[e & 1])) * il[e & 1];
+        }
+    }
   }
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
@@ -286,12 +367,27 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
   const int b = blockIdx.x, tid = threadIdx.x;
   const float* ib = imp + static_cast<int64_t>(b) * Hkv * S;
   float part = 0.f;
-  for (int j = tid; j < S; j += blockDim.x) {
-    float m = 0.f;
-    for (int h = 0; h < Hkv; ++h) m += ib[static_cast<int64_t>(h) * S + j];
-    m = fmaxf(m, 0.f);
-    ms[j] = m;
-    part += m;
+  // four tokens per thread per turn, so that 4 x Hkv loads are in flight
+  for (int jb = tid; jb < S; jb += 4 * blockDim.x) {
+    float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+    for (int h = 0; h < Hkv; ++h) {
+      const float* row = ib + static_cast<int64_t>(h) * S;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = jb + u * blockDim.x;
+        if (j < S) m[u] += row[j];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = jb + u * blockDim.x;
+      if (j < S) {
+        const float v = fmaxf(m[u], 0.f);
+        ms[j] = v;
+        part += v;
+      }
+    }
   }
 #pragma unroll
   for (int x = 16; x > 0; x >>= 1) part += __shfl_xor_sync(0xffffffffu, part, x);
@@ -313,9 +409,9 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
     }
     __syncthreads();
     const unsigned int prefix = prefix_sh;
-    // Most masses share a few buckets: lanes of a warp with the same bucket
-    // add their count and mass through one leader (one atomic per bucket per
-    // warp, not per element).
+    // Most masses share a few buckets: the lanes of a warp in the bucket of
+    // its first active lane add their count and mass by a warp reduction and
+    // one atomic each; the other lanes add theirs one by one.
     const int lane = tid & 31;
     for (int j0 = 0; j0 < S; j0 += blockDim.x) {
       const int j = j0 + tid;
@@ -328,44 +424,96 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
           m = ms[j];
         }
       }
-      const unsigned int peers = __match_any_sync(0xffffffffu, d);
-      const int leader = __ffs(peers) - 1;
-      float tot = 0.f;
-      for (unsigned int b = peers; b != 0u; b &= b - 1) {  // the group's masses, in lane order
-        const float v = __shfl_sync(peers, m, __ffs(b) - 1);
-        tot += v;
+      const unsigned int act = __ballot_sync(0xffffffffu, d >= 0);
+      if (act == 0u) continue;  // warp-uniform
+      const int d0 = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
+      const unsigned int same = __ballot_sync(0xffffffffu, d == d0);
+      float v = d == d0 ? m : 0.f;
+#pragma unroll
+      for (int x = 16; x > 0; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
+      if (lane == 0) {
+        atomicAdd(&hc[d0], static_cast<unsigned int>(__popc(same)));
+        atomicAdd(&hm[d0], v);
       }
-      if (d >= 0 && lane == leader) {
-        atomicAdd(&hc[d], static_cast<unsigned int>(__popc(peers)));
-        atomicAdd(&hm[d], tot);
+      if (d >= 0 && d != d0) {
+        atomicAdd(&hc[d], 1u);
+        atomicAdd(&hm[d], m);
       }
     }
     __syncthreads();
-    if (tid == 0) {
-      float am = above_m_sh;
-      unsigned int ac = above_c_sh;
+    // The bucket where the running mass from the top first reaches the
+    // target, by warp 0: lane L holds buckets 255 - 8L .. 248 - 8L, a scan
+    // over the lanes gives the mass and count above each lane's buckets.
+    if (tid < 32) {
+      float pm[8];
+      unsigned int pc[8];
+      float lm = 0.f;
+      unsigned int lc = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        pm[i] = hm[255 - 8 * lane - i];
+        pc[i] = hc[255 - 8 * lane - i];
+        lm += pm[i];
+        lc += pc[i];
+      }
+      float sm_ = lm;
+      unsigned int sc = lc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, sm_, o);
+        const unsigned int tc = __shfl_up_sync(0xffffffffu, sc, o);
+        if (lane >= o) {
+          sm_ += t;
+          sc += tc;
+        }
+      }
+      float em = __shfl_up_sync(0xffffffffu, sm_, 1);
+      unsigned int ec = __shfl_up_sync(0xffffffffu, sc, 1);
+      if (lane == 0) {
+        em = 0.f;
+        ec = 0u;
+      }
+      float am = above_m_sh + em;
+      unsigned int ac = above_c_sh + ec;
       int sel = -1, low = -1;
-      for (int d = 255; d >= 0; --d) {
-        if (hc[d] == 0u) continue;
-        if (am + hm[d] >= target) {
-          sel = d;
-          break;
+      float am_sel = 0.f, am_low = 0.f;
+      unsigned int ac_sel = 0u, ac_low = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (sel < 0 && pc[i] != 0u) {
+          if (am + pm[i] >= target) {
+            sel = 255 - 8 * lane - i;
+            am_sel = am;
+            ac_sel = ac;
+          } else {
+            am_low = am;  // the mass above this bucket, were it the cut
+            ac_low = ac;
+            am += pm[i];
+            ac += pc[i];
+            low = 255 - 8 * lane - i;
+          }
         }
-        am += hm[d];
-        ac += hc[d];
-        low = d;
       }
-      if (sel < 0) {  // the sums fell short of the target by rounding: cut in the lowest bucket
+      const unsigned int hit = __ballot_sync(0xffffffffu, sel >= 0);
+      int src;
+      if (hit != 0u) {
+        src = __ffs(hit) - 1;  // the first crossing from the top
+      } else {  // the sums fell short of the target by rounding: cut in the lowest bucket
+        const unsigned int nz = __ballot_sync(0xffffffffu, low >= 0);
+        src = nz != 0u ? 31 - __clz(nz) : 0;
         sel = low < 0 ? 0 : low;
-        if (low >= 0) {
-          am -= hm[low];
-          ac -= hc[low];
-        }
+        am_sel = low < 0 ? am : am_low;
+        ac_sel = low < 0 ? ac : ac_low;
       }
-      above_m_sh = am;
-      above_c_sh = ac;
-      sel_sh = static_cast<unsigned int>(sel);
-      prefix_sh = prefix | (static_cast<unsigned int>(sel) << shift);
+      sel = __shfl_sync(0xffffffffu, sel, src);
+      am_sel = __shfl_sync(0xffffffffu, am_sel, src);
+      ac_sel = __shfl_sync(0xffffffffu, ac_sel, src);
+      if (lane == 0) {
+        above_m_sh = am_sel;
+        above_c_sh = ac_sel;
+        sel_sh = static_cast<unsigned int>(sel);
+        prefix_sh = prefix | (static_cast<unsigned int>(sel) << shift);
+      }
     }
     __syncthreads();
     mask |= 255u << shift;
@@ -543,7 +691,7 @@ cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* 
   float* part = scratch;
   float* stats = scratch + static_cast<size_t>(B) * Hkv * nblk * R * 2;
   const size_t lds = static_cast<size_t>(D + 8) * 2;
-  const size_t sh1 = (R + kImpKeys) * lds + 4 * static_cast<size_t>(R) * 2 * 4;
+  const size_t sh1 = ((R + 31) / 32 * 32 + kImpKeys) * lds;
   const size_t sh2 = (R + kImpKeys) * lds + static_cast<size_t>(R) * 2 * 4;
   const dim3 grid(nblk, Hkv, B);
   const float sl2 = scale * kLog2eF;
@@ -554,7 +702,7 @@ cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* 
     e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<128>), sh1);
     if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<128>), sh2);
     if (e != cudaSuccess) return e;
-    imp_stats_kernel<128><<<grid, kImpThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
+    imp_stats_kernel<128><<<grid, kStatsThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
     imp_combine_kernel<<<B * Hkv, 256, 0, l.stream>>>(part, nblk, R, stats);
     imp_weight_kernel<128><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
                                                                  stats, imp);
@@ -562,7 +710,7 @@ cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* 
     e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<64>), sh1);
     if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<64>), sh2);
     if (e != cudaSuccess) return e;
-    imp_stats_kernel<64><<<grid, kImpThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
+    imp_stats_kernel<64><<<grid, kStatsThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
     imp_combine_kernel<<<B * Hkv, 256, 0, l.stream>>>(part, nblk, R, stats);
     imp_weight_kernel<64><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
                                                                 stats, imp);
