@@ -255,18 +255,40 @@ __global__ void __launch_bounds__(kStatsThreads) imp_stats_kernel(
   }
 }
 
-// The rows' max and sum over all key blocks: part -> stats [b, h, R, 2]
-// (one CTA per (b, h)).
-__global__ void imp_combine_kernel(const float* __restrict__ part, int nblk, int R,
-                                   float* __restrict__ stats) {
+// The rows' max and sum over all key blocks: part -> stats [b, h, R, 2].
+// CTA (b*Hkv + h, y) takes rows 32 y .. 32 y + 31; its 8 warps split the key
+// blocks (warp w: blocks w, w + 8, ...), lane = row, so the partials of a
+// turn are one coalesced 256-byte load per warp; the warps' results merge in
+// shared memory.
+constexpr int kCombineWarps = 8;
+__global__ void __launch_bounds__(kCombineWarps * 32) imp_combine_kernel(
+    const float* __restrict__ part, int nblk, int R, float* __restrict__ stats) {
+  __shared__ float2 red[kCombineWarps][32];
   const int64_t bh = blockIdx.x;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    float m = -INFINITY, l = 0.f;
-    for (int k = 0; k < nblk; ++k) {
-      const float mw = part[((bh * nblk + k) * R + r) * 2], lw = part[((bh * nblk + k) * R + r) * 2 + 1];
-      if (mw == -INFINITY) continue;
-      const float mn = fmaxf(m, mw);
-      l = l * exp2f(m - mn) + lw * exp2f(mw - mn);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int r = blockIdx.y * 32 + lane;
+  float m = -INFINITY, l = 0.f;
+  if (r < R) {
+    const float2* p2 = reinterpret_cast<const float2*>(part) + bh * nblk * R + r;
+#pragma unroll 4
+    for (int k = w; k < nblk; k += kCombineWarps) {
+      const float2 v = p2[static_cast<int64_t>(k) * R];
+      if (v.x == -INFINITY) continue;
+      const float mn = fmaxf(m, v.x);
+      l = l * exp2f(m - mn) + v.y * exp2f(v.x - mn);
+      m = mn;
+    }
+  }
+  red[w][lane] = make_float2(m, l);
+  __syncthreads();
+  if (w == 0 && r < R) {
+    m = -INFINITY;
+    l = 0.f;
+    for (int x = 0; x < kCombineWarps; ++x) {
+      const float2 v = red[x][lane];
+      if (v.x == -INFINITY) continue;
+      const float mn = fmaxf(m, v.x);
+      l = l * exp2f(m - mn) + v.y * exp2f(v.x - mn);
       m = mn;
     }
     stats[(bh * R + r) * 2] = m;
@@ -367,8 +389,25 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
   const int b = blockIdx.x, tid = threadIdx.x;
   const float* ib = imp + static_cast<int64_t>(b) * Hkv * S;
   float part = 0.f;
-  // four tokens per thread per turn, so that 4 x Hkv loads are in flight
-  for (int jb = tid; jb < S; jb += 4 * blockDim.x) {
+  // One SM reads all B*Hkv*S importances of the sequence: keep many bytes in
+  // flight per thread.  16-byte loads of four tokens, all heads at once,
+  // when the rows allow it; else four tokens per thread per turn.
+  const bool vec = S % 4 == 0 && (reinterpret_cast<uintptr_t>(ib) & 15u) == 0;
+  for (int j4 = tid; vec && j4 < S / 4; j4 += blockDim.x) {
+    float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int h = 0; h < Hkv; ++h) {
+      const float4 v = reinterpret_cast<const float4*>(ib + static_cast<int64_t>(h) * S)[j4];
+      m4.x += v.x;
+      m4.y += v.y;
+      m4.z += v.z;
+      m4.w += v.w;
+    }
+    m4 = make_float4(fmaxf(m4.x, 0.f), fmaxf(m4.y, 0.f), fmaxf(m4.z, 0.f), fmaxf(m4.w, 0.f));
+    reinterpret_cast<float4*>(ms)[j4] = m4;
+    part += (m4.x + m4.y) + (m4.z + m4.w);
+  }
+  for (int jb = tid; !vec && jb < S; jb += 4 * blockDim.x) {
     float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 2
     for (int h = 0; h < Hkv; ++h) {
@@ -409,9 +448,10 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
     }
     __syncthreads();
     const unsigned int prefix = prefix_sh;
-    // Most masses share a few buckets: the lanes of a warp in the bucket of
-    // its first active lane add their count and mass by a warp reduction and
-    // one atomic each; the other lanes add theirs one by one.
+    // Most masses share a few buckets: up to three times, the lanes of a
+    // warp in the bucket of its first remaining lane add their count and
+    // mass by a warp reduction and one atomic each; lanes left after that
+    // (buckets spread wide) add theirs one by one.
     const int lane = tid & 31;
     for (int j0 = 0; j0 < S; j0 += blockDim.x) {
       const int j = j0 + tid;
@@ -424,18 +464,22 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
           m = ms[j];
         }
       }
-      const unsigned int act = __ballot_sync(0xffffffffu, d >= 0);
-      if (act == 0u) continue;  // warp-uniform
-      const int d0 = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
-      const unsigned int same = __ballot_sync(0xffffffffu, d == d0);
-      float v = d == d0 ? m : 0.f;
 #pragma unroll
-      for (int x = 16; x > 0; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
-      if (lane == 0) {
-        atomicAdd(&hc[d0], static_cast<unsigned int>(__popc(same)));
-        atomicAdd(&hm[d0], v);
+      for (int round = 0; round < 3; ++round) {
+        const unsigned int act = __ballot_sync(0xffffffffu, d >= 0);
+        if (act == 0u) break;  // warp-uniform
+        const int d0 = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
+        const unsigned int same = __ballot_sync(0xffffffffu, d == d0);
+        float v = d == d0 ? m : 0.f;
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
+        if (lane == 0) {
+          atomicAdd(&hc[d0], static_cast<unsigned int>(__popc(same)));
+          atomicAdd(&hm[d0], v);
+        }
+        if (d == d0) d = -1;  // counted
       }
-      if (d >= 0 && d != d0) {
+      if (d >= 0) {
         atomicAdd(&hc[d], 1u);
         atomicAdd(&hm[d], m);
       }
@@ -555,26 +599,33 @@ __global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
                                   int kmax, int S, int Sc, int Hq, int Hkv, int D,
                                   __nv_bfloat16* __restrict__ Qc, __nv_bfloat16* __restrict__ Kc,
                                   __nv_bfloat16* __restrict__ Vc) {
+  // one warp per compressed row t of unit u = b * Hkv + h: its (G + 2) * D / 8
+  // pieces (G query rows, then K, then V) spread over the lanes
   const int G = Hq / Hkv, V8 = D / 8;
-  const int per_row = (G + 2) * V8;  // 16-byte pieces of one compressed row of (b, h)
-  const int64_t u = blockIdx.y;      // b * Hkv + h
+  const int per_row = (G + 2) * V8;
+  const int64_t u = blockIdx.y;
   const int b = static_cast<int>(u / Hkv), h = static_cast<int>(u % Hkv);
   const int n = count[u];
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-       e < static_cast<int64_t>(Sc) * per_row; e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(e / per_row), w = static_cast<int>(e % per_row);
-    const int part = w / V8, c = (w % V8) * 8;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < Sc; t += gridDim.x * wpb) {
     const int p = t < n ? idx[u * kmax + t] : -1;
-    int4 v = make_int4(0, 0, 0, 0);
-    if (part < G) {  // query head h*G + part
-      if (p >= 0)
-        v = *reinterpret_cast<const int4*>(Q + ((static_cast<int64_t>(b) * S + p) * Hq + h * G + part) * D + c);
-      *reinterpret_cast<int4*>(Qc + ((static_cast<int64_t>(b) * Sc + t) * Hq + h * G + part) * D + c) = v;
-    } else {
-      const __nv_bfloat16* src = part == G ? K : V;
-      __nv_bfloat16* dst = part == G ? Kc : Vc;
-      if (p >= 0) v = *reinterpret_cast<const int4*>(src + (u * S + p) * D + c);
-      *reinterpret_cast<int4*>(dst + (u * Sc + t) * D + c) = v;
+#pragma unroll 3
+    for (int w = lane; w < per_row; w += 32) {
+      const int part = w / V8, c = (w % V8) * 8;
+      int4 v = make_int4(0, 0, 0, 0);
+      if (part < G) {  // query head h*G + part
+        if (p >= 0)
+          v = *reinterpret_cast<const int4*>(
+              Q + ((static_cast<int64_t>(b) * S + p) * Hq + h * G + part) * D + c);
+        *reinterpret_cast<int4*>(Qc + ((static_cast<int64_t>(b) * Sc + t) * Hq + h * G + part) * D +
+                                 c) = v;
+      } else {
+        const __nv_bfloat16* src = part == G ? K : V;
+        __nv_bfloat16* dst = part == G ? Kc : Vc;
+        if (p >= 0) v = *reinterpret_cast<const int4*>(src + (u * S + p) * D + c);
+        *reinterpret_cast<int4*>(dst + (u * Sc + t) * D + c) = v;
+      }
     }
   }
 }
@@ -610,20 +661,23 @@ __global__ void tsa_inverse_kernel(const int32_t* __restrict__ idx,
 __global__ void tsa_scatter_kernel(const __nv_bfloat16* __restrict__ Oc,
                                    const int32_t* __restrict__ inv, int S, int Sc, int Hq, int Hkv,
                                    int D, int B, __nv_bfloat16* __restrict__ O) {
-  const int G = Hq / Hkv, V8 = D / 8;
-  const int64_t total = static_cast<int64_t>(B) * S * Hq * V8;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(e % V8) * 8;
-    const int64_t row = e / V8;  // (b * S + s) * Hq + hq
-    const int hq = static_cast<int>(row % Hq);
-    const int64_t bs = row / Hq;
-    const int s = static_cast<int>(bs % S), b = static_cast<int>(bs / S);
-    const int t = inv[(static_cast<int64_t>(b) * Hkv + hq / G) * S + s];
-    int4 v = make_int4(0, 0, 0, 0);
-    if (t >= 0)
-      v = *reinterpret_cast<const int4*>(Oc + ((static_cast<int64_t>(b) * Sc + t) * Hq + hq) * D + c);
-    *reinterpret_cast<int4*>(O + row * D + c) = v;
+  // one warp per output position (b, s): its Hq * D / 8 pieces over the lanes
+  const int G = Hq / Hkv, V8 = D / 8, per_row = Hq * V8;
+  const int lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  for (int64_t bs = blockIdx.x * wpb + (threadIdx.x >> 5); bs < static_cast<int64_t>(B) * S;
+       bs += gridDim.x * wpb) {
+    const int b = static_cast<int>(bs / S), s = static_cast<int>(bs % S);
+    const int32_t* invb = inv + static_cast<int64_t>(b) * Hkv * S + s;
+#pragma unroll 4
+    for (int q = lane; q < per_row; q += 32) {
+      const int hq = q / V8, c = (q % V8) * 8;
+      const int t = invb[static_cast<int64_t>(hq / G) * S];
+      int4 v = make_int4(0, 0, 0, 0);
+      if (t >= 0)
+        v = *reinterpret_cast<const int4*>(Oc + ((static_cast<int64_t>(b) * Sc + t) * Hq + hq) * D + c);
+      *reinterpret_cast<int4*>(O + (bs * Hq + hq) * D + c) = v;
+    }
   }
 }
 
@@ -649,7 +703,7 @@ cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, con
                               const int32_t* idx, const int32_t* count, int kmax, int B, int S,
                               int Sc, int Hq, int Hkv, int D, void* Qc, void* Kc, void* Vc) {
   if (B == 0 || Sc == 0) return cudaSuccess;
-  const dim3 grid(4 * l.num_sms / (B * Hkv) + 1, B * Hkv);
+  const dim3 grid(8 * l.num_sms / (B * Hkv) + 1, B * Hkv);
   tsa_gather_kernel<<<grid, 256, 0, l.stream>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
       static_cast<const __nv_bfloat16*>(V), idx, count, kmax, S, Sc, Hq, Hkv, D,
@@ -703,7 +757,8 @@ cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* 
     if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<128>), sh2);
     if (e != cudaSuccess) return e;
     imp_stats_kernel<128><<<grid, kStatsThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
-    imp_combine_kernel<<<B * Hkv, 256, 0, l.stream>>>(part, nblk, R, stats);
+    imp_combine_kernel<<<dim3(B * Hkv, (R + 31) / 32), kCombineWarps * 32, 0, l.stream>>>(
+        part, nblk, R, stats);
     imp_weight_kernel<128><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
                                                                  stats, imp);
   } else {
@@ -711,7 +766,8 @@ cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* 
     if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<64>), sh2);
     if (e != cudaSuccess) return e;
     imp_stats_kernel<64><<<grid, kStatsThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
-    imp_combine_kernel<<<B * Hkv, 256, 0, l.stream>>>(part, nblk, R, stats);
+    imp_combine_kernel<<<dim3(B * Hkv, (R + 31) / 32), kCombineWarps * 32, 0, l.stream>>>(
+        part, nblk, R, stats);
     imp_weight_kernel<64><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
                                                                 stats, imp);
   }
