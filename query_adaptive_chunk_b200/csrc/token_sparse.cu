@@ -45,14 +45,20 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, boo
                : "memory");
 }
 
-// Loads the observed query rows of (b, h) [R][D] and the key block [128][D]
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Asynchronous 16-byte copies of the observed query rows of (b, h) [R][D]
 // into padded shared memory (row stride D + 8 bf16: conflict-free fragment
-// loads) with asynchronous 16-byte copies, all in flight at once; waits for
-// them (the caller's barrier then publishes them).
+// loads); the caller commits and waits.
 template <int D>
-__device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, int h, int S,
-                         int Hq, int Hkv, int G, int n_obs, int j0, __nv_bfloat16* qs,
-                         __nv_bfloat16* ks) {
+__device__ __forceinline__ void imp_load_q(const __nv_bfloat16* Q, int b, int h, int S, int Hq,
+                                           int G, int n_obs, __nv_bfloat16* qs) {
   constexpr int LD = D + 8, V8 = D / 8;
   const int R = G * n_obs;
   for (int e = threadIdx.x; e < R * V8; e += blockDim.x) {
@@ -61,13 +67,32 @@ __device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, 
     cp_async16(qs + r * LD + c, Q + ((static_cast<int64_t>(b) * S + pos) * Hq + h * G + g) * D + c,
                true);
   }
+}
+
+// The same for the key block [kImpKeys][D] starting at key j0 (keys past S
+// are zero-filled).
+template <int D>
+__device__ __forceinline__ void imp_load_k(const __nv_bfloat16* K, int b, int h, int S, int Hkv,
+                                           int j0, __nv_bfloat16* ks) {
+  constexpr int LD = D + 8, V8 = D / 8;
   const __nv_bfloat16* kb = K + ((static_cast<int64_t>(b) * Hkv + h) * S) * D;
   for (int e = threadIdx.x; e < kImpKeys * V8; e += blockDim.x) {
     const int r = e / V8, c = (e % V8) * 8;
     const int j = j0 + r;
     cp_async16(ks + r * LD + c, kb + static_cast<int64_t>(j < S ? j : 0) * D + c, j < S);
   }
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+// Both, all in flight at once, then waits for them (the caller's barrier
+// then publishes them).
+template <int D>
+__device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, int h, int S,
+                         int Hq, int Hkv, int G, int n_obs, int j0, __nv_bfloat16* qs,
+                         __nv_bfloat16* ks) {
+  imp_load_q<D>(Q, b, h, S, Hq, G, n_obs, qs);
+  imp_load_k<D>(K, b, h, S, Hkv, j0, ks);
+  cp_async_commit();
+  cp_async_wait<0>();
 }
 
 // This warp's 32 keys (two 16-key m-tiles) as mma A fragments for every
@@ -96,135 +121,182 @@ template <int D>
 __device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const uint32_t (&af)[D / 16][2][4],
                                          int n0, float (&acc)[2][4]) {
   constexpr int LD = D + 8;
-  const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+  // B fragments of two 16-wide slices per ldmatrix: lanes 0-7 / 8-15 /
+  // 16-23 / 24-31 address rows n0 .. n0 + 7 at columns +0 / +8 / +16 / +24
+  const uint32_t qb_base =
+      smem_u32(qs + (n0 + (lane & 7)) * LD + (lane >> 4) * 16 + ((lane >> 3) & 1) * 8);
 #pragma unroll
-  for (int ks16 = 0; ks16 < D / 16; ++ks16) {
-    const __nv_bfloat16* qr = qs + (n0 + rr) * LD + ks16 * 16 + cc;
-    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qr);
-    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qr + 8);
+  for (int kp = 0; kp < D / 32; ++kp) {
+    uint32_t b[4];
+    ldsm_x4(qb_base + kp * 32 * 2, b[0], b[1], b[2], b[3]);
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-      mma_bf16_16816(acc[mt], af[ks16][mt][0], af[ks16][mt][1], af[ks16][mt][2], af[ks16][mt][3],
-                     b0, b1);
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+        mma_bf16_16816(acc[mt], af[2 * kp + t][mt][0], af[2 * kp + t][mt][1],
+                       af[2 * kp + t][mt][2], af[2 * kp + t][mt][3], b[2 * t], b[2 * t + 1]);
   }
 }
 
-// Pass 1: per (b, h, key block) and observed row, the max and the sum of
-// 2^(s - max) over the block's visible keys -> part [b, h, block, R, 2].
-// Here the observed rows are the mma M dimension and the keys N (the layout
-// of a flash-attention forward pass): a warp holds the A fragments of 32
-// rows, runs over the block's keys 64 at a time, and every lane keeps a
-// running (max, sum) of its rows over its own key columns; the four lanes of
-// a row merge once at the end, so no cross-lane reduction runs per tile.
-// Only blocks that reach past the first observed position need the causal
-// mask; the others take the unmasked path.
+// One warp's 32 observed rows r0 .. r0 + 31 against the key block at j0 in
+// `ks`: the rows are the mma M dimension and the keys N (the layout of a
+// flash-attention forward pass); the warp runs over the block's keys 64 at a
+// time and every lane folds its scores into the running (max, sum) of its
+// four rows over its own key columns, m/l [m-tile][row +0 / +8].  Only
+// blocks that reach past the first observed position need the causal mask.
 template <int D>
-__global__ void __launch_bounds__(kStatsThreads) imp_stats_kernel(
-    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, int S, int Hq,
-    int Hkv, int G, int n_obs, float sl2, float* __restrict__ part) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int LD = D + 8, V8 = D / 8;
-  const int R = G * n_obs, Rp = (R + 31) & ~31;
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);  // [Rp][LD]
-  __nv_bfloat16* ks = qs + Rp * LD;                          // [kImpKeys][LD]
-  const int nblk = gridDim.x, blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int j0 = blk * kImpKeys;
-  // rows R .. Rp - 1 of the last row group are zero (their results are dropped)
-  for (int e = threadIdx.x; e < (Rp - R) * V8; e += blockDim.x)
-    *reinterpret_cast<uint4*>(qs + (R + e / V8) * LD + (e % V8) * 8) = make_uint4(0u, 0u, 0u, 0u);
-  imp_load<D>(Q, K, b, h, S, Hq, Hkv, G, n_obs, j0, qs, ks);
-  __syncthreads();
+__device__ __forceinline__ void imp_stats_rows(const __nv_bfloat16* qs, const __nv_bfloat16* ks,
+                                               int r0, int R, int S, int n_obs, int j0,
+                                               bool masked, float sl2, float (&m)[2][2],
+                                               float (&l)[2][2]) {
+  constexpr int LD = D + 8;
+  const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
+  // A fragments by ldmatrix: lanes 0-7 / 8-15 / 16-23 / 24-31 address the
+  // rows of the (rows +0, cols +0) / (+8, +0) / (+0, +8) / (+8, +8) 8x8 blocks
+  uint32_t qa[D / 16][2][4];
+  const uint32_t qa_base =
+      smem_u32(qs + (r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * LD + (lane >> 4) * 8);
+#pragma unroll
+  for (int k16 = 0; k16 < D / 16; ++k16)
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+      ldsm_x4(qa_base + (mt * 16 * LD + k16 * 16) * 2, qa[k16][mt][0], qa[k16][mt][1],
+              qa[k16][mt][2], qa[k16][mt][3]);
   // key j is visible to row r iff j <= S - n_obs + r % n_obs (which also
-  // keeps j < S): every key of the block is visible to every row iff the
-  // block ends at or before the first observed position
-  const bool masked = j0 + kImpKeys - 1 > S - n_obs;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rr = lane >> 2, cc = 2 * (lane & 3);
-  float* out = part + ((static_cast<int64_t>(b) * Hkv + h) * nblk + blk) * R * 2;
-  for (int r0 = warp * 32; r0 < R; r0 += (kStatsThreads / 32) * 32) {
-    uint32_t qa[D / 16][2][4];
+  // keeps j < S); rows past R (zero padding) see nothing
+  int lim[2][2];
 #pragma unroll
-    for (int k16 = 0; k16 < D / 16; ++k16)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const __nv_bfloat16* qr = qs + (r0 + mt * 16 + rr) * LD + k16 * 16 + cc;
-        qa[k16][mt][0] = *reinterpret_cast<const uint32_t*>(qr);
-        qa[k16][mt][1] = *reinterpret_cast<const uint32_t*>(qr + 8 * LD);
-        qa[k16][mt][2] = *reinterpret_cast<const uint32_t*>(qr + 8);
-        qa[k16][mt][3] = *reinterpret_cast<const uint32_t*>(qr + 8 * LD + 8);
-      }
-    int lim[2][2];  // last key visible to this lane's rows [mt][+0 / +8]
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int r = r0 + mt * 16 + rr + 8 * hh;
-        lim[mt][hh] = r < R ? S - n_obs + r % n_obs : -1;
-      }
-    float m[2][2], l[2][2];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        m[mt][hh] = -INFINITY;
-        l[mt][hh] = 0.f;
-      }
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = r0 + mt * 16 + rr + 8 * hh;
+      lim[mt][hh] = r < R ? S - n_obs + r % n_obs : -1;
+    }
 #pragma unroll 1
-    for (int half = 0; half < kImpKeys / 64; ++half) {
-      float acc[8][2][4];
+  for (int half = 0; half < kImpKeys / 64; ++half) {
+    float acc[8][2][4];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
-#pragma unroll
-      for (int k16 = 0; k16 < D / 16; ++k16)
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const __nv_bfloat16* kr = ks + (half * 64 + nt * 8 + rr) * LD + k16 * 16 + cc;
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 8);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-            mma_bf16_16816(acc[nt][mt], qa[k16][mt][0], qa[k16][mt][1], qa[k16][mt][2],
-                           qa[k16][mt][3], b0, b1);
-        }
-      // C layout: acc[nt][mt][e] = row r0 + mt*16 + rr + 8 (e >> 1), key
-      // j0 + half*64 + nt*8 + cc + (e & 1); to the log2 domain, masked
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float v = acc[nt][mt][e] * sl2;
-            if (masked && j0 + half * 64 + nt * 8 + cc + (e & 1) > lim[mt][e >> 1]) v = -INFINITY;
-            acc[nt][mt][e] = v;
-          }
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float mx = -INFINITY;
+        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+    // B fragments of two n-tiles per ldmatrix: lanes 0-7 / 8-15 / 16-23 /
+    // 24-31 address the keys of (n-tile +0, cols +0) / (+0, +8) / (+1, +0) /
+    // (+1, +8)
+    const uint32_t kb_base = smem_u32(ks + (half * 64 + (lane >> 4) * 8 + (lane & 7)) * LD +
+                                      ((lane >> 3) & 1) * 8);
+#pragma unroll
+    for (int k16 = 0; k16 < D / 16; ++k16)
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t b[4];
+        ldsm_x4(kb_base + (np * 16 * LD + k16 * 16) * 2, b[0], b[1], b[2], b[3]);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+            mma_bf16_16816(acc[2 * np + t][mt], qa[k16][mt][0], qa[k16][mt][1], qa[k16][mt][2],
+                           qa[k16][mt][3], b[2 * t], b[2 * t + 1]);
+      }
+    // C layout: acc[nt][mt][e] = row r0 + mt*16 + rr + 8 (e >> 1), key
+    // j0 + half*64 + nt*8 + cc + (e & 1); to the log2 domain, masked
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v = acc[nt][mt][e] * sl2;
+          if (masked && j0 + half * 64 + nt * 8 + cc + (e & 1) > lim[mt][e >> 1]) v = -INFINITY;
+          acc[nt][mt][e] = v;
+        }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+          mx = fmaxf(mx, fmaxf(acc[nt][mt][2 * hh], acc[nt][mt][2 * hh + 1]));
+        const float mn = fmaxf(m[mt][hh], mx);
+        if (mn != -INFINITY) {
+          float sum = 0.f;
 #pragma unroll
           for (int nt = 0; nt < 8; ++nt)
-            mx = fmaxf(mx, fmaxf(acc[nt][mt][2 * hh], acc[nt][mt][2 * hh + 1]));
-          const float mn = fmaxf(m[mt][hh], mx);
-          if (mn != -INFINITY) {
-            float sum = 0.f;
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-              sum += fast_exp2(acc[nt][mt][2 * hh] - mn) + fast_exp2(acc[nt][mt][2 * hh + 1] - mn);
-            l[mt][hh] = l[mt][hh] * fast_exp2(m[mt][hh] - mn) + sum;
-            m[mt][hh] = mn;
-          }
+            sum += fast_exp2(acc[nt][mt][2 * hh] - mn) + fast_exp2(acc[nt][mt][2 * hh + 1] - mn);
+          l[mt][hh] = l[mt][hh] * fast_exp2(m[mt][hh] - mn) + sum;
+          m[mt][hh] = mn;
         }
+      }
+  }
+}
+
+// Pass 1: per (b, h) and observed row, the max and the sum of 2^(s - max)
+// over the visible keys of the key blocks this CTA takes -> part [b, h,
+// split, R, 2].  Persistent over the key blocks: CTA (split, h, b) takes
+// blocks split, split + nsplit, ...; the observed rows are loaded once and
+// the key tiles double-buffered, so the next tile's copy runs under this
+// tile's math.  Warp w takes the 32-row groups w, w + 8 (R <= 512) and keeps
+// their per-lane running statistics across all the CTA's blocks; the four
+// lanes of a row merge once at the end.
+template <int D>
+__global__ void __launch_bounds__(kStatsThreads) imp_stats_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, int S, int Hq,
+    int Hkv, int G, int n_obs, float sl2, int nblk, float* __restrict__ part) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  constexpr int LD = D + 8, V8 = D / 8;
+  constexpr int kRowsPerTurn = (kStatsThreads / 32) * 32;
+  const int R = G * n_obs, Rp = (R + 31) & ~31;
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);  // [Rp][LD]
+  __nv_bfloat16* ksb = qs + Rp * LD;                         // [2][kImpKeys][LD]
+  const int nsplit = gridDim.x, split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // rows R .. Rp - 1 of the last row group are zero (their results are dropped)
+  for (int e = threadIdx.x; e < (Rp - R) * V8; e += blockDim.x)
+    *reinterpret_cast<uint4*>(qs + (R + e / V8) * LD + (e % V8) * 8) = make_uint4(0u, 0u, 0u, 0u);
+  imp_load_q<D>(Q, b, h, S, Hq, G, n_obs, qs);
+  if (split < nblk) imp_load_k<D>(K, b, h, S, Hkv, split * kImpKeys, ksb);
+  cp_async_commit();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float m[2][2][2], l[2][2][2];  // [row group of this warp][m-tile][row +0 / +8]
+#pragma unroll
+  for (int g2 = 0; g2 < 2; ++g2)
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        m[g2][mt][hh] = -INFINITY;
+        l[g2][mt][hh] = 0.f;
+      }
+  int it = 0;
+  for (int blk = split; blk < nblk; blk += nsplit, ++it) {
+    const int nxt = blk + nsplit;
+    if (nxt < nblk) imp_load_k<D>(K, b, h, S, Hkv, nxt * kImpKeys, ksb + ((it + 1) & 1) * kImpKeys * LD);
+    cp_async_commit();
+    cp_async_wait<1>();  // all but the tile just issued
+    __syncthreads();
+    const __nv_bfloat16* ks = ksb + (it & 1) * kImpKeys * LD;
+    const int j0 = blk * kImpKeys;
+    const bool masked = j0 + kImpKeys - 1 > S - n_obs;
+#pragma unroll
+    for (int g2 = 0; g2 < 2; ++g2) {
+      const int r0 = warp * 32 + g2 * kRowsPerTurn;
+      if (r0 < R) imp_stats_rows<D>(qs, ks, r0, R, S, n_obs, j0, masked, sl2, m[g2], l[g2]);
     }
+    __syncthreads();  // this buffer takes the copy issued next turn
+  }
+  cp_async_wait<0>();
+  const int rr = lane >> 2;
+  float* out = part + ((static_cast<int64_t>(b) * Hkv + h) * nsplit + split) * R * 2;
+#pragma unroll
+  for (int g2 = 0; g2 < 2; ++g2) {
+    const int r0 = warp * 32 + g2 * kRowsPerTurn;
+    if (r0 >= R) continue;  // warp-uniform
     // merge the four lanes of each row (lanes 4 rr .. 4 rr + 3)
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
@@ -232,12 +304,12 @@ __global__ void __launch_bounds__(kStatsThreads) imp_stats_kernel(
       for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
         for (int x = 1; x <= 2; x <<= 1) {
-          const float mo = __shfl_xor_sync(0xffffffffu, m[mt][hh], x);
-          const float lo = __shfl_xor_sync(0xffffffffu, l[mt][hh], x);
-          const float mn = fmaxf(m[mt][hh], mo);
+          const float mo = __shfl_xor_sync(0xffffffffu, m[g2][mt][hh], x);
+          const float lo = __shfl_xor_sync(0xffffffffu, l[g2][mt][hh], x);
+          const float mn = fmaxf(m[g2][mt][hh], mo);
           if (mn != -INFINITY) {
-            l[mt][hh] = l[mt][hh] * fast_exp2(m[mt][hh] - mn) + lo * fast_exp2(mo - mn);
-            m[mt][hh] = mn;
+            l[g2][mt][hh] = l[g2][mt][hh] * fast_exp2(m[g2][mt][hh] - mn) + lo * fast_exp2(mo - mn);
+            m[g2][mt][hh] = mn;
           }
         }
     if ((lane & 3) == 0) {
@@ -247,8 +319,8 @@ __global__ void __launch_bounds__(kStatsThreads) imp_stats_kernel(
         for (int hh = 0; hh < 2; ++hh) {
           const int r = r0 + mt * 16 + rr + 8 * hh;
           if (r < R) {
-            out[r * 2] = m[mt][hh];
-            out[r * 2 + 1] = l[mt][hh];
+            out[r * 2] = m[g2][mt][hh];
+            out[r * 2 + 1] = l[g2][mt][hh];
           }
         }
     }
@@ -745,7 +817,9 @@ cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* 
   float* part = scratch;
   float* stats = scratch + static_cast<size_t>(B) * Hkv * nblk * R * 2;
   const size_t lds = static_cast<size_t>(D + 8) * 2;
-  const size_t sh1 = ((R + 31) / 32 * 32 + kImpKeys) * lds;
+  const size_t sh1 = ((R + 31) / 32 * 32 + 2 * kImpKeys) * lds;
+  // pass 1 is persistent: about one CTA per SM over the (b, h) pairs
+  const int nsplit = std::max(1, std::min(nblk, l.num_sms / std::max(1, B * Hkv)));
   const size_t sh2 = (R + kImpKeys) * lds + static_cast<size_t>(R) * 2 * 4;
   const dim3 grid(nblk, Hkv, B);
   const float sl2 = scale * kLog2eF;
@@ -756,18 +830,20 @@ cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* 
     e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<128>), sh1);
     if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<128>), sh2);
     if (e != cudaSuccess) return e;
-    imp_stats_kernel<128><<<grid, kStatsThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
+    imp_stats_kernel<128><<<dim3(nsplit, Hkv, B), kStatsThreads, sh1, l.stream>>>(
+        q, k, S, Hq, Hkv, G, n_obs, sl2, nblk, part);
     imp_combine_kernel<<<dim3(B * Hkv, (R + 31) / 32), kCombineWarps * 32, 0, l.stream>>>(
-        part, nblk, R, stats);
+        part, nsplit, R, stats);
     imp_weight_kernel<128><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
                                                                  stats, imp);
   } else {
     e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<64>), sh1);
     if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<64>), sh2);
     if (e != cudaSuccess) return e;
-    imp_stats_kernel<64><<<grid, kStatsThreads, sh1, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2, part);
+    imp_stats_kernel<64><<<dim3(nsplit, Hkv, B), kStatsThreads, sh1, l.stream>>>(
+        q, k, S, Hq, Hkv, G, n_obs, sl2, nblk, part);
     imp_combine_kernel<<<dim3(B * Hkv, (R + 31) / 32), kCombineWarps * 32, 0, l.stream>>>(
-        part, nblk, R, stats);
+        part, nsplit, R, stats);
     imp_weight_kernel<64><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
                                                                 stats, imp);
   }
