@@ -105,3 +105,20 @@ def test_decode_step_rejects_on_host(csa):
     assert csa.lib.csa_decode_step(ctypes.byref(d), ctypes.c_void_p(0)) == 1
     assert "mode" in csa.csa_last_error_string()
     assert csa.lib.csa_decode_step(None, ctypes.c_void_p(0)) == 1
+
+
+def test_decode_step_host_rejects_on_host(csa):
+    """csa_decode_step_host refuses a missing descriptor and the RoPE-aware
+    split (q_score set) before touching any buffer."""
+    lib = csa.lib
+    s0 = ctypes.c_void_p(0)
+    assert lib.csa_decode_step_host(None, None, None, None, s0) == 1
+    assert "descriptor" in csa.csa_last_error_string()
+    d = csa.decode_step_desc(B=1, Hq=4, Hkv=1, D=128, T=1024, L=64, scale=0.1, mode=0, kmax=4)
+    d.q_score = 4096
+    assert lib.csa_decode_step_host(ctypes.byref(d), None, None, None, s0) == 2
+    assert "q_score" in csa.csa_last_error_string()
+    d.q_score = None
+    # NULL host buffers
+    assert lib.csa_decode_step_host(ctypes.byref(d), None, None, None, s0) == 1
+    assert "q_host" in csa.csa_last_error_string()
