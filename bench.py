@@ -397,6 +397,45 @@ def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: f
             "tau": tau}
 
 
+def time_token_importance(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1):
+    """The first two stages of the Token Sparse call alone on the 32K prefill
+    inputs: the proxy importance (csa_token_importance) and the coverage
+    budget (csa_token_budget), each between its own events."""
+    from query_adaptive_chunk_b200 import csa
+    inp = synth.make_prefill_inputs(w, device="cuda")
+    Q, K = inp["Q"], inp["K"]
+    scale = 1.0 / math.sqrt(w.D)
+    imp = torch.empty(w.B, w.Hkv, w.S, dtype=torch.float32, device="cuda")
+    nb = csa.csa_token_importance_scratch_bytes(w.B, w.S, w.Hq, w.Hkv, n_obs)
+    scratch = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    k_seq = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    k_unit = torch.zeros(w.B * w.Hkv, dtype=torch.int32, device="cuda")
+
+    def call(e=None):
+        if e:
+            e[0].record()
+        csa.csa_token_importance(Q, K, w.B, w.S, w.Hq, w.Hkv, w.D, n_obs, scale, imp, scratch, nb)
+        if e:
+            e[1].record()
+        csa.csa_token_budget(imp, w.B, w.S, w.Hkv, tau, 64, k_seq, k_unit)
+        if e:
+            e[2].record()
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    imp_ms, bud_ms = [], []
+    for _ in range(steps):
+        flush()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        call(e)
+        torch.cuda.synchronize()
+        imp_ms.append(e[0].elapsed_time(e[1]))
+        bud_ms.append(e[1].elapsed_time(e[2]))
+    csa.csa_check_device_status()
+    return {"importance_ms": imp_ms, "budget_ms": bud_ms, "budget": int(k_seq.max())}
+
+
 def oracle_decode_seconds(w, inp, max_seconds: float = 20.0, max_steps: int = 5, threads: int = 1):
     """The CPU oracle's per-step work (score + select + attention, summaries
     precomputed) on this workload, a bounded number of steps.  threads == 1:
@@ -618,6 +657,12 @@ def run_only(args, flush, peaks):
         r = time_token_sparse(synth.PREFILL_32K, args.steps, args.warmup, flush)
         print(json.dumps({"workload": args.only, "ms": statistics.mean(r["ms"]),
                           "budget": r["budget"], "flops": r["flops"]}))
+        return 0
+    if args.only == "token_importance_bf16_seq32k":
+        r = time_token_importance(synth.PREFILL_32K, args.steps, args.warmup, flush)
+        print(json.dumps({"workload": args.only,
+                          "importance_ms": statistics.mean(r["importance_ms"]),
+                          "budget_ms": statistics.mean(r["budget_ms"]), "budget": r["budget"]}))
         return 0
     byname = {w.name: w for w in synth.ALL_WORKLOADS}
     w = byname[args.only]
