@@ -489,7 +489,9 @@ CSA_API csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream str
  * (one small copy kernel) and the decode stores the result straight into
  * it; d->out and d->lse_out are then left as they were.  Otherwise the
  * copies are cudaMemcpyAsync transfers and d->out / d->lse_out hold the
- * result too.  The call captures into a CUDA graph, whose replays read and
+ * result too.  Either way the transfers happen when the stream reaches
+ * them: q_host must keep the query, and out_host / lse_host must not be
+ * read, until the stream has passed the call.  The call captures into a CUDA graph, whose replays read and
  * write the same host buffers.  CSA_ERR_UNSUPPORTED with q_score set (the
  * RoPE-aware split rotates the query on the device: csa_rope, then
  * csa_decode_step).  Once the decode's own arguments have passed their
