@@ -109,6 +109,7 @@ class SparseDecoder:
                                 csa.csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts))
             self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
         self.desc = None
+        self.q_dev = None  # the device query buffer of step_host, made on first use
         if fused and self.dtype == csa.CSA_BF16:
             mode = {"topk": csa.CSA_SELECT_TOPK, "topp": csa.CSA_SELECT_TOPP,
                     "hier": csa.CSA_SELECT_HIER, "topk_union": csa.CSA_SELECT_TOPK_UNION}[select]
@@ -209,7 +210,7 @@ class SparseDecoder:
         Needs the one-call bf16 step without RoPE."""
         if self.desc is None or self.q_rot is not None:
             raise ValueError("step_host needs a fused bf16 decoder without RoPE")
-        if getattr(self, "q_dev", None) is None:
+        if self.q_dev is None:
             self.q_dev = torch.empty(self.B, self.Hq, self.D, dtype=torch.bfloat16,
                                      device=self.out.device)
         self.desc.q = self.q_dev.data_ptr()
