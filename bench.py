@@ -331,6 +331,26 @@ def time_e2e(w, dec, inp, steps: int, flush):
         out_host.numel() * out_host.element_size()
 
 
+def host_cpu_model() -> str:
+    """The host CPU's model name (first entry of /proc/cpuinfo), or ""."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
+def diagonal_blocks(idx: torch.Tensor, n_tiles: int) -> int:
+    """Executed diagonal blocks of a block-sparse prefill whose chunk equals
+    its tile (tile_m == L): the units u = (b * Hkv + h) * n_tiles + t whose
+    index row holds chunk t."""
+    t = torch.arange(idx.shape[0], dtype=torch.int64) % n_tiles
+    return int((idx.to(torch.int64) == t[:, None]).any(dim=1).sum())
+
+
 def time_prefill(w, steps: int, warmup: int, flush):
     from query_adaptive_chunk_b200.steps import BlockSparsePrefill
     inp = synth.make_prefill_inputs(w, device="cuda")
@@ -353,8 +373,12 @@ def time_prefill(w, steps: int, warmup: int, flush):
         att_ms.append(e[1].elapsed_time(e[2]))
     cnt = pf.count.cpu()
     blocks = int(cnt.sum())
-    flops = blocks * w.G * 2 * (2 * w.tile_m * w.L * w.D)
-    return {"select_ms": sel_ms, "attend_ms": att_ms, "blocks": blocks, "flops": flops}
+    per_block = w.G * 2 * (2 * w.tile_m * w.L * w.D)
+    flops = blocks * per_block
+    # causal-effective count: a diagonal block does about half the work
+    diag = diagonal_blocks(pf.idx.cpu(), pf.n_tiles) if w.tile_m == w.L else 0
+    return {"select_ms": sel_ms, "attend_ms": att_ms, "blocks": blocks, "flops": flops,
+            "causal_flops": (blocks - diag / 2) * per_block, "diagonal_blocks": diag}
 
 
 def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1):
@@ -564,7 +588,8 @@ def run_ours(args):
         t = oracle_decode_seconds(w, r["inp"], max_seconds=20.0, max_steps=5)
         cpu = {"value": 1e6 * statistics.mean(t), "unit": "us/step", "cores": 1, "kind": "oracle",
                "sample": f"{len(t)} whole decode steps of {w.name} (all {w.B * w.Hkv} units), "
-                         "summaries precomputed, numpy fp64 single-threaded"}
+                         "summaries precomputed, numpy fp64 single-threaded",
+               "cpu_model": host_cpu_model(), "host_cores": os.cpu_count()}
         n_thr = min(os.cpu_count() or 1, w.B * w.Hkv)
         if n_thr > 1:
             tp = oracle_decode_seconds(w, r["inp"], max_seconds=10.0, max_steps=5, threads=n_thr)
@@ -647,7 +672,10 @@ def other_workloads(args, flush, peaks):
                    "executed_blocks": r["blocks"], "flops": r["flops"],
                    "tflops": round(tflops, 1),
                    "frac_of_measured_bf16": round(tflops / peaks["bf16_tflops"], 4),
-                   "frac_of_sustained_bf16": round(tflops / peaks["bf16_tflops_sustained"], 4)}
+                   "frac_of_sustained_bf16": round(tflops / peaks["bf16_tflops_sustained"], 4),
+                   "diagonal_blocks": r["diagonal_blocks"],
+                   "causal_effective_flops": int(r["causal_flops"]),
+                   "causal_effective_tflops": round(r["causal_flops"] / (att_ms * 1e-3) / 1e12, 1)}
     return out
 
 
