@@ -536,7 +536,8 @@ def run_reference(args):
                        "full_heads": list(w.full_heads)},
             "cpu_baseline": {"value": us, "unit": "us/step", "cores": 1, "kind": "oracle",
                              "sample": f"{len(t)} whole decode steps of {w.name} (all 8 units), "
-                                       "summaries precomputed, numpy fp64 single-threaded"},
+                                       "summaries precomputed, numpy fp64 single-threaded",
+                             "cpu_model": host_cpu_model(), "host_cores": os.cpu_count()},
             "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
