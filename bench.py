@@ -628,6 +628,10 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "mode": e2e_mode,
                 "direct_launch_value": round(e2e_eager_us, 3)},
         "gpu_launches": 2 * args.steps,
+        "timing_stats": {"rank": 0, "step_us_median": round(1000 * statistics.median(r["step_ms"]), 3),
+                         "step_us_min": round(1000 * min(r["step_ms"]), 3),
+                         "decode_us_median": round(1000 * statistics.median(r["decode_ms"]), 3),
+                         "decode_us_min": round(1000 * min(r["decode_ms"]), 3)},
         "clocks": clocks,
         "cpu_baseline": cpu,
         "workloads": extra,
