@@ -678,6 +678,7 @@ def other_workloads(args, flush, peaks):
                    "tflops": round(tflops, 1),
                    "frac_of_measured_bf16": round(tflops / peaks["bf16_tflops"], 4),
                    "frac_of_sustained_bf16": round(tflops / peaks["bf16_tflops_sustained"], 4),
+                   "frac_of_2250_nominal_bf16": round(tflops / 2250.0, 4),
                    "diagonal_blocks": r["diagonal_blocks"],
                    "causal_effective_flops": int(r["causal_flops"]),
                    "causal_effective_tflops": round(r["causal_flops"] / (att_ms * 1e-3) / 1e12, 1)}
