@@ -319,7 +319,11 @@ def _pins_fail():
 @pytest.mark.parametrize("name,mutant", MUTANTS, ids=lambda x: getattr(x, "__name__", x))
 def test_mutant_is_caught(monkeypatch, name, mutant):
     monkeypatch.setattr(O, name, mutant)
-    assert _pins_fail(), f"no pin caught the planted mistake {mutant.__name__}"
+    # a planted mistake may leave a row with nothing visible (inf - inf):
+    # that is for the pins to catch, not a warning
+    with np.errstate(invalid="ignore"):
+        caught = _pins_fail()
+    assert caught, f"no pin caught the planted mistake {mutant.__name__}"
 
 
 def test_unmutated_oracle_passes():
