@@ -26,8 +26,10 @@ What it computes, in the order the pages give it:
   always kept.
 * Exact attention over the raw KV of the selected chunks (SSA summary,
   "방법론": standard attention over the hybrid context), and over the hybrid
-  context itself, the gist KV of every chunk plus the raw KV of the selected
-  ones ("방법론", "기술 상세"), computed as split-K
+  context itself: the gist KV and the raw KV of the selected chunks
+  ("방법론", "기술 상세"), or, read from the glossary entry "Selective
+  Unfolding", the gist KV of every chunk plus the raw KV of the selected
+  ones; computed as split-K
   partials combined afterwards (SSA summary, "핵심 기여": compact index list and
   split-K partial attention).
 * Block-sparse causal prefill over per-query-tile chunk sets (SSA summary,
@@ -326,23 +328,36 @@ def rope(x: np.ndarray, pos, theta: float) -> np.ndarray:
     return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
 
 
-def hybrid_unit(q_group, K_unit, V_unit, Kg_unit, Vg_unit, chunks, L: int, scale: float):
-    """Attention of one unit's query heads over its hybrid context (SSA
-    summary, "방법론" and "기술 상세": K_hybrid and V_hybrid are the gist KV
-    together with the raw KV of the selected chunks I_t, attended with
-    standard attention).
+GIST_SCOPES = ("selected", "all")
 
-    Reading: every chunk keeps its gist token in the context (glossary entry
-    "Selective Unfolding": the query first meets the gist tokens of all
-    chunks), and the raw tokens of the selected chunks are added next to
-    them.  One softmax runs over the union, with the same scale for gist and
-    raw logits.  K_unit/V_unit [T, D] raw; Kg_unit/Vg_unit [C, D], one gist
+
+def hybrid_unit(q_group, K_unit, V_unit, Kg_unit, Vg_unit, chunks, L: int, scale: float,
+                scope: str):
+    """Attention of one unit's query heads over its hybrid context (SSA
+    summary, "방법론" and "기술 상세").
+
+    scope = "selected" (the method and technical-details sections): the top-k
+    chunks I_t are the only ones brought back, each with its gist KV and its
+    raw KV; K_hybrid / V_hybrid are the union of the gist rows and the raw
+    rows of the chunks in I_t.
+    scope = "all" (the glossary entry "Selective Unfolding" read as the
+    context): the gist row of every chunk stays in the context and the raw
+    rows of the chunks in I_t are added next to them.
+
+    One softmax runs over the union, with the same scale for gist and raw
+    logits.  K_unit/V_unit [T, D] raw; Kg_unit/Vg_unit [C, D], one gist
     key/value per chunk -> o [G, D], lse [G]."""
-    tok = chunk_tokens(sorted(chunks), L)
+    if scope not in GIST_SCOPES:
+        raise ValueError(f"gist scope {scope!r}")
+    sel = sorted(chunks)
+    tok = chunk_tokens(sel, L)
+    Kg = np.asarray(Kg_unit, dtype=np.float64)
+    Vg = np.asarray(Vg_unit, dtype=np.float64)
+    gist_rows = np.asarray(sel, dtype=np.int64) if scope == "selected" else np.arange(Kg.shape[0])
     Kr = np.asarray(K_unit, dtype=np.float64)[tok]
     Vr = np.asarray(V_unit, dtype=np.float64)[tok]
-    Kh = np.concatenate([Kr, np.asarray(Kg_unit, dtype=np.float64)], axis=0)
-    Vh = np.concatenate([Vr, np.asarray(Vg_unit, dtype=np.float64)], axis=0)
+    Kh = np.concatenate([Kr, Kg[gist_rows]], axis=0)
+    Vh = np.concatenate([Vr, Vg[gist_rows]], axis=0)
     return attend(q_group, Kh, Vh, np.arange(Kh.shape[0]), scale)
 
 

@@ -33,22 +33,41 @@ def unit_summaries(K_unit, L: int, proj=None, block_chunks: int = 2048) -> np.nd
     return np.concatenate(parts, axis=0)
 
 
+def topp_logit_scale(D: int) -> float:
+    """Logit scale of the top-p chunk softmax: 1/sqrt(D), D the attention
+    head dimension, also when the scores come from a low-rank projection.
+    Reading: the HiLS review's chunk-mass surrogate (section 1) makes a
+    chunk's attention mass proportional to exp(q . k_mean / sqrt(D)); the
+    projected score stands in for q . k_mean (the Gaussian projection keeps
+    inner products in expectation), so the attention's own scale applies."""
+    return 1.0 / math.sqrt(D)
+
+
+def rope_query_position(T: int) -> int:
+    """Position of the decoding query in a context of T cached tokens: the
+    context's last token, T - 1 (the current token's key is the last row of
+    the cache)."""
+    return T - 1
+
+
 def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_local: int,
                 k_free: int = 0, proj=None, p: float = 0.0, budget: int = 0,
                 full_heads=(), Gm: int = 0, top_meta: int = 0, units=None,
-                with_attention: bool = True, gist=None, rope_theta: float = 0.0) -> dict:
+                with_attention: bool = True, gist=None, gist_scope: str = "",
+                rope_theta: float = 0.0) -> dict:
     """One decode step of the units (b, kvh) listed (default: all).
 
     q [B, Hq, D]; K, V [B, Hkv, T, D].  Returns a dict with, per unit, the
     ascending chunk set, the boundary gap(s), n_p for top-p, and when
     ``with_attention`` the output rows o [G, D] and lse [G].  gist = (Kg, Vg),
     each [B, Hkv, T // L, D]: the sparse units attend over the hybrid context
-    (their gist rows plus the raw KV of their chunks, ``hybrid_unit``).
+    of ``gist_scope`` ("selected": gist and raw rows of the chosen chunks;
+    "all": every chunk's gist row plus the raw rows of the chosen chunks;
+    ``hybrid_unit``).
     rope_theta > 0: the RoPE-aware split (RTPurbo review, section 1): q and K
     are the pre-RoPE ones and score as they are; attention runs on the
-    rotated query (position T - 1, the context's last token) and keys
-    (positions 0 .. T - 1), each stored in the cache's dtype as a decode
-    step would hold them."""
+    rotated query (at ``rope_query_position``) and keys (positions 0 .. T - 1),
+    each stored in the cache's dtype as a decode step would hold them."""
     B, Hkv, T, D = K.shape
     Hq = q.shape[1]
     G = Hq // Hkv
@@ -72,7 +91,7 @@ def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_lo
         elif select == "topp":
             summ = unit_summaries(K[b, h], L, projn)
             s = O.score_chunks(qg[None, None], summ[None, None], 1, projn)[0, 0, 0]
-            chunks, n_p, gap = O.select_topp(s, 1.0 / math.sqrt(D), p, budget, n_sink, n_local)
+            chunks, n_p, gap = O.select_topp(s, topp_logit_scale(D), p, budget, n_sink, n_local)
             res["n_p"][(b, h)] = n_p
         elif select == "hier":
             summ = unit_summaries(K[b, h], L)
@@ -86,14 +105,14 @@ def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_lo
         res["gap"][(b, h)] = gap
         if with_attention and rope_theta > 0:
             tok = O.chunk_tokens(chunks, L)
-            qr = _stored(O.rope(qg, np.full(G, T - 1), rope_theta), q)
+            qr = _stored(O.rope(qg, np.full(G, rope_query_position(T)), rope_theta), q)
             Kr = _stored(O.rope(to_np(K[b, h][_index(K, tok)]), tok, rope_theta), K)
             o, lse = O.attend(qr, Kr, to_np(V[b, h][_index(V, tok)]), np.arange(len(tok)), scale)
             res["o"][(b, h)] = o
             res["lse"][(b, h)] = lse
         elif with_attention and gist is not None and h not in tuple(full_heads):
             o, lse = O.hybrid_unit(qg, to_np(K[b, h]), to_np(V[b, h]), to_np(gist[0][b, h]),
-                                   to_np(gist[1][b, h]), chunks, L, scale)
+                                   to_np(gist[1][b, h]), chunks, L, scale, gist_scope)
             res["o"][(b, h)] = o
             res["lse"][(b, h)] = lse
         elif with_attention:
@@ -107,8 +126,9 @@ def decode_step(q, K, V, *, L: int, scale: float, select: str, n_sink: int, n_lo
 
 
 def _stored(x: np.ndarray, like) -> np.ndarray:
-    """x rounded to the element type of `like` (a bf16 cache holds bf16), as
-    fp64.  torch's round-to-nearest-even conversion is the library step."""
+    """x rounded to the element type of `like`, as fp64: a bf16 cache holds
+    its rotated keys (and the rotated query) in bf16, as a post-RoPE KV cache
+    does.  torch's round-to-nearest-even conversion is the library step."""
     if hasattr(like, "dtype") and str(like.dtype) == "torch.bfloat16":
         import torch
         return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()

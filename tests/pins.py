@@ -87,43 +87,109 @@ def check_empty_attention():
 
 
 def check_hybrid_golden():
-    """Hybrid context (gist KV of every chunk + raw KV of the selected ones):
-    the hand-worked cases of tests/golden/hybrid_cases.json."""
+    """Hybrid context in both gist scopes ("selected": gist and raw KV of the
+    chosen chunks; "all": every chunk's gist plus the raw KV of the chosen
+    ones): the hand-worked cases of tests/golden/hybrid_cases.json."""
     g = _golden("hybrid_cases.json")
     q, K, V = (np.array(g[k], dtype=np.float64) for k in ("q", "K", "V"))
     Kg, Vg = np.array(g["Kg"], dtype=np.float64), np.array(g["Vg"], dtype=np.float64)
-    for c in g["cases"]:
-        o, lse = O.hybrid_unit(q, K, V, Kg, Vg, c["chunks"], g["L"], g["scale"])
-        assert np.allclose(o, np.array(c["o"]), rtol=0, atol=1e-12), (c["chunks"], o)
-        assert np.allclose(lse, np.array(c["lse"]), rtol=0, atol=1e-12), (c["chunks"], lse)
+    for scope in ("all", "selected"):
+        for c in g["cases_" + scope]:
+            o, lse = O.hybrid_unit(q, K, V, Kg, Vg, c["chunks"], g["L"], g["scale"], scope)
+            want_lse = np.array([float(x) for x in c["lse"]])
+            assert np.allclose(o, np.array(c["o"]), rtol=0, atol=1e-12), (scope, c["chunks"], o)
+            assert np.array_equal(np.isinf(lse), np.isinf(want_lse)), (scope, c["chunks"], lse)
+            fin = np.isfinite(want_lse)
+            assert np.allclose(lse[fin], want_lse[fin], rtol=0, atol=1e-12), (scope, c["chunks"], lse)
 
 
 def check_hybrid_vs_sdpa(seed=16, G=4, D=16, T=256, L=32):
     """Hybrid context == fp64 SDPA over the raw cache with the C gist rows
-    appended, masked to keep the selected chunks' raw tokens and every gist
-    row; lse == logsumexp of the same masked logits.  Chunk sets from empty
-    to all chunks."""
+    appended, masked to keep the selected chunks' raw tokens and the gist
+    rows of the scope (the selected chunks' own, or every chunk's); lse ==
+    logsumexp of the same masked logits.  Chunk sets from empty to all
+    chunks (an empty set in the "selected" scope has nothing to attend)."""
     rng = np.random.default_rng(seed)
     C = T // L
-    for n_sel in (0, 1, 3, C):
-        q = rng.standard_normal((G, D))
-        K, V = rng.standard_normal((T, D)), rng.standard_normal((T, D))
-        Kg, Vg = rng.standard_normal((C, D)), rng.standard_normal((C, D))
-        chunks = sorted(rng.choice(C, size=n_sel, replace=False).tolist())
-        scale = 1.0 / math.sqrt(D)
-        o, lse = O.hybrid_unit(q, K, V, Kg, Vg, chunks, L, scale)
-        Ke, Ve = np.concatenate([K, Kg]), np.concatenate([V, Vg])
-        keep = np.zeros(T + C, dtype=bool)
-        keep[T:] = True
-        for c in chunks:
-            keep[c * L:(c + 1) * L] = True
-        mask = np.broadcast_to(keep, (G, 1, T + C))
-        ref = _sdpa(q[:, None, :], np.broadcast_to(Ke, (G, T + C, D)),
-                    np.broadcast_to(Ve, (G, T + C, D)), mask=mask, scale=scale)[:, 0]
-        assert np.allclose(o, ref, rtol=0, atol=1e-12), np.abs(o - ref).max()
-        logits = torch.as_tensor(q @ Ke.T * scale)
-        logits[:, ~torch.as_tensor(keep)] = -math.inf
-        assert np.allclose(lse, torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
+    for scope in ("all", "selected"):
+        for n_sel in (0, 1, 3, C):
+            q = rng.standard_normal((G, D))
+            K, V = rng.standard_normal((T, D)), rng.standard_normal((T, D))
+            Kg, Vg = rng.standard_normal((C, D)), rng.standard_normal((C, D))
+            chunks = sorted(rng.choice(C, size=n_sel, replace=False).tolist())
+            scale = 1.0 / math.sqrt(D)
+            o, lse = O.hybrid_unit(q, K, V, Kg, Vg, chunks, L, scale, scope)
+            Ke, Ve = np.concatenate([K, Kg]), np.concatenate([V, Vg])
+            keep = np.zeros(T + C, dtype=bool)
+            for c in chunks:
+                keep[c * L:(c + 1) * L] = True
+                keep[T + c] = scope == "selected"
+            if scope == "all":
+                keep[T:] = True
+            if not keep.any():
+                assert np.all(o == 0) and np.all(lse == -math.inf), (scope, o, lse)
+                continue
+            mask = np.broadcast_to(keep, (G, 1, T + C))
+            ref = _sdpa(q[:, None, :], np.broadcast_to(Ke, (G, T + C, D)),
+                        np.broadcast_to(Ve, (G, T + C, D)), mask=mask, scale=scale)[:, 0]
+            assert np.allclose(o, ref, rtol=0, atol=1e-12), (scope, np.abs(o - ref).max())
+            logits = torch.as_tensor(q @ Ke.T * scale)
+            logits[:, ~torch.as_tensor(keep)] = -math.inf
+            assert np.allclose(lse, torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
+
+
+def check_pipeline_topp_scale_under_projection():
+    """The decode step's top-p branch softmaxes the (projected) chunk scores
+    with the attention scale 1/sqrt(D) of the head dimension D, not
+    1/sqrt(R) of the projection rank and not the caller's attention scale.
+    Hand case: D = 4, R = 2, P = the first two unit vectors, q = e0, four
+    chunks of two identical keys, chunk 1's keys e0 * 2 ln 3, the others 0.
+    Scores (0, 2 ln 3, 0, 0).  With 1/sqrt(D) = 1/2 the weights are
+    (1, 3, 1, 1): chunk 1 holds 1/2 < p = 0.6, and chunk 0 (ties to the lower
+    index) brings the prefix to 2/3, so the set is {0, 1}.  With 1/sqrt(R)
+    the weight of chunk 1 is 3^sqrt(2) (mass 0.61 >= 0.6) and with scale 1
+    it is 9 (mass 3/4): both would give {1}."""
+    from oracle import pipeline as OP
+    D, L, C = 4, 2, 4
+    K = np.zeros((1, 1, C * L, D))
+    K[0, 0, 1 * L:2 * L, 0] = 2.0 * math.log(3.0)
+    q = np.zeros((1, 1, D))
+    q[0, 0, 0] = 1.0
+    P = np.zeros((D, 2))
+    P[0, 0] = P[1, 1] = 1.0
+    res = OP.decode_step(q, K, np.zeros_like(K), L=L, scale=1.0, select="topp", n_sink=0,
+                         n_local=0, proj=P, p=0.6, budget=C, with_attention=False)
+    assert res["sets"][(0, 0)] == [0, 1], res["sets"]
+    assert res["n_p"][(0, 0)] == 2, res["n_p"]
+
+
+def check_pipeline_rope_branch():
+    """The decode step's RoPE branch: the query sits at position T - 1 (the
+    context's last token), and with a bf16 cache the rotated query and keys
+    are held in bf16.  Hand case: D = 2 (one pair turning by pos radians),
+    L = 1, T = 2, q = e0, keys e0 and e0, values e0 and e1, scale 1.
+    fp64 inputs: the rotated query at position 1 meets k0 (position 0) with
+    cos(1 - 0) and k1 (position 1) with cos 0 = 1, so the weight of v0 is
+    1 / (1 + e^(1 - cos 1)); a query at position T = 2 would give
+    1 / (1 + e^(cos 1 - cos 2)).  bf16 inputs: cos 1 = 0.5403 and
+    sin 1 = 0.8415 lie in [0.5, 1), where bf16 steps by 2^-8, so they are
+    held as 138/256 and 215/256; the logits become 138/256 and
+    (138^2 + 215^2)/256^2 and the weight of v0 is
+    1 / (1 + e^((138^2 + 215^2)/65536 - 138/256))."""
+    from oracle import pipeline as OP
+    for dtype in (torch.float64, torch.bfloat16):
+        q = torch.tensor([[[1.0, 0.0]]], dtype=dtype)
+        K = torch.tensor([[[[1.0, 0.0], [1.0, 0.0]]]], dtype=dtype)
+        V = torch.tensor([[[[1.0, 0.0], [0.0, 1.0]]]], dtype=dtype)
+        res = OP.decode_step(q, K, V, L=1, scale=1.0, select="topk", n_sink=1, n_local=1,
+                             k_free=0, rope_theta=10000.0)
+        assert res["sets"][(0, 0)] == [0, 1]
+        if dtype == torch.float64:
+            w0 = 1.0 / (1.0 + math.exp(1.0 - math.cos(1.0)))
+        else:
+            w0 = 1.0 / (1.0 + math.exp((138 ** 2 + 215 ** 2) / 65536.0 - 138 / 256.0))
+        o = res["o"][(0, 0)]
+        assert np.allclose(o, [[w0, 1.0 - w0]], rtol=0, atol=1e-12), (dtype, o, w0)
 
 
 def check_rope_closed_forms(seed=18):
@@ -535,6 +601,7 @@ ALL_CHECKS = [
     check_topp_golden, check_topp_invariants, check_hier_golden, check_hier_all_metas_is_flat,
     check_meta_linearity, check_merge_closed_form, check_partition,
     check_prefill_dense_causal, check_prefill_masked, check_hybrid_golden, check_hybrid_vs_sdpa,
+    check_pipeline_topp_scale_under_projection, check_pipeline_rope_branch,
     check_rope_closed_forms, check_token_sparse_golden, check_token_sparse_invariants,
     check_token_sparse_vs_sdpa,
 ]

@@ -10,6 +10,7 @@ import pytest
 
 import pins
 from oracle import csa_oracle as O
+from oracle import pipeline as OP
 
 _orig = {name: getattr(O, name) for name in
          ["attend", "select_topk", "select_topp", "score_chunks", "lse_merge",
@@ -175,19 +176,46 @@ def per_head_scores_group_summed(q_group, summ_unit, proj=None):
     return np.repeat(per.sum(axis=0, keepdims=True), per.shape[0], axis=0)
 
 
-def hybrid_selected_gists_only(q, K, V, Kg, Vg, chunks, L, scale):
-    sel = sorted(chunks)
-    return _orig["hybrid_unit"](q, K, V, np.asarray(Kg)[sel], np.asarray(Vg)[sel], chunks, L,
-                                scale)
+def hybrid_scope_swapped(q, K, V, Kg, Vg, chunks, L, scale, scope):
+    other = "all" if scope == "selected" else "selected"
+    return _orig["hybrid_unit"](q, K, V, Kg, Vg, chunks, L, scale, other)
 
 
-def hybrid_no_gists(q, K, V, Kg, Vg, chunks, L, scale):
+def hybrid_no_gists(q, K, V, Kg, Vg, chunks, L, scale, scope):
     return O.decode_unit(q, K, V, chunks, L, scale)
 
 
-def hybrid_gist_logits_unscaled(q, K, V, Kg, Vg, chunks, L, scale):
+def hybrid_gist_logits_unscaled(q, K, V, Kg, Vg, chunks, L, scale, scope):
     return _orig["hybrid_unit"](q, K, V, np.asarray(Kg, dtype=np.float64) / scale, Vg, chunks,
-                                L, scale)
+                                L, scale, scope)
+
+
+def hybrid_selected_gists_shifted(q, K, V, Kg, Vg, chunks, L, scale, scope):
+    # the selected scope takes the gist row of the chunk after each chosen one
+    if scope != "selected":
+        return _orig["hybrid_unit"](q, K, V, Kg, Vg, chunks, L, scale, scope)
+    C = np.asarray(Kg).shape[0]
+    nxt = [(c + 1) % C for c in range(C)]
+    return _orig["hybrid_unit"](q, K, V, np.asarray(Kg, dtype=np.float64)[nxt],
+                                np.asarray(Vg, dtype=np.float64)[nxt], chunks, L, scale, scope)
+
+
+# decode-step composition (oracle/pipeline.py)
+
+def topp_scale_of_rank(D):
+    return 1.0 / math.sqrt(2.0)  # 1/sqrt(R) of the pin's rank-2 projection
+
+
+def topp_scale_unit(D):
+    return 1.0
+
+
+def rope_query_at_T(T):
+    return T
+
+
+def stored_unrounded(x, like):
+    return np.asarray(x, dtype=np.float64)
 
 
 def rope_sin_sign_flipped(x, pos, theta):
@@ -292,9 +320,14 @@ MUTANTS = [
     ("select_topk_union", union_first_head_only),
     ("select_topk_union", union_of_group_sum),
     ("score_chunks_per_head", per_head_scores_group_summed),
-    ("hybrid_unit", hybrid_selected_gists_only),
+    ("hybrid_unit", hybrid_scope_swapped),
     ("hybrid_unit", hybrid_no_gists),
     ("hybrid_unit", hybrid_gist_logits_unscaled),
+    ("hybrid_unit", hybrid_selected_gists_shifted),
+    ("pipeline.topp_logit_scale", topp_scale_of_rank),
+    ("pipeline.topp_logit_scale", topp_scale_unit),
+    ("pipeline.rope_query_position", rope_query_at_T),
+    ("pipeline._stored", stored_unrounded),
     ("rope", rope_sin_sign_flipped),
     ("rope", rope_adjacent_pairs),
     ("rope", rope_freq_exponent_off),
@@ -318,7 +351,10 @@ def _pins_fail():
 
 @pytest.mark.parametrize("name,mutant", MUTANTS, ids=lambda x: getattr(x, "__name__", x))
 def test_mutant_is_caught(monkeypatch, name, mutant):
-    monkeypatch.setattr(O, name, mutant)
+    if name.startswith("pipeline."):
+        monkeypatch.setattr(OP, name.split(".", 1)[1], mutant)
+    else:
+        monkeypatch.setattr(O, name, mutant)
     # a planted mistake may leave a row with nothing visible (inf - inf):
     # that is for the pins to catch, not a warning
     with np.errstate(invalid="ignore"):
