@@ -184,7 +184,8 @@ def decoder_for(w, inp):
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
                          n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
                          budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta,
-                         hybrid=w.hybrid, rope_theta=w.rope_theta)
+                         hybrid=w.hybrid, gist=(inp["Kg"], inp["Vg"]) if w.hybrid else None,
+                         gist_scope=w.gist_scope or "selected", rope_theta=w.rope_theta)
 
 
 def selected_bytes(w, dec) -> tuple:
@@ -197,8 +198,10 @@ def selected_bytes(w, dec) -> tuple:
         n += w.C if (u % w.Hkv) in w.full_heads else c
     kv = n * w.L * w.D * elt * 2
     U_sparse = sum(1 for u in range(w.B * w.Hkv) if (u % w.Hkv) not in w.full_heads)
-    if w.hybrid:  # every sparse unit also reads one gist key and value row per chunk
+    if w.hybrid and w.gist_scope == "all":  # a gist key and value row per chunk
         kv += U_sparse * w.C * w.D * elt * 2
+    elif w.hybrid:  # a gist key and value row per selected chunk
+        kv += sum(c for u, c in enumerate(cnt) if (u % w.Hkv) not in w.full_heads) * w.D * elt * 2
     if w.select == "hier":
         summ = U_sparse * (w.C // w.Gm + w.top_meta * w.Gm) * w.D * 4
     else:
@@ -381,44 +384,121 @@ def time_prefill(w, steps: int, warmup: int, flush):
             "causal_flops": (blocks - diag / 2) * per_block, "diagonal_blocks": diag}
 
 
+TOKEN_STAGES = ("importance", "budget", "select", "compress", "attend", "decompress")
+
+
 def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1):
-    """Token Sparse Attention prefill on the 32K prefill inputs: the whole
-    call (importance, budget, token choice, gather, dense causal attention of
-    the kept tokens, scatter) between two events.  The call reads the budget
-    back to the host once (so it is not graph-replayed)."""
+    """Token Sparse Attention prefill (importance, budget, each KV head's own
+    tokens, compress, dense causal attention of the kept tokens, decompress).
+
+    Two CUDA graphs replayed alternately, L2 flushed before each: G1 is the
+    whole call (csa_token_sparse_prefill) between events and gives the
+    per-call time; G2 runs the same six steps as the separate calls with an
+    event between each pair and gives each step's share."""
     from query_adaptive_chunk_b200 import csa
     inp = synth.make_prefill_inputs(w, device="cuda")
     Q, K, V = inp["Q"], inp["K"], inp["V"]
-    scale = 1.0 / math.sqrt(w.D)
-    nb = csa.csa_token_sparse_workspace_bytes(w.B, w.S, w.Hq, w.Hkv, w.D, n_obs)
-    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    B, S, Hq, Hkv, D = w.B, w.S, w.Hq, w.Hkv, w.D
+    dev = "cuda"
+    scale = 1.0 / math.sqrt(D)
+    nb = csa.csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
     O = torch.empty_like(Q)
-    budget = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    budget = torch.zeros(B, dtype=torch.int32, device=dev)
+    # buffers of the separate calls
+    U = B * Hkv
+    ni = csa.csa_token_importance_scratch_bytes(B, S, Hq, Hkv, n_obs)
+    si = torch.empty(ni, dtype=torch.uint8, device=dev)
+    imp = torch.empty(B, Hkv, S, device=dev)
+    k_seq = torch.empty(B, dtype=torch.int32, device=dev)
+    k_unit = torch.empty(U, dtype=torch.int32, device=dev)
+    idx = torch.empty(U, S, dtype=torch.int32, device=dev)
+    cnt = torch.empty(U, dtype=torch.int32, device=dev)
+    Qc, Oc = torch.empty_like(Q), torch.empty_like(Q)
+    Kc, Vc = torch.empty_like(K), torch.empty_like(V)
+    na = csa.csa_token_attend_scratch_bytes(B, S, Hkv)
+    sa = torch.empty(na, dtype=torch.uint8, device=dev)
+    nd = csa.csa_token_decompress_scratch_bytes(B, S, Hkv)
+    sd = torch.empty(nd, dtype=torch.uint8, device=dev)
+    O2 = torch.empty_like(Q)
+    ev = [_ext_event() for _ in range(len(TOKEN_STAGES) + 1)]
 
-    def call():
-        csa.csa_token_sparse_prefill(Q, K, V, w.B, w.S, w.Hq, w.Hkv, w.D, n_obs, tau, scale, ws,
-                                     nb, O, budget)
+    def whole():
+        csa.csa_token_sparse_prefill(Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale, ws, nb, O,
+                                     budget)
+
+    def staged():
+        ev[0].record()
+        csa.csa_token_importance(Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp, si, ni)
+        ev[1].record()
+        csa.csa_token_budget(imp, B, S, Hkv, tau, 64, k_seq, k_unit)
+        ev[2].record()
+        csa.csa_token_select(imp, B, S, Hkv, k_unit, idx, cnt)
+        ev[3].record()
+        csa.csa_token_compress(Q, K, V, idx, cnt, B, S, Hq, Hkv, D, Qc, Kc, Vc)
+        ev[4].record()
+        csa.csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, sa, na, Oc)
+        ev[5].record()
+        csa.csa_token_decompress(Oc, idx, cnt, B, S, Hq, Hkv, D, sd, nd, O2)
+        ev[6].record()
 
     for _ in range(warmup):
-        call()
+        whole()
+        staged()
     torch.cuda.synchronize()
-    ms = []
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=side):
+        whole()
+    with torch.cuda.graph(g2, stream=side, capture_error_mode="relaxed"):
+        staged()
+    for _ in range(warmup):
+        g1.replay()
+        g2.replay()
+    torch.cuda.synchronize()
+    ms, stage_ms = [], {k: [] for k in TOKEN_STAGES}
     for _ in range(steps):
         flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        call()
+        g1.replay()
         e1.record()
+        flush()
+        g2.replay()
         torch.cuda.synchronize()
         ms.append(e0.elapsed_time(e1))
+        for i, k in enumerate(TOKEN_STAGES):
+            stage_ms[k].append(ev[i].elapsed_time(ev[i + 1]))
     csa.csa_check_device_status()
+    assert torch.equal(O, O2), "the separate calls must give the whole call's output"
+    del g1, g2
     k = int(budget.max())
-    kt = min(w.S, (k + 63) // 64 * 64)
+    kt = min(S, (k + 63) // 64 * 64)
     n_t = kt // 64
     # dense causal attention of the kept tokens: tile t sees tiles 0..t
-    flops = w.B * w.Hkv * (n_t * (n_t + 1) // 2) * w.G * 2 * (2 * 64 * 64 * w.D)
-    return {"ms": ms, "budget": k, "kept_tokens": kt, "flops": flops, "n_obs": n_obs,
-            "tau": tau}
+    flops = B * Hkv * (n_t * (n_t + 1) // 2) * w.G * 2 * (2 * 64 * 64 * D)
+    return {"ms": ms, "stage_ms": stage_ms, "budget": k, "kept_tokens": kt, "flops": flops,
+            "n_obs": n_obs, "tau": tau}
+
+
+def token_sparse_line(w, r) -> dict:
+    """Bench entry of a Token Sparse run: per-call time, the kept fraction,
+    the attention TFLOP/s, and the time of each step with the share of the
+    steps other than the dense attention (importance, budget, token choice,
+    compress, decompress) in the sum of the steps."""
+    ms = statistics.mean(r["ms"])
+    st = {k: statistics.mean(v) for k, v in r["stage_ms"].items()}
+    tot = sum(st.values())
+    return {"ms_per_step": round(ms, 4), "n_obs": r["n_obs"], "tau": r["tau"],
+            "budget_tokens": r["budget"], "kept_tokens_per_head": r["kept_tokens"],
+            "kept_fraction": round(r["kept_tokens"] / w.S, 4),
+            "attention_flops": r["flops"],
+            "effective_tflops_whole_step": round(r["flops"] / (ms * 1e-3) / 1e12, 1),
+            "attend_tflops": round(r["flops"] / (st["attend"] * 1e-3) / 1e12, 1),
+            "stage_ms": {k: round(v, 4) for k, v in st.items()},
+            "overhead_share": round((tot - st["attend"]) / tot, 4),
+            "importance_budget_share": round((st["importance"] + st["budget"]) / tot, 4)}
 
 
 def time_token_importance(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1):
@@ -647,7 +727,7 @@ def other_workloads(args, flush, peaks):
     out = {}
     steps = max(5, args.steps // 2)
     for w in (synth.TOPK_32K, synth.HIER_1M, synth.TINY_F32, synth.TOPK_UNION_32K,
-              synth.HYBRID_TOPK_32K, synth.ROPE_TOPK_32K):
+              synth.HYBRID_TOPK_32K, synth.HYBRID_ALL_TOPK_32K, synth.ROPE_TOPK_32K):
         r = time_decode(w, steps, args.warmup, flush)
         us = 1000 * statistics.mean(r["step_ms"])
         dus = 1000 * statistics.mean(r["decode_ms"])
@@ -659,17 +739,13 @@ def other_workloads(args, flush, peaks):
                        "selected_kv_bytes": r["kv_bytes"], "summary_bytes": r["summ_bytes"]}
         del r
         torch.cuda.empty_cache()
+    for tw, name in ((synth.PREFILL_32K, "token_sparse_prefill_bf16_seq32k"),
+                     (synth.TOKEN_SPARSE_HEAVY_32K, synth.TOKEN_SPARSE_HEAVY_32K.name)):
+        r = time_token_sparse(tw, steps, args.warmup, flush)
+        out[name] = token_sparse_line(tw, r)
+        del r
+        torch.cuda.empty_cache()
     w = synth.PREFILL_32K
-    r = time_token_sparse(w, steps, args.warmup, flush)
-    ms = statistics.mean(r["ms"])
-    out["token_sparse_prefill_bf16_seq32k"] = {
-        "ms_per_step": round(ms, 4), "n_obs": r["n_obs"], "tau": r["tau"],
-        "budget_tokens": r["budget"], "kept_tokens_per_head": r["kept_tokens"],
-        "kept_fraction": round(r["kept_tokens"] / w.S, 4),
-        "attention_flops": r["flops"],
-        "effective_tflops_whole_step": round(r["flops"] / (ms * 1e-3) / 1e12, 1)}
-    del r
-    torch.cuda.empty_cache()
     r = time_prefill(w, steps, args.warmup, flush)
     att_ms = statistics.mean(r["attend_ms"])
     tflops = r["flops"] / (att_ms * 1e-3) / 1e12
@@ -687,10 +763,11 @@ def other_workloads(args, flush, peaks):
 
 def run_only(args, flush, peaks):
     """Time one named workload alone and print its figures (profiling aid)."""
-    if args.only == "token_sparse_prefill_bf16_seq32k":
-        r = time_token_sparse(synth.PREFILL_32K, args.steps, args.warmup, flush)
-        print(json.dumps({"workload": args.only, "ms": statistics.mean(r["ms"]),
-                          "budget": r["budget"], "flops": r["flops"]}))
+    if args.only in ("token_sparse_prefill_bf16_seq32k", synth.TOKEN_SPARSE_HEAVY_32K.name):
+        tw = synth.PREFILL_32K if args.only == "token_sparse_prefill_bf16_seq32k" else \
+            synth.TOKEN_SPARSE_HEAVY_32K
+        r = time_token_sparse(tw, args.steps, args.warmup, flush)
+        print(json.dumps({"workload": args.only, **token_sparse_line(tw, r)}))
         return 0
     if args.only == "token_importance_bf16_seq32k":
         r = time_token_importance(synth.PREFILL_32K, args.steps, args.warmup, flush)

@@ -176,14 +176,58 @@ CSA_API csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, flo
  *   O [B, S, Hq, D] bf16 (output); budget_out [B] int32 device (output, the
  *   unrounded k_seq).  D = 128, Hq/Hkv = 4, S % 64 == 0, S <= 32768.
  *   workspace >= csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs).
- * The call reads the budgets back to the host to size the dense attention:
- * it synchronises `stream` once and cannot be captured in a CUDA graph. */
+ * Every step runs on the device from the budgets the device computed: the
+ * compressed buffers are laid out for S kept tokens, and the dense attention
+ * runs over the tiles within each KV head's budget, skipping the rest.  The
+ * call never blocks the host; it enqueues only kernel launches on `stream`. */
 CSA_API int64_t csa_token_sparse_workspace_bytes(int B, int S, int Hq, int Hkv, int D, int n_obs);
 CSA_API csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V, int B,
                                             int S, int Hq, int Hkv, int D, int n_obs, float tau,
                                             float scale, void* workspace,
                                             int64_t workspace_bytes, void* O,
                                             int32_t* budget_out, csa_stream stream);
+
+/* The steps of csa_token_sparse_prefill after the budget, as separate calls
+ * (the same kernels, in the same order): compress ("핵심 아키텍처": gather
+ * the kept tokens), attend (dense causal attention of the compressed
+ * sequences) and decompress (scatter back).  Same shapes and limits as the
+ * whole call (D = 128, Hq/Hkv = 4, S % 64 == 0, S <= 32768); compressed
+ * buffers Qc [B, S, Hq, D], Kc/Vc [B, Hkv, S, D], Oc [B, S, Hq, D] bf16,
+ * laid out for S kept tokens.
+ *
+ * csa_token_select: each KV head's own k_unit[b*Hkv + h] most important
+ *   tokens (importance desc, lower position on ties), ascending, into
+ *   idx [B*Hkv, S] int32 (unused slots -1) and count [B*Hkv] int32 ("헤드별
+ *   선택"); imp and k_unit as csa_token_importance / csa_token_budget give
+ *   them.
+ * csa_token_compress: compressed row t < count[u] of unit u = b*Hkv + h gets
+ *   token idx[u, t]: its K and V rows into Kc/Vc[b, h, t], the query rows of
+ *   the group's heads into Qc[b, t, h*G .. h*G+G-1].  Rows past a unit's
+ *   count are not written.
+ * csa_token_attend: dense causal attention of each unit's first k_unit[u]
+ *   compressed rows (k_unit a multiple of 64, as csa_token_budget gives it);
+ *   the rows of Oc past a unit's k_unit are not written.  scratch >=
+ *   csa_token_attend_scratch_bytes(B, S, Hkv) (the per-tile causal lists).
+ * csa_token_decompress: O[b, s, h*G+g] = Oc[b, t, h*G+g] where idx[u, t] = s,
+ *   0 for the positions a head did not keep; every row of O is written.
+ *   scratch >= csa_token_decompress_scratch_bytes(B, S, Hkv) (the inverse
+ *   map). */
+CSA_API csa_status csa_token_select(const float* imp, int B, int S, int Hkv,
+                                    const int32_t* k_unit, int32_t* idx, int32_t* count,
+                                    csa_stream stream);
+CSA_API csa_status csa_token_compress(const void* Q, const void* K, const void* V,
+                                      const int32_t* idx, const int32_t* count, int B, int S,
+                                      int Hq, int Hkv, int D, void* Qc, void* Kc, void* Vc,
+                                      csa_stream stream);
+CSA_API int64_t csa_token_attend_scratch_bytes(int B, int S, int Hkv);
+CSA_API csa_status csa_token_attend(const void* Qc, const void* Kc, const void* Vc,
+                                    const int32_t* k_unit, int B, int S, int Hq, int Hkv, int D,
+                                    float scale, void* scratch, int64_t scratch_bytes, void* Oc,
+                                    csa_stream stream);
+CSA_API int64_t csa_token_decompress_scratch_bytes(int B, int S, int Hkv);
+CSA_API csa_status csa_token_decompress(const void* Oc, const int32_t* idx, const int32_t* count,
+                                        int B, int S, int Hq, int Hkv, int D, void* scratch,
+                                        int64_t scratch_bytes, void* O, csa_stream stream);
 
 /* ---------------------------------------------------------------- a7
  * Tile-mean queries for prefill (HiLS review section 3: adjacent queries
@@ -222,6 +266,19 @@ CSA_API csa_status csa_score_chunks(const void* q, csa_dtype q_dtype, const floa
 CSA_API csa_status csa_select_topk(const float* scores, int U, int C, const int32_t* n_valid,
                            int k_free, int n_sink, int n_local, int32_t* idx, int32_t* count,
                            int kmax, csa_stream stream);
+
+/* csa_select_topk for the query tiles of a causal prefill (SSA summary
+ * "핵심 기여": block-skip prefill; HiLS review section 3: one chunk union per
+ * group of adjacent queries): unit u is tile t = u mod n_tiles of its
+ * (sequence, KV head), and sees the chunks [0, v) with
+ *   v = min(C, ((t + 1) * tile_m - 1) / L + 1)
+ * (every chunk holding a key at or before the tile's last row), so that the
+ * forced local chunk (n_local = 1) is the diagonal one.  Arguments and
+ * results otherwise as csa_select_topk; U % n_tiles == 0. */
+CSA_API csa_status csa_select_topk_causal(const float* scores, int U, int C, int n_tiles,
+                                          int tile_m, int L, int k_free, int n_sink, int n_local,
+                                          int32_t* idx, int32_t* count, int kmax,
+                                          csa_stream stream);
 
 /* ---------------------------------------------------------------- a3
  * Dynamic top-p selection per unit (RTPurbo review section 1, "Dynamic Top-p
@@ -377,29 +434,42 @@ CSA_API csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K
                                                     float* lse_out, csa_stream stream);
 
 /* ---------------------------------------------------------------- hybrid context
- * The merged decode over the hybrid context of the SSA summary (sections
- * "방법론" and "기술 상세": K_hybrid / V_hybrid are the gist KV together with
- * the raw KV of the selected chunks, attended with standard attention): each
- * sparse unit's query heads attend, in one softmax, over the raw tokens of
- * its selected chunks and over the gist token of EVERY chunk of the unit
- * (reading: the gist tokens stay in the context, as the summary's glossary
- * entry "Selective Unfolding" describes; the raw tokens of the selected
- * chunks come next to them).  Full-attention KV heads (head_full) attend
- * over their raw tokens only.
- *   Kg, Vg [B, Hkv, C, D] bf16, C = T / L: gist key / value of chunk c of
- *   unit (b, h) at row c (the model's gist KV; the synthetic workloads use the
- *   chunk means as a stand-in).  Same scale for gist and raw logits.
+ * The merged decode over the hybrid context of the SSA summary: each sparse
+ * unit's query heads attend, in one softmax and with the same scale for gist
+ * and raw logits, over the raw tokens of its selected chunks and over gist
+ * rows, as `gist_scope` says:
+ *   CSA_GIST_SELECTED: the gist rows of the selected chunks only (SSA
+ *     summary, sections "방법론" and "기술 상세": only the top-k chunks are
+ *     brought back, each with its gist KV and its raw KV; K_hybrid / V_hybrid
+ *     are the union of the gist and raw KV of I_t).
+ *   CSA_GIST_ALL: the gist row of every chunk of the unit (the glossary entry
+ *     "Selective Unfolding" read as the context: the query meets every
+ *     chunk's gist token and the raw tokens of the top-k chunks are added).
+ * Full-attention KV heads (head_full) attend over their raw tokens only.  A
+ * sparse unit with no selected chunk gets out = 0, lse = -inf in the
+ * selected scope (an empty context), and its gist rows alone in the other.
+ *   Kg, Vg [B, Hkv, C, D] bf16, C = T / L, 16-byte aligned: gist key / value
+ *   of chunk c of unit (b, h) at row c (the model's gist KV; a synthetic
+ *   workload draws them or uses the chunk means as a stand-in).
  *   Other arguments, outputs, workspace and errors as
  *   csa_sparse_decode_merged; bf16 caches only (CSA_ERR_UNSUPPORTED for
- *   fp32).  The gist rows stream as ceil(C/L) extra chunks of each sparse
- *   unit (K and V: 2*C*D*2 bytes per unit). */
+ *   fp32); CSA_ERR_INVALID_ARG for a gist_scope outside the enum.  The gist
+ *   rows are read as extra chunks of each sparse unit: ceil(C/L) chunks of
+ *   contiguous rows (scope ALL, by TMA), or ceil(n/L) chunks of the n
+ *   selected chunks' rows gathered with 16-byte copies (scope SELECTED); K
+ *   and V: 2*D*2 bytes per gist row. */
+typedef enum csa_gist_scope {
+  CSA_GIST_SELECTED = 0,
+  CSA_GIST_ALL = 1
+} csa_gist_scope;
+
 CSA_API csa_status csa_sparse_decode_merged_hybrid(const void* q, const void* K, const void* V,
                                                    const void* Kg, const void* Vg,
-                                                   csa_dtype dtype, const int32_t* idx,
-                                                   const int32_t* count, int kmax,
-                                                   const uint8_t* head_full, int B, int Hq,
-                                                   int Hkv, int D, int64_t T, int L, float scale,
-                                                   int num_parts, void* workspace,
+                                                   int gist_scope, csa_dtype dtype,
+                                                   const int32_t* idx, const int32_t* count,
+                                                   int kmax, const uint8_t* head_full, int B,
+                                                   int Hq, int Hkv, int D, int64_t T, int L,
+                                                   float scale, int num_parts, void* workspace,
                                                    int64_t workspace_bytes, void* out,
                                                    csa_dtype out_dtype, float* lse_out,
                                                    csa_stream stream);
@@ -464,9 +534,11 @@ typedef struct csa_decode_step_desc {
   csa_dtype out_dtype;
   float* lse_out;        /* NULL or [B, Hq] (output) */
   /* hybrid context (as csa_sparse_decode_merged_hybrid): NULL, NULL = off,
-   * else both [B, Hkv, T/L, D] bf16 gist keys and values */
+   * else both [B, Hkv, T/L, D] bf16 gist keys and values, over the gist rows
+   * of gist_scope (csa_gist_scope; 0 = CSA_GIST_SELECTED) */
   const void* Kg;
   const void* Vg;
+  int gist_scope;
   /* RoPE-aware split (see csa_rope): NULL = score with q; else the pre-RoPE
    * query [B, Hq, D] bf16 the selection scores with (against summaries of
    * the pre-RoPE keys), while the decode attends with q (rotated) over the
@@ -494,9 +566,8 @@ CSA_API csa_status csa_decode_step(const csa_decode_step_desc* d, csa_stream str
  * read, until the stream has passed the call.  The call captures into a CUDA graph, whose replays read and
  * write the same host buffers.  CSA_ERR_UNSUPPORTED with q_score set (the
  * RoPE-aware split rotates the query on the device: csa_rope, then
- * csa_decode_step).  Once the decode's own arguments have passed their
- * checks the query copy is enqueued, so a selection argument rejected
- * after that leaves the copy enqueued (it writes only d->q). */
+ * csa_decode_step).  Every argument, the selection's included, is checked
+ * before the query copy: a rejected call enqueues nothing. */
 CSA_API csa_status csa_decode_step_host(const csa_decode_step_desc* d, const void* q_host,
                                         void* out_host, float* lse_host, csa_stream stream);
 

@@ -53,9 +53,16 @@ _SIGS = {
     "csa_token_sparse_workspace_bytes": (_i64, [_i, _i, _i, _i, _i, _i]),
     "csa_token_sparse_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _i64,
                                       _vp, _vp, _vp]),
+    "csa_token_select": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "csa_token_compress": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "csa_token_attend_scratch_bytes": (_i64, [_i, _i, _i]),
+    "csa_token_attend": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i64, _vp, _vp]),
+    "csa_token_decompress_scratch_bytes": (_i64, [_i, _i, _i]),
+    "csa_token_decompress": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i64, _vp, _vp]),
     "csa_score_chunks": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
                               _vp]),
     "csa_select_topk": (_i, [_vp, _i, _i, _vp, _i, _i, _i, _vp, _vp, _i, _vp]),
+    "csa_select_topk_causal": (_i, [_vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _i, _vp]),
     "csa_select_topp": (_i, [_vp, _i, _i, _f, _f, _i, _i, _i, _vp, _vp, _i, _vp, _vp]),
     "csa_select_hier": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
                              _i, _vp]),
@@ -71,9 +78,9 @@ _SIGS = {
     "csa_decode_workspace_bytes": (_i64, [_i, _i, _i, _i, _i]),
     "csa_sparse_decode_merged": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i64,
                                       _i, _f, _i, _vp, _i64, _vp, _i, _vp, _vp]),
-    "csa_sparse_decode_merged_hybrid": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i,
-                                             _i, _i, _i, _i64, _i, _f, _i, _vp, _i64, _vp, _i,
-                                             _vp, _vp]),
+    "csa_sparse_decode_merged_hybrid": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _i, _vp,
+                                             _i, _i, _i, _i, _i64, _i, _f, _i, _vp, _i64, _vp,
+                                             _i, _vp, _vp]),
     "csa_sparse_decode_merged_noalloc": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _i, _i, _i,
                                               _i64, _i, _f, _i, _vp, _i, _vp, _vp]),
     "csa_lse_merge": (_i, [_vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp]),
@@ -170,6 +177,12 @@ def csa_select_topk(scores, U, C, n_valid, k_free, n_sink, n_local, idx, count, 
                                _p(count), kmax, _s(stream)))
 
 
+def csa_select_topk_causal(scores, U, C, n_tiles, tile_m, L, k_free, n_sink, n_local, idx, count,
+                           kmax, stream=None):
+    _check(lib.csa_select_topk_causal(_p(scores), U, C, n_tiles, tile_m, L, k_free, n_sink,
+                                      n_local, _p(idx), _p(count), kmax, _s(stream)))
+
+
 def csa_select_topp(scores, U, C, logit_scale, p, budget, n_sink, n_local, idx, count, kmax,
                     n_p_out=None, stream=None):
     _check(lib.csa_select_topp(_p(scores), U, C, logit_scale, p, budget, n_sink, n_local, _p(idx),
@@ -258,6 +271,35 @@ def csa_token_sparse_prefill(Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale, works
                                         _s(stream)))
 
 
+def csa_token_select(imp, B, S, Hkv, k_unit, idx, count, stream=None):
+    _check(lib.csa_token_select(_p(imp), B, S, Hkv, _p(k_unit), _p(idx), _p(count), _s(stream)))
+
+
+def csa_token_compress(Q, K, V, idx, count, B, S, Hq, Hkv, D, Qc, Kc, Vc, stream=None):
+    _check(lib.csa_token_compress(_p(Q), _p(K), _p(V), _p(idx), _p(count), B, S, Hq, Hkv, D,
+                                  _p(Qc), _p(Kc), _p(Vc), _s(stream)))
+
+
+def csa_token_attend_scratch_bytes(B, S, Hkv) -> int:
+    return int(lib.csa_token_attend_scratch_bytes(B, S, Hkv))
+
+
+def csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, scratch, scratch_bytes, Oc,
+                     stream=None):
+    _check(lib.csa_token_attend(_p(Qc), _p(Kc), _p(Vc), _p(k_unit), B, S, Hq, Hkv, D, scale,
+                                _p(scratch), scratch_bytes, _p(Oc), _s(stream)))
+
+
+def csa_token_decompress_scratch_bytes(B, S, Hkv) -> int:
+    return int(lib.csa_token_decompress_scratch_bytes(B, S, Hkv))
+
+
+def csa_token_decompress(Oc, idx, count, B, S, Hq, Hkv, D, scratch, scratch_bytes, O,
+                         stream=None):
+    _check(lib.csa_token_decompress(_p(Oc), _p(idx), _p(count), B, S, Hq, Hkv, D, _p(scratch),
+                                    scratch_bytes, _p(O), _s(stream)))
+
+
 def csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts) -> int:
     n = lib.csa_decode_workspace_bytes(B, Hq, Hkv, D, num_parts)
     if n < 0:
@@ -274,12 +316,24 @@ def csa_sparse_decode_merged(q, K, V, dtype, idx, count, kmax, head_full, B, Hq,
                                         _p(lse_out), _s(stream)))
 
 
-def csa_sparse_decode_merged_hybrid(q, K, V, Kg, Vg, dtype, idx, count, kmax, head_full, B, Hq,
-                                    Hkv, D, T, L, scale, num_parts, workspace, workspace_bytes,
-                                    out, out_dtype, lse_out, stream=None):
-    """The merged decode over the hybrid context: gist K/V rows [B, Hkv, T/L, D]
-    of every chunk plus the raw KV of the selected chunks (see include/csa.h)."""
-    _check(lib.csa_sparse_decode_merged_hybrid(_p(q), _p(K), _p(V), _p(Kg), _p(Vg), _dt(dtype),
+CSA_GIST_SELECTED, CSA_GIST_ALL = 0, 1
+
+
+def _scope(gist_scope) -> int:
+    if isinstance(gist_scope, str):
+        return {"selected": CSA_GIST_SELECTED, "all": CSA_GIST_ALL}[gist_scope]
+    return int(gist_scope)
+
+
+def csa_sparse_decode_merged_hybrid(q, K, V, Kg, Vg, gist_scope, dtype, idx, count, kmax,
+                                    head_full, B, Hq, Hkv, D, T, L, scale, num_parts, workspace,
+                                    workspace_bytes, out, out_dtype, lse_out, stream=None):
+    """The merged decode over the hybrid context: the raw KV of the selected
+    chunks plus gist K/V rows (Kg, Vg [B, Hkv, T/L, D]) of the selected chunks
+    (gist_scope "selected" / CSA_GIST_SELECTED) or of every chunk ("all" /
+    CSA_GIST_ALL); see include/csa.h."""
+    _check(lib.csa_sparse_decode_merged_hybrid(_p(q), _p(K), _p(V), _p(Kg), _p(Vg),
+                                               _scope(gist_scope), _dt(dtype),
                                                _p(idx), _p(count), kmax, _p(head_full), B, Hq,
                                                Hkv, D, T, L, scale, num_parts, _p(workspace),
                                                workspace_bytes, _p(out), _dt(out_dtype),
@@ -312,7 +366,7 @@ class DecodeStepDesc(ctypes.Structure):
         ("idx", _vp), ("count", _vp), ("kmax", _i), ("n_p_out", _vp),
         ("num_parts", _i), ("workspace", _vp), ("workspace_bytes", _i64),
         ("out", _vp), ("out_dtype", _i), ("lse_out", _vp),
-        ("Kg", _vp), ("Vg", _vp), ("q_score", _vp),
+        ("Kg", _vp), ("Vg", _vp), ("gist_scope", _i), ("q_score", _vp),
     ]
 
 
@@ -322,6 +376,8 @@ def decode_step_desc(**kw) -> DecodeStepDesc:
     for k, v in kw.items():
         if k == "out_dtype":
             v = _dt(v)
+        elif k == "gist_scope":
+            v = _scope(v)
         elif isinstance(v, torch.Tensor) or (v is None and k not in ("scale", "p")):
             v = None if v is None else v.data_ptr()
         setattr(d, k, v)

@@ -284,6 +284,28 @@ csa_status csa_select_topk(const float* scores, int U, int C, const int32_t* n_v
                 "select_topk launch");
 }
 
+csa_status csa_select_topk_causal(const float* scores, int U, int C, int n_tiles, int tile_m,
+                                  int L, int k_free, int n_sink, int n_local, int32_t* idx,
+                                  int32_t* count, int kmax, csa_stream stream) {
+  CSA_REQUIRE(kmax > 0, "kmax must be positive");
+  CSA_REQUIRE(U >= 0 && C >= 0 && k_free >= 0 && n_sink >= 0 && n_local >= 0,
+              "U, C, k_free, n_sink and n_local must be non-negative");
+  CSA_REQUIRE(n_tiles > 0 && tile_m > 0 && L > 0, "n_tiles, tile_m and L must be positive");
+  CSA_REQUIRE(U % n_tiles == 0, "U must be a multiple of n_tiles");
+  CSA_SUPPORT(C <= 32768, "C must be <= 32768");
+  const int64_t need = std::min<int64_t>(C, static_cast<int64_t>(k_free) + n_sink + n_local);
+  CSA_REQUIRE(kmax >= need, "kmax < min(C, k_free + n_sink + n_local)");
+  if (U == 0) return CSA_OK;
+  CSA_TRY(check_ptr(scores, "scores", C > 0));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_select_topk(l, scores, U, C, nullptr, k_free, n_sink, n_local, idx,
+                                        count, kmax, nullptr, n_tiles, tile_m, L),
+                "select_topk_causal launch");
+}
+
 csa_status csa_select_topp(const float* scores, int U, int C, float logit_scale, float p, int budget,
                            int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
                            int32_t* n_p_out, csa_stream stream) {
@@ -307,10 +329,16 @@ csa_status csa_select_topp(const float* scores, int U, int C, float logit_scale,
                 "select_topp launch");
 }
 
-csa_status csa_select_hier(const void* q, csa_dtype q_dtype, const float* meta, const float* summ,
-                           int B, int Hq, int Hkv, int D, int C, int Gm, int top_meta, int k_free,
-                           int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
-                           csa_stream stream) {
+}  // extern "C"
+
+namespace {
+// The selection calls with `check_only`: every argument check, then return
+// before anything is enqueued (used by the one-call step to reject a bad
+// selection argument before its query copy).
+csa_status select_hier_impl(const void* q, csa_dtype q_dtype, const float* meta,
+                            const float* summ, int B, int Hq, int Hkv, int D, int C, int Gm,
+                            int top_meta, int k_free, int n_sink, int n_local, int32_t* idx,
+                            int32_t* count, int kmax, csa_stream stream, bool check_only) {
   CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
   CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && C > 0 && Gm > 0 && top_meta >= 0 && k_free >= 0 &&
                   n_sink >= 0 && n_local >= 0 && kmax > 0,
@@ -330,9 +358,21 @@ csa_status csa_select_hier(const void* q, csa_dtype q_dtype, const float* meta, 
   CSA_TRY(check_ptr(count, "count"));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
+  if (check_only) return CSA_OK;
   return finish(csa::launch_select_hier(l, q, q_dtype == CSA_BF16, meta, summ, B, Hq, Hkv, D, C, Gm,
                                         top_meta, k_free, n_sink, n_local, idx, count, kmax),
                 "select_hier launch");
+}
+}  // namespace
+
+extern "C" {
+
+csa_status csa_select_hier(const void* q, csa_dtype q_dtype, const float* meta, const float* summ,
+                           int B, int Hq, int Hkv, int D, int C, int Gm, int top_meta, int k_free,
+                           int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                           csa_stream stream) {
+  return select_hier_impl(q, q_dtype, meta, summ, B, Hq, Hkv, D, C, Gm, top_meta, k_free, n_sink,
+                          n_local, idx, count, kmax, stream, false);
 }
 
 csa_status csa_selftest_wait_timeout(uint64_t limit_ns, csa_stream stream) {
@@ -446,7 +486,7 @@ int64_t csa_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int num_parts)
 namespace {
 // csa_sparse_decode_merged, with the hybrid context when Kg/Vg are given.
 csa_status merged_decode(const void* q, const void* K, const void* V, const void* Kg,
-                         const void* Vg, csa_dtype dtype, const int32_t* idx,
+                         const void* Vg, int gist_scope, csa_dtype dtype, const int32_t* idx,
                          const int32_t* count, int kmax, const uint8_t* head_full, int B, int Hq,
                          int Hkv, int D, int64_t T, int L, float scale, int num_parts,
                          void* workspace, int64_t workspace_bytes, void* out,
@@ -454,7 +494,11 @@ csa_status merged_decode(const void* q, const void* K, const void* V, const void
   CSA_REQUIRE(valid_dtype(out_dtype), "out_dtype");
   CSA_TRY(decode_shape_checks(dtype, kmax, B, Hq, Hkv, D, T, L, scale, num_parts));
   CSA_SUPPORT(num_parts <= csa::kMergedMaxParts, "num_parts must be <= 256 for the merged decode");
-  if (hybrid) CSA_SUPPORT(dtype == CSA_BF16, "the hybrid context needs a bf16 cache");
+  if (hybrid) {
+    CSA_SUPPORT(dtype == CSA_BF16, "the hybrid context needs a bf16 cache");
+    CSA_REQUIRE(gist_scope == CSA_GIST_SELECTED || gist_scope == CSA_GIST_ALL,
+                "gist_scope must be CSA_GIST_SELECTED or CSA_GIST_ALL");
+  }
   if (B == 0) return CSA_OK;
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
@@ -476,6 +520,7 @@ csa_status merged_decode(const void* q, const void* K, const void* V, const void
   if (hybrid) {
     m.Kg = Kg;
     m.Vg = Vg;
+    m.gist_selected = gist_scope == CSA_GIST_SELECTED;
   }
   std::string why;
   cudaError_t e = csa::launch_decode(l, q, K, V, dtype == CSA_BF16, idx, count, kmax, head_full, B, Hq,
@@ -494,20 +539,21 @@ csa_status csa_sparse_decode_merged(const void* q, const void* K, const void* V,
                                     int64_t T, int L, float scale, int num_parts, void* workspace,
                                     int64_t workspace_bytes, void* out, csa_dtype out_dtype,
                                     float* lse_out, csa_stream stream) {
-  return merged_decode(q, K, V, nullptr, nullptr, dtype, idx, count, kmax, head_full, B, Hq, Hkv,
+  return merged_decode(q, K, V, nullptr, nullptr, 0, dtype, idx, count, kmax, head_full, B, Hq, Hkv,
                        D, T, L, scale, num_parts, workspace, workspace_bytes, out, out_dtype,
                        lse_out, stream, false);
 }
 
 csa_status csa_sparse_decode_merged_hybrid(const void* q, const void* K, const void* V,
-                                           const void* Kg, const void* Vg, csa_dtype dtype,
-                                           const int32_t* idx, const int32_t* count, int kmax,
+                                           const void* Kg, const void* Vg, int gist_scope,
+                                           csa_dtype dtype, const int32_t* idx,
+                                           const int32_t* count, int kmax,
                                            const uint8_t* head_full, int B, int Hq, int Hkv,
                                            int D, int64_t T, int L, float scale, int num_parts,
                                            void* workspace, int64_t workspace_bytes, void* out,
                                            csa_dtype out_dtype, float* lse_out,
                                            csa_stream stream) {
-  return merged_decode(q, K, V, Kg, Vg, dtype, idx, count, kmax, head_full, B, Hq, Hkv, D, T, L,
+  return merged_decode(q, K, V, Kg, Vg, gist_scope, dtype, idx, count, kmax, head_full, B, Hq, Hkv, D, T, L,
                        scale, num_parts, workspace, workspace_bytes, out, out_dtype, lse_out,
                        stream, true);
 }
@@ -517,7 +563,7 @@ csa_status score_select_topk_common(const void* q, csa_dtype q_dtype, const floa
                                     const float* summ, int B, int Hq, int Hkv, int D, int C,
                                     const uint8_t* head_full, int k_free, int n_sink, int n_local,
                                     int32_t* idx, int32_t* count, int kmax, csa_stream stream,
-                                    bool per_head_union) {
+                                    bool per_head_union, bool check_only = false) {
   CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
   CSA_REQUIRE(kmax > 0, "kmax must be positive");
   CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && D > 0 && C >= 0 && k_free >= 0 && n_sink >= 0 &&
@@ -544,6 +590,7 @@ csa_status score_select_topk_common(const void* q, csa_dtype q_dtype, const floa
   CSA_TRY(check_ptr(count, "count"));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
+  if (check_only) return CSA_OK;
   return finish(csa::launch_score_select_topk(l, q, q_dtype == CSA_BF16, proj, R, summ, B, Hq, Hkv, D,
                                               C, head_full, k_free, n_sink, n_local, idx, count, kmax,
                                               per_head_union),
@@ -568,11 +615,14 @@ csa_status csa_score_select_topk_union(const void* q, csa_dtype q_dtype, const f
                                   n_sink, n_local, idx, count, kmax, stream, true);
 }
 
-csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* proj, int R,
-                                 const float* summ, int B, int Hq, int Hkv, int D, int C,
-                                 const uint8_t* head_full, float logit_scale, float p, int budget,
-                                 int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
-                                 int32_t* n_p_out, csa_stream stream) {
+}  // extern "C"
+
+namespace {
+csa_status score_select_topp_impl(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                  const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                  const uint8_t* head_full, float logit_scale, float p, int budget,
+                                  int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                                  int32_t* n_p_out, csa_stream stream, bool check_only) {
   CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
   CSA_REQUIRE(kmax > 0, "kmax must be positive");
   CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && D > 0 && C > 0 && n_sink >= 0 && n_local >= 0,
@@ -596,10 +646,24 @@ csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* 
   CSA_TRY(check_ptr(n_p_out, "n_p_out", false));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
+  if (check_only) return CSA_OK;
   return finish(csa::launch_score_select_topp(l, q, q_dtype == CSA_BF16, proj, R, summ, B, Hq, Hkv, D,
                                               C, head_full, logit_scale, p, budget, n_sink, n_local,
                                               idx, count, kmax, n_p_out),
                 "score_select_topp launch");
+}
+}  // namespace
+
+extern "C" {
+
+csa_status csa_score_select_topp(const void* q, csa_dtype q_dtype, const float* proj, int R,
+                                 const float* summ, int B, int Hq, int Hkv, int D, int C,
+                                 const uint8_t* head_full, float logit_scale, float p, int budget,
+                                 int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
+                                 int32_t* n_p_out, csa_stream stream) {
+  return score_select_topp_impl(q, q_dtype, proj, R, summ, B, Hq, Hkv, D, C, head_full,
+                                logit_scale, p, budget, n_sink, n_local, idx, count, kmax, n_p_out,
+                                stream, false);
 }
 
 }  // extern "C"
@@ -683,11 +747,30 @@ csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stre
   if (hybrid) {  // both or neither
     CSA_TRY(check_ptr(d->Kg, "Kg"));
     CSA_TRY(check_ptr(d->Vg, "Vg"));
+    CSA_REQUIRE(d->gist_scope == CSA_GIST_SELECTED || d->gist_scope == CSA_GIST_ALL,
+                "gist_scope must be CSA_GIST_SELECTED or CSA_GIST_ALL");
   }
   const int C = static_cast<int>(d->T / d->L);
   // the selection scores with the pre-RoPE query when one is given
   const void* qs = d->q_score != nullptr ? d->q_score : d->q;
   if (d->q_score != nullptr) CSA_TRY(check_ptr(d->q_score, "q_score"));
+  auto selection = [&](bool check_only) -> csa_status {
+    if (d->mode == CSA_SELECT_TOPK || d->mode == CSA_SELECT_TOPK_UNION)
+      return score_select_topk_common(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
+                                      d->D, C, d->head_full, d->k_free, d->n_sink, d->n_local,
+                                      d->idx, d->count, d->kmax, stream,
+                                      d->mode == CSA_SELECT_TOPK_UNION, check_only);
+    if (d->mode == CSA_SELECT_TOPP)
+      return score_select_topp_impl(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
+                                    d->D, C, d->head_full, d->logit_scale, d->p, d->budget,
+                                    d->n_sink, d->n_local, d->idx, d->count, d->kmax, d->n_p_out,
+                                    stream, check_only);
+    return select_hier_impl(qs, CSA_BF16, d->meta, d->summ, d->B, d->Hq, d->Hkv, d->D, C, d->Gm,
+                            d->top_meta, d->k_free, d->n_sink, d->n_local, d->idx, d->count,
+                            d->kmax, stream, check_only);
+  };
+  // every argument of the selection too, before the query copy is enqueued
+  CSA_TRY(selection(true));
   if (io != nullptr && io->q != nullptr) {
     const size_t nq = static_cast<size_t>(d->B) * d->Hq * d->D * sizeof(__nv_bfloat16);
     if (io->q_mapped)
@@ -698,24 +781,7 @@ csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stre
                                      l.stream),
                      "query copy to the device"));
   }
-  // the selection (validates its own arguments before launching)
-  csa_status st;
-  if (d->mode == CSA_SELECT_TOPK)
-    st = csa_score_select_topk(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
-                               d->head_full, d->k_free, d->n_sink, d->n_local, d->idx, d->count,
-                               d->kmax, stream);
-  else if (d->mode == CSA_SELECT_TOPK_UNION)
-    st = csa_score_select_topk_union(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
-                                     d->D, C, d->head_full, d->k_free, d->n_sink, d->n_local,
-                                     d->idx, d->count, d->kmax, stream);
-  else if (d->mode == CSA_SELECT_TOPP)
-    st = csa_score_select_topp(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv, d->D, C,
-                               d->head_full, d->logit_scale, d->p, d->budget, d->n_sink, d->n_local,
-                               d->idx, d->count, d->kmax, d->n_p_out, stream);
-  else
-    st = csa_select_hier(qs, CSA_BF16, d->meta, d->summ, d->B, d->Hq, d->Hkv, d->D, C, d->Gm,
-                         d->top_meta, d->k_free, d->n_sink, d->n_local, d->idx, d->count, d->kmax,
-                         stream);
+  const csa_status st = selection(false);
   if (st != CSA_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(d->workspace);
   csa::MergeOut m{reinterpret_cast<int*>(ws + w.counters), d->out, d->out_dtype == CSA_BF16,
@@ -723,6 +789,7 @@ csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stre
   if (hybrid) {
     m.Kg = d->Kg;
     m.Vg = d->Vg;
+    m.gist_selected = d->gist_scope == CSA_GIST_SELECTED;
   }
   std::string why;
   cudaError_t e = csa::launch_decode(l, d->q, d->K, d->V, true, d->idx, d->count, d->kmax,
@@ -950,36 +1017,136 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
   if (e == cudaSuccess)  // each KV head's own top tokens under the (rounded) budget
     e = csa::launch_select_topk(l, imp, U, S, nullptr, 0, 0, 0, idx, cnt, S, k_unit);
   if (e != cudaSuccess) return finish(e, "token selection launch");
-  // The compressed length sizes the dense attention: read back the budgets.
-  std::vector<int32_t> ku(U);
-  e = cudaMemcpyAsync(ku.data(), k_unit, U * sizeof(int32_t), cudaMemcpyDeviceToHost, l.stream);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(l.stream);
-  if (e != cudaSuccess) return finish(e, "token budget read-back");
-  int Sc = 0;
-  for (int v : ku) Sc = std::max(Sc, v);
-  if (Sc <= 0 || Sc > S || Sc % 64 != 0) {
-    if (Sc != 0) return fail(CSA_ERR_CUDA, "token budget out of range");
-  }
+  // Compress, attend, decompress with no read-back of the budgets: the
+  // buffers are laid out for S kept tokens, the gather writes the kept rows
+  // of each unit only, the causal lists give the tiles past a unit's budget
+  // no chunk, and the dense attention skips those tiles without writing.
   void* Qc = ws + w.qc;
   void* Kc = ws + w.kc;
   void* Vc = ws + w.vc;
   void* Oc = ws + w.oc;
-  if (Sc > 0) {
-    e = csa::launch_tsa_gather(l, Q, K, V, idx, cnt, S, B, S, Sc, Hq, Hkv, D, Qc, Kc, Vc);
-    const int T = Sc / 64;
-    int32_t* lists = reinterpret_cast<int32_t*>(ws + w.lists);
-    int32_t* counts2 = reinterpret_cast<int32_t*>(ws + w.counts2);
-    if (e == cudaSuccess) e = csa::launch_tsa_lists(l, k_unit, U, T, 64, lists, counts2);
-    std::string why;
-    if (e == cudaSuccess)
-      e = csa::launch_prefill(l, Qc, Kc, Vc, lists, counts2, T, B, Sc, Hq, Hkv, D, 64, 64, scale,
-                              Oc, &why);
-    if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
-  }
+  const int T = S / 64;
+  int32_t* lists = reinterpret_cast<int32_t*>(ws + w.lists);
+  int32_t* counts2 = reinterpret_cast<int32_t*>(ws + w.counts2);
+  e = csa::launch_tsa_gather(l, Q, K, V, idx, cnt, S, B, S, S, Hq, Hkv, D, Qc, Kc, Vc);
+  if (e == cudaSuccess) e = csa::launch_tsa_lists(l, k_unit, U, T, 64, lists, counts2);
+  std::string why;
   if (e == cudaSuccess)
-    e = csa::launch_tsa_scatter(l, Oc, idx, cnt, S, B, S, Sc, Hq, Hkv, D,
+    e = csa::launch_prefill(l, Qc, Kc, Vc, lists, counts2, T, B, S, Hq, Hkv, D, 64, 64, scale, Oc,
+                            &why, /*skip_empty=*/true);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  if (e == cudaSuccess)
+    e = csa::launch_tsa_scatter(l, Oc, idx, cnt, S, B, S, S, Hq, Hkv, D,
                                 reinterpret_cast<int32_t*>(ws + w.inv), O);
   return finish(e, "token sparse prefill launch");
+}
+
+
+/* ---- the steps of csa_token_sparse_prefill as separate calls ---- */
+
+namespace {
+csa_status token_shape_checks(int B, int S, int Hq, int Hkv, int D) {
+  CSA_REQUIRE(B >= 0 && S >= 0 && Hq > 0 && Hkv > 0 && D > 0, "bad sizes");
+  CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
+  CSA_REQUIRE(S % 64 == 0, "S must be a multiple of 64");
+  CSA_SUPPORT(D == 128 && Hq / Hkv == 4 && S <= 32768,
+              "implemented for D = 128, Hq/Hkv = 4 and S <= 32768");
+  return CSA_OK;
+}
+}  // namespace
+
+csa_status csa_token_select(const float* imp, int B, int S, int Hkv, const int32_t* k_unit,
+                            int32_t* idx, int32_t* count, csa_stream stream) {
+  CSA_REQUIRE(B >= 0 && S >= 0 && Hkv > 0, "bad sizes");
+  CSA_SUPPORT(S <= 32768, "S must be <= 32768");
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  CSA_TRY(check_ptr(imp, "imp"));
+  CSA_TRY(check_ptr(k_unit, "k_unit"));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_select_topk(l, imp, B * Hkv, S, nullptr, 0, 0, 0, idx, count, S,
+                                        k_unit),
+                "token select launch");
+}
+
+csa_status csa_token_compress(const void* Q, const void* K, const void* V, const int32_t* idx,
+                              const int32_t* count, int B, int S, int Hq, int Hkv, int D,
+                              void* Qc, void* Kc, void* Vc, csa_stream stream) {
+  CSA_TRY(token_shape_checks(B, S, Hq, Hkv, D));
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  CSA_TRY(check_ptr(Q, "Q"));
+  CSA_TRY(check_ptr(K, "K"));
+  CSA_TRY(check_ptr(V, "V"));
+  CSA_TRY(check_ptr(Qc, "Qc"));
+  CSA_TRY(check_ptr(Kc, "Kc"));
+  CSA_TRY(check_ptr(Vc, "Vc"));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_tsa_gather(l, Q, K, V, idx, count, S, B, S, S, Hq, Hkv, D, Qc, Kc, Vc),
+                "token compress launch");
+}
+
+int64_t csa_token_attend_scratch_bytes(int B, int S, int Hkv) {
+  if (B < 0 || S < 0 || Hkv <= 0 || S % 64 != 0) return -1;
+  const int64_t U = static_cast<int64_t>(B) * Hkv, T = S / 64;
+  return (U * T * T + U * T) * 4;
+}
+
+csa_status csa_token_attend(const void* Qc, const void* Kc, const void* Vc,
+                            const int32_t* k_unit, int B, int S, int Hq, int Hkv, int D,
+                            float scale, void* scratch, int64_t scratch_bytes, void* Oc,
+                            csa_stream stream) {
+  CSA_TRY(token_shape_checks(B, S, Hq, Hkv, D));
+  CSA_REQUIRE(scale == scale && scale > 0.f, "scale must be positive");
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  CSA_REQUIRE(scratch_bytes >= csa_token_attend_scratch_bytes(B, S, Hkv),
+              "scratch smaller than csa_token_attend_scratch_bytes()");
+  CSA_TRY(check_ptr(Qc, "Qc"));
+  CSA_TRY(check_ptr(Kc, "Kc"));
+  CSA_TRY(check_ptr(Vc, "Vc"));
+  CSA_TRY(check_ptr(Oc, "Oc"));
+  CSA_TRY(check_ptr(k_unit, "k_unit"));
+  CSA_TRY(check_ptr(scratch, "scratch"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  const int U = B * Hkv, T = S / 64;
+  int32_t* lists = static_cast<int32_t*>(scratch);
+  int32_t* counts = lists + static_cast<int64_t>(U) * T * T;
+  cudaError_t e = csa::launch_tsa_lists(l, k_unit, U, T, 64, lists, counts);
+  std::string why;
+  if (e == cudaSuccess)
+    e = csa::launch_prefill(l, Qc, Kc, Vc, lists, counts, T, B, S, Hq, Hkv, D, 64, 64, scale, Oc,
+                            &why, /*skip_empty=*/true);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  return finish(e, "token attend launch");
+}
+
+int64_t csa_token_decompress_scratch_bytes(int B, int S, int Hkv) {
+  if (B < 0 || S < 0 || Hkv <= 0) return -1;
+  return static_cast<int64_t>(B) * Hkv * S * 4;
+}
+
+csa_status csa_token_decompress(const void* Oc, const int32_t* idx, const int32_t* count, int B,
+                                int S, int Hq, int Hkv, int D, void* scratch,
+                                int64_t scratch_bytes, void* O, csa_stream stream) {
+  CSA_TRY(token_shape_checks(B, S, Hq, Hkv, D));
+  if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
+  CSA_REQUIRE(scratch_bytes >= csa_token_decompress_scratch_bytes(B, S, Hkv),
+              "scratch smaller than csa_token_decompress_scratch_bytes()");
+  CSA_TRY(check_ptr(Oc, "Oc"));
+  CSA_TRY(check_ptr(idx, "idx"));
+  CSA_TRY(check_ptr(count, "count"));
+  CSA_TRY(check_ptr(scratch, "scratch"));
+  CSA_TRY(check_ptr(O, "O"));
+  csa::Launch l;
+  CSA_TRY(launch_ctx(stream, &l));
+  return finish(csa::launch_tsa_scatter(l, Oc, idx, count, S, B, S, S, Hq, Hkv, D,
+                                        static_cast<int32_t*>(scratch), O),
+                "token decompress launch");
 }
 
 }  // extern "C"

@@ -75,12 +75,20 @@ struct DecodeParams {
   // phased: the last `late` CTAs of the grid take no phase-1 work (they can
   // only start once the selection's CTAs have left their SMs)
   int late;
-  // hybrid context (bf16 merged): every sparse unit also attends over its
-  // gist rows, gist_rows (= C) per unit in [B*Hkv*gist_rows, D] bf16 tensors,
-  // streamed as n_gist = ceil(gist_rows / L) extra chunks after its selected
-  // ones (the last one ragged, its rows past gist_rows masked); 0 = off
+  // hybrid context (bf16 merged), over every chunk's gist row: every sparse
+  // unit also attends over its gist rows, gist_rows (= C) per unit in
+  // [B*Hkv*gist_rows, D] bf16 tensors, streamed as n_gist = ceil(gist_rows /
+  // L) extra chunks after its selected ones (the last one ragged, its rows
+  // past gist_rows masked); 0 = off
   int n_gist;
   int gist_rows;
+  // hybrid context over the selected chunks' own gist rows: each sparse unit
+  // with n selected chunks attends over their n gist rows (rows u*C + c of
+  // Kg/Vg), gathered by the producer warp with 16-byte cp.async copies into
+  // ceil(n / L) extra chunks after the selected ones; 0 = off
+  int gist_sel;
+  const __nv_bfloat16* Kg;
+  const __nv_bfloat16* Vg;
 };
 
 // Unit sets of a phase: 0 = every unit, 1 = full-head units, 2 = sparse units.
@@ -90,16 +98,31 @@ __device__ __forceinline__ bool unit_in(const DecodeParams& p, int u, int mode) 
   return mode == 1 ? full : !full;
 }
 
-__device__ __forceinline__ int unit_count(const DecodeParams& p, int u, int mode = 0) {
-  const bool full = p.head_full != nullptr && p.head_full[u % p.Hkv];
-  if (mode == 1) return full ? p.C : 0;
-  if (full) return mode == 2 ? 0 : p.C;
+// Selected chunks of sparse unit u (its count, clamped to [0, kmax]).
+__device__ __forceinline__ int sel_count(const DecodeParams& p, int u) {
   int n = p.count[u];
   if (n < 0 || n > p.kmax) {
     dev_flag(p.err, DEV_BAD_INDEX);
     n = max(0, min(n, p.kmax));
   }
-  return n + p.n_gist;  // a sparse unit's gist chunks come after its selected ones
+  return n;
+}
+
+// Gist chunks and gist rows of a hybrid sparse unit with n selected chunks
+// (both 0 without the hybrid context).
+__device__ __forceinline__ int gist_chunks(const DecodeParams& p, int n) {
+  return p.gist_sel ? (n + p.L - 1) / p.L : p.n_gist;
+}
+__device__ __forceinline__ int gist_rows_of(const DecodeParams& p, int n) {
+  return p.gist_sel ? n : p.gist_rows;
+}
+
+__device__ __forceinline__ int unit_count(const DecodeParams& p, int u, int mode = 0) {
+  const bool full = p.head_full != nullptr && p.head_full[u % p.Hkv];
+  if (mode == 1) return full ? p.C : 0;
+  if (full) return mode == 2 ? 0 : p.C;
+  const int n = sel_count(p, u);
+  return n + gist_chunks(p, n);  // a sparse unit's gist chunks come after its selected ones
 }
 
 __device__ __forceinline__ int unit_chunk(const DecodeParams& p, int u, int pos) {
@@ -112,16 +135,75 @@ __device__ __forceinline__ int unit_chunk(const DecodeParams& p, int u, int pos)
   return c;
 }
 
-// Row of the chunk at position pos of unit u (n = the unit's chunk count):
-// the raw K/V row of a selected (or, for a full unit, every) chunk, or for a
-// hybrid unit's gist chunk j the gist row, encoded as -(row + 1).
-__device__ __forceinline__ int unit_row(const DecodeParams& p, int u, int pos, int n, int L) {
-  if (p.n_gist > 0 && !(p.head_full != nullptr && p.head_full[u % p.Hkv])) {
-    const int j = pos - (n - p.n_gist);
-    if (j >= 0) return -(u * p.gist_rows + j * L) - 1;
+// Row of the chunk at position pos of unit u: the raw K/V row of a selected
+// (or, for a full unit, every) chunk, or for a hybrid unit's gist chunk j
+// the first gist row, encoded as -(row + 1).  In the selected-gist scope a
+// gist chunk has no contiguous rows: *gsel then gets the offset u*kmax + j*L
+// of its first chunk id in idx (else -1).
+__device__ __forceinline__ int unit_row(const DecodeParams& p, int u, int pos, int L, int* gsel) {
+  *gsel = -1;
+  if ((p.n_gist > 0 || p.gist_sel) && !(p.head_full != nullptr && p.head_full[u % p.Hkv])) {
+    const int j = pos - sel_count(p, u);
+    if (j >= 0) {
+      if (p.gist_sel) {
+        *gsel = u * p.kmax + j * L;
+        return 0;
+      }
+      return -(u * p.gist_rows + j * L) - 1;
+    }
   }
   const int c = unit_chunk(p, u, pos);
   return static_cast<int>(u * p.T + static_cast<int64_t>(c) * L);
+}
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// The arrive-on of `bar` waits for this thread's earlier cp.async copies (the
+// pending count goes up by one now and down by one when they land).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Selected-gist scope: the gist K and V rows of the chunk ids idx[off ..
+// off + L) of unit u = off / kmax (those below the unit's count; the rest of
+// the stage is zero-filled) into stage `dst`, laid out as the TMA boxes
+// ([L x 64] per 64 columns, 128-byte swizzle).  All 32 lanes of the calling
+// warp copy (lane r takes rows r, r + 32, ...) and arrive on `bar` through
+// cp.async.mbarrier.arrive; the caller then makes the barrier's own arrival.
+template <int D, int L>
+__device__ __forceinline__ void gather_gist_rows(const DecodeParams& p, int off, uint32_t dst,
+                                                 uint32_t bar) {
+  constexpr int KV_BYTES = L * D * 2, BOX_BYTES = L * 128, PIECES = D / 8;
+  const int lane = threadIdx.x & 31;
+  const int u = off / p.kmax, r0 = off - u * p.kmax;
+  const int n = sel_count(p, u);
+#pragma unroll 1
+  for (int r = lane; r < L; r += 32) {
+    const bool valid = r0 + r < n;
+    int c = valid ? p.idx[off + r] : 0;
+    if (c < 0 || c >= p.C) {
+      dev_flag(p.err, DEV_BAD_INDEX);
+      c = 0;
+    }
+    const int64_t row = static_cast<int64_t>(u) * p.C + c;
+    const __nv_bfloat16* ks = p.Kg + row * D;
+    const __nv_bfloat16* vs = p.Vg + row * D;
+    const uint32_t bytes = valid ? 16u : 0u;
+#pragma unroll
+    for (int pc = 0; pc < PIECES; ++pc) {
+      const uint32_t o = (pc >> 3) * BOX_BYTES + r * 128 + (((pc & 7) ^ (r & 7)) << 4);
+      cp_async_16(dst + o, ks + pc * 8, bytes);
+      cp_async_16(dst + KV_BYTES + o, vs + pc * 8, bytes);
+    }
+  }
+  cp_async_mbar_arrive(bar);
 }
 
 // prefix[0..U] of the effective chunk counts of a phase (all threads of the block).
@@ -471,6 +553,7 @@ __device__ void merge_bulk_issue(const DecodeParams& p, int u, int ns, const Mer
   float* st = reinterpret_cast<float*>(area);
   float* sl_rows = st + static_cast<size_t>(G) * ns * D;
   fence_proxy_async_global();  // read through the async proxy
+  fence_proxy_async_shared();  // the area may last have been written by cp.async
   mbar_arrive_expect_tx(bar, static_cast<uint32_t>(G) * (m.head_bytes + m.lse_bytes));
   for (int g = 0; g < G; ++g) {
     bulk_load(smem_u32(st + static_cast<size_t>(g) * ns * D),
@@ -701,6 +784,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // K/V is read once: first out of L2, so that what the kernel reads again
     // (its instructions, parameters, the partials and counters) stays there
     const uint64_t kv_policy = l2_policy_evict_first();
+    uint32_t cp_stages = 0;  // lane 0: stages last filled by cp.async (selected-gist chunks)
     int64_t issued = 0;
     bool ok = true;
     for (int ph = 0; ph < n_phase && ok; ++ph) {
@@ -716,31 +800,36 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       piece_range(N, phase_parts(ph), blockIdx.x, a, bnd);
       for (int64_t g0 = a; g0 < bnd && ok; g0 += 32) {
         const int64_t g = g0 + lane;
-        int row = 0, qu = -1;
+        int row = 0, qu = -1, gsel = -1;
         if (g < bnd) {
           const int u = unit_of(pre, p.U, g);
-          row = unit_row(p, u, static_cast<int>(g - pre[u]), pre[u + 1] - pre[u], L);
+          row = unit_row(p, u, static_cast<int>(g - pre[u]), L, &gsel);
           if (g == a || g == pre[u]) qu = u;  // first chunk of a unit here: its q rides along
         }
         const int nb = static_cast<int>(bnd - g0 < 32 ? bnd - g0 : 32);
         for (int j = 0; j < nb; ++j) {
           const int row_j = __shfl_sync(0xffffffffu, row, j);
           const int qu_j = __shfl_sync(0xffffffffu, qu, j);
+          const int gs_j = __shfl_sync(0xffffffffu, gsel, j);
+          const int64_t i = issued;
+          const int s = static_cast<int>(i % NS);
+          const uint32_t fb = full_bar + 8 * s;
+          const uint32_t dst = sbase + s * Sh::STAGE_BYTES;
           int good = 1;
           if (lane == 0) {
-            const int64_t i = issued;
-            const int s = static_cast<int>(i % NS);
             const uint32_t it = static_cast<uint32_t>(i / NS);
             if (!mbar_wait(empty_bar + 8 * s, (it & 1u) ^ 1u, p.err)) {
               good = 0;
-            } else {
-              const uint32_t fb = full_bar + 8 * s;
+            } else if (gs_j < 0) {
+              if (cp_stages & (1u << s)) {  // the copies that filled it last were cp.async
+                fence_proxy_async_shared();
+                cp_stages &= ~(1u << s);
+              }
               mbar_arrive_expect_tx(fb, Sh::STAGE_BYTES + (qu_j >= 0 ? q_bytes : 0u));
               if (qu_j >= 0) {
                 const int64_t qrow = static_cast<int64_t>(qu_j / p.Hkv) * p.Hq + (qu_j % p.Hkv) * G;
                 bulk_load(sbase + Y.q_off + s * Sh::QSLOT_BYTES, qg + qrow * D, q_bytes, fb);
               }
-              const uint32_t dst = sbase + s * Sh::STAGE_BYTES;
               const bool gist = row_j < 0;  // rows of a ragged last gist chunk past
               const int r = gist ? -row_j - 1 : row_j;  // the tensor read as zeros
               const CUtensorMap* mk = gist ? &tmKg : &tmK;
@@ -753,8 +842,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               }
             }
           }
-          issued = __shfl_sync(0xffffffffu, issued + good, 0);
           good = __shfl_sync(0xffffffffu, good, 0);
+          if (good && gs_j >= 0) {  // warp-uniform: a gathered gist chunk
+            gather_gist_rows<D, L>(p, gs_j, dst, fb);
+            __syncwarp();  // every lane's pending arrival before the barrier's own
+            if (lane == 0) {
+              cp_stages |= 1u << s;
+              if (qu_j >= 0) {
+                const int64_t qrow = static_cast<int64_t>(qu_j / p.Hkv) * p.Hq + (qu_j % p.Hkv) * G;
+                mbar_arrive_expect_tx(fb, q_bytes);
+                bulk_load(sbase + Y.q_off + s * Sh::QSLOT_BYTES, qg + qrow * D, q_bytes, fb);
+              } else {
+                mbar_arrive(fb);
+              }
+            }
+          }
+          issued = __shfl_sync(0xffffffffu, issued + good, 0);
           if (!good) {
             ok = false;
             break;
@@ -884,6 +987,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   int cur_u = -1, nflush = 0;
   bool cur_full = false;  // hybrid launches: the current unit is a full-attention one
+  int cur_ns = 0;         // hybrid launches: the current unit's selected chunks
+  const bool hybrid = p.n_gist > 0 || p.gist_sel;
   bool ok = true;
 
   // Hand this warp's (m, l, O) of unit u to the epilogue warp and go on.
@@ -957,7 +1062,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           break;
         }
         cur_u = unit_of(pre, p.U, g);
-        cur_full = p.n_gist > 0 && p.head_full != nullptr && p.head_full[cur_u % p.Hkv];
+        cur_full = hybrid && p.head_full != nullptr && p.head_full[cur_u % p.Hkv];
+        if (hybrid && !cur_full) cur_ns = sel_count(p, cur_u);
         // the unit's q arrived with this stage
         const __nv_bfloat16* qs =
             reinterpret_cast<const __nv_bfloat16*>(smem + Y.q_off + s * Sh::QSLOT_BYTES);
@@ -1000,12 +1106,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
         }
       }
-      if (p.n_gist > 0 && !cur_full) {
+      if (hybrid && !cur_full) {
         // a hybrid unit's last gist chunk is ragged: rows past its gist rows
-        // (the next unit's, or zeros past the tensor) take no part
-        const int n_all = pre[cur_u + 1] - pre[cur_u];
-        const int j = static_cast<int>(g - pre[cur_u]) - (n_all - p.n_gist);
-        const int valid = j >= 0 ? p.gist_rows - j * L : L;
+        // (the next unit's, zeros past the tensor, or the zero-filled rows of
+        // a gathered chunk) take no part
+        const int j = static_cast<int>(g - pre[cur_u]) - cur_ns;
+        const int valid = j >= 0 ? gist_rows_of(p, cur_ns) - j * L : L;
         if (valid < L) {
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt)
@@ -1362,8 +1468,14 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
     p.phased = (merge->phased && bf16) ? 1 : 0;
     p.late = p.phased ? merge->late : 0;
     if (merge->Kg != nullptr && bf16) {
-      p.gist_rows = static_cast<int>(T / L);
-      p.n_gist = (p.gist_rows + L - 1) / L;
+      if (merge->gist_selected) {
+        p.gist_sel = 1;
+        p.Kg = static_cast<const __nv_bfloat16*>(merge->Kg);
+        p.Vg = static_cast<const __nv_bfloat16*>(merge->Vg);
+      } else {
+        p.gist_rows = static_cast<int>(T / L);
+        p.n_gist = (p.gist_rows + L - 1) / L;
+      }
     }
   }
   p.D = D;

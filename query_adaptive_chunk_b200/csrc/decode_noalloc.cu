@@ -83,8 +83,11 @@ csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K, const 
   if (st != CSA_OK || B == 0) return st;
   // The area keeps whatever a call leaves behind.  Its arrival counters must
   // read zero when the next decode starts: the area is zero-initialised when
-  // the library loads, and every call clears the counters again after its
-  // decode (which also repairs them after a call that timed out).
+  // the library loads, a decode that completes leaves them zero, and every
+  // call also clears them after its decode, so that a call that ended early
+  // (a wait past its time limit, reported by csa_check_device_status) does
+  // not leave a count behind for the next one.  The clear is one memset node
+  // of B * Hkv counters on the stream (a few hundred bytes).
   const size_t counter_bytes = (static_cast<size_t>(B) * Hkv * 4 + 255) & ~size_t(255);
   cudaError_t e = cudaMemsetAsync(ws, 0, counter_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {

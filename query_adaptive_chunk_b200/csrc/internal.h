@@ -36,10 +36,14 @@ cudaError_t launch_score(const Launch& l, const void* q, bool bf16, const float*
                          float* scores);
 
 // select.cu
+// causal_tiles > 0: unit u is query tile u % causal_tiles of a causal
+// prefill and sees the chunks c < ((t + 1) * causal_tile_m - 1) / causal_L + 1
+// (n_valid is then ignored)
 cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax,
-                               const int32_t* k_dev = nullptr);
+                               const int32_t* k_dev = nullptr, int causal_tiles = 0,
+                               int causal_tile_m = 0, int causal_L = 0);
 cudaError_t launch_select_topp(const Launch& l, const float* scores, int U, int C,
                                float logit_scale, float p, int budget, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax, int32_t* n_p_out);
@@ -95,9 +99,12 @@ struct MergeOut {
   // start only after the selection's CTAs leave their SMs)
   int late = 0;
   // bf16 hybrid context: gist K/V rows [B, Hkv, C, D] (C = T / L) that every
-  // sparse unit attends over next to its selected chunks; null = off
+  // sparse unit attends over next to its selected chunks; null = off.
+  // gist_selected: only the gist rows of the unit's selected chunks, else
+  // every chunk's gist row
   const void* Kg = nullptr;
   const void* Vg = nullptr;
+  bool gist_selected = false;
 };
 constexpr int kMergedMaxParts = 256;
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,
@@ -113,10 +120,11 @@ cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_
 cudaError_t launch_copy16(const Launch& l, const void* src, void* dst, size_t bytes);
 
 // prefill.cu
+// skip_empty: units with no chunk write nothing (else their rows get 0)
 cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const void* V,
                            const int32_t* idx, const int32_t* count, int kmax, int B, int S,
                            int Hq, int Hkv, int D, int tile_m, int L, float scale, void* O,
-                           std::string* why);
+                           std::string* why, bool skip_empty = false);
 
 // tma_host.cu: 2-D bf16 tensor map over a row-major [rows, cols] matrix with
 // `row_stride` elements between rows, box [box_rows, box_cols], 128-byte swizzle.

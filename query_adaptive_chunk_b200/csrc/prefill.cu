@@ -132,6 +132,7 @@ struct PrefillParams {
   float scale_log2;
   __nv_bfloat16* O;
   DevErr err;
+  int skip_empty;  // units with no chunk write nothing (else their rows get 0)
 };
 
 __device__ __forceinline__ void unit_coords(const PrefillParams& p, int w, int& b, int& h, int& t) {
@@ -387,7 +388,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int qpos = t * 64 + i;
       __nv_bfloat16* orow = p.O + ((static_cast<int64_t>(b) * p.S + qpos) * p.Hq + h * 4 + g) * 128;
       if (n == 0) {
-        for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+        if (!p.skip_empty)
+          for (int c = 0; c < 128; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
       float m = -INFINITY, l = 0.f;  // running max of the raw scores, sum of 2^((s - m) sl)
@@ -542,7 +544,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const void* V,
                            const int32_t* idx, const int32_t* count, int kmax, int B, int S,
                            int Hq, int Hkv, int D, int tile_m, int L, float scale, void* O,
-                           std::string* why) {
+                           std::string* why, bool skip_empty) {
   (void)D;
   (void)tile_m;
   (void)L;
@@ -566,6 +568,7 @@ cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const 
   p.scale_log2 = scale * kLog2e;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.err = l.err;
+  p.skip_empty = skip_empty ? 1 : 0;
   const int n_units = B * Hkv * p.n_tiles;
   if (n_units == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -216,10 +216,16 @@ __device__ void topk_from_keys(const uint32_t* keys, uint8_t* flags, int v, int 
   emit_ascending(flags, v, row, cnt, kmax, s);
 }
 
+// Causal prefill units (causal_tiles > 0): unit u is query tile t = u mod
+// causal_tiles, which sees the chunks c < ((t + 1) * tile_m - 1) / L + 1.
+struct CausalRows {
+  int tiles, tile_m, L;
+};
+
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
     const float* __restrict__ scores, int C, const int32_t* __restrict__ n_valid, int k_free,
     int n_sink, int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax,
-    const int32_t* __restrict__ k_dev) {
+    const int32_t* __restrict__ k_dev, CausalRows causal) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
   __shared__ BucketScratch bs;
@@ -228,7 +234,12 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(
   uint32_t* keys = reinterpret_cast<uint32_t*>(sm + exch_bytes);
   uint8_t* flags = sm + exch_bytes + static_cast<size_t>(C) * 4;
   const int u = blockIdx.x;
-  const int v = n_valid ? max(0, min(C, n_valid[u])) : C;
+  int v = n_valid ? max(0, min(C, n_valid[u])) : C;
+  if (causal.tiles > 0) {
+    const int64_t t = u % causal.tiles;
+    const int64_t vis = ((t + 1) * causal.tile_m - 1) / causal.L + 1;
+    v = static_cast<int>(vis < C ? vis : C);
+  }
   const float* row = scores + static_cast<int64_t>(u) * C;
   for (int c = threadIdx.x; c < v; c += blockDim.x) {
     const bool f = is_forced(c, v, n_sink, n_local);
@@ -1194,13 +1205,15 @@ cudaError_t set_smem(const void* fn, size_t bytes) {
 
 cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
-                               int32_t* idx, int32_t* count, int kmax, const int32_t* k_dev) {
+                               int32_t* idx, int32_t* count, int kmax, const int32_t* k_dev,
+                               int causal_tiles, int causal_tile_m, int causal_L) {
   if (U == 0) return cudaSuccess;
   const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_topk_kernel), sh);
   if (e != cudaSuccess) return e;
+  const CausalRows causal{causal_tiles, causal_tile_m, causal_L};
   select_topk_kernel<<<U, kSelThreads, sh, l.stream>>>(scores, C, n_valid, k_free, n_sink, n_local,
-                                                       idx, count, kmax, k_dev);
+                                                       idx, count, kmax, k_dev, causal);
   return cudaGetLastError();
 }
 

@@ -661,8 +661,9 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
 
 // ---------------------------------------------------------------- gather / scatter
 
-// Compressed row t of (b, h): the kept token idx[u, t] (t < count[u]) or a
-// zero row.  Q^ [B, Sc, Hq, D] takes the G query heads of the group; K^, V^
+// Compressed row t < count[u] of (b, h): the kept token idx[u, t]; rows
+// past the unit's count are not written (no causal list reaches them).
+// Q^ [B, Sc, Hq, D] takes the G query heads of the group; K^, V^
 // [B, Hkv, Sc, D].  16 bytes per thread.
 __global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
                                   const __nv_bfloat16* __restrict__ K,
@@ -677,17 +678,17 @@ __global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
   const int per_row = (G + 2) * V8;
   const int64_t u = blockIdx.y;
   const int b = static_cast<int>(u / Hkv), h = static_cast<int>(u % Hkv);
-  const int n = count[u];
+  const int n = min(count[u], Sc);
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < Sc; t += gridDim.x * wpb) {
-    const int p = t < n ? idx[u * kmax + t] : -1;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < n; t += gridDim.x * wpb) {
+    const int p = idx[u * kmax + t];
 #pragma unroll 3
     for (int w = lane; w < per_row; w += 32) {
       const int part = w / V8, c = (w % V8) * 8;
       int4 v = make_int4(0, 0, 0, 0);
       if (part < G) {  // query head h*G + part
-        if (p >= 0)
+        if (p >= 0 && p < S)
           v = *reinterpret_cast<const int4*>(
               Q + ((static_cast<int64_t>(b) * S + p) * Hq + h * G + part) * D + c);
         *reinterpret_cast<int4*>(Qc + ((static_cast<int64_t>(b) * Sc + t) * Hq + h * G + part) * D +
@@ -695,7 +696,7 @@ __global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
       } else {
         const __nv_bfloat16* src = part == G ? K : V;
         __nv_bfloat16* dst = part == G ? Kc : Vc;
-        if (p >= 0) v = *reinterpret_cast<const int4*>(src + (u * S + p) * D + c);
+        if (p >= 0 && p < S) v = *reinterpret_cast<const int4*>(src + (u * S + p) * D + c);
         *reinterpret_cast<int4*>(dst + (u * Sc + t) * D + c) = v;
       }
     }
@@ -703,8 +704,9 @@ __global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
 }
 
 // Dense causal chunk lists of the compressed sequences: tile t of (b, h)
-// sees chunks 0..t (chunk = tile = 64 rows); tiles past the budget of
-// sequence b see none (their rows are padding and come out 0).
+// sees chunks 0..t (chunk = tile = 64 rows); tiles past the unit's budget
+// k_unit (a multiple of the tile) see none and are skipped by the dense
+// attention.
 __global__ void tsa_lists_kernel(const int32_t* __restrict__ k_unit, int n_tiles, int tile,
                                  int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
   const int64_t ut = blockIdx.x;  // (b * Hkv + h) * n_tiles + t

@@ -32,10 +32,12 @@ class SparseDecoder:
     ``step`` is one call of csa_decode_step, whose decode streams the
     full-attention heads while the selection runs.
 
-    hybrid=True (bf16, fused): every sparse head also attends over one gist
-    key/value row per chunk (the hybrid context of SSA).  The gist rows are
-    built here with the cache, as the chunk means of K and V in bf16: the
-    stand-in for a trained model's gist KV.
+    hybrid=True (bf16, fused): every sparse head also attends over gist
+    key/value rows (the hybrid context of SSA): those of its selected chunks
+    (gist_scope="selected", the method section's reading) or of every chunk
+    (gist_scope="all").  gist=(Kg, Vg), each [B, Hkv, T/L, D] bf16, is the
+    model's gist KV; when it is not given the rows are built here with the
+    cache, as the chunk means of K and V in bf16 (a stand-in).
 
     rope_theta > 0 (the RoPE-aware split): K and the queries given to ``step``
     are pre-RoPE; chunks are scored on them, and attention runs on rotated
@@ -46,7 +48,8 @@ class SparseDecoder:
                  n_sink: int, n_local: int, k_free: int = 0, proj: torch.Tensor | None = None,
                  p: float = 0.9, budget: int = 256, full_heads=(), Gm: int = 0, top_meta: int = 0,
                  scale: float | None = None, num_parts: int = 0, out_dtype=torch.float32,
-                 fused: bool = True, hybrid: bool = False, rope_theta: float = 0.0):
+                 fused: bool = True, hybrid: bool = False, gist=None, gist_scope: str = "selected",
+                 rope_theta: float = 0.0):
         assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
         self.K, self.V = K, V
         B, Hkv, T, D = K.shape
@@ -75,7 +78,11 @@ class SparseDecoder:
             csa.csa_rope(K, self.K_att, self.dtype, B * Hkv * T, D, T, 0, self.rope_theta)
             self.q_rot = torch.empty(B, Hq, D, dtype=K.dtype, device=dev)
         self.Kg = self.Vg = None
-        if hybrid:
+        self.gist_scope = gist_scope
+        if hybrid and gist is not None:
+            assert fused and K.dtype == torch.bfloat16, "the hybrid context needs a fused bf16 decode"
+            self.Kg, self.Vg = gist
+        elif hybrid:
             assert fused and K.dtype == torch.bfloat16, "the hybrid context needs a fused bf16 decode"
             means = torch.empty(B, Hkv, self.C, D, dtype=torch.float32, device=dev)
             csa.csa_chunk_summaries(K, self.dtype, B, Hkv, T, D, L, None, 0, means)
@@ -120,7 +127,8 @@ class SparseDecoder:
                 n_local=n_local, logit_scale=1.0 / math.sqrt(D), p=p, budget=budget, idx=self.idx,
                 count=self.count, kmax=self.kmax, n_p_out=self.n_p, num_parts=num_parts,
                 workspace=self.workspace, workspace_bytes=self.ws_bytes, out=self.out,
-                out_dtype=self.out.dtype, lse_out=self.lse, Kg=self.Kg, Vg=self.Vg)
+                out_dtype=self.out.dtype, lse_out=self.lse, Kg=self.Kg, Vg=self.Vg,
+                gist_scope=gist_scope)
 
     def select_chunks(self, q: torch.Tensor, stream=None):
         """Score + select: fills self.idx / self.count (and self.n_p for top-p)."""
@@ -165,7 +173,8 @@ class SparseDecoder:
         """Sparse split-K decode over the current index lists, then the LSE merge
         (one launch when fused)."""
         if self.Kg is not None:
-            csa.csa_sparse_decode_merged_hybrid(q, self.K_att, self.V, self.Kg, self.Vg, self.dtype,
+            csa.csa_sparse_decode_merged_hybrid(q, self.K_att, self.V, self.Kg, self.Vg,
+                                                self.gist_scope, self.dtype,
                                                 self.idx, self.count, self.kmax, self.head_full,
                                                 self.B, self.Hq, self.Hkv, self.D, self.T, self.L,
                                                 self.scale, self.P, self.workspace, self.ws_bytes,
@@ -255,9 +264,6 @@ class BlockSparsePrefill:
         self.qbar = torch.empty(B, self.n_tiles, Hq, D, dtype=torch.float32, device=dev)
         self.scores = torch.empty(B, Hkv, self.n_tiles, self.C, dtype=torch.float32, device=dev)
         U = B * Hkv * self.n_tiles
-        t = torch.arange(self.n_tiles, dtype=torch.int64)
-        n_valid = ((t + 1) * tile_m - 1) // L + 1
-        self.n_valid = n_valid.repeat(B * Hkv).to(torch.int32).to(dev)
         self.idx = torch.full((U, self.kmax), -1, dtype=torch.int32, device=dev)
         self.count = torch.zeros(U, dtype=torch.int32, device=dev)
         self.O = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=dev)
@@ -267,9 +273,9 @@ class BlockSparsePrefill:
         csa.csa_tile_mean_q(self.Q, _dt(self.Q), B, S, Hq, D, self.tile_m, self.qbar, stream=stream)
         csa.csa_score_chunks(self.qbar, csa.CSA_F32, None, 0, self.summ, B, self.n_tiles, Hq, Hkv,
                              D, self.C, None, self.tile_m, self.L, self.scores, stream=stream)
-        csa.csa_select_topk(self.scores, B * Hkv * self.n_tiles, self.C, self.n_valid, self.k_free,
-                            self.n_sink, self.n_local, self.idx, self.count, self.kmax,
-                            stream=stream)
+        csa.csa_select_topk_causal(self.scores, B * Hkv * self.n_tiles, self.C, self.n_tiles,
+                                   self.tile_m, self.L, self.k_free, self.n_sink, self.n_local,
+                                   self.idx, self.count, self.kmax, stream=stream)
 
     def attend(self, stream=None):
         csa.csa_block_sparse_prefill(self.Q, self.K, self.V, self.idx, self.count, self.kmax,

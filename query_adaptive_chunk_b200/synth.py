@@ -36,7 +36,8 @@ from typing import Optional
 
 import torch
 
-TENSOR_ID = {"q": 0, "k": 1, "v": 2, "proj": 3, "plant": 4, "perm": 5}
+TENSOR_ID = {"q": 0, "k": 1, "v": 2, "proj": 3, "plant": 4, "perm": 5, "gist_k": 6, "gist_v": 7,
+             "heavy_dir": 8, "heavy_pick": 9}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -65,7 +66,8 @@ class DecodeWorkload:
     full_heads: tuple = ()  # KV heads that attend to every chunk
     Gm: int = 0  # hierarchical: chunks per meta-chunk
     top_meta: int = 0  # hierarchical: meta-chunks kept
-    hybrid: bool = False  # sparse heads also attend over one gist row per chunk
+    hybrid: bool = False  # sparse heads also attend over gist rows (one per chunk)
+    gist_scope: str = ""  # hybrid: "selected" (the chosen chunks' gist rows) or "all"
     rope_theta: float = 0.0  # > 0: K/q are pre-RoPE; attention on the rotated ones
 
     @property
@@ -112,6 +114,13 @@ class PrefillWorkload:
     planted: int = 8
     strength: float = 3.0
     dtype: str = "bf16"
+    # heavy-hitter tokens: per sequence a seeded fraction of the token
+    # positions, shared by its KV heads, whose keys get +heavy_strength * w,
+    # with every query row of the group's heads also given +heavy_strength * w
+    # (w a seeded random unit direction per (b, kvh)), so that attention mass
+    # concentrates on them
+    heavy_frac: float = 0.0
+    heavy_strength: float = 0.0
 
     @property
     def C(self) -> int:
@@ -156,15 +165,26 @@ PREFILL_32K = PrefillWorkload(
     name="block_sparse_prefill_bf16_seq32k", seed=5, B=1, S=32768, Hq=32, Hkv=8, D=128,
     tile_m=64, L=64, k_free=16)
 
+# Token Sparse Attention in its high-sparsity regime: the 32K prefill shapes
+# with 20% heavy-hitter tokens per KV head (keys and queries share a planted
+# direction), so the coverage budget keeps a small part of the sequence
+TOKEN_SPARSE_HEAVY_32K = dataclasses.replace(
+    PREFILL_32K, name="token_sparse_heavy_prefill_bf16_seq32k", seed=9, planted=0,
+    heavy_frac=0.2, heavy_strength=8.0)
+
 # Per-head top-k with the GQA union on the 32K shapes: each of the 4 query
 # heads of a group keeps its own 29 best chunks, the group reads the union.
 TOPK_UNION_32K = dataclasses.replace(TOPK_32K, name="topk_union_decode_bf16_ctx32k", seed=6,
                                      select="topk_union")
 
-# SSA's hybrid context: the 32K top-k step with every chunk's gist row in the
-# context of each sparse head (8 extra 64-row chunks per unit)
+# SSA's hybrid context on the 32K top-k step: each sparse head attends over
+# the gist and raw KV of its 32 chosen chunks (one extra 64-row chunk of
+# gathered gist rows per unit), or, in the "all" scope, over every chunk's
+# gist row plus the raw KV of its chunks (8 extra 64-row chunks per unit)
 HYBRID_TOPK_32K = dataclasses.replace(TOPK_32K, name="hybrid_topk_decode_bf16_ctx32k", seed=7,
-                                      hybrid=True)
+                                      hybrid=True, gist_scope="selected")
+HYBRID_ALL_TOPK_32K = dataclasses.replace(TOPK_32K, name="hybrid_all_topk_decode_bf16_ctx32k",
+                                          seed=8, hybrid=True, gist_scope="all")
 
 # RTPurbo's RoPE-aware split: the 32K top-k step scored on the pre-RoPE keys
 # and query, attending with the rotated ones (base 500000)
@@ -172,8 +192,8 @@ ROPE_TOPK_32K = dataclasses.replace(TOPK_32K, name="rope_topk_decode_bf16_ctx32k
                                     rope_theta=500000.0)
 
 DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M, TOPK_UNION_32K, HYBRID_TOPK_32K,
-                    ROPE_TOPK_32K)
-ALL_WORKLOADS = DECODE_WORKLOADS + (PREFILL_32K,)
+                    HYBRID_ALL_TOPK_32K, ROPE_TOPK_32K)
+ALL_WORKLOADS = DECODE_WORKLOADS + (PREFILL_32K, TOKEN_SPARSE_HEAVY_32K)
 
 
 def _gen(device, seed: int, tid: int) -> torch.Generator:
@@ -239,6 +259,13 @@ def make_decode_inputs(w: DecodeWorkload, device="cpu") -> dict:
             K[b, h] = kb.to(dt)
             V[b, h] = vb.to(dt)
     out = {"q": q, "K": K, "V": V, "planted": planted}
+    if w.hybrid:
+        # gist key / value rows [B, Hkv, C, D]: a trained model's gist KV is an
+        # input of the step; drawn here N(0, 1/L), the spread of a mean of L
+        # N(0, 1) rows
+        shape = (w.B, w.Hkv, w.C, w.D)
+        out["Kg"] = (_randn(shape, device, w.seed, TENSOR_ID["gist_k"]) / math.sqrt(w.L)).to(dt)
+        out["Vg"] = (_randn(shape, device, w.seed, TENSOR_ID["gist_v"]) / math.sqrt(w.L)).to(dt)
     if w.proj_rank > 0:
         out["proj"] = (_randn((w.D, w.proj_rank), device, w.seed, TENSOR_ID["proj"]) / 4.0)
     return out
@@ -258,7 +285,18 @@ def make_prefill_inputs(w: PrefillWorkload, device="cpu") -> dict:
     V = torch.empty((w.B, w.Hkv, w.S, w.D), dtype=dt, device=device)
     free = torch.arange(1, max(w.C - 1, 1), dtype=torch.long)  # never the first or last chunk
     planted = []
+    heavy = []
+    if w.heavy_frac > 0:
+        gdir = torch.Generator(device="cpu")
+        gdir.manual_seed(w.seed * 1000 + TENSOR_ID["heavy_dir"])
+        ghp = torch.Generator(device="cpu")
+        ghp.manual_seed(w.seed * 1000 + TENSOR_ID["heavy_pick"])
+        Qf = Q.float()
     for b in range(w.B):
+        if w.heavy_frac > 0:
+            n_heavy = int(round(w.heavy_frac * w.S))
+            pos = torch.randperm(w.S, generator=ghp)[:n_heavy].sort().values
+            heavy.append(pos.tolist())
         for h in range(w.Hkv):
             kb = torch.randn((w.S, w.D), generator=gk, device=device, dtype=torch.float32)
             vb = torch.randn((w.S, w.D), generator=gv, device=device, dtype=torch.float32)
@@ -268,9 +306,16 @@ def make_prefill_inputs(w: PrefillWorkload, device="cpu") -> dict:
                 planted.append(pick.tolist())
             else:
                 planted.append([])
+            if w.heavy_frac > 0:
+                d = torch.randn(w.D, generator=gdir, dtype=torch.float64)
+                d = (d / d.norm()).to(torch.float32).to(device)
+                kb[pos.to(device)] += w.heavy_strength * d
+                Qf[b, :, h * w.G:(h + 1) * w.G] += w.heavy_strength * d
             K[b, h] = kb.to(dt)
             V[b, h] = vb.to(dt)
-    return {"Q": Q, "K": K, "V": V, "planted": planted}
+    if w.heavy_frac > 0:
+        Q = Qf.to(dt)
+    return {"Q": Q, "K": K, "V": V, "planted": planted, "heavy": heavy}
 
 
 def decode_units(w: DecodeWorkload):

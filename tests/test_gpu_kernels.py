@@ -149,6 +149,27 @@ def test_select_topk_n_valid(csa):
         assert got[u] == ref, (u, nv[u])
 
 
+@pytest.mark.parametrize("tile_m,L,C", [(64, 64, 64), (128, 64, 130), (64, 128, 40), (32, 96, 23)])
+def test_select_topk_causal(csa, tile_m, L, C):
+    """Query tiles of a causal prefill: tile t sees the chunks that hold a
+    key at or before its last row (t + 1) * tile_m - 1; the diagonal chunk is
+    the forced local one.  Two (sequence, KV head) rows of tiles."""
+    n_tiles = (C * L) // tile_m
+    U = 2 * n_tiles
+    s = _randn((U, C), 12)
+    kmax = min(C, 16 + 2)
+    idx = torch.full((U, kmax), 777, dtype=torch.int32, device="cuda")
+    cnt = torch.full((U,), 777, dtype=torch.int32, device="cuda")
+    csa.csa_select_topk_causal(s, U, C, n_tiles, tile_m, L, 16, 1, 1, idx, cnt, kmax)
+    got = parity.gpu_sets(idx, cnt)
+    sn = s.cpu().double().numpy()
+    for u in range(U):
+        last_row = (u % n_tiles + 1) * tile_m - 1
+        v = sum(1 for c in range(C) if c * L <= last_row)
+        ref, _ = O.select_topk(sn[u], 16, 1, 1, n_valid=v)
+        assert got[u] == ref, (u, v)
+
+
 def test_select_topk_golden(csa):
     for c in pins_golden("topk_cases.json"):
         s = torch.tensor([c["scores"]], dtype=torch.float32, device="cuda")
@@ -557,11 +578,12 @@ def test_merged_decode_second_wave(csa):
 
 
 def _hybrid_case(csa, B, Hkv, G, D, L, C, sets, full=(), num_parts=0, out_bf16=False,
-                 with_lse=True, seed=60, via_step=False):
+                 with_lse=True, seed=60, scope="selected"):
     """csa_sparse_decode_merged_hybrid against the oracle's hybrid context:
     random bf16 gist rows (any gist KV is a valid input), every sparse unit
-    over all its gist rows plus its selected chunks, full units over their
-    raw chunks only."""
+    over its selected chunks' raw KV plus the gist rows of the scope (its
+    selected chunks', or every chunk's), full units over their raw chunks
+    only."""
     Hq, T = G * Hkv, C * L
     dt = _dt("bf16")
     q = _randn((B, Hq, D), seed, dt)
@@ -589,8 +611,9 @@ def _hybrid_case(csa, B, Hkv, G, D, L, C, sets, full=(), num_parts=0, out_bf16=F
     out = torch.full((B, Hq, D), float("nan"), device="cuda").to(odt)
     lse = torch.full((B, Hq), float("nan"), device="cuda") if with_lse else None
     for _ in range(2):  # the second call sees the counters the first left
-        csa.csa_sparse_decode_merged_hybrid(q, K, V, Kg, Vg, dt, idx, cnt, kmax, hf, B, Hq, Hkv,
-                                            D, T, L, scale, num_parts, ws, nbytes, out, odt, lse)
+        csa.csa_sparse_decode_merged_hybrid(q, K, V, Kg, Vg, scope, dt, idx, cnt, kmax, hf, B, Hq,
+                                            Hkv, D, T, L, scale, num_parts, ws, nbytes, out, odt,
+                                            lse)
         csa.csa_check_device_status()
     qn = to_np(q)
     Kc, Vc, Kgc, Vgc = K.cpu(), V.cpu(), Kg.cpu(), Vg.cpu()
@@ -603,35 +626,47 @@ def _hybrid_case(csa, B, Hkv, G, D, L, C, sets, full=(), num_parts=0, out_bf16=F
                                    scale)
         else:
             ro, rl = O.hybrid_unit(qn[b, rows], to_np(Kc[b, h]), to_np(Vc[b, h]),
-                                   to_np(Kgc[b, h]), to_np(Vgc[b, h]), st, L, scale)
-        parity.assert_close(got, ro, "bf16", f"hybrid unit {u}")
+                                   to_np(Kgc[b, h]), to_np(Vgc[b, h]), st, L, scale, scope)
+        parity.assert_close(got, ro, "bf16", f"hybrid {scope} unit {u}")
         if lse is not None:
-            assert np.abs(lse[b, rows].cpu().double().numpy() - rl).max() < 1e-3, u
+            gl = lse[b, rows].cpu().double().numpy()
+            assert np.array_equal(np.isneginf(gl), np.isneginf(rl)), (u, gl, rl)
+            fin = np.isfinite(rl)
+            assert np.abs(gl[fin] - rl[fin]).max(initial=0.0) < 1e-3, u
     return out
 
 
+@pytest.mark.parametrize("scope", ["selected", "all"])
 @pytest.mark.parametrize("D,L,G,C,parts", [(128, 128, 4, 24, 0), (128, 64, 4, 150, 13),
                                            (64, 64, 8, 40, 7), (64, 128, 2, 300, 256),
                                            (128, 128, 1, 9, 3)])
-def test_hybrid_decode_shapes(csa, D, L, G, C, parts):
-    """Gist rows from one ragged chunk (C < L) to several with a ragged last
-    one (C % L != 0), GQA groups 1-8, few and many pieces."""
+def test_hybrid_decode_shapes(csa, D, L, G, C, parts, scope):
+    """Gist rows from one ragged chunk (fewer rows than L) to several with a
+    ragged last one, GQA groups 1-8, few and many pieces."""
     B, Hkv = 2, 3
     rng = np.random.default_rng(D + L + G + C)
     sets = [sorted(rng.choice(C, size=int(rng.integers(1, min(C, 14) + 1)),
                               replace=False).tolist()) for _ in range(B * Hkv)]
-    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=parts)
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=parts, scope=scope)
 
 
-def test_hybrid_decode_edge_cases(csa):
-    """A unit with no selected chunk attends over its gist rows alone; full
-    heads ignore the gist rows; bf16 output; one piece; no lse output."""
+@pytest.mark.parametrize("scope", ["selected", "all"])
+def test_hybrid_decode_edge_cases(csa, scope):
+    """A unit with no selected chunk: its gist rows alone (scope "all") or an
+    empty context, out = 0 and lse = -inf ("selected"); full heads ignore
+    the gist rows; bf16 output; one piece; no lse output; more selected
+    chunks than one gathered gist chunk holds (L = 64, 80 and 130 chunks)."""
     B, Hkv, G, D, L, C = 1, 4, 4, 128, 64, 9
     sets = [[], [0], [2, 5, 8], list(range(9))]
-    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=1)
-    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=200, out_bf16=True)
-    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, full=(2,), num_parts=7, with_lse=False)
-    _hybrid_case(csa, 2, 8, 4, 128, 128, 96, [list(range(0, 96, 5))] * 16, full=(0, 1))
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=1, scope=scope)
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, num_parts=200, out_bf16=True, scope=scope)
+    _hybrid_case(csa, B, Hkv, G, D, L, C, sets, full=(2,), num_parts=7, with_lse=False,
+                 scope=scope)
+    _hybrid_case(csa, 2, 8, 4, 128, 128, 96, [list(range(0, 96, 5))] * 16, full=(0, 1),
+                 scope=scope)
+    rng = np.random.default_rng(5)
+    big = [sorted(rng.choice(200, size=n, replace=False).tolist()) for n in (80, 130, 64, 1)]
+    _hybrid_case(csa, 1, 4, 4, 128, 64, 200, big, num_parts=0, scope=scope)
 
 
 def test_hybrid_decode_rejects_fp32_and_unaligned(csa):
@@ -648,14 +683,18 @@ def test_hybrid_decode_rejects_fp32_and_unaligned(csa):
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
     out = torch.zeros(B, Hq, D, device="cuda")
     with pytest.raises(CsaError):
-        csa.csa_sparse_decode_merged_hybrid(q, K, K, g, g, torch.float32, idx, cnt, 1, None, B, Hq,
-                                            Hkv, D, C * L, L, 0.1, 0, ws, nbytes, out,
+        csa.csa_sparse_decode_merged_hybrid(q, K, K, g, g, "all", torch.float32, idx, cnt, 1, None,
+                                            B, Hq, Hkv, D, C * L, L, 0.1, 0, ws, nbytes, out,
                                             torch.float32, None)
     qb, Kb, gb = q.bfloat16(), K.bfloat16(), g.bfloat16()
     with pytest.raises(CsaError):
-        csa.csa_sparse_decode_merged_hybrid(qb, Kb, Kb, gb.view(-1)[1:].data_ptr(), gb, torch.bfloat16,
-                                            idx, cnt, 1, None, B, Hq, Hkv, D, C * L, L, 0.1, 0, ws,
-                                            nbytes, out, torch.float32, None)
+        csa.csa_sparse_decode_merged_hybrid(qb, Kb, Kb, gb.view(-1)[1:].data_ptr(), gb, "selected",
+                                            torch.bfloat16, idx, cnt, 1, None, B, Hq, Hkv, D, C * L,
+                                            L, 0.1, 0, ws, nbytes, out, torch.float32, None)
+    with pytest.raises(CsaError, match="gist_scope"):
+        csa.csa_sparse_decode_merged_hybrid(qb, Kb, Kb, gb, gb, 2, torch.bfloat16, idx, cnt, 1,
+                                            None, B, Hq, Hkv, D, C * L, L, 0.1, 0, ws, nbytes, out,
+                                            torch.float32, None)
 
 
 def test_merged_decode_mixed_heads(csa):

@@ -118,13 +118,189 @@ def test_token_sparse_prefill_matches_oracle(B, S, Hq, Hkv, n_obs, tau, seed):
             got = Ob[b, :, h * G:(h + 1) * G].float().cpu().double().numpy()
             # rows the GPU kept: nonzero; ambiguous only at importance near-ties
             kept_gpu = np.abs(got).sum(axis=(1, 2)) > 0
-            kept_ref = np.zeros(S, dtype=bool)
-            kept_ref[toks] = True
-            diff = np.nonzero(kept_gpu != kept_ref)[0]
-            if len(diff):
-                cut = np.sort(imps[h])[::-1][kt - 1]
-                rel = np.abs(imps[h][diff] - cut) / cut
-                assert rel.max() < 1e-3, (h, diff[:8], rel.max())
-                parity.NEAR_TIE_LOG.append(("token sparse set", b, h, len(diff)))
-                continue  # outputs of later rows shift with the set: compared where sets agree
+            toks = _check_kept_set(kept_gpu, toks, imps[h], kt, S, f"b{b} h{h}")
+            if toks is not None:  # near-tie: the oracle over the GPU's own set
+                ref = O.token_sparse_head(to_np(Q[b, :, h * G:(h + 1) * G]), to_np(K[b, h]),
+                                          to_np(V[b, h]), toks, scale)
             parity.assert_close(got, ref, "bf16", f"token sparse b{b} h{h}")
+
+
+def _check_kept_set(kept_gpu, toks_ref, imp, kt, S, label):
+    """The GPU's kept rows against the oracle's top-kt tokens: identical, or
+    different only among tokens whose importance is within 1e-3 (relative)
+    of the cut, in which case the GPU's set (of the same size) is returned
+    for the oracle to recompute over; None when the sets agree."""
+    kept_ref = np.zeros(S, dtype=bool)
+    kept_ref[toks_ref] = True
+    diff = np.nonzero(kept_gpu != kept_ref)[0]
+    if len(diff) == 0:
+        return None
+    assert int(kept_gpu.sum()) == kt, (label, int(kept_gpu.sum()), kt)
+    cut = np.sort(imp)[::-1][kt - 1]
+    rel = np.abs(imp[diff] - cut) / cut
+    assert rel.max() < 1e-3, (label, diff[:8], rel.max())
+    parity.NEAR_TIE_LOG.append(("token sparse set", label, len(diff)))
+    print(f"near-tie: token sparse {label}: {len(diff)} tokens swapped at the cut")
+    return np.nonzero(kept_gpu)[0].tolist()
+
+
+def test_token_sparse_prefill_benched_workload():
+    """The benched Token Sparse call at full size: the 32K prefill inputs
+    (planted chunks), n_obs = 64, tau = 0.1, all 8 KV heads.  The importance
+    of every key of every head and the budget against the oracle; per head
+    the kept set, a sample of 40 output rows (the first, the last and random
+    kept rows, each against the oracle's causal attention over the kept
+    tokens) and 16 dropped rows (exactly 0)."""
+    from query_adaptive_chunk_b200 import csa, synth
+    w = synth.PREFILL_32K
+    inp = synth.make_prefill_inputs(w, device="cuda")
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    B, S, Hq, Hkv, D = w.B, w.S, w.Hq, w.Hkv, w.D
+    G, n_obs, tau, scale = w.G, 64, 0.1, w.scale
+    nb = csa.csa_token_importance_scratch_bytes(B, S, Hq, Hkv, n_obs)
+    scratch = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    imp = torch.full((B, Hkv, S), float("nan"), device="cuda")
+    csa.csa_token_importance(Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp, scratch, nb)
+    nbw = csa.csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs)
+    ws = torch.empty(nbw, dtype=torch.uint8, device="cuda")
+    Ob = torch.full((B, S, Hq, D), float("nan"), device="cuda").to(torch.bfloat16)
+    budget = torch.zeros(B, dtype=torch.int32, device="cuda")
+    csa.csa_token_sparse_prefill(Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale, ws, nbw, Ob, budget)
+    csa.csa_check_device_status()
+    imps = [_oracle_importance(Q, K, 0, h, G, n_obs, scale) for h in range(Hkv)]
+    for h in range(Hkv):
+        got = imp[0, h].cpu().double().numpy()
+        assert np.allclose(got, imps[h], rtol=1e-3, atol=1e-6), (h, np.abs(got - imps[h]).max())
+    mass = np.sum(imps, axis=0)
+    k_ref = O.coverage_budget(mass, tau)
+    k_got = int(budget[0])
+    cum = np.cumsum(np.sort(mass / mass.sum())[::-1])
+    assert k_got == k_ref or (cum[k_got - 1] >= (1 - tau) - 1e-6 and
+                              (k_got < 2 or cum[k_got - 2] <= (1 - tau) + 1e-6)), (k_got, k_ref)
+    kt = min(S, (k_got + 63) // 64 * 64)
+    rng = np.random.default_rng(32768)
+    Kc, Vc = K[0].cpu(), V[0].cpu()
+    for h in range(Hkv):
+        got = Ob[0, :, h * G:(h + 1) * G].float().cpu().double().numpy()  # [S, G, D]
+        kept_gpu = np.abs(got).sum(axis=(1, 2)) > 0
+        toks_ref = O.select_tokens(imps[h], kt)
+        toks = _check_kept_set(kept_gpu, toks_ref, imps[h], kt, S, f"h{h}")
+        tset = np.asarray(toks if toks is not None else toks_ref, dtype=np.int64)
+        picks = np.unique(np.concatenate([[0, kt - 1], rng.choice(kt, size=38, replace=False)]))
+        Kh, Vh = to_np(Kc[h][tset]), to_np(Vc[h][tset])
+        for i in picks:
+            t = int(tset[i])
+            qrows = to_np(Q[0, t, h * G:(h + 1) * G])  # [G, D]
+            ref = np.stack([O.causal_attend(qrows[g:g + 1], Kh, Vh, tset, t, scale)[0]
+                            for g in range(G)])
+            parity.assert_close(got[t], ref, "bf16", f"token sparse h{h} row {t}")
+        dropped = np.nonzero(~kept_gpu)[0]
+        if len(dropped):
+            pick = rng.choice(dropped, size=min(16, len(dropped)), replace=False)
+            assert np.all(got[pick] == 0), (h, pick)
+
+
+def _token_steps(csa, Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale):
+    """csa_token_importance, _budget, _select, _compress, _attend and
+    _decompress called one after the other; returns (O, k_seq)."""
+    dev = "cuda"
+    U = B * Hkv
+    nb = csa.csa_token_importance_scratch_bytes(B, S, Hq, Hkv, n_obs)
+    scratch = torch.empty(nb, dtype=torch.uint8, device=dev)
+    imp = torch.empty(B, Hkv, S, device=dev)
+    csa.csa_token_importance(Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp, scratch, nb)
+    k_seq = torch.empty(B, dtype=torch.int32, device=dev)
+    k_unit = torch.empty(U, dtype=torch.int32, device=dev)
+    csa.csa_token_budget(imp, B, S, Hkv, tau, 64, k_seq, k_unit)
+    idx = torch.empty(U, S, dtype=torch.int32, device=dev)
+    cnt = torch.empty(U, dtype=torch.int32, device=dev)
+    csa.csa_token_select(imp, B, S, Hkv, k_unit, idx, cnt)
+    Qc = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=dev)
+    Kc = torch.empty(B, Hkv, S, D, dtype=torch.bfloat16, device=dev)
+    Vc = torch.empty_like(Kc)
+    csa.csa_token_compress(Q, K, V, idx, cnt, B, S, Hq, Hkv, D, Qc, Kc, Vc)
+    na = csa.csa_token_attend_scratch_bytes(B, S, Hkv)
+    sa = torch.empty(na, dtype=torch.uint8, device=dev)
+    Oc = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=dev)
+    csa.csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, sa, na, Oc)
+    nd = csa.csa_token_decompress_scratch_bytes(B, S, Hkv)
+    sd = torch.empty(nd, dtype=torch.uint8, device=dev)
+    O = torch.full((B, S, Hq, D), float("nan"), device=dev).to(torch.bfloat16)
+    csa.csa_token_decompress(Oc, idx, cnt, B, S, Hq, Hkv, D, sd, nd, O)
+    return O, k_seq
+
+
+def test_token_sparse_steps_match_whole_call_and_graph():
+    """The separate step calls give the whole call's output bit for bit (two
+    sequences with different budgets), and the whole call captured in a CUDA
+    graph replays to the same output: the call never reads the budget back
+    on the host."""
+    from query_adaptive_chunk_b200 import csa
+    B, S, Hq, Hkv, D, n_obs, tau = 2, 2048, 8, 2, 128, 64, 0.05
+    Q, K, V = _inputs(B, S, Hq, Hkv, D, seed=77)
+    Q[1, :, :, :] *= 4  # sharper attention in sequence 1: a different budget
+    scale = 1.0 / math.sqrt(D)
+    nbw = csa.csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs)
+    ws = torch.empty(nbw, dtype=torch.uint8, device="cuda")
+    O1 = torch.full((B, S, Hq, D), float("nan"), device="cuda").to(torch.bfloat16)
+    bud = torch.zeros(B, dtype=torch.int32, device="cuda")
+    csa.csa_token_sparse_prefill(Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale, ws, nbw, O1, bud)
+    O2, k_seq = _token_steps(csa, Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale)
+    csa.csa_check_device_status()
+    assert torch.equal(bud, k_seq) and bud[0] != bud[1], (bud, k_seq)
+    assert torch.equal(O1, O2)
+    O3 = torch.full_like(O1, float("nan"))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        csa.csa_token_sparse_prefill(Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale, ws, nbw, O3,
+                                     bud)
+    g.replay()
+    torch.cuda.synchronize()
+    csa.csa_check_device_status()
+    assert torch.equal(O1, O3)
+    del g
+
+
+def test_token_sparse_heavy_workload():
+    """The high-sparsity workload at full size (32K, 20% heavy-hitter tokens
+    shared by the KV heads, n_obs = 64, tau = 0.1): the budget keeps a small
+    part of the sequence; importance, budget, kept sets and a sample of
+    output rows per head against the oracle (as for the benched 32K call)."""
+    from query_adaptive_chunk_b200 import csa, synth
+    w = synth.TOKEN_SPARSE_HEAVY_32K
+    inp = synth.make_prefill_inputs(w, device="cuda")
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    B, S, Hq, Hkv, D = w.B, w.S, w.Hq, w.Hkv, w.D
+    G, n_obs, tau, scale = w.G, 64, 0.1, w.scale
+    O_gpu, k_seq = _token_steps(csa, Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale)
+    csa.csa_check_device_status()
+    imps = [_oracle_importance(Q, K, 0, h, G, n_obs, scale) for h in range(Hkv)]
+    mass = np.sum(imps, axis=0)
+    k_ref = O.coverage_budget(mass, tau)
+    k_got = int(k_seq[0])
+    cum = np.cumsum(np.sort(mass / mass.sum())[::-1])
+    assert k_got == k_ref or (cum[k_got - 1] >= (1 - tau) - 1e-6 and
+                              (k_got < 2 or cum[k_got - 2] <= (1 - tau) + 1e-6)), (k_got, k_ref)
+    assert k_got <= 0.25 * S, k_got
+    kt = min(S, (k_got + 63) // 64 * 64)
+    rng = np.random.default_rng(9)
+    Kc, Vc = K[0].cpu(), V[0].cpu()
+    for h in range(Hkv):
+        got = O_gpu[0, :, h * G:(h + 1) * G].float().cpu().double().numpy()
+        kept_gpu = np.abs(got).sum(axis=(1, 2)) > 0
+        toks_ref = O.select_tokens(imps[h], kt)
+        toks = _check_kept_set(kept_gpu, toks_ref, imps[h], kt, S, f"heavy h{h}")
+        tset = np.asarray(toks if toks is not None else toks_ref, dtype=np.int64)
+        picks = np.unique(np.concatenate([[0, kt - 1], rng.choice(kt, size=30, replace=False)]))
+        Kh, Vh = to_np(Kc[h][tset]), to_np(Vc[h][tset])
+        for i in picks:
+            t = int(tset[i])
+            qrows = to_np(Q[0, t, h * G:(h + 1) * G])
+            ref = np.stack([O.causal_attend(qrows[g:g + 1], Kh, Vh, tset, t, scale)[0]
+                            for g in range(G)])
+            parity.assert_close(got[t], ref, "bf16", f"heavy h{h} row {t}")
+        dropped = np.nonzero(~kept_gpu)[0]
+        pick = rng.choice(dropped, size=min(16, len(dropped)), replace=False)
+        assert np.all(got[pick] == 0), (h, pick)

@@ -20,10 +20,15 @@ def _decoder(w, inp, fused=True):
     return SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
                          n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
                          budget=w.budget, full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta,
-                         fused=fused, hybrid=w.hybrid, rope_theta=w.rope_theta)
+                         fused=fused, hybrid=w.hybrid,
+                         gist=(inp["Kg"], inp["Vg"]) if w.hybrid else None,
+                         gist_scope=w.gist_scope or "selected", rope_theta=w.rope_theta)
 
 
-def run_and_check(w, units=None, fused=True):
+def run_and_check(w, units=None, fused=True, attention_units=None):
+    """One step through the library against the oracle.  Index sets are
+    compared on `units` (default: all); outputs on `attention_units`
+    (default: the same units)."""
     from query_adaptive_chunk_b200 import csa
     inp = synth.make_decode_inputs(w, device="cuda")
     dec = _decoder(w, inp, fused)
@@ -31,11 +36,18 @@ def run_and_check(w, units=None, fused=True):
     csa.csa_check_device_status()
     all_units = synth.decode_units(w)
     units = units or all_units
-    ref = OP.decode_step(inp["q"], inp["K"], inp["V"], L=w.L, scale=w.scale, select=w.select,
-                         n_sink=w.n_sink, n_local=w.n_local, k_free=w.k_free,
-                         proj=inp.get("proj"), p=w.p, budget=w.budget, full_heads=w.full_heads,
-                         Gm=w.Gm, top_meta=w.top_meta, units=units,
-                         gist=(dec.Kg, dec.Vg) if w.hybrid else None, rope_theta=w.rope_theta)
+    att = units if attention_units is None else attention_units
+    gist = (inp["Kg"], inp["Vg"]) if w.hybrid else None
+    kw = dict(L=w.L, scale=w.scale, select=w.select, n_sink=w.n_sink, n_local=w.n_local,
+              k_free=w.k_free, proj=inp.get("proj"), p=w.p, budget=w.budget,
+              full_heads=w.full_heads, Gm=w.Gm, top_meta=w.top_meta, gist=gist,
+              gist_scope=w.gist_scope, rope_theta=w.rope_theta)
+    ref = OP.decode_step(inp["q"], inp["K"], inp["V"], units=att, **kw)
+    rest = [u for u in units if u not in att]
+    if rest:  # index sets only
+        r2 = OP.decode_step(inp["q"], inp["K"], inp["V"], units=rest, with_attention=False, **kw)
+        for key in ("sets", "gap", "n_p"):
+            ref[key].update(r2[key])
     gsets_all = parity.gpu_sets(dec.idx, dec.count)
     sparse = [u for u in units if u[1] not in w.full_heads]
     uidx = {u: i for i, u in enumerate(all_units)}
@@ -44,7 +56,7 @@ def run_and_check(w, units=None, fused=True):
                                 [ref["gap"][u] for u in sparse], w.name)
     G = w.G
     worst = 0.0
-    for (b, h) in units:
+    for (b, h) in att:
         got = out[b, h * G:(h + 1) * G].cpu().double().numpy()
         gset = list(range(w.C)) if h in w.full_heads else gsets_all[uidx[(b, h)]]
         if gset == ref["sets"][(b, h)]:
@@ -52,13 +64,14 @@ def run_and_check(w, units=None, fused=True):
         elif w.rope_theta:  # near-tie: rotated attention over the GPU's own set
             tok = O.chunk_tokens(gset, w.L)
             qg = to_np(inp["q"][b, h * G:(h + 1) * G])
-            qr = OP._stored(O.rope(qg, np.full(G, w.T - 1), w.rope_theta), inp["q"])
+            qr = OP._stored(O.rope(qg, np.full(G, OP.rope_query_position(w.T)), w.rope_theta),
+                            inp["q"])
             Kr = OP._stored(O.rope(to_np(inp["K"][b, h][tok]), tok, w.rope_theta), inp["K"])
             ro, rl = O.attend(qr, Kr, to_np(inp["V"][b, h][tok]), np.arange(len(tok)), w.scale)
         elif w.hybrid:  # near-tie: the hybrid context over the GPU's own set
             ro, rl = O.hybrid_unit(to_np(inp["q"][b, h * G:(h + 1) * G]), to_np(inp["K"][b, h]),
-                                   to_np(inp["V"][b, h]), to_np(dec.Kg[b, h]),
-                                   to_np(dec.Vg[b, h]), gset, w.L, w.scale)
+                                   to_np(inp["V"][b, h]), to_np(inp["Kg"][b, h]),
+                                   to_np(inp["Vg"][b, h]), gset, w.L, w.scale, w.gist_scope)
         else:  # near-tie: check attention over the GPU's own set
             ro, rl = O.decode_unit(to_np(inp["q"][b, h * G:(h + 1) * G]), to_np(inp["K"][b, h]),
                                    to_np(inp["V"][b, h]), gset, w.L, w.scale)
@@ -73,7 +86,8 @@ def run_and_check(w, units=None, fused=True):
                 assert n_p[uidx[(b, h)]] == rn or ref["gap"][(b, h)] < parity.NEAR_TIE
             else:
                 assert n_p[uidx[(b, h)]] == w.budget + 1 or ref["gap"][(b, h)] < parity.NEAR_TIE
-    print(f"{w.name}: units {len(units)} near-ties {n_tie} worst max-abs {worst:.3g}")
+    print(f"{w.name}: units {len(units)} (attention {len(att)}) near-ties {n_tie} "
+          f"worst max-abs {worst:.3g}")
     return dec, inp
 
 
@@ -114,8 +128,9 @@ def test_hier_decode_reduced():
     run_and_check(synth.HIER_1M.scaled(T=131072, planted=8))
 
 
-def test_hier_decode_full_size_sampled():
-    run_and_check(synth.HIER_1M, units=[(0, 0), (0, 5)])
+def test_hier_decode_full_size():
+    """1M context: the index sets of all 8 units, the attention of 3."""
+    run_and_check(synth.HIER_1M, attention_units=[(0, 0), (0, 5), (0, 7)])
 
 
 def test_decode_batch_with_gqa8_and_d64():
@@ -158,23 +173,28 @@ def test_topk_union_with_projection_and_full_head():
     run_and_check(w)
 
 
-def test_hybrid_topk_decode_reduced():
+@pytest.mark.parametrize("w", [synth.HYBRID_TOPK_32K, synth.HYBRID_ALL_TOPK_32K],
+                         ids=lambda w: w.gist_scope)
+def test_hybrid_topk_decode_reduced(w):
     """SSA's hybrid context through the one-call step: each sparse head over
-    its top-k chunks plus the gist row of every chunk (chunk means of K and V
-    as the gist stand-in, built with the cache)."""
-    run_and_check(synth.HYBRID_TOPK_32K.scaled(B=2, T=8192))
+    the raw KV of its top-k chunks plus gist rows (the chosen chunks' own, or
+    every chunk's), the gist rows drawn by the workload generator."""
+    run_and_check(w.scaled(B=2, T=8192))
 
 
-def test_hybrid_topk_decode_full_size():
-    run_and_check(synth.HYBRID_TOPK_32K)
+@pytest.mark.parametrize("w", [synth.HYBRID_TOPK_32K, synth.HYBRID_ALL_TOPK_32K],
+                         ids=lambda w: w.gist_scope)
+def test_hybrid_topk_decode_full_size(w):
+    run_and_check(w)
 
 
-def test_hybrid_with_projection_full_head_and_topp():
+@pytest.mark.parametrize("scope", ["selected", "all"])
+def test_hybrid_with_projection_full_head_and_topp(scope):
     """Hybrid context next to a full-attention head, with projected top-p
     scores (the full head attends over its raw tokens only)."""
     import dataclasses
     w = dataclasses.replace(synth.TOPP_128K.scaled(B=1, T=16384), name="hybrid_topp_mixed",
-                            seed=17, hybrid=True)
+                            seed=17, hybrid=True, gist_scope=scope)
     run_and_check(w)
 
 
@@ -182,7 +202,7 @@ def test_hybrid_separate_decode_call_matches_step():
     """csa_sparse_decode_merged_hybrid over the step's own index lists gives
     the step's output (same chunk sets, same gist rows)."""
     from query_adaptive_chunk_b200 import csa
-    w = synth.HYBRID_TOPK_32K.scaled(B=2, T=8192)
+    w = synth.HYBRID_TOPK_32K.scaled(B=2, T=8192, planted=2, k_free=100)
     dec, inp = run_and_check(w)
     out_step = dec.out.clone()
     dec.attend(inp["q"])
@@ -265,4 +285,17 @@ def test_decode_step_host_rejects_pageable_and_rope():
     with pytest.raises(csa.CsaError, match="CSA_ERR_UNSUPPORTED"):
         csa.csa_decode_step_host(dec.desc, inp["q"].cpu().pin_memory(), out_host)
     dec.desc.q_score = None
+    # a selection argument rejected (kmax below the set size) enqueues
+    # nothing: the device query buffer keeps what it held
+    dec.step_host(inp["q"].cpu().pin_memory(), out_host)
+    torch.cuda.synchronize()
+    sentinel = torch.full_like(dec.q_dev, 7.0)
+    dec.q_dev.copy_(sentinel)
+    kmax = dec.desc.kmax
+    dec.desc.kmax = 1
+    with pytest.raises(csa.CsaError, match="kmax"):
+        csa.csa_decode_step_host(dec.desc, (inp["q"] * 0).cpu().pin_memory(), out_host)
+    dec.desc.kmax = kmax
+    torch.cuda.synchronize()
+    assert torch.equal(dec.q_dev, sentinel)
     csa.csa_check_device_status()
