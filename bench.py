@@ -235,7 +235,8 @@ def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
         dec.step(q)
     torch.cuda.synchronize()
     ev = [_ext_event() for _ in range(3)]
-    use_graph = graph and all(e is not None for e in ev)
+    evs = [_ext_event() for _ in range(2)]  # around the step, inside G1
+    use_graph = graph and all(e is not None for e in ev + evs)
     if use_graph:
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
@@ -245,7 +246,9 @@ def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
         torch.cuda.synchronize()
         g1 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g1, capture_error_mode="relaxed"):
+            evs[0].record()
             dec.step(q)
+            evs[1].record()
         g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2, capture_error_mode="relaxed"):
             ev[0].record()
@@ -257,7 +260,7 @@ def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
             g1.replay()
             g2.replay()
         torch.cuda.synchronize()
-    step_ms, dec_ms = [], []
+    step_ms, dec_ms, sel_ms, launch_ms = [], [], [], []
     for _ in range(steps):
         flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -268,8 +271,10 @@ def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
             flush()
             g2.replay()
             torch.cuda.synchronize()
-            step_ms.append(e0.elapsed_time(e1))
+            step_ms.append(evs[0].elapsed_time(evs[1]))
+            launch_ms.append(e0.elapsed_time(e1))
             dec_ms.append(ev[1].elapsed_time(ev[2]))
+            sel_ms.append(ev[0].elapsed_time(ev[1]))
         else:
             e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             e[0].record()
@@ -279,9 +284,13 @@ def time_decode(w, steps: int, warmup: int, flush, graph: bool = True):
             e[2].record()
             torch.cuda.synchronize()
             step_ms.append(e[0].elapsed_time(e[2]))
+            launch_ms.append(e[0].elapsed_time(e[2]))
             dec_ms.append(e[1].elapsed_time(e[2]))
+            sel_ms.append(e[0].elapsed_time(e[1]))
     kv, summ, n_chunks = selected_bytes(w, dec)
-    res = {"step_ms": step_ms, "decode_ms": dec_ms, "kv_bytes": kv, "summ_bytes": summ,
+    res = {"step_ms": step_ms, "decode_ms": dec_ms, "select_ms": sel_ms,
+           "step_with_launch_ms": launch_ms, "kv_bytes": kv,
+           "summ_bytes": summ,
            "chunks": n_chunks, "graph": use_graph, "dec": dec, "inp": inp}
     return res
 
@@ -691,9 +700,11 @@ def run_ours(args):
                    "L": w.L, "select": "top-p p=0.9 cap 256 + sink + 2 local",
                    "full_heads": list(w.full_heads), "proj_rank": w.proj_rank,
                    "l2": "flushed before every step (256 MB write + 256 MB read)",
-                   "timing": "CUDA-graph replay, events around the replay; decode kernel "
-                             "from events inside a second graph of the same step" if r["graph"]
-                             else "direct launches, CUDA events",
+                   "timing": "CUDA-graph replay; step from events captured at the start and "
+                             "end of the step inside the graph (device time, the host's graph "
+                             "launch excluded: step_with_graph_launch_us includes it); decode "
+                             "kernel from events inside a second graph of the same step"
+                             if r["graph"] else "direct launches, CUDA events",
                    "parallelism": f"replicas x{world} (units shard, no collective)"},
         "hbm_gbs": round(step_gbs, 1), "hbm_frac_of_measured": round(step_gbs / peaks["hbm_gbs"], 4),
         "hbm_frac_of_8tbs_nominal": round(step_gbs / 8000.0, 4),
@@ -708,6 +719,8 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "mode": e2e_mode,
                 "direct_launch_value": round(e2e_eager_us, 3)},
         "gpu_launches": 2 * args.steps,
+        "step_with_graph_launch_us": round(1000 * statistics.mean(r["step_with_launch_ms"]), 3),
+        "select_us": round(1000 * statistics.mean(r["select_ms"]), 3),
         "timing_stats": {"rank": 0, "step_us_median": round(1000 * statistics.median(r["step_ms"]), 3),
                          "step_us_min": round(1000 * min(r["step_ms"]), 3),
                          "decode_us_median": round(1000 * statistics.median(r["decode_ms"]), 3),
@@ -733,9 +746,14 @@ def other_workloads(args, flush, peaks):
         dus = 1000 * statistics.mean(r["decode_ms"])
         byt = r["kv_bytes"] + r["summ_bytes"]
         out[w.name] = {"us_per_step": round(us, 3), "step_gbs": round(byt / (us * 1e-6) / 1e9, 1),
+                       "us_per_step_with_graph_launch": round(
+                           1000 * statistics.mean(r["step_with_launch_ms"]), 3),
                        "step_frac_of_measured_hbm": round(byt / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
                        "decode_us": round(dus, 3),
                        "decode_gbs": round(r["kv_bytes"] / (dus * 1e-6) / 1e9, 1),
+                       "decode_frac_of_measured_hbm": round(
+                           r["kv_bytes"] / (dus * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                       "select_us": round(1000 * statistics.mean(r["select_ms"]), 3),
                        "selected_kv_bytes": r["kv_bytes"], "summary_bytes": r["summ_bytes"]}
         del r
         torch.cuda.empty_cache()
@@ -786,6 +804,7 @@ def run_only(args, flush, peaks):
         us = 1000 * statistics.mean(r["step_ms"])
         dus = 1000 * statistics.mean(r["decode_ms"])
         d = {"workload": w.name, "us_per_step": us, "decode_us": dus,
+             "select_us": 1000 * statistics.mean(r["select_ms"]),
              "decode_gbs": r["kv_bytes"] / (dus * 1e-6) / 1e9}
     print(json.dumps(d))
     return 0

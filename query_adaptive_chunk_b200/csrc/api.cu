@@ -522,6 +522,7 @@ csa_status merged_decode(const void* q, const void* K, const void* V, const void
     m.Vg = Vg;
     m.gist_selected = gist_scope == CSA_GIST_SELECTED;
   }
+  m.allow_cluster = num_parts == 0;
   std::string why;
   cudaError_t e = csa::launch_decode(l, q, K, V, dtype == CSA_BF16, idx, count, kmax, head_full, B, Hq,
                                      Hkv, D, T, L, scale, P, P, reinterpret_cast<float*>(ws + w.o),
@@ -791,6 +792,7 @@ csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stre
     m.Vg = d->Vg;
     m.gist_selected = d->gist_scope == CSA_GIST_SELECTED;
   }
+  m.allow_cluster = d->num_parts == 0;
   std::string why;
   cudaError_t e = csa::launch_decode(l, d->q, d->K, d->V, true, d->idx, d->count, d->kmax,
                                      d->head_full, d->B, d->Hq, d->Hkv, d->D, d->T, d->L, d->scale,

@@ -47,6 +47,12 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kDeferMax = 32;  // merges a CTA can postpone to the end of its work
 
+// e^x and ln x on the special-function unit (ex2.approx / lg2.approx): the
+// weights and lse of a merge need no more, and the short instruction
+// sequences keep the end-of-launch merge code small.
+__device__ __forceinline__ float sfu_exp(float x) { return fast_exp2(x * kLog2e); }
+__device__ __forceinline__ float sfu_log(float x) { return __log2f(x) * kLn2; }
+
 struct DecodeParams {
   const void* q;  // [B, Hq, D]
   const float* Kf;  // fp32 path only
@@ -70,8 +76,10 @@ struct DecodeParams {
   float* lse_out;  // [B, Hq] or null
   // phased: full-head units first (no dependency on the selection), then,
   // after griddepcontrol.wait, the sparse units (launched with programmatic
-  // dependent launch behind the selection kernel)
+  // dependent launch behind the selection kernel); pdl: that launch (the
+  // cluster kernel has no phases but waits the same way)
   int phased;
+  int pdl;
   // phased: the last `late` CTAs of the grid take no phase-1 work (they can
   // only start once the selection's CTAs have left their SMs)
   int late;
@@ -363,12 +371,12 @@ __device__ bool merge_unit(const DecodeParams& p, int u, int ns, float* wts, int
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
     float sum = 0.f;
-    for (int sl = lane; sl < ns; sl += 32) sum += expf(wts[g * ns + sl] - mx);
+    for (int sl = lane; sl < ns; sl += 32) sum += sfu_exp(wts[g * ns + sl] - mx);
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
-    const float lse = mx + logf(sum);
+    const float lse = mx + sfu_log(sum);
     __syncwarp();
-    for (int sl = lane; sl < ns; sl += 32) wts[g * ns + sl] = expf(wts[g * ns + sl] - lse);
+    for (int sl = lane; sl < ns; sl += 32) wts[g * ns + sl] = sfu_exp(wts[g * ns + sl] - lse);
     if (lane == 0 && p.lse_out) p.lse_out[row0 + g] = lse;
   }
   if (!sync()) return false;
@@ -432,7 +440,6 @@ struct DecodeShape {
   static constexpr int KV_BYTES = L * D * 2;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES;
   static constexpr int NS = kStageBudget / STAGE_BYTES;
-  static constexpr int BOX_BYTES = L * 128;
   static constexpr int QSLOT_BYTES = kQSlotHeads * D * 2;
 };
 
@@ -495,15 +502,15 @@ __device__ void merge_unit_warp(const DecodeParams& p, int u, int ns) {
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
     float sum = 0.f;
-    for (int s = lane; s < ns; s += 32) sum += expf(__ldcg(ls + s) - mx);
+    for (int s = lane; s < ns; s += 32) sum += sfu_exp(__ldcg(ls + s) - mx);
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
-    const float lse = mx + logf(sum);
+    const float lse = mx + sfu_log(sum);
     if (lane < D4) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       const float4* src = reinterpret_cast<const float4*>(p.o_part + row * p.max_splits * D) + lane;
       for (int s = 0; s < ns; ++s) {
-        const float wgt = expf(__ldcg(ls + s) - lse);
+        const float wgt = sfu_exp(__ldcg(ls + s) - lse);
         const float4 x = __ldcg(src + static_cast<int64_t>(s) * D4);
         acc.x += wgt * x.x;
         acc.y += wgt * x.y;
@@ -605,11 +612,11 @@ __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
     float sum = 0.f;
-    for (int sl = lane; sl < ns; sl += 32) sum += expf(ww[sl] - mx);
+    for (int sl = lane; sl < ns; sl += 32) sum += sfu_exp(ww[sl] - mx);
 #pragma unroll
     for (int x = 16; x > 0; x >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, x);
-    const float lse = mx + logf(sum);
-    for (int sl = lane; sl < ns; sl += 32) ww[sl] = expf(ww[sl] - lse);
+    const float lse = mx + sfu_log(sum);
+    for (int sl = lane; sl < ns; sl += 32) ww[sl] = sfu_exp(ww[sl] - lse);
     __syncwarp();
     if (lane == 0 && p.lse_out) p.lse_out[row0 + g] = lse;
     for (int c4 = lane; c4 < D4; c4 += 32) {
@@ -660,13 +667,13 @@ __device__ __forceinline__ int epilogue_unit(const DecodeParams& p, const float*
     for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + lane]);
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      wn[w] = exp2f(fm[w * 8 + lane] - M);
+      wn[w] = fast_exp2(fm[w * 8 + lane] - M);
       Ls += fl[w * 8 + lane] * wn[w];
     }
     const float inv = 1.0f / Ls;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) wn[w] *= inv;
-    const float lse = (M + log2f(Ls)) * kLn2;
+    const float lse = (M + __log2f(Ls)) * kLn2;
     if (!direct)
       p.lse_part[(row0 + lane) * p.max_splits + slot] = lse;
     else if (p.lse_out)
@@ -712,6 +719,240 @@ __device__ __forceinline__ int epilogue_unit(const DecodeParams& p, const float*
   return __shfl_sync(0xffffffffu, last, 0);
 }
 
+// ---------------------------------------------------------------- producer
+
+// The K/V tensor maps of a launch: raw rows [B*Hkv*T, D] and gist rows.
+struct KVMaps {
+  const CUtensorMap* K;
+  const CUtensorMap* V;
+  const CUtensorMap* Kg;
+  const CUtensorMap* Vg;
+};
+
+// Fill ring slot i % ns (stage at `dst`, barriers full/empty) with one chunk:
+// row >= 0 a raw K/V row block and row < 0 the gist rows -(row + 1).. (both
+// by TMA, issued by lane 0), or gsel >= 0 a gathered gist chunk (all 32
+// lanes).  qu >= 0: unit qu's query rows ride along into q slot `qdst`.
+// Called by the whole producer warp with warp-uniform arguments; false when
+// the wait for the slot ran out of time.
+template <int D, int L>
+__device__ __forceinline__ bool issue_stage(const DecodeParams& p, const KVMaps& m, int64_t i,
+                                            int ns, uint32_t dst, uint32_t full_bar,
+                                            uint32_t empty_bar, int row, int gsel, int qu,
+                                            uint32_t qdst, uint64_t kv_policy,
+                                            uint32_t& cp_stages) {
+  constexpr int KV_BYTES = L * D * 2, STAGE_BYTES = 2 * KV_BYTES, BOX_BYTES = L * 128;
+  const int lane = threadIdx.x & 31;
+  const int s = static_cast<int>(i % ns);
+  const uint32_t fb = full_bar + 8 * s;
+  const uint32_t q_bytes = static_cast<uint32_t>(p.G) * D * 2;
+  const __nv_bfloat16* qsrc = nullptr;
+  if (qu >= 0)
+    qsrc = static_cast<const __nv_bfloat16*>(p.q) +
+           (static_cast<int64_t>(qu / p.Hkv) * p.Hq + (qu % p.Hkv) * p.G) * D;
+  int good = 1;
+  if (lane == 0) {
+    const uint32_t it = static_cast<uint32_t>(i / ns);
+    if (!mbar_wait(empty_bar + 8 * s, (it & 1u) ^ 1u, p.err)) {
+      good = 0;
+    } else if (gsel < 0) {
+      if (cp_stages & (1u << s)) {  // the copies that filled it last were cp.async
+        fence_proxy_async_shared();
+        cp_stages &= ~(1u << s);
+      }
+      mbar_arrive_expect_tx(fb, STAGE_BYTES + (qu >= 0 ? q_bytes : 0u));
+      if (qu >= 0) bulk_load(qdst, qsrc, q_bytes, fb);
+      const bool gist = row < 0;  // rows of a ragged last gist chunk past
+      const int r = gist ? -row - 1 : row;  // the tensor read as zeros
+      const CUtensorMap* mk = gist ? m.Kg : m.K;
+      const CUtensorMap* mv = gist ? m.Vg : m.V;
+#pragma unroll
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_2d_hint(dst + bx * BOX_BYTES, mk, bx * 64, r, fb, kv_policy);
+        tma_load_2d_hint(dst + KV_BYTES + bx * BOX_BYTES, mv, bx * 64, r, fb, kv_policy);
+      }
+    }
+  }
+  good = __shfl_sync(0xffffffffu, good, 0);
+  if (good && gsel >= 0) {  // warp-uniform: a gathered gist chunk
+    gather_gist_rows<D, L>(p, gsel, dst, fb);
+    __syncwarp();  // every lane's pending arrival before the barrier's own
+    if (lane == 0) {
+      cp_stages |= 1u << s;
+      if (qu >= 0) {
+        mbar_arrive_expect_tx(fb, q_bytes);
+        bulk_load(qdst, qsrc, q_bytes, fb);
+      } else {
+        mbar_arrive(fb);
+      }
+    }
+  }
+  return good != 0;
+}
+
+// ---------------------------------------------------------------- per-warp attention
+//
+// A consumer warp takes L/4 tokens of every chunk.  S^T = K q^T runs as
+// mma.m16n8k16 with the tokens as M and the query heads of the GQA group as
+// N (lane l holds heads hA = 2 (l % 4) and hB = hA + 1); the online softmax
+// (log2 domain) stays in registers; P goes into the B layout with movmatrix
+// and O^T += V^T P^T runs as a second mma.
+
+template <int D>
+struct WarpAcc {
+  uint32_t qf[D / 16][2];  // the unit's query heads as B fragments
+  float o[D / 16][4];      // O^T tiles: d = 16 dt + lane/4 (+8), heads hA / hB
+  float m0, m1, l0, l1;    // running max (log2 domain) and sum of heads hA / hB
+};
+
+// Start a unit: its G query rows from a q slot ([8][D] bf16), accumulators zeroed.
+template <int D>
+__device__ __forceinline__ void acc_begin(WarpAcc<D>& w, const __nv_bfloat16* qs, int G,
+                                          int lane) {
+  const int n = lane >> 2;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const int d0 = ks * 16 + 2 * (lane & 3);
+    if (n < G) {
+      w.qf[ks][0] = *reinterpret_cast<const uint32_t*>(qs + n * D + d0);
+      w.qf[ks][1] = *reinterpret_cast<const uint32_t*>(qs + n * D + d0 + 8);
+    } else {
+      w.qf[ks][0] = 0u;
+      w.qf[ks][1] = 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w.o[ks][e] = 0.f;
+  }
+  w.m0 = w.m1 = -INFINITY;
+  w.l0 = w.l1 = 0.f;
+}
+
+// One stage (K at sK, V at sK + L*D*2, each as [L x 64] boxes with the
+// 128-byte swizzle) into the warp's accumulators; rows >= valid take no part.
+template <int D, int L>
+__device__ __forceinline__ void acc_stage(WarpAcc<D>& w, uint32_t sK, int warp, int lane,
+                                          float scale_log2, int valid) {
+  constexpr int TOK_W = L / kConsumerWarps;  // tokens per consumer warp
+  constexpr int MT = TOK_W / 16;             // 16-token m-tiles per warp
+  constexpr int KS = D / 16;                 // k-steps (QK) / d-tiles (PV)
+  constexpr int KV_BYTES = L * D * 2, BOX_BYTES = L * 128;
+  const uint32_t sV = sK + KV_BYTES;
+  const int tok0 = warp * TOK_W;
+  // S^T = K q^T over this warp's tokens
+  float sc[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int bx = ks >> 2, colb = (ks & 3) * 16;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int row = tok0 + mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int col = colb + (lane >> 4) * 8;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(sK + bx * BOX_BYTES + sw128_offset(row, col), a0, a1, a2, a3);
+      mma_bf16_16816(sc[mt], a0, a1, a2, a3, w.qf[ks][0], w.qf[ks][1]);
+    }
+  }
+  if (valid < L) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (tok0 + mt * 16 + (lane >> 2) + (e >> 1) * 8 >= valid) sc[mt][e] = -INFINITY;
+  }
+  // online softmax (log2 domain), per head hA / hB of this lane
+  float cm0 = -INFINITY, cm1 = -INFINITY;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[mt][e] *= scale_log2;
+    cm0 = fmaxf(cm0, fmaxf(sc[mt][0], sc[mt][2]));
+    cm1 = fmaxf(cm1, fmaxf(sc[mt][1], sc[mt][3]));
+  }
+#pragma unroll
+  for (int x = 4; x < 32; x <<= 1) {
+    cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, x));
+    cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, x));
+  }
+  const float mn0 = fmaxf(w.m0, cm0), mn1 = fmaxf(w.m1, cm1);
+  // exponent reference: 0 while every row this warp has seen was masked
+  // (max -inf), so that no -inf - -inf arises
+  const float rf0 = mn0 == -INFINITY ? 0.f : mn0, rf1 = mn1 == -INFINITY ? 0.f : mn1;
+  const float al0 = fast_exp2(w.m0 - rf0), al1 = fast_exp2(w.m1 - rf1);
+  w.m0 = mn0;
+  w.m1 = mn1;
+  uint32_t pb[MT][2];
+  float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const float p0 = fast_exp2(sc[mt][0] - rf0), p1 = fast_exp2(sc[mt][1] - rf1);
+    const float p2 = fast_exp2(sc[mt][2] - rf0), p3 = fast_exp2(sc[mt][3] - rf1);
+    ps0 += p0 + p2;
+    ps1 += p1 + p3;
+    pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+    pb[mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+  }
+  w.l0 = w.l0 * al0 + ps0;
+  w.l1 = w.l1 * al1 + ps1;
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    w.o[dt][0] *= al0;
+    w.o[dt][1] *= al1;
+    w.o[dt][2] *= al0;
+    w.o[dt][3] *= al1;
+  }
+  // O^T += V^T P^T
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const int bx = dt >> 2, colb = (dt & 3) * 16;
+      const int mi = lane >> 3;
+      const int tok = tok0 + mt * 16 + (lane & 7) + (mi >> 1) * 8;
+      const int col = colb + (mi & 1) * 8;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(sV + bx * BOX_BYTES + sw128_offset(tok, col), a0, a1, a2, a3);
+      mma_bf16_16816(w.o[dt], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+    }
+  }
+}
+
+// The warp's (m, l, O) into a flush buffer: O [kConsumerWarps][G][D], then
+// m [kConsumerWarps][8], l [kConsumerWarps][8] (fp32); the sums are reduced
+// over the lanes of a head first.
+template <int D>
+__device__ __forceinline__ void acc_write(WarpAcc<D>& w, float* fo, int G, int warp, int lane) {
+#pragma unroll
+  for (int x = 4; x < 32; x <<= 1) {
+    w.l0 += __shfl_xor_sync(0xffffffffu, w.l0, x);
+    w.l1 += __shfl_xor_sync(0xffffffffu, w.l1, x);
+  }
+  const int hA = 2 * (lane & 3), hB = hA + 1;
+  float* fm = fo + kConsumerWarps * G * D;
+  float* fl = fm + kConsumerWarps * 8;
+  if (lane < 4) {
+    fm[warp * 8 + hA] = w.m0;
+    fm[warp * 8 + hB] = w.m1;
+    fl[warp * 8 + hA] = w.l0;
+    fl[warp * 8 + hB] = w.l1;
+  }
+#pragma unroll
+  for (int dt = 0; dt < D / 16; ++dt) {
+    const int d = dt * 16 + (lane >> 2);
+    if (hA < G) {
+      fo[(warp * G + hA) * D + d] = w.o[dt][0];
+      fo[(warp * G + hA) * D + d + 8] = w.o[dt][2];
+    }
+    if (hB < G) {
+      fo[(warp * G + hB) * D + d] = w.o[dt][1];
+      fo[(warp * G + hB) * D + d + 8] = w.o[dt][3];
+    }
+  }
+}
+
 template <int D, int L>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -721,10 +962,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                        const __grid_constant__ DecodeParams p) {
   using Sh = DecodeShape<D, L>;
   constexpr int NS = Sh::NS;
-  constexpr int TOK_W = L / kConsumerWarps;  // tokens per consumer warp
-  constexpr int MT = TOK_W / 16;             // 16-token m-tiles per warp
-  constexpr int KS = D / 16;                 // k-steps (QK) / d-tiles (PV)
-  constexpr int NBOX = D / 64;
   const DecLayout Y = dec_layout(D, L, p.G, p.U);
   const int G = p.G;
 
@@ -779,8 +1016,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer
-    const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
-    const uint32_t q_bytes = static_cast<uint32_t>(G) * D * 2;
+    const KVMaps maps{&tmK, &tmV, &tmKg, &tmVg};
     // K/V is read once: first out of L2, so that what the kernel reads again
     // (its instructions, parameters, the partials and counters) stays there
     const uint64_t kv_policy = l2_policy_evict_first();
@@ -811,57 +1047,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           const int row_j = __shfl_sync(0xffffffffu, row, j);
           const int qu_j = __shfl_sync(0xffffffffu, qu, j);
           const int gs_j = __shfl_sync(0xffffffffu, gsel, j);
-          const int64_t i = issued;
-          const int s = static_cast<int>(i % NS);
-          const uint32_t fb = full_bar + 8 * s;
-          const uint32_t dst = sbase + s * Sh::STAGE_BYTES;
-          int good = 1;
-          if (lane == 0) {
-            const uint32_t it = static_cast<uint32_t>(i / NS);
-            if (!mbar_wait(empty_bar + 8 * s, (it & 1u) ^ 1u, p.err)) {
-              good = 0;
-            } else if (gs_j < 0) {
-              if (cp_stages & (1u << s)) {  // the copies that filled it last were cp.async
-                fence_proxy_async_shared();
-                cp_stages &= ~(1u << s);
-              }
-              mbar_arrive_expect_tx(fb, Sh::STAGE_BYTES + (qu_j >= 0 ? q_bytes : 0u));
-              if (qu_j >= 0) {
-                const int64_t qrow = static_cast<int64_t>(qu_j / p.Hkv) * p.Hq + (qu_j % p.Hkv) * G;
-                bulk_load(sbase + Y.q_off + s * Sh::QSLOT_BYTES, qg + qrow * D, q_bytes, fb);
-              }
-              const bool gist = row_j < 0;  // rows of a ragged last gist chunk past
-              const int r = gist ? -row_j - 1 : row_j;  // the tensor read as zeros
-              const CUtensorMap* mk = gist ? &tmKg : &tmK;
-              const CUtensorMap* mv = gist ? &tmVg : &tmV;
-#pragma unroll
-              for (int bx = 0; bx < NBOX; ++bx) {
-                tma_load_2d_hint(dst + bx * Sh::BOX_BYTES, mk, bx * 64, r, fb, kv_policy);
-                tma_load_2d_hint(dst + Sh::KV_BYTES + bx * Sh::BOX_BYTES, mv, bx * 64, r, fb,
-                                 kv_policy);
-              }
-            }
-          }
-          good = __shfl_sync(0xffffffffu, good, 0);
-          if (good && gs_j >= 0) {  // warp-uniform: a gathered gist chunk
-            gather_gist_rows<D, L>(p, gs_j, dst, fb);
-            __syncwarp();  // every lane's pending arrival before the barrier's own
-            if (lane == 0) {
-              cp_stages |= 1u << s;
-              if (qu_j >= 0) {
-                const int64_t qrow = static_cast<int64_t>(qu_j / p.Hkv) * p.Hq + (qu_j % p.Hkv) * G;
-                mbar_arrive_expect_tx(fb, q_bytes);
-                bulk_load(sbase + Y.q_off + s * Sh::QSLOT_BYTES, qg + qrow * D, q_bytes, fb);
-              } else {
-                mbar_arrive(fb);
-              }
-            }
-          }
-          issued = __shfl_sync(0xffffffffu, issued + good, 0);
+          const int s = static_cast<int>(issued % NS);
+          const bool good = issue_stage<D, L>(p, maps, issued, NS, sbase + s * Sh::STAGE_BYTES,
+                                              full_bar, empty_bar, row_j, gs_j, qu_j,
+                                              sbase + Y.q_off + s * Sh::QSLOT_BYTES, kv_policy,
+                                              cp_stages);
           if (!good) {
             ok = false;
             break;
           }
+          ++issued;
         }
       }
     }
@@ -981,10 +1176,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (p.merged) zero_empty_units(p, pre, p.phased ? 1 : 0, kConsumerWarps * 32);
   else fill_empty_slots(p, pre, kConsumerWarps * 32);
   const float scale_log2 = p.scale_log2;
-  const int hA = 2 * (lane & 3), hB = hA + 1;
-  uint32_t qf[KS][2];
-  float o[KS][4];
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  WarpAcc<D> acc;
   int cur_u = -1, nflush = 0;
   bool cur_full = false;  // hybrid launches: the current unit is a full-attention one
   int cur_ns = 0;         // hybrid launches: the current unit's selected chunks
@@ -993,37 +1185,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   // Hand this warp's (m, l, O) of unit u to the epilogue warp and go on.
   auto flush_async = [&](int u) -> bool {
-#pragma unroll
-    for (int x = 4; x < 32; x <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, x);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, x);
-    }
     (void)u;
     const int k = Y.nf == 2 ? (nflush & 1) : 0;
     const int use = Y.nf == 2 ? (nflush >> 1) : nflush;
     if (use > 0 && !warp_wait(fb_empty + 8 * k, static_cast<uint32_t>(use - 1) & 1u, p.err))
       return false;
-    float* fo = reinterpret_cast<float*>(smem + Y.fb_off + k * Y.fb_bytes);
-    float* fm = fo + kConsumerWarps * G * D;
-    float* fl = fm + kConsumerWarps * 8;
-    if (lane < 4) {
-      fm[warp * 8 + hA] = m0;
-      fm[warp * 8 + hB] = m1;
-      fl[warp * 8 + hA] = l0;
-      fl[warp * 8 + hB] = l1;
-    }
-#pragma unroll
-    for (int dt = 0; dt < KS; ++dt) {
-      const int d = dt * 16 + (lane >> 2);
-      if (hA < G) {
-        fo[(warp * G + hA) * D + d] = o[dt][0];
-        fo[(warp * G + hA) * D + d + 8] = o[dt][2];
-      }
-      if (hB < G) {
-        fo[(warp * G + hB) * D + d] = o[dt][1];
-        fo[(warp * G + hB) * D + d + 8] = o[dt][3];
-      }
-    }
+    acc_write<D>(acc, reinterpret_cast<float*>(smem + Y.fb_off + k * Y.fb_bytes), G, warp, lane);
     mbar_arrive(fb_full + 8 * k);
     ++nflush;
     return true;
@@ -1065,116 +1232,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         cur_full = hybrid && p.head_full != nullptr && p.head_full[cur_u % p.Hkv];
         if (hybrid && !cur_full) cur_ns = sel_count(p, cur_u);
         // the unit's q arrived with this stage
-        const __nv_bfloat16* qs =
-            reinterpret_cast<const __nv_bfloat16*>(smem + Y.q_off + s * Sh::QSLOT_BYTES);
-        const int n = lane >> 2;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          const int d0 = ks * 16 + 2 * (lane & 3);
-          if (n < G) {
-            qf[ks][0] = *reinterpret_cast<const uint32_t*>(qs + n * D + d0);
-            qf[ks][1] = *reinterpret_cast<const uint32_t*>(qs + n * D + d0 + 8);
-          } else {
-            qf[ks][0] = 0u;
-            qf[ks][1] = 0u;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) o[ks][e] = 0.f;
-        }
-        m0 = m1 = -INFINITY;
-        l0 = l1 = 0.f;
+        acc_begin<D>(acc,
+                     reinterpret_cast<const __nv_bfloat16*>(smem + Y.q_off + s * Sh::QSLOT_BYTES),
+                     G, lane);
       }
-      const uint32_t sK = sbase + s * Sh::STAGE_BYTES;
-      const uint32_t sV = sK + Sh::KV_BYTES;
-      const int tok0 = warp * TOK_W;
-
-      // S^T = K q^T over this warp's tokens
-      float sc[MT][4];
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const int bx = ks >> 2, colb = (ks & 3) * 16;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int row = tok0 + mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int col = colb + (lane >> 4) * 8;
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(sK + bx * Sh::BOX_BYTES + sw128_offset(row, col), a0, a1, a2, a3);
-          mma_bf16_16816(sc[mt], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
-        }
-      }
+      int valid = L;
       if (hybrid && !cur_full) {
         // a hybrid unit's last gist chunk is ragged: rows past its gist rows
         // (the next unit's, zeros past the tensor, or the zero-filled rows of
         // a gathered chunk) take no part
         const int j = static_cast<int>(g - pre[cur_u]) - cur_ns;
-        const int valid = j >= 0 ? gist_rows_of(p, cur_ns) - j * L : L;
-        if (valid < L) {
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (tok0 + mt * 16 + (lane >> 2) + (e >> 1) * 8 >= valid) sc[mt][e] = -INFINITY;
-        }
+        if (j >= 0) valid = min(L, gist_rows_of(p, cur_ns) - j * L);
       }
-      // online softmax (log2 domain), per head hA / hB of this lane
-      float cm0 = -INFINITY, cm1 = -INFINITY;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[mt][e] *= scale_log2;
-        cm0 = fmaxf(cm0, fmaxf(sc[mt][0], sc[mt][2]));
-        cm1 = fmaxf(cm1, fmaxf(sc[mt][1], sc[mt][3]));
-      }
-#pragma unroll
-      for (int x = 4; x < 32; x <<= 1) {
-        cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, x));
-        cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, x));
-      }
-      const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
-      // exponent reference: 0 while every row this warp has seen was masked
-      // (max -inf), so that no -inf - -inf arises
-      const float rf0 = mn0 == -INFINITY ? 0.f : mn0, rf1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float al0 = fast_exp2(m0 - rf0), al1 = fast_exp2(m1 - rf1);
-      m0 = mn0;
-      m1 = mn1;
-      uint32_t pb[MT][2];
-      float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const float p0 = fast_exp2(sc[mt][0] - rf0), p1 = fast_exp2(sc[mt][1] - rf1);
-        const float p2 = fast_exp2(sc[mt][2] - rf0), p3 = fast_exp2(sc[mt][3] - rf1);
-        ps0 += p0 + p2;
-        ps1 += p1 + p3;
-        pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
-        pb[mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
-      }
-      l0 = l0 * al0 + ps0;
-      l1 = l1 * al1 + ps1;
-#pragma unroll
-      for (int dt = 0; dt < KS; ++dt) {
-        o[dt][0] *= al0;
-        o[dt][1] *= al1;
-        o[dt][2] *= al0;
-        o[dt][3] *= al1;
-      }
-      // O^T += V^T P^T
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-        for (int dt = 0; dt < KS; ++dt) {
-          const int bx = dt >> 2, colb = (dt & 3) * 16;
-          const int mi = lane >> 3;
-          const int tok = tok0 + mt * 16 + (lane & 7) + (mi >> 1) * 8;
-          const int col = colb + (mi & 1) * 8;
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_trans(sV + bx * Sh::BOX_BYTES + sw128_offset(tok, col), a0, a1, a2, a3);
-          mma_bf16_16816(o[dt], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
-        }
-      }
+      acc_stage<D, L>(acc, sbase + s * Sh::STAGE_BYTES, warp, lane, scale_log2, valid);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar + 8 * s);
     }
@@ -1182,6 +1252,212 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   if (ok && cur_u >= 0) ok = flush_async(cur_u);
   if (!p.merged) return;
   final_merges(threadIdx.x);
+}
+
+// ------------------------------------------------------------------ cluster path
+//
+// Steps with few chunks per unit: one thread-block cluster of CS CTAs per
+// unit, CTA r of the cluster streaming the r-th of CS equal parts of the
+// unit's list (its chunks, then its gist chunks).  The parts are combined
+// through distributed shared memory: each CTA folds its four consumer
+// warps' (m, l, O) into one partial and writes it into a slot of the
+// cluster's first CTA, which writes the unit's output rows and lse after a
+// cluster barrier.  No partial leaves the cluster, so there is no global
+// workspace traffic, arrival counter or separate merge.  Warps 0-3 consume,
+// warp 4 produces (as in the persistent kernel).  Both cluster barriers are
+// reached by every thread on every path (a timed-out wait only skips work),
+// so a wait that ran out of time cannot leave the cluster waiting.
+
+constexpr int kClusterThreads = (kConsumerWarps + 1) * 32;
+constexpr int kClusterMax = 8;  // portable cluster size
+
+// Shared memory of the cluster kernel, offsets from the 1024-aligned base:
+// K/V stages | q slot | flush buffer | CS partial slots | mbarriers.
+struct ClLayout {
+  int ns;                                   // ring stages
+  int q_off, fo_off, part_off, part_stride, bar_off;
+  size_t total;
+};
+
+__host__ __device__ inline ClLayout cl_layout(int D, int L, int G, int CS) {
+  const int stage_bytes = 2 * L * D * 2;
+  ClLayout y;
+  const int fo_bytes = (kConsumerWarps * G * D + 2 * kConsumerWarps * 8) * 4;
+  y.part_stride = (G * D + 16) * 4;  // per slot: M [8], Lsum [8], O [G][D] (fp32)
+  const int fixed = kQSlotHeads * D * 2 + ((fo_bytes + 127) & ~127) +
+                    ((CS * y.part_stride + 127) & ~127) + 64 * 8;
+  int ns = kStageBudget / stage_bytes;
+  const int room = static_cast<int>(kMaxDynSmem) - 1024 - fixed;
+  if (ns * stage_bytes > room) ns = room / stage_bytes;
+  y.ns = ns;
+  y.q_off = ns * stage_bytes;
+  y.fo_off = y.q_off + kQSlotHeads * D * 2;
+  y.part_off = y.fo_off + ((fo_bytes + 127) & ~127);
+  y.bar_off = y.part_off + ((CS * y.part_stride + 127) & ~127);
+  y.total = 1024 + static_cast<size_t>(y.bar_off) + (2 * ns + 2) * 8;
+  return y;
+}
+
+template <int D, int L>
+__global__ void __launch_bounds__(kClusterThreads, 1)
+    decode_cluster_kernel(const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV,
+                          const __grid_constant__ CUtensorMap tmKg,
+                          const __grid_constant__ CUtensorMap tmVg,
+                          const __grid_constant__ DecodeParams p) {
+  cluster_arrive_relaxed();  // every CTA of the cluster has started by the matching wait
+  const int G = p.G;
+  const int CS = static_cast<int>(cluster_size());
+  const int rank = static_cast<int>(cluster_rank());
+  const int u = blockIdx.y;
+  const ClLayout Y = cl_layout(D, L, G, CS);
+  const int NS = Y.ns;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t full_bar = sbase + Y.bar_off;
+  const uint32_t empty_bar = full_bar + NS * 8;
+  const uint32_t fo_bar = empty_bar + NS * 8;
+  float* fo = reinterpret_cast<float*>(smem + Y.fo_off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < NS; ++k) {
+      mbar_init(full_bar + 8 * k, 1);
+      mbar_init(empty_bar + 8 * k, kConsumerWarps);
+    }
+    mbar_init(fo_bar, kConsumerWarps * 32);
+    fence_barrier_init();
+  }
+  if (warp == kConsumerWarps && lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+    if (p.n_gist > 0) {
+      prefetch_tensormap(&tmKg);
+      prefetch_tensormap(&tmVg);
+    }
+  }
+  __syncthreads();
+  const bool full = p.head_full != nullptr && p.head_full[u % p.Hkv];
+  if (!full && p.pdl) grid_dependency_wait();  // the selection's lists are complete
+  const int n_all = unit_count(p, u);
+  const int lo = static_cast<int>(static_cast<int64_t>(n_all) * rank / CS);
+  const int hi = static_cast<int>(static_cast<int64_t>(n_all) * (rank + 1) / CS);
+  const int STAGE_BYTES = 2 * L * D * 2;
+  bool ok = true;
+
+  if (warp == kConsumerWarps) {
+    // ---------------------------------------------------------------- producer
+    const KVMaps maps{&tmK, &tmV, &tmKg, &tmVg};
+    const uint64_t kv_policy = l2_policy_evict_first();
+    uint32_t cp_stages = 0;
+    int64_t issued = 0;
+    for (int g0 = lo; g0 < hi && ok; g0 += 32) {
+      int row = 0, gsel = -1;
+      if (g0 + lane < hi) row = unit_row(p, u, g0 + lane, L, &gsel);
+      const int nb = min(32, hi - g0);
+      for (int j = 0; j < nb; ++j) {
+        const int row_j = __shfl_sync(0xffffffffu, row, j);
+        const int gs_j = __shfl_sync(0xffffffffu, gsel, j);
+        const int s = static_cast<int>(issued % NS);
+        if (!issue_stage<D, L>(p, maps, issued, NS, sbase + s * STAGE_BYTES, full_bar,
+                               empty_bar, row_j, gs_j, g0 + j == lo ? u : -1,
+                               sbase + Y.q_off, kv_policy, cp_stages)) {
+          ok = false;
+          break;
+        }
+        ++issued;
+      }
+    }
+    // no copy may still be landing when the CTA retires
+    if (lane == 0) {
+      const int64_t first = issued > NS ? issued - NS : 0;
+      for (int64_t i = first; i < issued; ++i)
+        mbar_wait(full_bar + 8 * static_cast<int>(i % NS), static_cast<uint32_t>(i / NS) & 1u,
+                  p.err);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- consumers
+    WarpAcc<D> acc;
+    acc.m0 = acc.m1 = -INFINITY;
+    acc.l0 = acc.l1 = 0.f;
+    for (int ks = 0; ks < D / 16; ++ks)
+      for (int e = 0; e < 4; ++e) acc.o[ks][e] = 0.f;
+    const bool hybrid = (p.n_gist > 0 || p.gist_sel) && !full;
+    const int ns_sel = hybrid ? sel_count(p, u) : 0;
+    for (int g = lo; g < hi; ++g) {
+      const int64_t i = g - lo;
+      const int s = static_cast<int>(i % NS);
+      if (!warp_wait(full_bar + 8 * s, static_cast<uint32_t>(i / NS) & 1u, p.err)) {
+        ok = false;
+        break;
+      }
+      if (g == lo)  // the unit's q arrived with the first stage
+        acc_begin<D>(acc, reinterpret_cast<const __nv_bfloat16*>(smem + Y.q_off), G, lane);
+      int valid = L;
+      if (hybrid) {
+        const int j = g - ns_sel;
+        if (j >= 0) valid = min(L, gist_rows_of(p, ns_sel) - j * L);
+      }
+      acc_stage<D, L>(acc, sbase + s * STAGE_BYTES, warp, lane, p.scale_log2, valid);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar + 8 * s);
+    }
+    acc_write<D>(acc, fo, G, warp, lane);
+    mbar_arrive(fo_bar);
+    const bool have = warp_wait(fo_bar, 0u, p.err);
+    // this CTA's part: the four warps folded into one (M, Lsum, O) per head
+    const float* fm = fo + kConsumerWarps * G * D;
+    const float* fl = fm + kConsumerWarps * 8;
+    cluster_wait();  // (phase 1) every CTA of the cluster is running
+    const uint32_t slot = cluster_map(smem_u32(smem + Y.part_off + rank * Y.part_stride), 0);
+    const int tid = threadIdx.x;  // 0 .. 127
+    for (int e = tid; e < G * D && have; e += kConsumerWarps * 32) {
+      const int g = e / D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, fm[w * 8 + g]);
+      float O = 0.f, Ls = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float wt = fast_exp2(fm[w * 8 + g] - M);
+          O += fo[(w * G + g) * D + (e % D)] * wt;
+          Ls += fl[w * 8 + g] * wt;
+        }
+      }
+      st_cluster_f32(slot + (16 + e) * 4, O);
+      if (e % D == 0) {
+        st_cluster_f32(slot + g * 4, M);
+        st_cluster_f32(slot + (8 + g) * 4, Ls);
+      }
+    }
+  }
+  if (warp == kConsumerWarps) cluster_wait();  // (phase 1) for the producer warp
+  cluster_arrive();  // (phase 2) the parts are in the first CTA's slots
+  cluster_wait();
+  if (rank != 0) return;
+  // ---------------------------------------------------------------- the unit's rows
+  const float* part = reinterpret_cast<const float*>(smem + Y.part_off);
+  const int pst = Y.part_stride / 4;
+  const int64_t row0 = static_cast<int64_t>(u / p.Hkv) * p.Hq + (u % p.Hkv) * G;
+  for (int e = threadIdx.x; e < G * D; e += kClusterThreads) {
+    const int g = e / D;
+    float M = -INFINITY;
+    for (int r = 0; r < CS; ++r) M = fmaxf(M, part[r * pst + g]);
+    float O = 0.f, Ls = 0.f;
+    if (M != -INFINITY) {
+      for (int r = 0; r < CS; ++r) {
+        const float wt = fast_exp2(part[r * pst + g] - M);
+        O += part[r * pst + 16 + e] * wt;
+        Ls += part[r * pst + 8 + g] * wt;
+      }
+    }
+    store_out(p, row0 * D + e, Ls > 0.f ? O / Ls : 0.f);
+    if (e % D == 0 && p.lse_out)
+      p.lse_out[row0 + g] = Ls > 0.f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+  }
 }
 
 // ------------------------------------------------------------------ fp32 path
@@ -1420,7 +1696,7 @@ cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, c
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sh));
   if (e != cudaSuccess) return e;
-  if (!p.phased) {
+  if (!p.pdl) {
     fn<<<P, kDecodeThreads, sh, l.stream>>>(tmK, tmV, tmKg, tmVg, p);
     return cudaGetLastError();
   }
@@ -1438,6 +1714,66 @@ cudaError_t launch_bf16(const Launch& l, const DecodeParams& p, const void* K, c
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, fn, tmK, tmV, tmKg, tmVg, p);
+}
+
+template <int D, int L>
+cudaError_t launch_cluster(const Launch& l, const DecodeParams& p, const void* K, const void* V,
+                           const void* Kg, const void* Vg, int B, int Hkv, int CS,
+                           std::string* why) {
+  CUtensorMap tmK, tmV, tmKg, tmVg;
+  const uint64_t rows = static_cast<uint64_t>(B) * Hkv * p.T;
+  if (!make_tmap_bf16_2d(&tmK, K, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tmV, V, rows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+  if (p.n_gist > 0) {
+    const uint64_t grows = static_cast<uint64_t>(B) * Hkv * p.gist_rows;
+    if (!make_tmap_bf16_2d(&tmKg, Kg, grows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tmVg, Vg, grows, D, D, L, 64, why)) return cudaErrorInvalidValue;
+  } else {
+    tmKg = tmK;
+    tmVg = tmV;
+  }
+  const size_t sh = cl_layout(D, L, p.G, CS).total;
+  auto fn = decode_cluster_kernel<D, L>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sh));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, p.U);
+  cfg.blockDim = dim3(kClusterThreads);
+  cfg.dynamicSmemBytes = sh;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  int na = 1;
+  if (p.pdl) {  // behind the selection: wait for it on the device (griddepcontrol.wait)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    na = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, fn, tmK, tmV, tmKg, tmVg, p);
+}
+
+// Cluster size for the cluster path, or 0 for the persistent one.  Without
+// full-attention heads (which the host cannot see without reading device
+// memory) and with at most ~512 KB of K/V per CTA at the largest possible
+// list (kmax chunks plus the gist chunks), CS is the largest power of two
+// <= 8 with B*Hkv*CS CTAs on the SMs.
+int cluster_size_for(const DecodeParams& p, bool head_full, int num_sms) {
+  if (head_full || p.U <= 0 || p.U > 65535) return 0;
+  int CS = kClusterMax;
+  while (CS > 1 && static_cast<int64_t>(p.U) * CS > num_sms) CS >>= 1;
+  if (static_cast<int64_t>(p.U) * CS > num_sms) return 0;
+  int n_max = std::min(p.C, p.kmax);
+  n_max += p.gist_sel ? (std::min(p.C, p.kmax) + p.L - 1) / p.L : p.n_gist;
+  const int64_t per_cta = static_cast<int64_t>((n_max + CS - 1) / CS) * 2 * p.L * p.D * 2;
+  if (per_cta > 512 * 1024) return 0;
+  if (cl_layout(p.D, p.L, p.G, CS).ns < 2) return 0;
+  return CS;
 }
 
 }  // namespace
@@ -1465,7 +1801,8 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
     p.out = merge->out;
     p.out_bf16 = merge->out_bf16 ? 1 : 0;
     p.lse_out = merge->lse_out;
-    p.phased = (merge->phased && bf16) ? 1 : 0;
+    p.pdl = (merge->phased && bf16) ? 1 : 0;
+    p.phased = p.pdl;
     p.late = p.phased ? merge->late : 0;
     if (merge->Kg != nullptr && bf16) {
       if (merge->gist_selected) {
@@ -1516,6 +1853,15 @@ cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const v
   }
   const void* Kg = merge != nullptr ? merge->Kg : nullptr;
   const void* Vg = merge != nullptr ? merge->Vg : nullptr;
+  const int CS = (merge != nullptr && merge->allow_cluster)
+                     ? cluster_size_for(p, head_full != nullptr, l.num_sms)
+                     : 0;
+  if (CS > 0) {
+    if (D == 128 && L == 128) return launch_cluster<128, 128>(l, p, K, V, Kg, Vg, B, Hkv, CS, why);
+    if (D == 128 && L == 64) return launch_cluster<128, 64>(l, p, K, V, Kg, Vg, B, Hkv, CS, why);
+    if (D == 64 && L == 128) return launch_cluster<64, 128>(l, p, K, V, Kg, Vg, B, Hkv, CS, why);
+    return launch_cluster<64, 64>(l, p, K, V, Kg, Vg, B, Hkv, CS, why);
+  }
   if (D == 128 && L == 128) return launch_bf16<128, 128>(l, p, K, V, Kg, Vg, B, Hkv, P, why);
   if (D == 128 && L == 64) return launch_bf16<128, 64>(l, p, K, V, Kg, Vg, B, Hkv, P, why);
   if (D == 64 && L == 128) return launch_bf16<64, 128>(l, p, K, V, Kg, Vg, B, Hkv, P, why);

@@ -105,6 +105,10 @@ struct MergeOut {
   const void* Kg = nullptr;
   const void* Vg = nullptr;
   bool gist_selected = false;
+  // the caller left the number of pieces to the library: steps with few
+  // chunks per unit and no full-attention heads may run as one cluster of
+  // CTAs per unit (its parts combined in distributed shared memory)
+  bool allow_cluster = false;
 };
 constexpr int kMergedMaxParts = 256;
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,

@@ -36,13 +36,15 @@ namespace csa {
 namespace {
 
 constexpr int kPfThreads = 384;
-constexpr int kNS = 5;                         // K/V stages
+constexpr int kNS = 4;                         // K/V stages
 constexpr int kQHalfBytes = 128 * 128 * 2;     // 32 KB: one 128-row half of the Q tile
 constexpr int kKVBytes = 64 * 128 * 2;         // 16 KB per K (or V) chunk
 constexpr int kStageBytes = 2 * kKVBytes;
 constexpr int kQOff = 0;
 constexpr int kKVOff = 2 * kQHalfBytes;
-constexpr int kBarOff = kKVOff + kNS * kStageBytes;
+constexpr int kOStageBytes = 16384;            // per half: 64 output columns of its 128 rows
+constexpr int kOOff = kKVOff + kNS * kStageBytes;
+constexpr int kBarOff = kOOff + 2 * kOStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
@@ -93,6 +95,30 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Bulk tensor store of a [64 x 64] bf16 box from shared memory (128-byte
+// swizzle) at (col, row) of the output map; completion tracked per thread
+// by bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The shared-memory sources of this thread's stores have been read.
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// This thread's stores are complete.
+__device__ __forceinline__ void bulk_wait0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 #define CSA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
@@ -188,7 +214,8 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -203,7 +230,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t p_full = s_free + 16;                      // [2]
   const uint32_t pv_done = p_full + 16;                     // [2]
   const uint32_t drain = pv_done + 16;                      // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + (drain + 16 - bar));
+  const uint32_t o_full = drain + 16;                       // [2] a half's staged O columns
+  const uint32_t o_free = o_full + 16;                      // [2] ... have been read by the store
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + (o_free + 16 - bar));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -221,6 +250,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     mbar_init(drain, 1);
     mbar_init(drain + 8, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(o_full + 8 * h, 128);
+      mbar_init(o_free + 8 * h, 1);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -378,7 +411,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int g = half * 2 + (r >> 6);  // query head within the group
     const int i = r & 63;               // row within the tile
     const float sl = p.scale_log2;
-    uint32_t s_cnt = 0, pv_phase = 0;
+    uint32_t s_cnt = 0, pv_phase = 0, o_cnt = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       int b, h, t;
@@ -507,30 +540,75 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       pv_phase ^= 1u;
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
-      // two 32-column loads in flight at a time
+      // O / l as bf16 into this half's staging area, laid out as the output
+      // map's [64 x 64] boxes (128-byte swizzle), kOStageBytes / 256 columns
+      // per round; one thread then writes the boxes with bulk tensor stores.
+      constexpr int CW = kOStageBytes / 256, NBX = CW / 64;
+      const uint32_t so = sb + kOOff + half * kOStageBytes;
+      const uint32_t srow = so + (r >> 6) * NBX * 8192 + i * 128;
 #pragma unroll 1
-      for (int cc = 0; cc < 128; cc += 64) {
-        uint32_t ov[2][32];
-        tmem_ld32(tO + cc, ov[0]);
-        tmem_ld32(tO + cc + 32, ov[1]);
-        tmem_wait_ld();
+      for (int cc = 0; cc < 128; cc += CW) {
+        uint32_t pk[CW / 2];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[16];
+        for (int c0 = 0; c0 < CW; c0 += 64) {
+          uint32_t ov[2][32];
+          tmem_ld32(tO + cc + c0, ov[0]);
+          tmem_ld32(tO + cc + c0 + 32, ov[1]);
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(ov[hh][2 * e]) * inv,
-                                __uint_as_float(ov[hh][2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc + 32 * hh);
+          for (int e = 0; e < 32; ++e)
+            pk[c0 / 2 + e] = pack_bf16x2(__uint_as_float(ov[e >> 4][2 * (e & 15)]) * inv,
+                                         __uint_as_float(ov[e >> 4][2 * (e & 15) + 1]) * inv);
+        }
+        // the area is free once the bulk store of the previous round has read it
+        if (o_cnt > 0) {
+          if (r == 0) {
+            bulk_wait_read0();
+            mbar_arrive(o_free + 8 * half);
+          }
+          __syncwarp();
+          if (!warp_wait(o_free + 8 * half, (o_cnt - 1) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+        }
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        for (int j = 0; j < CW / 8; ++j) {
+          const uint32_t dst = srow + (j >> 3) * 8192 + (((j & 7) ^ (i & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[4 * j]),
+                       "r"(pk[4 * j + 1]), "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();  // the writes, for the bulk store
+        mbar_arrive(o_full + 8 * half);
+        if (r == 0) {
+          if (mbar_wait(o_full + 8 * half, o_cnt & 1u, p.err)) {
+            const int orow0 = b * p.S + t * 64;
+#pragma unroll
+            for (int gq = 0; gq < 2; ++gq)
+#pragma unroll
+              for (int bx = 0; bx < NBX; ++bx)
+                tma_store_2d(&tmO, so + (gq * NBX + bx) * 8192,
+                             (h * 4 + half * 2 + gq) * 128 + cc + bx * 64, orow0);
+            bulk_commit();
+          } else {
+            ok = false;
+          }
+        }
+        __syncwarp();
+        ++o_cnt;
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
         }
       }
+      if (!ok) break;
       // the next unit's first PV overwrites O: it is issued after this
       // warpgroup's next p_full arrival, which follows these loads
       tc_fence_before();
     }
+    if (r == 0) bulk_wait0();  // the last bulk stores are complete before the CTA retires
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -548,7 +626,10 @@ cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const 
   (void)D;
   (void)tile_m;
   (void)L;
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ, tmK, tmV, tmO;
+  if (!make_tmap_bf16_2d(&tmO, O, static_cast<uint64_t>(B) * S, static_cast<uint64_t>(Hq) * 128,
+                         static_cast<uint64_t>(Hq) * 128, 64, 64, why))
+    return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tmQ, Q, static_cast<uint64_t>(B) * S, static_cast<uint64_t>(Hq) * 128,
                          static_cast<uint64_t>(Hq) * 128, 64, 64, why))
     return cudaErrorInvalidValue;
@@ -575,7 +656,7 @@ cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const 
                                        kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = std::min(n_units, l.num_sms);
-  prefill_kernel<<<grid, kPfThreads, kSmemBytes, l.stream>>>(tmQ, tmK, tmV, p);
+  prefill_kernel<<<grid, kPfThreads, kSmemBytes, l.stream>>>(tmQ, tmK, tmV, tmO, p);
   return cudaGetLastError();
 }
 

@@ -1189,6 +1189,295 @@ __global__ void __launch_bounds__(kSelThreads) score_select_topp_kernel(
               count, kmax, n_p_out, SN, u, s, bs);
 }
 
+// ---------------------------------------------------------------- cluster score + top-k
+//
+// Short selections: one cluster of CS CTAs per unit.  CTA r scores the r-th
+// of CS equal ranges of the unit's chunks (one round of summary loads) and
+// keeps its best min(k_free, candidates) by rank: the 64-bit composites
+// (score key << 32 | ~index) are unique, so a chunk is kept when fewer than
+// k_free composites of the range exceed its own.  The kept candidates meet
+// in the first CTA's shared memory, which ranks them again the same way,
+// adds the forced chunks and writes the ascending list.  The result is the
+// unit's top-k: a chunk among the best k_free overall is among the best
+// k_free of its own range.
+
+constexpr int kClSelThreads = 256;
+constexpr int kClRangeMax = 512;  // chunks scored by one CTA
+constexpr int kClCandMax = 512;   // candidates meeting in the first CTA
+constexpr int kClRowBatch = 16;   // summary rows per warp in flight
+
+// One warp's round of summary rows: local rows base + b * RPI + (lane /
+// (DS/4)), b < kClRowBatch, each lane holding one float4 of its row.
+template <int DS>
+__device__ __forceinline__ void rows_issue(const float* __restrict__ summ_u, int lo, int n,
+                                           const int* rows, int base, float4 (&v)[kClRowBatch]) {
+  constexpr int LPR = DS / 4, RPI = 32 / LPR;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane % LPR, rsub = lane / LPR;
+#pragma unroll
+  for (int b = 0; b < kClRowBatch; ++b) {
+    const int i = base + b * RPI + rsub;
+    const int r = i < n ? (rows ? rows[lo + i] : lo + i) : 0;
+    v[b] = i < n ? __ldg(reinterpret_cast<const float4*>(summ_u + static_cast<int64_t>(r) * DS) + sub)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+template <int DS>
+__device__ __forceinline__ int rows_first(int n) {
+  constexpr int RPI = 32 / (DS / 4);
+  return (threadIdx.x >> 5) * RPI * kClRowBatch;
+}
+
+// Composite keys of n summary rows of a unit (row of local index i: lo + i,
+// or rows[lo + i] when a row list is given) against the (projected,
+// group-summed) query qv; forced chunks (skip_forced) get 0.  `pre` holds
+// this warp's first round when `prefetched` (rows_issue before the query
+// was ready).
+template <int DS>
+__device__ __forceinline__ void cluster_scores(const float* __restrict__ summ_u, int lo, int n,
+                                               int C, const float* qv, int n_sink, int n_local,
+                                               uint64_t* comp, const int* rows, bool skip_forced,
+                                               const float4 (&pre)[kClRowBatch], bool prefetched) {
+  constexpr int LPR = DS / 4, RPI = 32 / LPR;  // lanes per row, rows per warp step
+  const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int sub = lane % LPR, rsub = lane / LPR;
+  const float4 q4 = make_float4(qv[sub * 4], qv[sub * 4 + 1], qv[sub * 4 + 2], qv[sub * 4 + 3]);
+  const int first = rows_first<DS>(n);
+  for (int base = first; base < n; base += nw * RPI * kClRowBatch) {
+    float4 v[kClRowBatch];
+    if (prefetched && base == first) {
+#pragma unroll
+      for (int b = 0; b < kClRowBatch; ++b) v[b] = pre[b];
+    } else {
+      rows_issue<DS>(summ_u, lo, n, rows, base, v);
+    }
+#pragma unroll
+    for (int b = 0; b < kClRowBatch; ++b) {
+      float x = v[b].x * q4.x + v[b].y * q4.y + v[b].z * q4.z + v[b].w * q4.w;
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      const int i = base + b * RPI + rsub;
+      if (sub == 0 && i < n) {
+        const int c = rows ? rows[lo + i] : lo + i;
+        comp[i] = (skip_forced && is_forced(c, C, n_sink, n_local)) ? 0ull
+                                                                     : composite(float_key(x), c);
+      }
+    }
+  }
+}
+
+// comp[0, n) -> kept[0, *n_kept): the composites with fewer than k of the
+// others above them (all composites distinct, 0 = none).  Ends with a barrier.
+__device__ __forceinline__ void rank_keep(const uint64_t* comp, int n, int k, uint64_t* kept,
+                                          int* n_kept) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint64_t me = comp[i];
+    if (me == 0ull) continue;
+    int above = 0;
+    for (int j = 0; j < n; ++j) above += comp[j] > me;
+    if (above < k) kept[atomicAdd(n_kept, 1)] = me;
+  }
+  __syncthreads();
+}
+
+// The first CTA's ascending list of the chosen chunks sel[0, n_sel) and the
+// forced ones (the first n_sink and last n_local of C), written to the
+// unit's index row.  The chunks are distinct; `buf` has room for all.
+__device__ void emit_with_forced(int32_t* buf, int n_sel, int C, int n_sink, int n_local,
+                                 int32_t* row, int32_t* cnt, int kmax) {
+  const int ns_ = min(n_sink, C), loc0 = max(C - n_local, ns_);
+  for (int j = threadIdx.x; j < ns_; j += blockDim.x) buf[n_sel + j] = j;
+  for (int j = threadIdx.x; j < C - loc0; j += blockDim.x) buf[n_sel + ns_ + j] = loc0 + j;
+  const int total = n_sel + ns_ + (C - loc0);
+  __syncthreads();
+  // each chunk's place is the number of smaller ones
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int me = buf[i];
+    int pos = 0;
+    for (int j = 0; j < total; ++j) pos += buf[j] < me;
+    if (pos < kmax) row[pos] = me;
+  }
+  for (int i = total + threadIdx.x; i < kmax; i += blockDim.x) row[i] = -1;
+  if (threadIdx.x == 0) *cnt = min(total, kmax);
+}
+
+template <int DS>
+__global__ void __launch_bounds__(kClSelThreads) score_select_topk_cluster_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ proj, int R,
+    const float* __restrict__ summ, int Hq, int Hkv, int D, int C,
+    const uint8_t* __restrict__ head_full, int k_free, int n_sink, int n_local,
+    int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
+  allow_dependent_launch();
+  cluster_arrive_relaxed();  // every CTA of the cluster runs by the matching wait
+  __shared__ FusedSmem f;
+  __shared__ uint64_t comp[kClRangeMax];
+  __shared__ uint64_t kept[kClRangeMax];
+  __shared__ uint64_t cand[kClCandMax];
+  __shared__ int32_t out_l[kClCandMax + 64];
+  __shared__ int n_kept, n_out;
+  const int CS = static_cast<int>(cluster_size());
+  const int rank = static_cast<int>(cluster_rank());
+  const int u = blockIdx.y, h = u % Hkv, b = u / Hkv, G = Hq / Hkv;
+  const int lo = static_cast<int>(static_cast<int64_t>(C) * rank / CS);
+  const int n = static_cast<int>(static_cast<int64_t>(C) * (rank + 1) / CS) - lo;
+  const int KL = (k_free < (C + CS - 1) / CS) ? k_free : (C + CS - 1) / CS;  // slots per CTA
+  const bool full = head_full != nullptr && head_full[h];
+  if (threadIdx.x == 0) n_kept = 0;
+  if (!full) {
+    const float* summ_u = summ + static_cast<int64_t>(u) * C * DS;
+    float4 pre[kClRowBatch];
+    rows_issue<DS>(summ_u, lo, n, nullptr, rows_first<DS>(n), pre);  // in flight with the query
+    unit_query(q, q_bf16, static_cast<int64_t>(b) * Hq + h * G, G, D, proj, R, f.qs, f.qv,
+               f.part);  // ends with a barrier
+    cluster_scores<DS>(summ_u, lo, n, C, proj ? f.qv : f.qs, n_sink, n_local, comp, nullptr, true,
+                       pre, true);
+    __syncthreads();
+    rank_keep(comp, n, k_free, kept, &n_kept);
+  }
+  __syncthreads();
+  cluster_wait();  // (phase 1)
+  if (!full) {  // this CTA's kept candidates into its slots of the first CTA (zeros pad)
+    const uint32_t dst = cluster_map(smem_u32(cand + rank * KL), 0);
+    const int nk = n_kept;
+    for (int i = threadIdx.x; i < KL; i += blockDim.x)
+      st_cluster_u64(dst + i * 8, i < nk ? kept[i] : 0ull);
+  }
+  cluster_arrive();  // (phase 2)
+  cluster_wait();
+  if (rank != 0) return;
+  int32_t* row = idx + static_cast<int64_t>(u) * kmax;
+  if (full) {  // full heads read every chunk: no list
+    for (int i = threadIdx.x; i < kmax; i += blockDim.x) row[i] = -1;
+    if (threadIdx.x == 0) count[u] = 0;
+    return;
+  }
+  // the unit's best k_free among the candidates, then the forced chunks
+  const int nc = CS * KL;
+  if (threadIdx.x == 0) n_out = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+    const uint64_t me = cand[i];
+    if (me == 0ull) continue;
+    int above = 0;
+    for (int j = 0; j < nc; ++j) above += cand[j] > me;
+    if (above < k_free) out_l[atomicAdd(&n_out, 1)] = comp_index(me);
+  }
+  __syncthreads();
+  emit_with_forced(out_l, n_out, C, n_sink, n_local, row, count + u, kmax);
+}
+
+// Two-level selection by a cluster of CS CTAs per unit: the meta-chunks'
+// scores split over the CTAs, each keeping its best by rank; the first CTA
+// ranks the kept metas and hands the ascending list of the top_meta best to
+// every CTA of the cluster; the children of those metas split over the CTAs
+// the same way (forced chunks out of the pool); the first CTA ranks the kept
+// children and writes them with the forced chunks, ascending.
+__global__ void __launch_bounds__(kClSelThreads) select_hier_cluster_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ meta,
+    const float* __restrict__ summ, int Hq, int Hkv, int D, int C, int Gm, int top_meta,
+    int k_free, int n_sink, int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count,
+    int kmax) {
+  allow_dependent_launch();
+  cluster_arrive_relaxed();
+  __shared__ float qs[128];
+  __shared__ uint64_t comp[kClRangeMax];
+  __shared__ uint64_t kept[kClRangeMax];
+  __shared__ uint64_t cand[kClCandMax];
+  __shared__ uint8_t chosen[kClCandMax];
+  __shared__ int32_t mlist[kClRangeMax];
+  __shared__ int32_t out_l[kClCandMax + 64];
+  __shared__ int n_kept, n_out;
+  const int CS = static_cast<int>(cluster_size());
+  const int rank = static_cast<int>(cluster_rank());
+  const int u = blockIdx.y, h = u % Hkv, b = u / Hkv, G = Hq / Hkv;
+  const int M = C / Gm, k1 = min(top_meta, M), NCH = k1 * Gm;
+  // level 1: this CTA's share of the metas (every meta is a candidate); its
+  // rows are in flight while the query is summed
+  const int lo1 = static_cast<int>(static_cast<int64_t>(M) * rank / CS);
+  const int n1 = static_cast<int>(static_cast<int64_t>(M) * (rank + 1) / CS) - lo1;
+  const int KL1 = min(k1, (M + CS - 1) / CS);
+  const float* meta_u = meta + static_cast<int64_t>(u) * M * D;
+  float4 pre[kClRowBatch];
+  rows_issue<128>(meta_u, lo1, n1, nullptr, rows_first<128>(n1), pre);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int g = 0; g < G; ++g) {
+      const int64_t off = (static_cast<int64_t>(b) * Hq + h * G + g) * D + d;
+      acc += q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
+                    : static_cast<const float*>(q)[off];
+    }
+    qs[d] = acc;
+  }
+  if (threadIdx.x == 0) n_kept = 0;
+  __syncthreads();
+  cluster_scores<128>(meta_u, lo1, n1, C, qs, 0, 0, comp, nullptr, false, pre, true);
+  __syncthreads();
+  rank_keep(comp, n1, k1, kept, &n_kept);
+  cluster_wait();  // (phase 1)
+  {
+    const uint32_t dst = cluster_map(smem_u32(cand + rank * KL1), 0);
+    for (int i = threadIdx.x; i < KL1; i += blockDim.x)
+      st_cluster_u64(dst + i * 8, i < n_kept ? kept[i] : 0ull);
+  }
+  cluster_arrive();  // (phase 2) the meta candidates are in the first CTA
+  cluster_wait();
+  if (rank == 0) {  // the top_meta best metas, ascending, into every CTA's mlist
+    const int nc = CS * KL1;
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      const uint64_t me = cand[i];
+      int above = 0;
+      if (me != 0ull)
+        for (int j = 0; j < nc; ++j) above += cand[j] > me;
+      chosen[i] = me != 0ull && above < k1;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      if (!chosen[i]) continue;
+      const int m = comp_index(cand[i]);
+      int pos = 0;
+      for (int j = 0; j < nc; ++j) pos += chosen[j] && comp_index(cand[j]) < m;
+      for (int r = 0; r < CS; ++r) st_cluster_u32(cluster_map(smem_u32(mlist + pos), r), m);
+    }
+  }
+  cluster_arrive();  // (phase 3) every CTA holds the kept metas
+  cluster_wait();
+  // level 2: this CTA's share of the kept metas' children
+  if (threadIdx.x == 0) n_kept = 0;
+  const int lo2 = static_cast<int>(static_cast<int64_t>(NCH) * rank / CS);
+  const int n2 = static_cast<int>(static_cast<int64_t>(NCH) * (rank + 1) / CS) - lo2;
+  const int KL2 = min(k_free, (NCH + CS - 1) / CS);
+  int32_t* clist = out_l;  // chunk of child i: meta mlist[i / Gm], child i % Gm
+  for (int i = threadIdx.x; i < n2; i += blockDim.x)
+    clist[lo2 + i - lo2] = mlist[(lo2 + i) / Gm] * Gm + (lo2 + i) % Gm;
+  __syncthreads();
+  cluster_scores<128>(summ + static_cast<int64_t>(u) * C * D, 0, n2, C, qs, n_sink, n_local,
+                      comp, clist, true, pre, false);
+  __syncthreads();
+  rank_keep(comp, n2, k_free, kept, &n_kept);
+  {
+    const uint32_t dst = cluster_map(smem_u32(cand + rank * KL2), 0);
+    for (int i = threadIdx.x; i < KL2; i += blockDim.x)
+      st_cluster_u64(dst + i * 8, i < n_kept ? kept[i] : 0ull);
+  }
+  cluster_arrive();  // (phase 4) the child candidates are in the first CTA
+  cluster_wait();
+  if (rank != 0) return;
+  if (threadIdx.x == 0) n_out = 0;
+  __syncthreads();
+  const int nc2 = CS * KL2;
+  for (int i = threadIdx.x; i < nc2; i += blockDim.x) {
+    const uint64_t me = cand[i];
+    if (me == 0ull) continue;
+    int above = 0;
+    for (int j = 0; j < nc2; ++j) above += cand[j] > me;
+    if (above < k_free) out_l[atomicAdd(&n_out, 1)] = comp_index(me);
+  }
+  __syncthreads();
+  emit_with_forced(out_l, n_out, C, n_sink, n_local, idx + static_cast<int64_t>(u) * kmax,
+                   count + u, kmax);
+}
+
 int next_pow2(int x) {
   int p = 1;
   while (p < x) p <<= 1;
@@ -1239,6 +1528,29 @@ cudaError_t launch_select_hier(const Launch& l, const void* q, bool bf16, const 
   const int M = C / Gm;
   const int k1 = std::min(top_meta, M);
   const int NCH = k1 * Gm;
+  if (D == 128 && n_sink + n_local <= 64 && U <= 65535) {  // one cluster per unit
+    for (int CS = 8; CS >= 2; CS >>= 1) {
+      if (static_cast<int64_t>(U) * CS > l.num_sms) continue;
+      const int per1 = (M + CS - 1) / CS, per2 = (NCH + CS - 1) / CS;
+      if (per1 > kClRangeMax || per2 > kClRangeMax || CS * std::min(k1, per1) > kClCandMax ||
+          CS * std::min(k_free, per2) > kClCandMax || k1 > kClRangeMax)
+        continue;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(CS, U);
+      cfg.blockDim = dim3(kClSelThreads);
+      cfg.stream = l.stream;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = CS;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, select_hier_cluster_kernel, q, bf16 ? 1 : 0, meta, summ, Hq,
+                                Hkv, D, C, Gm, top_meta, k_free, n_sink, n_local, idx, count,
+                                kmax);
+    }
+  }
   if (M <= kRankMax && NCH <= kRankMax && D <= 128) {
     select_hier_rank_kernel<<<U, kSelThreads, 0, l.stream>>>(q, bf16 ? 1 : 0, meta, summ, Hq, Hkv,
                                                              D, C, Gm, top_meta, k_free, n_sink,
@@ -1301,12 +1613,59 @@ cudaError_t fused_topp_ds(const Launch& l, const void* q, bool bf16, const float
 }
 }  // namespace
 
+namespace {
+// Cluster size for the cluster top-k, or 0: the largest power of two <= 8
+// with B*Hkv*CS CTAs on the SMs, each CTA scoring at most kClRangeMax chunks
+// and the kept candidates fitting the first CTA's kClCandMax slots.
+int select_cluster_size(int U, int C, int k_free, int n_sink, int n_local, int num_sms) {
+  if (U <= 0 || U > 65535 || C <= 0 || n_sink + n_local > 64) return 0;
+  for (int CS = 8; CS >= 2; CS >>= 1) {
+    if (static_cast<int64_t>(U) * CS > num_sms) continue;
+    const int per = (C + CS - 1) / CS;
+    const int KL = std::min(k_free, per);
+    if (per <= kClRangeMax && CS * KL <= kClCandMax) return CS;
+  }
+  return 0;
+}
+
+template <int DS>
+cudaError_t cluster_topk_kernel(const Launch& l, const void* q, bool bf16, const float* proj,
+                                int R, const float* summ, int U, int Hq, int Hkv, int D, int C,
+                                const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                                int32_t* idx, int32_t* count, int kmax, int CS) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, U);
+  cfg.blockDim = dim3(kClSelThreads);
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_select_topk_cluster_kernel<DS>, q, bf16 ? 1 : 0, proj, R,
+                            summ, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count,
+                            kmax);
+}
+}  // namespace
+
 cudaError_t launch_score_select_topk(const Launch& l, const void* q, bool bf16, const float* proj,
                                      int R, const float* summ, int B, int Hq, int Hkv, int D, int C,
                                      const uint8_t* head_full, int k_free, int n_sink, int n_local,
                                      int32_t* idx, int32_t* count, int kmax, bool per_head_union) {
   const int U = B * Hkv;
   if (U == 0) return cudaSuccess;
+  const int CS = per_head_union ? 0 : select_cluster_size(U, C, k_free, n_sink, n_local, l.num_sms);
+  if (CS > 0) {
+    switch (proj ? R : D) {
+      case 16: return cluster_topk_kernel<16>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CS);
+      case 32: return cluster_topk_kernel<32>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CS);
+      case 64: return cluster_topk_kernel<64>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CS);
+      case 128: return cluster_topk_kernel<128>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CS);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   const bool pu = per_head_union;
   switch (proj ? R : D) {
     case 16: return fused_topk_ds<16>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, pu);

@@ -177,13 +177,14 @@ class SparseDecoder:
                                                 self.gist_scope, self.dtype,
                                                 self.idx, self.count, self.kmax, self.head_full,
                                                 self.B, self.Hq, self.Hkv, self.D, self.T, self.L,
-                                                self.scale, self.P, self.workspace, self.ws_bytes,
-                                                self.out, _dt(self.out), self.lse, stream=stream)
+                                                self.scale, self.num_parts, self.workspace,
+                                                self.ws_bytes, self.out, _dt(self.out), self.lse,
+                                                stream=stream)
             return
         if self.fused:
             csa.csa_sparse_decode_merged(q, self.K_att, self.V, self.dtype, self.idx, self.count,
                                          self.kmax, self.head_full, self.B, self.Hq, self.Hkv,
-                                         self.D, self.T, self.L, self.scale, self.P,
+                                         self.D, self.T, self.L, self.scale, self.num_parts,
                                          self.workspace, self.ws_bytes, self.out, _dt(self.out),
                                          self.lse, stream=stream)
             return

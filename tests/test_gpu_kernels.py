@@ -256,11 +256,13 @@ def test_select_hier_vs_oracle(csa, D, C, Gm, top_meta, k_free, G):
     parity.compare_sets(got, refs, gaps, "hier")
 
 
-def test_select_hier_golden(csa):
+@pytest.mark.parametrize("D", [64, 128])
+def test_select_hier_golden(csa, D):
+    """The hand-worked cases, scalars in the first dimension (D = 128 takes
+    the cluster path: the metas and the children split over CTAs)."""
     for c in pins_golden("hier_cases.json"):
         qv = np.array(c["q"], dtype=np.float32)  # [G, 1] scalars
         G = qv.shape[0]
-        D = 64
         summ_s = np.array(c["summ"], dtype=np.float32)
         C = len(summ_s)
         q = torch.zeros(1, G, D, device="cuda")
@@ -439,17 +441,26 @@ def test_host_pointer_rejected(csa):
 
 # ---------------------------------------------------------------- fused paths
 
-@pytest.mark.parametrize("select,R,G,C", [("topk", 0, 4, 512), ("topk", 32, 8, 300),
-                                          ("topp", 16, 4, 1024), ("topp", 0, 2, 700)])
-def test_fused_score_select_equals_two_calls(csa, select, R, G, C):
-    """One CTA per unit computing scores into shared memory gives the same
-    index lists as csa_score_chunks followed by csa_select_*."""
+@pytest.mark.parametrize("select,R,G,C,ties", [("topk", 0, 4, 512, False), ("topk", 32, 8, 300, False),
+                                               ("topk", 0, 4, 4096, False), ("topk", 16, 4, 2048, True),
+                                               ("topk", 0, 4, 13, True),
+                                               ("topp", 16, 4, 1024, False), ("topp", 0, 2, 700, False)])
+def test_fused_score_select_equals_two_calls(csa, select, R, G, C, ties):
+    """Scores computed next to the selection (one CTA per unit, or for top-k
+    one cluster of CTAs per unit whose best candidates meet in one CTA) give
+    the same index lists as csa_score_chunks followed by csa_select_*; with
+    integer summaries and queries many scores tie exactly (lower index
+    first)."""
     B, Hkv, D = 2, 4, 128
     Hq = G * Hkv
     q = _randn((B, Hq, D), 30, torch.bfloat16)
     P = _randn((D, R), 31) / 4 if R else None
     Ds = R or D
     summ = _randn((B, Hkv, C, Ds), 32) * 0.3
+    if ties:
+        q = torch.randint(-1, 2, (B, Hq, D), generator=_gen(33), device="cuda").to(torch.bfloat16)
+        summ = torch.randint(-1, 2, (B, Hkv, C, Ds), generator=_gen(34), device="cuda").float()
+        P = torch.randint(-1, 2, (D, R), generator=_gen(35), device="cuda").float() if R else None
     full = torch.tensor([0, 1, 0, 0], dtype=torch.uint8, device="cuda")
     U = B * Hkv
     kmax = min(C, (20 if select == "topk" else 64) + 3)
@@ -531,8 +542,11 @@ def _merged_case(csa, dtype, B, Hkv, G, D, T, L, sets, full=(), num_parts=0, out
         parity.assert_close(got, ro, tol, f"merged unit {u}")
         if lse is not None:
             assert np.abs(lse[b, rows].cpu().double().numpy() - rl).max() < 1e-3
-    # same result as the split path (decode + separate merge), to fp32 rounding
-    if not out_bf16:
+    # same result as the split path (decode + separate merge) with the same
+    # pieces, to fp32 rounding (num_parts = 0 lets the library pick a cluster
+    # per unit instead: other parts, other bf16 roundings of P, checked
+    # against the oracle above)
+    if not out_bf16 and num_parts != 0:
         P = num_parts or csa.csa_decode_default_parts(dt, D, L)
         o_part = torch.empty(B, Hq, P, D, device="cuda")
         l_part = torch.empty(B, Hq, P, device="cuda")
@@ -541,6 +555,7 @@ def _merged_case(csa, dtype, B, Hkv, G, D, T, L, sets, full=(), num_parts=0, out
         ref = torch.empty(B, Hq, D, device="cuda")
         csa.csa_lse_merge(o_part, l_part, B * Hq, P, D, ref, torch.float32, None)
         assert (out - ref).abs().max().item() < 1e-5
+    return out
 
 
 @pytest.mark.parametrize("dtype,D,L,G,parts", [("bf16", 128, 128, 4, 0), ("bf16", 128, 64, 4, 13),
@@ -562,6 +577,29 @@ def test_merged_decode_edge_cases(csa):
     _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, [[3], [0, 8], [], [1]], full=(2,), num_parts=7)
     _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=5, out_bf16=True)
     _merged_case(csa, "f32", B, Hkv, G, 64, C * L, L, sets, num_parts=3, with_lse=False)
+
+
+@pytest.mark.parametrize("B,Hkv,G,D,L,C,nmax", [(1, 4, 4, 128, 64, 9, 9), (2, 8, 4, 128, 64, 512, 32),
+                                                 (1, 8, 4, 128, 128, 300, 35), (3, 2, 8, 64, 64, 40, 20),
+                                                 (2, 3, 1, 64, 128, 24, 5), (1, 1, 4, 128, 64, 70, 64),
+                                                 (20, 8, 4, 128, 64, 64, 12)])
+def test_merged_decode_cluster_path(csa, B, Hkv, G, D, L, C, nmax):
+    """Library-chosen pieces (num_parts = 0) on short lists without full
+    heads: one cluster of CTAs per unit whose parts meet in distributed
+    shared memory (parts of one chunk or none; an empty unit; GQA 1-8; L 64
+    and 128).  160 units are more than the SMs: the persistent kernel takes
+    them.  Two calls in a row, against the oracle, and against the
+    persistent kernel with explicit pieces on the same lists."""
+    rng = np.random.default_rng(B * 1000 + Hkv * 100 + C)
+    sets = [sorted(rng.choice(C, size=int(rng.integers(1, nmax + 1)), replace=False).tolist())
+            for _ in range(B * Hkv)]
+    sets[-1] = []  # one unit with no chunk
+    out0 = _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=0)
+    out1 = _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=148)
+    parity.assert_close(out0.cpu().double().numpy(), out1.cpu().double().numpy(), "bf16",
+                        "cluster vs persistent")
+    _merged_case(csa, "bf16", B, Hkv, G, D, C * L, L, sets, num_parts=0, out_bf16=True,
+                 with_lse=False)
 
 
 def test_merged_decode_second_wave(csa):
