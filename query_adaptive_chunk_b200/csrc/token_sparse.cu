@@ -659,6 +659,231 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
   }
 }
 
+// ---------------------------------------------------------------- budget, one cluster per sequence
+//
+// The same cut as budget_kernel, over a cluster of kBudgetCS CTAs: CTA r
+// holds the masses of tokens [r S / CS, (r + 1) S / CS) in shared memory and
+// builds its own 256-bucket histogram (count and mass) per radix pass; the
+// CTAs then read every CTA's histogram through distributed shared memory and
+// add them in rank order, so each finds the same cut bucket, and the next
+// pass narrows the prefix.  The first CTA writes the budgets.
+
+constexpr int kBudgetCS = 8;
+constexpr int kBudgetCThreads = 512;
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kBudgetCThreads) budget_cluster_kernel(
+    const float* __restrict__ imp, int S, int Hkv, float tau, int tile, int32_t* __restrict__ k_seq,
+    int32_t* __restrict__ k_unit) {
+  cluster_arrive_relaxed();
+  extern __shared__ __align__(16) uint8_t sm[];
+  float* ms = reinterpret_cast<float*>(sm);  // [S / CS] this CTA's masses
+  __shared__ unsigned int hc[256];           // this CTA's histogram of the pass
+  __shared__ float hm[256];
+  __shared__ unsigned int gc[256];           // the cluster's
+  __shared__ float gm[256];
+  __shared__ float wsum[32], tot_parts[kBudgetCS];
+  __shared__ unsigned int prefix_sh, sel_sh;
+  __shared__ float above_m_sh;
+  __shared__ unsigned int above_c_sh;
+  const int CS = static_cast<int>(cluster_size());
+  const int rank = static_cast<int>(cluster_rank());
+  const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int lo = static_cast<int>(static_cast<int64_t>(S) * rank / CS);
+  const int n = static_cast<int>(static_cast<int64_t>(S) * (rank + 1) / CS) - lo;
+  const float* ib = imp + static_cast<int64_t>(b) * Hkv * S + lo;
+  float part = 0.f;
+  for (int j = tid; j < n; j += blockDim.x) {
+    float m = 0.f;
+#pragma unroll 8
+    for (int h = 0; h < Hkv; ++h) m += ib[static_cast<int64_t>(h) * S + j];
+    m = fmaxf(m, 0.f);
+    ms[j] = m;
+    part += m;
+  }
+#pragma unroll
+  for (int x = 16; x > 0; x >>= 1) part += __shfl_xor_sync(0xffffffffu, part, x);
+  if (lane == 0) wsum[tid >> 5] = part;
+  if (tid == 0) {
+    prefix_sh = 0u;
+    above_m_sh = 0.f;
+    above_c_sh = 0u;
+  }
+  __syncthreads();
+  cluster_wait();  // (phase 1) every CTA is running: its part of the total to all
+  if (tid == 0) {
+    float t = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += wsum[w];
+    for (int r = 0; r < CS; ++r) st_cluster_f32(cluster_map(smem_u32(tot_parts + rank), r), t);
+  }
+  cluster_arrive();
+  cluster_wait();
+  float total = 0.f;
+  for (int r = 0; r < CS; ++r) total += tot_parts[r];  // rank order: the same sum in every CTA
+  const float target = (1.0f - tau) * total;
+  unsigned int mask = 0u;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int d = tid; d < 256; d += blockDim.x) {
+      hc[d] = 0u;
+      hm[d] = 0.f;
+    }
+    __syncthreads();
+    const unsigned int prefix = prefix_sh;
+    for (int j0 = 0; j0 < n; j0 += blockDim.x) {
+      const int j = j0 + tid;
+      int d = -1;
+      float m = 0.f;
+      if (j < n) {
+        const unsigned int key = __float_as_uint(ms[j]);
+        if ((key & mask) == prefix) {
+          d = (key >> shift) & 255u;
+          m = ms[j];
+        }
+      }
+#pragma unroll
+      for (int round = 0; round < 3; ++round) {
+        const unsigned int act = __ballot_sync(0xffffffffu, d >= 0);
+        if (act == 0u) break;  // warp-uniform
+        const int d0 = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
+        const unsigned int same = __ballot_sync(0xffffffffu, d == d0);
+        float v = d == d0 ? m : 0.f;
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
+        if (lane == 0) {
+          atomicAdd(&hc[d0], static_cast<unsigned int>(__popc(same)));
+          atomicAdd(&hm[d0], v);
+        }
+        if (d == d0) d = -1;  // counted
+      }
+      if (d >= 0) {
+        atomicAdd(&hc[d], 1u);
+        atomicAdd(&hm[d], m);
+      }
+    }
+    cluster_arrive();  // every CTA's histogram of this pass is complete
+    cluster_wait();
+    for (int d = tid; d < 256; d += blockDim.x) {  // the cluster's, added in rank order
+      unsigned int c = 0u;
+      float mm = 0.f;
+      for (int r = 0; r < CS; ++r) {
+        c += ld_cluster_u32(cluster_map(smem_u32(hc + d), r));
+        mm += ld_cluster_f32(cluster_map(smem_u32(hm + d), r));
+      }
+      gc[d] = c;
+      gm[d] = mm;
+    }
+    cluster_arrive();  // every CTA has read the others' histograms (they may be cleared)
+    cluster_wait();
+    // the bucket where the running mass from the top first reaches the
+    // target, by warp 0 (as budget_kernel), on the cluster's histogram
+    if (tid < 32) {
+      float pm[8];
+      unsigned int pc[8];
+      float lm = 0.f;
+      unsigned int lc = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        pm[i] = gm[255 - 8 * lane - i];
+        pc[i] = gc[255 - 8 * lane - i];
+        lm += pm[i];
+        lc += pc[i];
+      }
+      float sm_ = lm;
+      unsigned int sc = lc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, sm_, o);
+        const unsigned int tc = __shfl_up_sync(0xffffffffu, sc, o);
+        if (lane >= o) {
+          sm_ += t;
+          sc += tc;
+        }
+      }
+      float em = __shfl_up_sync(0xffffffffu, sm_, 1);
+      unsigned int ec = __shfl_up_sync(0xffffffffu, sc, 1);
+      if (lane == 0) {
+        em = 0.f;
+        ec = 0u;
+      }
+      float am = above_m_sh + em;
+      unsigned int ac = above_c_sh + ec;
+      int sel = -1, low = -1;
+      float am_sel = 0.f, am_low = 0.f;
+      unsigned int ac_sel = 0u, ac_low = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (sel < 0 && pc[i] != 0u) {
+          if (am + pm[i] >= target) {
+            sel = 255 - 8 * lane - i;
+            am_sel = am;
+            ac_sel = ac;
+          } else {
+            am_low = am;
+            ac_low = ac;
+            am += pm[i];
+            ac += pc[i];
+            low = 255 - 8 * lane - i;
+          }
+        }
+      }
+      const unsigned int hit = __ballot_sync(0xffffffffu, sel >= 0);
+      int src;
+      if (hit != 0u) {
+        src = __ffs(hit) - 1;
+      } else {
+        const unsigned int nz = __ballot_sync(0xffffffffu, low >= 0);
+        src = nz != 0u ? 31 - __clz(nz) : 0;
+        sel = low < 0 ? 0 : low;
+        am_sel = low < 0 ? am : am_low;
+        ac_sel = low < 0 ? ac : ac_low;
+      }
+      sel = __shfl_sync(0xffffffffu, sel, src);
+      am_sel = __shfl_sync(0xffffffffu, am_sel, src);
+      ac_sel = __shfl_sync(0xffffffffu, ac_sel, src);
+      if (lane == 0) {
+        above_m_sh = am_sel;
+        above_c_sh = ac_sel;
+        sel_sh = static_cast<unsigned int>(sel);
+        prefix_sh = prefix | (static_cast<unsigned int>(sel) << shift);
+      }
+    }
+    __syncthreads();
+    mask |= 255u << shift;
+  }
+  if (rank == 0 && tid == 0) {
+    int k;
+    if (!(target > 0.f)) {
+      k = 0;
+    } else {
+      const float v = __uint_as_float(prefix_sh);
+      const unsigned int n_eq = gc[sel_sh];
+      const float need = target - above_m_sh;
+      unsigned int take = n_eq;
+      if (v > 0.f && need > 0.f) {
+        const float t = ceilf(need / v);
+        take = t < static_cast<float>(n_eq) ? static_cast<unsigned int>(fmaxf(t, 1.f)) : n_eq;
+      } else if (!(need > 0.f)) {
+        take = 0u;
+      }
+      k = static_cast<int>(above_c_sh + take);
+    }
+    k = min(k, S);
+    k_seq[b] = k;
+    const int kt = min(S, (k + tile - 1) / tile * tile);
+    for (int h = 0; h < Hkv; ++h) k_unit[static_cast<int64_t>(b) * Hkv + h] = kt;
+  }
+}
+
 // ---------------------------------------------------------------- gather / scatter
 
 // Compressed row t < count[u] of (b, h): the kept token idx[u, t]; rows
@@ -766,6 +991,24 @@ cudaError_t set_smem_ts(const void* fn, size_t bytes) {
 cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S, int Hkv,
                                 float tau, int tile, int32_t* k_seq, int32_t* k_unit) {
   if (B == 0) return cudaSuccess;
+  if (B <= 65535 && static_cast<int64_t>(B) * kBudgetCS <= l.num_sms) {  // one cluster per sequence
+    const size_t shc = static_cast<size_t>((S + kBudgetCS - 1) / kBudgetCS) * 4;
+    cudaError_t e = set_smem_ts(reinterpret_cast<const void*>(budget_cluster_kernel), shc);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kBudgetCS, B);
+    cfg.blockDim = dim3(kBudgetCThreads);
+    cfg.dynamicSmemBytes = shc;
+    cfg.stream = l.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kBudgetCS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, budget_cluster_kernel, imp, S, Hkv, tau, tile, k_seq, k_unit);
+  }
   const size_t sh = static_cast<size_t>(S) * 4;
   cudaError_t e = set_smem_ts(reinterpret_cast<const void*>(budget_kernel), sh);
   if (e != cudaSuccess) return e;
