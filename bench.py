@@ -621,8 +621,10 @@ def run_reference(args):
             "ms_per_step": us / 1000, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                       "ctx": w.T, "L": w.L, "p": w.p, "budget": w.budget,
-                       "full_heads": list(w.full_heads)},
+                       "ctx": w.T, "L": w.L, "select": "top-p p=0.9 cap 256 + sink + 2 local",
+                       "full_heads": list(w.full_heads), "proj_rank": w.proj_rank,
+                       "timing": "wall clock around each whole oracle step (host)",
+                       "parallelism": "one process on the host cores"},
             "cpu_baseline": {"value": us, "unit": "us/step", "cores": 1, "kind": "oracle",
                              "sample": f"{len(t)} whole decode steps of {w.name} (all 8 units), "
                                        "summaries precomputed, numpy fp64 single-threaded",

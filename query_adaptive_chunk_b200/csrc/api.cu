@@ -935,9 +935,11 @@ csa_status csa_token_importance(const void* Q, const void* K, int B, int S, int 
   CSA_TRY(check_ptr(scratch, "scratch"));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
-  return finish(csa::launch_token_importance(l, Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp,
-                                             static_cast<float*>(scratch)),
-                "token importance launch");
+  std::string why;
+  const cudaError_t e = csa::launch_token_importance(l, Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp,
+                                                     static_cast<float*>(scratch), &why);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
+  return finish(e, "token importance launch");
 }
 
 csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, float tau, int tile,
@@ -1013,8 +1015,10 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
   int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + w.count);
   const int U = B * Hkv;
+  std::string why;
   cudaError_t e = csa::launch_token_importance(l, Q, K, B, S, Hq, Hkv, D, n_obs, scale, imp,
-                                               reinterpret_cast<float*>(ws + w.scratch));
+                                               reinterpret_cast<float*>(ws + w.scratch), &why);
+  if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
   if (e == cudaSuccess) e = csa::launch_token_budget(l, imp, B, S, Hkv, tau, 64, budget_out, k_unit);
   if (e == cudaSuccess)  // each KV head's own top tokens under the (rounded) budget
     e = csa::launch_select_topk(l, imp, U, S, nullptr, 0, 0, 0, idx, cnt, S, k_unit);
@@ -1032,7 +1036,6 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
   int32_t* counts2 = reinterpret_cast<int32_t*>(ws + w.counts2);
   e = csa::launch_tsa_gather(l, Q, K, V, idx, cnt, S, B, S, S, Hq, Hkv, D, Qc, Kc, Vc);
   if (e == cudaSuccess) e = csa::launch_tsa_lists(l, k_unit, U, T, 64, lists, counts2);
-  std::string why;
   if (e == cudaSuccess)
     e = csa::launch_prefill(l, Qc, Kc, Vc, lists, counts2, T, B, S, Hq, Hkv, D, 64, 64, scale, Oc,
                             &why, /*skip_empty=*/true);

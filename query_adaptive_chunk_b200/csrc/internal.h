@@ -67,7 +67,7 @@ cudaError_t launch_score_select_topp(const Launch& l, const void* q, bool bf16, 
 size_t token_importance_scratch_bytes(int B, int S, int Hkv, int G, int n_obs);
 cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* K, int B, int S,
                                     int Hq, int Hkv, int D, int n_obs, float scale, float* imp,
-                                    float* scratch);
+                                    float* scratch, std::string* why);
 cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S, int Hkv,
                                 float tau, int tile, int32_t* k_seq, int32_t* k_unit);
 cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, const void* V,

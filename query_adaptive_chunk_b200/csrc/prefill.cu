@@ -29,8 +29,8 @@
 // SM, the whole 512-column TMEM), heaviest tiles first.
 #include <algorithm>
 
-#include "exp2_poly.h"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace csa {
 namespace {
@@ -54,48 +54,10 @@ constexpr int kEmuPeriod = 3;  // one pair of exponentials in kEmuPeriod on the 
 // O of half h at 256 + 128 h
 constexpr uint32_t kColP = 128, kColO = 256;
 
-// instruction descriptors (kind::f16): D fp32, A/B bf16, M = 128
-constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (0u << 16) |
-                              ((64u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
-                              ((128u >> 3) << 17) | ((128u >> 4) << 24);
-
-// shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((addr & 0x3ffffu) >> 4) |
-         (static_cast<uint64_t>(lbo >> 4) << 16) | (static_cast<uint64_t>(sbo >> 4) << 32) |
-         (1ull << 46) | (2ull << 61);
-}
-
-__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                        uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
+// instruction descriptors: QK^T M = 128, N = 64 (both K-major); PV M = 128,
+// N = 128 (V MN-major)
+constexpr uint32_t kIdescQK = idesc_bf16(128, 64, 0);
+constexpr uint32_t kIdescPV = idesc_bf16(128, 128, 1);
 
 // Bulk tensor store of a [64 x 64] bf16 box from shared memory (128-byte
 // swizzle) at (col, row) of the output map; completion tracked per thread
@@ -116,38 +78,6 @@ __device__ __forceinline__ void bulk_wait_read0() {
 // This thread's stores are complete.
 __device__ __forceinline__ void bulk_wait0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-#define CSA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
-                  "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
-#define CSA_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \
-                  "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
-
-// 32 consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : CSA_R8(0), CSA_R8(8), CSA_R8(16), CSA_R8(24)
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      CSA_W8(0), CSA_W8(8), CSA_W8(16), CSA_W8(24)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 struct PrefillParams {
@@ -185,31 +115,6 @@ __device__ __forceinline__ int unit_chunk(const PrefillParams& p, int sel_row, i
     c = 0;
   }
   return c;
-}
-
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// 2^x for a pair, x <= 8, on the FMA and integer pipes (Cody-Waite range
-// reduction): j = rint(x) by the round-to-nearest of adding 1.5 * 2^23,
-// f = x - j in [-1/2, 1/2], 2^f by the minimax cubic of exp2_poly.h (relative
-// error < 1e-4), and 2^j added to the exponent field.  Inputs below -125
-// give 2^-125 (the result stays a normal number).
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 magic = make_float2(12582912.f, 12582912.f);
-  const float2 t = __fadd2_rn(x, magic);
-  const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(jf, make_float2(-1.f, -1.f), x);
-  float2 q = __ffma2_rn(f, make_float2(CSA_EXP2_C3, CSA_EXP2_C3), make_float2(CSA_EXP2_C2, CSA_EXP2_C2));
-  q = __ffma2_rn(q, f, make_float2(CSA_EXP2_C1, CSA_EXP2_C1));
-  q = __ffma2_rn(q, f, make_float2(CSA_EXP2_C0, CSA_EXP2_C0));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -257,10 +162,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
-                     smem_u32(tmem_slot))
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc<512>(tmem_slot);
   }
   tc_fence_before();
   __syncthreads();
@@ -614,7 +516,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    tmem_dealloc<512>(tmem);
 }
 
 }  // namespace

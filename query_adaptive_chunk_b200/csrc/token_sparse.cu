@@ -7,10 +7,10 @@
 //                of key j is the sum over those rows of its softmax weight
 //                (the rows of the GQA group's heads summed: one importance
 //                per KV head).  Two passes over K on the tensor cores
-//                (mma.m16n8k16): per-row max and sum over key blocks (rows
-//                as M, keys as N), then, with the rows' final max and sum,
-//                the weights summed per key (keys as M, rows as N).  K is
-//                read twice from HBM.
+//                (tcgen05, accumulators in tensor memory): per-row max and
+//                sum over key blocks (rows as M, keys as N), then, with the
+//                rows' final max and sum, the weights summed per key (keys
+//                as M, rows as N).  K is read twice.
 //   budget       Dynamic Token Coverage: the fewest tokens whose importance
 //                (summed over the KV heads, normalised) reaches 1 - tau, i.e.
 //                the least important ones are dropped while their mass stays
@@ -24,415 +24,419 @@
 //   scatter      the compressed output back to the kept positions; every
 //                other row of the output is 0 (the residual path carries the
 //                skipped tokens in the model).
+#include <algorithm>
+
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace csa {
 namespace {
 
-constexpr int kImpThreads = 128;    // pass 2: 4 warps, 32 keys each
-constexpr int kStatsThreads = 256;  // pass 1: 8 warps, 32 observed rows each per turn
-constexpr int kImpKeys = 128;       // keys per CTA
+// ---------------------------------------------------------------- importance
+//
+// Both passes are persistent over blocks of kTcKeys keys: CTA (split, h, b)
+// takes blocks split, split + nsplit, ... of KV head h of sequence b.  The
+// head's observed query rows (R = G * n_obs of them, padded with zero rows
+// to Rp, a multiple of 128) are copied once into shared memory by TMA as
+// 64-column slabs with the 128-byte swizzle; the key blocks stream through a
+// ring of TMA stages; one thread issues the MMAs into a double-buffered
+// accumulator in tensor memory:
+//   pass 1   S = Q_obs K_blk^T, M = 128 observed rows per MMA (Rp / 128 of
+//            them), N = 128 keys.  TMEM lane = row: each epilogue thread
+//            keeps its row's running max and sum of 2^(s - max).
+//   pass 2   S^T = K_blk Q_obs^T, M = 128 keys, N = the observed rows (up to
+//            256 per MMA).  TMEM lane = key: each thread sums its key's
+//            weights 2^(s - max_r - log2 sum_r) along its own TMEM lane.
+// Warp 0 issues the TMA copies, warp 1 owns the tensor memory and one of its
+// threads issues the MMAs, warps 2-9 are two warpgroups that read the
+// accumulators (warp w reaches TMEM lanes 32 (w % 4) .. + 31): in pass 1
+// warpgroup g takes the 128-row tiles g and g + 2; in pass 2 it takes half
+// of the observed rows, and the halves' sums meet in shared memory.  A third
+// of the exponentials run on the FMA pipe.  Pass 2 is launched behind pass 1
+// with programmatic dependent launch: its copies and MMAs start while pass 1
+// drains, and its epilogue waits (griddepcontrol.wait) for pass 1's per-split
+// row statistics, which it combines itself.  Pass 1 reads K with the default
+// L2 policy so that pass 2, which reads it last, finds much of it in L2.
+
+constexpr int kTcKeys = 128;
+constexpr int kTcEpiWarps = 8;
+constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;
+constexpr int kTcMaxNS = 4;
+constexpr size_t kTcMinSmem = 120 * 1024;  // one CTA per SM: it allocates all 512 TMEM columns
+constexpr size_t kTcMaxSmem = 232448;      // 227 KB per block
+constexpr int kTcEmuPeriod = 3;            // one pair of exponentials in 3 on the FMA pipe
 constexpr float kLog2eF = 1.4426950408889634f;
 
-// Row r of the observed block of KV head h: query head h*G + r / n_obs at
-// position S - n_obs + r % n_obs.
-__device__ __forceinline__ int obs_pos(int r, int n_obs, int S) { return S - n_obs + r % n_obs; }
+struct ImpParams {
+  int S, Hkv, G, n_obs, R, Rp, D, nblk, nsplit, NS, qbox;
+  float sl2;    // scale * log2(e)
+  float2* part;  // [B, Hkv, nsplit, R]: (max, sum of 2^(s - max)) per split, log2 units
+  float* imp;    // [B, Hkv, S]
+  DevErr err;
+};
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
-  // 16-byte asynchronous copy; src-size 0 fills the destination with zeros
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
-               "l"(gsrc), "r"(valid ? 16 : 0)
-               : "memory");
+// Shared-memory layout, offsets from the 1024-aligned base: Q slabs | K
+// stages | mbarriers + TMEM slot | pass 2: bias[Rp], lim[Rp], red[2][128].
+struct ImpLayout {
+  int kv_off, stage_bytes, bar_off, bias_off, lim_off, red_off;
+  size_t total;
+};
+
+__host__ __device__ inline ImpLayout imp_layout(int Rp, int D, int NS) {
+  ImpLayout y;
+  y.kv_off = Rp * D * 2;
+  y.stage_bytes = kTcKeys * D * 2;
+  y.bar_off = y.kv_off + NS * y.stage_bytes;
+  y.bias_off = y.bar_off + 256;
+  y.lim_off = y.bias_off + Rp * 4;
+  y.red_off = y.lim_off + Rp * 4;
+  y.total = 1024 + static_cast<size_t>(y.red_off) + 2 * kTcKeys * 4;
+  return y;
 }
 
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Asynchronous 16-byte copies of the observed query rows of (b, h) [R][D]
-// into padded shared memory (row stride D + 8 bf16: conflict-free fragment
-// loads); the caller commits and waits.
-template <int D>
-__device__ __forceinline__ void imp_load_q(const __nv_bfloat16* Q, int b, int h, int S, int Hq,
-                                           int G, int n_obs, __nv_bfloat16* qs) {
-  constexpr int LD = D + 8, V8 = D / 8;
-  const int R = G * n_obs;
-  for (int e = threadIdx.x; e < R * V8; e += blockDim.x) {
-    const int r = e / V8, c = (e % V8) * 8;
-    const int g = r / n_obs, pos = obs_pos(r, n_obs, S);
-    cp_async16(qs + r * LD + c, Q + ((static_cast<int64_t>(b) * S + pos) * Hq + h * G + g) * D + c,
-               true);
-  }
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// The same for the key block [kImpKeys][D] starting at key j0 (keys past S
-// are zero-filled).
-template <int D>
-__device__ __forceinline__ void imp_load_k(const __nv_bfloat16* K, int b, int h, int S, int Hkv,
-                                           int j0, __nv_bfloat16* ks) {
-  constexpr int LD = D + 8, V8 = D / 8;
-  const __nv_bfloat16* kb = K + ((static_cast<int64_t>(b) * Hkv + h) * S) * D;
-  for (int e = threadIdx.x; e < kImpKeys * V8; e += blockDim.x) {
-    const int r = e / V8, c = (e % V8) * 8;
-    const int j = j0 + r;
-    cp_async16(ks + r * LD + c, kb + static_cast<int64_t>(j < S ? j : 0) * D + c, j < S);
-  }
+// Named barrier over the eight epilogue warps.
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kTcEpiWarps * 32) : "memory");
 }
 
-// Both, all in flight at once, then waits for them (the caller's barrier
-// then publishes them).
-template <int D>
-__device__ void imp_load(const __nv_bfloat16* Q, const __nv_bfloat16* K, int b, int h, int S,
-                         int Hq, int Hkv, int G, int n_obs, int j0, __nv_bfloat16* qs,
-                         __nv_bfloat16* ks) {
-  imp_load_q<D>(Q, b, h, S, Hq, G, n_obs, qs);
-  imp_load_k<D>(K, b, h, S, Hkv, j0, ks);
-  cp_async_commit();
-  cp_async_wait<0>();
+__device__ __forceinline__ int imp_blocks(const ImpParams& p, int split) {
+  return split < p.nblk ? (p.nblk - split + p.nsplit - 1) / p.nsplit : 0;
 }
 
-// This warp's 32 keys (two 16-key m-tiles) as mma A fragments for every
-// 16-wide slice of D, loaded once and reused for every block of query rows.
-template <int D>
-__device__ __forceinline__ void imp_load_a(const __nv_bfloat16* ks, int kw,
-                                           uint32_t (&af)[D / 16][2][4]) {
-  constexpr int LD = D + 8;
-  const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
-#pragma unroll
-  for (int ks16 = 0; ks16 < D / 16; ++ks16)
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      const __nv_bfloat16* kr = ks + (kw + mt * 16 + rr) * LD + ks16 * 16 + cc;
-      af[ks16][mt][0] = *reinterpret_cast<const uint32_t*>(kr);
-      af[ks16][mt][1] = *reinterpret_cast<const uint32_t*>(kr + 8 * LD);
-      af[ks16][mt][2] = *reinterpret_cast<const uint32_t*>(kr + 8);
-      af[ks16][mt][3] = *reinterpret_cast<const uint32_t*>(kr + 8 * LD + 8);
+// Warp 0, lane 0: the observed rows once, then this CTA's key blocks into
+// the ring.  Returns the number of key blocks issued.
+__device__ uint32_t imp_produce(const ImpParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                                uint32_t sQ, uint32_t sKV, uint32_t stage_bytes, uint32_t q_full,
+                                uint32_t kv_full, uint32_t kv_empty, int b, int h, int split,
+                                bool evict_first) {
+  const int nslab = p.D / 64;
+  mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.R) * p.D * 2);
+  for (int g = 0; g < p.G; ++g)
+    for (int i = 0; i < p.n_obs; i += p.qbox)
+      for (int sl = 0; sl < nslab; ++sl)
+        tma_load_2d(sQ + sl * p.Rp * 128 + (g * p.n_obs + i) * 128, tmQ,
+                    (h * p.G + g) * p.D + sl * 64, b * p.S + p.S - p.n_obs + i, q_full);
+  const uint64_t pol = evict_first ? l2_policy_evict_first() : 0;
+  const int krow0 = (b * p.Hkv + h) * p.S;
+  uint32_t it = 0;
+  for (int blk = split; blk < p.nblk; blk += p.nsplit, ++it) {
+    const uint32_t s = it % p.NS;
+    if (!mbar_wait(kv_empty + 8 * s, ((it / p.NS) & 1u) ^ 1u, p.err)) break;
+    const uint32_t fb = kv_full + 8 * s;
+    mbar_arrive_expect_tx(fb, stage_bytes);
+    for (int sl = 0; sl < nslab; ++sl) {
+      const uint32_t dst = sKV + s * stage_bytes + sl * (kTcKeys * 128);
+      if (evict_first)
+        tma_load_2d_hint(dst, tmK, sl * 64, krow0 + blk * kTcKeys, fb, pol);
+      else
+        tma_load_2d(dst, tmK, sl * 64, krow0 + blk * kTcKeys, fb);
     }
-}
-
-// S^T tile of this warp's 32 keys against query rows [n0 .. n0 + 8):
-// acc[mt][0..3] as the mma C layout (key = lane/4 (+8), row = n0 + 2 (lane%4)
-// (+1)), unscaled.
-template <int D>
-__device__ __forceinline__ void imp_tile(const __nv_bfloat16* qs, const uint32_t (&af)[D / 16][2][4],
-                                         int n0, float (&acc)[2][4]) {
-  constexpr int LD = D + 8;
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
-  // B fragments of two 16-wide slices per ldmatrix: lanes 0-7 / 8-15 /
-  // 16-23 / 24-31 address rows n0 .. n0 + 7 at columns +0 / +8 / +16 / +24
-  const uint32_t qb_base =
-      smem_u32(qs + (n0 + (lane & 7)) * LD + (lane >> 4) * 16 + ((lane >> 3) & 1) * 8);
-#pragma unroll
-  for (int kp = 0; kp < D / 32; ++kp) {
-    uint32_t b[4];
-    ldsm_x4(qb_base + kp * 32 * 2, b[0], b[1], b[2], b[3]);
-#pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-        mma_bf16_16816(acc[mt], af[2 * kp + t][mt][0], af[2 * kp + t][mt][1],
-                       af[2 * kp + t][mt][2], af[2 * kp + t][mt][3], b[2 * t], b[2 * t + 1]);
   }
+  // no copy may still be landing when the CTA retires
+  const uint32_t first = it > static_cast<uint32_t>(p.NS) ? it - p.NS : 0u;
+  for (uint32_t i = first; i < it; ++i)
+    mbar_wait(kv_full + 8 * (i % p.NS), (i / p.NS) & 1u, p.err);
+  mbar_wait(q_full, 0u, p.err);
+  return it;
 }
 
-// One warp's 32 observed rows r0 .. r0 + 31 against the key block at j0 in
-// `ks`: the rows are the mma M dimension and the keys N (the layout of a
-// flash-attention forward pass); the warp runs over the block's keys 64 at a
-// time and every lane folds its scores into the running (max, sum) of its
-// four rows over its own key columns, m/l [m-tile][row +0 / +8].  Only
-// blocks that reach past the first observed position need the causal mask.
-template <int D>
-__device__ __forceinline__ void imp_stats_rows(const __nv_bfloat16* qs, const __nv_bfloat16* ks,
-                                               int r0, int R, int S, int n_obs, int j0,
-                                               bool masked, float sl2, float (&m)[2][2],
-                                               float (&l)[2][2]) {
-  constexpr int LD = D + 8;
-  const int lane = threadIdx.x & 31, rr = lane >> 2, cc = 2 * (lane & 3);
-  // A fragments by ldmatrix: lanes 0-7 / 8-15 / 16-23 / 24-31 address the
-  // rows of the (rows +0, cols +0) / (+8, +0) / (+0, +8) / (+8, +8) 8x8 blocks
-  uint32_t qa[D / 16][2][4];
-  const uint32_t qa_base =
-      smem_u32(qs + (r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * LD + (lane >> 4) * 8);
-#pragma unroll
-  for (int k16 = 0; k16 < D / 16; ++k16)
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-      ldsm_x4(qa_base + (mt * 16 * LD + k16 * 16) * 2, qa[k16][mt][0], qa[k16][mt][1],
-              qa[k16][mt][2], qa[k16][mt][3]);
-  // key j is visible to row r iff j <= S - n_obs + r % n_obs (which also
-  // keeps j < S); rows past R (zero padding) see nothing
-  int lim[2][2];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int r = r0 + mt * 16 + rr + 8 * hh;
-      lim[mt][hh] = r < R ? S - n_obs + r % n_obs : -1;
-    }
-#pragma unroll 1
-  for (int half = 0; half < kImpKeys / 64; ++half) {
-    float acc[8][2][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
-    // B fragments of two n-tiles per ldmatrix: lanes 0-7 / 8-15 / 16-23 /
-    // 24-31 address the keys of (n-tile +0, cols +0) / (+0, +8) / (+1, +0) /
-    // (+1, +8)
-    const uint32_t kb_base = smem_u32(ks + (half * 64 + (lane >> 4) * 8 + (lane & 7)) * LD +
-                                      ((lane >> 3) & 1) * 8);
-#pragma unroll
-    for (int k16 = 0; k16 < D / 16; ++k16)
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t b[4];
-        ldsm_x4(kb_base + (np * 16 * LD + k16 * 16) * 2, b[0], b[1], b[2], b[3]);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-            mma_bf16_16816(acc[2 * np + t][mt], qa[k16][mt][0], qa[k16][mt][1], qa[k16][mt][2],
-                           qa[k16][mt][3], b[2 * t], b[2 * t + 1]);
-      }
-    // C layout: acc[nt][mt][e] = row r0 + mt*16 + rr + 8 (e >> 1), key
-    // j0 + half*64 + nt*8 + cc + (e & 1); to the log2 domain, masked
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v = acc[nt][mt][e] * sl2;
-          if (masked && j0 + half * 64 + nt * 8 + cc + (e & 1) > lim[mt][e >> 1]) v = -INFINITY;
-          acc[nt][mt][e] = v;
+// Warp 1, lane 0: the MMAs of every key block this CTA takes.  Pass 1:
+// D[buf][128 mt .. + 128) = Q rows of tile mt x K_blk^T for each 128-row
+// tile; pass 2: D[buf][n0 .. + N) = K_blk x Q rows n0 .. n0 + N - 1.  Each
+// block's stage is released and its accumulator published by commits.
+template <bool kPass2>
+__device__ void imp_mma(const ImpParams& p, uint32_t tmem, uint32_t sQ, uint32_t sKV,
+                        uint32_t stage_bytes, uint32_t q_full, uint32_t kv_full,
+                        uint32_t kv_empty, uint32_t tm_full, uint32_t tm_free, uint32_t drain,
+                        int nb) {
+  const int nbuf = 2 * p.Rp <= 512 ? 2 : 1;
+  const int ksteps = p.D / 16;
+  bool ok = mbar_wait(q_full, 0u, p.err);
+  for (int i = 0; i < nb && ok; ++i) {
+    const uint32_t s = i % p.NS;
+    const int buf = i % nbuf, use = i / nbuf;
+    if (!mbar_wait(kv_full + 8 * s, (i / p.NS) & 1u, p.err)) break;
+    if (use > 0 && !mbar_wait(tm_free + 8 * buf, (use - 1) & 1u, p.err)) break;
+    tc_fence_after();
+    const uint32_t kb = sKV + s * stage_bytes;
+    const uint32_t d0 = tmem + buf * p.Rp;
+    if (!kPass2) {
+      const uint32_t idesc = idesc_bf16(128, kTcKeys, 0);
+      for (int mt = 0; mt < p.Rp / 128; ++mt)
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const uint32_t qa = sQ + (kk >> 2) * (p.Rp * 128) + mt * 16384 + (kk & 3) * 32;
+          const uint32_t ka = kb + (kk >> 2) * (kTcKeys * 128) + (kk & 3) * 32;
+          umma_ss(d0 + mt * 128, smem_desc(qa, 16, 1024), smem_desc(ka, 16, 1024), idesc,
+                  kk > 0 ? 1u : 0u);
         }
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-          mx = fmaxf(mx, fmaxf(acc[nt][mt][2 * hh], acc[nt][mt][2 * hh + 1]));
-        const float mn = fmaxf(m[mt][hh], mx);
-        if (mn != -INFINITY) {
-          float sum = 0.f;
-#pragma unroll
-          for (int nt = 0; nt < 8; ++nt)
-            sum += fast_exp2(acc[nt][mt][2 * hh] - mn) + fast_exp2(acc[nt][mt][2 * hh + 1] - mn);
-          l[mt][hh] = l[mt][hh] * fast_exp2(m[mt][hh] - mn) + sum;
-          m[mt][hh] = mn;
-        }
-      }
-  }
-}
-
-// Pass 1: per (b, h) and observed row, the max and the sum of 2^(s - max)
-// over the visible keys of the key blocks this CTA takes -> part [b, h,
-// split, R, 2].  Persistent over the key blocks: CTA (split, h, b) takes
-// blocks split, split + nsplit, ...; the observed rows are loaded once and
-// the key tiles double-buffered, so the next tile's copy runs under this
-// tile's math.  Warp w takes the 32-row groups w, w + 8 (R <= 512) and keeps
-// their per-lane running statistics across all the CTA's blocks; the four
-// lanes of a row merge once at the end.
-template <int D>
-__global__ void __launch_bounds__(kStatsThreads) imp_stats_kernel(
-    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, int S, int Hq,
-    int Hkv, int G, int n_obs, float sl2, int nblk, float* __restrict__ part) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int LD = D + 8, V8 = D / 8;
-  constexpr int kRowsPerTurn = (kStatsThreads / 32) * 32;
-  const int R = G * n_obs, Rp = (R + 31) & ~31;
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);  // [Rp][LD]
-  __nv_bfloat16* ksb = qs + Rp * LD;                         // [2][kImpKeys][LD]
-  const int nsplit = gridDim.x, split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  // rows R .. Rp - 1 of the last row group are zero (their results are dropped)
-  for (int e = threadIdx.x; e < (Rp - R) * V8; e += blockDim.x)
-    *reinterpret_cast<uint4*>(qs + (R + e / V8) * LD + (e % V8) * 8) = make_uint4(0u, 0u, 0u, 0u);
-  imp_load_q<D>(Q, b, h, S, Hq, G, n_obs, qs);
-  if (split < nblk) imp_load_k<D>(K, b, h, S, Hkv, split * kImpKeys, ksb);
-  cp_async_commit();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float m[2][2][2], l[2][2][2];  // [row group of this warp][m-tile][row +0 / +8]
-#pragma unroll
-  for (int g2 = 0; g2 < 2; ++g2)
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        m[g2][mt][hh] = -INFINITY;
-        l[g2][mt][hh] = 0.f;
-      }
-  int it = 0;
-  for (int blk = split; blk < nblk; blk += nsplit, ++it) {
-    const int nxt = blk + nsplit;
-    if (nxt < nblk) imp_load_k<D>(K, b, h, S, Hkv, nxt * kImpKeys, ksb + ((it + 1) & 1) * kImpKeys * LD);
-    cp_async_commit();
-    cp_async_wait<1>();  // all but the tile just issued
-    __syncthreads();
-    const __nv_bfloat16* ks = ksb + (it & 1) * kImpKeys * LD;
-    const int j0 = blk * kImpKeys;
-    const bool masked = j0 + kImpKeys - 1 > S - n_obs;
-#pragma unroll
-    for (int g2 = 0; g2 < 2; ++g2) {
-      const int r0 = warp * 32 + g2 * kRowsPerTurn;
-      if (r0 < R) imp_stats_rows<D>(qs, ks, r0, R, S, n_obs, j0, masked, sl2, m[g2], l[g2]);
-    }
-    __syncthreads();  // this buffer takes the copy issued next turn
-  }
-  cp_async_wait<0>();
-  const int rr = lane >> 2;
-  float* out = part + ((static_cast<int64_t>(b) * Hkv + h) * nsplit + split) * R * 2;
-#pragma unroll
-  for (int g2 = 0; g2 < 2; ++g2) {
-    const int r0 = warp * 32 + g2 * kRowsPerTurn;
-    if (r0 >= R) continue;  // warp-uniform
-    // merge the four lanes of each row (lanes 4 rr .. 4 rr + 3)
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int x = 1; x <= 2; x <<= 1) {
-          const float mo = __shfl_xor_sync(0xffffffffu, m[g2][mt][hh], x);
-          const float lo = __shfl_xor_sync(0xffffffffu, l[g2][mt][hh], x);
-          const float mn = fmaxf(m[g2][mt][hh], mo);
-          if (mn != -INFINITY) {
-            l[g2][mt][hh] = l[g2][mt][hh] * fast_exp2(m[g2][mt][hh] - mn) + lo * fast_exp2(mo - mn);
-            m[g2][mt][hh] = mn;
-          }
-        }
-    if ((lane & 3) == 0) {
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int r = r0 + mt * 16 + rr + 8 * hh;
-          if (r < R) {
-            out[r * 2] = m[g2][mt][hh];
-            out[r * 2 + 1] = l[g2][mt][hh];
-          }
-        }
-    }
-  }
-}
-
-// The rows' max and sum over all key blocks: part -> stats [b, h, R, 2].
-// CTA (b*Hkv + h, y) takes rows 32 y .. 32 y + 31; its 8 warps split the key
-// blocks (warp w: blocks w, w + 8, ...), lane = row, so the partials of a
-// turn are one coalesced 256-byte load per warp; the warps' results merge in
-// shared memory.
-constexpr int kCombineWarps = 8;
-__global__ void __launch_bounds__(kCombineWarps * 32) imp_combine_kernel(
-    const float* __restrict__ part, int nblk, int R, float* __restrict__ stats) {
-  __shared__ float2 red[kCombineWarps][32];
-  const int64_t bh = blockIdx.x;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int r = blockIdx.y * 32 + lane;
-  float m = -INFINITY, l = 0.f;
-  if (r < R) {
-    const float2* p2 = reinterpret_cast<const float2*>(part) + bh * nblk * R + r;
-#pragma unroll 4
-    for (int k = w; k < nblk; k += kCombineWarps) {
-      const float2 v = p2[static_cast<int64_t>(k) * R];
-      if (v.x == -INFINITY) continue;
-      const float mn = fmaxf(m, v.x);
-      l = l * exp2f(m - mn) + v.y * exp2f(v.x - mn);
-      m = mn;
-    }
-  }
-  red[w][lane] = make_float2(m, l);
-  __syncthreads();
-  if (w == 0 && r < R) {
-    m = -INFINITY;
-    l = 0.f;
-    for (int x = 0; x < kCombineWarps; ++x) {
-      const float2 v = red[x][lane];
-      if (v.x == -INFINITY) continue;
-      const float mn = fmaxf(m, v.x);
-      l = l * exp2f(m - mn) + v.y * exp2f(v.x - mn);
-      m = mn;
-    }
-    stats[(bh * R + r) * 2] = m;
-    stats[(bh * R + r) * 2 + 1] = l;
-  }
-}
-
-// Pass 2: importance of each key = sum over the observed rows of
-// 2^(s - max_r) / sum_r -> imp [b, h, S].
-template <int D>
-__global__ void __launch_bounds__(kImpThreads) imp_weight_kernel(
-    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, int S, int Hq,
-    int Hkv, int G, int n_obs, float sl2, const float* __restrict__ stats, float* __restrict__ imp) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int LD = D + 8;
-  const int R = G * n_obs;
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm);
-  __nv_bfloat16* ks = qs + R * LD;
-  float* st = reinterpret_cast<float*>(ks + kImpKeys * LD);  // [R][2]: max, 1/sum
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int j0 = blk * kImpKeys;
-  const int64_t bh = static_cast<int64_t>(b) * Hkv + h;
-  imp_load<D>(Q, K, b, h, S, Hq, Hkv, G, n_obs, j0, qs, ks);
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    st[r * 2] = stats[(bh * R + r) * 2];
-    const float l = stats[(bh * R + r) * 2 + 1];
-    st[r * 2 + 1] = l > 0.f ? 1.0f / l : 0.f;
-  }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kw = warp * 32, rr = lane >> 2, cc = 2 * (lane & 3);
-  float wsum[4] = {0.f, 0.f, 0.f, 0.f};  // keys kw + rr + 8 t
-  uint32_t af[D / 16][2][4];
-  imp_load_a<D>(ks, kw, af);
-  // as in pass 1: only blocks reaching past the first observed position mask
-  const bool masked = j0 + kImpKeys - 1 > S - n_obs;
-  const float2* st2 = reinterpret_cast<const float2*>(st);
-  for (int n0 = 0; n0 < R; n0 += 8) {
-    float acc[2][4];
-    imp_tile<D>(qs, af, n0, acc);
-    // (max, 1/sum) of this lane's two rows
-    const float2 s0 = st2[n0 + cc], s1 = st2[n0 + cc + 1];
-    const float nm[2] = {-s0.x, -s1.x}, il[2] = {s0.y, s1.y};
-    if (!masked) {
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          wsum[mt * 2 + (e >> 1)] += fast_exp2(fmaf(acc[mt][e], sl2, nm[e & 1])) * il[e & 1];
     } else {
-      const int lim[2] = {obs_pos(n0 + cc, n_obs, S), obs_pos(n0 + cc + 1, n_obs, S)};
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int t = mt * 2 + (e >> 1);
-          if (j0 + kw + rr + t * 8 <= lim[e & 1])
-            wsum[t] += fast_exp2(fmaf(acc[mt][e], sl2, nm[e & 1])) * il[e & 1];
+      for (int n0 = 0; n0 < p.Rp; n0 += 256) {
+        const int n = min(256, p.Rp - n0);
+        const uint32_t idesc = idesc_bf16(128, n, 0);
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const uint32_t ka = kb + (kk >> 2) * (kTcKeys * 128) + (kk & 3) * 32;
+          const uint32_t qa = sQ + (kk >> 2) * (p.Rp * 128) + n0 * 128 + (kk & 3) * 32;
+          umma_ss(d0 + n0, smem_desc(ka, 16, 1024), smem_desc(qa, 16, 1024), idesc,
+                  kk > 0 ? 1u : 0u);
         }
+      }
+    }
+    umma_commit(kv_empty + 8 * s);
+    umma_commit(tm_full + 8 * buf);
+  }
+  // every MMA issued here has finished before the tensor memory is freed
+  umma_commit(drain);
+  mbar_wait(drain, 0u, p.err);
+}
+
+// 2^x of a pair, every kTcEmuPeriod-th pair on the FMA pipe.
+template <int PAIR>
+__device__ __forceinline__ float2 exp2_pair(float2 a) {
+  if (PAIR % kTcEmuPeriod == kTcEmuPeriod - 1) return exp2_fma2(a);
+  return make_float2(fast_exp2(a.x), fast_exp2(a.y));
+}
+
+// Pass 1 epilogue, one 128-key block for one row: x = the row's raw scores
+// against the block's keys, keys i <= lim visible (lim >= 127: all); folds
+// them into the running (m: max of s * sl2, l: sum of 2^(s sl2 - m)).
+__device__ __forceinline__ void stats_fold(const uint32_t (&r)[4][32], int lim, float sl2,
+                                           float& m, float& l) {
+  float x[128];
+#pragma unroll
+  for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(r[i >> 5][i & 31]);
+  if (lim < 127) {
+#pragma unroll
+    for (int i = 0; i < 128; ++i) x[i] = i <= lim ? x[i] : -INFINITY;
+  }
+  float mq[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    float v = fmax3(x[32 * a], x[32 * a + 1], x[32 * a + 2]);
+#pragma unroll
+    for (int k = 3; k < 31; k += 2) v = fmax3(v, x[32 * a + k], x[32 * a + k + 1]);
+    mq[a] = fmaxf(v, x[32 * a + 31]);
+  }
+  const float mn = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]) * sl2;
+  const float mnew = fmaxf(m, mn);
+  if (mnew == -INFINITY) return;  // no visible key yet
+  const float2 sc = make_float2(sl2, sl2), nb = make_float2(-mnew, -mnew);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < 64; q += kTcEmuPeriod * 2) {
+#pragma unroll
+    for (int t = 0; t < kTcEmuPeriod * 2; ++t) {
+      if (q + t < 64) {
+        const float2 a = __ffma2_rn(make_float2(x[2 * (q + t)], x[2 * (q + t) + 1]), sc, nb);
+        float2 e;
+        if (t % kTcEmuPeriod == kTcEmuPeriod - 1) e = exp2_fma2(a);
+        else e = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+        if (t & 1) acc1 = __fadd2_rn(acc1, e);
+        else acc0 = __fadd2_rn(acc0, e);
+      }
     }
   }
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    wsum[t] += __shfl_xor_sync(0xffffffffu, wsum[t], 1);
-    wsum[t] += __shfl_xor_sync(0xffffffffu, wsum[t], 2);
-  }
-  if ((lane & 3) == 0) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int j = j0 + kw + rr + t * 8;
-      if (j < S) imp[bh * S + j] = wsum[t];
+  l = l * fast_exp2(m - mnew) + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
+  m = mnew;
+}
+
+template <bool kPass2>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    imp_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ ImpParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const ImpLayout Y = imp_layout(p.Rp, p.D, p.NS);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t sQ = sb, sKV = sb + Y.kv_off;
+  const uint32_t kv_full = sb + Y.bar_off, kv_empty = kv_full + 8 * kTcMaxNS;
+  const uint32_t tm_full = kv_empty + 8 * kTcMaxNS, tm_free = tm_full + 16;  // [2] each
+  const uint32_t q_full = tm_free + 16, drain = q_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Y.bar_off + 8 * (2 * kTcMaxNS + 6));
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = imp_blocks(p, split);
+  const int nbuf = 2 * p.Rp <= 512 ? 2 : 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.NS; ++s) {
+      mbar_init(kv_full + 8 * s, 1);
+      mbar_init(kv_empty + 8 * s, 1);
     }
+    // pass 1: the warps of each warpgroup that has a 128-row tile read the
+    // accumulator; pass 2: all eight
+    const int readers = kPass2 ? kTcEpiWarps : 4 * min(2, p.Rp / 128);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(tm_full + 8 * k, 1);
+      mbar_init(tm_free + 8 * k, readers);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmQ);
+    prefetch_tensormap(&tmK);
+  }
+  if (warp == 1) tmem_alloc<512>(tmem_slot);
+  if (warp >= 2 && p.Rp > p.R) {  // zero the padding rows of every slab (MMA operands)
+    const int pad16 = (p.Rp - p.R) * 8;  // 16-byte pieces per slab
+    for (int e = threadIdx.x - 64; e < pad16 * (p.D / 64); e += kTcEpiWarps * 32) {
+      const int sl = e / pad16, o = e % pad16;
+      *reinterpret_cast<uint4*>(smem + sl * p.Rp * 128 + p.R * 128 + o * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (!kPass2) grid_dependents_launch();  // pass 2 may start its copies as SMs free up
+
+  if (warp == 0) {
+    if (lane == 0)
+      imp_produce(p, &tmQ, &tmK, sQ, sKV, Y.stage_bytes, q_full, kv_full, kv_empty, b, h, split,
+                  kPass2);
+  } else if (warp == 1) {
+    if (lane == 0)
+      imp_mma<kPass2>(p, tmem, sQ, sKV, Y.stage_bytes, q_full, kv_full, kv_empty, tm_full, tm_free,
+                      drain, nb);
+    __syncwarp();
+  } else {
+    const int e = warp - 2, grp = e >> 2, quarter = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const int64_t bh = static_cast<int64_t>(b) * p.Hkv + h;
+    if (!kPass2) {
+      // ------------------------------------------------ pass 1: row statistics
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      const int nmt = p.Rp / 128;
+      for (int i = 0; i < nb && grp < nmt; ++i) {
+        const int buf = i % nbuf, use = i / nbuf;
+        const int j0 = (split + i * p.nsplit) * kTcKeys;
+        if (!warp_wait(tm_full + 8 * buf, use & 1u, p.err)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int mt = grp + 2 * k;
+          if (mt >= nmt) break;
+          uint32_t r[4][32];
+          const uint32_t ta = tmem + lane_base + buf * p.Rp + mt * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(ta + 32 * c, r[c]);
+          tmem_wait_ld();
+          if (mt + 2 >= nmt) {  // this warp's last read of the buffer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tm_free + 8 * buf);
+          }
+          const int row = mt * 128 + quarter * 32 + lane;
+          // keys past the first observed position are masked per row
+          const int lim = (j0 + kTcKeys - 1 > p.S - p.n_obs)
+                              ? p.S - p.n_obs + (row % p.n_obs) - j0
+                              : kTcKeys - 1;
+          stats_fold(r, lim, p.sl2, m[k], l[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int row = (grp + 2 * k) * 128 + quarter * 32 + lane;
+        if (grp + 2 * k < nmt && row < p.R)
+          p.part[(bh * p.nsplit + split) * p.R + row] = make_float2(m[k], l[k]);
+      }
+    } else {
+      // ------------------------------------------------ pass 2: weights per key
+      float* bias = reinterpret_cast<float*>(smem + Y.bias_off);
+      int* lim = reinterpret_cast<int*>(smem + Y.lim_off);
+      float* red = reinterpret_cast<float*>(smem + Y.red_off);
+      grid_dependency_wait();  // pass 1's statistics are complete and visible
+      for (int r = threadIdx.x - 64; r < p.Rp; r += kTcEpiWarps * 32) {
+        float bv = -INFINITY;
+        int lv = -1;
+        if (r < p.R) {
+          const float2* pr = p.part + bh * p.nsplit * p.R + r;
+          float M = -INFINITY;
+          for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, pr[static_cast<int64_t>(s) * p.R].x);
+          float Ls = 0.f;
+          for (int s = 0; s < p.nsplit; ++s) {
+            const float2 v = pr[static_cast<int64_t>(s) * p.R];
+            if (v.x != -INFINITY) Ls += v.y * exp2f(v.x - M);
+          }
+          // weight of score s: 2^(s sl2 - M) / Ls = 2^(s sl2 + bias)
+          bv = Ls > 0.f ? -(M + log2f(Ls)) : -INFINITY;
+          lv = p.S - p.n_obs + r % p.n_obs;
+        }
+        bias[r] = bv;
+        lim[r] = lv;
+      }
+      epi_sync();
+      const int half = p.Rp / 2, c_begin = grp * half;
+      const int key = quarter * 32 + lane;
+      const float2 sc = make_float2(p.sl2, p.sl2);
+      // every epilogue warp meets the others once per block, also after a
+      // timed-out wait (it then reads nothing more), so the named barrier
+      // never waits for a warp that left
+      bool ok = true;
+      for (int i = 0; i < nb; ++i) {
+        const int buf = i % nbuf, use = i / nbuf;
+        const int j0 = (split + i * p.nsplit) * kTcKeys, j = j0 + key;
+        const bool masked = j0 + kTcKeys - 1 > p.S - p.n_obs;
+        if (ok) ok = warp_wait(tm_full + 8 * buf, use & 1u, p.err);
+        tc_fence_after();
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        for (int c0 = c_begin; ok && c0 < c_begin + half; c0 += 64) {
+          uint32_t r[2][32];
+          const uint32_t ta = tmem + lane_base + buf * p.Rp + c0;
+          tmem_ld32(ta, r[0]);
+          tmem_ld32(ta + 32, r[1]);
+          tmem_wait_ld();
+          if (c0 + 64 >= c_begin + half) {  // this warp's last read of the buffer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tm_free + 8 * buf);
+          }
+#pragma unroll
+          for (int q = 0; q < 32; q += kTcEmuPeriod * 2) {
+#pragma unroll
+            for (int t = 0; t < kTcEmuPeriod * 2; ++t) {
+              if (q + t < 32) {
+                const int pr = q + t, c = c0 + 2 * pr;
+                const float2 bb = *reinterpret_cast<const float2*>(bias + c);
+                const float2 a = __ffma2_rn(make_float2(__uint_as_float(r[pr >> 4][(2 * pr) & 31]),
+                                                        __uint_as_float(r[pr >> 4][(2 * pr + 1) & 31])),
+                                            sc, bb);
+                float2 ev;
+                if (t % kTcEmuPeriod == kTcEmuPeriod - 1) ev = exp2_fma2(a);
+                else ev = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+                if (masked) {
+                  ev.x = j <= lim[c] ? ev.x : 0.f;
+                  ev.y = j <= lim[c + 1] ? ev.y : 0.f;
+                }
+                if (t & 1) acc1 = __fadd2_rn(acc1, ev);
+                else acc0 = __fadd2_rn(acc0, ev);
+              }
+            }
+          }
+        }
+        const float w = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        float* rb = red + (i & 1) * kTcKeys;
+        if (grp == 1) rb[key] = w;
+        epi_sync();
+        if (ok && grp == 0 && j < p.S) p.imp[bh * p.S + j] = w + rb[key];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<512>(tmem);
   }
 }
 
@@ -1048,51 +1052,69 @@ cudaError_t launch_tsa_scatter(const Launch& l, const void* Oc, const int32_t* i
 }
 
 size_t token_importance_scratch_bytes(int B, int S, int Hkv, int G, int n_obs) {
-  const int64_t nblk = (S + kImpKeys - 1) / kImpKeys;
+  // per-split row statistics of pass 1: at most one split per key block
+  const int64_t nblk = (S + kTcKeys - 1) / kTcKeys;
   const int64_t R = static_cast<int64_t>(G) * n_obs;
-  return static_cast<size_t>(B) * Hkv * R * 2 * 4 * (nblk + 1);
+  return static_cast<size_t>(B) * Hkv * R * 2 * 4 * nblk;
 }
 
 cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* K, int B, int S,
                                     int Hq, int Hkv, int D, int n_obs, float scale, float* imp,
-                                    float* scratch) {
+                                    float* scratch, std::string* why) {
   if (B == 0 || S == 0) return cudaSuccess;
-  const int G = Hq / Hkv, R = G * n_obs;
-  const int nblk = (S + kImpKeys - 1) / kImpKeys;
-  float* part = scratch;
-  float* stats = scratch + static_cast<size_t>(B) * Hkv * nblk * R * 2;
-  const size_t lds = static_cast<size_t>(D + 8) * 2;
-  const size_t sh1 = ((R + 31) / 32 * 32 + 2 * kImpKeys) * lds;
-  // pass 1 is persistent: about one CTA per SM over the (b, h) pairs
-  const int nsplit = std::max(1, std::min(nblk, l.num_sms / std::max(1, B * Hkv)));
-  const size_t sh2 = (R + kImpKeys) * lds + static_cast<size_t>(R) * 2 * 4;
-  const dim3 grid(nblk, Hkv, B);
-  const float sl2 = scale * kLog2eF;
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
-  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K);
-  cudaError_t e;
-  if (D == 128) {
-    e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<128>), sh1);
-    if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<128>), sh2);
-    if (e != cudaSuccess) return e;
-    imp_stats_kernel<128><<<dim3(nsplit, Hkv, B), kStatsThreads, sh1, l.stream>>>(
-        q, k, S, Hq, Hkv, G, n_obs, sl2, nblk, part);
-    imp_combine_kernel<<<dim3(B * Hkv, (R + 31) / 32), kCombineWarps * 32, 0, l.stream>>>(
-        part, nsplit, R, stats);
-    imp_weight_kernel<128><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
-                                                                 stats, imp);
-  } else {
-    e = set_smem_ts(reinterpret_cast<const void*>(imp_stats_kernel<64>), sh1);
-    if (e == cudaSuccess) e = set_smem_ts(reinterpret_cast<const void*>(imp_weight_kernel<64>), sh2);
-    if (e != cudaSuccess) return e;
-    imp_stats_kernel<64><<<dim3(nsplit, Hkv, B), kStatsThreads, sh1, l.stream>>>(
-        q, k, S, Hq, Hkv, G, n_obs, sl2, nblk, part);
-    imp_combine_kernel<<<dim3(B * Hkv, (R + 31) / 32), kCombineWarps * 32, 0, l.stream>>>(
-        part, nsplit, R, stats);
-    imp_weight_kernel<64><<<grid, kImpThreads, sh2, l.stream>>>(q, k, S, Hq, Hkv, G, n_obs, sl2,
-                                                                stats, imp);
+  ImpParams p{};
+  p.S = S;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_obs = n_obs;
+  p.R = p.G * n_obs;
+  p.Rp = (p.R + 127) & ~127;
+  p.D = D;
+  p.nblk = (S + kTcKeys - 1) / kTcKeys;
+  // about one CTA per SM over the (b, h) pairs
+  p.nsplit = std::max(1, std::min(p.nblk, l.num_sms / std::max(1, B * Hkv)));
+  p.qbox = std::min(256, n_obs & -n_obs);  // n_obs is a multiple of 8
+  p.sl2 = scale * kLog2eF;
+  p.part = reinterpret_cast<float2*>(scratch);
+  p.imp = imp;
+  p.err = l.err;
+  const int stage = kTcKeys * D * 2;
+  const size_t fixed = imp_layout(p.Rp, D, 0).total;
+  p.NS = static_cast<int>(std::min<size_t>(kTcMaxNS, (kTcMaxSmem - fixed) / stage));
+  if (p.NS < 2) {
+    if (why) *why = "token importance: observed rows do not fit in shared memory";
+    return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  const size_t smem = std::max(kTcMinSmem, imp_layout(p.Rp, D, p.NS).total);
+  CUtensorMap tmQ, tmK;
+  if (!make_tmap_bf16_2d(&tmQ, Q, static_cast<uint64_t>(B) * S, static_cast<uint64_t>(Hq) * D,
+                         static_cast<uint64_t>(Hq) * D, p.qbox, 64, why))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tmK, K, static_cast<uint64_t>(B) * Hkv * S, D, D, kTcKeys, 64, why))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(imp_tc_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(imp_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(p.nsplit, Hkv, B);
+  imp_tc_kernel<false><<<grid, kTcThreads, smem, l.stream>>>(tmQ, tmK, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // pass 2 behind pass 1 (programmatic dependent launch)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, imp_tc_kernel<true>, tmQ, tmK, p);
 }
 
 }  // namespace csa

@@ -36,8 +36,14 @@ def _oracle_importance(Q, K, b, h, G, n_obs, scale):
     return O.token_importance(np.concatenate(rows), to_np(K[b, h]), pos, scale)
 
 
+# observed rows R = (Hq/Hkv) n_obs: 256 (two 128-row tiles, double-buffered
+# accumulators), 128, 512 (single-buffered), 384, 8 (one tile, mostly zero
+# padding), 512 with n_obs = 512 (two 256-row copies per head), 48 with
+# n_obs = 24 (8-row copies); ragged key blocks (S % 128 != 0) and B > 1
 @pytest.mark.parametrize("B,S,Hq,Hkv,D,n_obs", [(1, 2048, 8, 2, 128, 64), (2, 1000, 4, 1, 64, 32),
-                                                (1, 4096, 16, 2, 128, 64)])
+                                                (1, 4096, 16, 2, 128, 64), (1, 777, 12, 2, 128, 64),
+                                                (1, 600, 2, 2, 64, 8), (1, 1536, 2, 2, 128, 512),
+                                                (3, 300, 8, 4, 128, 24)])
 def test_token_importance_matches_oracle(B, S, Hq, Hkv, D, n_obs):
     from query_adaptive_chunk_b200 import csa
     Q, K, _ = _inputs(B, S, Hq, Hkv, D, seed=S + D)
