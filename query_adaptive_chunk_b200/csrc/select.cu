@@ -1484,6 +1484,167 @@ int next_pow2(int x) {
   return p;
 }
 
+// ------------------------------------------------------------------ long rows (cluster)
+//
+// Top-k over long score rows with no forced entries (the Token Sparse
+// tokens, C >= kClTopkMinC): one cluster of kClTopkCS CTAs per unit, CTA r
+// holding the keys of positions [C r / CS, C (r + 1) / CS) in shared memory.
+// An MSB-first radix select over the keys' four bytes finds the k-th largest
+// key tau, the CTAs' 256-bucket histograms of each pass added through
+// distributed shared memory in rank order (integer counts: every CTA takes
+// the same bucket); the keys equal to tau are taken lowest position first
+// (the CTAs' counts of them meet the same way), and each CTA writes its kept
+// positions, ascending, after those of the CTAs before it.
+constexpr int kClTopkCS = 8;
+constexpr int kClTopkThreads = 512;
+constexpr int kClTopkMinC = 8192;
+
+__global__ void __launch_bounds__(kClTopkThreads) topk_cluster_kernel(
+    const float* __restrict__ scores, int C, int k_free, const int32_t* __restrict__ k_dev,
+    int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
+  cluster_arrive_relaxed();
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm);  // this CTA's positions
+  __shared__ unsigned int hc[256];                   // this CTA's histogram of the pass
+  __shared__ unsigned int gc[256];                   // the cluster's
+  __shared__ unsigned int part_eq[kClTopkCS], part_sel[kClTopkCS];
+  __shared__ int scan_sh[33];
+  __shared__ unsigned int pick_sh[2];  // the pass's bucket and the count above it
+  const int CS = static_cast<int>(cluster_size());
+  const int rank = static_cast<int>(cluster_rank());
+  const int u = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int lo = static_cast<int>(static_cast<int64_t>(C) * rank / CS);
+  const int n = static_cast<int>(static_cast<int64_t>(C) * (rank + 1) / CS) - lo;
+  const float* row = scores + static_cast<int64_t>(u) * C + lo;
+  for (int j = tid; j < n; j += blockDim.x) keys[j] = float_key(row[j]);
+  const int k = min(k_dev ? max(0, min(k_dev[u], kmax)) : max(0, min(k_free, kmax)), C);
+  __syncthreads();
+  cluster_wait();  // (phase 1) every CTA of the cluster is running
+  // keys > tau are taken, and the first `need` keys equal to tau
+  uint32_t tau = 0u;
+  unsigned int need = 0u;
+  if (k == 0) {
+    tau = 0xffffffffu;
+  } else if (k < C) {
+    uint32_t prefix = 0u, mask = 0u;
+    need = static_cast<unsigned int>(k);
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int d = tid; d < 256; d += blockDim.x) hc[d] = 0u;
+      __syncthreads();
+      for (int j0 = 0; j0 < n; j0 += blockDim.x) {
+        const int j = j0 + tid;
+        int d = -1;
+        if (j < n) {
+          const uint32_t key = keys[j];
+          if ((key & mask) == prefix) d = static_cast<int>((key >> shift) & 255u);
+        }
+        const unsigned int act = __ballot_sync(0xffffffffu, d >= 0);
+        if (d >= 0) {  // one shared atomic per distinct bucket of the warp
+          const unsigned int peers = __match_any_sync(act, d);
+          if (lane == __ffs(peers) - 1) atomicAdd(&hc[d], static_cast<unsigned int>(__popc(peers)));
+        }
+      }
+      cluster_arrive();  // every CTA's histogram of this pass is complete
+      cluster_wait();
+      for (int d = tid; d < 256; d += blockDim.x) {
+        unsigned int c = 0u;
+        for (int r = 0; r < CS; ++r) c += ld_cluster_u32(cluster_map(smem_u32(hc + d), r));
+        gc[d] = c;
+      }
+      cluster_arrive();  // every CTA has read the others' histograms (they may be cleared)
+      cluster_wait();
+      if (tid < 32) {  // the bucket where the count from the top reaches `need`
+        unsigned int pc[8], lc = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          pc[i] = gc[255 - 8 * lane - i];
+          lc += pc[i];
+        }
+        unsigned int sc = lc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned int t = __shfl_up_sync(0xffffffffu, sc, o);
+          if (lane >= o) sc += t;
+        }
+        unsigned int above = sc - lc;  // count in the buckets above this lane's eight
+        int sel = -1;
+        unsigned int above_sel = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (sel < 0) {
+            if (above + pc[i] >= need) {
+              sel = 255 - 8 * lane - i;
+              above_sel = above;
+            } else {
+              above += pc[i];
+            }
+          }
+        }
+        // `need` never exceeds the count of keys under the prefix: a bucket is hit
+        const unsigned int hit = __ballot_sync(0xffffffffu, sel >= 0);
+        if (lane == (hit ? __ffs(hit) - 1 : 0)) {
+          pick_sh[0] = sel < 0 ? 0u : static_cast<unsigned int>(sel);
+          pick_sh[1] = above_sel;
+        }
+      }
+      __syncthreads();
+      prefix |= pick_sh[0] << shift;
+      mask |= 255u << shift;
+      need -= pick_sh[1];
+      __syncthreads();  // pick_sh read before the next pass writes it
+    }
+    tau = prefix;
+  }
+  // this thread's segment of the CTA's positions: keys above tau, keys at tau
+  const int seg = (n + blockDim.x - 1) / blockDim.x;
+  const int s0 = min(n, tid * seg), s1 = min(n, s0 + seg);
+  int c_gt = 0, c_eq = 0;
+  for (int j = s0; j < s1; ++j) {
+    const uint32_t key = keys[j];
+    c_gt += key > tau;
+    c_eq += key == tau;
+  }
+  int eq_tot = 0;
+  const int eq_base = block_exclusive_scan(c_eq, scan_sh, &eq_tot);
+  if (tid < CS) st_cluster_u32(cluster_map(smem_u32(part_eq + rank), tid), static_cast<unsigned int>(eq_tot));
+  cluster_arrive();
+  cluster_wait();
+  int eq_before = 0;
+  for (int r = 0; r < rank; ++r) eq_before += static_cast<int>(part_eq[r]);
+  const int take = max(0, min(static_cast<int>(need) - eq_before, eq_tot));  // ties kept here
+  const int c_sel = c_gt + max(0, min(take - eq_base, c_eq));
+  int sel_tot = 0;
+  const int sel_base = block_exclusive_scan(c_sel, scan_sh, &sel_tot);
+  if (tid < CS) st_cluster_u32(cluster_map(smem_u32(part_sel + rank), tid), static_cast<unsigned int>(sel_tot));
+  cluster_arrive();
+  cluster_wait();  // the last access to another CTA's shared memory is before this barrier
+  int sel_before = 0, total = 0;
+  for (int r = 0; r < CS; ++r) {
+    const int v = static_cast<int>(part_sel[r]);
+    if (r < rank) sel_before += v;
+    total += v;
+  }
+  int32_t* out = idx + static_cast<int64_t>(u) * kmax;
+  int pos = sel_before + sel_base, eq_seen = eq_base;
+  for (int j = s0; j < s1; ++j) {
+    const uint32_t key = keys[j];
+    bool t = key > tau;
+    if (key == tau) {
+      t = eq_seen < take;
+      ++eq_seen;
+    }
+    if (t) {
+      if (pos < kmax) out[pos] = lo + j;
+      ++pos;
+    }
+  }
+  const int tot = min(total, kmax);
+  const int f0 = tot + static_cast<int>(static_cast<int64_t>(kmax - tot) * rank / CS);
+  const int f1 = tot + static_cast<int>(static_cast<int64_t>(kmax - tot) * (rank + 1) / CS);
+  for (int i = f0 + tid; i < f1; i += blockDim.x) out[i] = -1;
+  if (rank == 0 && tid == 0) count[u] = tot;
+}
+
 cudaError_t set_smem(const void* fn, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1497,6 +1658,27 @@ cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int 
                                int32_t* idx, int32_t* count, int kmax, const int32_t* k_dev,
                                int causal_tiles, int causal_tile_m, int causal_L) {
   if (U == 0) return cudaSuccess;
+  if (n_valid == nullptr && causal_tiles == 0 && n_sink == 0 && n_local == 0 &&
+      C >= kClTopkMinC && U <= 65535 && static_cast<int64_t>(U) * kClTopkCS <= l.num_sms) {
+    // long rows, nothing forced: one cluster per unit
+    const size_t shc = static_cast<size_t>((C + kClTopkCS - 1) / kClTopkCS) * 4;
+    cudaError_t e = set_smem(reinterpret_cast<const void*>(topk_cluster_kernel), shc);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClTopkCS, U);
+    cfg.blockDim = dim3(kClTopkThreads);
+    cfg.dynamicSmemBytes = shc;
+    cfg.stream = l.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClTopkCS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, C, k_free, k_dev, idx, count,
+                              kmax);
+  }
   const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_topk_kernel), sh);
   if (e != cudaSuccess) return e;

@@ -675,17 +675,6 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const float* __r
 constexpr int kBudgetCS = 8;
 constexpr int kBudgetCThreads = 512;
 
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-
 __global__ void __launch_bounds__(kBudgetCThreads) budget_cluster_kernel(
     const float* __restrict__ imp, int S, int Hkv, float tau, int tile, int32_t* __restrict__ k_seq,
     int32_t* __restrict__ k_unit) {

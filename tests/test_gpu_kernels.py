@@ -137,6 +137,51 @@ def test_select_topk_exact(csa, C, U, kind):
             assert got[u] == ref, (u, k_free, n_sink, n_local)
 
 
+@pytest.mark.parametrize("C,U,kind", [(8192, 3, "normal"), (20000, 2, "ints"), (32768, 18, "ints"),
+                                      (9000, 4, "zeros")])
+def test_select_topk_long_rows_cluster(csa, C, U, kind):
+    """Long rows with nothing forced (one cluster per unit, radix select over
+    the cluster, ties to the lower index across the CTAs' ranges): the same
+    sets as the oracle for k from 0 to past C, many equal scores included."""
+    if kind == "normal":
+        s = _randn((U, C), 31)
+    elif kind == "ints":
+        s = torch.randint(-3, 4, (U, C), generator=_gen(32), device="cuda").float()
+    else:
+        s = torch.zeros(U, C, device="cuda")
+        s[:, ::3] = -0.0
+        s[:, 5::7] = 1.0
+    sn = s.cpu().double().numpy()
+    rng = np.random.default_rng(C + U)
+    for k_free in [0, 1, 7, C // 3, C - 1, C, C + 5, int(rng.integers(1, C))]:
+        got = _run_topk(csa, s, k_free, 0, 0, kmax=C)
+        for u in range(U):
+            ref, _ = O.select_topk(sn[u], k_free, 0, 0)
+            assert got[u] == ref, (u, k_free)
+
+
+@pytest.mark.parametrize("S,B,Hkv", [(32768, 1, 8), (8192, 2, 3)])
+def test_token_select_per_unit_k(csa, S, B, Hkv):
+    """csa_token_select: each unit's own k from device memory (0, 1, ties at
+    the cut, S) through the cluster path, against the oracle's top-k."""
+    U = B * Hkv
+    g = _gen(33)
+    imp = torch.randint(0, 50, (B, Hkv, S), generator=g, device="cuda").float() / 7.0
+    ks = [0, 1, S, S // 2, S - 1] + [int(x) for x in np.random.default_rng(S).integers(1, S, U)]
+    k_unit = torch.tensor(ks[:U], dtype=torch.int32, device="cuda")
+    idx = torch.full((U, S), 777, dtype=torch.int32, device="cuda")
+    cnt = torch.full((U,), 777, dtype=torch.int32, device="cuda")
+    csa.csa_token_select(imp, B, S, Hkv, k_unit, idx, cnt)
+    csa.csa_check_device_status()
+    got = parity.gpu_sets(idx, cnt)
+    isn = imp.reshape(U, S).cpu().double().numpy()
+    idx_h = idx.cpu().numpy()
+    for u in range(U):
+        ref, _ = O.select_topk(isn[u], ks[u], 0, 0)
+        assert got[u] == ref, (u, ks[u])
+        assert np.all(idx_h[u, len(ref):] == -1)
+
+
 def test_select_topk_n_valid(csa):
     """Causal units: each sees only chunks [0, n_valid) (0, 1, 2 and ragged)."""
     C, U = 515, 40
