@@ -1020,8 +1020,10 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
                                                reinterpret_cast<float*>(ws + w.scratch), &why);
   if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
   if (e == cudaSuccess) e = csa::launch_token_budget(l, imp, B, S, Hkv, tau, 64, budget_out, k_unit);
+  bool inv_ready = false;  // the selection may write the position -> slot map itself
   if (e == cudaSuccess)  // each KV head's own top tokens under the (rounded) budget
-    e = csa::launch_select_topk(l, imp, U, S, nullptr, 0, 0, 0, idx, cnt, S, k_unit);
+    e = csa::launch_select_topk(l, imp, U, S, nullptr, 0, 0, 0, idx, cnt, S, k_unit, 0, 0, 0,
+                                reinterpret_cast<int32_t*>(ws + w.inv), &inv_ready);
   if (e != cudaSuccess) return finish(e, "token selection launch");
   // Compress, attend, decompress with no read-back of the budgets: the
   // buffers are laid out for S kept tokens, the gather writes the kept rows
@@ -1042,7 +1044,7 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
   if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
   if (e == cudaSuccess)
     e = csa::launch_tsa_scatter(l, Oc, idx, cnt, S, B, S, S, Hq, Hkv, D,
-                                reinterpret_cast<int32_t*>(ws + w.inv), O);
+                                reinterpret_cast<int32_t*>(ws + w.inv), O, inv_ready);
   return finish(e, "token sparse prefill launch");
 }
 

@@ -38,12 +38,15 @@ cudaError_t launch_score(const Launch& l, const void* q, bool bf16, const float*
 // select.cu
 // causal_tiles > 0: unit u is query tile u % causal_tiles of a causal
 // prefill and sees the chunks c < ((t + 1) * causal_tile_m - 1) / causal_L + 1
-// (n_valid is then ignored)
+// (n_valid is then ignored).  inv (optional, [U, C]): when the long-row
+// cluster kernel runs, it also writes every position's slot in its unit's
+// list (or -1) and sets *inv_done; otherwise *inv_done is false.
 cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax,
                                const int32_t* k_dev = nullptr, int causal_tiles = 0,
-                               int causal_tile_m = 0, int causal_L = 0);
+                               int causal_tile_m = 0, int causal_L = 0, int32_t* inv = nullptr,
+                               bool* inv_done = nullptr);
 cudaError_t launch_select_topp(const Launch& l, const float* scores, int U, int C,
                                float logit_scale, float p, int budget, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax, int32_t* n_p_out);
@@ -75,9 +78,11 @@ cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, con
                               int Sc, int Hq, int Hkv, int D, void* Qc, void* Kc, void* Vc);
 cudaError_t launch_tsa_lists(const Launch& l, const int32_t* k_unit, int U, int n_tiles, int tile,
                              int32_t* lists, int32_t* counts);
+// inv [B*Hkv, S] (scratch): built here from idx/count unless inv_ready (the
+// selection wrote it)
 cudaError_t launch_tsa_scatter(const Launch& l, const void* Oc, const int32_t* idx,
                                const int32_t* count, int kmax, int B, int S, int Sc, int Hq,
-                               int Hkv, int D, int32_t* inv, void* O);
+                               int Hkv, int D, int32_t* inv, void* O, bool inv_ready = false);
 
 // rope.cu
 cudaError_t launch_rope(const Launch& l, const void* x, void* y, bool bf16, int64_t rows, int D,

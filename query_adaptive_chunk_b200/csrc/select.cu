@@ -1367,6 +1367,158 @@ __global__ void __launch_bounds__(kClSelThreads) score_select_topk_cluster_kerne
   emit_with_forced(out_l, n_out, C, n_sink, n_local, row, count + u, kmax);
 }
 
+// Per-head top-k with the GQA union by a cluster of CS CTAs per unit: CTA r
+// loads the summary rows of the r-th range of the unit's chunks once and
+// scores them against each of the G query heads' own (projected) queries;
+// per head it keeps its best min(k_free, candidates) by rank.  The first
+// CTA gathers every head's candidates, takes each head's k_free best (the
+// same argument as for one head: a chunk among a head's best k_free overall
+// is among that head's best of its own range), marks their union, adds the
+// forced chunks and writes the ascending list.
+template <int DS>
+__device__ __forceinline__ void cluster_scores_heads(const float* __restrict__ summ_u, int lo,
+                                                     int n, int C, const float* qall, int G,
+                                                     int n_sink, int n_local, uint64_t* comp,
+                                                     int stride,
+                                                     const float4 (&pre)[kClRowBatch]) {
+  constexpr int LPR = DS / 4, RPI = 32 / LPR;
+  const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int sub = lane % LPR, rsub = lane / LPR;
+  const int first = rows_first<DS>(n);
+  for (int base = first; base < n; base += nw * RPI * kClRowBatch) {
+    float4 v[kClRowBatch];
+    if (base == first) {
+#pragma unroll
+      for (int b = 0; b < kClRowBatch; ++b) v[b] = pre[b];
+    } else {
+      rows_issue<DS>(summ_u, lo, n, nullptr, base, v);
+    }
+    for (int g = 0; g < G; ++g) {
+      const float* qv = qall + g * DS;
+      const float4 q4 = make_float4(qv[sub * 4], qv[sub * 4 + 1], qv[sub * 4 + 2], qv[sub * 4 + 3]);
+#pragma unroll
+      for (int b = 0; b < kClRowBatch; ++b) {
+        float x = v[b].x * q4.x + v[b].y * q4.y + v[b].z * q4.z + v[b].w * q4.w;
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        const int i = base + b * RPI + rsub;
+        if (sub == 0 && i < n) {
+          const int c = lo + i;
+          comp[g * stride + i] = is_forced(c, C, n_sink, n_local) ? 0ull : composite(float_key(x), c);
+        }
+      }
+    }
+  }
+}
+
+// Dynamic shared memory of the union kernel: qall [G][DS] f32 | comp
+// [G][per] | kept [G][KL] | cand [G][CS][KL] (u64) | out_l [C + 64] i32 |
+// flags [C] u8.
+__host__ __device__ inline size_t union_cl_bytes(int G, int DS, int per, int KL, int CS, int C) {
+  return static_cast<size_t>(G) * DS * 4 + static_cast<size_t>(G) * (per + KL + CS * KL) * 8 +
+         static_cast<size_t>(C + 64) * 4 + static_cast<size_t>(C + 15) / 16 * 16;
+}
+
+template <int DS>
+__global__ void __launch_bounds__(kClSelThreads) score_select_union_cluster_kernel(
+    const void* __restrict__ q, int q_bf16, const float* __restrict__ proj, int R,
+    const float* __restrict__ summ, int Hq, int Hkv, int D, int C,
+    const uint8_t* __restrict__ head_full, int k_free, int n_sink, int n_local,
+    int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
+  allow_dependent_launch();
+  cluster_arrive_relaxed();  // every CTA of the cluster runs by the matching wait
+  __shared__ FusedSmem f;
+  __shared__ int n_kept[8];
+  __shared__ int n_out;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int CS = static_cast<int>(cluster_size());
+  const int rank = static_cast<int>(cluster_rank());
+  const int u = blockIdx.y, h = u % Hkv, b = u / Hkv, G = Hq / Hkv;
+  const int per = (C + CS - 1) / CS;
+  const int lo = static_cast<int>(static_cast<int64_t>(C) * rank / CS);
+  const int n = static_cast<int>(static_cast<int64_t>(C) * (rank + 1) / CS) - lo;
+  const int KL = k_free < per ? k_free : per;  // slots per CTA and head
+  float* qall = reinterpret_cast<float*>(dsm);
+  uint64_t* comp = reinterpret_cast<uint64_t*>(dsm + static_cast<size_t>(G) * DS * 4);
+  uint64_t* kept = comp + static_cast<size_t>(G) * per;
+  uint64_t* cand = kept + static_cast<size_t>(G) * KL;
+  int32_t* out_l = reinterpret_cast<int32_t*>(cand + static_cast<size_t>(G) * CS * KL);
+  uint8_t* flags = reinterpret_cast<uint8_t*>(out_l + C + 64);
+  const bool full = head_full != nullptr && head_full[h];
+  if (threadIdx.x < 8) n_kept[threadIdx.x] = 0;
+  if (!full) {
+    const float* summ_u = summ + static_cast<int64_t>(u) * C * DS;
+    float4 pre[kClRowBatch];
+    rows_issue<DS>(summ_u, lo, n, nullptr, rows_first<DS>(n), pre);  // in flight with the queries
+    // the G heads' queries in one round of loads, then each projected (the
+    // same partition and order as unit_query)
+    const int64_t head0 = static_cast<int64_t>(b) * Hq + h * G;
+    float* qs_all = proj ? f.qs : qall;  // [G][D]
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+      const int64_t off = head0 * D + e;
+      qs_all[e] = q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
+                         : static_cast<const float*>(q)[off];
+    }
+    __syncthreads();
+    if (proj) {
+      const int parts = 256 / R;
+      for (int g = 0; g < G; ++g) {
+        if (threadIdx.x < 256) {
+          const int r = threadIdx.x / parts, pt = threadIdx.x % parts;
+          const int dchunk = (D + parts - 1) / parts;
+          const int d0 = pt * dchunk, d1 = min(D, d0 + dchunk);
+          float acc = 0.f;
+#pragma unroll 4
+          for (int d = d0; d < d1; ++d)
+            acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * qs_all[g * D + d];
+          for (int o = parts >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (pt == 0) qall[g * DS + r] = acc;
+        }
+      }
+      __syncthreads();
+    }
+    cluster_scores_heads<DS>(summ_u, lo, n, C, qall, G, n_sink, n_local, comp, per, pre);
+    __syncthreads();
+    for (int g = 0; g < G; ++g) rank_keep(comp + g * per, n, k_free, kept + g * KL, &n_kept[g]);
+  }
+  __syncthreads();
+  cluster_wait();  // (phase 1)
+  if (!full) {  // each head's kept candidates into this CTA's slots of the first CTA
+    for (int g = 0; g < G; ++g) {
+      const uint32_t dst = cluster_map(smem_u32(cand + (static_cast<size_t>(g) * CS + rank) * KL), 0);
+      const int nk = n_kept[g];
+      for (int i = threadIdx.x; i < KL; i += blockDim.x)
+        st_cluster_u64(dst + i * 8, i < nk ? kept[g * KL + i] : 0ull);
+    }
+  }
+  cluster_arrive();  // (phase 2)
+  cluster_wait();
+  if (rank != 0) return;
+  int32_t* row = idx + static_cast<int64_t>(u) * kmax;
+  if (full) {  // full heads read every chunk: no list
+    for (int i = threadIdx.x; i < kmax; i += blockDim.x) row[i] = -1;
+    if (threadIdx.x == 0) count[u] = 0;
+    return;
+  }
+  for (int c = threadIdx.x; c < C; c += blockDim.x) flags[c] = 0;
+  if (threadIdx.x == 0) n_out = 0;
+  __syncthreads();
+  const int nc = CS * KL;
+  for (int e = threadIdx.x; e < G * nc; e += blockDim.x) {  // each head's k_free best
+    const uint64_t* hc = cand + static_cast<size_t>(e / nc) * nc;
+    const uint64_t me = hc[e % nc];
+    if (me == 0ull) continue;
+    int above = 0;
+    for (int j = 0; j < nc; ++j) above += hc[j] > me;
+    if (above < k_free) flags[comp_index(me)] = 1;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x)
+    if (flags[c]) out_l[atomicAdd(&n_out, 1)] = c;
+  __syncthreads();
+  emit_with_forced(out_l, n_out, C, n_sink, n_local, row, count + u, kmax);
+}
+
 // Two-level selection by a cluster of CS CTAs per unit: the meta-chunks'
 // scores split over the CTAs, each keeping its best by rank; the first CTA
 // ranks the kept metas and hands the ascending list of the top_meta best to
@@ -1494,14 +1646,15 @@ int next_pow2(int x) {
 // distributed shared memory in rank order (integer counts: every CTA takes
 // the same bucket); the keys equal to tau are taken lowest position first
 // (the CTAs' counts of them meet the same way), and each CTA writes its kept
-// positions, ascending, after those of the CTAs before it.
+// positions, ascending, after those of the CTAs before it.  `inv` (optional,
+// [U, C]): for every position its slot in the unit's list, or -1.
 constexpr int kClTopkCS = 8;
 constexpr int kClTopkThreads = 512;
 constexpr int kClTopkMinC = 8192;
 
 __global__ void __launch_bounds__(kClTopkThreads) topk_cluster_kernel(
     const float* __restrict__ scores, int C, int k_free, const int32_t* __restrict__ k_dev,
-    int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax) {
+    int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax, int32_t* __restrict__ inv) {
   cluster_arrive_relaxed();
   extern __shared__ __align__(16) uint8_t sm[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(sm);  // this CTA's positions
@@ -1625,6 +1778,7 @@ __global__ void __launch_bounds__(kClTopkThreads) topk_cluster_kernel(
     total += v;
   }
   int32_t* out = idx + static_cast<int64_t>(u) * kmax;
+  int32_t* inv_row = inv ? inv + static_cast<int64_t>(u) * C + lo : nullptr;
   int pos = sel_before + sel_base, eq_seen = eq_base;
   for (int j = s0; j < s1; ++j) {
     const uint32_t key = keys[j];
@@ -1633,6 +1787,7 @@ __global__ void __launch_bounds__(kClTopkThreads) topk_cluster_kernel(
       t = eq_seen < take;
       ++eq_seen;
     }
+    if (inv_row) inv_row[j] = t && pos < kmax ? pos : -1;
     if (t) {
       if (pos < kmax) out[pos] = lo + j;
       ++pos;
@@ -1656,7 +1811,9 @@ cudaError_t set_smem(const void* fn, size_t bytes) {
 cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax, const int32_t* k_dev,
-                               int causal_tiles, int causal_tile_m, int causal_L) {
+                               int causal_tiles, int causal_tile_m, int causal_L, int32_t* inv,
+                               bool* inv_done) {
+  if (inv_done) *inv_done = false;
   if (U == 0) return cudaSuccess;
   if (n_valid == nullptr && causal_tiles == 0 && n_sink == 0 && n_local == 0 &&
       C >= kClTopkMinC && U <= 65535 && static_cast<int64_t>(U) * kClTopkCS <= l.num_sms) {
@@ -1676,8 +1833,10 @@ cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, C, k_free, k_dev, idx, count,
-                              kmax);
+    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, C, k_free, k_dev, idx, count, kmax,
+                           inv);
+    if (e == cudaSuccess && inv_done) *inv_done = inv != nullptr;
+    return e;
   }
   const size_t sh = sort_exch_bytes(C) + static_cast<size_t>(C) * 5 + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_topk_kernel), sh);
@@ -1810,6 +1969,48 @@ int select_cluster_size(int U, int C, int k_free, int n_sink, int n_local, int n
   return 0;
 }
 
+// Cluster size for the per-head union (G query heads per unit), or 0.
+int union_cluster_size(int U, int G, int C, int k_free, int n_sink, int n_local, int DS,
+                       bool projected, int D, int num_sms) {
+  if (U <= 0 || U > 65535 || C <= 0 || G > 8 || n_sink + n_local > 64) return 0;
+  if (projected && G * D > 1024) return 0;  // the heads' raw queries share one 1024-float buffer
+  for (int CS = 8; CS >= 2; CS >>= 1) {
+    if (static_cast<int64_t>(U) * CS > num_sms) continue;
+    const int per = (C + CS - 1) / CS;
+    const int KL = std::min(k_free, per);
+    if (per <= kClRangeMax && CS * KL <= kClCandMax &&
+        union_cl_bytes(G, DS, per, KL, CS, C) <= 160 * 1024)
+      return CS;
+  }
+  return 0;
+}
+
+template <int DS>
+cudaError_t cluster_union_kernel(const Launch& l, const void* q, bool bf16, const float* proj,
+                                 int R, const float* summ, int U, int Hq, int Hkv, int D, int C,
+                                 const uint8_t* head_full, int k_free, int n_sink, int n_local,
+                                 int32_t* idx, int32_t* count, int kmax, int CS) {
+  const int G = Hq / Hkv, per = (C + CS - 1) / CS;
+  const size_t sh = union_cl_bytes(G, DS, per, std::min(k_free, per), CS, C);
+  cudaError_t e = set_smem(reinterpret_cast<const void*>(score_select_union_cluster_kernel<DS>), sh);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, U);
+  cfg.blockDim = dim3(kClSelThreads);
+  cfg.dynamicSmemBytes = sh;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_select_union_cluster_kernel<DS>, q, bf16 ? 1 : 0, proj, R,
+                            summ, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count,
+                            kmax);
+}
+
 template <int DS>
 cudaError_t cluster_topk_kernel(const Launch& l, const void* q, bool bf16, const float* proj,
                                 int R, const float* summ, int U, int Hq, int Hkv, int D, int C,
@@ -1838,6 +2039,19 @@ cudaError_t launch_score_select_topk(const Launch& l, const void* q, bool bf16, 
                                      int32_t* idx, int32_t* count, int kmax, bool per_head_union) {
   const int U = B * Hkv;
   if (U == 0) return cudaSuccess;
+  const int DSel = proj ? R : D;
+  const int CSu = per_head_union ? union_cluster_size(U, Hq / Hkv, C, k_free, n_sink, n_local,
+                                                      DSel, proj != nullptr, D, l.num_sms)
+                                 : 0;
+  if (CSu > 0) {
+    switch (DSel) {
+      case 16: return cluster_union_kernel<16>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CSu);
+      case 32: return cluster_union_kernel<32>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CSu);
+      case 64: return cluster_union_kernel<64>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CSu);
+      case 128: return cluster_union_kernel<128>(l, q, bf16, proj, R, summ, U, Hq, Hkv, D, C, head_full, k_free, n_sink, n_local, idx, count, kmax, CSu);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   const int CS = per_head_union ? 0 : select_cluster_size(U, C, k_free, n_sink, n_local, l.num_sms);
   if (CS > 0) {
     switch (proj ? R : D) {

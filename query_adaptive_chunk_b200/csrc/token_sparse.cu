@@ -48,18 +48,20 @@ namespace {
 //            256 per MMA).  TMEM lane = key: each thread sums its key's
 //            weights 2^(s - max_r - log2 sum_r) along its own TMEM lane.
 // Warp 0 issues the TMA copies, warp 1 owns the tensor memory and one of its
-// threads issues the MMAs, warps 2-9 are two warpgroups that read the
+// threads issues the MMAs, warps 2-17 are four warpgroups that read the
 // accumulators (warp w reaches TMEM lanes 32 (w % 4) .. + 31): in pass 1
-// warpgroup g takes the 128-row tiles g and g + 2; in pass 2 it takes half
-// of the observed rows, and the halves' sums meet in shared memory.  A third
-// of the exponentials run on the FMA pipe.  Pass 2 is launched behind pass 1
+// warpgroup g takes the 128-row tiles g % 2 and g % 2 + 2, keys of half g / 2
+// of each block (the halves keep separate row statistics, written as two
+// splits); in pass 2 it takes a quarter of the observed rows, and the
+// quarters' sums meet in shared memory.  A third of the exponentials run on
+// the FMA pipe.  Pass 2 is launched behind pass 1
 // with programmatic dependent launch: its copies and MMAs start while pass 1
 // drains, and its epilogue waits (griddepcontrol.wait) for pass 1's per-split
 // row statistics, which it combines itself.  Pass 1 reads K with the default
 // L2 policy so that pass 2, which reads it last, finds much of it in L2.
 
 constexpr int kTcKeys = 128;
-constexpr int kTcEpiWarps = 8;
+constexpr int kTcEpiWarps = 16;
 constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;
 constexpr int kTcMaxNS = 4;
 constexpr size_t kTcMinSmem = 120 * 1024;  // one CTA per SM: it allocates all 512 TMEM columns
@@ -70,13 +72,13 @@ constexpr float kLog2eF = 1.4426950408889634f;
 struct ImpParams {
   int S, Hkv, G, n_obs, R, Rp, D, nblk, nsplit, NS, qbox;
   float sl2;    // scale * log2(e)
-  float2* part;  // [B, Hkv, nsplit, R]: (max, sum of 2^(s - max)) per split, log2 units
+  float2* part;  // [B, Hkv, 2 nsplit, R]: (max, sum of 2^(s - max)) per split and key half, log2 units
   float* imp;    // [B, Hkv, S]
   DevErr err;
 };
 
 // Shared-memory layout, offsets from the 1024-aligned base: Q slabs | K
-// stages | mbarriers + TMEM slot | pass 2: bias[Rp], lim[Rp], red[2][128].
+// stages | mbarriers + TMEM slot | pass 2: bias[Rp], lim[Rp], red[2][3][128].
 struct ImpLayout {
   int kv_off, stage_bytes, bar_off, bias_off, lim_off, red_off;
   size_t total;
@@ -90,7 +92,7 @@ __host__ __device__ inline ImpLayout imp_layout(int Rp, int D, int NS) {
   y.bias_off = y.bar_off + 256;
   y.lim_off = y.bias_off + Rp * 4;
   y.red_off = y.lim_off + Rp * 4;
-  y.total = 1024 + static_cast<size_t>(y.red_off) + 2 * kTcKeys * 4;
+  y.total = 1024 + static_cast<size_t>(y.red_off) + 2 * 3 * kTcKeys * 4;
   return y;
 }
 
@@ -197,53 +199,89 @@ __device__ void imp_mma(const ImpParams& p, uint32_t tmem, uint32_t sQ, uint32_t
 }
 
 // 2^x of a pair, every kTcEmuPeriod-th pair on the FMA pipe.
-template <int PAIR>
-__device__ __forceinline__ float2 exp2_pair(float2 a) {
-  if (PAIR % kTcEmuPeriod == kTcEmuPeriod - 1) return exp2_fma2(a);
-  return make_float2(fast_exp2(a.x), fast_exp2(a.y));
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ int2 lds_s2(uint32_t addr) {
+  int2 v;
+  asm volatile("ld.shared.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
 }
 
-// Pass 1 epilogue, one 128-key block for one row: x = the row's raw scores
-// against the block's keys, keys i <= lim visible (lim >= 127: all); folds
-// them into the running (m: max of s * sl2, l: sum of 2^(s sl2 - m)).
-__device__ __forceinline__ void stats_fold(const uint32_t (&r)[4][32], int lim, float sl2,
+// Pass 1 epilogue, one row against 64 keys of a block: x = the raw scores,
+// keys i <= lim visible (lim >= 63: all); folds them into the running (m:
+// max of s * sl2, l: sum of 2^(s sl2 - m)).
+__device__ __forceinline__ void stats_fold(const uint32_t (&r)[2][32], int lim, float sl2,
                                            float& m, float& l) {
-  float x[128];
+  float x[64];
 #pragma unroll
-  for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(r[i >> 5][i & 31]);
-  if (lim < 127) {
+  for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(r[i >> 5][i & 31]);
+  if (lim < 63) {
 #pragma unroll
-    for (int i = 0; i < 128; ++i) x[i] = i <= lim ? x[i] : -INFINITY;
+    for (int i = 0; i < 64; ++i) x[i] = i <= lim ? x[i] : -INFINITY;
   }
-  float mq[4];
+  float mq[2];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
+  for (int a = 0; a < 2; ++a) {
     float v = fmax3(x[32 * a], x[32 * a + 1], x[32 * a + 2]);
 #pragma unroll
     for (int k = 3; k < 31; k += 2) v = fmax3(v, x[32 * a + k], x[32 * a + k + 1]);
     mq[a] = fmaxf(v, x[32 * a + 31]);
   }
-  const float mn = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]) * sl2;
+  const float mn = fmaxf(mq[0], mq[1]) * sl2;
   const float mnew = fmaxf(m, mn);
   if (mnew == -INFINITY) return;  // no visible key yet
   const float2 sc = make_float2(sl2, sl2), nb = make_float2(-mnew, -mnew);
-  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int q = 0; q < 64; q += kTcEmuPeriod * 2) {
+  for (int q = 0; q < 32; q += kTcEmuPeriod * 2) {
 #pragma unroll
     for (int t = 0; t < kTcEmuPeriod * 2; ++t) {
-      if (q + t < 64) {
+      if (q + t < 32) {
         const float2 a = __ffma2_rn(make_float2(x[2 * (q + t)], x[2 * (q + t) + 1]), sc, nb);
         float2 e;
         if (t % kTcEmuPeriod == kTcEmuPeriod - 1) e = exp2_fma2(a);
         else e = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-        if (t & 1) acc1 = __fadd2_rn(acc1, e);
-        else acc0 = __fadd2_rn(acc0, e);
+        acc[(q + t) & 3] = __fadd2_rn(acc[(q + t) & 3], e);
       }
     }
   }
-  l = l * fast_exp2(m - mnew) + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
+  const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+  l = l * fast_exp2(m - mnew) + ((s01.x + s01.y) + (s23.x + s23.y));
   m = mnew;
+}
+
+// Pass 2 epilogue, one key against 32 observed rows c0 .. c0 + 31: adds
+// 2^(s sl2 + bias_c) over the rows it may see (all unless `masked`: then
+// only rows whose position lim_c >= j).
+__device__ __forceinline__ void weight_fold(const uint32_t (&r)[32], uint32_t bias_a,
+                                            uint32_t lim_a, int c0, bool masked, int j, float sl2,
+                                            float2 (&acc)[4]) {
+  const float2 sc = make_float2(sl2, sl2);
+#pragma unroll
+  for (int q = 0; q < 16; q += kTcEmuPeriod * 2) {
+#pragma unroll
+    for (int t = 0; t < kTcEmuPeriod * 2; ++t) {
+      if (q + t < 16) {
+        const int pr = q + t, c = c0 + 2 * pr;
+        const float2 bb = lds_f2(bias_a + c * 4);
+        const float2 a =
+            __ffma2_rn(make_float2(__uint_as_float(r[2 * pr]), __uint_as_float(r[2 * pr + 1])), sc, bb);
+        float2 ev;
+        if (t % kTcEmuPeriod == kTcEmuPeriod - 1) ev = exp2_fma2(a);
+        else ev = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+        if (masked) {
+          const int2 lm = lds_s2(lim_a + c * 4);
+          ev.x = j <= lm.x ? ev.x : 0.f;
+          ev.y = j <= lm.y ? ev.y : 0.f;
+        }
+        acc[pr & 3] = __fadd2_rn(acc[pr & 3], ev);
+      }
+    }
+  }
 }
 
 template <bool kPass2>
@@ -270,9 +308,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(kv_full + 8 * s, 1);
       mbar_init(kv_empty + 8 * s, 1);
     }
-    // pass 1: the warps of each warpgroup that has a 128-row tile read the
-    // accumulator; pass 2: all eight
-    const int readers = kPass2 ? kTcEpiWarps : 4 * min(2, p.Rp / 128);
+    // pass 1: the warps of the warpgroups that have a 128-row tile read the
+    // accumulator (two per tile parity); pass 2: all of them
+    const int readers = kPass2 ? kTcEpiWarps : 8 * min(2, p.Rp / 128);
     for (int k = 0; k < 2; ++k) {
       mbar_init(tm_full + 8 * k, 1);
       mbar_init(tm_free + 8 * k, readers);
@@ -315,21 +353,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int64_t bh = static_cast<int64_t>(b) * p.Hkv + h;
     if (!kPass2) {
       // ------------------------------------------------ pass 1: row statistics
+      const int tp = grp & 1, kh = grp >> 1;  // tile parity, key half
       float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
       const int nmt = p.Rp / 128;
-      for (int i = 0; i < nb && grp < nmt; ++i) {
+      for (int i = 0; i < nb && tp < nmt; ++i) {
         const int buf = i % nbuf, use = i / nbuf;
-        const int j0 = (split + i * p.nsplit) * kTcKeys;
+        const int j0 = (split + i * p.nsplit) * kTcKeys + kh * 64;
         if (!warp_wait(tm_full + 8 * buf, use & 1u, p.err)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const int mt = grp + 2 * k;
+          const int mt = tp + 2 * k;
           if (mt >= nmt) break;
-          uint32_t r[4][32];
-          const uint32_t ta = tmem + lane_base + buf * p.Rp + mt * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(ta + 32 * c, r[c]);
+          uint32_t r[2][32];
+          const uint32_t ta = tmem + lane_base + buf * p.Rp + mt * 128 + kh * 64;
+          tmem_ld32(ta, r[0]);
+          tmem_ld32(ta + 32, r[1]);
           tmem_wait_ld();
           if (mt + 2 >= nmt) {  // this warp's last read of the buffer
             tc_fence_before();
@@ -338,33 +377,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           const int row = mt * 128 + quarter * 32 + lane;
           // keys past the first observed position are masked per row
-          const int lim = (j0 + kTcKeys - 1 > p.S - p.n_obs)
-                              ? p.S - p.n_obs + (row % p.n_obs) - j0
-                              : kTcKeys - 1;
+          const int lim = (j0 + 63 > p.S - p.n_obs) ? p.S - p.n_obs + (row % p.n_obs) - j0 : 63;
           stats_fold(r, lim, p.sl2, m[k], l[k]);
         }
       }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const int row = (grp + 2 * k) * 128 + quarter * 32 + lane;
-        if (grp + 2 * k < nmt && row < p.R)
-          p.part[(bh * p.nsplit + split) * p.R + row] = make_float2(m[k], l[k]);
+        const int row = (tp + 2 * k) * 128 + quarter * 32 + lane;
+        if (tp + 2 * k < nmt && row < p.R)
+          p.part[(bh * 2 * p.nsplit + 2 * split + kh) * p.R + row] = make_float2(m[k], l[k]);
       }
     } else {
       // ------------------------------------------------ pass 2: weights per key
       float* bias = reinterpret_cast<float*>(smem + Y.bias_off);
       int* lim = reinterpret_cast<int*>(smem + Y.lim_off);
-      float* red = reinterpret_cast<float*>(smem + Y.red_off);
+      float* red = reinterpret_cast<float*>(smem + Y.red_off);  // [2][3][128]
       grid_dependency_wait();  // pass 1's statistics are complete and visible
+      const int nparts = 2 * p.nsplit;
       for (int r = threadIdx.x - 64; r < p.Rp; r += kTcEpiWarps * 32) {
         float bv = -INFINITY;
         int lv = -1;
         if (r < p.R) {
-          const float2* pr = p.part + bh * p.nsplit * p.R + r;
+          const float2* pr = p.part + bh * nparts * p.R + r;
           float M = -INFINITY;
-          for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, pr[static_cast<int64_t>(s) * p.R].x);
+          for (int s = 0; s < nparts; ++s) M = fmaxf(M, pr[static_cast<int64_t>(s) * p.R].x);
           float Ls = 0.f;
-          for (int s = 0; s < p.nsplit; ++s) {
+          for (int s = 0; s < nparts; ++s) {
             const float2 v = pr[static_cast<int64_t>(s) * p.R];
             if (v.x != -INFINITY) Ls += v.y * exp2f(v.x - M);
           }
@@ -376,9 +414,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         lim[r] = lv;
       }
       epi_sync();
-      const int half = p.Rp / 2, c_begin = grp * half;
+      const uint32_t bias_a = smem_u32(bias), lim_a = smem_u32(lim);
+      const int quarter_cols = p.Rp / 4, c_begin = grp * quarter_cols;
       const int key = quarter * 32 + lane;
-      const float2 sc = make_float2(p.sl2, p.sl2);
       // every epilogue warp meets the others once per block, also after a
       // timed-out wait (it then reads nothing more), so the named barrier
       // never waits for a warp that left
@@ -389,46 +427,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool masked = j0 + kTcKeys - 1 > p.S - p.n_obs;
         if (ok) ok = warp_wait(tm_full + 8 * buf, use & 1u, p.err);
         tc_fence_after();
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-        for (int c0 = c_begin; ok && c0 < c_begin + half; c0 += 64) {
-          uint32_t r[2][32];
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+        // this warpgroup's columns, two 32-column loads in flight when there are two
+        for (int c0 = c_begin; ok && c0 < c_begin + quarter_cols; c0 += 64) {
+          const bool two = c0 + 32 < c_begin + quarter_cols;
+          uint32_t r0[32], r1[32];
           const uint32_t ta = tmem + lane_base + buf * p.Rp + c0;
-          tmem_ld32(ta, r[0]);
-          tmem_ld32(ta + 32, r[1]);
+          tmem_ld32(ta, r0);
+          if (two) tmem_ld32(ta + 32, r1);
           tmem_wait_ld();
-          if (c0 + 64 >= c_begin + half) {  // this warp's last read of the buffer
+          if (c0 + 64 >= c_begin + quarter_cols) {  // this warp's last read of the buffer
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tm_free + 8 * buf);
           }
-#pragma unroll
-          for (int q = 0; q < 32; q += kTcEmuPeriod * 2) {
-#pragma unroll
-            for (int t = 0; t < kTcEmuPeriod * 2; ++t) {
-              if (q + t < 32) {
-                const int pr = q + t, c = c0 + 2 * pr;
-                const float2 bb = *reinterpret_cast<const float2*>(bias + c);
-                const float2 a = __ffma2_rn(make_float2(__uint_as_float(r[pr >> 4][(2 * pr) & 31]),
-                                                        __uint_as_float(r[pr >> 4][(2 * pr + 1) & 31])),
-                                            sc, bb);
-                float2 ev;
-                if (t % kTcEmuPeriod == kTcEmuPeriod - 1) ev = exp2_fma2(a);
-                else ev = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-                if (masked) {
-                  ev.x = j <= lim[c] ? ev.x : 0.f;
-                  ev.y = j <= lim[c + 1] ? ev.y : 0.f;
-                }
-                if (t & 1) acc1 = __fadd2_rn(acc1, ev);
-                else acc0 = __fadd2_rn(acc0, ev);
-              }
-            }
-          }
+          weight_fold(r0, bias_a, lim_a, c0, masked, j, p.sl2, acc);
+          if (two) weight_fold(r1, bias_a, lim_a, c0 + 32, masked, j, p.sl2, acc);
         }
-        const float w = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-        float* rb = red + (i & 1) * kTcKeys;
-        if (grp == 1) rb[key] = w;
+        const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+        const float w = (s01.x + s01.y) + (s23.x + s23.y);
+        float* rb = red + (i & 1) * 3 * kTcKeys;
+        if (grp > 0) rb[(grp - 1) * kTcKeys + key] = w;
         epi_sync();
-        if (ok && grp == 0 && j < p.S) p.imp[bh * p.S + j] = w + rb[key];
+        if (ok && grp == 0 && j < p.S)
+          p.imp[bh * p.S + j] = ((w + rb[key]) + rb[kTcKeys + key]) + rb[2 * kTcKeys + key];
       }
     }
   }
@@ -949,26 +972,40 @@ __global__ void tsa_inverse_kernel(const int32_t* __restrict__ idx,
   }
 }
 
-// O[b, s, h*G + g] = O^[b, inv, h*G + g] for kept positions, else 0.
-__global__ void tsa_scatter_kernel(const __nv_bfloat16* __restrict__ Oc,
-                                   const int32_t* __restrict__ inv, int S, int Sc, int Hq, int Hkv,
-                                   int D, int B, __nv_bfloat16* __restrict__ O) {
-  // one warp per output position (b, s): its Hq * D / 8 pieces over the lanes
-  const int G = Hq / Hkv, V8 = D / 8, per_row = Hq * V8;
-  const int lane = threadIdx.x & 31;
-  const int64_t wpb = blockDim.x >> 5;
-  for (int64_t bs = blockIdx.x * wpb + (threadIdx.x >> 5); bs < static_cast<int64_t>(B) * S;
-       bs += gridDim.x * wpb) {
-    const int b = static_cast<int>(bs / S), s = static_cast<int>(bs % S);
-    const int32_t* invb = inv + static_cast<int64_t>(b) * Hkv * S + s;
+// O[b, s, h*G + g] = O^[b, inv, h*G + g] for kept positions, else 0.  CTA
+// (chunk, b) takes kScatterRows positions: the inverse entries of every KV
+// head for them into shared memory (one coalesced row per head), then the
+// threads move independent 16-byte pieces, consecutive threads consecutive
+// pieces of an output row (coalesced stores; a kept row reads each head's
+// D contiguous elements of O^), four rows in flight per thread.
+constexpr int kScatterRows = 32;
+constexpr int kScatterThreads = 256;
+template <int D>
+__global__ void __launch_bounds__(kScatterThreads) tsa_scatter_kernel(
+    const __nv_bfloat16* __restrict__ Oc, const int32_t* __restrict__ inv, int S, int Sc, int Hq,
+    int Hkv, __nv_bfloat16* __restrict__ O) {
+  extern __shared__ int inv_s[];  // [Hkv][kScatterRows]
+  constexpr int V8 = D / 8;
+  const int b = blockIdx.y, s0 = blockIdx.x * kScatterRows;
+  const int nrow = min(kScatterRows, S - s0);
+  for (int e = threadIdx.x; e < Hkv * kScatterRows; e += blockDim.x) {
+    const int h = e / kScatterRows, r = e % kScatterRows;
+    int t = r < nrow ? inv[(static_cast<int64_t>(b) * Hkv + h) * S + s0 + r] : -1;
+    inv_s[e] = t < Sc ? t : -1;
+  }
+  __syncthreads();
+  const int G = Hq / Hkv, per_row = Hq * V8;
+  const __nv_bfloat16* ob = Oc + static_cast<int64_t>(b) * Sc * Hq * D;
+  __nv_bfloat16* dst = O + (static_cast<int64_t>(b) * S + s0) * Hq * D;
+  for (int q = threadIdx.x; q < per_row; q += blockDim.x) {
+    const int hq = q / V8, c = (q % V8) * 8;
+    const int* it = inv_s + (hq / G) * kScatterRows;
 #pragma unroll 4
-    for (int q = lane; q < per_row; q += 32) {
-      const int hq = q / V8, c = (q % V8) * 8;
-      const int t = invb[static_cast<int64_t>(hq / G) * S];
+    for (int r = 0; r < nrow; ++r) {
+      const int t = it[r];
       int4 v = make_int4(0, 0, 0, 0);
-      if (t >= 0)
-        v = *reinterpret_cast<const int4*>(Oc + ((static_cast<int64_t>(b) * Sc + t) * Hq + hq) * D + c);
-      *reinterpret_cast<int4*>(O + (bs * Hq + hq) * D + c) = v;
+      if (t >= 0) v = *reinterpret_cast<const int4*>(ob + (static_cast<int64_t>(t) * Hq + hq) * D + c);
+      *reinterpret_cast<int4*>(dst + (static_cast<int64_t>(r) * Hq + hq) * D + c) = v;
     }
   }
 }
@@ -1031,20 +1068,31 @@ cudaError_t launch_tsa_lists(const Launch& l, const int32_t* k_unit, int U, int 
 
 cudaError_t launch_tsa_scatter(const Launch& l, const void* Oc, const int32_t* idx,
                                const int32_t* count, int kmax, int B, int S, int Sc, int Hq,
-                               int Hkv, int D, int32_t* inv, void* O) {
+                               int Hkv, int D, int32_t* inv, void* O, bool inv_ready) {
   if (B == 0 || S == 0) return cudaSuccess;
-  tsa_inverse_kernel<<<B * Hkv, 512, 0, l.stream>>>(idx, count, kmax, S, inv);
-  tsa_scatter_kernel<<<8 * l.num_sms, 256, 0, l.stream>>>(
-      static_cast<const __nv_bfloat16*>(Oc), inv, S, Sc, Hq, Hkv, D, B,
-      static_cast<__nv_bfloat16*>(O));
+  if (!inv_ready) tsa_inverse_kernel<<<B * Hkv, 512, 0, l.stream>>>(idx, count, kmax, S, inv);
+  const dim3 grid((S + kScatterRows - 1) / kScatterRows, B);
+  const size_t sh = static_cast<size_t>(Hkv) * kScatterRows * 4;
+  const auto* oc = static_cast<const __nv_bfloat16*>(Oc);
+  auto* o = static_cast<__nv_bfloat16*>(O);
+  if (D == 128) {
+    cudaError_t e = set_smem_ts(reinterpret_cast<const void*>(tsa_scatter_kernel<128>), sh);
+    if (e != cudaSuccess) return e;
+    tsa_scatter_kernel<128><<<grid, kScatterThreads, sh, l.stream>>>(oc, inv, S, Sc, Hq, Hkv, o);
+  } else {
+    cudaError_t e = set_smem_ts(reinterpret_cast<const void*>(tsa_scatter_kernel<64>), sh);
+    if (e != cudaSuccess) return e;
+    tsa_scatter_kernel<64><<<grid, kScatterThreads, sh, l.stream>>>(oc, inv, S, Sc, Hq, Hkv, o);
+  }
   return cudaGetLastError();
 }
 
 size_t token_importance_scratch_bytes(int B, int S, int Hkv, int G, int n_obs) {
-  // per-split row statistics of pass 1: at most one split per key block
+  // row statistics of pass 1 per split and key half: at most one split per
+  // key block
   const int64_t nblk = (S + kTcKeys - 1) / kTcKeys;
   const int64_t R = static_cast<int64_t>(G) * n_obs;
-  return static_cast<size_t>(B) * Hkv * R * 2 * 4 * nblk;
+  return static_cast<size_t>(B) * Hkv * R * 2 * 4 * 2 * nblk;
 }
 
 cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* K, int B, int S,
