@@ -425,8 +425,6 @@ def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: f
     cnt = torch.empty(U, dtype=torch.int32, device=dev)
     Qc, Oc = torch.empty_like(Q), torch.empty_like(Q)
     Kc, Vc = torch.empty_like(K), torch.empty_like(V)
-    na = csa.csa_token_attend_scratch_bytes(B, S, Hkv)
-    sa = torch.empty(na, dtype=torch.uint8, device=dev)
     nd = csa.csa_token_decompress_scratch_bytes(B, S, Hkv)
     sd = torch.empty(nd, dtype=torch.uint8, device=dev)
     O2 = torch.empty_like(Q)
@@ -446,7 +444,7 @@ def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: f
         ev[3].record()
         csa.csa_token_compress(Q, K, V, idx, cnt, B, S, Hq, Hkv, D, Qc, Kc, Vc)
         ev[4].record()
-        csa.csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, sa, na, Oc)
+        csa.csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, Oc)
         ev[5].record()
         csa.csa_token_decompress(Oc, idx, cnt, B, S, Hq, Hkv, D, sd, nd, O2)
         ev[6].record()

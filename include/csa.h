@@ -205,9 +205,10 @@ CSA_API csa_status csa_token_sparse_prefill(const void* Q, const void* K, const 
  *   the group's heads into Qc[b, t, h*G .. h*G+G-1].  Rows past a unit's
  *   count are not written.
  * csa_token_attend: dense causal attention of each unit's first k_unit[u]
- *   compressed rows (k_unit a multiple of 64, as csa_token_budget gives it);
- *   the rows of Oc past a unit's k_unit are not written.  scratch >=
- *   csa_token_attend_scratch_bytes(B, S, Hkv) (the per-tile causal lists).
+ *   compressed rows (k_unit a multiple of 64, as csa_token_budget gives it),
+ *   64-row tile t attending to tiles 0 .. t; the rows of Oc past a unit's
+ *   k_unit are not written.  No scratch: the tiles are read from k_unit on
+ *   the device.
  * csa_token_decompress: O[b, s, h*G+g] = Oc[b, t, h*G+g] where idx[u, t] = s,
  *   0 for the positions a head did not keep; every row of O is written.
  *   scratch >= csa_token_decompress_scratch_bytes(B, S, Hkv) (the inverse
@@ -219,11 +220,9 @@ CSA_API csa_status csa_token_compress(const void* Q, const void* K, const void* 
                                       const int32_t* idx, const int32_t* count, int B, int S,
                                       int Hq, int Hkv, int D, void* Qc, void* Kc, void* Vc,
                                       csa_stream stream);
-CSA_API int64_t csa_token_attend_scratch_bytes(int B, int S, int Hkv);
 CSA_API csa_status csa_token_attend(const void* Qc, const void* Kc, const void* Vc,
                                     const int32_t* k_unit, int B, int S, int Hq, int Hkv, int D,
-                                    float scale, void* scratch, int64_t scratch_bytes, void* Oc,
-                                    csa_stream stream);
+                                    float scale, void* Oc, csa_stream stream);
 CSA_API int64_t csa_token_decompress_scratch_bytes(int B, int S, int Hkv);
 CSA_API csa_status csa_token_decompress(const void* Oc, const int32_t* idx, const int32_t* count,
                                         int B, int S, int Hq, int Hkv, int D, void* scratch,

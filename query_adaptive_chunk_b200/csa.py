@@ -55,8 +55,7 @@ _SIGS = {
                                       _vp, _vp, _vp]),
     "csa_token_select": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "csa_token_compress": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
-    "csa_token_attend_scratch_bytes": (_i64, [_i, _i, _i]),
-    "csa_token_attend": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _i64, _vp, _vp]),
+    "csa_token_attend": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp]),
     "csa_token_decompress_scratch_bytes": (_i64, [_i, _i, _i]),
     "csa_token_decompress": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i64, _vp, _vp]),
     "csa_score_chunks": (_i, [_vp, _i, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
@@ -280,14 +279,9 @@ def csa_token_compress(Q, K, V, idx, count, B, S, Hq, Hkv, D, Qc, Kc, Vc, stream
                                   _p(Qc), _p(Kc), _p(Vc), _s(stream)))
 
 
-def csa_token_attend_scratch_bytes(B, S, Hkv) -> int:
-    return int(lib.csa_token_attend_scratch_bytes(B, S, Hkv))
-
-
-def csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, scratch, scratch_bytes, Oc,
-                     stream=None):
+def csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, Oc, stream=None):
     _check(lib.csa_token_attend(_p(Qc), _p(Kc), _p(Vc), _p(k_unit), B, S, Hq, Hkv, D, scale,
-                                _p(scratch), scratch_bytes, _p(Oc), _s(stream)))
+                                _p(Oc), _s(stream)))
 
 
 def csa_token_decompress_scratch_bytes(B, S, Hkv) -> int:

@@ -959,11 +959,11 @@ csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, float tau, 
 
 namespace {
 struct TsaLayout {
-  size_t imp, scratch, k_unit, idx, count, qc, kc, vc, oc, lists, counts2, inv, total;
+  size_t imp, scratch, k_unit, idx, count, qc, kc, vc, oc, inv, total;
 };
 TsaLayout tsa_layout(int B, int S, int Hq, int Hkv, int D, int n_obs) {
   auto r = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t U = static_cast<size_t>(B) * Hkv, T = S / 64;
+  const size_t U = static_cast<size_t>(B) * Hkv;
   TsaLayout w;
   size_t o = 0;
   w.imp = o; o += r(U * S * 4);
@@ -975,8 +975,6 @@ TsaLayout tsa_layout(int B, int S, int Hq, int Hkv, int D, int n_obs) {
   w.kc = o; o += r(U * S * D * 2);
   w.vc = o; o += r(U * S * D * 2);
   w.oc = o; o += r(static_cast<size_t>(B) * S * Hq * D * 2);
-  w.lists = o; o += r(U * T * T * 4);
-  w.counts2 = o; o += r(U * T * 4);
   w.inv = o; o += r(U * S * 4);
   w.total = o;
   return w;
@@ -1027,20 +1025,16 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
   if (e != cudaSuccess) return finish(e, "token selection launch");
   // Compress, attend, decompress with no read-back of the budgets: the
   // buffers are laid out for S kept tokens, the gather writes the kept rows
-  // of each unit only, the causal lists give the tiles past a unit's budget
-  // no chunk, and the dense attention skips those tiles without writing.
+  // of each unit only, and the dense causal attention takes the tiles below
+  // each unit's budget (tiles past it are never visited and write nothing).
   void* Qc = ws + w.qc;
   void* Kc = ws + w.kc;
   void* Vc = ws + w.vc;
   void* Oc = ws + w.oc;
-  const int T = S / 64;
-  int32_t* lists = reinterpret_cast<int32_t*>(ws + w.lists);
-  int32_t* counts2 = reinterpret_cast<int32_t*>(ws + w.counts2);
   e = csa::launch_tsa_gather(l, Q, K, V, idx, cnt, S, B, S, S, Hq, Hkv, D, Qc, Kc, Vc);
-  if (e == cudaSuccess) e = csa::launch_tsa_lists(l, k_unit, U, T, 64, lists, counts2);
   if (e == cudaSuccess)
-    e = csa::launch_prefill(l, Qc, Kc, Vc, lists, counts2, T, B, S, Hq, Hkv, D, 64, 64, scale, Oc,
-                            &why, /*skip_empty=*/true);
+    e = csa::launch_prefill(l, Qc, Kc, Vc, nullptr, nullptr, 0, B, S, Hq, Hkv, D, 64, 64, scale, Oc,
+                            &why, /*skip_empty=*/true, k_unit);
   if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
   if (e == cudaSuccess)
     e = csa::launch_tsa_scatter(l, Oc, idx, cnt, S, B, S, S, Hq, Hkv, D,
@@ -1097,37 +1091,22 @@ csa_status csa_token_compress(const void* Q, const void* K, const void* V, const
                 "token compress launch");
 }
 
-int64_t csa_token_attend_scratch_bytes(int B, int S, int Hkv) {
-  if (B < 0 || S < 0 || Hkv <= 0 || S % 64 != 0) return -1;
-  const int64_t U = static_cast<int64_t>(B) * Hkv, T = S / 64;
-  return (U * T * T + U * T) * 4;
-}
-
 csa_status csa_token_attend(const void* Qc, const void* Kc, const void* Vc,
                             const int32_t* k_unit, int B, int S, int Hq, int Hkv, int D,
-                            float scale, void* scratch, int64_t scratch_bytes, void* Oc,
-                            csa_stream stream) {
+                            float scale, void* Oc, csa_stream stream) {
   CSA_TRY(token_shape_checks(B, S, Hq, Hkv, D));
   CSA_REQUIRE(scale == scale && scale > 0.f, "scale must be positive");
   if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
-  CSA_REQUIRE(scratch_bytes >= csa_token_attend_scratch_bytes(B, S, Hkv),
-              "scratch smaller than csa_token_attend_scratch_bytes()");
   CSA_TRY(check_ptr(Qc, "Qc"));
   CSA_TRY(check_ptr(Kc, "Kc"));
   CSA_TRY(check_ptr(Vc, "Vc"));
   CSA_TRY(check_ptr(Oc, "Oc"));
   CSA_TRY(check_ptr(k_unit, "k_unit"));
-  CSA_TRY(check_ptr(scratch, "scratch"));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
-  const int U = B * Hkv, T = S / 64;
-  int32_t* lists = static_cast<int32_t*>(scratch);
-  int32_t* counts = lists + static_cast<int64_t>(U) * T * T;
-  cudaError_t e = csa::launch_tsa_lists(l, k_unit, U, T, 64, lists, counts);
   std::string why;
-  if (e == cudaSuccess)
-    e = csa::launch_prefill(l, Qc, Kc, Vc, lists, counts, T, B, S, Hq, Hkv, D, 64, 64, scale, Oc,
-                            &why, /*skip_empty=*/true);
+  const cudaError_t e = csa::launch_prefill(l, Qc, Kc, Vc, nullptr, nullptr, 0, B, S, Hq, Hkv, D,
+                                            64, 64, scale, Oc, &why, /*skip_empty=*/true, k_unit);
   if (e != cudaSuccess && !why.empty()) return fail(CSA_ERR_CUDA, why);
   return finish(e, "token attend launch");
 }

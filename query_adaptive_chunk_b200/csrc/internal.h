@@ -76,8 +76,6 @@ cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S,
 cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, const void* V,
                               const int32_t* idx, const int32_t* count, int kmax, int B, int S,
                               int Sc, int Hq, int Hkv, int D, void* Qc, void* Kc, void* Vc);
-cudaError_t launch_tsa_lists(const Launch& l, const int32_t* k_unit, int U, int n_tiles, int tile,
-                             int32_t* lists, int32_t* counts);
 // inv [B*Hkv, S] (scratch): built here from idx/count unless inv_ready (the
 // selection wrote it)
 cudaError_t launch_tsa_scatter(const Launch& l, const void* Oc, const int32_t* idx,
@@ -129,11 +127,14 @@ cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_
 cudaError_t launch_copy16(const Launch& l, const void* src, void* dst, size_t bytes);
 
 // prefill.cu
-// skip_empty: units with no chunk write nothing (else their rows get 0)
+// skip_empty: units with no chunk write nothing (else their rows get 0).
+// dense_k (dense causal mode; idx/count unused): tile t of (b, h) attends
+// to chunks 0 .. t when t * 64 < dense_k[b * Hkv + h], else it is empty.
 cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const void* V,
                            const int32_t* idx, const int32_t* count, int kmax, int B, int S,
                            int Hq, int Hkv, int D, int tile_m, int L, float scale, void* O,
-                           std::string* why, bool skip_empty = false);
+                           std::string* why, bool skip_empty = false,
+                           const int32_t* dense_k = nullptr);
 
 // tma_host.cu: 2-D bf16 tensor map over a row-major [rows, cols] matrix with
 // `row_stride` elements between rows, box [box_rows, box_cols], 128-byte swizzle.

@@ -89,17 +89,35 @@ struct PrefillParams {
   __nv_bfloat16* O;
   DevErr err;
   int skip_empty;  // units with no chunk write nothing (else their rows get 0)
+  // dense causal mode (no index lists): unit (b, h, t) holds chunks 0 .. t
+  // when t * 64 < dense_k[b * Hkv + h], else none
+  const int32_t* dense_k;
 };
 
-__device__ __forceinline__ void unit_coords(const PrefillParams& p, int w, int& b, int& h, int& t) {
+// Tiles that can hold work: all of them, or in dense causal mode those below
+// the largest dense_k (the launch's units beyond it are never visited).
+__device__ __forceinline__ int active_tiles(const PrefillParams& p) {
+  if (p.dense_k == nullptr) return p.n_tiles;
+  int mx = 0;
+  for (int bh = 0; bh < p.B * p.Hkv; ++bh) mx = max(mx, __ldg(p.dense_k + bh));
+  return min(p.n_tiles, (mx + 63) / 64);
+}
+
+// Unit w of T active tiles: heaviest (latest) tiles first.
+__device__ __forceinline__ void unit_coords(const PrefillParams& p, int T, int w, int& b, int& h,
+                                            int& t) {
   const int bh = p.B * p.Hkv;
-  t = p.n_tiles - 1 - w / bh;  // heaviest (latest) tiles first
+  t = T - 1 - w / bh;
   const int r = w % bh;
   b = r / p.Hkv;
   h = r % p.Hkv;
 }
 
 __device__ __forceinline__ int unit_n(const PrefillParams& p, int sel_row) {
+  if (p.dense_k != nullptr) {
+    const int t = sel_row % p.n_tiles;
+    return t * 64 < __ldg(p.dense_k + sel_row / p.n_tiles) ? t + 1 : 0;
+  }
   int n = p.count[sel_row];
   if (n < 0 || n > p.kmax) {
     dev_flag(p.err, DEV_BAD_INDEX);
@@ -109,6 +127,7 @@ __device__ __forceinline__ int unit_n(const PrefillParams& p, int sel_row) {
 }
 
 __device__ __forceinline__ int unit_chunk(const PrefillParams& p, int sel_row, int j) {
+  if (p.dense_k != nullptr) return j;
   int c = p.idx[static_cast<int64_t>(sel_row) * p.kmax + j];
   if (c < 0 || c >= p.C) {
     dev_flag(p.err, DEV_BAD_INDEX);
@@ -161,14 +180,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     fence_barrier_init();
   }
+  __shared__ int tiles_sh;
   if (warp == 1) {
     tmem_alloc<512>(tmem_slot);
   }
+  if (threadIdx.x == 64) tiles_sh = active_tiles(p);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int n_units = p.B * p.Hkv * p.n_tiles;
+  const int T = tiles_sh;
+  const int n_units = p.B * p.Hkv * T;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -176,7 +198,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       int b, h, t;
-      unit_coords(p, w, b, h, t);
+      unit_coords(p, T, w, b, h, t);
       const int sel = (b * p.Hkv + h) * p.n_tiles + t;
       const int n = unit_n(p, sel);
       if (n == 0) continue;
@@ -271,7 +293,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
         int b, h, t;
-        unit_coords(p, w, b, h, t);
+        unit_coords(p, T, w, b, h, t);
         const int n = unit_n(p, (b * p.Hkv + h) * p.n_tiles + t);
         if (n == 0) continue;
         const uint32_t st0 = kv_it % kNS;
@@ -317,7 +339,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     bool ok = true;
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       int b, h, t;
-      unit_coords(p, w, b, h, t);
+      unit_coords(p, T, w, b, h, t);
       const int sel = (b * p.Hkv + h) * p.n_tiles + t;
       const int n = unit_n(p, sel);
       const int qpos = t * 64 + i;
@@ -524,7 +546,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const void* V,
                            const int32_t* idx, const int32_t* count, int kmax, int B, int S,
                            int Hq, int Hkv, int D, int tile_m, int L, float scale, void* O,
-                           std::string* why, bool skip_empty) {
+                           std::string* why, bool skip_empty, const int32_t* dense_k) {
   (void)D;
   (void)tile_m;
   (void)L;
@@ -552,6 +574,7 @@ cudaError_t launch_prefill(const Launch& l, const void* Q, const void* K, const 
   p.O = static_cast<__nv_bfloat16*>(O);
   p.err = l.err;
   p.skip_empty = skip_empty ? 1 : 0;
+  p.dense_k = dense_k;
   const int n_units = B * Hkv * p.n_tiles;
   if (n_units == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -944,21 +944,6 @@ __global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
   }
 }
 
-// Dense causal chunk lists of the compressed sequences: tile t of (b, h)
-// sees chunks 0..t (chunk = tile = 64 rows); tiles past the unit's budget
-// k_unit (a multiple of the tile) see none and are skipped by the dense
-// attention.
-__global__ void tsa_lists_kernel(const int32_t* __restrict__ k_unit, int n_tiles, int tile,
-                                 int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
-  const int64_t ut = blockIdx.x;  // (b * Hkv + h) * n_tiles + t
-  const int t = static_cast<int>(ut % n_tiles);
-  const int64_t u = ut / n_tiles;
-  const bool live = t * tile < k_unit[u];
-  for (int c = threadIdx.x; c < n_tiles; c += blockDim.x)
-    lists[ut * n_tiles + c] = (live && c <= t) ? c : -1;
-  if (threadIdx.x == 0) counts[ut] = live ? t + 1 : 0;
-}
-
 __global__ void tsa_inverse_kernel(const int32_t* __restrict__ idx,
                                    const int32_t* __restrict__ count, int kmax, int S,
                                    int32_t* __restrict__ inv) {
@@ -1056,13 +1041,6 @@ cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, con
       static_cast<const __nv_bfloat16*>(V), idx, count, kmax, S, Sc, Hq, Hkv, D,
       static_cast<__nv_bfloat16*>(Qc), static_cast<__nv_bfloat16*>(Kc),
       static_cast<__nv_bfloat16*>(Vc));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_tsa_lists(const Launch& l, const int32_t* k_unit, int U, int n_tiles, int tile,
-                             int32_t* lists, int32_t* counts) {
-  if (U == 0 || n_tiles == 0) return cudaSuccess;
-  tsa_lists_kernel<<<U * n_tiles, 128, 0, l.stream>>>(k_unit, n_tiles, tile, lists, counts);
   return cudaGetLastError();
 }
 

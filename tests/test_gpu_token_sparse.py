@@ -225,10 +225,8 @@ def _token_steps(csa, Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale):
     Kc = torch.empty(B, Hkv, S, D, dtype=torch.bfloat16, device=dev)
     Vc = torch.empty_like(Kc)
     csa.csa_token_compress(Q, K, V, idx, cnt, B, S, Hq, Hkv, D, Qc, Kc, Vc)
-    na = csa.csa_token_attend_scratch_bytes(B, S, Hkv)
-    sa = torch.empty(na, dtype=torch.uint8, device=dev)
     Oc = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=dev)
-    csa.csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, sa, na, Oc)
+    csa.csa_token_attend(Qc, Kc, Vc, k_unit, B, S, Hq, Hkv, D, scale, Oc)
     nd = csa.csa_token_decompress_scratch_bytes(B, S, Hkv)
     sd = torch.empty(nd, dtype=torch.uint8, device=dev)
     O = torch.full((B, S, Hq, D), float("nan"), device=dev).to(torch.bfloat16)
