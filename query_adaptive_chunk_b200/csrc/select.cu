@@ -1701,7 +1701,11 @@ __global__ void __launch_bounds__(kClTopkThreads) topk_cluster_kernel(
       cluster_wait();
       for (int d = tid; d < 256; d += blockDim.x) {
         unsigned int c = 0u;
-        for (int r = 0; r < CS; ++r) c += ld_cluster_u32(cluster_map(smem_u32(hc + d), r));
+        unsigned int cr[kClTopkCS];  // the launch's cluster has kClTopkCS CTAs: all loads in flight
+#pragma unroll
+        for (int r = 0; r < kClTopkCS; ++r) cr[r] = ld_cluster_u32(cluster_map(smem_u32(hc + d), r));
+#pragma unroll
+        for (int r = 0; r < kClTopkCS; ++r) c += cr[r];
         gc[d] = c;
       }
       cluster_arrive();  // every CTA has read the others' histograms (they may be cleared)

@@ -791,9 +791,19 @@ __global__ void __launch_bounds__(kBudgetCThreads) budget_cluster_kernel(
     for (int d = tid; d < 256; d += blockDim.x) {  // the cluster's, added in rank order
       unsigned int c = 0u;
       float mm = 0.f;
-      for (int r = 0; r < CS; ++r) {
-        c += ld_cluster_u32(cluster_map(smem_u32(hc + d), r));
-        mm += ld_cluster_f32(cluster_map(smem_u32(hm + d), r));
+      // all the cluster's loads in flight at once (the launch's cluster has
+      // kBudgetCS CTAs), then added in rank order
+      unsigned int cr[kBudgetCS];
+      float mr[kBudgetCS];
+#pragma unroll
+      for (int r = 0; r < kBudgetCS; ++r) {
+        cr[r] = ld_cluster_u32(cluster_map(smem_u32(hc + d), r));
+        mr[r] = ld_cluster_f32(cluster_map(smem_u32(hm + d), r));
+      }
+#pragma unroll
+      for (int r = 0; r < kBudgetCS; ++r) {
+        c += cr[r];
+        mm += mr[r];
       }
       gc[d] = c;
       gm[d] = mm;
