@@ -487,6 +487,14 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// An opaque copy of v: the compiler cannot tell which loop pass a flag made
+// from it is set on, so it keeps one copy of the loop body for all passes
+// (a dry first pass then runs the same instructions as the real ones).
+__device__ __forceinline__ int opaque(int v) {
+  asm volatile("" : "+r"(v));
+  return v;
+}
+
 // Merge of unit u by one warp, straight from global memory (rarely used:
 // more merges fell to one CTA than its deferred list holds).
 template <int D>
@@ -646,12 +654,14 @@ __device__ bool merge_staged(const DecodeParams& p, int u, int ns, uint8_t* area
 // its output when ns == 1), release the buffer, and count the split in.
 // Returns 1 when this CTA brought the unit's last split (its merge is
 // deferred), 2 when it also started the merge's copy already (the CTA's last
-// flush), else 0.
+// flush), else 0.  `dry`: the same instructions with every write, release
+// and count left out (a first pass that only fetches the code).
 template <int D>
 __device__ __forceinline__ int epilogue_unit(const DecodeParams& p, const float* fo, int u,
                                              int slot, int ns, bool final_flush, uint8_t* area,
                                              int area_bytes, uint32_t merge_bar,
-                                             uint32_t fb_empty, int* pre_u, int* pre_ns) {
+                                             uint32_t fb_empty, int* pre_u, int* pre_ns,
+                                             bool dry) {
   static_assert(kConsumerWarps == 4, "four partials per head");
   const int lane = threadIdx.x & 31, G = p.G;
   const float* fm = fo + kConsumerWarps * G * D;
@@ -674,10 +684,12 @@ __device__ __forceinline__ int epilogue_unit(const DecodeParams& p, const float*
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) wn[w] *= inv;
     const float lse = (M + __log2f(Ls)) * kLn2;
-    if (!direct)
+    if (dry) {
+    } else if (!direct) {
       p.lse_part[(row0 + lane) * p.max_splits + slot] = lse;
-    else if (p.lse_out)
+    } else if (p.lse_out) {
       p.lse_out[row0 + lane] = lse;
+    }
   }
   // Every lane: columns lane + 32 j of every head, all independent (the
   // weights of all heads first, then the loads and stores).
@@ -695,12 +707,14 @@ __device__ __forceinline__ int epilogue_unit(const DecodeParams& p, const float*
         float acc = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) acc += fo[(w * G + g) * D + d] * wg[g][w];
+        if (dry) continue;
         if (direct) store_out(p, row * D + d, acc);
         else p.o_part[(row * p.max_splits + slot) * D + d] = acc;
       }
     }
   }
   __syncwarp();
+  if (dry) return 0;
   if (lane == 0) mbar_arrive(fb_empty);  // the consumers may refill it
   if (!p.merged || direct) return 0;
   fence_acq_rel_gpu();  // this lane's partial writes before the arrival count
@@ -1129,24 +1143,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       piece_range(N, P, blockIdx.x, a, bnd);
       if (a >= bnd) continue;
       const int u0 = unit_of(pre, p.U, a), u1 = unit_of(pre, p.U, bnd - 1);
-      for (int u = u0; u <= u1 && ok; ++u) {
-        if (pre[u + 1] <= pre[u]) continue;  // no chunk: never flushed
+      // phase 0 starts with a dry pass of the loop body (no wait, nothing
+      // written) while the first stages are in flight: its code is then in
+      // the instruction caches for the real flushes
+      for (int u = u0 - (ph == 0 ? 1 : 0); u <= u1 && ok; ++u) {
+        const bool dry = opaque(u < u0 ? 1 : 0) != 0;
+        if (!dry && pre[u + 1] <= pre[u]) continue;  // no chunk: never flushed
         // the split's slot and count before the wait (64-bit divisions)
-        const int slot = split_slot(pre[u], a, blockIdx.x, N, P);
-        const int ns = split_count(pre[u], pre[u + 1], N, P);
-        const int k = Y.nf == 2 ? (nseen & 1) : 0;
+        const int slot = dry ? 0 : split_slot(pre[u], a, blockIdx.x, N, P);
+        const int ns = dry ? 2 : split_count(pre[u], pre[u + 1], N, P);
+        const int k = dry ? 0 : (Y.nf == 2 ? (nseen & 1) : 0);
         const int use = Y.nf == 2 ? (nseen >> 1) : nseen;
-        if (!warp_wait(fb_full + 8 * k, static_cast<uint32_t>(use) & 1u, p.err)) {
+        if (!dry && !warp_wait(fb_full + 8 * k, static_cast<uint32_t>(use) & 1u, p.err)) {
           ok = false;
           break;
         }
-        ++nseen;
+        if (!dry) ++nseen;
         const float* fo = reinterpret_cast<const float*>(smem + Y.fb_off + k * Y.fb_bytes);
         // the CTA's last flush: the consumers are done with the stage ring
-        const bool final_flush = ph == n_phase - 1 && u == u1;
-        int last = epilogue_unit<D>(p, fo, u, slot, ns, final_flush, smem, NS * Sh::STAGE_BYTES,
-                                    merge_bar, fb_empty + 8 * k, &pre_u_sh, &pre_ns_sh);
-        if (last != 1) continue;
+        const bool final_flush = !dry && ph == n_phase - 1 && u == u1;
+        int last = epilogue_unit<D>(p, fo, dry ? u0 : u, slot, ns, final_flush, smem,
+                                    NS * Sh::STAGE_BYTES, merge_bar, fb_empty + 8 * k, &pre_u_sh,
+                                    &pre_ns_sh, dry);
+        if (dry || last != 1) continue;
         if (n_defer < kDeferMax) {  // merged after the main loop, off the hot path
           if (lane == 0) {
             defer_u[n_defer] = u;
@@ -1216,14 +1235,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       piece_range(N, phase_parts(1), blockIdx.x, a, bnd);
       zero_empty_units(p, pre, 2, kConsumerWarps * 32);
     }
-    for (int64_t g = a; g < bnd; ++g, ++i) {
-      const int s = static_cast<int>(i % NS);
+    // phase 0 starts with a dry pass of the loop body over stage 0 (no
+    // wait, nothing released or kept; the accumulator is set up again by the
+    // first real chunk) while the first stages are in flight: its code is
+    // then in the instruction caches when the data arrives
+    for (int64_t g = (ph == 0 && a < bnd) ? a - 1 : a; g < bnd; ++g) {
+      const bool dry = opaque(g < a ? 1 : 0) != 0;
+      const int s = dry ? 0 : static_cast<int>(i % NS);
       const uint32_t it = static_cast<uint32_t>(i / NS);
-      if (!warp_wait(full_bar + 8 * s, it & 1u, p.err)) {
+      if (!dry && !warp_wait(full_bar + 8 * s, it & 1u, p.err)) {
         ok = false;
         break;
       }
-      if (cur_u < 0 || g >= pre[cur_u + 1]) {
+      if (!dry && (cur_u < 0 || g >= pre[cur_u + 1])) {
         if (cur_u >= 0 && !flush_async(cur_u)) {
           ok = false;
           break;
@@ -1237,7 +1261,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                      G, lane);
       }
       int valid = L;
-      if (hybrid && !cur_full) {
+      if (!dry && hybrid && !cur_full) {
         // a hybrid unit's last gist chunk is ragged: rows past its gist rows
         // (the next unit's, zeros past the tensor, or the zero-filled rows of
         // a gathered chunk) take no part
@@ -1246,7 +1270,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       acc_stage<D, L>(acc, sbase + s * Sh::STAGE_BYTES, warp, lane, scale_log2, valid);
       __syncwarp();
+      if (dry) continue;
       if (lane == 0) mbar_arrive(empty_bar + 8 * s);
+      ++i;
     }
   }
   if (ok && cur_u >= 0) ok = flush_async(cur_u);
