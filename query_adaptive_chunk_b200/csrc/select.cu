@@ -1000,6 +1000,18 @@ __global__ void __launch_bounds__(kSelThreads) select_hier_rank_kernel(
 __device__ void unit_query(const void* __restrict__ q, int q_bf16, int64_t head0, int G, int D,
                            const float* __restrict__ proj, int R, float* qs, float* qv,
                            float* part) {
+  // this thread's projection entries are loaded together with the query
+  // (they do not depend on it), so the two global round trips overlap
+  constexpr int kPre = 8;
+  float pw[kPre];
+  const int parts = proj != nullptr ? 256 / R : 1;
+  const int pr = threadIdx.x / parts, ppt = threadIdx.x % parts;
+  const int dchunk = (D + parts - 1) / parts;
+  const int pd0 = ppt * dchunk, pd1 = min(D, pd0 + dchunk);
+  const bool pre_ok = proj != nullptr && threadIdx.x < 256 && dchunk <= kPre;
+#pragma unroll
+  for (int k = 0; k < kPre; ++k)
+    pw[k] = pre_ok && pd0 + k < pd1 ? __ldg(proj + static_cast<int64_t>(pd0 + k) * R + pr) : 0.f;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float acc = 0.f;
     for (int g = 0; g < G; ++g) {
@@ -1014,16 +1026,18 @@ __device__ void unit_query(const void* __restrict__ q, int q_bf16, int64_t head0
   // 256 threads: thread t handles r = t / parts over the d range of part
   // t % parts; the parts of one r sit in adjacent lanes and are added by an
   // xor-shuffle tree (same order as the score kernel)
-  const int parts = 256 / R;
   if (threadIdx.x < 256) {
-    const int r = threadIdx.x / parts, pt = threadIdx.x % parts;
-    const int dchunk = (D + parts - 1) / parts;
-    const int d0 = pt * dchunk, d1 = min(D, d0 + dchunk);
     float acc = 0.f;
+    if (pre_ok) {
+#pragma unroll
+      for (int k = 0; k < kPre; ++k)
+        if (pd0 + k < pd1) acc += pw[k] * qs[pd0 + k];
+    } else {
 #pragma unroll 4
-    for (int d = d0; d < d1; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * qs[d];
+      for (int d = pd0; d < pd1; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + pr) * qs[d];
+    }
     for (int o = parts >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (pt == 0) qv[r] = acc;
+    if (ppt == 0) qv[pr] = acc;
   }
   (void)part;
   __syncthreads();
