@@ -19,7 +19,7 @@
 // special-function unit, which otherwise needs as many cycles per chunk as
 // the tensor core, stops being the bound.
 // Warp roles: warp 0 issues TMA (each half of the Q tile once per unit, K/V
-// per chunk into a 5-stage ring), warp 1 allocates TMEM, one thread of warp
+// per chunk into a 3-stage ring), warp 1 allocates TMEM, one thread of warp
 // 1 issues the MMAs of half 0 and one thread of warp 2 those of half 1 (in
 // the order QK(j+1) PV(j) per chunk j, so that neither half's chain waits
 // on the other's softmax), warps 4-7 and 8-11 are the softmax/epilogue
@@ -36,13 +36,13 @@ namespace csa {
 namespace {
 
 constexpr int kPfThreads = 384;
-constexpr int kNS = 4;                         // K/V stages
+constexpr int kNS = 3;                         // K/V stages
 constexpr int kQHalfBytes = 128 * 128 * 2;     // 32 KB: one 128-row half of the Q tile
 constexpr int kKVBytes = 64 * 128 * 2;         // 16 KB per K (or V) chunk
 constexpr int kStageBytes = 2 * kKVBytes;
 constexpr int kQOff = 0;
 constexpr int kKVOff = 2 * kQHalfBytes;
-constexpr int kOStageBytes = 16384;            // per half: 64 output columns of its 128 rows
+constexpr int kOStageBytes = 32768;            // per half: all 128 output columns of its 128 rows
 constexpr int kOOff = kKVOff + kNS * kStageBytes;
 constexpr int kBarOff = kOOff + 2 * kOStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;
