@@ -14,7 +14,7 @@
 // The softmax releases S as soon as it holds it in registers, so QK^T of
 // chunk j+1 runs while it computes the exponentials of chunk j; the running
 // max is lazily updated (O is rescaled in TMEM only when a row max grows by
-// more than 2^8).  A third of the exponentials are
+// more than 2^8).  Half of the exponentials are
 // computed on the FMA pipe (2^x = 2^rint(x) * cubic(x - rint(x))) so that the
 // special-function unit, which otherwise needs as many cycles per chunk as
 // the tensor core, stops being the bound.
@@ -48,7 +48,7 @@ constexpr int kBarOff = kOOff + 2 * kOStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kEmuPeriod = 3;  // one pair of exponentials in kEmuPeriod on the FMA pipe
+constexpr int kEmuPeriod = 2;  // one pair of exponentials in kEmuPeriod on the FMA pipe
 
 // TMEM columns: S of half h at 64 h, P (bf16 pairs) of half h at 128 + 32 h,
 // O of half h at 256 + 128 h

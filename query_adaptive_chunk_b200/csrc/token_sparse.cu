@@ -932,8 +932,13 @@ __global__ void tsa_gather_kernel(const __nv_bfloat16* __restrict__ Q,
   const int n = min(count[u], Sc);
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < n; t += gridDim.x * wpb) {
-    const int p = idx[u * kmax + t];
+  const int stride = gridDim.x * wpb;
+  int t = blockIdx.x * wpb + (threadIdx.x >> 5);
+  int p_next = t < n ? idx[u * kmax + t] : 0;
+  for (; t < n; t += stride) {
+    const int p = p_next;
+    // the next row's position is loaded while this row's pieces move
+    if (t + stride < n) p_next = idx[u * kmax + t + stride];
 #pragma unroll 3
     for (int w = lane; w < per_row; w += 32) {
       const int part = w / V8, c = (w % V8) * 8;
