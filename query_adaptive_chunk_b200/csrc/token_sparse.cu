@@ -977,7 +977,7 @@ __global__ void tsa_inverse_kernel(const int32_t* __restrict__ idx,
 // head for them into shared memory (one coalesced row per head), then the
 // threads move independent 16-byte pieces, consecutive threads consecutive
 // pieces of an output row (coalesced stores; a kept row reads each head's
-// D contiguous elements of O^), four rows in flight per thread.
+// D contiguous elements of O^), eight rows in flight per thread.
 constexpr int kScatterRows = 32;
 constexpr int kScatterThreads = 256;
 template <int D>
@@ -1000,7 +1000,7 @@ __global__ void __launch_bounds__(kScatterThreads) tsa_scatter_kernel(
   for (int q = threadIdx.x; q < per_row; q += blockDim.x) {
     const int hq = q / V8, c = (q % V8) * 8;
     const int* it = inv_s + (hq / G) * kScatterRows;
-#pragma unroll 4
+#pragma unroll 8
     for (int r = 0; r < nrow; ++r) {
       const int t = it[r];
       int4 v = make_int4(0, 0, 0, 0);

@@ -61,6 +61,54 @@ def test_token_importance_matches_oracle(B, S, Hq, Hkv, D, n_obs):
             assert np.allclose(got, ref, rtol=1e-3, atol=1e-6), np.abs(got - ref).max()
 
 
+def test_token_budget_one_cta_per_sequence():
+    """More sequences than the SMs hold 8-CTA clusters of (B * 8 > SMs): the
+    one-CTA-per-sequence budget kernel, against the oracle's cut."""
+    from query_adaptive_chunk_b200 import csa
+    B, S, Hkv, tau = 20, 1536, 2, 0.2
+    assert B * 8 > torch.cuda.get_device_properties(0).multi_processor_count
+    rng = np.random.default_rng(11)
+    imp_np = (rng.random((B, Hkv, S)) ** 5).astype(np.float32)
+    imp = torch.tensor(imp_np, device="cuda")
+    k_seq = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    k_unit = torch.full((B * Hkv,), -7, dtype=torch.int32, device="cuda")
+    csa.csa_token_budget(imp, B, S, Hkv, tau, 64, k_seq, k_unit)
+    csa.csa_check_device_status()
+    for b in range(B):
+        mass = imp_np[b].astype(np.float64).sum(axis=0)
+        ref = O.coverage_budget(mass, tau)
+        got = int(k_seq[b])
+        if got != ref:
+            cum = np.cumsum(np.sort(mass / mass.sum())[::-1])
+            top = cum[got - 1] if got > 0 else 0.0
+            below = cum[got - 2] if got > 1 else 0.0
+            assert top >= (1 - tau) - 1e-6 and below <= (1 - tau) + 1e-6, (b, got, ref)
+            parity.NEAR_TIE_LOG.append(("token budget", b, got, ref))
+        assert k_unit[b * Hkv:(b + 1) * Hkv].tolist() == [min(S, (got + 63) // 64 * 64)] * Hkv
+
+
+def test_token_select_one_cta_per_unit():
+    """More units than the SMs hold 8-CTA clusters of (B * Hkv * 8 > SMs): the
+    one-CTA-per-unit top-k with each unit's k from device memory."""
+    from query_adaptive_chunk_b200 import csa
+    B, S, Hkv = 5, 8192, 4
+    U = B * Hkv
+    assert U * 8 > torch.cuda.get_device_properties(0).multi_processor_count
+    g = _gen(12)
+    imp = torch.randint(0, 40, (B, Hkv, S), generator=g, device="cuda").float() / 9.0
+    ks = [0, 1, S, S // 3] + [int(x) for x in np.random.default_rng(13).integers(1, S, U - 4)]
+    k_unit = torch.tensor(ks, dtype=torch.int32, device="cuda")
+    idx = torch.full((U, S), 777, dtype=torch.int32, device="cuda")
+    cnt = torch.full((U,), 777, dtype=torch.int32, device="cuda")
+    csa.csa_token_select(imp, B, S, Hkv, k_unit, idx, cnt)
+    csa.csa_check_device_status()
+    got = parity.gpu_sets(idx, cnt)
+    isn = imp.reshape(U, S).cpu().double().numpy()
+    for u in range(U):
+        ref, _ = O.select_topk(isn[u], ks[u], 0, 0)
+        assert got[u] == ref, (u, ks[u])
+
+
 @pytest.mark.parametrize("S,tau,seed", [(1000, 0.1, 1), (32768, 0.05, 2), (4096, 0.0, 3),
                                         (4096, 0.9, 4), (333, 0.3, 5)])
 def test_token_budget_matches_oracle(S, tau, seed):
