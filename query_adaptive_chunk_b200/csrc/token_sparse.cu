@@ -398,13 +398,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float bv = -INFINITY;
         int lv = -1;
         if (r < p.R) {
+          // the row's (max, sum) over the splits, kStatBatch splits' loads in
+          // flight at a time and folded online (each batch rescales the sum)
+          constexpr int kStatBatch = 16;
           const float2* pr = p.part + bh * nparts * p.R + r;
-          float M = -INFINITY;
-          for (int s = 0; s < nparts; ++s) M = fmaxf(M, pr[static_cast<int64_t>(s) * p.R].x);
-          float Ls = 0.f;
-          for (int s = 0; s < nparts; ++s) {
-            const float2 v = pr[static_cast<int64_t>(s) * p.R];
-            if (v.x != -INFINITY) Ls += v.y * exp2f(v.x - M);
+          float M = -INFINITY, Ls = 0.f;
+          for (int s0 = 0; s0 < nparts; s0 += kStatBatch) {
+            float2 v[kStatBatch];
+#pragma unroll
+            for (int k = 0; k < kStatBatch; ++k)
+              v[k] = s0 + k < nparts ? pr[static_cast<int64_t>(s0 + k) * p.R]
+                                     : make_float2(-INFINITY, 0.f);
+            float bm = M;
+#pragma unroll
+            for (int k = 0; k < kStatBatch; ++k) bm = fmaxf(bm, v[k].x);
+            if (bm == -INFINITY) continue;
+            Ls = M == -INFINITY ? 0.f : Ls * exp2f(M - bm);
+#pragma unroll
+            for (int k = 0; k < kStatBatch; ++k)
+              if (v[k].x != -INFINITY) Ls += v[k].y * exp2f(v[k].x - bm);
+            M = bm;
           }
           // weight of score s: 2^(s sl2 - M) / Ls = 2^(s sl2 + bias)
           bv = Ls > 0.f ? -(M + log2f(Ls)) : -INFINITY;
@@ -703,7 +716,10 @@ __global__ void __launch_bounds__(kBudgetCThreads) budget_cluster_kernel(
     int32_t* __restrict__ k_unit) {
   cluster_arrive_relaxed();
   extern __shared__ __align__(16) uint8_t sm[];
-  float* ms = reinterpret_cast<float*>(sm);  // [S / CS] this CTA's masses
+  constexpr int kWarps = kBudgetCThreads / 32;
+  unsigned int* whc = reinterpret_cast<unsigned int*>(sm);  // [kWarps][256] per-warp counts
+  float* whm = reinterpret_cast<float*>(whc + kWarps * 256);  // [kWarps][256] per-warp masses
+  float* ms = whm + kWarps * 256;            // [S / CS] this CTA's masses
   __shared__ unsigned int hc[256];           // this CTA's histogram of the pass
   __shared__ float hm[256];
   __shared__ unsigned int gc[256];           // the cluster's
@@ -719,13 +735,20 @@ __global__ void __launch_bounds__(kBudgetCThreads) budget_cluster_kernel(
   const int n = static_cast<int>(static_cast<int64_t>(S) * (rank + 1) / CS) - lo;
   const float* ib = imp + static_cast<int64_t>(b) * Hkv * S + lo;
   float part = 0.f;
-  for (int j = tid; j < n; j += blockDim.x) {
-    float m = 0.f;
+  // n <= kBudgetJ * blockDim.x (S <= 32768 over kBudgetCS CTAs): the loop is
+  // unrolled so that every load of the thread is in flight together
+  constexpr int kBudgetJ = 8;
+#pragma unroll
+  for (int k = 0; k < kBudgetJ; ++k) {
+    const int j = tid + k * kBudgetCThreads;
+    if (j < n) {
+      float m = 0.f;
 #pragma unroll 8
-    for (int h = 0; h < Hkv; ++h) m += ib[static_cast<int64_t>(h) * S + j];
-    m = fmaxf(m, 0.f);
-    ms[j] = m;
-    part += m;
+      for (int h = 0; h < Hkv; ++h) m += ib[static_cast<int64_t>(h) * S + j];
+      m = fmaxf(m, 0.f);
+      ms[j] = m;
+      part += m;
+    }
   }
 #pragma unroll
   for (int x = 16; x > 0; x >>= 1) part += __shfl_xor_sync(0xffffffffu, part, x);
@@ -749,42 +772,36 @@ __global__ void __launch_bounds__(kBudgetCThreads) budget_cluster_kernel(
   const float target = (1.0f - tau) * total;
   unsigned int mask = 0u;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int d = tid; d < 256; d += blockDim.x) {
-      hc[d] = 0u;
-      hm[d] = 0.f;
+    // each warp's own histogram (shared-memory atomics contend only within
+    // the warp: the masses' high bytes take few values), then the CTA's as
+    // their sum in warp order
+    unsigned int* wc = whc + (tid >> 5) * 256;
+    float* wm = whm + (tid >> 5) * 256;
+    for (int d = lane; d < 256; d += 32) {
+      wc[d] = 0u;
+      wm[d] = 0.f;
+    }
+    __syncwarp();
+    const unsigned int prefix = prefix_sh;
+    for (int j = tid; j < n; j += blockDim.x) {
+      const unsigned int key = __float_as_uint(ms[j]);
+      if ((key & mask) == prefix) {
+        const int d = static_cast<int>((key >> shift) & 255u);
+        atomicAdd(&wc[d], 1u);
+        atomicAdd(&wm[d], ms[j]);
+      }
     }
     __syncthreads();
-    const unsigned int prefix = prefix_sh;
-    for (int j0 = 0; j0 < n; j0 += blockDim.x) {
-      const int j = j0 + tid;
-      int d = -1;
-      float m = 0.f;
-      if (j < n) {
-        const unsigned int key = __float_as_uint(ms[j]);
-        if ((key & mask) == prefix) {
-          d = (key >> shift) & 255u;
-          m = ms[j];
-        }
+    for (int d = tid; d < 256; d += blockDim.x) {
+      unsigned int c = 0u;
+      float mm = 0.f;
+#pragma unroll 4
+      for (int w = 0; w < kWarps; ++w) {
+        c += whc[w * 256 + d];
+        mm += whm[w * 256 + d];
       }
-#pragma unroll
-      for (int round = 0; round < 3; ++round) {
-        const unsigned int act = __ballot_sync(0xffffffffu, d >= 0);
-        if (act == 0u) break;  // warp-uniform
-        const int d0 = __shfl_sync(0xffffffffu, d, __ffs(act) - 1);
-        const unsigned int same = __ballot_sync(0xffffffffu, d == d0);
-        float v = d == d0 ? m : 0.f;
-#pragma unroll
-        for (int x = 16; x > 0; x >>= 1) v += __shfl_xor_sync(0xffffffffu, v, x);
-        if (lane == 0) {
-          atomicAdd(&hc[d0], static_cast<unsigned int>(__popc(same)));
-          atomicAdd(&hm[d0], v);
-        }
-        if (d == d0) d = -1;  // counted
-      }
-      if (d >= 0) {
-        atomicAdd(&hc[d], 1u);
-        atomicAdd(&hm[d], m);
-      }
+      hc[d] = c;
+      hm[d] = mm;
     }
     cluster_arrive();  // every CTA's histogram of this pass is complete
     cluster_wait();
@@ -1022,8 +1039,12 @@ cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S,
                                 float tau, int tile, int32_t* k_seq, int32_t* k_unit) {
   if (B == 0) return cudaSuccess;
   if (B <= 65535 && static_cast<int64_t>(B) * kBudgetCS <= l.num_sms) {  // one cluster per sequence
-    const size_t shc = static_cast<size_t>((S + kBudgetCS - 1) / kBudgetCS) * 4;
-    cudaError_t e = set_smem_ts(reinterpret_cast<const void*>(budget_cluster_kernel), shc);
+    const size_t shc = static_cast<size_t>((S + kBudgetCS - 1) / kBudgetCS) * 4 +
+                       static_cast<size_t>(kBudgetCThreads / 32) * 256 * 8;
+    // always set: with its static histograms the kernel may pass 48 KB in all
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(budget_cluster_kernel),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(shc));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kBudgetCS, B);
