@@ -341,9 +341,9 @@ CSA_API csa_status csa_sparse_decode(const void* q, const void* K, const void* V
 CSA_API int csa_decode_default_parts(csa_dtype dtype, int D, int L);
 
 /* Fused a1 + a2 (decode, Nq = 1): the scores of csa_score_chunks computed
- * straight into shared memory, one CTA per unit, then the top-k of
- * csa_select_topk; same arithmetic, so the index lists equal the two-call
- * path's bit for bit.  Units of heads with head_full[h] != 0 get count 0 and
+ * straight into shared memory (one CTA per unit, or one thread-block cluster
+ * per unit when the lists are short), then the top-k of csa_select_topk;
+ * same arithmetic, so the index lists equal the two-call path's bit for bit.  Units of heads with head_full[h] != 0 get count 0 and
  * an all -1 row (csa_sparse_decode reads every chunk for them).
  *   q [B, Hq, D];  proj NULL or [D, R];  summ [B, Hkv, C, Ds] fp32
  *   idx [B*Hkv, kmax], count [B*Hkv] (outputs);  same limits as the two calls. */
