@@ -18,6 +18,10 @@
 // computed on the FMA pipe (2^x = 2^rint(x) * cubic(x - rint(x))) so that the
 // special-function unit, which otherwise needs as many cycles per chunk as
 // the tensor core, stops being the bound.
+// P is double-buffered in tensor memory: the softmax of chunk j + 1 writes
+// its P while the PV of chunk j still reads the other buffer, so it waits
+// only for the PV two chunks back (and for the previous one when O has to be
+// rescaled).
 // Warp roles: warp 0 issues TMA (each half of the Q tile once per unit, K/V
 // per chunk into a 3-stage ring), warp 1 allocates TMEM, one thread of warp
 // 1 issues the MMAs of half 0 and one thread of warp 2 those of half 1 (in
@@ -50,8 +54,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kEmuPeriod = 2;  // one pair of exponentials in kEmuPeriod on the FMA pipe
 
-// TMEM columns: S of half h at 64 h, P (bf16 pairs) of half h at 128 + 32 h,
-// O of half h at 256 + 128 h
+// TMEM columns: S of half h at 64 h, P buffer u (bf16 pairs) of half h at
+// 128 + 64 u + 32 h, O of half h at 256 + 128 h
 constexpr uint32_t kColP = 128, kColO = 256;
 
 // instruction descriptors: QK^T M = 128, N = 64 (both K-major); PV M = 128,
@@ -151,9 +155,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t kv_full = bar + 32, kv_empty = kv_full + 8 * kNS;
   const uint32_t s_full = kv_empty + 8 * kNS;               // [2]
   const uint32_t s_free = s_full + 16;                      // [2]
-  const uint32_t p_full = s_free + 16;                      // [2]
-  const uint32_t pv_done = p_full + 16;                     // [2]
-  const uint32_t drain = pv_done + 16;                      // [2]
+  const uint32_t p_full = s_free + 16;                      // [2 halves][2 P buffers]
+  const uint32_t pv_done = p_full + 32;                     // [2][2]
+  const uint32_t drain = pv_done + 32;                      // [2]
   const uint32_t o_full = drain + 16;                       // [2] a half's staged O columns
   const uint32_t o_free = o_full + 16;                      // [2] ... have been read by the store
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + (o_free + 16 - bar));
@@ -165,8 +169,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(q_empty + 8 * h, 1);
       mbar_init(s_full + 8 * h, 1);
       mbar_init(s_free + 8 * h, 128);
-      mbar_init(p_full + 8 * h, 128);
-      mbar_init(pv_done + 8 * h, 1);
+      for (int u = 0; u < 2; ++u) {
+        mbar_init(p_full + 8 * (2 * h + u), 128);
+        mbar_init(pv_done + 8 * (2 * h + u), 1);
+      }
     }
     for (int s = 0; s < kNS; ++s) {
       mbar_init(kv_full + 8 * s, 1);
@@ -260,7 +266,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // half's QK^T -> softmax -> PV chain runs at its own pace.
     const int hf = warp - 1;
     if (lane == 0) {
-      uint32_t q_phase = 0, p_phase = 0, s_cnt = 0, kv_it = 0;
+      uint32_t q_phase = 0, s_cnt = 0, kv_it = 0;
       bool ok = true;
       const uint32_t qa = sQ + hf * kQHalfBytes;
       // S of this half is overwritten only after the softmax has loaded the
@@ -281,15 +287,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ++s_cnt;
         return true;
       };
-      auto pv = [&](uint32_t stage, bool acc) {
+      // PV of this half's chunk k (kv_it) reads P buffer k & 1 and signals
+      // pv_done[hf][k & 1]
+      auto pv = [&](uint32_t stage, bool acc, uint32_t k) {
         const uint32_t d = tmem + kColO + hf * 128;
-        const uint32_t pa = tmem + kColP + hf * 32;
+        const uint32_t pa = tmem + kColP + (k & 1u) * 64 + hf * 32;
         const uint32_t vb = sKV + stage * kStageBytes + kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_ts(d, pa + kk * 8, smem_desc(vb + kk * 2048, 8192, 1024), kIdescPV,
                   (acc || kk > 0) ? 1u : 0u);
-        umma_commit(pv_done + 8 * hf);
+        umma_commit(pv_done + 8 * (2 * hf + (k & 1u)));
       };
       for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
         int b, h, t;
@@ -309,11 +317,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!qk(nxt)) { ok = false; break; }
             if (j + 2 == n) umma_commit(q_empty + 8 * hf);
           }
-          // P of chunk j written, and (implied) the PV of chunk j - 1 done
-          if (!mbar_wait(p_full + 8 * hf, p_phase, p.err)) { ok = false; break; }
-          p_phase ^= 1u;
+          // P of chunk j written (its buffer's (kv_it / 2)-th fill)
+          if (!mbar_wait(p_full + 8 * (2 * hf + (kv_it & 1u)), (kv_it >> 1) & 1u, p.err)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          pv(cur, j > 0);
+          pv(cur, j > 0, kv_it);
           umma_commit(kv_empty + 8 * cur);  // the stage is free once both halves' reads are done
           ++kv_it;
         }
@@ -329,14 +339,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int r = ((warp & 3) << 5) + lane;  // row within the half == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + half * 64;
-    const uint32_t tP = tmem + lane_base + kColP + half * 32;
+    const uint32_t tP = tmem + lane_base + kColP + half * 32;  // + 64 per buffer
     const uint32_t tO = tmem + lane_base + kColO + half * 128;
-    const uint32_t my_p_full = p_full + 8 * half, my_pv_done = pv_done + 8 * half;
     const int g = half * 2 + (r >> 6);  // query head within the group
     const int i = r & 63;               // row within the tile
     const float sl = p.scale_log2;
-    uint32_t s_cnt = 0, pv_phase = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0;  // s_cnt: this half's chunks so far (chunk k has PV k)
+    int64_t pv_seen = -1;            // the latest PV known complete (all earlier ones too)
     bool ok = true;
+    // Wait until PV k is complete: the (k / 2)-th completion of pv_done[half][k & 1];
+    // waits come in increasing k, and PV k + 2 needs a P written after this wait
+    auto wait_pv = [&](int64_t k) -> bool {
+      if (k <= pv_seen) return true;
+      if (!warp_wait(pv_done + 8 * (2 * half + static_cast<int>(k & 1)),
+                     static_cast<uint32_t>(k >> 1) & 1u, p.err))
+        return false;
+      pv_seen = k;
+      tc_fence_after();
+      return true;
+    };
     for (int w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       int b, h, t;
       unit_coords(p, T, w, b, h, t);
@@ -355,6 +376,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int c = c_next;
         if (j + 1 < n) c_next = unit_chunk(p, sel, j + 1);
         const uint32_t sph = s_cnt & 1u;
+        const int64_t kc = s_cnt;  // this chunk's index: P buffer kc & 1, PV kc
         ++s_cnt;
         // wait results are made warp-uniform: the TMEM accesses below are
         // warp-collective
@@ -388,14 +410,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           mq[a] = fmaxf(v, x[16 * a + 15]);
         }
         const float mnew = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmaxf(mq[3], m));
-        // P and O of this half are free once the previous chunk's PV is done
-        if (j > 0) {
-          if (!warp_wait(my_pv_done, pv_phase, p.err)) {
-            ok = false;
-            break;
-          }
-          pv_phase ^= 1u;
-          tc_fence_after();
+        // this chunk's P buffer is free once the PV two chunks back is done
+        if (!wait_pv(kc - 2)) {
+          ok = false;
+          break;
         }
         // Lazy rescale: a row moves its max only when it grew by more than
         // 2^8.  tcgen05.ld/st are warp-collective, so the warp rescales
@@ -409,6 +427,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         if (m == -INFINITY) m = mnew;  // first visible keys: nothing accumulated in O yet
         if (__any_sync(0xffffffffu, grow)) {
+          // O is rescaled in place: every PV issued so far has to be done
+          if (!wait_pv(kc - 1)) {
+            ok = false;
+            break;
+          }
 #pragma unroll 1
           for (int cc = 0; cc < 128; cc += 32) {
             uint32_t ov[32];
@@ -450,19 +473,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
              (acc[3].x + acc[3].y);
-        tmem_st32(tP, pk);  // P row r (bf16 pairs), the A operand of this half's PV
+        // P row r (bf16 pairs), the A operand of this half's PV
+        tmem_st32(tP + static_cast<uint32_t>(kc & 1) * 64, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(my_p_full);
+        mbar_arrive(p_full + 8 * (2 * half + static_cast<int>(kc & 1)));
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 rows, once the unit's last PV is done
-      if (!warp_wait(my_pv_done, pv_phase, p.err)) {
+      if (!wait_pv(static_cast<int64_t>(s_cnt) - 1)) {
         ok = false;
         break;
       }
-      pv_phase ^= 1u;
-      tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
       // O / l as bf16 into this half's staging area, laid out as the output
       // map's [64 x 64] boxes (128-byte swizzle), kOStageBytes / 256 columns
