@@ -1,38 +1,79 @@
 // Precompute kernels: chunk summaries (chunk-mean keys, optionally projected
 // to a low rank), meta-summaries (mean of Gm chunk summaries) and tile-mean
 // queries.  These run once per cache / per prefill, outside the per-step path;
-// each is a coalesced reduction over rows.
+// each is a reduction over rows with 16-byte loads, several rows in flight
+// per thread.
 #include "internal.h"
 
 namespace csa {
 namespace {
 
-template <typename T>
-__device__ __forceinline__ float ld_f(const T* p);
-template <>
-__device__ __forceinline__ float ld_f<float>(const float* p) { return __ldg(p); }
-template <>
-__device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16* p) {
-  return __bfloat162float(*p);
+// Sums the E values of a 16-byte vector into acc (bf16: 8 values, fp32: 4).
+__device__ __forceinline__ void add16(float* acc, const uint4& v, const __nv_bfloat16*) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    acc[2 * e] += f.x;
+    acc[2 * e + 1] += f.y;
+  }
+}
+__device__ __forceinline__ void add16(float* acc, const uint4& v, const float*) {
+  acc[0] += __uint_as_float(v.x);
+  acc[1] += __uint_as_float(v.y);
+  acc[2] += __uint_as_float(v.z);
+  acc[3] += __uint_as_float(v.w);
 }
 
-// One CTA per (chunk, unit); thread d sums column d over the chunk's L rows,
-// in row order, in fp32.  With a projection the mean goes through shared
-// memory and R threads form the [R] outputs.
-template <typename T>
-__global__ void chunk_summaries_kernel(const T* __restrict__ K, int64_t T_len, int D, int L,
-                                       const float* __restrict__ proj, int R,
-                                       float* __restrict__ summ) {
-  extern __shared__ float mean_sh[];
+// One CTA of kSummThreads per (chunk, unit).  A key row of D values is D / E
+// 16-byte pieces (E = 8 bf16 or 4 fp32 values); thread t takes piece
+// t % (D / E) of the rows rg, rg + RG, ... (rg = t / (D / E), RG row groups
+// side by side), eight rows in flight, summing in fp32 in row order; the RG
+// partial sums of each column then meet in shared memory and are added in
+// row-group order.  With a projection R threads form the [R] outputs from
+// the mean.
+constexpr int kSummThreads = 128;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSummThreads, 8) chunk_summaries_kernel(
+    const T* __restrict__ K, int64_t T_len, int L, const float* __restrict__ proj, int R,
+    float* __restrict__ summ) {
+  constexpr int E = 16 / sizeof(T);
+  constexpr int TPR = D / E;                 // threads per row
+  constexpr int RG = kSummThreads / TPR;     // rows in parallel
+  constexpr int UNROLL = 8;
+  __shared__ float part[RG][D];
+  __shared__ float mean_sh[D];
   const int c = blockIdx.x;
   const int u = blockIdx.y;
   const int C = static_cast<int>(T_len / L);
-  const T* base = K + (static_cast<int64_t>(u) * T_len + static_cast<int64_t>(c) * L) * D;
+  const int piece = threadIdx.x % TPR, rg = threadIdx.x / TPR;
+  const T* base =
+      K + (static_cast<int64_t>(u) * T_len + static_cast<int64_t>(c) * L) * D + piece * E;
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  int j = rg;
+  for (; j + (UNROLL - 1) * RG < L; j += UNROLL * RG) {
+    uint4 v[UNROLL];
+#pragma unroll
+    for (int k = 0; k < UNROLL; ++k)
+      v[k] = __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(j + k * RG) * D));
+#pragma unroll
+    for (int k = 0; k < UNROLL; ++k) add16(acc, v[k], static_cast<const T*>(nullptr));
+  }
+  for (; j < L; j += RG)
+    add16(acc, __ldg(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(j) * D)),
+          static_cast<const T*>(nullptr));
+#pragma unroll
+  for (int e = 0; e < E; ++e) part[rg][piece * E + e] = acc[e];
+  __syncthreads();
   const float invL = 1.0f / static_cast<float>(L);
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int j = 0; j < L; ++j) acc += ld_f<T>(base + static_cast<int64_t>(j) * D + d);
-    float m = acc * invL;
+  for (int d = threadIdx.x; d < D; d += kSummThreads) {
+    float m = 0.f;
+#pragma unroll
+    for (int r = 0; r < RG; ++r) m += part[r][d];
+    m *= invL;
     if (proj == nullptr)
       summ[(static_cast<int64_t>(u) * C + c) * D + d] = m;
     else
@@ -40,10 +81,10 @@ __global__ void chunk_summaries_kernel(const T* __restrict__ K, int64_t T_len, i
   }
   if (proj == nullptr) return;
   __syncthreads();
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    float acc = 0.f;
-    for (int d = 0; d < D; ++d) acc += __ldg(proj + static_cast<int64_t>(d) * R + r) * mean_sh[d];
-    summ[(static_cast<int64_t>(u) * C + c) * R + r] = acc;
+  for (int r = threadIdx.x; r < R; r += kSummThreads) {
+    float a = 0.f;
+    for (int d = 0; d < D; ++d) a += __ldg(proj + static_cast<int64_t>(d) * R + r) * mean_sh[d];
+    summ[(static_cast<int64_t>(u) * C + c) * R + r] = a;
   }
 }
 
@@ -66,21 +107,6 @@ __global__ void meta_summaries_kernel(const float* __restrict__ summ, int C, int
 // eight rows in flight.  Grid: (tiles, row segments of 128 threads, batch).
 constexpr int kTileMeanThreads = 128;
 
-__device__ __forceinline__ void add16(float* acc, const uint4& v, const __nv_bfloat16*) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __bfloat1622float2(h[e]);
-    acc[2 * e] += f.x;
-    acc[2 * e + 1] += f.y;
-  }
-}
-__device__ __forceinline__ void add16(float* acc, const uint4& v, const float*) {
-  acc[0] += __uint_as_float(v.x);
-  acc[1] += __uint_as_float(v.y);
-  acc[2] += __uint_as_float(v.z);
-  acc[3] += __uint_as_float(v.w);
-}
 
 template <typename T>
 __global__ void __launch_bounds__(kTileMeanThreads) tile_mean_kernel(
@@ -120,14 +146,20 @@ cudaError_t launch_chunk_summaries(const Launch& l, const void* K, bool bf16, in
   const int C = static_cast<int>(T / L);
   if (C == 0 || U == 0) return cudaSuccess;
   dim3 grid(C, U);
-  const int threads = D >= 128 ? 128 : 64;
-  const size_t sh = proj ? D * sizeof(float) : 0;
-  if (bf16)
-    chunk_summaries_kernel<__nv_bfloat16><<<grid, threads, sh, l.stream>>>(
-        static_cast<const __nv_bfloat16*>(K), T, D, L, proj, R, summ);
-  else
-    chunk_summaries_kernel<float><<<grid, threads, sh, l.stream>>>(static_cast<const float*>(K), T,
-                                                                   D, L, proj, R, summ);
+  const auto* kb = static_cast<const __nv_bfloat16*>(K);
+  const auto* kf = static_cast<const float*>(K);
+  const int th = kSummThreads;
+  if (D == 128 && bf16)
+    chunk_summaries_kernel<__nv_bfloat16, 128><<<grid, th, 0, l.stream>>>(kb, T, L, proj, R, summ);
+  else if (D == 128)
+    chunk_summaries_kernel<float, 128><<<grid, th, 0, l.stream>>>(kf, T, L, proj, R, summ);
+  else if (D == 64 && bf16)
+    chunk_summaries_kernel<__nv_bfloat16, 64><<<grid, th, 0, l.stream>>>(kb, T, L, proj, R, summ);
+  else if (D == 64)
+    chunk_summaries_kernel<float, 64><<<grid, th, 0, l.stream>>>(kf, T, L, proj, R, summ);
+  else {
+    return cudaErrorInvalidValue;  // D is 64 or 128 (checked by the caller)
+  }
   return cudaGetLastError();
 }
 
