@@ -87,7 +87,9 @@ csa_status csa_sparse_decode_merged_noalloc(const void* q, const void* K, const 
   // call also clears them after its decode, so that a call that ended early
   // (a wait past its time limit, reported by csa_check_device_status) does
   // not leave a count behind for the next one.  The clear is one memset node
-  // of B * Hkv counters on the stream (a few hundred bytes).
+  // of B * Hkv counters on the stream (a few hundred bytes).  No test makes a
+  // decode's waits run out on purpose: a limit short enough for that would
+  // also cut short the wait for its own copies in flight before it retires.
   const size_t counter_bytes = (static_cast<size_t>(B) * Hkv * 4 + 255) & ~size_t(255);
   cudaError_t e = cudaMemsetAsync(ws, 0, counter_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
