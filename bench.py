@@ -891,7 +891,8 @@ def run_only(args, flush, peaks):
     if isinstance(w, synth.PrefillWorkload):
         r = time_prefill(w, args.steps, args.warmup, flush)
         ms = statistics.mean(r["attend_ms"])
-        d = {"workload": w.name, "attend_ms": ms, "tflops": r["flops"] / (ms * 1e-3) / 1e12}
+        d = {"workload": w.name, "attend_ms": ms, "tflops": r["flops"] / (ms * 1e-3) / 1e12,
+             "select_ms": statistics.mean(r["select_ms"])}
     else:
         r = time_decode(w, args.steps, args.warmup, flush)
         us = 1000 * statistics.mean(r["step_ms"])

@@ -1500,7 +1500,9 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
   float* lh = mh + 8;                              // [8]
   float* ah = lh + 8;                              // [8]
   float* wts = ah + 8;                             // [kMergeWts] merge weights
-  int* prefix = reinterpret_cast<int*>(wts + kMergeWts);  // [U+1]
+  float* ks = wts + kMergeWts;                     // [L][D + 1] the chunk's keys (padded rows)
+  float* vs = ks + 128 * (D + 1);                  // [L][D] its values (16-byte aligned)
+  int* prefix = reinterpret_cast<int*>(vs + 128 * D);  // [U+1]
   __shared__ int scan_sh[33];
   __shared__ int last_sh;
   build_prefix(p, prefix, scan_sh);
@@ -1563,8 +1565,40 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
     const int u = cur_u;
     const int c = unit_chunk(p, u, static_cast<int>(g - prefix[u]));
     const int64_t row0 = u * p.T + static_cast<int64_t>(c) * L;
+    {
+      // the chunk's K and V rows into shared memory: 16-byte loads, up to
+      // eight of each in flight per thread (one round for L = D = 64)
+      constexpr int D4 = D / 4;
+      const float4* kg = reinterpret_cast<const float4*>(p.Kf + row0 * D);
+      const float4* vg = reinterpret_cast<const float4*>(p.Vf + row0 * D);
+      const int n4 = L * D4;
+      for (int e0 = 0; e0 < n4; e0 += 8 * kF32Threads) {
+        float4 kv[8], vv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int e = e0 + k * kF32Threads + tid;
+          if (e < n4) {
+            kv[k] = __ldg(kg + e);
+            vv[k] = __ldg(vg + e);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int e = e0 + k * kF32Threads + tid;
+          if (e < n4) {
+            float* kd = ks + (e / D4) * (D + 1) + (e % D4) * 4;
+            kd[0] = kv[k].x;
+            kd[1] = kv[k].y;
+            kd[2] = kv[k].z;
+            kd[3] = kv[k].w;
+            reinterpret_cast<float4*>(vs)[e] = vv[k];
+          }
+        }
+      }
+    }
+    __syncthreads();
     if (tid < L) {
-      const float* kr = p.Kf + (row0 + tid) * D;
+      const float* kr = ks + tid * (D + 1);
       for (int x = 0; x < G; ++x) {
         float acc = 0.f;
         for (int d = 0; d < D; ++d) acc += qs[x * D + d] * kr[d];
@@ -1591,7 +1625,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
     if (tid < D) {
       for (int x = 0; x < G; ++x) {
         float acc = 0.f;
-        for (int j = 0; j < L; ++j) acc += sc[x * 128 + j] * p.Vf[(row0 + j) * D + tid];
+        for (int j = 0; j < L; ++j) acc += sc[x * 128 + j] * vs[j * D + tid];
         o[x] = o[x] * ah[x] + acc;
       }
     }
@@ -1812,7 +1846,8 @@ int decode_default_parts(bool bf16, int D, int L, int num_sms) {
 }
 
 size_t decode_f32_smem_bytes(int D, int U) {
-  return static_cast<size_t>(8 * D + 8 * 128 + 24 + kMergeWts + U + 1) * 4;
+  return static_cast<size_t>(8 * D + 8 * 128 + 24 + kMergeWts + 128 * (D + 1) + 128 * D + U + 1) *
+         4;
 }
 
 cudaError_t launch_decode(const Launch& l, const void* q, const void* K, const void* V, bool bf16,

@@ -1860,8 +1860,11 @@ cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int 
   cudaError_t e = set_smem(reinterpret_cast<const void*>(select_topk_kernel), sh);
   if (e != cudaSuccess) return e;
   const CausalRows causal{causal_tiles, causal_tile_m, causal_L};
-  select_topk_kernel<<<U, kSelThreads, sh, l.stream>>>(scores, C, n_valid, k_free, n_sink, n_local,
-                                                       idx, count, kmax, k_dev, causal);
+  // short rows (C <= 1024: at most 8 sort positions per thread) take 128
+  // threads, so four times as many units are in flight per SM
+  const int threads = C <= 1024 ? 128 : kSelThreads;
+  select_topk_kernel<<<U, threads, sh, l.stream>>>(scores, C, n_valid, k_free, n_sink, n_local,
+                                                   idx, count, kmax, k_dev, causal);
   return cudaGetLastError();
 }
 
