@@ -461,14 +461,17 @@ def time_prefill(w, steps: int, warmup: int, flush):
 TOKEN_STAGES = ("importance", "budget", "select", "compress", "attend", "decompress")
 
 
-def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1):
+def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1,
+                      dense: bool = False):
     """Token Sparse Attention prefill (importance, budget, each KV head's own
     tokens, compress, dense causal attention of the kept tokens, decompress).
 
     Two CUDA graphs replayed alternately, L2 flushed before each: G1 is the
     whole call (csa_token_sparse_prefill) between events and gives the
     per-call time; G2 runs the same six steps as the separate calls with an
-    event between each pair and gives each step's share."""
+    event between each pair and gives each step's share.  `dense`: also time
+    the dense causal attention of every token (the same attention kernel with
+    every KV head keeping all S tokens), the attention the method replaces."""
     from query_adaptive_chunk_b200 import csa
     inp = synth.make_prefill_inputs(w, device="cuda")
     Q, K, V = inp["Q"], inp["K"], inp["V"]
@@ -545,13 +548,30 @@ def time_token_sparse(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: f
     csa.csa_check_device_status()
     assert torch.equal(O, O2), "the separate calls must give the whole call's output"
     del g1, g2
+    dense_ms = []
+    if dense:
+        k_all = torch.full((U,), S, dtype=torch.int32, device=dev)
+        for _ in range(max(1, warmup)):
+            csa.csa_token_attend(Q, K, V, k_all, B, S, Hq, Hkv, D, scale, Oc)
+        torch.cuda.synchronize()
+        for _ in range(max(3, steps // 2)):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            csa.csa_token_attend(Q, K, V, k_all, B, S, Hq, Hkv, D, scale, Oc)
+            e1.record()
+            torch.cuda.synchronize()
+            dense_ms.append(e0.elapsed_time(e1))
+        csa.csa_check_device_status()
     k = int(budget.max())
     kt = min(S, (k + 63) // 64 * 64)
     n_t = kt // 64
     # dense causal attention of the kept tokens: tile t sees tiles 0..t
     flops = B * Hkv * (n_t * (n_t + 1) // 2) * w.G * 2 * (2 * 64 * 64 * D)
+    n_all = S // 64
+    dense_flops = B * Hkv * (n_all * (n_all + 1) // 2) * w.G * 2 * (2 * 64 * 64 * D)
     return {"ms": ms, "stage_ms": stage_ms, "budget": k, "kept_tokens": kt, "flops": flops,
-            "n_obs": n_obs, "tau": tau}
+            "n_obs": n_obs, "tau": tau, "dense_ms": dense_ms, "dense_flops": dense_flops}
 
 
 def token_sparse_line(w, r) -> dict:
@@ -570,7 +590,12 @@ def token_sparse_line(w, r) -> dict:
             "attend_tflops": round(r["flops"] / (st["attend"] * 1e-3) / 1e12, 1),
             "stage_ms": {k: round(v, 4) for k, v in st.items()},
             "overhead_share": round((tot - st["attend"]) / tot, 4),
-            "importance_budget_share": round((st["importance"] + st["budget"]) / tot, 4)}
+            "importance_budget_share": round((st["importance"] + st["budget"]) / tot, 4),
+            **({"dense_attention_ms": round(statistics.mean(r["dense_ms"]), 3),
+                "dense_attention_tflops": round(
+                    r["dense_flops"] / (statistics.mean(r["dense_ms"]) * 1e-3) / 1e12, 1),
+                "speedup_vs_dense_attention": round(statistics.mean(r["dense_ms"]) / ms, 2)}
+               if r["dense_ms"] else {})}
 
 
 def time_token_importance(w, steps: int, warmup: int, flush, n_obs: int = 64, tau: float = 0.1):
@@ -851,8 +876,10 @@ def other_workloads(args, flush, peaks):
         del r
         torch.cuda.empty_cache()
     for tw, name in ((synth.PREFILL_32K, "token_sparse_prefill_bf16_seq32k"),
-                     (synth.TOKEN_SPARSE_HEAVY_32K, synth.TOKEN_SPARSE_HEAVY_32K.name)):
-        r = time_token_sparse(tw, steps, args.warmup, flush)
+                     (synth.TOKEN_SPARSE_HEAVY_32K, synth.TOKEN_SPARSE_HEAVY_32K.name),
+                     (synth.TOKEN_SPARSE_HEAVY_128K, synth.TOKEN_SPARSE_HEAVY_128K.name)):
+        r = time_token_sparse(tw, steps, args.warmup, flush,
+                              dense=tw is synth.TOKEN_SPARSE_HEAVY_128K)
         out[name] = token_sparse_line(tw, r)
         del r
         torch.cuda.empty_cache()
@@ -874,6 +901,11 @@ def other_workloads(args, flush, peaks):
 
 def run_only(args, flush, peaks):
     """Time one named workload alone and print its figures (profiling aid)."""
+    if args.only == synth.TOKEN_SPARSE_HEAVY_128K.name:
+        tw = synth.TOKEN_SPARSE_HEAVY_128K
+        r = time_token_sparse(tw, args.steps, args.warmup, flush, dense=True)
+        print(json.dumps({"workload": args.only, **token_sparse_line(tw, r)}))
+        return 0
     if args.only in ("token_sparse_prefill_bf16_seq32k", synth.TOKEN_SPARSE_HEAVY_32K.name):
         tw = synth.PREFILL_32K if args.only == "token_sparse_prefill_bf16_seq32k" else \
             synth.TOKEN_SPARSE_HEAVY_32K

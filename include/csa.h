@@ -161,7 +161,9 @@ CSA_API csa_status csa_token_importance(const void* Q, const void* K, int B, int
  * reaches 1 - tau.  k_unit[b*Hkv + h] = k_seq[b] rounded up to a multiple of
  * `tile` (at most S): the token count every KV head of sequence b keeps.
  * Float sums: a cut within rounding of a tie may land one token apart from
- * exact arithmetic.  tau in [0, 1); S <= 32768. */
+ * exact arithmetic.  tau in [0, 1); S <= 32768, or up to 131072 when B * 8
+ * <= the number of SMs (one cluster of 8 CTAs per sequence); other sizes
+ * return CSA_ERR_UNSUPPORTED. */
 CSA_API csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, float tau, int tile,
                                     int32_t* k_seq, int32_t* k_unit, csa_stream stream);
 
@@ -174,7 +176,9 @@ CSA_API csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, flo
  * with every earlier tile visible); decompress: each output row back to its
  * position, every other row of O set to 0.
  *   O [B, S, Hq, D] bf16 (output); budget_out [B] int32 device (output, the
- *   unrounded k_seq).  D = 128, Hq/Hkv = 4, S % 64 == 0, S <= 32768.
+ *   unrounded k_seq).  D = 128, Hq/Hkv = 4, S % 64 == 0, S <= 32768, or up
+ *   to 131072 when B * Hkv * 8 <= the number of SMs (the budget and the
+ *   token choice then run on their cluster paths); else CSA_ERR_UNSUPPORTED.
  *   workspace >= csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs).
  * Every step runs on the device from the budgets the device computed: the
  * compressed buffers are laid out for S kept tokens, and the dense attention
@@ -191,7 +195,8 @@ CSA_API csa_status csa_token_sparse_prefill(const void* Q, const void* K, const 
  * (the same kernels, in the same order): compress ("핵심 아키텍처": gather
  * the kept tokens), attend (dense causal attention of the compressed
  * sequences) and decompress (scatter back).  Same shapes and limits as the
- * whole call (D = 128, Hq/Hkv = 4, S % 64 == 0, S <= 32768); compressed
+ * whole call (D = 128, Hq/Hkv = 4, S % 64 == 0, S <= 131072; csa_token_select
+ * above 32768 only when B * Hkv * 8 <= the number of SMs); compressed
  * buffers Qc [B, S, Hq, D], Kc/Vc [B, Hkv, S, D], Oc [B, S, Hq, D] bf16,
  * laid out for S kept tokens.
  *

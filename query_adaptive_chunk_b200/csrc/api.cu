@@ -922,6 +922,22 @@ csa_status importance_checks(const void* Q, const void* K, int B, int S, int Hq,
   CSA_TRY(check_ptr(K, "K"));
   return CSA_OK;
 }
+
+// Sequences longer than 32768 tokens (up to 131072): the coverage budget and
+// the per-head token choice then run only on their cluster paths, which hold
+// S / 8 values per CTA and need B * 8 and B * Hkv * 8 CTAs on the SMs.
+constexpr int kTokenMaxS = 131072;
+csa_status token_long_check(int B, int Hkv, int S, const csa::Launch& l, bool budget, bool select) {
+  if (S <= 32768) return CSA_OK;
+  CSA_SUPPORT(S <= kTokenMaxS, "S must be <= 131072");
+  if (budget)
+    CSA_SUPPORT(csa::token_budget_cluster_fits(B, l.num_sms),
+                "S > 32768 needs B * 8 <= the number of SMs");
+  if (select)
+    CSA_SUPPORT(csa::topk_cluster_fits(B * Hkv, S, l.num_sms),
+                "S > 32768 needs B * Hkv * 8 <= the number of SMs");
+  return CSA_OK;
+}
 }  // namespace
 
 csa_status csa_token_importance(const void* Q, const void* K, int B, int S, int Hq, int Hkv,
@@ -946,13 +962,14 @@ csa_status csa_token_budget(const float* imp, int B, int S, int Hkv, float tau, 
                             int32_t* k_seq, int32_t* k_unit, csa_stream stream) {
   CSA_REQUIRE(B >= 0 && S >= 0 && Hkv > 0 && tile > 0, "bad sizes");
   CSA_REQUIRE(tau == tau && tau >= 0.f && tau < 1.f, "tau must be in [0, 1)");
-  CSA_SUPPORT(S <= 32768, "S must be <= 32768");
+  CSA_SUPPORT(S <= kTokenMaxS, "S must be <= 131072");
   if (B == 0) return CSA_OK;
   CSA_TRY(check_ptr(imp, "imp"));
   CSA_TRY(check_ptr(k_seq, "k_seq"));
   CSA_TRY(check_ptr(k_unit, "k_unit"));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
+  CSA_TRY(token_long_check(B, Hkv, S, l, true, false));
   return finish(csa::launch_token_budget(l, imp, B, S, Hkv, tau, tile, k_seq, k_unit),
                 "token budget launch");
 }
@@ -995,8 +1012,8 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
   CSA_TRY(importance_checks(Q, K, B, S, Hq, Hkv, D, n_obs, scale));
   CSA_REQUIRE(tau == tau && tau >= 0.f && tau < 1.f, "tau must be in [0, 1)");
   CSA_REQUIRE(S % 64 == 0, "S must be a multiple of 64");
-  CSA_SUPPORT(D == 128 && Hq / Hkv == 4 && S <= 32768,
-              "implemented for D = 128, Hq/Hkv = 4 and S <= 32768");
+  CSA_SUPPORT(D == 128 && Hq / Hkv == 4 && S <= kTokenMaxS,
+              "implemented for D = 128, Hq/Hkv = 4 and S <= 131072");
   if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
   const TsaLayout w = tsa_layout(B, S, Hq, Hkv, D, n_obs);
   CSA_REQUIRE(workspace_bytes >= static_cast<int64_t>(w.total),
@@ -1007,6 +1024,7 @@ csa_status csa_token_sparse_prefill(const void* Q, const void* K, const void* V,
   CSA_TRY(check_ptr(budget_out, "budget_out"));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
+  CSA_TRY(token_long_check(B, Hkv, S, l, true, true));
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* imp = reinterpret_cast<float*>(ws + w.imp);
   int32_t* k_unit = reinterpret_cast<int32_t*>(ws + w.k_unit);
@@ -1050,8 +1068,8 @@ csa_status token_shape_checks(int B, int S, int Hq, int Hkv, int D) {
   CSA_REQUIRE(B >= 0 && S >= 0 && Hq > 0 && Hkv > 0 && D > 0, "bad sizes");
   CSA_REQUIRE(Hq % Hkv == 0, "Hq must be a multiple of Hkv");
   CSA_REQUIRE(S % 64 == 0, "S must be a multiple of 64");
-  CSA_SUPPORT(D == 128 && Hq / Hkv == 4 && S <= 32768,
-              "implemented for D = 128, Hq/Hkv = 4 and S <= 32768");
+  CSA_SUPPORT(D == 128 && Hq / Hkv == 4 && S <= kTokenMaxS,
+              "implemented for D = 128, Hq/Hkv = 4 and S <= 131072");
   return CSA_OK;
 }
 }  // namespace
@@ -1059,7 +1077,7 @@ csa_status token_shape_checks(int B, int S, int Hq, int Hkv, int D) {
 csa_status csa_token_select(const float* imp, int B, int S, int Hkv, const int32_t* k_unit,
                             int32_t* idx, int32_t* count, csa_stream stream) {
   CSA_REQUIRE(B >= 0 && S >= 0 && Hkv > 0, "bad sizes");
-  CSA_SUPPORT(S <= 32768, "S must be <= 32768");
+  CSA_SUPPORT(S <= kTokenMaxS, "S must be <= 131072");
   if (static_cast<int64_t>(B) * S == 0) return CSA_OK;
   CSA_TRY(check_ptr(imp, "imp"));
   CSA_TRY(check_ptr(k_unit, "k_unit"));
@@ -1067,6 +1085,7 @@ csa_status csa_token_select(const float* imp, int B, int S, int Hkv, const int32
   CSA_TRY(check_ptr(count, "count"));
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
+  CSA_TRY(token_long_check(B, Hkv, S, l, false, true));
   return finish(csa::launch_select_topk(l, imp, B * Hkv, S, nullptr, 0, 0, 0, idx, count, S,
                                         k_unit),
                 "token select launch");

@@ -41,6 +41,9 @@ cudaError_t launch_score(const Launch& l, const void* q, bool bf16, const float*
 // (n_valid is then ignored).  inv (optional, [U, C]): when the long-row
 // cluster kernel runs, it also writes every position's slot in its unit's
 // list (or -1) and sets *inv_done; otherwise *inv_done is false.
+// The long-row top-k (one cluster of 8 CTAs per unit) runs for these sizes
+// (rows of C >= 8192 keys, nothing forced).
+bool topk_cluster_fits(int U, int C, int num_sms);
 cudaError_t launch_select_topk(const Launch& l, const float* scores, int U, int C,
                                const int32_t* n_valid, int k_free, int n_sink, int n_local,
                                int32_t* idx, int32_t* count, int kmax,
@@ -71,6 +74,9 @@ size_t token_importance_scratch_bytes(int B, int S, int Hkv, int G, int n_obs);
 cudaError_t launch_token_importance(const Launch& l, const void* Q, const void* K, int B, int S,
                                     int Hq, int Hkv, int D, int n_obs, float scale, float* imp,
                                     float* scratch, std::string* why);
+// The coverage budget runs one cluster of 8 CTAs per sequence for these
+// sizes (else one CTA per sequence, S <= 32768).
+bool token_budget_cluster_fits(int B, int num_sms);
 cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S, int Hkv,
                                 float tau, int tile, int32_t* k_seq, int32_t* k_unit);
 cudaError_t launch_tsa_gather(const Launch& l, const void* Q, const void* K, const void* V,

@@ -735,19 +735,22 @@ __global__ void __launch_bounds__(kBudgetCThreads) budget_cluster_kernel(
   const int n = static_cast<int>(static_cast<int64_t>(S) * (rank + 1) / CS) - lo;
   const float* ib = imp + static_cast<int64_t>(b) * Hkv * S + lo;
   float part = 0.f;
-  // n <= kBudgetJ * blockDim.x (S <= 32768 over kBudgetCS CTAs): the loop is
-  // unrolled so that every load of the thread is in flight together
+  // rounds of kBudgetJ * blockDim.x tokens (one round up to S = 32768 over
+  // kBudgetCS CTAs), each unrolled so that every load of the thread in the
+  // round is in flight together
   constexpr int kBudgetJ = 8;
+  for (int j0 = 0; j0 < n; j0 += kBudgetJ * kBudgetCThreads) {
 #pragma unroll
-  for (int k = 0; k < kBudgetJ; ++k) {
-    const int j = tid + k * kBudgetCThreads;
-    if (j < n) {
-      float m = 0.f;
+    for (int k = 0; k < kBudgetJ; ++k) {
+      const int j = j0 + tid + k * kBudgetCThreads;
+      if (j < n) {
+        float m = 0.f;
 #pragma unroll 8
-      for (int h = 0; h < Hkv; ++h) m += ib[static_cast<int64_t>(h) * S + j];
-      m = fmaxf(m, 0.f);
-      ms[j] = m;
-      part += m;
+        for (int h = 0; h < Hkv; ++h) m += ib[static_cast<int64_t>(h) * S + j];
+        m = fmaxf(m, 0.f);
+        ms[j] = m;
+        part += m;
+      }
     }
   }
 #pragma unroll
@@ -1035,10 +1038,14 @@ cudaError_t set_smem_ts(const void* fn, size_t bytes) {
 
 }  // namespace
 
+bool token_budget_cluster_fits(int B, int num_sms) {
+  return B <= 65535 && static_cast<int64_t>(B) * kBudgetCS <= num_sms;
+}
+
 cudaError_t launch_token_budget(const Launch& l, const float* imp, int B, int S, int Hkv,
                                 float tau, int tile, int32_t* k_seq, int32_t* k_unit) {
   if (B == 0) return cudaSuccess;
-  if (B <= 65535 && static_cast<int64_t>(B) * kBudgetCS <= l.num_sms) {  // one cluster per sequence
+  if (token_budget_cluster_fits(B, l.num_sms)) {  // one cluster per sequence
     const size_t shc = static_cast<size_t>((S + kBudgetCS - 1) / kBudgetCS) * 4 +
                        static_cast<size_t>(kBudgetCThreads / 32) * 256 * 8;
     // always set: with its static histograms the kernel may pass 48 KB in all

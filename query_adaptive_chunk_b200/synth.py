@@ -172,6 +172,11 @@ TOKEN_SPARSE_HEAVY_32K = dataclasses.replace(
     PREFILL_32K, name="token_sparse_heavy_prefill_bf16_seq32k", seed=9, planted=0,
     heavy_frac=0.2, heavy_strength=8.0)
 
+# The same recipe at the 128K context the Token Sparse page reports its
+# speed-up and index overhead at (B=1, Hq=32, Hkv=8, D=128)
+TOKEN_SPARSE_HEAVY_128K = dataclasses.replace(
+    TOKEN_SPARSE_HEAVY_32K, name="token_sparse_heavy_prefill_bf16_seq128k", seed=10, S=131072)
+
 # Per-head top-k with the GQA union on the 32K shapes: each of the 4 query
 # heads of a group keeps its own 29 best chunks, the group reads the union.
 TOPK_UNION_32K = dataclasses.replace(TOPK_32K, name="topk_union_decode_bf16_ctx32k", seed=6,
@@ -193,7 +198,7 @@ ROPE_TOPK_32K = dataclasses.replace(TOPK_32K, name="rope_topk_decode_bf16_ctx32k
 
 DECODE_WORKLOADS = (TINY_F32, TOPK_32K, TOPP_128K, HIER_1M, TOPK_UNION_32K, HYBRID_TOPK_32K,
                     HYBRID_ALL_TOPK_32K, ROPE_TOPK_32K)
-ALL_WORKLOADS = DECODE_WORKLOADS + (PREFILL_32K, TOKEN_SPARSE_HEAVY_32K)
+ALL_WORKLOADS = DECODE_WORKLOADS + (PREFILL_32K, TOKEN_SPARSE_HEAVY_32K, TOKEN_SPARSE_HEAVY_128K)
 
 
 def _gen(device, seed: int, tid: int) -> torch.Generator:

@@ -315,13 +315,15 @@ def test_token_sparse_steps_match_whole_call_and_graph():
     del g
 
 
-def test_token_sparse_heavy_workload():
-    """The high-sparsity workload at full size (32K, 20% heavy-hitter tokens
-    shared by the KV heads, n_obs = 64, tau = 0.1): the budget keeps a small
-    part of the sequence; importance, budget, kept sets and a sample of
-    output rows per head against the oracle (as for the benched 32K call)."""
+@pytest.mark.parametrize("wname", ["TOKEN_SPARSE_HEAVY_32K", "TOKEN_SPARSE_HEAVY_128K"])
+def test_token_sparse_heavy_workload(wname):
+    """The high-sparsity workloads at full size (32K and 128K, 20% heavy-hitter
+    tokens shared by the KV heads, n_obs = 64, tau = 0.1): the budget keeps a
+    small part of the sequence; importance, budget, kept sets and a sample of
+    output rows per head against the oracle (as for the benched 32K call).
+    At 128K the budget and the token choice run on their cluster paths."""
     from query_adaptive_chunk_b200 import csa, synth
-    w = synth.TOKEN_SPARSE_HEAVY_32K
+    w = getattr(synth, wname)
     inp = synth.make_prefill_inputs(w, device="cuda")
     Q, K, V = inp["Q"], inp["K"], inp["V"]
     B, S, Hq, Hkv, D = w.B, w.S, w.Hq, w.Hkv, w.D
@@ -356,3 +358,28 @@ def test_token_sparse_heavy_workload():
         dropped = np.nonzero(~kept_gpu)[0]
         pick = rng.choice(dropped, size=min(16, len(dropped)), replace=False)
         assert np.all(got[pick] == 0), (h, pick)
+
+
+def test_token_sparse_long_sequences_need_the_cluster_paths():
+    """Beyond 32768 tokens the budget and the token choice hold S / 8 values
+    per CTA of their cluster paths: with more sequences than the SMs hold
+    8-CTA clusters for, the calls are refused (CSA_ERR_UNSUPPORTED) before
+    anything is enqueued; above 131072 tokens always."""
+    from query_adaptive_chunk_b200 import csa
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, Hkv, S = sms // 8 + 1, 1, 65536
+    imp = torch.zeros(B, Hkv, S, device="cuda")
+    k_seq = torch.zeros(B, dtype=torch.int32, device="cuda")
+    k_unit = torch.zeros(B * Hkv, dtype=torch.int32, device="cuda")
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_token_budget(imp, B, S, Hkv, 0.1, 64, k_seq, k_unit)
+    assert ei.value.status == 2
+    idx = torch.zeros(B * Hkv, S, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B * Hkv, dtype=torch.int32, device="cuda")
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_token_select(imp, B, S, Hkv, k_unit, idx, cnt)
+    assert ei.value.status == 2
+    imp1 = torch.zeros(1, 1, 2 * 131072, device="cuda")
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_token_budget(imp1, 1, 2 * 131072, 1, 0.1, 64, k_seq[:1], k_unit[:1])
+    assert ei.value.status == 2
