@@ -1024,8 +1024,10 @@ __global__ void __launch_bounds__(kScatterThreads) tsa_scatter_kernel(
     for (int r = 0; r < nrow; ++r) {
       const int t = it[r];
       int4 v = make_int4(0, 0, 0, 0);
-      if (t >= 0) v = *reinterpret_cast<const int4*>(ob + (static_cast<int64_t>(t) * Hq + hq) * D + c);
-      *reinterpret_cast<int4*>(dst + (static_cast<int64_t>(r) * Hq + hq) * D + c) = v;
+      if (t >= 0)
+        v = __ldcs(reinterpret_cast<const int4*>(ob + (static_cast<int64_t>(t) * Hq + hq) * D + c));
+      // O is written once and not read again here: streaming (evict-first) stores
+      __stcs(reinterpret_cast<int4*>(dst + (static_cast<int64_t>(r) * Hq + hq) * D + c), v);
     }
   }
 }
