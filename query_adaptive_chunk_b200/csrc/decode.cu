@@ -483,6 +483,12 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* ptr, int v) {
   return old;
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -993,7 +999,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   int* prefix2 = prefix + (p.U + 1);  // phase 2 (sparse units), built by the producer
   __shared__ int scan_sh[33];
   __shared__ int defer_u[kDeferMax], defer_ns[kDeferMax];
-  __shared__ int n_defer_sh, pre_u_sh, pre_ns_sh;
+  __shared__ int n_defer_sh, pre_u_sh, pre_ns_sh, own_ok_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -1027,6 +1033,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   auto phase_parts = [&](int ph) -> int64_t {
     return (p.phased && ph == 0) ? P_all - p.late : P_all;
   };
+  // merged phased launches: the late CTAs merge the full-head units
+  const bool own_full = p.merged && p.phased && p.late > 0;
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer
@@ -1100,24 +1108,58 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   auto final_merges = [&](int tid) {
     if (!end_sync()) return;
     const int nd = n_defer_sh, pu = pre_u_sh;
-    if (nd == 0 && pu < 0) return;
-    // the arrival counts seen (by the epilogue's atomics) before partials are
-    // read by these threads; not needed when the only merge's partials and
-    // lse rows come by the bulk copy its own issuer ordered
-    if (nd > 0 || (p.max_splits & 3) != 0) fence_acq_rel_gpu();
     uint32_t n_bulk = 0;
-    if (pu >= 0) {  // the last unit of the CTA: its copy is already in flight
-      if (!merge_staged<D>(p, pu, pre_ns_sh, smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk, true,
-                           tid, (kConsumerWarps + 1) * 32, end_sync))
-        return;
-      if (tid == 0) p.counters[pu] = 0;  // ready for the next call
+    if (nd > 0 || pu >= 0) {
+      // the arrival counts seen (by the epilogue's atomics) before partials are
+      // read by these threads; not needed when the only merge's partials and
+      // lse rows come by the bulk copy its own issuer ordered
+      if (nd > 0 || (p.max_splits & 3) != 0) fence_acq_rel_gpu();
+      if (pu >= 0) {  // the last unit of the CTA: its copy is already in flight
+        if (!merge_staged<D>(p, pu, pre_ns_sh, smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk,
+                             true, tid, (kConsumerWarps + 1) * 32, end_sync))
+          return;
+        if (tid == 0) p.counters[pu] = 0;  // ready for the next call
+      }
+      for (int k = 0; k < nd; ++k) {
+        const int u = defer_u[k];
+        if (!merge_staged<D>(p, u, defer_ns[k], smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk,
+                             false, tid, (kConsumerWarps + 1) * 32, end_sync))
+          return;
+        if (tid == 0) p.counters[u] = 0;  // ready for the next call
+      }
     }
-    for (int k = 0; k < nd; ++k) {
-      const int u = defer_u[k];
-      if (!merge_staged<D>(p, u, defer_ns[k], smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk, false,
-                           tid, (kConsumerWarps + 1) * 32, end_sync))
-        return;
-      if (tid == 0) p.counters[u] = 0;  // ready for the next call
+    // A late CTA of a merged phased launch merges the full-head units assigned
+    // to it (the k-th such unit to late CTA k mod late): their splits all come
+    // in phase 1, while the late CTAs' own work is phase 2 only, so these
+    // merges run beside the other CTAs' streaming instead of at the end.
+    if (own_full && static_cast<int64_t>(blockIdx.x) >= P_all - p.late) {
+      const int64_t N1 = prefix[p.U], P1 = P_all - p.late;
+      const int li = static_cast<int>(blockIdx.x - P1);
+      int kf = 0;
+      for (int u = 0; u < p.U; ++u) {
+        if (prefix[u + 1] <= prefix[u]) continue;  // not a phase-1 unit
+        if (kf++ % p.late != li) continue;
+        const int ns = split_count(prefix[u], prefix[u + 1], N1, P1);
+        if (ns <= 1) continue;  // one split writes the unit's rows itself
+        if (tid == 0) {  // every split counted in (bounded)
+          int ok = 1;
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(p.counters + u) < ns) {
+            if (globaltimer_ns() - t0 > p.err.wait_ns) {
+              dev_flag(p.err, DEV_TIMEOUT);
+              ok = 0;
+              break;
+            }
+            __nanosleep(64);
+          }
+          own_ok_sh = ok;
+        }
+        if (!end_sync() || !own_ok_sh) return;
+        if (!merge_staged<D>(p, u, ns, smem, NS * Sh::STAGE_BYTES, merge_bar, n_bulk, false, tid,
+                             (kConsumerWarps + 1) * 32, end_sync))
+          return;
+        if (tid == 0) p.counters[u] = 0;  // ready for the next call
+      }
     }
   };
 
@@ -1166,6 +1208,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                                     NS * Sh::STAGE_BYTES, merge_bar, fb_empty + 8 * k, &pre_u_sh,
                                     &pre_ns_sh, dry);
         if (dry || last != 1) continue;
+        if (ph == 0 && own_full) continue;  // a late CTA merges it
         if (n_defer < kDeferMax) {  // merged after the main loop, off the hot path
           if (lane == 0) {
             defer_u[n_defer] = u;
