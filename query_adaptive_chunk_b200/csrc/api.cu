@@ -623,7 +623,8 @@ csa_status score_select_topp_impl(const void* q, csa_dtype q_dtype, const float*
                                   const float* summ, int B, int Hq, int Hkv, int D, int C,
                                   const uint8_t* head_full, float logit_scale, float p, int budget,
                                   int n_sink, int n_local, int32_t* idx, int32_t* count, int kmax,
-                                  int32_t* n_p_out, csa_stream stream, bool check_only) {
+                                  int32_t* n_p_out, csa_stream stream, bool check_only,
+                                  bool after_query_copy = false) {
   CSA_REQUIRE(valid_dtype(q_dtype), "q_dtype");
   CSA_REQUIRE(kmax > 0, "kmax must be positive");
   CSA_REQUIRE(B >= 0 && Hq > 0 && Hkv > 0 && D > 0 && C > 0 && n_sink >= 0 && n_local >= 0,
@@ -648,6 +649,7 @@ csa_status score_select_topp_impl(const void* q, csa_dtype q_dtype, const float*
   csa::Launch l;
   CSA_TRY(launch_ctx(stream, &l));
   if (check_only) return CSA_OK;
+  l.after_query_copy = after_query_copy;
   return finish(csa::launch_score_select_topp(l, q, q_dtype == CSA_BF16, proj, R, summ, B, Hq, Hkv, D,
                                               C, head_full, logit_scale, p, budget, n_sink, n_local,
                                               idx, count, kmax, n_p_out),
@@ -755,7 +757,9 @@ csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stre
   // the selection scores with the pre-RoPE query when one is given
   const void* qs = d->q_score != nullptr ? d->q_score : d->q;
   if (d->q_score != nullptr) CSA_TRY(check_ptr(d->q_score, "q_score"));
-  auto selection = [&](bool check_only) -> csa_status {
+  // after_copy: the query copy kernel runs right before the selection (the
+  // top-p selection then starts behind it with programmatic dependent launch)
+  auto selection = [&](bool check_only, bool after_copy) -> csa_status {
     if (d->mode == CSA_SELECT_TOPK || d->mode == CSA_SELECT_TOPK_UNION)
       return score_select_topk_common(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
                                       d->D, C, d->head_full, d->k_free, d->n_sink, d->n_local,
@@ -765,15 +769,17 @@ csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stre
       return score_select_topp_impl(qs, CSA_BF16, d->proj, d->R, d->summ, d->B, d->Hq, d->Hkv,
                                     d->D, C, d->head_full, d->logit_scale, d->p, d->budget,
                                     d->n_sink, d->n_local, d->idx, d->count, d->kmax, d->n_p_out,
-                                    stream, check_only);
+                                    stream, check_only, after_copy);
     return select_hier_impl(qs, CSA_BF16, d->meta, d->summ, d->B, d->Hq, d->Hkv, d->D, C, d->Gm,
                             d->top_meta, d->k_free, d->n_sink, d->n_local, d->idx, d->count,
                             d->kmax, stream, check_only);
   };
   // every argument of the selection too, before the query copy is enqueued
-  CSA_TRY(selection(true));
+  CSA_TRY(selection(true, false));
+  bool q_by_kernel = false;  // the query copied by a kernel just before the selection
   if (io != nullptr && io->q != nullptr) {
     const size_t nq = static_cast<size_t>(d->B) * d->Hq * d->D * sizeof(__nv_bfloat16);
+    q_by_kernel = io->q_mapped && nq >= 16;
     if (io->q_mapped)
       CSA_TRY(finish(csa::launch_copy16(l, io->q, const_cast<void*>(d->q), nq),
                      "query copy to the device"));
@@ -782,7 +788,7 @@ csa_status decode_step(const csa_decode_step_desc* d, const HostIO* io, csa_stre
                                      l.stream),
                      "query copy to the device"));
   }
-  const csa_status st = selection(false);
+  const csa_status st = selection(false, q_by_kernel && d->q_score == nullptr);
   if (st != CSA_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(d->workspace);
   csa::MergeOut m{reinterpret_cast<int*>(ws + w.counters), d->out, d->out_dtype == CSA_BF16,

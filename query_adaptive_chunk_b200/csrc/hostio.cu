@@ -10,8 +10,11 @@
 namespace csa {
 namespace {
 
-// 16-byte words from src to dst, one word per thread.
+// 16-byte words from src to dst, one word per thread.  A kernel launched
+// behind it with programmatic dependent launch may start at once (it waits
+// for this grid's completion before reading dst).
 __global__ void copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < n) dst[i] = src[i];
 }

@@ -19,6 +19,10 @@ struct Launch {
   cudaStream_t stream;
   DevErr err;
   int num_sms;
+  // the launch follows a kernel that writes the query it reads (a host-query
+  // copy): a launcher that supports it starts behind that kernel with
+  // programmatic dependent launch and waits for it before reading the query
+  bool after_query_copy = false;
 };
 
 // summaries.cu

@@ -40,6 +40,12 @@ __device__ __forceinline__ void allow_dependent_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Waits until the grid this one was launched behind (programmatic dependent
+// launch) has completed and its writes are visible; returns at once otherwise.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   uint32_t b = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
   return __uint_as_float(b);
@@ -1170,8 +1176,11 @@ __global__ void __launch_bounds__(kSelThreads) score_select_topp_kernel(
     const float* __restrict__ summ, int Hq, int Hkv, int D, int C,
     const uint8_t* __restrict__ head_full, float logit_scale, float p, int budget, int n_sink,
     int n_local, int32_t* __restrict__ idx, int32_t* __restrict__ count, int kmax,
-    int32_t* __restrict__ n_p_out, int SN) {
-  allow_dependent_launch();
+    int32_t* __restrict__ n_p_out, int SN, int q_after_copy) {
+  // q_after_copy: launched behind the kernel that writes q (programmatic
+  // dependent launch); the grid behind this one may start only once q is
+  // complete, since it reads q without waiting for this grid
+  if (!q_after_copy) allow_dependent_launch();
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ SelScratch s;
   __shared__ BucketScratch bs;
@@ -1194,6 +1203,10 @@ __global__ void __launch_bounds__(kSelThreads) score_select_topp_kernel(
   const float* summ_u = summ + static_cast<int64_t>(u) * C * DS;
   float4 pre[kRowBatch];
   rows_load<DS>(summ_u, C, rows_first_base<DS>(), pre);  // in flight during the query phase
+  if (q_after_copy) {
+    grid_dependency_wait();  // the query copy is complete and visible
+    allow_dependent_launch();
+  }
   unit_query(q, q_bf16, static_cast<int64_t>(b) * Hq + h * G, G, D, proj, R, f.qs, f.qv, f.part);
   for (int c = threadIdx.x; c < C; c += blockDim.x) flags[c] = 0;
   float mx = -INFINITY, Z = 0.f;
@@ -1973,10 +1986,26 @@ cudaError_t fused_topp_ds(const Launch& l, const void* q, bool bf16, const float
   const size_t sh = topp_head_bytes(C, SN) + static_cast<size_t>(C) * 5 + 16;
   cudaError_t e = set_smem(reinterpret_cast<const void*>(score_select_topp_kernel<DS>), sh);
   if (e != cudaSuccess) return e;
-  score_select_topp_kernel<DS><<<U, kSelThreads, sh, l.stream>>>(
-      q, bf16 ? 1 : 0, proj, R, summ, Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink,
-      n_local, idx, count, kmax, n_p_out, SN);
-  return cudaGetLastError();
+  if (!l.after_query_copy) {
+    score_select_topp_kernel<DS><<<U, kSelThreads, sh, l.stream>>>(
+        q, bf16 ? 1 : 0, proj, R, summ, Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink,
+        n_local, idx, count, kmax, n_p_out, SN, 0);
+    return cudaGetLastError();
+  }
+  // behind the query copy: start now, wait for it before reading q
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(U);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = sh;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_select_topp_kernel<DS>, q, bf16 ? 1 : 0, proj, R, summ,
+                            Hq, Hkv, D, C, head_full, logit_scale, p, budget, n_sink, n_local, idx,
+                            count, kmax, n_p_out, SN, 1);
 }
 }  // namespace
 
