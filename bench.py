@@ -360,6 +360,76 @@ def time_decode_rotating(w, inp, steps: int, warmup: int, copies: int = 8):
     return {"decode_ms": dec_ms, "step_ms": step_ms, "cache_bytes": cache_bytes}
 
 
+def time_separate_calls(w, steps: int, warmup: int, flush):
+    """The headline step as the separate boundary calls (the unfused path):
+    csa_score_chunks, csa_select_topp, csa_sparse_decode (split partials) and
+    csa_lse_merge, in one CUDA graph with an event between each pair (L2
+    flushed before each replay).  Returns each call's times (ms) and the
+    partials' bytes the merge reads."""
+    from query_adaptive_chunk_b200 import csa
+    from query_adaptive_chunk_b200.steps import SparseDecoder, _dt
+    assert w.select == "topp"
+    inp = synth.make_decode_inputs(w, device="cuda")
+    d = SparseDecoder(inp["K"], inp["V"], Hq=w.Hq, L=w.L, select=w.select, n_sink=w.n_sink,
+                      n_local=w.n_local, k_free=w.k_free, proj=inp.get("proj"), p=w.p,
+                      budget=w.budget, full_heads=w.full_heads, fused=False)
+    q = inp["q"]
+    qd = _dt(q)
+    B, Hq, Hkv, D, C = d.B, d.Hq, d.Hkv, d.D, d.C
+    ev = [_ext_event() for _ in range(5)]
+    if any(e is None for e in ev):
+        return None
+
+    def calls(with_events):
+        if with_events:
+            ev[0].record()
+        csa.csa_score_chunks(q, qd, d.proj, d.R, d.summ, B, 1, Hq, Hkv, D, C, d.head_full, 0, 0,
+                             d.scores)
+        if with_events:
+            ev[1].record()
+        csa.csa_select_topp(d.scores, B * Hkv, C, 1.0 / math.sqrt(D), d.p, d.budget, d.n_sink,
+                            d.n_local, d.idx, d.count, d.kmax, d.n_p)
+        if with_events:
+            ev[2].record()
+        csa.csa_sparse_decode(q, d.K_att, d.V, d.dtype, d.idx, d.count, d.kmax, d.head_full, B,
+                              Hq, Hkv, D, d.T, d.L, d.scale, d.P, d.max_splits, d.o_part,
+                              d.lse_part)
+        if with_events:
+            ev[3].record()
+        csa.csa_lse_merge(d.o_part, d.lse_part, B * Hq, d.max_splits, D, d.out, _dt(d.out),
+                          d.lse)
+        if with_events:
+            ev[4].record()
+
+    for _ in range(warmup):
+        calls(False)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        calls(False)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        calls(True)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    names = ("score", "select", "decode", "merge")
+    ms = {k: [] for k in names}
+    for _ in range(steps):
+        flush()
+        g.replay()
+        torch.cuda.synchronize()
+        for i, k in enumerate(names):
+            ms[k].append(ev[i].elapsed_time(ev[i + 1]))
+    csa.csa_check_device_status()
+    del g
+    part_bytes = (d.o_part.numel() + d.lse_part.numel()) * 4
+    return {"ms": ms, "merge_read_bytes": part_bytes, "dec": d}
+
+
 def time_e2e(w, dec, inp, steps: int, flush):
     """Same step through the public API with the query in pinned host memory
     and the output read back to pinned host memory, every step
@@ -890,6 +960,23 @@ def other_workloads(args, flush, peaks):
                     "copies": n_cp, "resident_bytes": n_cp * rr["cache_bytes"],
                     "note": f"no flush: {n_cp} copies of the K/V cache in rotation"}
             del rr
+        del r
+        torch.cuda.empty_cache()
+    # the headline step as the separate boundary calls (split partials and the
+    # stand-alone log-sum-exp merge)
+    r = time_separate_calls(synth.TOPP_128K, steps, args.warmup, flush)
+    if r is not None:
+        st = {k: 1000 * statistics.mean(v) for k, v in r["ms"].items()}
+        kv = selected_bytes(synth.TOPP_128K, r["dec"])[0]
+        out["topp_mixed_decode_bf16_ctx128k_separate_calls"] = {
+            "score_us": round(st["score"], 3), "select_us": round(st["select"], 3),
+            "decode_split_partials_us": round(st["decode"], 3), "merge_us": round(st["merge"], 3),
+            "sum_us": round(sum(st.values()), 3),
+            "decode_gbs": round(kv / (st["decode"] * 1e-6) / 1e9, 1),
+            "decode_frac_of_measured_hbm": round(kv / (st["decode"] * 1e-6) / 1e9 /
+                                                 peaks["hbm_gbs"], 4),
+            "merge_read_bytes": r["merge_read_bytes"],
+            "merge_gbs": round(r["merge_read_bytes"] / (st["merge"] * 1e-6) / 1e9, 1)}
         del r
         torch.cuda.empty_cache()
     for tw, name in ((synth.PREFILL_32K, "token_sparse_prefill_bf16_seq32k"),
