@@ -376,11 +376,11 @@ def time_separate_calls(w, steps: int, warmup: int, flush):
     q = inp["q"]
     qd = _dt(q)
     B, Hq, Hkv, D, C = d.B, d.Hq, d.Hkv, d.D, d.C
-    ev = [_ext_event() for _ in range(5)]
+    ev = [_ext_event() for _ in range(7)]
     if any(e is None for e in ev):
         return None
 
-    def calls(with_events):
+    def calls(with_events, pair=False):
         if with_events:
             ev[0].record()
         csa.csa_score_chunks(q, qd, d.proj, d.R, d.summ, B, 1, Hq, Hkv, D, C, d.head_full, 0, 0,
@@ -391,6 +391,8 @@ def time_separate_calls(w, steps: int, warmup: int, flush):
                             d.n_local, d.idx, d.count, d.kmax, d.n_p)
         if with_events:
             ev[2].record()
+        if pair:
+            ev[5].record()
         csa.csa_sparse_decode(q, d.K_att, d.V, d.dtype, d.idx, d.count, d.kmax, d.head_full, B,
                               Hq, Hkv, D, d.T, d.L, d.scale, d.P, d.max_splits, d.o_part,
                               d.lse_part)
@@ -400,6 +402,8 @@ def time_separate_calls(w, steps: int, warmup: int, flush):
                           d.lse)
         if with_events:
             ev[4].record()
+        if pair:
+            ev[6].record()
 
     for _ in range(warmup):
         calls(False)
@@ -413,19 +417,30 @@ def time_separate_calls(w, steps: int, warmup: int, flush):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, capture_error_mode="relaxed"):
         calls(True)
+    # the decode and the merge with no event between them (the merge is
+    # launched behind the decode with programmatic dependent launch)
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, capture_error_mode="relaxed"):
+        calls(False, pair=True)
     for _ in range(warmup):
         g.replay()
+        g2.replay()
     torch.cuda.synchronize()
     names = ("score", "select", "decode", "merge")
     ms = {k: [] for k in names}
+    ms["decode_merge"] = []
     for _ in range(steps):
         flush()
         g.replay()
         torch.cuda.synchronize()
         for i, k in enumerate(names):
             ms[k].append(ev[i].elapsed_time(ev[i + 1]))
+        flush()
+        g2.replay()
+        torch.cuda.synchronize()
+        ms["decode_merge"].append(ev[5].elapsed_time(ev[6]))
     csa.csa_check_device_status()
-    del g
+    del g, g2
     part_bytes = (d.o_part.numel() + d.lse_part.numel()) * 4
     return {"ms": ms, "merge_read_bytes": part_bytes, "dec": d}
 
@@ -971,7 +986,8 @@ def other_workloads(args, flush, peaks):
         out["topp_mixed_decode_bf16_ctx128k_separate_calls"] = {
             "score_us": round(st["score"], 3), "select_us": round(st["select"], 3),
             "decode_split_partials_us": round(st["decode"], 3), "merge_us": round(st["merge"], 3),
-            "sum_us": round(sum(st.values()), 3),
+            "sum_us": round(st["score"] + st["select"] + st["decode"] + st["merge"], 3),
+            "decode_then_merge_us": round(st["decode_merge"], 3),
             "decode_gbs": round(kv / (st["decode"] * 1e-6) / 1e9, 1),
             "decode_frac_of_measured_hbm": round(kv / (st["decode"] * 1e-6) / 1e9 /
                                                  peaks["hbm_gbs"], 4),

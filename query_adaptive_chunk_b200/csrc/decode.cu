@@ -1002,6 +1002,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __shared__ int n_defer_sh, pre_u_sh, pre_ns_sh, own_ok_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // split partials out (no merge here): the merge kernel launched behind this
+  // one may become resident now; it waits for this grid before reading them
+  if (!p.merged) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full_bar + 8 * s, 1);
@@ -1548,6 +1551,8 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(const DecodePar
   int* prefix = reinterpret_cast<int*>(vs + 128 * D);  // [U+1]
   __shared__ int scan_sh[33];
   __shared__ int last_sh;
+  // split partials out: the merge kernel behind this one may become resident
+  if (!p.merged) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   build_prefix(p, prefix, scan_sh);
   fill_empty_slots(p, prefix, kF32Threads);
   const int64_t N = prefix[p.U], P = gridDim.x;
@@ -1699,6 +1704,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   const int r = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* lrow = lse_part + static_cast<int64_t>(r) * S;
+  // launched behind the split decode (programmatic dependent launch): the
+  // CTAs wait here, resident, until its partials are complete and visible
+  grid_dependency_wait();
   // row max
   float mx = -INFINITY;
   for (int s = threadIdx.x; s < S; s += kMergeThreads) mx = fmaxf(mx, lrow[s]);
@@ -1981,9 +1989,20 @@ cudaError_t launch_merge(const Launch& l, const float* o_part, const float* lse_
                                          static_cast<int>(sh));
     if (e != cudaSuccess) return e;
   }
-  merge_kernel<<<rows, kMergeThreads, sh, l.stream>>>(o_part, lse_part, rows, max_splits, D, out,
-                                                      out_bf16 ? 1 : 0, lse_out);
-  return cudaGetLastError();
+  // behind the kernel that writes the partials: may start early (it waits
+  // on the device for that kernel to complete)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = sh;
+  cfg.stream = l.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_kernel, o_part, lse_part, rows, max_splits, D, out,
+                            out_bf16 ? 1 : 0, lse_out);
 }
 
 }  // namespace csa
