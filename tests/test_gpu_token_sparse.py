@@ -360,6 +360,54 @@ def test_token_sparse_heavy_workload(wname):
         assert np.all(got[pick] == 0), (h, pick)
 
 
+def test_token_sparse_long_batch_on_the_cluster_paths():
+    """Two sequences of 65536 tokens (beyond 32768: the budget and the token
+    choice on their cluster paths, one cluster per sequence and per KV head),
+    with different budgets: budget, kept sets and sampled rows against the
+    oracle, dropped rows exactly 0."""
+    from query_adaptive_chunk_b200 import csa
+    B, S, Hq, Hkv, D, n_obs, tau = 2, 65536, 8, 2, 128, 64, 0.1
+    Q, K, V = _inputs(B, S, Hq, Hkv, D, seed=65)
+    Q[1] *= 3  # sharper attention in sequence 1: a different budget
+    G, scale = Hq // Hkv, 1.0 / math.sqrt(D)
+    nbw = csa.csa_token_sparse_workspace_bytes(B, S, Hq, Hkv, D, n_obs)
+    ws = torch.empty(nbw, dtype=torch.uint8, device="cuda")
+    Ob = torch.full((B, S, Hq, D), float("nan"), device="cuda").to(torch.bfloat16)
+    budget = torch.zeros(B, dtype=torch.int32, device="cuda")
+    csa.csa_token_sparse_prefill(Q, K, V, B, S, Hq, Hkv, D, n_obs, tau, scale, ws, nbw, Ob, budget)
+    csa.csa_check_device_status()
+    rng = np.random.default_rng(65536)
+    for b in range(B):
+        imps = [_oracle_importance(Q, K, b, h, G, n_obs, scale) for h in range(Hkv)]
+        mass = np.sum(imps, axis=0)
+        k_ref = O.coverage_budget(mass, tau)
+        k_got = int(budget[b])
+        cum = np.cumsum(np.sort(mass / mass.sum())[::-1])
+        assert k_got == k_ref or (cum[k_got - 1] >= (1 - tau) - 1e-6 and
+                                  (k_got < 2 or cum[k_got - 2] <= (1 - tau) + 1e-6)), (b, k_got, k_ref)
+        kt = min(S, (k_got + 63) // 64 * 64)
+        Kb, Vb = K[b].cpu(), V[b].cpu()
+        for h in range(Hkv):
+            got = Ob[b, :, h * G:(h + 1) * G].float().cpu().double().numpy()
+            kept_gpu = np.abs(got).sum(axis=(1, 2)) > 0
+            toks_ref = O.select_tokens(imps[h], kt)
+            toks = _check_kept_set(kept_gpu, toks_ref, imps[h], kt, S, f"long b{b} h{h}")
+            tset = np.asarray(toks if toks is not None else toks_ref, dtype=np.int64)
+            picks = np.unique(np.concatenate([[0, kt - 1], rng.choice(kt, size=14, replace=False)]))
+            Kh, Vh = to_np(Kb[h][tset]), to_np(Vb[h][tset])
+            for i in picks:
+                t = int(tset[i])
+                qrows = to_np(Q[b, t, h * G:(h + 1) * G])
+                ref = np.stack([O.causal_attend(qrows[g:g + 1], Kh, Vh, tset, t, scale)[0]
+                                for g in range(G)])
+                parity.assert_close(got[t], ref, "bf16", f"long b{b} h{h} row {t}")
+            dropped = np.nonzero(~kept_gpu)[0]
+            if len(dropped):
+                pick = rng.choice(dropped, size=min(16, len(dropped)), replace=False)
+                assert np.all(got[pick] == 0), (b, h, pick)
+    assert int(budget[0]) != int(budget[1]), budget
+
+
 def test_token_sparse_long_sequences_need_the_cluster_paths():
     """Beyond 32768 tokens the budget and the token choice hold S / 8 values
     per CTA of their cluster paths: with more sequences than the SMs hold

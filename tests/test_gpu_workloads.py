@@ -128,6 +128,13 @@ def test_hier_decode_reduced():
     run_and_check(synth.HIER_1M.scaled(T=131072, planted=8))
 
 
+def test_topp_mixed_step_batch3_late_merges():
+    """The one-call phased step with three sequences (24 units, 6 of them
+    full-head): the late CTAs merge the full-head units while the others
+    stream the sparse ones; every unit's set and output against the oracle."""
+    run_and_check(synth.TOPP_128K.scaled(B=3, T=8192, seed=31))
+
+
 def test_hier_decode_full_size():
     """1M context: the index sets of all 8 units, the attention of 3."""
     run_and_check(synth.HIER_1M, attention_units=[(0, 0), (0, 5), (0, 7)])
